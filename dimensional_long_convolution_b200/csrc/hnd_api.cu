@@ -1,0 +1,291 @@
+// hnd_api.cu -- the C ABI declared in include/hyena_nd.h: argument checks,
+// workspace planning, tier selection and launch sequencing.  Every arithmetic
+// step of the convolution runs in the kernels of hnd_kernels.cuh.
+#include "hyena_nd.h"
+#include "hnd_launch.h"
+
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+
+namespace hnd {
+cudaError_t launch_fused2d_f32(const ConvArgs& a);
+cudaError_t launch_fused2d_bf16(const ConvArgs& a);
+}  // namespace hnd
+
+namespace {
+
+thread_local int g_last_launches = 0;
+
+constexpr size_t kStatusBytes = 256;                  // status word + padding
+constexpr size_t kWaveBudget = size_t(48) << 20;      // multi-pass intermediate per wave
+constexpr size_t kFilterBudget = size_t(64) << 20;    // filter grid per channel chunk
+constexpr int kFilterMaxChunk = 16;
+
+enum Tier { kRows1D = 0, kFused2D = 1, kMulti2D = 2, kMulti3D = 3 };
+
+struct Plan {
+  int ndim = 0;
+  int n[3] = {1, 1, 1};
+  long long B = 0, C = 0;
+  int bf16 = 0;
+  long long L = 1;          // voxels per volume
+  long long gsz = 1;        // padded grid points per channel
+  long long spec_per = 0;   // complex values per channel spectrum
+  int tier = 0;
+  long long wave = 0;       // pairs per wave (multi-pass tiers)
+  int filter_chunk = 1;
+  size_t ws_total = 0;
+  size_t spec_bytes = 0;
+};
+
+bool pow2_in(long long x, long long lo, long long hi) { return x >= lo && x <= hi && (x & (x - 1)) == 0; }
+
+hyena_nd_status make_plan(const hyena_nd_problem* p, Plan* pl) {
+  if (!p) return HYENA_ND_ERR_INVALID_ARG;
+  if (p->ndim < 1 || p->ndim > 3) return HYENA_ND_ERR_INVALID_ARG;
+  if (p->B < 1 || p->C < 1) return HYENA_ND_ERR_INVALID_ARG;
+  if (p->io_dtype != HYENA_ND_F32 && p->io_dtype != HYENA_ND_BF16) return HYENA_ND_ERR_INVALID_ARG;
+  for (int a = 0; a < p->ndim; ++a)
+    if (p->n[a] < 1) return HYENA_ND_ERR_INVALID_ARG;
+  if (p->circular != 0) return HYENA_ND_ERR_UNSUPPORTED;
+  for (int a = 0; a < p->ndim; ++a)
+    if (!pow2_in(p->n[a], 8, 256)) return HYENA_ND_ERR_UNSUPPORTED;
+  if (p->ndim == 3 && (p->n[0] > 128 || p->n[1] > 128)) return HYENA_ND_ERR_UNSUPPORTED;
+  if (p->B > INT_MAX / p->C) return HYENA_ND_ERR_UNSUPPORTED;
+  pl->ndim = p->ndim;
+  pl->B = p->B;
+  pl->C = p->C;
+  pl->bf16 = p->io_dtype == HYENA_ND_BF16;
+  pl->L = 1;
+  pl->gsz = 1;
+  for (int a = 0; a < 3; ++a) pl->n[a] = 1;
+  for (int a = 0; a < p->ndim; ++a) {
+    pl->n[a] = static_cast<int>(p->n[a]);
+    pl->L *= p->n[a];
+    pl->gsz *= 2 * p->n[a];
+  }
+  const int nl = pl->n[p->ndim - 1];
+  if (p->ndim == 1) pl->spec_per = nl + 1;
+  else if (p->ndim == 2) pl->spec_per = static_cast<long long>(nl + 1) * 2 * pl->n[0];
+  else pl->spec_per = static_cast<long long>(nl + 1) * 4 * pl->n[0] * pl->n[1];
+  pl->spec_bytes = static_cast<size_t>(pl->spec_per) * 8 * static_cast<size_t>(p->C);
+
+  const long long pairs = p->B * p->C;
+  size_t ws_conv = 0;
+  if (p->ndim == 1) {
+    pl->tier = kRows1D;
+  } else if (p->ndim == 2 && pl->n[0] <= 128 && pl->n[1] <= 128) {
+    pl->tier = kFused2D;
+  } else {
+    pl->tier = p->ndim == 2 ? kMulti2D : kMulti3D;
+    const size_t per_pair = static_cast<size_t>(8) * static_cast<size_t>(pl->L);
+    long long w = static_cast<long long>(kWaveBudget / per_pair);
+    if (w < 1) w = 1;
+    if (w > pairs) w = pairs;
+    if (w >= p->B) w -= w % p->B;        // keep a channel's samples in one wave
+    pl->wave = w;
+    ws_conv = per_pair * static_cast<size_t>(w);
+  }
+  long long chunk = static_cast<long long>(kFilterBudget / (8 * static_cast<size_t>(pl->gsz)));
+  if (chunk < 1) chunk = 1;
+  if (chunk > kFilterMaxChunk) chunk = kFilterMaxChunk;
+  if (chunk > p->C) chunk = p->C;
+  pl->filter_chunk = static_cast<int>(chunk);
+  const size_t ws_filter = static_cast<size_t>(chunk) * static_cast<size_t>(pl->gsz) * 8;
+  pl->ws_total = kStatusBytes + (ws_conv > ws_filter ? ws_conv : ws_filter);
+  return HYENA_ND_OK;
+}
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+bool overlaps(const void* a, const void* b, size_t bytes) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + bytes && y < x + bytes;
+}
+
+hyena_nd_status cuda_status(cudaError_t e) { return e == cudaSuccess ? HYENA_ND_OK : HYENA_ND_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t hyena_nd_spectrum_bytes(const hyena_nd_problem* p) {
+  Plan pl;
+  return make_plan(p, &pl) == HYENA_ND_OK ? pl.spec_bytes : 0;
+}
+
+size_t hyena_nd_workspace_bytes(const hyena_nd_problem* p) {
+  Plan pl;
+  return make_plan(p, &pl) == HYENA_ND_OK ? pl.ws_total : 0;
+}
+
+hyena_nd_status hyena_nd_workspace_init(void* ws, size_t ws_bytes, void* cuda_stream) {
+  if (!ws) return HYENA_ND_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return HYENA_ND_ERR_MISALIGNED;
+  if (ws_bytes < kStatusBytes) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
+  return cuda_status(cudaMemsetAsync(ws, 0, 16, static_cast<cudaStream_t>(cuda_stream)));
+}
+
+hyena_nd_status hyena_nd_fftconv_batched(const hyena_nd_problem* p, const void* q, const void* k, const void* v,
+                                         const void* spectrum, int64_t spectrum_batch_stride, void* y, void* ws,
+                                         size_t ws_bytes, void* cuda_stream) {
+  Plan pl;
+  hyena_nd_status st = make_plan(p, &pl);
+  if (st != HYENA_ND_OK) return st;
+  if (!q || !k || !v || !spectrum || !y || !ws) return HYENA_ND_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(spectrum) || !aligned16(y) || !aligned16(ws))
+    return HYENA_ND_ERR_MISALIGNED;
+  if (spectrum_batch_stride < 0) return HYENA_ND_ERR_INVALID_ARG;
+  if (spectrum_batch_stride % 16 != 0) return HYENA_ND_ERR_MISALIGNED;
+  if (ws_bytes < pl.ws_total) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
+  const size_t act_bytes = static_cast<size_t>(pl.B * pl.C * pl.L) * (pl.bf16 ? 2 : 4);
+  if (overlaps(y, q, act_bytes) || overlaps(y, k, act_bytes) || overlaps(y, v, act_bytes))
+    return HYENA_ND_ERR_INVALID_ARG;
+
+  hnd::ConvArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.spec = spectrum;
+  a.sbs = spectrum_batch_stride / 8;
+  a.y = y;
+  a.B = static_cast<int>(pl.B);
+  a.C = static_cast<int>(pl.C);
+  a.bf16 = pl.bf16;
+  a.ndim = pl.ndim;
+  for (int i = 0; i < 3; ++i) a.n[i] = pl.n[i];
+  a.stream = static_cast<cudaStream_t>(cuda_stream);
+
+  int launches = 0;
+  cudaError_t e = cudaSuccess;
+  if (pl.tier == kRows1D) {
+    e = hnd::launch_rows1d(a);
+    launches = 1;
+  } else if (pl.tier == kFused2D) {
+    e = pl.bf16 ? hnd::launch_fused2d_bf16(a) : hnd::launch_fused2d_f32(a);
+    launches = 1;
+  } else {
+    float2* zt = reinterpret_cast<float2*>(static_cast<char*>(ws) + kStatusBytes);
+    const long long pairs = pl.B * pl.C;
+    const int nl = pl.n[pl.ndim - 1];
+    const int rp_total = static_cast<int>(pl.L / nl / 2);
+    for (long long ord0 = 0; ord0 < pairs && e == cudaSuccess; ord0 += pl.wave) {
+      const int np = static_cast<int>(pairs - ord0 < pl.wave ? pairs - ord0 : pl.wave);
+      e = hnd::launch_rowfwd(a, nl, zt, ord0, np, rp_total);
+      if (e == cudaSuccess) e = pl.tier == kMulti2D ? hnd::launch_mid1(a, zt, ord0, np) : hnd::launch_mid2(a, zt, ord0, np);
+      if (e == cudaSuccess) e = hnd::launch_rowinv(a, nl, zt, ord0, np, rp_total);
+      launches += 3;
+    }
+  }
+  if (e != cudaSuccess) return HYENA_ND_ERR_CUDA;
+  g_last_launches = launches;
+  return HYENA_ND_OK;
+}
+
+hyena_nd_status hyena_nd_fftconv(const hyena_nd_problem* p, const void* q, const void* k, const void* v,
+                                 const void* spectrum_c, void* y, void* ws, size_t ws_bytes, void* cuda_stream) {
+  if (!p) return HYENA_ND_ERR_INVALID_ARG;
+  if (p->B != 1 || p->C != 1) return HYENA_ND_ERR_INVALID_ARG;
+  return hyena_nd_fftconv_batched(p, q, k, v, spectrum_c, 0, y, ws, ws_bytes, cuda_stream);
+}
+
+hyena_nd_status hyena_nd_filter_spectrum(const hyena_nd_problem* p, const hyena_nd_filter* f, void* spectrum,
+                                         void* ws, size_t ws_bytes, void* cuda_stream) {
+  Plan pl;
+  hyena_nd_status st = make_plan(p, &pl);
+  if (st != HYENA_ND_OK) return st;
+  if (!f || !spectrum || !ws || !f->W1 || !f->b1 || !f->W2 || !f->b2 || !f->alpha) return HYENA_ND_ERR_INVALID_ARG;
+  if (f->window != 0) return HYENA_ND_ERR_UNSUPPORTED;
+  if (f->num_freqs < 1 || f->num_freqs > 16 || f->hidden < 1 || f->hidden > 128) return HYENA_ND_ERR_UNSUPPORTED;
+  if (!(f->decay_scale > 0.f) || !std::isfinite(f->decay_scale)) return HYENA_ND_ERR_INVALID_ARG;
+  if (!aligned16(spectrum) || !aligned16(ws)) return HYENA_ND_ERR_MISALIGNED;
+  const void* wp[5] = {f->W1, f->b1, f->W2, f->b2, f->alpha};
+  for (const void* w : wp)
+    if (reinterpret_cast<uintptr_t>(w) & 3u) return HYENA_ND_ERR_MISALIGNED;
+  if (ws_bytes < pl.ws_total) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
+  hnd::FilterLaunch fl;
+  fl.W1 = f->W1;
+  fl.b1 = f->b1;
+  fl.W2 = f->W2;
+  fl.b2 = f->b2;
+  fl.alpha = f->alpha;
+  fl.num_freqs = f->num_freqs;
+  fl.hidden = f->hidden;
+  fl.decay_scale = f->decay_scale;
+  float2* grid = reinterpret_cast<float2*>(static_cast<char*>(ws) + kStatusBytes);
+  for (long long c0 = 0; c0 < pl.C; c0 += pl.filter_chunk) {
+    const int nc = static_cast<int>(pl.C - c0 < pl.filter_chunk ? pl.C - c0 : pl.filter_chunk);
+    cudaError_t e = hnd::launch_filter_chunk(fl, pl.ndim, pl.n, static_cast<int>(c0), nc, grid, spectrum,
+                                             static_cast<cudaStream_t>(cuda_stream));
+    if (e != cudaSuccess) return HYENA_ND_ERR_CUDA;
+  }
+  return HYENA_ND_OK;
+}
+
+static hyena_nd_status spec_convert(const hyena_nd_problem* p, const void* src, void* dst, bool to_natural,
+                                    void* cuda_stream) {
+  Plan pl;
+  hyena_nd_status st = make_plan(p, &pl);
+  if (st != HYENA_ND_OK) return st;
+  if (!src || !dst) return HYENA_ND_ERR_INVALID_ARG;
+  if (!aligned16(src) || !aligned16(dst)) return HYENA_ND_ERR_MISALIGNED;
+  if (overlaps(src, dst, pl.spec_bytes)) return HYENA_ND_ERR_INVALID_ARG;
+  return cuda_status(hnd::launch_spec_convert(pl.ndim, pl.n, pl.C, src, dst, to_natural,
+                                              static_cast<cudaStream_t>(cuda_stream)));
+}
+
+hyena_nd_status hyena_nd_spectrum_export(const hyena_nd_problem* p, const void* spectrum, void* natural_c64,
+                                         void* cuda_stream) {
+  return spec_convert(p, spectrum, natural_c64, true, cuda_stream);
+}
+
+hyena_nd_status hyena_nd_spectrum_import(const hyena_nd_problem* p, const void* natural_c64, void* spectrum,
+                                         void* cuda_stream) {
+  return spec_convert(p, natural_c64, spectrum, false, cuda_stream);
+}
+
+hyena_nd_status hyena_nd_device_status(void* ws, void* cuda_stream) {
+  if (!ws) return HYENA_ND_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return HYENA_ND_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return HYENA_ND_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return HYENA_ND_ERR_CUDA;
+  if (v != 0 && cudaMemset(ws, 0, sizeof(int)) != cudaSuccess) return HYENA_ND_ERR_CUDA;
+  if (v < 0 || v > HYENA_ND_ERR_DEVICE_BOUNDS) return HYENA_ND_ERR_CUDA;
+  return static_cast<hyena_nd_status>(v);
+}
+
+hyena_nd_status hyena_nd_debug_bounded_wait(void* ws, size_t ws_bytes, int limit_us, void* cuda_stream) {
+  if (!ws) return HYENA_ND_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return HYENA_ND_ERR_MISALIGNED;
+  if (ws_bytes < kStatusBytes) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
+  if (limit_us < 1 || limit_us > 1000000) return HYENA_ND_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  int* status = static_cast<int*>(ws);
+  int* flag = status + 1;                       // never set by anyone
+  if (cudaMemsetAsync(flag, 0, sizeof(int), s) != cudaSuccess) return HYENA_ND_ERR_CUDA;
+  const long long limit_cycles = static_cast<long long>(limit_us) * 2000;   // about 2 GHz
+  return cuda_status(hnd::launch_bounded_wait(status, flag, limit_cycles, s));
+}
+
+const char* hyena_nd_status_string(hyena_nd_status s) {
+  switch (s) {
+    case HYENA_ND_OK: return "HYENA_ND_OK";
+    case HYENA_ND_ERR_INVALID_ARG: return "HYENA_ND_ERR_INVALID_ARG";
+    case HYENA_ND_ERR_UNSUPPORTED: return "HYENA_ND_ERR_UNSUPPORTED";
+    case HYENA_ND_ERR_MISALIGNED: return "HYENA_ND_ERR_MISALIGNED";
+    case HYENA_ND_ERR_WORKSPACE_TOO_SMALL: return "HYENA_ND_ERR_WORKSPACE_TOO_SMALL";
+    case HYENA_ND_ERR_CUDA: return "HYENA_ND_ERR_CUDA";
+    case HYENA_ND_ERR_DEVICE_TIMEOUT: return "HYENA_ND_ERR_DEVICE_TIMEOUT";
+    case HYENA_ND_ERR_DEVICE_BOUNDS: return "HYENA_ND_ERR_DEVICE_BOUNDS";
+  }
+  return "HYENA_ND_ERR_UNKNOWN";
+}
+
+int hyena_nd_last_launch_count(void) { return g_last_launches; }
+
+}  // extern "C"

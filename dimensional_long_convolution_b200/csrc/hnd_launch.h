@@ -1,0 +1,53 @@
+// hnd_launch.h -- host-side launchers shared by the instantiation units and
+// the C ABI (hnd_api.cu).  Each launcher switches on the runtime sizes and
+// returns cudaErrorInvalidValue for a size it has no instantiation for.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace hnd {
+
+struct ConvArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* spec;
+  long long sbs;          // per-sample spectrum stride in complex elements (0 = shared)
+  void* y;
+  int B, C;
+  int bf16;               // 0 = fp32 activations, 1 = bf16
+  int n[3];
+  int ndim;
+  cudaStream_t stream;
+};
+
+// Maximum dynamic shared memory per CTA on sm_100 (227 KB).
+constexpr size_t kMaxSmem = 232448;
+
+// Fused tiers (one launch).
+cudaError_t launch_fused2d(const ConvArgs& a);
+cudaError_t launch_rows1d(const ConvArgs& a);
+size_t fused2d_smem(int n0, int n1);
+
+// Multi-pass tier, one wave of pairs [ord0, ord0 + np) in channel-major order.
+cudaError_t launch_rowfwd(const ConvArgs& a, int nl, float2* zt, long long ord0, int np, int rp_total);
+cudaError_t launch_rowinv(const ConvArgs& a, int nl, const float2* zt, long long ord0, int np, int rp_total);
+cudaError_t launch_mid1(const ConvArgs& a, float2* zt, long long ord0, int np);
+cudaError_t launch_mid2(const ConvArgs& a, float2* zt, long long ord0, int np);
+size_t mid2_smem(int n0, int n1, bool* pair_variant);
+
+// Filter spectrum and layout conversion.
+struct FilterLaunch {
+  const float *W1, *b1, *W2, *b2, *alpha;
+  int num_freqs, hidden;
+  float decay_scale;
+};
+cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, int c0, int nc, float2* grid,
+                                void* spectrum, cudaStream_t st);
+cudaError_t launch_spec_convert(int ndim, const int* n, long long C, const void* src, void* dst, bool to_natural,
+                                cudaStream_t st);
+cudaError_t launch_bounded_wait(int* status, const int* flag, long long limit_cycles, cudaStream_t st);
+
+}  // namespace hnd

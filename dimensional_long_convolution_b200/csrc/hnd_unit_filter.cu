@@ -1,0 +1,78 @@
+// Filter spectrum (call 1), spectrum layout conversion, diagnostics.
+#include "hnd_kernels.cuh"
+#include "hnd_launch.h"
+#include "hnd_host_util.h"
+
+namespace hnd {
+
+static SpecDims make_dims(int ndim, const int* n) {
+  SpecDims d;
+  d.ndim = ndim;
+  for (int a = 0; a < 3; ++a) d.n[a] = a < ndim ? n[a] : 1;
+  return d;
+}
+
+static unsigned grid_for(long long work, int threads) {
+  long long b = (work + threads - 1) / threads;
+  if (b < 1) b = 1;
+  if (b > 148LL * 32) b = 148LL * 32;
+  return static_cast<unsigned>(b);
+}
+
+cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, int c0, int nc, float2* grid,
+                                void* spectrum, cudaStream_t st) {
+  const SpecDims d = make_dims(ndim, n);
+  long long gsz = 1, noff = 1;
+  for (int a = 0; a < ndim; ++a) {
+    gsz *= 2 * n[a];
+    noff *= 2 * n[a] - 1;
+  }
+  cudaError_t e = cudaMemsetAsync(grid, 0, sizeof(float2) * gsz * nc, st);
+  if (e != cudaSuccess) return e;
+  FilterArgs fa;
+  fa.W1 = f.W1;
+  fa.b1 = f.b1;
+  fa.W2 = f.W2;
+  fa.b2 = f.b2;
+  fa.alpha = f.alpha;
+  fa.num_freqs = f.num_freqs;
+  fa.hidden = f.hidden;
+  fa.fin = 2 * f.num_freqs * ndim;
+  fa.decay_scale = f.decay_scale;
+  k_filter_mlp<<<grid_for(noff, 128), 128, 0, st>>>(fa, d, c0, nc, grid);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  long long stride = gsz;
+  for (int a = 0; a < ndim; ++a) {
+    const int P = 2 * n[a];
+    stride /= P;
+    int logP = 0;
+    while ((1 << logP) < P) ++logP;
+    const long long npen = gsz * nc / P;
+    const long long per_cta = 512 / P;
+    k_fft_axis<<<static_cast<unsigned>((npen + per_cta - 1) / per_cta), 256, 0, st>>>(grid, P, logP, stride, npen);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  const long long per = spec_per_channel(d);
+  k_spec_pack<<<grid_for(per * nc, 256), 256, 0, st>>>(grid, static_cast<float2*>(spectrum), d, c0, nc,
+                                                       static_cast<float>(1.0 / static_cast<double>(gsz)));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_spec_convert(int ndim, const int* n, long long C, const void* src, void* dst, bool to_natural,
+                                cudaStream_t st) {
+  const SpecDims d = make_dims(ndim, n);
+  const long long total = spec_per_channel(d) * C;
+  if (to_natural)
+    k_spec_export<<<grid_for(total, 256), 256, 0, st>>>(static_cast<const float2*>(src), static_cast<float2*>(dst), d, C);
+  else
+    k_spec_import<<<grid_for(total, 256), 256, 0, st>>>(static_cast<const float2*>(src), static_cast<float2*>(dst), d, C);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bounded_wait(int* status, const int* flag, long long limit_cycles, cudaStream_t st) {
+  const long long max_it = limit_cycles / 1000 + 16;
+  k_bounded_wait<<<1, 32, 0, st>>>(status, flag, limit_cycles, max_it);
+  return cudaGetLastError();
+}
+
+}  // namespace hnd

@@ -1,0 +1,77 @@
+// Instantiations: multi-pass column stages (2D pencils, 3D slabs).
+#include "hnd_kernels.cuh"
+#include "hnd_launch.h"
+#include "hnd_host_util.h"
+
+namespace hnd {
+
+template <int N0>
+static cudaError_t mid1_go(const ConvArgs& a, float2* zt, long long ord0, int np) {
+  auto kern = k_mid1<N0>;
+  const size_t sm = kMidSmemBase;
+  cudaError_t e = ensure_smem(kern, sm);
+  if (e != cudaSuccess) return e;
+  constexpr int PPW = 32 / (N0 / 8);
+  const int n1 = a.n[1];
+  dim3 grid(np, (n1 + kWarps * PPW - 1) / (kWarps * PPW));
+  kern<<<grid, kThreads, sm, a.stream>>>(zt, static_cast<const float2*>(a.spec), a.sbs, n1, ord0, a.B, a.C);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mid1(const ConvArgs& a, float2* zt, long long ord0, int np) {
+  switch (a.n[0]) {
+    case 8: return mid1_go<8>(a, zt, ord0, np);
+    case 16: return mid1_go<16>(a, zt, ord0, np);
+    case 32: return mid1_go<32>(a, zt, ord0, np);
+    case 64: return mid1_go<64>(a, zt, ord0, np);
+    case 128: return mid1_go<128>(a, zt, ord0, np);
+    case 256: return mid1_go<256>(a, zt, ord0, np);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int N0, int N1>
+static cudaError_t mid2_go(const ConvArgs& a, float2* zt, long long ord0, int np) {
+  const int n2 = a.n[2];
+  if (SlabSmem<N0, N1>::kBytes <= kMaxSmem) {
+    auto kern = k_mid2<N0, N1>;
+    const size_t sm = SlabSmem<N0, N1>::kBytes;
+    cudaError_t e = ensure_smem(kern, sm);
+    if (e != cudaSuccess) return e;
+    dim3 grid(np, n2 + 1);
+    kern<<<grid, kThreads, sm, a.stream>>>(zt, static_cast<const float2*>(a.spec), a.sbs, n2, ord0, a.B, a.C);
+  } else {
+    auto kern = k_mid2_pair<N0, N1>;
+    const size_t sm = SlabSmem<N0, N1>::kHalfBytes;
+    cudaError_t e = ensure_smem(kern, sm);
+    if (e != cudaSuccess) return e;
+    dim3 grid(2 * np, n2 + 1);
+    kern<<<grid, kThreads, sm, a.stream>>>(zt, static_cast<const float2*>(a.spec), a.sbs, n2, ord0, a.B, a.C);
+  }
+  return cudaGetLastError();
+}
+
+template <int N0>
+static cudaError_t mid2_n1(const ConvArgs& a, float2* zt, long long ord0, int np) {
+  switch (a.n[1]) {
+    case 8: return mid2_go<N0, 8>(a, zt, ord0, np);
+    case 16: return mid2_go<N0, 16>(a, zt, ord0, np);
+    case 32: return mid2_go<N0, 32>(a, zt, ord0, np);
+    case 64: return mid2_go<N0, 64>(a, zt, ord0, np);
+    case 128: return mid2_go<N0, 128>(a, zt, ord0, np);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_mid2(const ConvArgs& a, float2* zt, long long ord0, int np) {
+  switch (a.n[0]) {
+    case 8: return mid2_n1<8>(a, zt, ord0, np);
+    case 16: return mid2_n1<16>(a, zt, ord0, np);
+    case 32: return mid2_n1<32>(a, zt, ord0, np);
+    case 64: return mid2_n1<64>(a, zt, ord0, np);
+    case 128: return mid2_n1<128>(a, zt, ord0, np);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace hnd

@@ -1,0 +1,95 @@
+// Instantiations: 1D fused rows, multi-pass row stages.
+#include "hnd_kernels.cuh"
+#include "hnd_launch.h"
+#include "hnd_host_util.h"
+
+namespace hnd {
+
+template <int N, class IO>
+static cudaError_t rows1d_go(const ConvArgs& a) {
+  using TT = typename IO::T;
+  auto kern = k_rows1d<N, IO>;
+  const size_t sm = kMidSmemBase;
+  cudaError_t e = ensure_smem(kern, sm);
+  if (e != cudaSuccess) return e;
+  constexpr int PPW = 32 / (N / 8);
+  const long long rpairs = (static_cast<long long>(a.B) * a.C + 1) / 2;
+  long long blocks = (rpairs + kWarps * PPW - 1) / (kWarps * PPW);
+  if (blocks > 148LL * 64) blocks = 148LL * 64;
+  kern<<<static_cast<unsigned>(blocks), kThreads, sm, a.stream>>>(
+      static_cast<const TT*>(a.q), static_cast<const TT*>(a.k), static_cast<const TT*>(a.v),
+      static_cast<const float2*>(a.spec), a.sbs, static_cast<TT*>(a.y), a.B, a.C);
+  return cudaGetLastError();
+}
+
+template <class IO>
+static cudaError_t rows1d_io(const ConvArgs& a) {
+  switch (a.n[0]) {
+    case 8: return rows1d_go<8, IO>(a);
+    case 16: return rows1d_go<16, IO>(a);
+    case 32: return rows1d_go<32, IO>(a);
+    case 64: return rows1d_go<64, IO>(a);
+    case 128: return rows1d_go<128, IO>(a);
+    case 256: return rows1d_go<256, IO>(a);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_rows1d(const ConvArgs& a) { return a.bf16 ? rows1d_io<IOBF16>(a) : rows1d_io<IOF32>(a); }
+
+template <int NL, class IO>
+static cudaError_t rowfwd_go(const ConvArgs& a, float2* zt, long long ord0, int np, int rp_total) {
+  using TT = typename IO::T;
+  auto kern = k_rowfwd<NL, IO>;
+  const size_t sm = RowTile<NL>::kBytes;
+  cudaError_t e = ensure_smem(kern, sm);
+  if (e != cudaSuccess) return e;
+  constexpr int RPB = RowTile<NL>::RPB;
+  dim3 grid(np, (rp_total + RPB - 1) / RPB);
+  kern<<<grid, kThreads, sm, a.stream>>>(static_cast<const TT*>(a.k), static_cast<const TT*>(a.v), zt, ord0,
+                                         rp_total, a.B, a.C);
+  return cudaGetLastError();
+}
+
+template <int NL, class IO>
+static cudaError_t rowinv_go(const ConvArgs& a, const float2* zt, long long ord0, int np, int rp_total) {
+  using TT = typename IO::T;
+  auto kern = k_rowinv<NL, IO>;
+  const size_t sm = RowTile<NL>::kBytes;
+  cudaError_t e = ensure_smem(kern, sm);
+  if (e != cudaSuccess) return e;
+  constexpr int RPB = RowTile<NL>::RPB;
+  dim3 grid(np, (rp_total + RPB - 1) / RPB);
+  kern<<<grid, kThreads, sm, a.stream>>>(zt, static_cast<const TT*>(a.q), static_cast<TT*>(a.y), ord0, rp_total,
+                                         a.B, a.C);
+  return cudaGetLastError();
+}
+
+#define HND_ROWS_SWITCH(FN, IO, ...)                  \
+  switch (nl) {                                       \
+    case 8: return FN<8, IO>(__VA_ARGS__);            \
+    case 16: return FN<16, IO>(__VA_ARGS__);          \
+    case 32: return FN<32, IO>(__VA_ARGS__);          \
+    case 64: return FN<64, IO>(__VA_ARGS__);          \
+    case 128: return FN<128, IO>(__VA_ARGS__);        \
+    case 256: return FN<256, IO>(__VA_ARGS__);        \
+    default: return cudaErrorInvalidValue;            \
+  }
+
+cudaError_t launch_rowfwd(const ConvArgs& a, int nl, float2* zt, long long ord0, int np, int rp_total) {
+  if (a.bf16) {
+    HND_ROWS_SWITCH(rowfwd_go, IOBF16, a, zt, ord0, np, rp_total)
+  } else {
+    HND_ROWS_SWITCH(rowfwd_go, IOF32, a, zt, ord0, np, rp_total)
+  }
+}
+
+cudaError_t launch_rowinv(const ConvArgs& a, int nl, const float2* zt, long long ord0, int np, int rp_total) {
+  if (a.bf16) {
+    HND_ROWS_SWITCH(rowinv_go, IOBF16, a, zt, ord0, np, rp_total)
+  } else {
+    HND_ROWS_SWITCH(rowinv_go, IOF32, a, zt, ord0, np, rp_total)
+  }
+}
+
+}  // namespace hnd

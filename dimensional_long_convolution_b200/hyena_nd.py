@@ -1,0 +1,247 @@
+"""Thin ctypes binding of libhyena_nd.so (the C ABI in include/hyena_nd.h).
+
+Argument marshalling only: every step of the convolution runs in the CUDA
+kernels of the shared library.  The functions carry the C names without the
+``hyena_nd_`` prefix and take raw integers (device pointers, byte counts,
+stream handles).  ``HyenaND`` below wraps them for torch tensors: torch
+provides device memory and the current stream, nothing else.
+
+Importing this module never falls back to anything: if the shared library is
+missing or fails to load, ``load()`` raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhyena_nd.so")
+
+OK = 0
+ERR_INVALID_ARG = 1
+ERR_UNSUPPORTED = 2
+ERR_MISALIGNED = 3
+ERR_WORKSPACE_TOO_SMALL = 4
+ERR_CUDA = 5
+ERR_DEVICE_TIMEOUT = 6
+ERR_DEVICE_BOUNDS = 7
+
+F32 = 0
+BF16 = 1
+
+EXPORTED = (
+    "hyena_nd_spectrum_bytes",
+    "hyena_nd_workspace_bytes",
+    "hyena_nd_workspace_init",
+    "hyena_nd_filter_spectrum",
+    "hyena_nd_fftconv",
+    "hyena_nd_fftconv_batched",
+    "hyena_nd_spectrum_export",
+    "hyena_nd_spectrum_import",
+    "hyena_nd_device_status",
+    "hyena_nd_debug_bounded_wait",
+    "hyena_nd_status_string",
+    "hyena_nd_last_launch_count",
+)
+
+
+class Problem(ctypes.Structure):
+    _fields_ = [
+        ("ndim", ctypes.c_int),
+        ("n", ctypes.c_int64 * 3),
+        ("B", ctypes.c_int64),
+        ("C", ctypes.c_int64),
+        ("io_dtype", ctypes.c_int),
+        ("circular", ctypes.c_int),
+    ]
+
+
+class Filter(ctypes.Structure):
+    _fields_ = [
+        ("num_freqs", ctypes.c_int),
+        ("hidden", ctypes.c_int),
+        ("W1", ctypes.c_void_p),
+        ("b1", ctypes.c_void_p),
+        ("W2", ctypes.c_void_p),
+        ("b2", ctypes.c_void_p),
+        ("alpha", ctypes.c_void_p),
+        ("decay_scale", ctypes.c_float),
+        ("window", ctypes.c_int),
+    ]
+
+
+class HyenaNDError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__("%s failed: %s" % (what, status_string(code)))
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the shared library (once).  Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError("libhyena_nd.so not built at %s (run python -m dimensional_long_convolution_b200.build)" % path)
+    lib = ctypes.CDLL(path)
+    P = ctypes.POINTER(Problem)
+    vp, sz, i64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int64
+    sigs = {
+        "hyena_nd_spectrum_bytes": (sz, [P]),
+        "hyena_nd_workspace_bytes": (sz, [P]),
+        "hyena_nd_workspace_init": (ctypes.c_int, [vp, sz, vp]),
+        "hyena_nd_filter_spectrum": (ctypes.c_int, [P, ctypes.POINTER(Filter), vp, vp, sz, vp]),
+        "hyena_nd_fftconv": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "hyena_nd_fftconv_batched": (ctypes.c_int, [P, vp, vp, vp, vp, i64, vp, vp, sz, vp]),
+        "hyena_nd_spectrum_export": (ctypes.c_int, [P, vp, vp, vp]),
+        "hyena_nd_spectrum_import": (ctypes.c_int, [P, vp, vp, vp]),
+        "hyena_nd_device_status": (ctypes.c_int, [vp, vp]),
+        "hyena_nd_debug_bounded_wait": (ctypes.c_int, [vp, sz, ctypes.c_int, vp]),
+        "hyena_nd_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "hyena_nd_last_launch_count": (ctypes.c_int, []),
+    }
+    for name, (res, args) in sigs.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def problem(dims: Sequence[int], B: int, C: int, io_dtype: int = F32, circular: int = 0) -> Problem:
+    p = Problem()
+    p.ndim = len(dims)
+    for i in range(3):
+        p.n[i] = int(dims[i]) if i < len(dims) else 0
+    p.B, p.C, p.io_dtype, p.circular = int(B), int(C), int(io_dtype), int(circular)
+    return p
+
+
+# ------------------------------------------------------------ raw C calls
+def spectrum_bytes(p: Problem) -> int:
+    return int(load().hyena_nd_spectrum_bytes(ctypes.byref(p)))
+
+
+def workspace_bytes(p: Problem) -> int:
+    return int(load().hyena_nd_workspace_bytes(ctypes.byref(p)))
+
+
+def workspace_init(ws: int, ws_bytes: int, stream: int = 0) -> int:
+    return load().hyena_nd_workspace_init(ws, ws_bytes, stream)
+
+
+def filter_spectrum(p: Problem, f: Filter, spectrum: int, ws: int, ws_bytes: int, stream: int = 0) -> int:
+    return load().hyena_nd_filter_spectrum(ctypes.byref(p), ctypes.byref(f), spectrum, ws, ws_bytes, stream)
+
+
+def fftconv(p: Problem, q: int, k: int, v: int, spectrum_c: int, y: int, ws: int, ws_bytes: int,
+            stream: int = 0) -> int:
+    return load().hyena_nd_fftconv(ctypes.byref(p), q, k, v, spectrum_c, y, ws, ws_bytes, stream)
+
+
+def fftconv_batched(p: Problem, q: int, k: int, v: int, spectrum: int, spectrum_batch_stride: int, y: int,
+                    ws: int, ws_bytes: int, stream: int = 0) -> int:
+    return load().hyena_nd_fftconv_batched(ctypes.byref(p), q, k, v, spectrum, spectrum_batch_stride, y, ws,
+                                           ws_bytes, stream)
+
+
+def spectrum_export(p: Problem, spectrum: int, natural: int, stream: int = 0) -> int:
+    return load().hyena_nd_spectrum_export(ctypes.byref(p), spectrum, natural, stream)
+
+
+def spectrum_import(p: Problem, natural: int, spectrum: int, stream: int = 0) -> int:
+    return load().hyena_nd_spectrum_import(ctypes.byref(p), natural, spectrum, stream)
+
+
+def device_status(ws: int, stream: int = 0) -> int:
+    return load().hyena_nd_device_status(ws, stream)
+
+
+def debug_bounded_wait(ws: int, ws_bytes: int, limit_us: int, stream: int = 0) -> int:
+    return load().hyena_nd_debug_bounded_wait(ws, ws_bytes, int(limit_us), stream)
+
+
+def status_string(code: int) -> str:
+    return load().hyena_nd_status_string(int(code)).decode()
+
+
+def last_launch_count() -> int:
+    return int(load().hyena_nd_last_launch_count())
+
+
+def check(code: int, what: str) -> None:
+    if code != OK:
+        raise HyenaNDError(code, what)
+
+
+# ------------------------------------------------------------ torch wrapper
+class HyenaND:
+    """One problem shape bound to a device: owns the spectrum and workspace
+    tensors (allocated by torch) and calls the C ABI on the current stream."""
+
+    def __init__(self, dims: Sequence[int], B: int, C: int, io_dtype: str = "f32", device=None):
+        import torch
+
+        self.torch = torch
+        self.dims = tuple(int(d) for d in dims)
+        self.B, self.C = int(B), int(C)
+        self.io_dtype = io_dtype
+        self.tdtype = torch.bfloat16 if io_dtype == "bf16" else torch.float32
+        self.p = problem(self.dims, B, C, BF16 if io_dtype == "bf16" else F32)
+        self.device = torch.device(device if device is not None else "cuda")
+        nbytes = workspace_bytes(self.p)
+        if nbytes == 0:
+            raise HyenaNDError(ERR_UNSUPPORTED, "workspace_bytes")
+        self.ws_bytes = nbytes
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        self.spec_bytes = spectrum_bytes(self.p)
+        self.spectrum = torch.empty(self.spec_bytes // 8, dtype=torch.complex64, device=self.device)
+        check(workspace_init(self.ws.data_ptr(), nbytes, self._stream()), "workspace_init")
+
+    def _stream(self) -> int:
+        return int(self.torch.cuda.current_stream(self.device).cuda_stream)
+
+    def natural_shape(self):
+        P = [2 * n for n in self.dims]
+        return (self.C,) + tuple(P[:-1]) + (self.dims[-1] + 1,)
+
+    def set_filter(self, W1, b1, W2, b2, alpha, decay_scale: float, num_freqs: int = 8) -> None:
+        t = [x.to(self.device, self.torch.float32).contiguous() for x in (W1, b1, W2, b2, alpha)]
+        self._filter_params = t        # keep alive until the call has run
+        f = Filter()
+        f.num_freqs = int(num_freqs)
+        f.hidden = int(t[0].shape[0])
+        f.W1, f.b1, f.W2, f.b2, f.alpha = (x.data_ptr() for x in t)
+        f.decay_scale = float(decay_scale)
+        f.window = 0
+        check(filter_spectrum(self.p, f, self.spectrum.data_ptr(), self.ws.data_ptr(), self.ws_bytes,
+                              self._stream()), "filter_spectrum")
+
+    def import_spectrum(self, natural) -> None:
+        nat = natural.to(self.device, self.torch.complex64).contiguous()
+        check(spectrum_import(self.p, nat.data_ptr(), self.spectrum.data_ptr(), self._stream()), "spectrum_import")
+        self._import_keep = nat
+
+    def export_spectrum(self):
+        out = self.torch.empty(self.natural_shape(), dtype=self.torch.complex64, device=self.device)
+        check(spectrum_export(self.p, self.spectrum.data_ptr(), out.data_ptr(), self._stream()), "spectrum_export")
+        return out
+
+    def __call__(self, q, k, v, y=None, spectrum=None, spectrum_batch_stride: int = 0):
+        for t in (q, k, v):
+            if t.dtype != self.tdtype or not t.is_contiguous() or t.device != self.device:
+                raise ValueError("q, k, v must be contiguous %s tensors on %s" % (self.tdtype, self.device))
+        if y is None:
+            y = self.torch.empty_like(q)
+        spec = self.spectrum if spectrum is None else spectrum
+        check(fftconv_batched(self.p, q.data_ptr(), k.data_ptr(), v.data_ptr(), spec.data_ptr(),
+                              int(spectrum_batch_stride), y.data_ptr(), self.ws.data_ptr(), self.ws_bytes,
+                              self._stream()), "fftconv_batched")
+        return y
+
+    def status(self) -> int:
+        return device_status(self.ws.data_ptr(), self._stream())

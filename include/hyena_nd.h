@@ -1,0 +1,177 @@
+/*
+ * hyena_nd.h -- C ABI of the B200 (sm_100a) gated nD FFT long-convolution library.
+ *
+ * The operation (HyenaND pages):
+ *   * autognosis blog "Native multi-dimensional subquadratic operators via
+ *     input-dependent long convolutions", section "HyenaND", output equation
+ *     y[i] = sum_j phi(x[j]) x[j] K[i - j]: a global convolution of a gated input
+ *     with an implicitly parameterised kernel, evaluated through FFTs.
+ *   * gist.science summary of arXiv 2607.19378, section "Methodologie": native
+ *     N-dimensional grids L1 x ... x LN (no rasterisation), a kernel given by a
+ *     sine-activated coordinate MLP times a window, and zero padding to twice
+ *     the grid for the non-circular (linear) convolution; section
+ *     "Implementation: nSubQ": forward FFT, spectral modulation, inverse FFT and
+ *     output cropping fused in one kernel with intermediates kept on chip.
+ *
+ * In Hyena form, per batch b and channel c, with u = k (.) v:
+ *     y[b,c,i] = q[b,c,i] * sum_{j in [0,n)^d} u[b,c,j] * K_c[i - j],   i in [0,n)^d,
+ * where K_c is defined on every offset t in [-(n_a - 1), n_a - 1] per axis.
+ *
+ * Conventions shared by every call:
+ *   * All device memory is owned by the caller; the library never allocates
+ *     or frees.  Every call is asynchronous on the given CUDA stream
+ *     (cudaStream_t passed as void*; NULL = legacy default stream) and
+ *     performs no host synchronisation, except hyena_nd_device_status.
+ *   * Argument errors are detected on the host before anything is launched
+ *     and returned synchronously.  A failed launch returns HYENA_ND_ERR_CUDA.
+ *     Errors detected on the device are written to a status word held in the
+ *     first 16 bytes of the workspace and read by hyena_nd_device_status.
+ *   * Activations q, k, v, y: contiguous [B, C, n_1, ..., n_d], last axis
+ *     fastest, all of one dtype (fp32 or bf16; bf16 outputs are rounded to
+ *     nearest even).  Arithmetic is fp32 throughout.
+ *   * Every device pointer must be 16-byte aligned.
+ *   * The spectrum is complex64 in an order private to this library: write it
+ *     with hyena_nd_filter_spectrum or hyena_nd_spectrum_import and read it
+ *     back with hyena_nd_spectrum_export.  It already carries the inverse
+ *     transform's 1 / prod(P) scale (P_a = 2 n_a).
+ */
+#ifndef HYENA_ND_H_
+#define HYENA_ND_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HYENA_ND_API __attribute__((visibility("default")))
+#else
+#define HYENA_ND_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HYENA_ND_OK = 0,
+  HYENA_ND_ERR_INVALID_ARG = 1,        /* null pointer, bad rank, B or C < 1, ... */
+  HYENA_ND_ERR_UNSUPPORTED = 2,        /* valid problem outside the supported sizes */
+  HYENA_ND_ERR_MISALIGNED = 3,         /* a device pointer is not 16-byte aligned */
+  HYENA_ND_ERR_WORKSPACE_TOO_SMALL = 4,
+  HYENA_ND_ERR_CUDA = 5,               /* a CUDA runtime call or launch failed */
+  HYENA_ND_ERR_DEVICE_TIMEOUT = 6,     /* a bounded device-side wait gave up */
+  HYENA_ND_ERR_DEVICE_BOUNDS = 7       /* a checked build caught an out-of-range index */
+} hyena_nd_status;
+
+typedef enum { HYENA_ND_F32 = 0, HYENA_ND_BF16 = 1 } hyena_nd_dtype;
+
+/* Problem descriptor.
+ *   ndim     1, 2 or 3.
+ *   n[a]     grid extent of axis a (a < ndim), a power of two in [8, 256];
+ *            for ndim == 3 the two outer axes are limited to [8, 128].
+ *   B, C     batch and channel counts (>= 1).
+ *   io_dtype dtype of q, k, v and y.
+ *   circular must be 0 (zero-padded linear convolution); the periodic mode of
+ *            the pages is not implemented and returns HYENA_ND_ERR_UNSUPPORTED. */
+typedef struct {
+  int ndim;
+  int64_t n[3];
+  int64_t B, C;
+  hyena_nd_dtype io_dtype;
+  int circular;
+} hyena_nd_problem;
+
+/* Implicit filter (pages: coordinate MLP with sine activation times a window).
+ * For every offset t in [-(n_a-1), n_a-1]^d:
+ *   phi(t)  = [sin(pi m t_a / n_a), cos(pi m t_a / n_a)] for a < ndim, m = 1..num_freqs,
+ *             ordered [axis][m][sin, cos]            (2 * num_freqs * ndim features)
+ *   h       = sin(W1 phi + b1)                       (hidden units)
+ *   K_c(t)  = ((W2 h + b2)_c) * exp(-alpha_c * ||t||_2 / decay_scale)
+ * Device pointers, fp32, row-major: W1 [hidden, 2*num_freqs*ndim], b1 [hidden],
+ * W2 [C, hidden], b2 [C], alpha [C].  Limits: 1 <= num_freqs <= 16,
+ * 1 <= hidden <= 128, decay_scale > 0.  window must be 0 (exponential decay);
+ * the Gaussian window of the pages is not implemented (HYENA_ND_ERR_UNSUPPORTED). */
+typedef struct {
+  int num_freqs;
+  int hidden;
+  const float *W1, *b1, *W2, *b2, *alpha;
+  float decay_scale;
+  int window;
+} hyena_nd_filter;
+
+/* Size in bytes of the spectrum buffer for `p` (C channels of
+ * prod_{a<d-1} P_a * (P_d/2 + 1) complex64 values).  0 if `p` is invalid. */
+HYENA_ND_API size_t hyena_nd_spectrum_bytes(const hyena_nd_problem* p);
+
+/* Workspace bytes needed by every call below for problem `p` (a pure
+ * function of the descriptor, at least 256 bytes; the first 16 bytes hold the
+ * device status word).  0 if `p` is invalid or unsupported.  The same
+ * workspace may be reused by consecutive calls on one stream. */
+HYENA_ND_API size_t hyena_nd_workspace_bytes(const hyena_nd_problem* p);
+
+/* Clear the device status word (enqueues a 16-byte memset on `stream`).  Call
+ * once on a fresh workspace before the first call that uses it. */
+HYENA_ND_API hyena_nd_status hyena_nd_workspace_init(void* ws, size_t ws_bytes, void* cuda_stream);
+
+/* Call 1: evaluate the implicit filter on the offset grid, place it on the
+ * zero-padded periodic grid P^d (offset t at slot t mod P_a, slot n_a zero),
+ * take its real-input DFT, scale by 1/prod(P) and store it in the library's
+ * spectrum order.  `spectrum`: hyena_nd_spectrum_bytes(p) bytes, written.
+ * Pages: blog sections "nSubQ" (parameter computation) and "Implementation
+ * patterns" (neural parameterisation); arXiv summary "Methodologie". */
+HYENA_ND_API hyena_nd_status hyena_nd_filter_spectrum(const hyena_nd_problem* p, const hyena_nd_filter* f,
+                                         void* spectrum, void* ws, size_t ws_bytes,
+                                         void* cuda_stream);
+
+/* Call 2 (one volume): the gated linear convolution for one (b, c) pair.
+ * `p->B` and `p->C` must both be 1; `spectrum_c` holds that channel's
+ * spectrum.  Same semantics as the batched call. */
+HYENA_ND_API hyena_nd_status hyena_nd_fftconv(const hyena_nd_problem* p, const void* q, const void* k,
+                                 const void* v, const void* spectrum_c, void* y, void* ws,
+                                 size_t ws_bytes, void* cuda_stream);
+
+/* Call 3 (batched over B and C): for every (b, c),
+ *   y[b,c] = q[b,c] (.) crop_n( IFFT_P( FFT_P(pad_P(k[b,c] (.) v[b,c])) (.) S[b,c] ) )
+ * i.e. the linear convolution defined at the top of this header.
+ * q, k, v: read; y: written (may not alias q, k or v); all [B, C, n...].
+ * `spectrum`: C spectra laid out as hyena_nd_filter_spectrum writes them.
+ * `spectrum_batch_stride`: 0 = one spectrum per channel shared by every b;
+ * otherwise sample b uses spectrum + b * spectrum_batch_stride bytes (a
+ * per-sample spectrum set, multiple of 16 bytes).
+ * `ws`: hyena_nd_workspace_bytes(p) bytes of device scratch. */
+HYENA_ND_API hyena_nd_status hyena_nd_fftconv_batched(const hyena_nd_problem* p, const void* q,
+                                         const void* k, const void* v, const void* spectrum,
+                                         int64_t spectrum_batch_stride, void* y, void* ws,
+                                         size_t ws_bytes, void* cuda_stream);
+
+/* Convert between the library's spectrum order and the natural order
+ * [C, P_1, ..., P_{d-1}, P_d/2 + 1] complex64 (scale included, i.e. the
+ * natural array is DFT(wrap-placed K) / prod(P)).  Both buffers are device
+ * memory of hyena_nd_spectrum_bytes(p) bytes and may not alias. */
+HYENA_ND_API hyena_nd_status hyena_nd_spectrum_export(const hyena_nd_problem* p, const void* spectrum,
+                                         void* natural_c64, void* cuda_stream);
+HYENA_ND_API hyena_nd_status hyena_nd_spectrum_import(const hyena_nd_problem* p, const void* natural_c64,
+                                         void* spectrum, void* cuda_stream);
+
+/* Synchronise `stream`, then read and clear the device status word in `ws`.
+ * Returns HYENA_ND_OK, the recorded device error, or HYENA_ND_ERR_CUDA. */
+HYENA_ND_API hyena_nd_status hyena_nd_device_status(void* ws, void* cuda_stream);
+
+/* Test hook for bounded device waits: launches one CTA that waits on a flag
+ * nothing will ever set, with an iteration and clock limit of about
+ * `limit_us` microseconds, after which it records HYENA_ND_ERR_DEVICE_TIMEOUT
+ * in the status word and returns.  It never traps and never hangs. */
+HYENA_ND_API hyena_nd_status hyena_nd_debug_bounded_wait(void* ws, size_t ws_bytes, int limit_us,
+                                            void* cuda_stream);
+
+/* Human-readable name of a status code (static string). */
+HYENA_ND_API const char* hyena_nd_status_string(hyena_nd_status s);
+
+/* Number of kernels the most recent successful call to hyena_nd_fftconv or
+ * hyena_nd_fftconv_batched on this host thread enqueued. */
+HYENA_ND_API int hyena_nd_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HYENA_ND_H_ */

@@ -64,23 +64,28 @@ def fourier_features(t: np.ndarray, dims: Sequence[int], num_freqs: int) -> np.n
     return np.stack(cols, axis=-1)
 
 
-def implicit_kernel(filt, dims: Sequence[int]) -> np.ndarray:
-    """K_c(t) for every channel c and offset t (pages: coordinate MLP with sine
-    activation times a decay window; reading 4).  Computed in float64 from the
-    fp32 parameters.  Returns [C, 2n_1-1, ..., 2n_d-1]; index t + (n - 1)."""
-    t = offsets_grid(dims)
-    phi = fourier_features(t, dims, filt.num_freqs)
+def implicit_kernel(filt, dims: Sequence[int], channels=None, chunk: int = 1 << 18) -> np.ndarray:
+    """K_c(t) for every channel c (or the listed ``channels``) and offset t
+    (pages: coordinate MLP with sine activation times a decay window; reading
+    4).  Computed in float64 from the fp32 parameters, ``chunk`` offsets at a
+    time to bound memory.  Returns [C, 2n_1-1, ..., 2n_d-1]; index t + (n - 1)."""
+    t_all = offsets_grid(dims)
     W1 = filt.W1.astype(np.float64)
     b1 = filt.b1.astype(np.float64)
-    W2 = filt.W2.astype(np.float64)
-    b2 = filt.b2.astype(np.float64)
-    h = np.sin(phi @ W1.T + b1)                      # [N, H]
-    mlp = h @ W2.T + b2                              # [N, C]
-    r = np.sqrt(np.sum(t * t, axis=-1))              # ||t||_2
-    alpha = filt.alpha.astype(np.float64)
-    window = np.exp(-np.outer(r, alpha) / float(filt.decay_scale))
-    K = (mlp * window).T                             # [C, N]
-    return K.reshape((K.shape[0],) + tuple(2 * n - 1 for n in dims))
+    sel = np.arange(filt.W2.shape[0]) if channels is None else np.asarray(channels)
+    W2 = filt.W2.astype(np.float64)[sel]
+    b2 = filt.b2.astype(np.float64)[sel]
+    alpha = filt.alpha.astype(np.float64)[sel]
+    K = np.empty((len(sel), t_all.shape[0]), dtype=np.float64)
+    for s0 in range(0, t_all.shape[0], chunk):
+        t = t_all[s0: s0 + chunk]
+        phi = fourier_features(t, dims, filt.num_freqs)
+        h = np.sin(phi @ W1.T + b1)                      # [N, H]
+        mlp = h @ W2.T + b2                              # [N, C]
+        r = np.sqrt(np.sum(t * t, axis=-1))              # ||t||_2
+        window = np.exp(-np.outer(r, alpha) / float(filt.decay_scale))
+        K[:, s0: s0 + chunk] = (mlp * window).T
+    return K.reshape((len(sel),) + tuple(2 * n - 1 for n in dims))
 
 
 def wrap_place(K: np.ndarray, dims: Sequence[int]) -> np.ndarray:

@@ -1,0 +1,151 @@
+"""Host-only checks of the C ABI: the library loads, exports every symbol that
+include/hyena_nd.h declares, reports sizes, and rejects bad arguments before
+touching the GPU (no call here reaches a kernel launch)."""
+import os
+import re
+
+import pytest
+
+from dimensional_long_convolution_b200 import hyena_nd as H
+from dimensional_long_convolution_b200 import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "hyena_nd.h")).read()
+    return sorted(set(re.findall(r"HYENA_ND_API\s+[\w\s\*]+?\b(hyena_nd_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = H.load()
+    names = _declared()
+    assert len(names) == len(H.EXPORTED) == 12
+    assert set(names) == set(H.EXPORTED)
+    for n in names:
+        assert getattr(lib, n) is not None
+
+
+def test_status_strings():
+    assert H.status_string(0) == "HYENA_ND_OK"
+    assert H.status_string(6) == "HYENA_ND_ERR_DEVICE_TIMEOUT"
+    assert H.status_string(99) == "HYENA_ND_ERR_UNKNOWN"
+
+
+@pytest.mark.parametrize("i", range(5))
+def test_sizes_of_the_benchmark_grids(i):
+    wl = W.workload(i)
+    p = H.problem(wl.dims, wl.B, wl.C, H.BF16 if wl.io_dtype == "bf16" else H.F32)
+    P = [2 * n for n in wl.dims]
+    half = 1
+    for a in P[:-1]:
+        half *= a
+    half *= P[-1] // 2 + 1
+    assert H.spectrum_bytes(p) == wl.C * half * 8
+    ws = H.workspace_bytes(p)
+    assert ws >= 256 and ws % 16 == 0
+    assert H.workspace_bytes(p) == ws          # pure function of the descriptor
+
+
+@pytest.mark.parametrize("dims,B,C,dt,circ,want", [
+    ((64, 64), 1, 1, 0, 0, True),
+    ((300, 300), 1, 1, 0, 0, False),          # not a power of two
+    ((512,), 1, 1, 0, 0, False),              # above 256
+    ((4, 8), 1, 1, 0, 0, False),              # below 8
+    ((256, 64, 64), 1, 1, 0, 0, False),       # outer 3D axis above 128
+    ((64, 64), 0, 1, 0, 0, False),            # B < 1
+    ((64, 64), 1, 1, 7, 0, False),            # unknown dtype
+    ((64, 64), 1, 1, 0, 1, False),            # circular mode not implemented
+])
+def test_workspace_bytes_is_zero_for_invalid_problems(dims, B, C, dt, circ, want):
+    p = H.problem(dims, B, C, dt, circ)
+    assert (H.workspace_bytes(p) > 0) == want
+    assert (H.spectrum_bytes(p) > 0) == want
+
+
+def test_rank_zero_and_four_are_invalid():
+    p = H.problem((64, 64), 1, 1)
+    p.ndim = 0
+    assert H.workspace_bytes(p) == 0
+    p.ndim = 4
+    assert H.workspace_bytes(p) == 0
+
+
+# fake, never dereferenced device addresses (argument checks run first)
+A = 0x7F0000000000
+STEP = 1 << 30
+
+
+def _ptrs():
+    return [A + i * STEP for i in range(6)]
+
+
+def _call(p, q, k, v, s, y, ws, wsb, sbs=0):
+    return H.fftconv_batched(p, q, k, v, s, sbs, y, ws, wsb, 0)
+
+
+def test_invalid_arguments_are_rejected_before_launch():
+    p = H.problem((64, 64), 2, 3)
+    q, k, v, s, y, ws = _ptrs()
+    wsb = H.workspace_bytes(p)
+    assert _call(p, 0, k, v, s, y, ws, wsb) == H.ERR_INVALID_ARG
+    assert _call(p, q, k, v, 0, y, ws, wsb) == H.ERR_INVALID_ARG
+    assert _call(p, q, k, v, s, y, 0, wsb) == H.ERR_INVALID_ARG
+    assert _call(p, q + 4, k, v, s, y, ws, wsb) == H.ERR_MISALIGNED
+    assert _call(p, q, k, v, s, y + 8, ws, wsb) == H.ERR_MISALIGNED
+    assert _call(p, q, k, v, s, y, ws, wsb - 16) == H.ERR_WORKSPACE_TOO_SMALL
+    assert _call(p, q, k, v, s, q, ws, wsb) == H.ERR_INVALID_ARG          # y aliases q
+    assert _call(p, q, k, v, s, k + 64, ws, wsb) == H.ERR_INVALID_ARG     # y overlaps k
+    assert _call(p, q, k, v, s, y, ws, wsb, sbs=-16) == H.ERR_INVALID_ARG
+    assert _call(p, q, k, v, s, y, ws, wsb, sbs=8) == H.ERR_MISALIGNED
+    bad = H.problem((48, 64), 2, 3)
+    assert _call(bad, q, k, v, s, y, ws, wsb) == H.ERR_UNSUPPORTED
+    circ = H.problem((64, 64), 2, 3, circular=1)
+    assert _call(circ, q, k, v, s, y, ws, wsb) == H.ERR_UNSUPPORTED
+
+
+def test_single_volume_call_needs_b_and_c_of_one():
+    q, k, v, s, y, ws = _ptrs()
+    p = H.problem((32, 32), 2, 1)
+    assert H.fftconv(p, q, k, v, s, y, ws, 1 << 30, 0) == H.ERR_INVALID_ARG
+
+
+def test_filter_arguments_are_checked():
+    p = H.problem((32, 32), 1, 4)
+    _, _, _, s, _, ws = _ptrs()
+    wsb = H.workspace_bytes(p)
+    f = H.Filter()
+    f.num_freqs, f.hidden = 8, 64
+    f.W1 = f.b1 = f.W2 = f.b2 = f.alpha = A + 7 * STEP
+    f.decay_scale, f.window = 32.0, 0
+    f.window = 1
+    assert H.filter_spectrum(p, f, s, ws, wsb) == H.ERR_UNSUPPORTED      # Gaussian window
+    f.window = 0
+    f.hidden = 0
+    assert H.filter_spectrum(p, f, s, ws, wsb) == H.ERR_UNSUPPORTED
+    f.hidden = 64
+    f.decay_scale = 0.0
+    assert H.filter_spectrum(p, f, s, ws, wsb) == H.ERR_INVALID_ARG
+    f.decay_scale = 32.0
+    f.W2 = 0
+    assert H.filter_spectrum(p, f, s, ws, wsb) == H.ERR_INVALID_ARG
+    f.W2 = A + 7 * STEP + 2
+    assert H.filter_spectrum(p, f, s, ws, wsb) == H.ERR_MISALIGNED
+    f.W2 = A + 7 * STEP
+    assert H.filter_spectrum(p, f, s, ws, wsb - 1) == H.ERR_WORKSPACE_TOO_SMALL
+
+
+def test_spectrum_conversion_checks():
+    p = H.problem((32, 32), 1, 4)
+    nb = H.spectrum_bytes(p)
+    assert H.spectrum_export(p, A, A + nb // 2, 0) == H.ERR_INVALID_ARG     # overlap
+    assert H.spectrum_import(p, A + 4, A + STEP, 0) == H.ERR_MISALIGNED
+    assert H.spectrum_import(p, 0, A + STEP, 0) == H.ERR_INVALID_ARG
+
+
+def test_status_and_debug_calls_check_arguments():
+    assert H.device_status(0, 0) == H.ERR_INVALID_ARG
+    assert H.device_status(A + 4, 0) == H.ERR_MISALIGNED
+    assert H.workspace_init(A, 16, 0) == H.ERR_WORKSPACE_TOO_SMALL
+    assert H.debug_bounded_wait(A, 4096, 0, 0) == H.ERR_INVALID_ARG
+    assert H.debug_bounded_wait(A, 8, 100, 0) == H.ERR_WORKSPACE_TOO_SMALL
