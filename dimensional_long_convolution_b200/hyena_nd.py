@@ -192,7 +192,10 @@ class HyenaND:
         self.io_dtype = io_dtype
         self.tdtype = torch.bfloat16 if io_dtype == "bf16" else torch.float32
         self.p = problem(self.dims, B, C, BF16 if io_dtype == "bf16" else F32)
-        self.device = torch.device(device if device is not None else "cuda")
+        dev = torch.device(device if device is not None else "cuda")
+        if dev.type == "cuda" and dev.index is None:
+            dev = torch.device("cuda", torch.cuda.current_device())
+        self.device = dev
         nbytes = workspace_bytes(self.p)
         if nbytes == 0:
             raise HyenaNDError(ERR_UNSUPPORTED, "workspace_bytes")

@@ -241,7 +241,10 @@ def reference_output(inputs, S_full=None, K=None) -> np.ndarray:
 
 
 def rel_l2(a: np.ndarray, b: np.ndarray) -> float:
-    a = np.asarray(a, dtype=np.float64)
-    b = np.asarray(b, dtype=np.float64)
+    """||a - b||_2 / ||b||_2 over all elements (complex values compared as
+    complex numbers)."""
+    cplx = np.iscomplexobj(a) or np.iscomplexobj(b)
+    a = np.asarray(a, dtype=np.complex128 if cplx else np.float64)
+    b = np.asarray(b, dtype=np.complex128 if cplx else np.float64)
     den = np.linalg.norm(b.reshape(-1))
     return float(np.linalg.norm((a - b).reshape(-1)) / (den if den > 0 else 1.0))

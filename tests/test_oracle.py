@@ -304,3 +304,9 @@ def test_workload_zero_full_direct_vs_dft():
     y1 = O.conv_direct(q, k, v, K, dims)
     y2 = O.conv_dft(q, k, v, O.spectrum_full(K, dims), dims)
     assert O.rel_l2(y2, y1) < 1e-12
+
+
+def test_rel_l2_compares_complex_values_as_complex():
+    a = np.array([1.0 + 1.0j, 2.0])
+    b = np.array([1.0 + 0.0j, 2.0])
+    assert abs(O.rel_l2(a, b) - 1.0 / np.sqrt(5.0)) < 1e-15
