@@ -43,7 +43,10 @@ EXPORTED = (
     "hyena_nd_debug_bounded_wait",
     "hyena_nd_status_string",
     "hyena_nd_last_launch_count",
+    "hyena_nd_fftconv_batched_static",
 )
+
+STATIC_SCRATCH_BYTES = 16 << 20
 
 
 class Problem(ctypes.Structure):
@@ -103,6 +106,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "hyena_nd_debug_bounded_wait": (ctypes.c_int, [vp, sz, ctypes.c_int, vp]),
         "hyena_nd_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "hyena_nd_last_launch_count": (ctypes.c_int, []),
+        "hyena_nd_fftconv_batched_static": (ctypes.c_int, [P, vp, vp, vp, vp, i64, vp, vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -147,6 +151,14 @@ def fftconv_batched(p: Problem, q: int, k: int, v: int, spectrum: int, spectrum_
                     ws: int, ws_bytes: int, stream: int = 0) -> int:
     return load().hyena_nd_fftconv_batched(ctypes.byref(p), q, k, v, spectrum, spectrum_batch_stride, y, ws,
                                            ws_bytes, stream)
+
+
+def fftconv_batched_static(p: Problem, q: int, k: int, v: int, spectrum: int, spectrum_batch_stride: int,
+                           y: int, stream: int = 0) -> int:
+    """The batched call without a workspace argument: its scratch is a fixed
+    16 MiB array inside the library (for callers that cannot allocate)."""
+    return load().hyena_nd_fftconv_batched_static(ctypes.byref(p), q, k, v, spectrum, spectrum_batch_stride, y,
+                                                  stream)
 
 
 def spectrum_export(p: Problem, spectrum: int, natural: int, stream: int = 0) -> int:

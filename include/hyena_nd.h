@@ -143,6 +143,32 @@ HYENA_ND_API hyena_nd_status hyena_nd_fftconv_batched(const hyena_nd_problem* p,
                                          int64_t spectrum_batch_stride, void* y, void* ws,
                                          size_t ws_bytes, void* cuda_stream);
 
+/* Same operation as hyena_nd_fftconv_batched, for callers that cannot
+ * allocate device memory and so have no workspace to pass: for instance a
+ * plugin whose interface carries only input and output buffers, or an
+ * application that reserves all device memory at start-up and allows no
+ * allocation afterwards.  (The HyenaND pages have no counterpart; this is a
+ * deployment convenience of this library.)
+ * Scratch: a fixed array of HYENA_ND_STATIC_SCRATCH_BYTES (16 MiB) inside the
+ * library's device image, held by every GPU that loads the library until the
+ * process exits.  Nothing is allocated or freed by the call.
+ *   * A problem whose single (b, c) volume needs more than that (8 bytes per
+ *     voxel in the multi-pass tiers, e.g. a 128 x 128 x 256 volume) returns
+ *     HYENA_ND_ERR_WORKSPACE_TOO_SMALL before anything is launched.
+ *   * The first call on a device looks up the array's device address once;
+ *     make that first call before any stream capture.
+ *   * Every call shares the array and it keeps the previous call's contents
+ *     (each call writes what it reads, so nothing has to start at zero).
+ *     Calls whose kernels overlap on one GPU race on it: serialise them.
+ *   * Device-side status words are not used by this call.
+ * Other arguments and errors: as hyena_nd_fftconv_batched. */
+#define HYENA_ND_STATIC_SCRATCH_BYTES (16u << 20)
+HYENA_ND_API hyena_nd_status hyena_nd_fftconv_batched_static(const hyena_nd_problem* p, const void* q,
+                                                             const void* k, const void* v,
+                                                             const void* spectrum,
+                                                             int64_t spectrum_batch_stride, void* y,
+                                                             void* cuda_stream);
+
 /* Convert between the library's spectrum order and the natural order
  * [C, P_1, ..., P_{d-1}, P_d/2 + 1] complex64 (scale included, i.e. the
  * natural array is DFT(wrap-placed K) / prod(P)).  Both buffers are device
