@@ -158,6 +158,7 @@ hyena_nd_status hyena_nd_fftconv_batched(const hyena_nd_problem* p, const void* 
   a.ndim = pl.ndim;
   for (int i = 0; i < 3; ++i) a.n[i] = pl.n[i];
   a.stream = static_cast<cudaStream_t>(cuda_stream);
+  a.status = static_cast<int*>(ws);
 
   int launches = 0;
   cudaError_t e = cudaSuccess;

@@ -1,0 +1,339 @@
+// hnd_fft2.cuh -- packed two-path FFT core for sm_100a.
+//
+// The zero-padded length-2N transform of a pencil whose last N inputs are 0
+// (HyenaND pages: zero padding to twice the grid gives the linear
+// convolution) splits into two length-N transforms that share every twiddle:
+//   X[2m]   = FFT_N(x)[m]                (path 0)
+//   X[2m+1] = FFT_N(x W_2N^j)[m]         (path 1)
+// and the inverse that keeps outputs [0, N):
+//   y[i]    = IFFT_N(Y0)[i] + W_2N^-i IFFT_N(Y1)[i].
+// Both paths live in the two lanes of float2 registers ("cp": re = (path0.re,
+// path1.re), im = (path0.im, path1.im)), so every butterfly is one packed
+// FADD2/FFMA2 for both paths: the fp32 work is unchanged, the issue slots
+// halve.
+//
+// A length-N transform (N = R1 * R2, R1 = 8) is owned by G = R2 lanes; each
+// lane holds R1 slots.  Pass 1 is a radix-R1 DFT on x[g + r G]; the lanes
+// trade values once through a swizzled shared buffer; pass 2 is a radix-R2
+// DFT with twiddles W_N^{j r}.  Layouts:
+//   natural  (forward input, inverse output):  slot s <-> index g + s G
+//   spectral (forward output, inverse input):  slot s <-> g + G (s / R2) + (s % R2) R1
+// The spectral order is never reordered: the channel spectrum is stored in
+// it, so the pointwise product needs no bit reversal.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace hnd2 {
+
+// ------------------------------------------------------------ packed fp32
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
+__device__ __forceinline__ float2 padd(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 psub(float2 a, float2 b) { return __fadd2_rn(a, make_float2(-b.x, -b.y)); }
+__device__ __forceinline__ float2 pmul(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 pfma(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
+struct cp {
+  float2 re, im;
+};
+__device__ __forceinline__ cp cadd(cp a, cp b) { return {padd(a.re, b.re), padd(a.im, b.im)}; }
+__device__ __forceinline__ cp csub(cp a, cp b) { return {psub(a.re, b.re), psub(a.im, b.im)}; }
+
+// x * (c + i s) for both paths (w4 = (c, c, s, s)); INV: x * (c - i s)
+template <bool INV>
+__device__ __forceinline__ cp ctw(cp x, float4 w4) {
+  const float2 cc = make_float2(w4.x, w4.y), ss = make_float2(w4.z, w4.w);
+  const float2 nss = make_float2(-w4.z, -w4.w);
+  if (INV) return {pfma(x.im, ss, pmul(x.re, cc)), pfma(x.re, nss, pmul(x.im, cc))};
+  return {pfma(x.im, nss, pmul(x.re, cc)), pfma(x.re, ss, pmul(x.im, cc))};
+}
+// x * s with a different complex factor per path (s = (s0.re, s1.re), (s0.im, s1.im))
+__device__ __forceinline__ cp cmulp(cp x, float2 sre, float2 sim) {
+  const float2 nsim = make_float2(-sim.x, -sim.y);
+  return {pfma(x.im, nsim, pmul(x.re, sre)), pfma(x.re, sim, pmul(x.im, sre))};
+}
+
+// ------------------------------------------------------------ small DFTs
+// Natural-order DFT4 of (a0, a1, a2, a3); forward sign -i, inverse +i.
+template <bool INV>
+__device__ __forceinline__ void dft4(cp& a0, cp& a1, cp& a2, cp& a3) {
+  const cp c0 = cadd(a0, a2), c2 = csub(a0, a2), c1 = cadd(a1, a3), d = csub(a1, a3);
+  a0 = cadd(c0, c1);
+  a2 = csub(c0, c1);
+  if (!INV) {   // c2 -/+ i d
+    a1 = {padd(c2.re, d.im), psub(c2.im, d.re)};
+    a3 = {psub(c2.re, d.im), padd(c2.im, d.re)};
+  } else {
+    a1 = {psub(c2.re, d.im), padd(c2.im, d.re)};
+    a3 = {padd(c2.re, d.im), psub(c2.im, d.re)};
+  }
+}
+
+__device__ __forceinline__ void dft2(cp& a0, cp& a1) {
+  const cp t = csub(a0, a1);
+  a0 = cadd(a0, a1);
+  a1 = t;
+}
+
+// Natural-order DFT8, 52 packed operations (the 1/sqrt2 factors ride in FMAs).
+template <bool INV>
+__device__ __forceinline__ void dft8(cp* a) {
+  const float2 h = f2(0.70710678118654752440f), nh = f2(-0.70710678118654752440f);
+  cp b0 = cadd(a[0], a[4]), b4 = csub(a[0], a[4]);
+  cp b1 = cadd(a[1], a[5]), b5 = csub(a[1], a[5]);
+  cp b2 = cadd(a[2], a[6]), b6 = csub(a[2], a[6]);
+  cp b3 = cadd(a[3], a[7]), b7 = csub(a[3], a[7]);
+  dft4<INV>(b0, b1, b2, b3);                // even outputs 0, 2, 4, 6
+  cp c0, c2;
+  float2 u1, u2, u3, u4;                   // odd half: b5 W8, b6 W8^2, b7 W8^3 folded in
+  if (!INV) {
+    c0 = {padd(b4.re, b6.im), psub(b4.im, b6.re)};          // b4 + (-i) b6
+    c2 = {psub(b4.re, b6.im), padd(b4.im, b6.re)};
+    const float2 s5 = padd(b5.re, b5.im), t5 = psub(b5.im, b5.re);
+    const float2 s7 = padd(b7.re, b7.im), t7 = psub(b7.im, b7.re);
+    u1 = padd(s5, t7);
+    u2 = psub(t5, s7);      // c1 = h (u1, u2)
+    u3 = psub(s5, t7);
+    u4 = padd(t5, s7);      // d  = h (u3, u4)
+    a[0] = b0; a[2] = b1; a[4] = b2; a[6] = b3;
+    a[1] = {pfma(h, u1, c0.re), pfma(h, u2, c0.im)};
+    a[5] = {pfma(nh, u1, c0.re), pfma(nh, u2, c0.im)};
+    a[3] = {pfma(h, u4, c2.re), pfma(nh, u3, c2.im)};       // c2 + (-i) d
+    a[7] = {pfma(nh, u4, c2.re), pfma(h, u3, c2.im)};
+  } else {
+    c0 = {psub(b4.re, b6.im), padd(b4.im, b6.re)};          // b4 + (+i) b6
+    c2 = {padd(b4.re, b6.im), psub(b4.im, b6.re)};
+    // b5 (1 + i) h, b7 (-1 + i) h
+    const float2 s5 = psub(b5.re, b5.im), t5 = padd(b5.re, b5.im);
+    const float2 s7 = padd(b7.re, b7.im), t7 = psub(b7.re, b7.im);
+    // p1 = h (s5, t5); p3 = h (-s7, t7)
+    u1 = psub(s5, s7);
+    u2 = padd(t5, t7);      // c1 = p1 + p3
+    u3 = padd(s5, s7);
+    u4 = psub(t5, t7);      // d  = p1 - p3
+    a[0] = b0; a[2] = b1; a[4] = b2; a[6] = b3;
+    a[1] = {pfma(h, u1, c0.re), pfma(h, u2, c0.im)};
+    a[5] = {pfma(nh, u1, c0.re), pfma(nh, u2, c0.im)};
+    a[3] = {pfma(nh, u4, c2.re), pfma(h, u3, c2.im)};       // c2 + (+i) d
+    a[7] = {pfma(h, u4, c2.re), pfma(nh, u3, c2.im)};
+  }
+  // the even DFT4 left its outputs in b0..b3 = X0, X2, X4, X6 (set above)
+}
+
+// ------------------------------------------------------------------- plan
+template <int N>
+struct P2 {
+  static_assert(N == 8 || N == 16 || N == 32 || N == 64, "packed core: N in {8,16,32,64}");
+  static constexpr int R1 = 8;
+  static constexpr int R2 = N / 8;          // 1 (single pass), 2, 4, 8
+  static constexpr int G = (N == 8) ? 1 : R2;
+  static constexpr bool TWO = N > 8;
+};
+
+template <int N>
+__host__ __device__ __forceinline__ int spec_idx(int g, int s) {
+  if constexpr (N == 8) {
+    return s;
+  } else {
+    constexpr int G = P2<N>::G, R2 = P2<N>::R2, R1 = P2<N>::R1;
+    return g + G * (s / R2) + (s % R2) * R1;
+  }
+}
+
+// Swizzled float4 index inside a pencil's exchange buffer: the low three bits
+// are XORed with bits 3-5 and 4-6, which keeps every pass's 8-lane phase on
+// distinct 16-byte bank groups (a bijection inside each aligned block of 8).
+__host__ __device__ __forceinline__ int swz(int i) { return i ^ (((i >> 3) ^ (i >> 4)) & 7); }
+
+// Per-pencil key XORed into the low bits so that pencils sharing an 8-lane
+// phase (G < 8) land on disjoint bank groups.
+template <int N>
+__device__ __forceinline__ int pkey(int pen) {
+  constexpr int G = N / 8 < 1 ? 1 : N / 8;
+  return (pen * G) & 7;
+}
+
+template <int N>
+__device__ __forceinline__ unsigned pmask(int lane) {
+  constexpr int G = P2<N>::G;
+  if constexpr (G >= 32) {
+    return 0xffffffffu;
+  } else {
+    const unsigned m = (1u << G) - 1u;
+    return m << ((lane / G) * G);
+  }
+}
+
+// Per-size twiddle tables in shared memory (built once per CTA):
+//   tw2[(b R2 + r) G + g] = W_N^{(g + G b) r}   pass-2 twiddles, (c, c, s, s)
+//   twi[r G + g]          = W_N^{g r}           inverse pass-2 twiddles
+//   tst[s G + g]          = W_2N^{g + s G}      twist factors, (c, s)
+template <int N>
+struct Tabs {
+  static constexpr int G = P2<N>::G;
+  static constexpr int kTw2 = 8 * G;        // float4
+  static constexpr int kTwi = 8 * G;        // float4
+  static constexpr int kTst = 8 * G;        // float2
+  static constexpr size_t kBytes = 16 * (kTw2 + kTwi) + 8 * kTst;
+  float4* tw2;
+  float4* twi;
+  float2* tst;
+};
+
+// W_M^e from the 512-entry table W_512^k.
+__device__ __forceinline__ float2 wtab(const float2* __restrict__ W512, int M, int e) {
+  return W512[(e % M) * (512 / M)];
+}
+
+template <int N>
+__device__ __forceinline__ Tabs<N> tabs_at(unsigned char* base) {
+  Tabs<N> t;
+  t.tw2 = reinterpret_cast<float4*>(base);
+  t.twi = t.tw2 + Tabs<N>::kTw2;
+  t.tst = reinterpret_cast<float2*>(t.twi + Tabs<N>::kTwi);
+  return t;
+}
+
+template <int N>
+__device__ __forceinline__ void tabs_build(Tabs<N> t, const float2* __restrict__ W512) {
+  constexpr int G = P2<N>::G, R2 = P2<N>::R2;
+  for (int e = threadIdx.x; e < 8 * G; e += blockDim.x) {
+    const int g = e % G, sr = e / G;              // sr = b R2 + r (pass 2) or r (inverse) or s (twist)
+    const int b = sr / (R2 > 0 ? R2 : 1), r = sr % (R2 > 0 ? R2 : 1);
+    const float2 w = wtab(W512, N, (g + G * b) * r);
+    t.tw2[e] = make_float4(w.x, w.x, w.y, w.y);
+    const float2 wi = wtab(W512, N, g * sr);
+    t.twi[e] = make_float4(wi.x, wi.x, wi.y, wi.y);
+    t.tst[e] = wtab(W512, 2 * N, g + sr * G);
+  }
+}
+
+// ------------------------------------------------------------------- FFTs
+// Forward: natural -> spectral.  buf: this pencil's N float4 (swizzled).
+template <int N>
+__device__ __forceinline__ void fft_fwd(cp (&x)[8], int g, float4* buf, int key, Tabs<N> t, unsigned mask) {
+  dft8<false>(x);
+  if constexpr (P2<N>::TWO) {
+    constexpr int G = P2<N>::G, R2 = P2<N>::R2;
+    // pass-1 output index j*8 + r (j = g): write, then read pass-2 inputs j' + r*8
+    __syncwarp(mask);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) buf[swz(g * 8 + r) ^ key] = make_float4(x[r].re.x, x[r].re.y, x[r].im.x, x[r].im.y);
+    __syncwarp(mask);
+#pragma unroll
+    for (int b = 0; b < 8 / R2; ++b) {
+#pragma unroll
+      for (int r = 0; r < R2; ++r) {
+        const float4 v = buf[swz(g + G * b + r * 8) ^ key];
+        cp y = {make_float2(v.x, v.y), make_float2(v.z, v.w)};
+        if (r > 0) y = ctw<false>(y, t.tw2[(b * R2 + r) * G + g]);
+        x[b * R2 + r] = y;
+      }
+      if constexpr (R2 == 8) dft8<false>(&x[b * 8]);
+      else if constexpr (R2 == 4) dft4<false>(x[b * 4], x[b * 4 + 1], x[b * 4 + 2], x[b * 4 + 3]);
+      else dft2(x[b * 2], x[b * 2 + 1]);
+    }
+  }
+}
+
+// Inverse (unnormalised): spectral -> natural.
+template <int N>
+__device__ __forceinline__ void fft_inv(cp (&x)[8], int g, float4* buf, int key, Tabs<N> t, unsigned mask) {
+  if constexpr (!P2<N>::TWO) {
+    dft8<true>(x);
+  } else {
+    constexpr int G = P2<N>::G, R2 = P2<N>::R2;
+    // inverse pass 1: radix R2 on slots b*R2 + r (inputs j + r*8, j = g + G b)
+#pragma unroll
+    for (int b = 0; b < 8 / R2; ++b) {
+      if constexpr (R2 == 8) dft8<true>(&x[b * 8]);
+      else if constexpr (R2 == 4) dft4<true>(x[b * 4], x[b * 4 + 1], x[b * 4 + 2], x[b * 4 + 3]);
+      else dft2(x[b * 2], x[b * 2 + 1]);
+    }
+    // output index (j) * R2 + r ; read pass-2 inputs g + r*G with twiddle W_N^{-g r}
+    __syncwarp(mask);
+#pragma unroll
+    for (int b = 0; b < 8 / R2; ++b) {
+#pragma unroll
+      for (int r = 0; r < R2; ++r) {
+        const int s = b * R2 + r;
+        buf[swz((g + G * b) * R2 + r) ^ key] = make_float4(x[s].re.x, x[s].re.y, x[s].im.x, x[s].im.y);
+      }
+    }
+    __syncwarp(mask);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const float4 v = buf[swz(g + r * G) ^ key];
+      cp y = {make_float2(v.x, v.y), make_float2(v.z, v.w)};
+      if (r > 0) y = ctw<true>(y, t.twi[r * G + g]);
+      x[r] = y;
+    }
+    dft8<true>(x);
+  }
+}
+
+// Forward padded transform: on entry z[s] = input at natural index g + s G
+// (a complex value, the same for both paths); on exit x[s] holds
+// (Z[2f], Z[2f+1]) with f = spec_idx<N>(g, s).
+template <int N>
+__device__ __forceinline__ void padded_fwd(const float2 (&z)[8], cp (&x)[8], int g, float4* buf, int key, Tabs<N> t,
+                                           unsigned mask) {
+  constexpr int G = P2<N>::G;
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const float2 w = t.tst[s * G + g];
+    const float ore = fmaf(z[s].x, w.x, -z[s].y * w.y);
+    const float oim = fmaf(z[s].x, w.y, z[s].y * w.x);
+    x[s] = {make_float2(z[s].x, ore), make_float2(z[s].y, oim)};
+  }
+  fft_fwd<N>(x, g, buf, key, t, mask);
+}
+
+// Inverse padded transform keeping outputs [0, N): on entry x[s] =
+// (Y[2f], Y[2f+1]); on exit out[s] = y[g + s G] (unnormalised).
+template <int N>
+__device__ __forceinline__ void padded_inv(cp (&x)[8], float2 (&out)[8], int g, float4* buf, int key, Tabs<N> t,
+                                           unsigned mask) {
+  constexpr int G = P2<N>::G;
+  fft_inv<N>(x, g, buf, key, t, mask);
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const float2 w = t.tst[s * G + g];   // untwist by conj(W_2N^{g + s G})
+    const float re = fmaf(x[s].re.y, w.x, fmaf(x[s].im.y, w.y, x[s].re.x));
+    const float im = fmaf(x[s].im.y, w.x, fmaf(-x[s].re.y, w.y, x[s].im.x));
+    out[s] = make_float2(re, im);
+  }
+}
+
+// Partner frequency -k (mod 2N) of spectral slot (f, path): path 0 -> (N - f)
+// mod N, path 1 -> N - 1 - f (both as natural half-frequency indices).
+template <int N>
+__device__ __forceinline__ void fetch_partner(const cp (&x)[8], cp (&xp)[8], int g, float4* buf, int key, unsigned mask) {
+  __syncwarp(mask);
+#pragma unroll
+  for (int s = 0; s < 8; ++s)
+    buf[swz(spec_idx<N>(g, s)) ^ key] = make_float4(x[s].re.x, x[s].re.y, x[s].im.x, x[s].im.y);
+  __syncwarp(mask);
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const int f = spec_idx<N>(g, s);
+    const float4 a = buf[swz((N - f) & (N - 1)) ^ key];
+    const float4 b = buf[swz(N - 1 - f) ^ key];
+    xp[s] = {make_float2(a.x, b.y), make_float2(a.z, b.w)};
+  }
+}
+
+// Row-pair packing: X_a = (Z[k] + conj Z[-k]) / 2, X_b = (Z[k] - conj Z[-k]) / (2i)
+__device__ __forceinline__ float2 unpack_a(float2 z, float2 zm) {
+  return make_float2(0.5f * (z.x + zm.x), 0.5f * (z.y - zm.y));
+}
+__device__ __forceinline__ float2 unpack_b(float2 z, float2 zm) {
+  return make_float2(0.5f * (z.y + zm.y), 0.5f * (zm.x - z.x));
+}
+// W[k] = Y_a + i Y_b ; W[-k] = conj(Y_a) + i conj(Y_b)
+__device__ __forceinline__ float2 pack_pos(float2 ya, float2 yb) { return make_float2(ya.x - yb.y, ya.y + yb.x); }
+__device__ __forceinline__ float2 pack_neg(float2 ya, float2 yb) { return make_float2(ya.x + yb.y, yb.x - ya.y); }
+
+}  // namespace hnd2

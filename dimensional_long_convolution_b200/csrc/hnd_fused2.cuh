@@ -1,0 +1,416 @@
+// hnd_fused2.cuh -- persistent fused 2D tier on the packed two-path FFT core.
+//
+// One CTA (256 threads, two per SM) walks (b, c) volumes.  Per volume, all
+// in shared memory (HyenaND arXiv summary, "Implementation: nSubQ": forward
+// FFT, spectral modulation, inverse FFT and output cropping fused, with the
+// intermediates on chip):
+//   stage 1  rows r and r + n0/2 packed as one complex row, zero-padded
+//            forward transform along axis 1 -> Zb[kk][rp]
+//   stage 2  per last-axis frequency: unpack both rows, zero-padded
+//            convolution along axis 0 with the channel spectrum, repack
+//   stage 3  inverse row transforms, crop, output gate q, store y
+// k and v of the next volume are prefetched with bulk asynchronous copies
+// (one per row, into a padded staging pitch) while stages 2-3 run.
+#pragma once
+
+#include "hnd_fft2.cuh"
+
+namespace hnd2 {
+
+static __device__ const float2 g_tw512[512] =
+#include "hnd_twiddles.inc"
+;
+
+constexpr int kT = 256;          // threads per CTA
+constexpr int kW = kT / 32;      // warps per CTA
+
+// ------------------------------------------------------- async copy (TMA)
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+
+// Bounded wait on a phase of an mbarrier: gives up after about `limit`
+// cycles, records a timeout in the status word and returns false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity, int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  const long long limit = 4000000000LL;     // about 2 s at 2 GHz
+  for (long long it = 0; it < (1LL << 28); ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (clock64() - t0 > limit) break;
+  }
+  if (status) atomicCAS(status, 0, 6 /* HYENA_ND_ERR_DEVICE_TIMEOUT */);
+  return false;
+}
+
+// ------------------------------------------------------------ activations
+template <class T>
+struct Act;
+template <>
+struct Act<float> {
+  static __device__ __forceinline__ float ld_s(const float* p) { return *p; }
+  static __device__ __forceinline__ float ld_g(const float* p) { return __ldcs(p); }
+  static __device__ __forceinline__ void st_g(float* p, float x) { __stcs(p, x); }
+};
+template <>
+struct Act<__nv_bfloat16> {
+  static __device__ __forceinline__ float ld_s(const __nv_bfloat16* p) {
+    return __uint_as_float(static_cast<unsigned>(*reinterpret_cast<const unsigned short*>(p)) << 16);
+  }
+  static __device__ __forceinline__ float ld_g(const __nv_bfloat16* p) {
+    return __uint_as_float(static_cast<unsigned>(__ldcs(reinterpret_cast<const unsigned short*>(p))) << 16);
+  }
+  static __device__ __forceinline__ void st_g(__nv_bfloat16* p, float x) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    __stcs(reinterpret_cast<unsigned short*>(p), *reinterpret_cast<const unsigned short*>(&h));
+  }
+};
+
+// ------------------------------------------------------------ the kernel
+template <int N0, int N1, class T>
+struct F2 {
+  static constexpr int PITCH = (N1 * static_cast<int>(sizeof(T)) / 4 + 8) * 4 / static_cast<int>(sizeof(T));
+  static constexpr int RPS = N0 / 2 + 1;                 // Zb pitch (float2) per frequency row
+  static constexpr size_t kTabs = Tabs<N0>::kBytes + (N0 == N1 ? 0 : Tabs<N1>::kBytes);
+  static constexpr size_t kStage = static_cast<size_t>(N0) * PITCH * sizeof(T);
+  static constexpr size_t kZb = sizeof(float2) * 2 * N1 * RPS;
+  static constexpr size_t kX = 4096 * kW;                // exchange buffers (float4 per pencil slot)
+  static constexpr size_t kBytes = 16 + kTabs + 2 * kStage + kZb + kX;
+};
+
+template <int N0, int N1, class T>
+__global__ void __launch_bounds__(kT, 2)
+    k_fused2d_v2(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+                 const float4* __restrict__ spec, long long sbs4, T* __restrict__ y, int B, int C, int* status) {
+  using L = F2<N0, N1, T>;
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem);
+  unsigned char* p = smem + 16;
+  const Tabs<N0> t0 = tabs_at<N0>(p);
+  Tabs<N1> t1;
+  if constexpr (N0 == N1) {
+    t1 = t0;
+  } else {
+    t1 = tabs_at<N1>(p + Tabs<N0>::kBytes);
+  }
+  p += L::kTabs;
+  T* kst = reinterpret_cast<T*>(p);
+  T* vst = reinterpret_cast<T*>(p + L::kStage);
+  float2* Zb = reinterpret_cast<float2*>(p + 2 * L::kStage);
+  float4* xb = reinterpret_cast<float4*>(p + 2 * L::kStage + L::kZb);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nvol = B * C;
+  int vol = blockIdx.x;
+  if (vol >= nvol) return;
+  constexpr long long Lv = static_cast<long long>(N0) * N1;
+  constexpr unsigned kvBytes = 2u * N0 * N1 * sizeof(T);
+
+  tabs_build<N0>(t0, g_tw512);
+  if constexpr (N0 != N1) tabs_build<N1>(t1, g_tw512);
+
+  // issue the bulk copies of k and v rows of volume `vv` into the staging pitch
+  auto issue_kv = [&](int vv) {
+    const int cc = vv / B, bb = vv % B;
+    const long long base = (static_cast<long long>(bb) * C + cc) * Lv;
+    if (lane == 0) mbar_expect_tx(bar, kvBytes);
+    __syncwarp();
+    for (int r = lane; r < 2 * N0; r += 32) {
+      const int row = r % N0;
+      const T* src = (r < N0 ? k : v) + base + static_cast<long long>(row) * N1;
+      T* dst = (r < N0 ? kst : vst) + row * L::PITCH;
+      bulk_g2s(dst, src, N1 * sizeof(T), bar);
+    }
+  };
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == 0) issue_kv(vol);
+  unsigned phase = 0;
+
+  for (; vol < nvol; vol += gridDim.x) {
+    const int c = vol / B, b = vol % B;
+    const long long pair = static_cast<long long>(b) * C + c;
+    const T* qp = q + pair * Lv;
+    T* yp = y + pair * Lv;
+    const int next = vol + gridDim.x;
+
+    if (!mbar_wait_bounded(bar, phase, status)) {
+      mbar_wait_bounded(bar, phase, nullptr);     // one more bounded wait for copies in flight
+      return;
+    }
+    phase ^= 1u;
+
+    // ---- stage 1: row pairs (rp, rp + N0/2) forward along axis 1
+    {
+      constexpr int G = P2<N1>::G, PPW = 32 / G;
+      const int pen = lane / G, g = lane % G;
+      const unsigned mask = pmask<N1>(lane);
+      const int key = pkey<N1>(pen);
+      float4* buf = xb + warp * 256 + pen * N1;
+      for (int r0 = warp * PPW; r0 < N0 / 2; r0 += kW * PPW) {
+        const int rp = r0 + pen;
+        const bool act = rp < N0 / 2;
+        float2 z[8];
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+          const int j = g + s * G;
+          const int ra = rp * L::PITCH + j, rb = (rp + N0 / 2) * L::PITCH + j;
+          z[s] = act ? make_float2(Act<T>::ld_s(kst + ra) * Act<T>::ld_s(vst + ra),
+                                   Act<T>::ld_s(kst + rb) * Act<T>::ld_s(vst + rb))
+                     : make_float2(0.f, 0.f);
+        }
+        cp x[8];
+        padded_fwd<N1>(z, x, g, buf, key, t1, mask);
+        if (act) {
+#pragma unroll
+          for (int s = 0; s < 8; ++s) {
+            const int kk = 2 * spec_idx<N1>(g, s);
+            Zb[kk * L::RPS + rp] = make_float2(x[s].re.x, x[s].im.x);
+            Zb[(kk + 1) * L::RPS + rp] = make_float2(x[s].re.y, x[s].im.y);
+          }
+        }
+      }
+    }
+    __syncthreads();
+    if (warp == 0 && next < nvol) {
+      fence_proxy_async();
+      issue_kv(next);
+    }
+
+    // ---- stage 2: columns; pencils of a warp take units 8 apart
+    {
+      constexpr int G = P2<N0>::G, PPW = 32 / G;
+      const int pen = lane / G, g = lane % G;
+      const unsigned mask = pmask<N0>(lane);
+      const int key = pkey<N0>(pen);
+      float4* buf = xb + warp * 256 + pen * N0;
+      const float4* sp = spec + static_cast<long long>(b) * sbs4 + static_cast<long long>(c) * (N1 + 1) * N0;
+      for (int round = 0; round * kW * PPW < N1; ++round) {
+        const int cu = round * kW * PPW + pen * kW + warp;
+        const bool act = cu < N1;
+        const int kx = cu, kxm = 2 * N1 - cu;
+        float2 z[8];
+        cp x[8];
+        if (cu == 0) {
+          // DC and Nyquist columns (both real) as one complex column
+#pragma unroll
+          for (int s = 0; s < 4; ++s) {
+            const int rp = g + s * G;
+            const float2 z0 = Zb[rp], zn = Zb[N1 * L::RPS + rp];
+            z[s] = make_float2(z0.x, zn.x);
+            z[s + 4] = make_float2(z0.y, zn.y);
+          }
+          padded_fwd<N0>(z, x, g, buf, key, t0, mask);
+          cp xp[8];
+          fetch_partner<N0>(x, xp, g, buf, key, mask);
+#pragma unroll
+          for (int s = 0; s < 8; ++s) {
+            const float4 A = __ldg(sp + s * G + g), Bc = __ldg(sp + N0 + s * G + g);
+            const cp a = cmulp(x[s], make_float2(A.x, A.y), make_float2(A.z, A.w));
+            const cp xc = {xp[s].re, make_float2(-xp[s].im.x, -xp[s].im.y)};
+            const cp bb = cmulp(xc, make_float2(Bc.x, Bc.y), make_float2(Bc.z, Bc.w));
+            x[s] = cadd(a, bb);
+          }
+        } else {
+          float4 S[8];
+          if (act) {
+            const float4* su = sp + static_cast<long long>(cu + 1) * N0;
+#pragma unroll
+            for (int s = 0; s < 8; ++s) S[s] = __ldg(su + s * G + g);
+          }
+#pragma unroll
+          for (int s = 0; s < 4; ++s) {
+            const int rp = g + s * G;
+            float2 z1 = make_float2(0.f, 0.f), z2 = z1;
+            if (act) {
+              z1 = Zb[kx * L::RPS + rp];
+              z2 = Zb[kxm * L::RPS + rp];
+            }
+            z[s] = unpack_a(z1, z2);
+            z[s + 4] = unpack_b(z1, z2);
+          }
+          padded_fwd<N0>(z, x, g, buf, key, t0, mask);
+          if (act) {
+#pragma unroll
+            for (int s = 0; s < 8; ++s) x[s] = cmulp(x[s], make_float2(S[s].x, S[s].y), make_float2(S[s].z, S[s].w));
+          }
+        }
+        float2 o[8];
+        padded_inv<N0>(x, o, g, buf, key, t0, mask);
+        if (act) {
+#pragma unroll
+          for (int s = 0; s < 4; ++s) {
+            const int rp = g + s * G;
+            const float2 ya = o[s], yb = o[s + 4];
+            if (cu == 0) {
+              Zb[rp] = make_float2(ya.x, yb.x);
+              Zb[N1 * L::RPS + rp] = make_float2(ya.y, yb.y);
+            } else {
+              Zb[kx * L::RPS + rp] = pack_pos(ya, yb);
+              Zb[kxm * L::RPS + rp] = pack_neg(ya, yb);
+            }
+          }
+        }
+      }
+    }
+    __syncthreads();
+
+    // ---- stage 3: inverse rows, crop, output gate
+    {
+      constexpr int G = P2<N1>::G, PPW = 32 / G;
+      const int pen = lane / G, g = lane % G;
+      const unsigned mask = pmask<N1>(lane);
+      const int key = pkey<N1>(pen);
+      float4* buf = xb + warp * 256 + pen * N1;
+      for (int r0 = warp * PPW; r0 < N0 / 2; r0 += kW * PPW) {
+        const int rp = r0 + pen;
+        const bool act = rp < N0 / 2;
+        float qa[8], qb[8];
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+          const long long ja = static_cast<long long>(rp) * N1 + g + s * G;
+          qa[s] = act ? Act<T>::ld_g(qp + ja) : 0.f;
+          qb[s] = act ? Act<T>::ld_g(qp + ja + (N0 / 2) * N1) : 0.f;
+        }
+        cp x[8];
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+          const int kk = 2 * spec_idx<N1>(g, s);
+          const float2 e = act ? Zb[kk * L::RPS + rp] : make_float2(0.f, 0.f);
+          const float2 d = act ? Zb[(kk + 1) * L::RPS + rp] : make_float2(0.f, 0.f);
+          x[s] = {make_float2(e.x, d.x), make_float2(e.y, d.y)};
+        }
+        float2 o[8];
+        padded_inv<N1>(x, o, g, buf, key, t1, mask);
+        if (act) {
+#pragma unroll
+          for (int s = 0; s < 8; ++s) {
+            const long long ja = static_cast<long long>(rp) * N1 + g + s * G;
+            Act<T>::st_g(yp + ja, o[s].x * qa[s]);
+            Act<T>::st_g(yp + ja + (N0 / 2) * N1, o[s].y * qb[s]);
+          }
+        }
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------ spectrum layout (2D)
+// Library order of a 2D problem with n0 <= 64, per channel, in float4 units:
+// unit 0 (DC and Nyquist columns combined) holds A then B, n0 float4 each;
+// unit u >= 1 (column kx = u) holds n0 float4 at offset (u + 1) n0.  Inside a
+// unit, float4 m = s G + g holds (S[2f].re, S[2f+1].re, S[2f].im, S[2f+1].im)
+// with f = spec_idx(g, s) the z-pencil frequency of lane g, slot s.
+__host__ __device__ __forceinline__ int spec_idx_rt(int N, int g, int s) {
+  if (N == 8) return s;
+  const int G = N / 8;
+  return g + G * (s / G) + (s % G) * 8;
+}
+
+struct Pos2 {
+  int kind;      // 0 plain column, 1 = A (combined), 2 = B (combined)
+  int kx;        // plain column index
+  int ky0, ky1;  // padded frequencies held by path 0 and path 1
+};
+
+__host__ __device__ __forceinline__ Pos2 pos2_of(int n0, int n1, long long e4) {
+  Pos2 r;
+  long long m;
+  if (e4 < 2LL * n0) {
+    r.kind = 1 + static_cast<int>(e4 / n0);
+    r.kx = 0;
+    m = e4 % n0;
+  } else {
+    r.kind = 0;
+    r.kx = static_cast<int>((e4 - 2LL * n0) / n0) + 1;
+    m = (e4 - 2LL * n0) % n0;
+  }
+  const int G = n0 / 8 < 1 ? 1 : n0 / 8;
+  const int s = static_cast<int>(m / G), g = static_cast<int>(m % G);
+  const int f = spec_idx_rt(n0, g, s);
+  r.ky0 = 2 * f;
+  r.ky1 = 2 * f + 1;
+  return r;
+}
+
+// natural half spectrum [C][2 n0][n1 + 1] -> library order (v2)
+static __global__ void k_spec_import_v2(const float2* __restrict__ nat, float4* __restrict__ out, int n0, int n1,
+                                 long long C, long long full_pitch, float scale) {
+  // full_pitch: row length of the source (n1 + 1 for a half spectrum, 2 n1 for a full grid)
+  const long long per = static_cast<long long>(n1 + 1) * n0;         // float4 per channel
+  const long long src_per = static_cast<long long>(2 * n0) * full_pitch;
+  for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < per * C;
+       e += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long c = e / per, e4 = e % per;
+    const Pos2 ps = pos2_of(n0, n1, e4);
+    const float2* src = nat + c * src_per;
+    float2 s0, s1;
+    if (ps.kind == 0) {
+      s0 = src[ps.ky0 * full_pitch + ps.kx];
+      s1 = src[ps.ky1 * full_pitch + ps.kx];
+    } else {
+      const float sg = ps.kind == 1 ? 1.f : -1.f;
+      const float2 a0 = src[ps.ky0 * full_pitch], b0 = src[ps.ky0 * full_pitch + n1];
+      const float2 a1 = src[ps.ky1 * full_pitch], b1 = src[ps.ky1 * full_pitch + n1];
+      s0 = make_float2(0.5f * (a0.x + sg * b0.x), 0.5f * (a0.y + sg * b0.y));
+      s1 = make_float2(0.5f * (a1.x + sg * b1.x), 0.5f * (a1.y + sg * b1.y));
+    }
+    out[e] = make_float4(scale * s0.x, scale * s1.x, scale * s0.y, scale * s1.y);
+  }
+}
+
+// library order (v2) -> natural half spectrum [C][2 n0][n1 + 1]
+static __global__ void k_spec_export_v2(const float4* __restrict__ lib, float2* __restrict__ nat, int n0, int n1,
+                                 long long C) {
+  const long long per = static_cast<long long>(n1 + 1) * n0;
+  const long long W = n1 + 1;
+  for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < per * C;
+       e += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long c = e / per, e4 = e % per;
+    const Pos2 ps = pos2_of(n0, n1, e4);
+    float2* dst = nat + c * per * 2;
+    const float4 f = lib[e];
+    if (ps.kind == 0) {
+      dst[ps.ky0 * W + ps.kx] = make_float2(f.x, f.z);
+      dst[ps.ky1 * W + ps.kx] = make_float2(f.y, f.w);
+    } else if (ps.kind == 1) {
+      const float4 g = lib[e + n0];     // the B payload at the same position
+      dst[ps.ky0 * W] = make_float2(f.x + g.x, f.z + g.z);
+      dst[ps.ky0 * W + n1] = make_float2(f.x - g.x, f.z - g.z);
+      dst[ps.ky1 * W] = make_float2(f.y + g.y, f.w + g.w);
+      dst[ps.ky1 * W + n1] = make_float2(f.y - g.y, f.w - g.w);
+    }
+  }
+}
+
+}  // namespace hnd2

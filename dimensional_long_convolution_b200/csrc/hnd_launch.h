@@ -21,7 +21,15 @@ struct ConvArgs {
   int n[3];
   int ndim;
   cudaStream_t stream;
+  int* status = nullptr;  // device status word (may be null)
 };
+
+// 2D problems whose axes are both <= 64 run on the packed persistent fused
+// kernel and use the packed (v2) spectrum order.
+inline bool use_v2_2d(int ndim, const int* n) { return ndim == 2 && n[0] <= 64 && n[1] <= 64; }
+
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count();
 
 // Maximum dynamic shared memory per CTA on sm_100 (227 KB).
 constexpr size_t kMaxSmem = 232448;

@@ -1,5 +1,6 @@
 // Filter spectrum (call 1), spectrum layout conversion, diagnostics.
 #include "hnd_kernels.cuh"
+#include "hnd_fused2.cuh"
 #include "hnd_launch.h"
 #include "hnd_host_util.h"
 
@@ -53,8 +54,14 @@ cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, i
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   const long long per = spec_per_channel(d);
-  k_spec_pack<<<grid_for(per * nc, 256), 256, 0, st>>>(grid, static_cast<float2*>(spectrum), d, c0, nc,
-                                                       static_cast<float>(1.0 / static_cast<double>(gsz)));
+  const float scale = static_cast<float>(1.0 / static_cast<double>(gsz));
+  if (use_v2_2d(ndim, n)) {
+    float4* out = static_cast<float4*>(spectrum) + static_cast<long long>(c0) * (per / 2);
+    hnd2::k_spec_import_v2<<<grid_for(per / 2 * nc, 256), 256, 0, st>>>(grid, out, n[0], n[1], nc, 2LL * n[1],
+                                                                        scale);
+  } else {
+    k_spec_pack<<<grid_for(per * nc, 256), 256, 0, st>>>(grid, static_cast<float2*>(spectrum), d, c0, nc, scale);
+  }
   return cudaGetLastError();
 }
 
@@ -62,11 +69,33 @@ cudaError_t launch_spec_convert(int ndim, const int* n, long long C, const void*
                                 cudaStream_t st) {
   const SpecDims d = make_dims(ndim, n);
   const long long total = spec_per_channel(d) * C;
+  if (use_v2_2d(ndim, n)) {
+    if (to_natural)
+      hnd2::k_spec_export_v2<<<grid_for(total / 2, 256), 256, 0, st>>>(static_cast<const float4*>(src),
+                                                                      static_cast<float2*>(dst), n[0], n[1], C);
+    else
+      hnd2::k_spec_import_v2<<<grid_for(total / 2, 256), 256, 0, st>>>(static_cast<const float2*>(src),
+                                                                      static_cast<float4*>(dst), n[0], n[1], C,
+                                                                      n[1] + 1, 1.0f);
+    return cudaGetLastError();
+  }
   if (to_natural)
     k_spec_export<<<grid_for(total, 256), 256, 0, st>>>(static_cast<const float2*>(src), static_cast<float2*>(dst), d, C);
   else
     k_spec_import<<<grid_for(total, 256), 256, 0, st>>>(static_cast<const float2*>(src), static_cast<float2*>(dst), d, C);
   return cudaGetLastError();
+}
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    cached[dev] = v;
+  }
+  return cached[dev];
 }
 
 cudaError_t launch_bounded_wait(int* status, const int* flag, long long limit_cycles, cudaStream_t st) {
