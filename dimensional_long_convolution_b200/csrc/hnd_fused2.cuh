@@ -92,25 +92,187 @@ struct Act<__nv_bfloat16> {
 };
 
 // ------------------------------------------------------------ the kernel
+// 512 threads = two groups of 8 warps.  Volumes are software-pipelined with
+// two Zb buffers: in phase A group 0 finishes volume i (inverse rows, crop,
+// gate, store) while group 1 starts volume i+1 (forward rows); in phase B all
+// 16 warps run the column stage of volume i+1.  Two barriers per volume and
+// every warp busy in both phases.  k, v (for the forward rows) and q (for the
+// output gate) arrive by bulk asynchronous copies one phase ahead.
+constexpr int kT3 = 512;
+constexpr int kW3 = kT3 / 32;
+
 template <int N0, int N1, class T>
-struct F2 {
+struct F3 {
   static constexpr int PITCH = (N1 * static_cast<int>(sizeof(T)) / 4 + 8) * 4 / static_cast<int>(sizeof(T));
   static constexpr int RPS = N0 / 2 + 1;                 // Zb pitch (float2) per frequency row
   static constexpr size_t kTabs = Tabs<N0>::kBytes + (N0 == N1 ? 0 : Tabs<N1>::kBytes);
-  static constexpr size_t kStage = static_cast<size_t>(N0) * PITCH * sizeof(T);
+  static constexpr size_t kStage = static_cast<size_t>(N0) * PITCH * sizeof(T);   // one plane
   static constexpr size_t kZb = sizeof(float2) * 2 * N1 * RPS;
-  static constexpr size_t kX = 4096 * kW;                // exchange buffers (float4 per pencil slot)
-  static constexpr size_t kBytes = 16 + kTabs + 2 * kStage + kZb + kX;
+  static constexpr size_t kX = 4096 * kW3;
+  static constexpr size_t kBytes = 32 + kTabs + 3 * kStage + 2 * kZb + kX;
 };
 
+// Row-stage work of one warp group (8 warps): forward rows of a volume.
 template <int N0, int N1, class T>
-__global__ void __launch_bounds__(kT, 2)
-    k_fused2d_v2(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+__device__ __forceinline__ void rows_fwd(const T* kst, const T* vst, float2* Zb, float4* xb, Tabs<N1> t1, int gw,
+                                         int lane) {
+  using L = F3<N0, N1, T>;
+  constexpr int G = P2<N1>::G, PPW = 32 / G;
+  const int pen = lane / G, g = lane % G;
+  const unsigned mask = pmask<N1>(lane);
+  const int key = pkey<N1>(pen);
+  float4* buf = xb + pen * N1;
+  for (int r0 = gw * PPW; r0 < N0 / 2; r0 += 8 * PPW) {
+    const int rp = r0 + pen;
+    const bool act = rp < N0 / 2;
+    float2 z[8];
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      const int j = g + s * G;
+      const int ra = rp * L::PITCH + j, rb = (rp + N0 / 2) * L::PITCH + j;
+      z[s] = act ? make_float2(Act<T>::ld_s(kst + ra) * Act<T>::ld_s(vst + ra),
+                               Act<T>::ld_s(kst + rb) * Act<T>::ld_s(vst + rb))
+                 : make_float2(0.f, 0.f);
+    }
+    cp x[8];
+    padded_fwd<N1>(z, x, g, buf, key, t1, mask);
+    if (act) {
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        const int kk = 2 * spec_idx<N1>(g, s);
+        Zb[kk * L::RPS + rp] = make_float2(x[s].re.x, x[s].im.x);
+        Zb[(kk + 1) * L::RPS + rp] = make_float2(x[s].re.y, x[s].im.y);
+      }
+    }
+  }
+}
+
+// Inverse rows, crop, output gate and store of one volume (8 warps).
+template <int N0, int N1, class T>
+__device__ __forceinline__ void rows_inv(const T* qst, const float2* Zb, T* yp, float4* xb, Tabs<N1> t1, int gw,
+                                         int lane) {
+  using L = F3<N0, N1, T>;
+  constexpr int G = P2<N1>::G, PPW = 32 / G;
+  const int pen = lane / G, g = lane % G;
+  const unsigned mask = pmask<N1>(lane);
+  const int key = pkey<N1>(pen);
+  float4* buf = xb + pen * N1;
+  for (int r0 = gw * PPW; r0 < N0 / 2; r0 += 8 * PPW) {
+    const int rp = r0 + pen;
+    const bool act = rp < N0 / 2;
+    cp x[8];
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      const int kk = 2 * spec_idx<N1>(g, s);
+      const float2 e = act ? Zb[kk * L::RPS + rp] : make_float2(0.f, 0.f);
+      const float2 d = act ? Zb[(kk + 1) * L::RPS + rp] : make_float2(0.f, 0.f);
+      x[s] = {make_float2(e.x, d.x), make_float2(e.y, d.y)};
+    }
+    float2 o[8];
+    padded_inv<N1>(x, o, g, buf, key, t1, mask);
+    if (act) {
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        const int j = g + s * G;
+        const float qa = Act<T>::ld_s(qst + rp * L::PITCH + j);
+        const float qb = Act<T>::ld_s(qst + (rp + N0 / 2) * L::PITCH + j);
+        Act<T>::st_g(yp + static_cast<long long>(rp) * N1 + j, o[s].x * qa);
+        Act<T>::st_g(yp + static_cast<long long>(rp + N0 / 2) * N1 + j, o[s].y * qb);
+      }
+    }
+  }
+}
+
+// Column stage of one volume by all 16 warps.  Unit cu = last-axis frequency
+// kx (cu >= 1) or the combined DC/Nyquist unit (cu = 0).  The pencils of a
+// warp take units 8 apart (bank groups of Zb reads); the warp that owns unit
+// 0 runs the general product A Z + B conj(Z[-k]) for all its pencils so the
+// warp does not diverge.
+template <int N0, int N1, class T>
+__device__ __forceinline__ void columns(float2* Zb, float4* xb, const float4* __restrict__ sp, Tabs<N0> t0,
+                                        int warp, int lane) {
+  using L = F3<N0, N1, T>;
+  constexpr int G = P2<N0>::G, PPW = 32 / G;
+  constexpr int SLOTS = kW3 * PPW;
+  const int pen = lane / G, g = lane % G;
+  const unsigned mask = pmask<N0>(lane);
+  const int key = pkey<N0>(pen);
+  float4* buf = xb + pen * N0;
+  const int sidx = pen * 8 + (warp & 7) + (warp >> 3) * (8 * PPW);
+  for (int round = 0; round * SLOTS < N1; ++round) {
+    const int cu = round * SLOTS + sidx;
+    const bool act = cu < N1;
+    const bool general = round == 0 && warp == 0;      // this warp holds unit 0
+    const int kx = cu, kxm = 2 * N1 - cu;
+    float4 S[8];
+    if (act) {
+      const float4* su = sp + (cu == 0 ? 0LL : static_cast<long long>(cu + 1) * N0);
+#pragma unroll
+      for (int s = 0; s < 8; ++s) S[s] = __ldg(su + s * G + g);
+    }
+    float2 z[8];
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const int rp = g + s * G;
+      float2 z1 = make_float2(0.f, 0.f), z2 = z1;
+      if (act) {
+        z1 = Zb[kx * L::RPS + rp];
+        z2 = Zb[(cu == 0 ? N1 : kxm) * L::RPS + rp];
+      }
+      if (cu == 0) {
+        z[s] = make_float2(z1.x, z2.x);       // row a: (DC, Nyquist)
+        z[s + 4] = make_float2(z1.y, z2.y);   // row b
+      } else {
+        z[s] = unpack_a(z1, z2);
+        z[s + 4] = unpack_b(z1, z2);
+      }
+    }
+    cp x[8];
+    padded_fwd<N0>(z, x, g, buf, key, t0, mask);
+    if (general) {
+      cp xp[8];
+      fetch_partner<N0>(x, xp, g, buf, key, mask);
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        float4 Bc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (cu == 0) Bc = __ldg(sp + N0 + s * G + g);
+        const cp a = cmulp(x[s], make_float2(S[s].x, S[s].y), make_float2(S[s].z, S[s].w));
+        const cp xc = {xp[s].re, make_float2(-xp[s].im.x, -xp[s].im.y)};
+        const cp bb = cmulp(xc, make_float2(Bc.x, Bc.y), make_float2(Bc.z, Bc.w));
+        x[s] = cadd(a, bb);
+      }
+    } else if (act) {
+#pragma unroll
+      for (int s = 0; s < 8; ++s) x[s] = cmulp(x[s], make_float2(S[s].x, S[s].y), make_float2(S[s].z, S[s].w));
+    }
+    float2 o[8];
+    padded_inv<N0>(x, o, g, buf, key, t0, mask);
+    if (act) {
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        const int rp = g + s * G;
+        const float2 ya = o[s], yb = o[s + 4];
+        if (cu == 0) {
+          Zb[rp] = make_float2(ya.x, yb.x);
+          Zb[N1 * L::RPS + rp] = make_float2(ya.y, yb.y);
+        } else {
+          Zb[kx * L::RPS + rp] = pack_pos(ya, yb);
+          Zb[kxm * L::RPS + rp] = pack_neg(ya, yb);
+        }
+      }
+    }
+  }
+}
+
+template <int N0, int N1, class T>
+__global__ void __launch_bounds__(kT3, 1)
+    k_fused2d_v3(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                  const float4* __restrict__ spec, long long sbs4, T* __restrict__ y, int B, int C, int* status) {
-  using L = F2<N0, N1, T>;
+  using L = F3<N0, N1, T>;
   extern __shared__ __align__(16) unsigned char smem[];
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem);
-  unsigned char* p = smem + 16;
+  uint64_t* bar_kv = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* bar_q = bar_kv + 1;
+  unsigned char* p = smem + 32;
   const Tabs<N0> t0 = tabs_at<N0>(p);
   Tabs<N1> t1;
   if constexpr (N0 == N1) {
@@ -121,207 +283,109 @@ __global__ void __launch_bounds__(kT, 2)
   p += L::kTabs;
   T* kst = reinterpret_cast<T*>(p);
   T* vst = reinterpret_cast<T*>(p + L::kStage);
-  float2* Zb = reinterpret_cast<float2*>(p + 2 * L::kStage);
-  float4* xb = reinterpret_cast<float4*>(p + 2 * L::kStage + L::kZb);
+  T* qst = reinterpret_cast<T*>(p + 2 * L::kStage);
+  float2* Zb0 = reinterpret_cast<float2*>(p + 3 * L::kStage);
+  float2* Zb1 = reinterpret_cast<float2*>(p + 3 * L::kStage + L::kZb);
+  float4* xb = reinterpret_cast<float4*>(p + 3 * L::kStage + 2 * L::kZb);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = warp >> 3, gw = warp & 7;
+  float4* xw = xb + warp * 256;
   const int nvol = B * C;
-  int vol = blockIdx.x;
-  if (vol >= nvol) return;
+  const int v0 = blockIdx.x;
+  if (v0 >= nvol) return;
   constexpr long long Lv = static_cast<long long>(N0) * N1;
-  constexpr unsigned kvBytes = 2u * N0 * N1 * sizeof(T);
 
   tabs_build<N0>(t0, g_tw512);
   if constexpr (N0 != N1) tabs_build<N1>(t1, g_tw512);
 
-  // issue the bulk copies of k and v rows of volume `vv` into the staging pitch
-  auto issue_kv = [&](int vv) {
+  auto vol_base = [&](int vv) {
     const int cc = vv / B, bb = vv % B;
-    const long long base = (static_cast<long long>(bb) * C + cc) * Lv;
-    if (lane == 0) mbar_expect_tx(bar, kvBytes);
-    __syncwarp();
-    for (int r = lane; r < 2 * N0; r += 32) {
+    return (static_cast<long long>(bb) * C + cc) * Lv;
+  };
+  // Bulk row copies, one row per thread.  Every copying thread first arrives
+  // on the barrier with the bytes it will deliver (barrier counts: 2 N0 for
+  // k and v, N0 for q), so a phase completes only when all rows have landed.
+  // Copies are only issued after a CTA barrier that follows the previous
+  // phase's completion and the last reads of the staging buffer.
+  auto copy_kv = [&](int vv) {
+    const long long base = vol_base(vv);
+    const int r = threadIdx.x;
+    if (r < 2 * N0) {
       const int row = r % N0;
       const T* src = (r < N0 ? k : v) + base + static_cast<long long>(row) * N1;
-      T* dst = (r < N0 ? kst : vst) + row * L::PITCH;
-      bulk_g2s(dst, src, N1 * sizeof(T), bar);
+      fence_proxy_async();
+      mbar_expect_tx(bar_kv, N1 * sizeof(T));
+      bulk_g2s((r < N0 ? kst : vst) + row * L::PITCH, src, N1 * sizeof(T), bar_kv);
+    }
+  };
+  auto copy_q = [&](int vv) {
+    const long long base = vol_base(vv);
+    const int r = threadIdx.x;
+    if (r < N0) {
+      fence_proxy_async();
+      mbar_expect_tx(bar_q, N1 * sizeof(T));
+      bulk_g2s(qst + r * L::PITCH, q + base + static_cast<long long>(r) * N1, N1 * sizeof(T), bar_q);
     }
   };
 
   if (threadIdx.x == 0) {
-    mbar_init(bar, 1);
+    mbar_init(bar_kv, 2 * N0);
+    mbar_init(bar_q, N0);
     fence_mbar_init();
   }
   __syncthreads();
-  if (warp == 0) issue_kv(vol);
-  unsigned phase = 0;
+  copy_kv(v0);
+  copy_q(v0);
+  unsigned ph_kv = 0, ph_q = 0;
+  bool ok = true;
 
-  for (; vol < nvol; vol += gridDim.x) {
+  // prologue: forward rows of the first volume by group 1
+  if (grp == 1) {
+    ok = mbar_wait_bounded(bar_kv, ph_kv, status);
+    if (ok) rows_fwd<N0, N1, T>(kst, vst, Zb0, xw, t1, gw, lane);
+  }
+  int vol = v0;
+  int next = vol + gridDim.x;
+  if (!__syncthreads_and(ok)) {
+    // a copy never arrived: one more bounded wait for the copies in flight, then stop
+    mbar_wait_bounded(bar_kv, ph_kv, nullptr);
+    mbar_wait_bounded(bar_q, ph_q, nullptr);
+    return;
+  }
+  ph_kv ^= 1u;
+  if (next < nvol) copy_kv(next);
+
+  for (int i = 0; vol < nvol; ++i, vol = next, next += gridDim.x) {
     const int c = vol / B, b = vol % B;
-    const long long pair = static_cast<long long>(b) * C + c;
-    const T* qp = q + pair * Lv;
-    T* yp = y + pair * Lv;
-    const int next = vol + gridDim.x;
+    float2* Zc = (i & 1) ? Zb1 : Zb0;
+    float2* Zn = (i & 1) ? Zb0 : Zb1;
+    const float4* sp = spec + static_cast<long long>(b) * sbs4 + static_cast<long long>(c) * (N1 + 1) * N0;
 
-    if (!mbar_wait_bounded(bar, phase, status)) {
-      mbar_wait_bounded(bar, phase, nullptr);     // one more bounded wait for copies in flight
+    // phase B: columns of `vol`
+    columns<N0, N1, T>(Zc, xw, sp, t0, warp, lane);
+    __syncthreads();
+
+    // phase A: group 0 finishes `vol`, group 1 starts `next`
+    ok = true;
+    if (grp == 0) {
+      ok = mbar_wait_bounded(bar_q, ph_q, status);
+      if (ok) rows_inv<N0, N1, T>(qst, Zc, y + (static_cast<long long>(b) * C + c) * Lv, xw, t1, gw, lane);
+    } else if (next < nvol) {
+      ok = mbar_wait_bounded(bar_kv, ph_kv, status);
+      if (ok) rows_fwd<N0, N1, T>(kst, vst, Zn, xw, t1, gw, lane);
+    }
+    const int next2 = next + gridDim.x;
+    if (!__syncthreads_and(ok)) {
+      // a copy never arrived: one more bounded wait for the copies in flight, then stop
+      mbar_wait_bounded(bar_q, ph_q, nullptr);
+      if (next < nvol) mbar_wait_bounded(bar_kv, ph_kv, nullptr);
       return;
     }
-    phase ^= 1u;
-
-    // ---- stage 1: row pairs (rp, rp + N0/2) forward along axis 1
-    {
-      constexpr int G = P2<N1>::G, PPW = 32 / G;
-      const int pen = lane / G, g = lane % G;
-      const unsigned mask = pmask<N1>(lane);
-      const int key = pkey<N1>(pen);
-      float4* buf = xb + warp * 256 + pen * N1;
-      for (int r0 = warp * PPW; r0 < N0 / 2; r0 += kW * PPW) {
-        const int rp = r0 + pen;
-        const bool act = rp < N0 / 2;
-        float2 z[8];
-#pragma unroll
-        for (int s = 0; s < 8; ++s) {
-          const int j = g + s * G;
-          const int ra = rp * L::PITCH + j, rb = (rp + N0 / 2) * L::PITCH + j;
-          z[s] = act ? make_float2(Act<T>::ld_s(kst + ra) * Act<T>::ld_s(vst + ra),
-                                   Act<T>::ld_s(kst + rb) * Act<T>::ld_s(vst + rb))
-                     : make_float2(0.f, 0.f);
-        }
-        cp x[8];
-        padded_fwd<N1>(z, x, g, buf, key, t1, mask);
-        if (act) {
-#pragma unroll
-          for (int s = 0; s < 8; ++s) {
-            const int kk = 2 * spec_idx<N1>(g, s);
-            Zb[kk * L::RPS + rp] = make_float2(x[s].re.x, x[s].im.x);
-            Zb[(kk + 1) * L::RPS + rp] = make_float2(x[s].re.y, x[s].im.y);
-          }
-        }
-      }
-    }
-    __syncthreads();
-    if (warp == 0 && next < nvol) {
-      fence_proxy_async();
-      issue_kv(next);
-    }
-
-    // ---- stage 2: columns; pencils of a warp take units 8 apart
-    {
-      constexpr int G = P2<N0>::G, PPW = 32 / G;
-      const int pen = lane / G, g = lane % G;
-      const unsigned mask = pmask<N0>(lane);
-      const int key = pkey<N0>(pen);
-      float4* buf = xb + warp * 256 + pen * N0;
-      const float4* sp = spec + static_cast<long long>(b) * sbs4 + static_cast<long long>(c) * (N1 + 1) * N0;
-      for (int round = 0; round * kW * PPW < N1; ++round) {
-        const int cu = round * kW * PPW + pen * kW + warp;
-        const bool act = cu < N1;
-        const int kx = cu, kxm = 2 * N1 - cu;
-        float2 z[8];
-        cp x[8];
-        if (cu == 0) {
-          // DC and Nyquist columns (both real) as one complex column
-#pragma unroll
-          for (int s = 0; s < 4; ++s) {
-            const int rp = g + s * G;
-            const float2 z0 = Zb[rp], zn = Zb[N1 * L::RPS + rp];
-            z[s] = make_float2(z0.x, zn.x);
-            z[s + 4] = make_float2(z0.y, zn.y);
-          }
-          padded_fwd<N0>(z, x, g, buf, key, t0, mask);
-          cp xp[8];
-          fetch_partner<N0>(x, xp, g, buf, key, mask);
-#pragma unroll
-          for (int s = 0; s < 8; ++s) {
-            const float4 A = __ldg(sp + s * G + g), Bc = __ldg(sp + N0 + s * G + g);
-            const cp a = cmulp(x[s], make_float2(A.x, A.y), make_float2(A.z, A.w));
-            const cp xc = {xp[s].re, make_float2(-xp[s].im.x, -xp[s].im.y)};
-            const cp bb = cmulp(xc, make_float2(Bc.x, Bc.y), make_float2(Bc.z, Bc.w));
-            x[s] = cadd(a, bb);
-          }
-        } else {
-          float4 S[8];
-          if (act) {
-            const float4* su = sp + static_cast<long long>(cu + 1) * N0;
-#pragma unroll
-            for (int s = 0; s < 8; ++s) S[s] = __ldg(su + s * G + g);
-          }
-#pragma unroll
-          for (int s = 0; s < 4; ++s) {
-            const int rp = g + s * G;
-            float2 z1 = make_float2(0.f, 0.f), z2 = z1;
-            if (act) {
-              z1 = Zb[kx * L::RPS + rp];
-              z2 = Zb[kxm * L::RPS + rp];
-            }
-            z[s] = unpack_a(z1, z2);
-            z[s + 4] = unpack_b(z1, z2);
-          }
-          padded_fwd<N0>(z, x, g, buf, key, t0, mask);
-          if (act) {
-#pragma unroll
-            for (int s = 0; s < 8; ++s) x[s] = cmulp(x[s], make_float2(S[s].x, S[s].y), make_float2(S[s].z, S[s].w));
-          }
-        }
-        float2 o[8];
-        padded_inv<N0>(x, o, g, buf, key, t0, mask);
-        if (act) {
-#pragma unroll
-          for (int s = 0; s < 4; ++s) {
-            const int rp = g + s * G;
-            const float2 ya = o[s], yb = o[s + 4];
-            if (cu == 0) {
-              Zb[rp] = make_float2(ya.x, yb.x);
-              Zb[N1 * L::RPS + rp] = make_float2(ya.y, yb.y);
-            } else {
-              Zb[kx * L::RPS + rp] = pack_pos(ya, yb);
-              Zb[kxm * L::RPS + rp] = pack_neg(ya, yb);
-            }
-          }
-        }
-      }
-    }
-    __syncthreads();
-
-    // ---- stage 3: inverse rows, crop, output gate
-    {
-      constexpr int G = P2<N1>::G, PPW = 32 / G;
-      const int pen = lane / G, g = lane % G;
-      const unsigned mask = pmask<N1>(lane);
-      const int key = pkey<N1>(pen);
-      float4* buf = xb + warp * 256 + pen * N1;
-      for (int r0 = warp * PPW; r0 < N0 / 2; r0 += kW * PPW) {
-        const int rp = r0 + pen;
-        const bool act = rp < N0 / 2;
-        float qa[8], qb[8];
-#pragma unroll
-        for (int s = 0; s < 8; ++s) {
-          const long long ja = static_cast<long long>(rp) * N1 + g + s * G;
-          qa[s] = act ? Act<T>::ld_g(qp + ja) : 0.f;
-          qb[s] = act ? Act<T>::ld_g(qp + ja + (N0 / 2) * N1) : 0.f;
-        }
-        cp x[8];
-#pragma unroll
-        for (int s = 0; s < 8; ++s) {
-          const int kk = 2 * spec_idx<N1>(g, s);
-          const float2 e = act ? Zb[kk * L::RPS + rp] : make_float2(0.f, 0.f);
-          const float2 d = act ? Zb[(kk + 1) * L::RPS + rp] : make_float2(0.f, 0.f);
-          x[s] = {make_float2(e.x, d.x), make_float2(e.y, d.y)};
-        }
-        float2 o[8];
-        padded_inv<N1>(x, o, g, buf, key, t1, mask);
-        if (act) {
-#pragma unroll
-          for (int s = 0; s < 8; ++s) {
-            const long long ja = static_cast<long long>(rp) * N1 + g + s * G;
-            Act<T>::st_g(yp + ja, o[s].x * qa[s]);
-            Act<T>::st_g(yp + ja + (N0 / 2) * N1, o[s].y * qb[s]);
-          }
-        }
-      }
-    }
-    __syncthreads();
+    ph_q ^= 1u;
+    if (next < nvol) ph_kv ^= 1u;
+    if (next < nvol) copy_q(next);
+    if (next2 < nvol) copy_kv(next2);
   }
 }
 
