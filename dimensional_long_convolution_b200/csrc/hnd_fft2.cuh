@@ -142,18 +142,19 @@ __host__ __device__ __forceinline__ int spec_idx(int g, int s) {
   }
 }
 
-// Swizzled float4 index inside a pencil's exchange buffer: the low three bits
-// are XORed with bits 3-5 and 4-6, which keeps every pass's 8-lane phase on
-// distinct 16-byte bank groups (a bijection inside each aligned block of 8).
-__host__ __device__ __forceinline__ int swz(int i) { return i ^ (((i >> 3) ^ (i >> 4)) & 7); }
+// Padded float4 index inside a pencil's exchange buffer (one pad slot every
+// 8): for the 8-lane phases of both passes the lanes land on distinct
+// 16-byte bank groups, and with the thread's lane index folded into a base
+// pointer every access is a compile-time offset.  A pencil's buffer holds
+// N + N/8 float4.
+__host__ __device__ __forceinline__ int swz(int i) { return i + (i >> 3); }
 
-// Per-pencil key XORed into the low bits so that pencils sharing an 8-lane
-// phase (G < 8) land on disjoint bank groups.
+// Exchange-buffer float4 per pencil; the pencil stride keeps pencils that
+// share an 8-lane phase (G < 8) on different bank groups.
 template <int N>
-__device__ __forceinline__ int pkey(int pen) {
-  constexpr int G = N / 8 < 1 ? 1 : N / 8;
-  return (pen * G) & 7;
-}
+struct XB { static constexpr int kPen = N + N / 8; };
+template <int N>
+__device__ __forceinline__ int pkey(int) { return 0; }
 
 template <int N>
 __device__ __forceinline__ unsigned pmask(int lane) {
@@ -218,10 +219,10 @@ __device__ __forceinline__ void fft_fwd(cp (&x)[8], int g, float4* buf, int key,
   if constexpr (P2<N>::TWO) {
     constexpr int G = P2<N>::G, R2 = P2<N>::R2;
     // pass-1 output index j*8 + r (j = g): write, then read pass-2 inputs j' + r*8
-    __syncwarp(mask);
+    __syncwarp();
 #pragma unroll
     for (int r = 0; r < 8; ++r) buf[swz(g * 8 + r) ^ key] = make_float4(x[r].re.x, x[r].re.y, x[r].im.x, x[r].im.y);
-    __syncwarp(mask);
+    __syncwarp();
 #pragma unroll
     for (int b = 0; b < 8 / R2; ++b) {
 #pragma unroll
@@ -253,7 +254,7 @@ __device__ __forceinline__ void fft_inv(cp (&x)[8], int g, float4* buf, int key,
       else dft2(x[b * 2], x[b * 2 + 1]);
     }
     // output index (j) * R2 + r ; read pass-2 inputs g + r*G with twiddle W_N^{-g r}
-    __syncwarp(mask);
+    __syncwarp();
 #pragma unroll
     for (int b = 0; b < 8 / R2; ++b) {
 #pragma unroll
@@ -262,7 +263,7 @@ __device__ __forceinline__ void fft_inv(cp (&x)[8], int g, float4* buf, int key,
         buf[swz((g + G * b) * R2 + r) ^ key] = make_float4(x[s].re.x, x[s].re.y, x[s].im.x, x[s].im.y);
       }
     }
-    __syncwarp(mask);
+    __syncwarp();
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const float4 v = buf[swz(g + r * G) ^ key];
@@ -311,11 +312,11 @@ __device__ __forceinline__ void padded_inv(cp (&x)[8], float2 (&out)[8], int g, 
 // mod N, path 1 -> N - 1 - f (both as natural half-frequency indices).
 template <int N>
 __device__ __forceinline__ void fetch_partner(const cp (&x)[8], cp (&xp)[8], int g, float4* buf, int key, unsigned mask) {
-  __syncwarp(mask);
+  __syncwarp();
 #pragma unroll
   for (int s = 0; s < 8; ++s)
     buf[swz(spec_idx<N>(g, s)) ^ key] = make_float4(x[s].re.x, x[s].re.y, x[s].im.x, x[s].im.y);
-  __syncwarp(mask);
+  __syncwarp();
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
     const int f = spec_idx<N>(g, s);

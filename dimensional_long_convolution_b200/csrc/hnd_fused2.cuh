@@ -107,21 +107,21 @@ struct F3 {
   static constexpr int RPS = N0 / 2 + 1;                 // Zb pitch (float2) per frequency row
   static constexpr size_t kTabs = Tabs<N0>::kBytes + (N0 == N1 ? 0 : Tabs<N1>::kBytes);
   static constexpr size_t kStage = static_cast<size_t>(N0) * PITCH * sizeof(T);   // one plane
-  static constexpr size_t kZb = sizeof(float2) * 2 * N1 * RPS;
-  static constexpr size_t kX = 4096 * kW3;
+  static constexpr size_t kZb = sizeof(float4) * N1 * RPS;    // [f][rp] float4
+  static constexpr size_t kX = 4608 * kW3;
   static constexpr size_t kBytes = 32 + kTabs + 3 * kStage + 2 * kZb + kX;
 };
 
 // Row-stage work of one warp group (8 warps): forward rows of a volume.
 template <int N0, int N1, class T>
-__device__ __forceinline__ void rows_fwd(const T* kst, const T* vst, float2* Zb, float4* xb, Tabs<N1> t1, int gw,
+__device__ __forceinline__ void rows_fwd(const T* kst, const T* vst, float4* Zb, float4* xb, Tabs<N1> t1, int gw,
                                          int lane) {
   using L = F3<N0, N1, T>;
   constexpr int G = P2<N1>::G, PPW = 32 / G;
   const int pen = lane / G, g = lane % G;
   const unsigned mask = pmask<N1>(lane);
   const int key = pkey<N1>(pen);
-  float4* buf = xb + pen * N1;
+  float4* buf = xb + pen * XB<N1>::kPen;
   for (int r0 = gw * PPW; r0 < N0 / 2; r0 += 8 * PPW) {
     const int rp = r0 + pen;
     const bool act = rp < N0 / 2;
@@ -138,35 +138,30 @@ __device__ __forceinline__ void rows_fwd(const T* kst, const T* vst, float2* Zb,
     padded_fwd<N1>(z, x, g, buf, key, t1, mask);
     if (act) {
 #pragma unroll
-      for (int s = 0; s < 8; ++s) {
-        const int kk = 2 * spec_idx<N1>(g, s);
-        Zb[kk * L::RPS + rp] = make_float2(x[s].re.x, x[s].im.x);
-        Zb[(kk + 1) * L::RPS + rp] = make_float2(x[s].re.y, x[s].im.y);
-      }
+      for (int s = 0; s < 8; ++s)
+        Zb[spec_idx<N1>(g, s) * L::RPS + rp] = make_float4(x[s].re.x, x[s].im.x, x[s].re.y, x[s].im.y);
     }
   }
 }
 
 // Inverse rows, crop, output gate and store of one volume (8 warps).
 template <int N0, int N1, class T>
-__device__ __forceinline__ void rows_inv(const T* qst, const float2* Zb, T* yp, float4* xb, Tabs<N1> t1, int gw,
+__device__ __forceinline__ void rows_inv(const T* qst, const float4* Zb, T* yp, float4* xb, Tabs<N1> t1, int gw,
                                          int lane) {
   using L = F3<N0, N1, T>;
   constexpr int G = P2<N1>::G, PPW = 32 / G;
   const int pen = lane / G, g = lane % G;
   const unsigned mask = pmask<N1>(lane);
   const int key = pkey<N1>(pen);
-  float4* buf = xb + pen * N1;
+  float4* buf = xb + pen * XB<N1>::kPen;
   for (int r0 = gw * PPW; r0 < N0 / 2; r0 += 8 * PPW) {
     const int rp = r0 + pen;
     const bool act = rp < N0 / 2;
     cp x[8];
 #pragma unroll
     for (int s = 0; s < 8; ++s) {
-      const int kk = 2 * spec_idx<N1>(g, s);
-      const float2 e = act ? Zb[kk * L::RPS + rp] : make_float2(0.f, 0.f);
-      const float2 d = act ? Zb[(kk + 1) * L::RPS + rp] : make_float2(0.f, 0.f);
-      x[s] = {make_float2(e.x, d.x), make_float2(e.y, d.y)};
+      const float4 e = act ? Zb[spec_idx<N1>(g, s) * L::RPS + rp] : make_float4(0.f, 0.f, 0.f, 0.f);
+      x[s] = {make_float2(e.x, e.z), make_float2(e.y, e.w)};
     }
     float2 o[8];
     padded_inv<N1>(x, o, g, buf, key, t1, mask);
@@ -184,26 +179,31 @@ __device__ __forceinline__ void rows_inv(const T* qst, const float2* Zb, T* yp, 
 }
 
 // Column stage of one volume by all 16 warps.  Unit cu = last-axis frequency
-// kx (cu >= 1) or the combined DC/Nyquist unit (cu = 0).  The pencils of a
-// warp take units 8 apart (bank groups of Zb reads); the warp that owns unit
-// 0 runs the general product A Z + B conj(Z[-k]) for all its pencils so the
-// warp does not diverge.
+// kx (cu >= 1) or the combined DC/Nyquist unit (cu = 0).  Zb holds, per
+// half-frequency f and row pair, the two padded frequencies 2f and 2f+1 side
+// by side, so frequency kx lives at float2 (f RPS + rp) 2 + (kx & 1); the
+// pencils of a warp take adjacent units, which puts the two pencils of a
+// 16-lane phase on opposite bank parities.  The warp that owns unit 0 runs the
+// general product A Z + B conj(Z[-k]) for all its pencils so it does not
+// diverge.
 template <int N0, int N1, class T>
-__device__ __forceinline__ void columns(float2* Zb, float4* xb, const float4* __restrict__ sp, Tabs<N0> t0,
+__device__ __forceinline__ void columns(float4* Zb4, float4* xb, const float4* __restrict__ sp, Tabs<N0> t0,
                                         int warp, int lane) {
   using L = F3<N0, N1, T>;
   constexpr int G = P2<N0>::G, PPW = 32 / G;
   constexpr int SLOTS = kW3 * PPW;
+  float2* Zb = reinterpret_cast<float2*>(Zb4);
   const int pen = lane / G, g = lane % G;
   const unsigned mask = pmask<N0>(lane);
   const int key = pkey<N0>(pen);
-  float4* buf = xb + pen * N0;
-  const int sidx = pen * 8 + (warp & 7) + (warp >> 3) * (8 * PPW);
+  float4* buf = xb + pen * XB<N0>::kPen;
+  const int sidx = warp * PPW + pen;
+  auto zidx = [](int kk, int rp) { return ((kk >> 1) * L::RPS + rp) * 2 + (kk & 1); };
   for (int round = 0; round * SLOTS < N1; ++round) {
     const int cu = round * SLOTS + sidx;
     const bool act = cu < N1;
     const bool general = round == 0 && warp == 0;      // this warp holds unit 0
-    const int kx = cu, kxm = 2 * N1 - cu;
+    const int kx = cu, kxm = cu == 0 ? N1 : 2 * N1 - cu;
     float4 S[8];
     if (act) {
       const float4* su = sp + (cu == 0 ? 0LL : static_cast<long long>(cu + 1) * N0);
@@ -216,8 +216,8 @@ __device__ __forceinline__ void columns(float2* Zb, float4* xb, const float4* __
       const int rp = g + s * G;
       float2 z1 = make_float2(0.f, 0.f), z2 = z1;
       if (act) {
-        z1 = Zb[kx * L::RPS + rp];
-        z2 = Zb[(cu == 0 ? N1 : kxm) * L::RPS + rp];
+        z1 = Zb[zidx(kx, rp)];
+        z2 = Zb[zidx(kxm, rp)];
       }
       if (cu == 0) {
         z[s] = make_float2(z1.x, z2.x);       // row a: (DC, Nyquist)
@@ -253,15 +253,22 @@ __device__ __forceinline__ void columns(float2* Zb, float4* xb, const float4* __
         const int rp = g + s * G;
         const float2 ya = o[s], yb = o[s + 4];
         if (cu == 0) {
-          Zb[rp] = make_float2(ya.x, yb.x);
-          Zb[N1 * L::RPS + rp] = make_float2(ya.y, yb.y);
+          Zb[zidx(0, rp)] = make_float2(ya.x, yb.x);
+          Zb[zidx(N1, rp)] = make_float2(ya.y, yb.y);
         } else {
-          Zb[kx * L::RPS + rp] = pack_pos(ya, yb);
-          Zb[kxm * L::RPS + rp] = pack_neg(ya, yb);
+          Zb[zidx(kx, rp)] = pack_pos(ya, yb);
+          Zb[zidx(kxm, rp)] = pack_neg(ya, yb);
         }
       }
     }
   }
+}
+
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ void named_arrive(int id, int nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 template <int N0, int N1, class T>
@@ -284,13 +291,13 @@ __global__ void __launch_bounds__(kT3, 1)
   T* kst = reinterpret_cast<T*>(p);
   T* vst = reinterpret_cast<T*>(p + L::kStage);
   T* qst = reinterpret_cast<T*>(p + 2 * L::kStage);
-  float2* Zb0 = reinterpret_cast<float2*>(p + 3 * L::kStage);
-  float2* Zb1 = reinterpret_cast<float2*>(p + 3 * L::kStage + L::kZb);
+  float4* Zb0 = reinterpret_cast<float4*>(p + 3 * L::kStage);
+  float4* Zb1 = reinterpret_cast<float4*>(p + 3 * L::kStage + L::kZb);
   float4* xb = reinterpret_cast<float4*>(p + 3 * L::kStage + 2 * L::kZb);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = warp >> 3, gw = warp & 7;
-  float4* xw = xb + warp * 256;
+  float4* xw = xb + warp * 288;
   const int nvol = B * C;
   const int v0 = blockIdx.x;
   if (v0 >= nvol) return;
@@ -358,13 +365,16 @@ __global__ void __launch_bounds__(kT3, 1)
 
   for (int i = 0; vol < nvol; ++i, vol = next, next += gridDim.x) {
     const int c = vol / B, b = vol % B;
-    float2* Zc = (i & 1) ? Zb1 : Zb0;
-    float2* Zn = (i & 1) ? Zb0 : Zb1;
+    float4* Zc = (i & 1) ? Zb1 : Zb0;
+    float4* Zn = (i & 1) ? Zb0 : Zb1;
     const float4* sp = spec + static_cast<long long>(b) * sbs4 + static_cast<long long>(c) * (N1 + 1) * N0;
 
-    // phase B: columns of `vol`
+    // phase B: columns of `vol`.  Group 0 needs every column before its
+    // inverse rows; group 1 only signals and goes on to the next volume's
+    // forward rows (they touch the other Zb buffer and the staging planes).
     columns<N0, N1, T>(Zc, xw, sp, t0, warp, lane);
-    __syncthreads();
+    if (grp == 0) named_sync(1, kT3);
+    else named_arrive(1, kT3);
 
     // phase A: group 0 finishes `vol`, group 1 starts `next`
     ok = true;
