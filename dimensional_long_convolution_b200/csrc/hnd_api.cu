@@ -77,7 +77,7 @@ hyena_nd_status make_plan(const hyena_nd_problem* p, Plan* pl) {
   size_t ws_conv = 0;
   if (p->ndim == 1) {
     pl->tier = kRows1D;
-  } else if (p->ndim == 2 && pl->n[0] <= 128 && pl->n[1] <= 128) {
+  } else if (hnd::fused_2d(p->ndim, pl->n)) {
     pl->tier = kFused2D;
   } else {
     pl->tier = p->ndim == 2 ? kMulti2D : kMulti3D;

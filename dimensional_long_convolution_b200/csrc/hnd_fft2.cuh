@@ -122,13 +122,51 @@ __device__ __forceinline__ void dft8(cp* a) {
   // the even DFT4 left its outputs in b0..b3 = X0, X2, X4, X6 (set above)
 }
 
+// Natural-order DFT16 as 4 x 4: DFT4 over stride-4 inputs, twiddles
+// W16^{r1 k1}, DFT4 across; the result is read back in natural order.
+template <bool INV>
+__device__ __forceinline__ void cmul_const(cp& x, float c, float sn) {
+  // x * (c + i sn)
+  const float2 cc = f2(c), ss = f2(sn), nss = f2(-sn);
+  x = {pfma(x.im, nss, pmul(x.re, cc)), pfma(x.re, ss, pmul(x.im, cc))};
+}
+
+template <bool INV>
+__device__ __forceinline__ void dft16(cp* a) {
+  const float c1 = 0.92387953251128675613f, s1 = 0.38268343236508977173f, h = 0.70710678118654752440f;
+  const float sg = INV ? 1.f : -1.f;      // forward W16^e = exp(-2 pi i e / 16)
+#pragma unroll
+  for (int r1 = 0; r1 < 4; ++r1) dft4<INV>(a[r1], a[r1 + 4], a[r1 + 8], a[r1 + 12]);
+  // B[r1][k1] at a[r1 + 4 k1]; twiddles W16^{r1 k1}
+  cmul_const<INV>(a[1 + 4], c1, sg * s1);            // e = 1
+  cmul_const<INV>(a[2 + 4], h, sg * h);              // e = 2
+  cmul_const<INV>(a[3 + 4], s1, sg * c1);            // e = 3
+  cmul_const<INV>(a[1 + 8], h, sg * h);              // e = 2
+  a[2 + 8] = INV ? cp{make_float2(-a[10].im.x, -a[10].im.y), a[10].re}
+                 : cp{a[10].im, make_float2(-a[10].re.x, -a[10].re.y)};   // e = 4: -+i
+  cmul_const<INV>(a[3 + 8], -h, sg * h);             // e = 6
+  cmul_const<INV>(a[1 + 12], s1, sg * c1);           // e = 3
+  cmul_const<INV>(a[2 + 12], -h, sg * h);            // e = 6
+  cmul_const<INV>(a[3 + 12], -c1, -sg * s1);         // e = 9
+#pragma unroll
+  for (int k1 = 0; k1 < 4; ++k1) dft4<INV>(a[4 * k1], a[4 * k1 + 1], a[4 * k1 + 2], a[4 * k1 + 3]);
+  // X[k1 + 4 k2] sits at a[4 k1 + k2]: transpose the 4 x 4 block
+  cp t[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) t[i] = a[i];
+#pragma unroll
+  for (int k1 = 0; k1 < 4; ++k1)
+#pragma unroll
+    for (int k2 = 0; k2 < 4; ++k2) a[k1 + 4 * k2] = t[4 * k1 + k2];
+}
+
 // ------------------------------------------------------------------- plan
 template <int N>
 struct P2 {
-  static_assert(N == 8 || N == 16 || N == 32 || N == 64, "packed core: N in {8,16,32,64}");
-  static constexpr int R1 = 8;
-  static constexpr int R2 = N / 8;          // 1 (single pass), 2, 4, 8
-  static constexpr int G = (N == 8) ? 1 : R2;
+  static_assert(N == 8 || N == 16 || N == 32 || N == 64 || N == 128 || N == 256, "packed core: N in 8..256");
+  static constexpr int R1 = N >= 128 ? 16 : 8;     // slots per lane, pass-1 radix
+  static constexpr int R2 = N / R1;                // pass-2 radix: 1 (single pass), 2, 4, 8, 16
+  static constexpr int G = (N == 8) ? 1 : R2;      // lanes per pencil
   static constexpr bool TWO = N > 8;
 };
 
@@ -148,11 +186,17 @@ __host__ __device__ __forceinline__ int spec_idx(int g, int s) {
 // pointer every access is a compile-time offset.  A pencil's buffer holds
 // N + N/8 float4.
 __host__ __device__ __forceinline__ int swz(int i) { return i + (i >> 3); }
+// pad by d: one pad slot every d entries (d = 8 or 16)
+template <int D>
+__host__ __device__ __forceinline__ int padx(int i) { return i + i / D; }
 
 // Exchange-buffer float4 per pencil; the pencil stride keeps pencils that
 // share an 8-lane phase (G < 8) on different bank groups.
 template <int N>
-struct XB { static constexpr int kPen = N + N / 8; };
+struct XB {
+  static constexpr int kPen = N + N / 8;                  // float4 per pencil (covers both pads)
+  static constexpr int kWarp = (32 / P2<N>::G) * kPen;     // float4 per warp (all its pencils)
+};
 template <int N>
 __device__ __forceinline__ int pkey(int) { return 0; }
 
@@ -173,10 +217,10 @@ __device__ __forceinline__ unsigned pmask(int lane) {
 //   tst[s G + g]          = W_2N^{g + s G}      twist factors, (c, s)
 template <int N>
 struct Tabs {
-  static constexpr int G = P2<N>::G;
-  static constexpr int kTw2 = 8 * G;        // float4
-  static constexpr int kTwi = 8 * G;        // float4
-  static constexpr int kTst = 8 * G;        // float2
+  static constexpr int G = P2<N>::G, R1 = P2<N>::R1;
+  static constexpr int kTw2 = R1 * G;       // float4
+  static constexpr int kTwi = R1 * G;       // float4
+  static constexpr int kTst = R1 * G;       // float2
   static constexpr size_t kBytes = 16 * (kTw2 + kTwi) + 8 * kTst;
   float4* tw2;
   float4* twi;
@@ -199,8 +243,8 @@ __device__ __forceinline__ Tabs<N> tabs_at(unsigned char* base) {
 
 template <int N>
 __device__ __forceinline__ void tabs_build(Tabs<N> t, const float2* __restrict__ W512) {
-  constexpr int G = P2<N>::G, R2 = P2<N>::R2;
-  for (int e = threadIdx.x; e < 8 * G; e += blockDim.x) {
+  constexpr int G = P2<N>::G, R2 = P2<N>::R2, R1 = P2<N>::R1;
+  for (int e = threadIdx.x; e < R1 * G; e += blockDim.x) {
     const int g = e % G, sr = e / G;              // sr = b R2 + r (pass 2) or r (inverse) or s (twist)
     const int b = sr / (R2 > 0 ? R2 : 1), r = sr % (R2 > 0 ? R2 : 1);
     const float2 w = wtab(W512, N, (g + G * b) * r);
@@ -212,27 +256,33 @@ __device__ __forceinline__ void tabs_build(Tabs<N> t, const float2* __restrict__
 }
 
 // ------------------------------------------------------------------- FFTs
-// Forward: natural -> spectral.  buf: this pencil's N float4 (swizzled).
+// Forward: natural -> spectral.  buf: this pencil's XB<N>::kPen float4.
+// The forward exchange pads by R1, the inverse exchange by max(R2, 8): with the
+// lane index in the low bits, each 8-lane phase hits distinct 16-byte bank
+// groups, and every padded index stays below N + N/8.
 template <int N>
-__device__ __forceinline__ void fft_fwd(cp (&x)[8], int g, float4* buf, int key, Tabs<N> t, unsigned mask) {
-  dft8<false>(x);
+__device__ __forceinline__ void fft_fwd(cp (&x)[P2<N>::R1], int g, float4* buf, int key, Tabs<N> t, unsigned mask) {
+  constexpr int R1 = P2<N>::R1;
+  if constexpr (R1 == 16) dft16<false>(x);
+  else dft8<false>(x);
   if constexpr (P2<N>::TWO) {
     constexpr int G = P2<N>::G, R2 = P2<N>::R2;
-    // pass-1 output index j*8 + r (j = g): write, then read pass-2 inputs j' + r*8
     __syncwarp();
 #pragma unroll
-    for (int r = 0; r < 8; ++r) buf[swz(g * 8 + r) ^ key] = make_float4(x[r].re.x, x[r].re.y, x[r].im.x, x[r].im.y);
+    for (int r = 0; r < R1; ++r)
+      buf[padx<R1>(g * R1 + r)] = make_float4(x[r].re.x, x[r].re.y, x[r].im.x, x[r].im.y);
     __syncwarp();
 #pragma unroll
-    for (int b = 0; b < 8 / R2; ++b) {
+    for (int b = 0; b < R1 / R2; ++b) {
 #pragma unroll
       for (int r = 0; r < R2; ++r) {
-        const float4 v = buf[swz(g + G * b + r * 8) ^ key];
+        const float4 v = buf[padx<R1>(g + G * b + r * R1)];
         cp y = {make_float2(v.x, v.y), make_float2(v.z, v.w)};
         if (r > 0) y = ctw<false>(y, t.tw2[(b * R2 + r) * G + g]);
         x[b * R2 + r] = y;
       }
-      if constexpr (R2 == 8) dft8<false>(&x[b * 8]);
+      if constexpr (R2 == 16) dft16<false>(&x[b * 16]);
+      else if constexpr (R2 == 8) dft8<false>(&x[b * 8]);
       else if constexpr (R2 == 4) dft4<false>(x[b * 4], x[b * 4 + 1], x[b * 4 + 2], x[b * 4 + 3]);
       else dft2(x[b * 2], x[b * 2 + 1]);
     }
@@ -241,37 +291,39 @@ __device__ __forceinline__ void fft_fwd(cp (&x)[8], int g, float4* buf, int key,
 
 // Inverse (unnormalised): spectral -> natural.
 template <int N>
-__device__ __forceinline__ void fft_inv(cp (&x)[8], int g, float4* buf, int key, Tabs<N> t, unsigned mask) {
+__device__ __forceinline__ void fft_inv(cp (&x)[P2<N>::R1], int g, float4* buf, int key, Tabs<N> t, unsigned mask) {
+  constexpr int R1 = P2<N>::R1;
   if constexpr (!P2<N>::TWO) {
     dft8<true>(x);
   } else {
     constexpr int G = P2<N>::G, R2 = P2<N>::R2;
-    // inverse pass 1: radix R2 on slots b*R2 + r (inputs j + r*8, j = g + G b)
+    constexpr int PD = R2 < 8 ? 8 : R2;      // pad stride; keeps the buffer within N + N/8
 #pragma unroll
-    for (int b = 0; b < 8 / R2; ++b) {
-      if constexpr (R2 == 8) dft8<true>(&x[b * 8]);
+    for (int b = 0; b < R1 / R2; ++b) {
+      if constexpr (R2 == 16) dft16<true>(&x[b * 16]);
+      else if constexpr (R2 == 8) dft8<true>(&x[b * 8]);
       else if constexpr (R2 == 4) dft4<true>(x[b * 4], x[b * 4 + 1], x[b * 4 + 2], x[b * 4 + 3]);
       else dft2(x[b * 2], x[b * 2 + 1]);
     }
-    // output index (j) * R2 + r ; read pass-2 inputs g + r*G with twiddle W_N^{-g r}
     __syncwarp();
 #pragma unroll
-    for (int b = 0; b < 8 / R2; ++b) {
+    for (int b = 0; b < R1 / R2; ++b) {
 #pragma unroll
       for (int r = 0; r < R2; ++r) {
         const int s = b * R2 + r;
-        buf[swz((g + G * b) * R2 + r) ^ key] = make_float4(x[s].re.x, x[s].re.y, x[s].im.x, x[s].im.y);
+        buf[padx<PD>((g + G * b) * R2 + r)] = make_float4(x[s].re.x, x[s].re.y, x[s].im.x, x[s].im.y);
       }
     }
     __syncwarp();
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const float4 v = buf[swz(g + r * G) ^ key];
+    for (int r = 0; r < R1; ++r) {
+      const float4 v = buf[padx<PD>(g + r * G)];
       cp y = {make_float2(v.x, v.y), make_float2(v.z, v.w)};
       if (r > 0) y = ctw<true>(y, t.twi[r * G + g]);
       x[r] = y;
     }
-    dft8<true>(x);
+    if constexpr (R1 == 16) dft16<true>(x);
+    else dft8<true>(x);
   }
 }
 
@@ -279,11 +331,11 @@ __device__ __forceinline__ void fft_inv(cp (&x)[8], int g, float4* buf, int key,
 // (a complex value, the same for both paths); on exit x[s] holds
 // (Z[2f], Z[2f+1]) with f = spec_idx<N>(g, s).
 template <int N>
-__device__ __forceinline__ void padded_fwd(const float2 (&z)[8], cp (&x)[8], int g, float4* buf, int key, Tabs<N> t,
-                                           unsigned mask) {
+__device__ __forceinline__ void padded_fwd(const float2 (&z)[P2<N>::R1], cp (&x)[P2<N>::R1], int g, float4* buf,
+                                           int key, Tabs<N> t, unsigned mask) {
   constexpr int G = P2<N>::G;
 #pragma unroll
-  for (int s = 0; s < 8; ++s) {
+  for (int s = 0; s < P2<N>::R1; ++s) {
     const float2 w = t.tst[s * G + g];
     const float ore = fmaf(z[s].x, w.x, -z[s].y * w.y);
     const float oim = fmaf(z[s].x, w.y, z[s].y * w.x);
@@ -295,12 +347,12 @@ __device__ __forceinline__ void padded_fwd(const float2 (&z)[8], cp (&x)[8], int
 // Inverse padded transform keeping outputs [0, N): on entry x[s] =
 // (Y[2f], Y[2f+1]); on exit out[s] = y[g + s G] (unnormalised).
 template <int N>
-__device__ __forceinline__ void padded_inv(cp (&x)[8], float2 (&out)[8], int g, float4* buf, int key, Tabs<N> t,
-                                           unsigned mask) {
+__device__ __forceinline__ void padded_inv(cp (&x)[P2<N>::R1], float2 (&out)[P2<N>::R1], int g, float4* buf, int key,
+                                           Tabs<N> t, unsigned mask) {
   constexpr int G = P2<N>::G;
   fft_inv<N>(x, g, buf, key, t, mask);
 #pragma unroll
-  for (int s = 0; s < 8; ++s) {
+  for (int s = 0; s < P2<N>::R1; ++s) {
     const float2 w = t.tst[s * G + g];   // untwist by conj(W_2N^{g + s G})
     const float re = fmaf(x[s].re.y, w.x, fmaf(x[s].im.y, w.y, x[s].re.x));
     const float im = fmaf(x[s].im.y, w.x, fmaf(-x[s].re.y, w.y, x[s].im.x));
@@ -311,14 +363,15 @@ __device__ __forceinline__ void padded_inv(cp (&x)[8], float2 (&out)[8], int g, 
 // Partner frequency -k (mod 2N) of spectral slot (f, path): path 0 -> (N - f)
 // mod N, path 1 -> N - 1 - f (both as natural half-frequency indices).
 template <int N>
-__device__ __forceinline__ void fetch_partner(const cp (&x)[8], cp (&xp)[8], int g, float4* buf, int key, unsigned mask) {
+__device__ __forceinline__ void fetch_partner(const cp (&x)[P2<N>::R1], cp (&xp)[P2<N>::R1], int g, float4* buf,
+                                              int key, unsigned mask) {
   __syncwarp();
 #pragma unroll
-  for (int s = 0; s < 8; ++s)
+  for (int s = 0; s < P2<N>::R1; ++s)
     buf[swz(spec_idx<N>(g, s)) ^ key] = make_float4(x[s].re.x, x[s].re.y, x[s].im.x, x[s].im.y);
   __syncwarp();
 #pragma unroll
-  for (int s = 0; s < 8; ++s) {
+  for (int s = 0; s < P2<N>::R1; ++s) {
     const int f = spec_idx<N>(g, s);
     const float4 a = buf[swz((N - f) & (N - 1)) ^ key];
     const float4 b = buf[swz(N - 1 - f) ^ key];

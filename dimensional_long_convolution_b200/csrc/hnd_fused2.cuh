@@ -108,7 +108,8 @@ struct F3 {
   static constexpr size_t kTabs = Tabs<N0>::kBytes + (N0 == N1 ? 0 : Tabs<N1>::kBytes);
   static constexpr size_t kStage = static_cast<size_t>(N0) * PITCH * sizeof(T);   // one plane
   static constexpr size_t kZb = sizeof(float4) * N1 * RPS;    // [f][rp] float4
-  static constexpr size_t kX = 4608 * kW3;
+  static constexpr int XW = XB<N0>::kWarp > XB<N1>::kWarp ? XB<N0>::kWarp : XB<N1>::kWarp;
+  static constexpr size_t kX = 16ull * XW * kW3;
   static constexpr size_t kBytes = 32 + kTabs + 3 * kStage + 2 * kZb + kX;
 };
 
@@ -297,7 +298,7 @@ __global__ void __launch_bounds__(kT3, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = warp >> 3, gw = warp & 7;
-  float4* xw = xb + warp * 288;
+  float4* xw = xb + warp * L::XW;
   const int nvol = B * C;
   const int v0 = blockIdx.x;
   if (v0 >= nvol) return;
@@ -400,15 +401,15 @@ __global__ void __launch_bounds__(kT3, 1)
 }
 
 // ------------------------------------------------------ spectrum layout (2D)
-// Library order of a 2D problem with n0 <= 64, per channel, in float4 units:
+// Library order of a 2D problem, per channel, in float4 units:
 // unit 0 (DC and Nyquist columns combined) holds A then B, n0 float4 each;
 // unit u >= 1 (column kx = u) holds n0 float4 at offset (u + 1) n0.  Inside a
 // unit, float4 m = s G + g holds (S[2f].re, S[2f+1].re, S[2f].im, S[2f+1].im)
 // with f = spec_idx(g, s) the z-pencil frequency of lane g, slot s.
 __host__ __device__ __forceinline__ int spec_idx_rt(int N, int g, int s) {
   if (N == 8) return s;
-  const int G = N / 8;
-  return g + G * (s / G) + (s % G) * 8;
+  const int R1 = N >= 128 ? 16 : 8, G = N / R1;
+  return g + G * (s / G) + (s % G) * R1;
 }
 
 struct Pos2 {
@@ -429,7 +430,7 @@ __host__ __device__ __forceinline__ Pos2 pos2_of(int n0, int n1, long long e4) {
     r.kx = static_cast<int>((e4 - 2LL * n0) / n0) + 1;
     m = (e4 - 2LL * n0) % n0;
   }
-  const int G = n0 / 8 < 1 ? 1 : n0 / 8;
+  const int G = n0 == 8 ? 1 : n0 / (n0 >= 128 ? 16 : 8);
   const int s = static_cast<int>(m / G), g = static_cast<int>(m % G);
   const int f = spec_idx_rt(n0, g, s);
   r.ky0 = 2 * f;

@@ -24,9 +24,10 @@ struct ConvArgs {
   int* status = nullptr;  // device status word (may be null)
 };
 
-// 2D problems whose axes are both <= 64 run on the packed persistent fused
-// kernel and use the packed (v2) spectrum order.
-inline bool use_v2_2d(int ndim, const int* n) { return ndim == 2 && n[0] <= 64 && n[1] <= 64; }
+// 2D problems whose axes are both <= 64 run on the persistent fused kernel;
+// larger 2D grids and every 3D grid run the multi-pass tier.  2D and 3D
+// spectra use the packed order of the two-path FFT core.
+inline bool fused_2d(int ndim, const int* n) { return ndim == 2 && n[0] <= 64 && n[1] <= 64; }
 
 // Streaming multiprocessors of the current device (cached per device).
 int sm_count();

@@ -1,0 +1,506 @@
+// hnd_multi2.cuh -- multi-pass tiers on the packed two-path FFT core, for
+// volumes whose padded transform does not fit one SM (2D with an axis >= 128,
+// every 3D grid).  One wave of (b, c) volumes at a time:
+//   k_rowfwd2   rows along the last axis, packed two at a time, zero-padded
+//               forward transform -> Zt[kk][rp] (an L2-sized workspace)
+//   k_mid1v2    2D: per last-axis frequency, zero-padded convolution along
+//               axis 0 with the channel spectrum
+//   k_mid2v2    3D: per last-axis frequency, zero-padded 2D convolution over
+//               axes (0, 1)
+//   k_rowinv2   inverse rows, crop, output gate q
+// (HyenaND pages: zero padding to twice the grid; forward FFT, spectral
+// modulation, inverse FFT and output cropping.)
+#pragma once
+
+#include "hnd_fused2.cuh"
+
+#include <cooperative_groups.h>
+
+namespace hnd2 {
+
+namespace cg = cooperative_groups;
+
+constexpr int kTM = 256;          // threads per CTA in the multi-pass kernels
+constexpr int kWM = kTM / 32;
+
+// Row pair rp = rows (ra, ra + ps): 2D pairs row r with r + n0/2 (ps = n0/2),
+// 3D pairs neighbouring rows (ps = 1).
+__device__ __forceinline__ long long pair_row(long long rp, int ps) { return (rp / ps) * 2 * ps + (rp % ps); }
+
+template <int NL>
+struct RT {
+  static constexpr int G = P2<NL>::G, PPW = 32 / G;
+  static constexpr int RPB = (kWM * PPW) * ((kWM * PPW) < 16 ? 2 : 1);   // row pairs per CTA
+  static constexpr int TS = RPB + 1;                                     // tile pitch (float2)
+  static constexpr size_t kBytes = Tabs<NL>::kBytes + sizeof(float2) * 2 * NL * TS + 16ull * XB<NL>::kWarp * kWM;
+};
+
+// ------------------------------------------------------------- forward rows
+template <int NL, class T>
+__global__ void __launch_bounds__(kTM) k_rowfwd2(const T* __restrict__ k, const T* __restrict__ v,
+                                                 float2* __restrict__ Zt, long long ord0, int rp_total, int ps,
+                                                 int B, int C) {
+  using R = RT<NL>;
+  constexpr int G = R::G, PPW = R::PPW, R1 = P2<NL>::R1, RPB = R::RPB, TS = R::TS;
+  extern __shared__ __align__(16) unsigned char smem[];
+  const Tabs<NL> t = tabs_at<NL>(smem);
+  float2* tile = reinterpret_cast<float2*>(smem + Tabs<NL>::kBytes);
+  float4* xb = reinterpret_cast<float4*>(smem + Tabs<NL>::kBytes + sizeof(float2) * 2 * NL * TS);
+  tabs_build<NL>(t, g_tw512);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long ord = ord0 + blockIdx.x;
+  const int c = static_cast<int>(ord / B), b = static_cast<int>(ord % B);
+  const long long L = static_cast<long long>(rp_total) * 2 * NL;
+  const long long base = (static_cast<long long>(b) * C + c) * L;
+  const int rpb = blockIdx.y * RPB;
+  const int nrp = min(RPB, rp_total - rpb);
+  const int pen = lane / G, g = lane % G;
+  float4* buf = xb + warp * XB<NL>::kWarp + pen * XB<NL>::kPen;
+  __syncthreads();
+  for (int r0 = warp * PPW; r0 < RPB; r0 += kWM * PPW) {
+    const int rl = r0 + pen;
+    const bool act = rl < nrp;
+    const long long ra = pair_row(rpb + rl, ps) * NL, rb = ra + static_cast<long long>(ps) * NL;
+    float2 z[R1];
+#pragma unroll
+    for (int s = 0; s < R1; ++s) {
+      const long long j = g + s * G;
+      z[s] = act ? make_float2(Act<T>::ld_g(k + base + ra + j) * Act<T>::ld_g(v + base + ra + j),
+                               Act<T>::ld_g(k + base + rb + j) * Act<T>::ld_g(v + base + rb + j))
+                 : make_float2(0.f, 0.f);
+    }
+    cp x[R1];
+    padded_fwd<NL>(z, x, g, buf, 0, t, 0u);
+#pragma unroll
+    for (int s = 0; s < R1; ++s) {
+      const int kk = 2 * spec_idx<NL>(g, s);
+      tile[kk * TS + rl] = make_float2(x[s].re.x, x[s].im.x);
+      tile[(kk + 1) * TS + rl] = make_float2(x[s].re.y, x[s].im.y);
+    }
+  }
+  __syncthreads();
+  float2* zt = Zt + static_cast<long long>(blockIdx.x) * L;
+  for (int e = threadIdx.x; e < 2 * NL * RPB; e += kTM) {
+    const int kk = e / RPB, rl = e % RPB;
+    if (rl < nrp) zt[static_cast<long long>(kk) * rp_total + rpb + rl] = tile[kk * TS + rl];
+  }
+}
+
+// ------------------------------------------------------------- inverse rows
+template <int NL, class T>
+__global__ void __launch_bounds__(kTM) k_rowinv2(const float2* __restrict__ Zt, const T* __restrict__ q,
+                                                 T* __restrict__ y, long long ord0, int rp_total, int ps, int B,
+                                                 int C) {
+  using R = RT<NL>;
+  constexpr int G = R::G, PPW = R::PPW, R1 = P2<NL>::R1, RPB = R::RPB, TS = R::TS;
+  extern __shared__ __align__(16) unsigned char smem[];
+  const Tabs<NL> t = tabs_at<NL>(smem);
+  float2* tile = reinterpret_cast<float2*>(smem + Tabs<NL>::kBytes);
+  float4* xb = reinterpret_cast<float4*>(smem + Tabs<NL>::kBytes + sizeof(float2) * 2 * NL * TS);
+  tabs_build<NL>(t, g_tw512);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long ord = ord0 + blockIdx.x;
+  const int c = static_cast<int>(ord / B), b = static_cast<int>(ord % B);
+  const long long L = static_cast<long long>(rp_total) * 2 * NL;
+  const long long base = (static_cast<long long>(b) * C + c) * L;
+  const int rpb = blockIdx.y * RPB;
+  const int nrp = min(RPB, rp_total - rpb);
+  const float2* zt = Zt + static_cast<long long>(blockIdx.x) * L;
+  for (int e = threadIdx.x; e < 2 * NL * RPB; e += kTM) {
+    const int kk = e / RPB, rl = e % RPB;
+    tile[kk * TS + rl] = (rl < nrp) ? zt[static_cast<long long>(kk) * rp_total + rpb + rl] : make_float2(0.f, 0.f);
+  }
+  __syncthreads();
+  const int pen = lane / G, g = lane % G;
+  float4* buf = xb + warp * XB<NL>::kWarp + pen * XB<NL>::kPen;
+  for (int r0 = warp * PPW; r0 < RPB; r0 += kWM * PPW) {
+    const int rl = r0 + pen;
+    const bool act = rl < nrp;
+    const long long ra = pair_row(rpb + rl, ps) * NL, rb = ra + static_cast<long long>(ps) * NL;
+    float qa[R1], qb[R1];
+#pragma unroll
+    for (int s = 0; s < R1; ++s) {
+      const long long j = g + s * G;
+      qa[s] = act ? Act<T>::ld_g(q + base + ra + j) : 0.f;
+      qb[s] = act ? Act<T>::ld_g(q + base + rb + j) : 0.f;
+    }
+    cp x[R1];
+#pragma unroll
+    for (int s = 0; s < R1; ++s) {
+      const int kk = 2 * spec_idx<NL>(g, s);
+      const float2 e = tile[kk * TS + rl], d = tile[(kk + 1) * TS + rl];
+      x[s] = {make_float2(e.x, d.x), make_float2(e.y, d.y)};
+    }
+    float2 o[R1];
+    padded_inv<NL>(x, o, g, buf, 0, t, 0u);
+    if (act) {
+#pragma unroll
+      for (int s = 0; s < R1; ++s) {
+        const long long j = g + s * G;
+        Act<T>::st_g(y + base + ra + j, o[s].x * qa[s]);
+        Act<T>::st_g(y + base + rb + j, o[s].y * qb[s]);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------- 2D column units
+// Zt[kk][rp] per volume, rp in [0, n0/2) with row pair (rp, rp + n0/2); unit cu
+// = last-axis frequency kx (cu >= 1) or the combined DC/Nyquist unit (cu = 0).
+template <int N0>
+struct M1 {
+  static constexpr int G = P2<N0>::G, PPW = 32 / G;
+  static constexpr int UPB = kWM * PPW;                  // units per CTA
+  static constexpr size_t kBytes = Tabs<N0>::kBytes + 16ull * XB<N0>::kWarp * kWM;
+};
+
+template <int N0>
+__global__ void __launch_bounds__(kTM) k_mid1v2(float2* __restrict__ Zt, const float4* __restrict__ spec,
+                                                long long sbs4, int N1, long long ord0, int B, int C) {
+  using M = M1<N0>;
+  constexpr int G = M::G, PPW = M::PPW, R1 = P2<N0>::R1, RP = N0 / 2, HS = R1 / 2;
+  extern __shared__ __align__(16) unsigned char smem[];
+  const Tabs<N0> t = tabs_at<N0>(smem);
+  float4* xb = reinterpret_cast<float4*>(smem + Tabs<N0>::kBytes);
+  tabs_build<N0>(t, g_tw512);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long ord = ord0 + blockIdx.x;
+  const int c = static_cast<int>(ord / B), b = static_cast<int>(ord % B);
+  const int u0 = blockIdx.y * M::UPB;
+  const float4* sp = spec + static_cast<long long>(b) * sbs4 + static_cast<long long>(c) * (N1 + 1) * N0;
+  __syncthreads();
+  float2* zt = Zt + static_cast<long long>(blockIdx.x) * 2 * N1 * RP;
+  const int pen = lane / G, g = lane % G;
+  float4* buf = xb + warp * XB<N0>::kWarp + pen * XB<N0>::kPen;
+  const int cu = u0 + warp * PPW + pen;
+  const bool act = cu < N1;
+  const bool general = u0 == 0 && warp == 0;
+  const int kx = act ? cu : 1, kxm = cu == 0 ? N1 : 2 * N1 - kx;
+  float2 z[R1];
+#pragma unroll
+  for (int s = 0; s < HS; ++s) {
+    const int rp = g + s * G;
+    float2 z1 = make_float2(0.f, 0.f), z2 = z1;
+    if (act) {
+      z1 = zt[static_cast<long long>(kx) * RP + rp];
+      z2 = zt[static_cast<long long>(kxm) * RP + rp];
+    }
+    if (cu == 0) {
+      z[s] = make_float2(z1.x, z2.x);
+      z[s + HS] = make_float2(z1.y, z2.y);
+    } else {
+      z[s] = unpack_a(z1, z2);
+      z[s + HS] = unpack_b(z1, z2);
+    }
+  }
+  cp x[R1];
+  padded_fwd<N0>(z, x, g, buf, 0, t, 0u);
+  const float4* su = sp + (cu == 0 ? 0LL : static_cast<long long>(cu + 1) * N0);
+  if (general) {
+    cp xp[R1];
+    fetch_partner<N0>(x, xp, g, buf, 0, 0u);
+#pragma unroll
+    for (int s = 0; s < R1; ++s) {
+      const float4 S = act ? __ldg(su + s * G + g) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 Bc = (cu == 0) ? __ldg(sp + N0 + s * G + g) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const cp a = cmulp(x[s], make_float2(S.x, S.y), make_float2(S.z, S.w));
+      const cp xc = {xp[s].re, make_float2(-xp[s].im.x, -xp[s].im.y)};
+      const cp bb = cmulp(xc, make_float2(Bc.x, Bc.y), make_float2(Bc.z, Bc.w));
+      x[s] = cadd(a, bb);
+    }
+  } else if (act) {
+#pragma unroll
+    for (int s = 0; s < R1; ++s) {
+      const float4 S = __ldg(su + s * G + g);
+      x[s] = cmulp(x[s], make_float2(S.x, S.y), make_float2(S.z, S.w));
+    }
+  }
+  float2 o[R1];
+  padded_inv<N0>(x, o, g, buf, 0, t, 0u);
+  if (act) {
+#pragma unroll
+    for (int s = 0; s < HS; ++s) {
+      const int rp = g + s * G;
+      const float2 ya = o[s], yb = o[s + HS];
+      if (cu == 0) {
+        zt[rp] = make_float2(ya.x, yb.x);
+        zt[static_cast<long long>(N1) * RP + rp] = make_float2(ya.y, yb.y);
+      } else {
+        zt[static_cast<long long>(kx) * RP + rp] = pack_pos(ya, yb);
+        zt[static_cast<long long>(kxm) * RP + rp] = pack_neg(ya, yb);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- 3D slabs
+// For one last-axis frequency kx: the (axis 0, axis 1) slab of both packed
+// rows' spectra (rows y and y + 1 share one Zt entry), zero-padded 2D
+// convolution with the channel's slab spectrum, written back packed.
+//   step 1  y transforms (one pencil per z)       -> F[ky][z]
+//   step 2  z-pencil convolution per ky (spectrum payload [s][g] per ky)
+//   step 3  inverse y transforms, repack, write Zt
+// With HALF = true the slab is split over a 2-CTA cluster by ky parity: CTA h
+// keeps ky = 2m + h and finishes rows z in [h n0/2, (h + 1) n0/2), reading the
+// other parity through distributed shared memory.
+template <int N0, int N1, bool HALF>
+struct M2 {
+  static constexpr int FS = N0 + 1;
+  static constexpr int NKY = HALF ? N1 : 2 * N1;         // ky rows held by this CTA
+  static constexpr size_t kTabs = Tabs<N0>::kBytes + (N0 == N1 ? 0 : Tabs<N1>::kBytes);
+  static constexpr int XW = XB<N0>::kWarp > XB<N1>::kWarp ? XB<N0>::kWarp : XB<N1>::kWarp;
+  static constexpr size_t kBytes = kTabs + sizeof(float2) * NKY * FS + 16ull * XW * kWM;
+};
+
+template <int N0, int N1>
+__device__ __forceinline__ void slab_rows_in(const float2* __restrict__ zt, long long RPn, int kx, int kxm,
+                                            bool self_conj, int z, int g, float2 (&x)[P2<N1>::R1]) {
+  constexpr int G = P2<N1>::G, R1 = P2<N1>::R1;
+#pragma unroll
+  for (int s = 0; s < R1; ++s) {
+    const int yy = g + s * G;
+    const long long rp = (static_cast<long long>(z) * N1 + yy) >> 1;
+    const float2 z1 = zt[kx * RPn + rp];
+    const float2 z2 = self_conj ? z1 : zt[kxm * RPn + rp];
+    x[s] = (yy & 1) ? unpack_b(z1, z2) : unpack_a(z1, z2);
+  }
+}
+
+template <int N0, int N1>
+__device__ __forceinline__ void slab_rows_out(float2* __restrict__ zt, long long RPn, int kx, int kxm, bool self_conj,
+                                             int z, int g, bool act, const float2 (&o)[P2<N1>::R1]) {
+  constexpr int G = P2<N1>::G, R1 = P2<N1>::R1;
+#pragma unroll
+  for (int s = 0; s < R1; ++s) {
+    const float2 own = o[s];
+    float2 oth;
+    if constexpr (G >= 2) {
+      oth.x = __shfl_xor_sync(0xffffffffu, own.x, 1);
+      oth.y = __shfl_xor_sync(0xffffffffu, own.y, 1);
+    } else {
+      oth = o[s ^ 1];
+    }
+    const int yy = g + s * G;
+    const long long rp = (static_cast<long long>(z) * N1 + yy) >> 1;
+    const bool odd = yy & 1;
+    const float2 ya = odd ? oth : own, yb = odd ? own : oth;
+    if (!act) continue;
+    if (self_conj) {
+      if (!odd) zt[kx * RPn + rp] = make_float2(ya.x, yb.x);
+    } else {
+      if (!odd) zt[kx * RPn + rp] = pack_pos(ya, yb);
+      else zt[kxm * RPn + rp] = pack_neg(ya, yb);
+    }
+  }
+}
+
+template <int N0, int N1, bool HALF>
+__device__ __forceinline__ void k_mid2_body(float2* __restrict__ Zt, const float4* __restrict__ spec, long long sbs4,
+                                            int N2, long long ord0, int B, int C, int vol_local, int h) {
+  using M = M2<N0, N1, HALF>;
+  constexpr int FS = M::FS, NKY = M::NKY;
+  constexpr int G0 = P2<N0>::G, R0 = P2<N0>::R1, G1 = P2<N1>::G, R1 = P2<N1>::R1;
+  extern __shared__ __align__(16) unsigned char smem[];
+  const Tabs<N0> t0 = tabs_at<N0>(smem);
+  Tabs<N1> t1;
+  if constexpr (N0 == N1) {
+    t1 = t0;
+  } else {
+    t1 = tabs_at<N1>(smem + Tabs<N0>::kBytes);
+  }
+  float2* F = reinterpret_cast<float2*>(smem + M::kTabs);
+  float4* xb = reinterpret_cast<float4*>(smem + M::kTabs + sizeof(float2) * NKY * FS);
+  tabs_build<N0>(t0, g_tw512);
+  if constexpr (N0 != N1) tabs_build<N1>(t1, g_tw512);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long ord = ord0 + vol_local;
+  const int c = static_cast<int>(ord / B), b = static_cast<int>(ord % B);
+  const long long RPn = static_cast<long long>(N0) * N1 / 2;
+  float2* zt = Zt + static_cast<long long>(vol_local) * 2 * N2 * RPn;
+  const int kx = blockIdx.y;
+  const bool self_conj = (kx == 0) || (kx == N2);
+  const int kxm = self_conj ? kx : 2 * N2 - kx;
+  const long long slab = 2LL * N1 * N0;                 // float4 per slab
+  const float4* sslab = spec + static_cast<long long>(b) * sbs4 + static_cast<long long>(c) * (N2 + 1) * slab +
+                        static_cast<long long>(kx) * slab;
+  __syncthreads();
+  // step 1: y transforms, one pencil per z
+  {
+    constexpr int PPW = 32 / G1;
+    const int pen = lane / G1, g = lane % G1;
+    float4* buf = xb + warp * M::XW + pen * XB<N1>::kPen;
+    for (int z0 = warp * PPW; z0 < N0; z0 += kWM * PPW) {
+      const int z = z0 + pen;
+      const bool act = z < N0;
+      float2 in[R1];
+      if (act) {
+        slab_rows_in<N0, N1>(zt, RPn, kx, kxm, self_conj, z, g, in);
+      } else {
+#pragma unroll
+        for (int s = 0; s < R1; ++s) in[s] = make_float2(0.f, 0.f);
+      }
+      cp x[R1];
+      padded_fwd<N1>(in, x, g, buf, 0, t1, 0u);
+      if (act) {
+#pragma unroll
+        for (int s = 0; s < R1; ++s) {
+          const int f = spec_idx<N1>(g, s);
+          if (HALF) {
+            F[f * FS + z] = h == 0 ? make_float2(x[s].re.x, x[s].im.x) : make_float2(x[s].re.y, x[s].im.y);
+          } else {
+            F[(2 * f) * FS + z] = make_float2(x[s].re.x, x[s].im.x);
+            F[(2 * f + 1) * FS + z] = make_float2(x[s].re.y, x[s].im.y);
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();
+  // step 2: z-pencil convolution per ky row held here; pencils of a warp
+  // take rows 8 apart (bank groups of F)
+  {
+    constexpr int PPW = 32 / G0, SLOTS = kWM * PPW;
+    const int pen = lane / G0, g = lane % G0;
+    float4* buf = xb + warp * XB<N0>::kWarp + pen * XB<N0>::kPen;
+    for (int r0 = 0; r0 < NKY; r0 += SLOTS) {
+      const int kyl = r0 + warp + pen * kWM;
+      const bool act = kyl < NKY;
+      const int ky = HALF ? 2 * kyl + h : kyl;
+      const float4* su = sslab + static_cast<long long>(act ? ky : 0) * N0;
+      constexpr int NPF = R0 == 8 ? 8 : 1;             // prefetch the payload when registers allow
+      float4 S[NPF];
+      if (R0 == 8 && act) {
+#pragma unroll
+        for (int s = 0; s < NPF; ++s) S[s] = __ldg(su + s * G0 + g);
+      }
+      float2 in[R0];
+#pragma unroll
+      for (int s = 0; s < R0; ++s) in[s] = act ? F[kyl * FS + g + s * G0] : make_float2(0.f, 0.f);
+      cp x[R0];
+      padded_fwd<N0>(in, x, g, buf, 0, t0, 0u);
+      if (act) {
+#pragma unroll
+        for (int s = 0; s < R0; ++s) {
+          const float4 Sv = (R0 == 8) ? S[s % NPF] : __ldg(su + s * G0 + g);
+          x[s] = cmulp(x[s], make_float2(Sv.x, Sv.y), make_float2(Sv.z, Sv.w));
+        }
+      }
+      float2 o[R0];
+      padded_inv<N0>(x, o, g, buf, 0, t0, 0u);
+      if (act) {
+#pragma unroll
+        for (int s = 0; s < R0; ++s) F[kyl * FS + g + s * G0] = o[s];
+      }
+    }
+  }
+  if constexpr (HALF) {
+    cg::this_cluster().sync();
+  } else {
+    __syncthreads();
+  }
+  // step 3: inverse y transforms, repack, write back
+  {
+    constexpr int PPW = 32 / G1;
+    const int pen = lane / G1, g = lane % G1;
+    float4* buf = xb + warp * M::XW + pen * XB<N1>::kPen;
+    const float2* Fe = F;
+    const float2* Fo = F;
+    if constexpr (HALF) {
+      float2* other = cg::this_cluster().map_shared_rank(F, h ^ 1);
+      Fe = h == 0 ? F : other;
+      Fo = h == 0 ? other : F;
+    }
+    constexpr int NZ = HALF ? N0 / 2 : N0;
+    for (int z0 = warp * PPW; z0 < NZ; z0 += kWM * PPW) {
+      const int zl = z0 + pen;
+      const bool act = zl < NZ;
+      const int z = HALF ? h * (N0 / 2) + zl : zl;
+      cp x[R1];
+#pragma unroll
+      for (int s = 0; s < R1; ++s) {
+        const int f = spec_idx<N1>(g, s);
+        float2 e = make_float2(0.f, 0.f), d = e;
+        if (act) {
+          if (HALF) {
+            e = Fe[f * FS + z];
+            d = Fo[f * FS + z];
+          } else {
+            e = F[(2 * f) * FS + z];
+            d = F[(2 * f + 1) * FS + z];
+          }
+        }
+        x[s] = {make_float2(e.x, d.x), make_float2(e.y, d.y)};
+      }
+      float2 o[R1];
+      padded_inv<N1>(x, o, g, buf, 0, t1, 0u);
+      slab_rows_out<N0, N1>(zt, RPn, kx, kxm, self_conj, z, g, act, o);
+    }
+  }
+  if constexpr (HALF) cg::this_cluster().sync();
+}
+
+template <int N0, int N1>
+__global__ void __launch_bounds__(kTM) k_mid2v2(float2* __restrict__ Zt, const float4* __restrict__ spec,
+                                                long long sbs4, int N2, long long ord0, int B, int C) {
+  k_mid2_body<N0, N1, false>(Zt, spec, sbs4, N2, ord0, B, C, blockIdx.x, 0);
+}
+
+template <int N0, int N1>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTM)
+    k_mid2v2_pair(float2* __restrict__ Zt, const float4* __restrict__ spec, long long sbs4, int N2, long long ord0,
+                  int B, int C) {
+  const int h = static_cast<int>(cg::this_cluster().block_rank());
+  k_mid2_body<N0, N1, true>(Zt, spec, sbs4, N2, ord0, B, C, blockIdx.x / 2, h);
+}
+
+// --------------------------------------------------- spectrum layouts (v2)
+// 3D, per channel, float4 units: for kx in [0, n2], for ky in [0, 2 n1), n0
+// float4 at [s][g] of the z-pencil plan: (S[2f].re, S[2f+1].re, S[2f].im,
+// S[2f+1].im), f = spec_idx(g, s), the z frequency of lane g, slot s.
+__host__ __device__ __forceinline__ int spec_idx_gen(int N, int g, int s) {
+  if (N == 8) return s;
+  const int R1 = N >= 128 ? 16 : 8, R2 = N / R1, G = R2;
+  return g + G * (s / R2) + (s % R2) * R1;
+}
+__host__ __device__ __forceinline__ int lanes_of(int N) { return N == 8 ? 1 : N / (N >= 128 ? 16 : 8); }
+
+// natural half spectrum [C][2n0][2n1][n2 + 1] (pitch = last-axis length of the
+// source: n2 + 1 for a half spectrum, 2 n2 for a full grid) -> library order
+static __global__ void k_spec3_in(const float2* __restrict__ nat, float4* __restrict__ out, int n0, int n1, int n2,
+                                  long long C, long long pitch, float scale) {
+  const long long per = static_cast<long long>(n2 + 1) * 2 * n1 * n0;     // float4 per channel
+  const long long src_per = 4LL * n0 * n1 * pitch;
+  const int G = lanes_of(n0);
+  for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < per * C;
+       e += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long c = e / per, r = e % per;
+    const int kx = static_cast<int>(r / (2LL * n1 * n0));
+    const long long r2 = r % (2LL * n1 * n0);
+    const int ky = static_cast<int>(r2 / n0), m = static_cast<int>(r2 % n0);
+    const int f = spec_idx_gen(n0, m % G, m / G);
+    const float2* src = nat + c * src_per;
+    const float2 s0 = src[((2LL * f) * (2 * n1) + ky) * pitch + kx];
+    const float2 s1 = src[((2LL * f + 1) * (2 * n1) + ky) * pitch + kx];
+    out[e] = make_float4(scale * s0.x, scale * s1.x, scale * s0.y, scale * s1.y);
+  }
+}
+
+static __global__ void k_spec3_out(const float4* __restrict__ lib, float2* __restrict__ nat, int n0, int n1, int n2,
+                                   long long C) {
+  const long long per = static_cast<long long>(n2 + 1) * 2 * n1 * n0;
+  const int G = lanes_of(n0);
+  for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < per * C;
+       e += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long c = e / per, r = e % per;
+    const int kx = static_cast<int>(r / (2LL * n1 * n0));
+    const long long r2 = r % (2LL * n1 * n0);
+    const int ky = static_cast<int>(r2 / n0), m = static_cast<int>(r2 % n0);
+    const int f = spec_idx_gen(n0, m % G, m / G);
+    float2* dst = nat + c * per * 2;
+    const float4 v = lib[e];
+    dst[((2LL * f) * (2 * n1) + ky) * (n2 + 1) + kx] = make_float2(v.x, v.z);
+    dst[((2LL * f + 1) * (2 * n1) + ky) * (n2 + 1) + kx] = make_float2(v.y, v.w);
+  }
+}
+
+}  // namespace hnd2

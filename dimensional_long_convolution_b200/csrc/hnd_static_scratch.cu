@@ -107,7 +107,7 @@ extern "C" HYENA_ND_API hyena_nd_status hyena_nd_fftconv_batched_static(
   if (overlaps(y, q, act_bytes) || overlaps(y, k, act_bytes) || overlaps(y, v, act_bytes))
     return HYENA_ND_ERR_INVALID_ARG;
 
-  const bool fused = p->ndim == 1 || (p->ndim == 2 && n[0] <= 128 && n[1] <= 128);
+  const bool fused = p->ndim == 1 || hnd::fused_2d(p->ndim, n);
   const size_t per_pair = static_cast<size_t>(8) * static_cast<size_t>(L);
   if (!fused && per_pair > kStaticScratchBytes) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
 

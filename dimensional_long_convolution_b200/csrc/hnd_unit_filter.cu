@@ -1,6 +1,6 @@
 // Filter spectrum (call 1), spectrum layout conversion, diagnostics.
 #include "hnd_kernels.cuh"
-#include "hnd_fused2.cuh"
+#include "hnd_multi2.cuh"
 #include "hnd_launch.h"
 #include "hnd_host_util.h"
 
@@ -55,10 +55,13 @@ cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, i
   }
   const long long per = spec_per_channel(d);
   const float scale = static_cast<float>(1.0 / static_cast<double>(gsz));
-  if (use_v2_2d(ndim, n)) {
+  if (ndim == 2) {
     float4* out = static_cast<float4*>(spectrum) + static_cast<long long>(c0) * (per / 2);
     hnd2::k_spec_import_v2<<<grid_for(per / 2 * nc, 256), 256, 0, st>>>(grid, out, n[0], n[1], nc, 2LL * n[1],
                                                                         scale);
+  } else if (ndim == 3) {
+    float4* out = static_cast<float4*>(spectrum) + static_cast<long long>(c0) * (per / 2);
+    hnd2::k_spec3_in<<<grid_for(per / 2 * nc, 256), 256, 0, st>>>(grid, out, n[0], n[1], n[2], nc, 2LL * n[2], scale);
   } else {
     k_spec_pack<<<grid_for(per * nc, 256), 256, 0, st>>>(grid, static_cast<float2*>(spectrum), d, c0, nc, scale);
   }
@@ -69,7 +72,17 @@ cudaError_t launch_spec_convert(int ndim, const int* n, long long C, const void*
                                 cudaStream_t st) {
   const SpecDims d = make_dims(ndim, n);
   const long long total = spec_per_channel(d) * C;
-  if (use_v2_2d(ndim, n)) {
+  if (ndim == 3) {
+    if (to_natural)
+      hnd2::k_spec3_out<<<grid_for(total / 2, 256), 256, 0, st>>>(static_cast<const float4*>(src),
+                                                                 static_cast<float2*>(dst), n[0], n[1], n[2], C);
+    else
+      hnd2::k_spec3_in<<<grid_for(total / 2, 256), 256, 0, st>>>(static_cast<const float2*>(src),
+                                                                static_cast<float4*>(dst), n[0], n[1], n[2], C,
+                                                                n[2] + 1, 1.0f);
+    return cudaGetLastError();
+  }
+  if (ndim == 2) {
     if (to_natural)
       hnd2::k_spec_export_v2<<<grid_for(total / 2, 256), 256, 0, st>>>(static_cast<const float4*>(src),
                                                                       static_cast<float2*>(dst), n[0], n[1], C);

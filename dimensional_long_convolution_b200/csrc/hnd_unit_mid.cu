@@ -1,5 +1,6 @@
-// Instantiations: multi-pass column stages (2D pencils, 3D slabs).
-#include "hnd_kernels.cuh"
+// Instantiations: multi-pass column stages (2D pencils, 3D slabs) on the
+// packed two-path FFT core.
+#include "hnd_multi2.cuh"
 #include "hnd_launch.h"
 #include "hnd_host_util.h"
 
@@ -7,14 +8,14 @@ namespace hnd {
 
 template <int N0>
 static cudaError_t mid1_go(const ConvArgs& a, float2* zt, long long ord0, int np) {
-  auto kern = k_mid1<N0>;
-  const size_t sm = kMidSmemBase;
+  auto kern = hnd2::k_mid1v2<N0>;
+  const size_t sm = hnd2::M1<N0>::kBytes;
   cudaError_t e = ensure_smem(kern, sm);
   if (e != cudaSuccess) return e;
-  constexpr int PPW = 32 / (N0 / 8);
+  constexpr int UPB = hnd2::M1<N0>::UPB;
   const int n1 = a.n[1];
-  dim3 grid(np, (n1 + kWarps * PPW - 1) / (kWarps * PPW));
-  kern<<<grid, kThreads, sm, a.stream>>>(zt, static_cast<const float2*>(a.spec), a.sbs, n1, ord0, a.B, a.C);
+  dim3 grid(np, (n1 + UPB - 1) / UPB);
+  kern<<<grid, hnd2::kTM, sm, a.stream>>>(zt, static_cast<const float4*>(a.spec), a.sbs / 2, n1, ord0, a.B, a.C);
   return cudaGetLastError();
 }
 
@@ -33,20 +34,20 @@ cudaError_t launch_mid1(const ConvArgs& a, float2* zt, long long ord0, int np) {
 template <int N0, int N1>
 static cudaError_t mid2_go(const ConvArgs& a, float2* zt, long long ord0, int np) {
   const int n2 = a.n[2];
-  if (SlabSmem<N0, N1>::kBytes <= kMaxSmem) {
-    auto kern = k_mid2<N0, N1>;
-    const size_t sm = SlabSmem<N0, N1>::kBytes;
+  if (hnd2::M2<N0, N1, false>::kBytes <= kMaxSmem) {
+    auto kern = hnd2::k_mid2v2<N0, N1>;
+    const size_t sm = hnd2::M2<N0, N1, false>::kBytes;
     cudaError_t e = ensure_smem(kern, sm);
     if (e != cudaSuccess) return e;
     dim3 grid(np, n2 + 1);
-    kern<<<grid, kThreads, sm, a.stream>>>(zt, static_cast<const float2*>(a.spec), a.sbs, n2, ord0, a.B, a.C);
+    kern<<<grid, hnd2::kTM, sm, a.stream>>>(zt, static_cast<const float4*>(a.spec), a.sbs / 2, n2, ord0, a.B, a.C);
   } else {
-    auto kern = k_mid2_pair<N0, N1>;
-    const size_t sm = SlabSmem<N0, N1>::kHalfBytes;
+    auto kern = hnd2::k_mid2v2_pair<N0, N1>;
+    const size_t sm = hnd2::M2<N0, N1, true>::kBytes;
     cudaError_t e = ensure_smem(kern, sm);
     if (e != cudaSuccess) return e;
     dim3 grid(2 * np, n2 + 1);
-    kern<<<grid, kThreads, sm, a.stream>>>(zt, static_cast<const float2*>(a.spec), a.sbs, n2, ord0, a.B, a.C);
+    kern<<<grid, hnd2::kTM, sm, a.stream>>>(zt, static_cast<const float4*>(a.spec), a.sbs / 2, n2, ord0, a.B, a.C);
   }
   return cudaGetLastError();
 }

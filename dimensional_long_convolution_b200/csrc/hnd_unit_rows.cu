@@ -1,5 +1,6 @@
 // Instantiations: 1D fused rows, multi-pass row stages.
 #include "hnd_kernels.cuh"
+#include "hnd_multi2.cuh"
 #include "hnd_launch.h"
 #include "hnd_host_util.h"
 
@@ -37,31 +38,44 @@ static cudaError_t rows1d_io(const ConvArgs& a) {
 
 cudaError_t launch_rows1d(const ConvArgs& a) { return a.bf16 ? rows1d_io<IOBF16>(a) : rows1d_io<IOF32>(a); }
 
+template <class IO>
+struct TypeOf;
+template <>
+struct TypeOf<IOF32> {
+  using T = float;
+};
+template <>
+struct TypeOf<IOBF16> {
+  using T = __nv_bfloat16;
+};
+
+static int pair_stride(const ConvArgs& a) { return a.ndim == 2 ? a.n[0] / 2 : 1; }
+
 template <int NL, class IO>
 static cudaError_t rowfwd_go(const ConvArgs& a, float2* zt, long long ord0, int np, int rp_total) {
-  using TT = typename IO::T;
-  auto kern = k_rowfwd<NL, IO>;
-  const size_t sm = RowTile<NL>::kBytes;
+  using TT = typename TypeOf<IO>::T;
+  auto kern = hnd2::k_rowfwd2<NL, TT>;
+  const size_t sm = hnd2::RT<NL>::kBytes;
   cudaError_t e = ensure_smem(kern, sm);
   if (e != cudaSuccess) return e;
-  constexpr int RPB = RowTile<NL>::RPB;
+  constexpr int RPB = hnd2::RT<NL>::RPB;
   dim3 grid(np, (rp_total + RPB - 1) / RPB);
-  kern<<<grid, kThreads, sm, a.stream>>>(static_cast<const TT*>(a.k), static_cast<const TT*>(a.v), zt, ord0,
-                                         rp_total, a.B, a.C);
+  kern<<<grid, hnd2::kTM, sm, a.stream>>>(static_cast<const TT*>(a.k), static_cast<const TT*>(a.v), zt, ord0,
+                                          rp_total, pair_stride(a), a.B, a.C);
   return cudaGetLastError();
 }
 
 template <int NL, class IO>
 static cudaError_t rowinv_go(const ConvArgs& a, const float2* zt, long long ord0, int np, int rp_total) {
-  using TT = typename IO::T;
-  auto kern = k_rowinv<NL, IO>;
-  const size_t sm = RowTile<NL>::kBytes;
+  using TT = typename TypeOf<IO>::T;
+  auto kern = hnd2::k_rowinv2<NL, TT>;
+  const size_t sm = hnd2::RT<NL>::kBytes;
   cudaError_t e = ensure_smem(kern, sm);
   if (e != cudaSuccess) return e;
-  constexpr int RPB = RowTile<NL>::RPB;
+  constexpr int RPB = hnd2::RT<NL>::RPB;
   dim3 grid(np, (rp_total + RPB - 1) / RPB);
-  kern<<<grid, kThreads, sm, a.stream>>>(zt, static_cast<const TT*>(a.q), static_cast<TT*>(a.y), ord0, rp_total,
-                                         a.B, a.C);
+  kern<<<grid, hnd2::kTM, sm, a.stream>>>(zt, static_cast<const TT*>(a.q), static_cast<TT*>(a.y), ord0, rp_total,
+                                          pair_stride(a), a.B, a.C);
   return cudaGetLastError();
 }
 
