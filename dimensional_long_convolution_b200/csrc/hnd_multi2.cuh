@@ -32,12 +32,16 @@ struct RT {
   static constexpr int G = P2<NL>::G, PPW = 32 / G;
   static constexpr int RPB = (kWM * PPW) * ((kWM * PPW) < 16 ? 2 : 1);   // row pairs per CTA
   static constexpr int TS = RPB + 1;                                     // tile pitch (float2)
-  static constexpr size_t kBytes = Tabs<NL>::kBytes + sizeof(float2) * 2 * NL * TS + 16ull * XB<NL>::kWarp * kWM;
+  // The row tile and the FFT exchange buffers are never live together, so
+  // they share one region.
+  static constexpr size_t kTile = sizeof(float2) * 2 * NL * TS;
+  static constexpr size_t kXb = 16ull * XB<NL>::kWarp * kWM;
+  static constexpr size_t kBytes = Tabs<NL>::kBytes + (kTile > kXb ? kTile : kXb);
 };
 
 // ------------------------------------------------------------- forward rows
 template <int NL, class T>
-__global__ void __launch_bounds__(kTM) k_rowfwd2(const T* __restrict__ k, const T* __restrict__ v,
+__global__ void __launch_bounds__(kTM, 2) k_rowfwd2(const T* __restrict__ k, const T* __restrict__ v,
                                                  float2* __restrict__ Zt, long long ord0, int rp_total, int ps,
                                                  int B, int C) {
   using R = RT<NL>;
@@ -45,7 +49,7 @@ __global__ void __launch_bounds__(kTM) k_rowfwd2(const T* __restrict__ k, const 
   extern __shared__ __align__(16) unsigned char smem[];
   const Tabs<NL> t = tabs_at<NL>(smem);
   float2* tile = reinterpret_cast<float2*>(smem + Tabs<NL>::kBytes);
-  float4* xb = reinterpret_cast<float4*>(smem + Tabs<NL>::kBytes + sizeof(float2) * 2 * NL * TS);
+  float4* xb = reinterpret_cast<float4*>(smem + Tabs<NL>::kBytes);     // shares the tile region
   tabs_build<NL>(t, g_tw512);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long ord = ord0 + blockIdx.x;
@@ -57,7 +61,11 @@ __global__ void __launch_bounds__(kTM) k_rowfwd2(const T* __restrict__ k, const 
   const int pen = lane / G, g = lane % G;
   float4* buf = xb + warp * XB<NL>::kWarp + pen * XB<NL>::kPen;
   __syncthreads();
-  for (int r0 = warp * PPW; r0 < RPB; r0 += kWM * PPW) {
+  static_assert(RPB == kWM * PPW || RPB == 2 * kWM * PPW, "row tile covers one or two rounds");
+  constexpr int ROUNDS = RPB / (kWM * PPW);
+  cp keep[ROUNDS > 1 ? R1 : 1];
+  for (int round = 0; round < ROUNDS; ++round) {
+    const int r0 = round * kWM * PPW + warp * PPW;
     const int rl = r0 + pen;
     const bool act = rl < nrp;
     const long long ra = pair_row(rpb + rl, ps) * NL, rb = ra + static_cast<long long>(ps) * NL;
@@ -71,12 +79,22 @@ __global__ void __launch_bounds__(kTM) k_rowfwd2(const T* __restrict__ k, const 
     }
     cp x[R1];
     padded_fwd<NL>(z, x, g, buf, 0, t, 0u);
+    if (ROUNDS > 1 && round == 0) {
 #pragma unroll
-    for (int s = 0; s < R1; ++s) {
-      const int kk = 2 * spec_idx<NL>(g, s);
-      tile[kk * TS + rl] = make_float2(x[s].re.x, x[s].im.x);
-      tile[(kk + 1) * TS + rl] = make_float2(x[s].re.y, x[s].im.y);
+      for (int s = 0; s < R1; ++s) keep[ROUNDS > 1 ? s : 0] = x[s];
+      continue;
     }
+    __syncthreads();      // every pencil's exchange buffer is free: reuse it as the tile
+    auto put = [&](const cp (&xx)[R1], int rl_) {
+#pragma unroll
+      for (int s = 0; s < R1; ++s) {
+        const int kk = 2 * spec_idx<NL>(g, s);
+        tile[kk * TS + rl_] = make_float2(xx[s].re.x, xx[s].im.x);
+        tile[(kk + 1) * TS + rl_] = make_float2(xx[s].re.y, xx[s].im.y);
+      }
+    };
+    if constexpr (ROUNDS > 1) put(keep, warp * PPW + pen);
+    put(x, rl);
   }
   __syncthreads();
   float2* zt = Zt + static_cast<long long>(blockIdx.x) * L;
@@ -88,7 +106,7 @@ __global__ void __launch_bounds__(kTM) k_rowfwd2(const T* __restrict__ k, const 
 
 // ------------------------------------------------------------- inverse rows
 template <int NL, class T>
-__global__ void __launch_bounds__(kTM) k_rowinv2(const float2* __restrict__ Zt, const T* __restrict__ q,
+__global__ void __launch_bounds__(kTM, 2) k_rowinv2(const float2* __restrict__ Zt, const T* __restrict__ q,
                                                  T* __restrict__ y, long long ord0, int rp_total, int ps, int B,
                                                  int C) {
   using R = RT<NL>;
@@ -96,7 +114,7 @@ __global__ void __launch_bounds__(kTM) k_rowinv2(const float2* __restrict__ Zt, 
   extern __shared__ __align__(16) unsigned char smem[];
   const Tabs<NL> t = tabs_at<NL>(smem);
   float2* tile = reinterpret_cast<float2*>(smem + Tabs<NL>::kBytes);
-  float4* xb = reinterpret_cast<float4*>(smem + Tabs<NL>::kBytes + sizeof(float2) * 2 * NL * TS);
+  float4* xb = reinterpret_cast<float4*>(smem + Tabs<NL>::kBytes);     // shares the tile region
   tabs_build<NL>(t, g_tw512);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long ord = ord0 + blockIdx.x;
@@ -113,7 +131,24 @@ __global__ void __launch_bounds__(kTM) k_rowinv2(const float2* __restrict__ Zt, 
   __syncthreads();
   const int pen = lane / G, g = lane % G;
   float4* buf = xb + warp * XB<NL>::kWarp + pen * XB<NL>::kPen;
-  for (int r0 = warp * PPW; r0 < RPB; r0 += kWM * PPW) {
+  static_assert(RPB == kWM * PPW || RPB == 2 * kWM * PPW, "row tile covers one or two rounds");
+  constexpr int ROUNDS = RPB / (kWM * PPW);
+  // pull every round's inputs out of the tile before the tile region turns
+  // into exchange buffers
+  cp xin[ROUNDS][R1];
+#pragma unroll
+  for (int round = 0; round < ROUNDS; ++round) {
+    const int rl = round * kWM * PPW + warp * PPW + pen;
+#pragma unroll
+    for (int s = 0; s < R1; ++s) {
+      const int kk = 2 * spec_idx<NL>(g, s);
+      const float2 e = tile[kk * TS + rl], d = tile[(kk + 1) * TS + rl];
+      xin[round][s] = {make_float2(e.x, d.x), make_float2(e.y, d.y)};
+    }
+  }
+  __syncthreads();
+  for (int round = 0; round < ROUNDS; ++round) {
+    const int r0 = round * kWM * PPW + warp * PPW;
     const int rl = r0 + pen;
     const bool act = rl < nrp;
     const long long ra = pair_row(rpb + rl, ps) * NL, rb = ra + static_cast<long long>(ps) * NL;
@@ -126,11 +161,7 @@ __global__ void __launch_bounds__(kTM) k_rowinv2(const float2* __restrict__ Zt, 
     }
     cp x[R1];
 #pragma unroll
-    for (int s = 0; s < R1; ++s) {
-      const int kk = 2 * spec_idx<NL>(g, s);
-      const float2 e = tile[kk * TS + rl], d = tile[(kk + 1) * TS + rl];
-      x[s] = {make_float2(e.x, d.x), make_float2(e.y, d.y)};
-    }
+    for (int s = 0; s < R1; ++s) x[s] = xin[round][s];
     float2 o[R1];
     padded_inv<NL>(x, o, g, buf, 0, t, 0u);
     if (act) {
@@ -155,7 +186,7 @@ struct M1 {
 };
 
 template <int N0>
-__global__ void __launch_bounds__(kTM) k_mid1v2(float2* __restrict__ Zt, const float4* __restrict__ spec,
+__global__ void __launch_bounds__(kTM, 2) k_mid1v2(float2* __restrict__ Zt, const float4* __restrict__ spec,
                                                 long long sbs4, int N1, long long ord0, int B, int C) {
   using M = M1<N0>;
   constexpr int G = M::G, PPW = M::PPW, R1 = P2<N0>::R1, RP = N0 / 2, HS = R1 / 2;
@@ -440,7 +471,7 @@ __device__ __forceinline__ void k_mid2_body(float2* __restrict__ Zt, const float
 }
 
 template <int N0, int N1>
-__global__ void __launch_bounds__(kTM) k_mid2v2(float2* __restrict__ Zt, const float4* __restrict__ spec,
+__global__ void __launch_bounds__(kTM, 2) k_mid2v2(float2* __restrict__ Zt, const float4* __restrict__ spec,
                                                 long long sbs4, int N2, long long ord0, int B, int C) {
   k_mid2_body<N0, N1, false>(Zt, spec, sbs4, N2, ord0, B, C, blockIdx.x, 0);
 }
