@@ -39,6 +39,54 @@ struct RT {
   static constexpr size_t kBytes = Tabs<NL>::kBytes + (kTile > kXb ? kTile : kXb);
 };
 
+// Tile <-> workspace copies: rows of RPB row pairs (float2) per frequency kk,
+// moved as float4 pairs, every load of a thread issued before its stores.
+template <int NL, int RPB, int TS>
+__device__ __forceinline__ void tile_from_ws(float2* tile, const float2* __restrict__ zt, int rp_total, int rpb,
+                                             int nrp) {
+  constexpr int PER = NL * RPB / kTM;                     // float4 per thread
+  static_assert(PER * kTM == NL * RPB && RPB % 2 == 0, "tile split");
+  float4 v[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = 2 * (threadIdx.x + i * kTM);
+    const int kk = e / RPB, rl = e % RPB;
+    const float2* src = zt + static_cast<long long>(kk) * rp_total + rpb + rl;
+    if (rl + 1 < nrp) {
+      v[i] = __ldcg(reinterpret_cast<const float4*>(src));
+    } else {
+      const float2 a = rl < nrp ? __ldcg(src) : make_float2(0.f, 0.f);
+      v[i] = make_float4(a.x, a.y, 0.f, 0.f);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = 2 * (threadIdx.x + i * kTM);
+    const int kk = e / RPB, rl = e % RPB;
+    tile[kk * TS + rl] = make_float2(v[i].x, v[i].y);
+    tile[kk * TS + rl + 1] = make_float2(v[i].z, v[i].w);
+  }
+}
+
+template <int NL, int RPB, int TS>
+__device__ __forceinline__ void tile_to_ws(const float2* tile, float2* __restrict__ zt, int rp_total, int rpb,
+                                           int nrp) {
+  constexpr int PER = NL * RPB / kTM;
+  static_assert(PER * kTM == NL * RPB && RPB % 2 == 0, "tile split");
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = 2 * (threadIdx.x + i * kTM);
+    const int kk = e / RPB, rl = e % RPB;
+    const float2 a = tile[kk * TS + rl], b = tile[kk * TS + rl + 1];
+    float2* dst = zt + static_cast<long long>(kk) * rp_total + rpb + rl;
+    if (rl + 1 < nrp) {
+      __stcg(reinterpret_cast<float4*>(dst), make_float4(a.x, a.y, b.x, b.y));
+    } else if (rl < nrp) {
+      __stcg(dst, a);
+    }
+  }
+}
+
 // ------------------------------------------------------------- forward rows
 template <int NL, class T>
 __global__ void __launch_bounds__(kTM, 2) k_rowfwd2(const T* __restrict__ k, const T* __restrict__ v,
@@ -97,11 +145,7 @@ __global__ void __launch_bounds__(kTM, 2) k_rowfwd2(const T* __restrict__ k, con
     put(x, rl);
   }
   __syncthreads();
-  float2* zt = Zt + static_cast<long long>(blockIdx.x) * L;
-  for (int e = threadIdx.x; e < 2 * NL * RPB; e += kTM) {
-    const int kk = e / RPB, rl = e % RPB;
-    if (rl < nrp) zt[static_cast<long long>(kk) * rp_total + rpb + rl] = tile[kk * TS + rl];
-  }
+  tile_to_ws<NL, RPB, TS>(tile, Zt + static_cast<long long>(blockIdx.x) * L, rp_total, rpb, nrp);
 }
 
 // ------------------------------------------------------------- inverse rows
@@ -123,11 +167,7 @@ __global__ void __launch_bounds__(kTM, 2) k_rowinv2(const float2* __restrict__ Z
   const long long base = (static_cast<long long>(b) * C + c) * L;
   const int rpb = blockIdx.y * RPB;
   const int nrp = min(RPB, rp_total - rpb);
-  const float2* zt = Zt + static_cast<long long>(blockIdx.x) * L;
-  for (int e = threadIdx.x; e < 2 * NL * RPB; e += kTM) {
-    const int kk = e / RPB, rl = e % RPB;
-    tile[kk * TS + rl] = (rl < nrp) ? zt[static_cast<long long>(kk) * rp_total + rpb + rl] : make_float2(0.f, 0.f);
-  }
+  tile_from_ws<NL, RPB, TS>(tile, Zt + static_cast<long long>(blockIdx.x) * L, rp_total, rpb, nrp);
   __syncthreads();
   const int pen = lane / G, g = lane % G;
   float4* buf = xb + warp * XB<NL>::kWarp + pen * XB<NL>::kPen;
