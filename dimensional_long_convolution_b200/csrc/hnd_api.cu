@@ -20,7 +20,7 @@ namespace {
 thread_local int g_last_launches = 0;
 
 constexpr size_t kStatusBytes = 256;                  // status word + padding
-constexpr size_t kWaveBudget = size_t(48) << 20;      // multi-pass intermediate per wave
+constexpr size_t kWaveBudget = size_t(96) << 20;      // multi-pass intermediate per wave (measured best of 24/48/96 MiB)
 constexpr size_t kFilterBudget = size_t(64) << 20;    // filter grid per channel chunk
 constexpr int kFilterMaxChunk = 16;
 

@@ -208,14 +208,14 @@ def test_launch_counts_per_tier():
 
 
 def test_multi_wave_schedule():
-    """More pairs than one wave of the multi-pass tier holds (2D 256^2: 96
-    pairs per wave), so several waves run back to back."""
+    """More pairs than one wave of the multi-pass tier holds (2D 256^2: 192
+    pairs per wave), so several waves run back to back (192, 192, 16)."""
     dims = (256, 256)
-    wl = W.custom(dims, 2, 100, io_dtype="bf16", seed=31)
+    wl = W.custom(dims, 2, 200, io_dtype="bf16", seed=31)
     inp = W.make_inputs(wl)
     got, _ = run(inp)
     assert H.last_launch_count() == 9
-    chans = [0, 49, 99]
+    chans = [0, 99, 199]
     pts = sample_points(wl, 12, seed=2, channels=chans)
     K = O.implicit_kernel(inp.filt, dims, channels=chans)
     Kfull = np.zeros((wl.C,) + K.shape[1:])
