@@ -86,6 +86,11 @@ hyena_nd_status make_plan(const hyena_nd_problem* p, Plan* pl) {
     if (w < 1) w = 1;
     if (w > pairs) w = pairs;
     if (w >= p->B) w -= w % p->B;        // keep a channel's samples in one wave
+    // equal waves: no short last wave
+    const long long nw = (pairs + w - 1) / w;
+    long long we = (pairs + nw - 1) / nw;
+    if (we >= p->B && we % p->B) we += p->B - we % p->B;
+    if (we < w) w = we;
     pl->wave = w;
     ws_conv = per_pair * static_cast<size_t>(w);
   }
@@ -126,7 +131,7 @@ hyena_nd_status hyena_nd_workspace_init(void* ws, size_t ws_bytes, void* cuda_st
   if (!ws) return HYENA_ND_ERR_INVALID_ARG;
   if (!aligned16(ws)) return HYENA_ND_ERR_MISALIGNED;
   if (ws_bytes < kStatusBytes) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
-  return cuda_status(cudaMemsetAsync(ws, 0, 16, static_cast<cudaStream_t>(cuda_stream)));
+  return cuda_status(cudaMemsetAsync(ws, 0, kStatusBytes, static_cast<cudaStream_t>(cuda_stream)));
 }
 
 hyena_nd_status hyena_nd_fftconv_batched(const hyena_nd_problem* p, const void* q, const void* k, const void* v,

@@ -22,6 +22,8 @@
 // it, so the pointwise product needs no bit reversal.
 #pragma once
 
+#include <type_traits>
+
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -211,21 +213,33 @@ __device__ __forceinline__ unsigned pmask(int lane) {
   }
 }
 
-// Per-size twiddle tables in shared memory (built once per CTA):
-//   tw2[(b R2 + r) G + g] = W_N^{(g + G b) r}   pass-2 twiddles, (c, c, s, s)
-//   twi[r G + g]          = W_N^{g r}           inverse pass-2 twiddles
-//   tst[s G + g]          = W_2N^{g + s G}      twist factors, (c, s)
+// Per-size twiddle bases in shared memory (built once per CTA), [j][g]:
+//   b[j G + g] = W_N^{2^j g}  (j = 0..3: u, u^2, u^4, u^8 for u = W_N^g)
+//   b[4 G + g] = W_2N^g
+// Every twiddle of a lane follows from these and the roots W_32^e (constant
+// memory, compile-time indices):
+//   pass-2 twiddle  W_N^{(g + G b) r} = u^r W_R1^{b r}   (G / N = 1 / R1)
+//   inverse pass 2  W_N^{g r}         = u^r
+//   twist           W_2N^{g + s G}    = W_2N^g W_{2 R1}^s
+// with u^r the product of the bases of r's set bits (at most three complex
+// products).
 template <int N>
 struct Tabs {
-  static constexpr int G = P2<N>::G, R1 = P2<N>::R1;
-  static constexpr int kTw2 = R1 * G;       // float4
-  static constexpr int kTwi = R1 * G;       // float4
-  static constexpr int kTst = R1 * G;       // float2
-  static constexpr size_t kBytes = 16 * (kTw2 + kTwi) + 8 * kTst;
-  float4* tw2;
-  float4* twi;
-  float2* tst;
+  static constexpr int G = P2<N>::G;
+  static constexpr size_t kBytes = (8 * 5 * G + 15) / 16 * 16;
+  float2* b;
 };
+
+static __constant__ float2 c_w32[32] =
+#include "hnd_w32.inc"
+    ;
+
+template <int N>
+__device__ __forceinline__ Tabs<N> tabs_at(unsigned char* base) {
+  Tabs<N> t;
+  t.b = reinterpret_cast<float2*>(base);
+  return t;
+}
 
 // W_M^e from the 512-entry table W_512^k.
 __device__ __forceinline__ float2 wtab(const float2* __restrict__ W512, int M, int e) {
@@ -233,25 +247,54 @@ __device__ __forceinline__ float2 wtab(const float2* __restrict__ W512, int M, i
 }
 
 template <int N>
-__device__ __forceinline__ Tabs<N> tabs_at(unsigned char* base) {
-  Tabs<N> t;
-  t.tw2 = reinterpret_cast<float4*>(base);
-  t.twi = t.tw2 + Tabs<N>::kTw2;
-  t.tst = reinterpret_cast<float2*>(t.twi + Tabs<N>::kTwi);
-  return t;
+__device__ __forceinline__ void tabs_build(Tabs<N> t, const float2* __restrict__ W512) {
+  constexpr int G = P2<N>::G;
+  for (int e = threadIdx.x; e < 5 * G; e += blockDim.x) {
+    const int j = e / G, g = e % G;
+    t.b[e] = j < 4 ? wtab(W512, N, g << j) : wtab(W512, 2 * N, g);
+  }
+}
+
+__device__ __forceinline__ float2 cmul1(float2 a, float2 b) {
+  return make_float2(fmaf(a.x, b.x, -a.y * b.y), fmaf(a.x, b.y, a.y * b.x));
+}
+
+// u^R (1 <= R < 16): product of the bases u^{2^j} of R's set bits j >= J.
+template <int R, int J = 0>
+__device__ __forceinline__ float2 upow(const float2 (&u)[4]) {
+  static_assert(R >= 1 && R < 16, "power range");
+  if constexpr ((R >> J) == 1) return u[J];
+  else if constexpr (((R >> J) & 1) == 0) return upow<R, J + 1>(u);
+  else return cmul1(u[J], upow<R, J + 1>(u));
+}
+
+// x * W_32^E (E compile-time; E == 0: x)
+template <int E>
+__device__ __forceinline__ float2 mul_w32(float2 x) {
+  if constexpr ((E & 31) == 0) return x;
+  else if constexpr ((E & 31) == 8) return make_float2(x.y, -x.x);       // W_32^8 = -i
+  else if constexpr ((E & 31) == 16) return make_float2(-x.x, -x.y);
+  else if constexpr ((E & 31) == 24) return make_float2(-x.y, x.x);      // W_32^24 = i
+  else return cmul1(x, c_w32[E & 31]);
 }
 
 template <int N>
-__device__ __forceinline__ void tabs_build(Tabs<N> t, const float2* __restrict__ W512) {
-  constexpr int G = P2<N>::G, R2 = P2<N>::R2, R1 = P2<N>::R1;
-  for (int e = threadIdx.x; e < R1 * G; e += blockDim.x) {
-    const int g = e % G, sr = e / G;              // sr = b R2 + r (pass 2) or r (inverse) or s (twist)
-    const int b = sr / (R2 > 0 ? R2 : 1), r = sr % (R2 > 0 ? R2 : 1);
-    const float2 w = wtab(W512, N, (g + G * b) * r);
-    t.tw2[e] = make_float4(w.x, w.x, w.y, w.y);
-    const float2 wi = wtab(W512, N, g * sr);
-    t.twi[e] = make_float4(wi.x, wi.x, wi.y, wi.y);
-    t.tst[e] = wtab(W512, 2 * N, g + sr * G);
+__device__ __forceinline__ void load_bases(Tabs<N> t, int g, float2 (&u)[4]) {
+  constexpr int G = P2<N>::G, R1 = P2<N>::R1;
+  u[0] = t.b[g];
+  u[1] = t.b[G + g];
+  u[2] = t.b[2 * G + g];
+  u[3] = R1 == 16 ? t.b[3 * G + g] : make_float2(1.f, 0.f);
+}
+
+__device__ __forceinline__ float4 w4of(float2 w) { return make_float4(w.x, w.x, w.y, w.y); }
+
+// Compile-time loops (the twiddle exponents must be constants).
+template <int I, int E, class F>
+__device__ __forceinline__ void sfor(F&& f) {
+  if constexpr (I < E) {
+    f(std::integral_constant<int, I>{});
+    sfor<I + 1, E>(f);
   }
 }
 
@@ -272,20 +315,25 @@ __device__ __forceinline__ void fft_fwd(cp (&x)[P2<N>::R1], int g, float4* buf, 
     for (int r = 0; r < R1; ++r)
       buf[padx<R1>(g * R1 + r)] = make_float4(x[r].re.x, x[r].re.y, x[r].im.x, x[r].im.y);
     __syncwarp();
-#pragma unroll
-    for (int b = 0; b < R1 / R2; ++b) {
-#pragma unroll
-      for (int r = 0; r < R2; ++r) {
+    float2 u[4];
+    load_bases<N>(t, g, u);
+    sfor<0, R1 / R2>([&](auto bc) {
+      constexpr int b = decltype(bc)::value;
+      sfor<0, R2>([&](auto rc) {
+        constexpr int r = decltype(rc)::value;
         const float4 v = buf[padx<R1>(g + G * b + r * R1)];
         cp y = {make_float2(v.x, v.y), make_float2(v.z, v.w)};
-        if (r > 0) y = ctw<false>(y, t.tw2[(b * R2 + r) * G + g]);
+        if constexpr (r > 0) {
+          // W_N^{(g + G b) r} = u^r W_R1^{b r}
+          y = ctw<false>(y, w4of(mul_w32<(b * r % R1) * (32 / R1)>(upow<r>(u))));
+        }
         x[b * R2 + r] = y;
-      }
+      });
       if constexpr (R2 == 16) dft16<false>(&x[b * 16]);
       else if constexpr (R2 == 8) dft8<false>(&x[b * 8]);
       else if constexpr (R2 == 4) dft4<false>(x[b * 4], x[b * 4 + 1], x[b * 4 + 2], x[b * 4 + 3]);
       else dft2(x[b * 2], x[b * 2 + 1]);
-    }
+    });
   }
 }
 
@@ -315,13 +363,15 @@ __device__ __forceinline__ void fft_inv(cp (&x)[P2<N>::R1], int g, float4* buf, 
       }
     }
     __syncwarp();
-#pragma unroll
-    for (int r = 0; r < R1; ++r) {
+    float2 u[4];
+    load_bases<N>(t, g, u);
+    sfor<0, R1>([&](auto rc) {
+      constexpr int r = decltype(rc)::value;
       const float4 v = buf[padx<PD>(g + r * G)];
       cp y = {make_float2(v.x, v.y), make_float2(v.z, v.w)};
-      if (r > 0) y = ctw<true>(y, t.twi[r * G + g]);
+      if constexpr (r > 0) y = ctw<true>(y, w4of(upow<r>(u)));     // W_N^{g r}
       x[r] = y;
-    }
+    });
     if constexpr (R1 == 16) dft16<true>(x);
     else dft8<true>(x);
   }
@@ -333,14 +383,15 @@ __device__ __forceinline__ void fft_inv(cp (&x)[P2<N>::R1], int g, float4* buf, 
 template <int N>
 __device__ __forceinline__ void padded_fwd(const float2 (&z)[P2<N>::R1], cp (&x)[P2<N>::R1], int g, float4* buf,
                                            int key, Tabs<N> t, unsigned mask) {
-  constexpr int G = P2<N>::G;
-#pragma unroll
-  for (int s = 0; s < P2<N>::R1; ++s) {
-    const float2 w = t.tst[s * G + g];
+  constexpr int G = P2<N>::G, R1 = P2<N>::R1;
+  const float2 tg = t.b[4 * G + g];
+  sfor<0, R1>([&](auto sc) {
+    constexpr int s = decltype(sc)::value;
+    const float2 w = mul_w32<s * (16 / R1)>(tg);     // W_2N^{g + s G} = W_2N^g W_{2 R1}^s
     const float ore = fmaf(z[s].x, w.x, -z[s].y * w.y);
     const float oim = fmaf(z[s].x, w.y, z[s].y * w.x);
     x[s] = {make_float2(z[s].x, ore), make_float2(z[s].y, oim)};
-  }
+  });
   fft_fwd<N>(x, g, buf, key, t, mask);
 }
 
@@ -349,15 +400,16 @@ __device__ __forceinline__ void padded_fwd(const float2 (&z)[P2<N>::R1], cp (&x)
 template <int N>
 __device__ __forceinline__ void padded_inv(cp (&x)[P2<N>::R1], float2 (&out)[P2<N>::R1], int g, float4* buf, int key,
                                            Tabs<N> t, unsigned mask) {
-  constexpr int G = P2<N>::G;
+  constexpr int G = P2<N>::G, R1 = P2<N>::R1;
   fft_inv<N>(x, g, buf, key, t, mask);
-#pragma unroll
-  for (int s = 0; s < P2<N>::R1; ++s) {
-    const float2 w = t.tst[s * G + g];   // untwist by conj(W_2N^{g + s G})
+  const float2 tg = t.b[4 * G + g];
+  sfor<0, R1>([&](auto sc) {
+    constexpr int s = decltype(sc)::value;
+    const float2 w = mul_w32<s * (16 / R1)>(tg);   // untwist by conj(W_2N^{g + s G})
     const float re = fmaf(x[s].re.y, w.x, fmaf(x[s].im.y, w.y, x[s].re.x));
     const float im = fmaf(x[s].im.y, w.x, fmaf(-x[s].re.y, w.y, x[s].im.x));
     out[s] = make_float2(re, im);
-  }
+  });
 }
 
 // Partner frequency -k (mod 2N) of spectral slot (f, path): path 0 -> (N - f)

@@ -26,6 +26,27 @@ inline cudaError_t ensure_smem(K kernel, size_t bytes) {
   return e;
 }
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel on the stream finishes; it must wait for that grid
+// (griddepcontrol.wait) before touching memory the previous work wrote.
+// `early` = false launches normally (the kernel's griddepcontrol calls are
+// then no-ops).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(bool early, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = early ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 }  // namespace hnd
 
 // Switch over the power-of-two extents 8..256 (LIST_N) or 8..128 (LIST_S).

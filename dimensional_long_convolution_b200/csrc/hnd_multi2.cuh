@@ -23,6 +23,20 @@ namespace cg = cooperative_groups;
 constexpr int kTM = 256;          // threads per CTA in the multi-pass kernels
 constexpr int kWM = kTM / 32;
 
+// Barrier over the kTM task threads (named barrier 1).  In the stage kernels
+// these are all the threads of the CTA; the persistent pipeline adds a
+// scheduler warp that does not take part.
+__device__ __forceinline__ void task_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kTM) : "memory"); }
+
+// Programmatic dependent launch: the stage kernels run back to back on one
+// stream.  Each lets the next stage's CTAs be scheduled as soon as all of its
+// own CTAs have started (they then build their tables on SMs freed by this
+// stage's tail), and waits for the previous grid to complete, with its
+// memory visible, before its first global access.  Both are no-ops for a
+// launch without the programmatic-serialization attribute.
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Row pair rp = rows (ra, ra + ps): 2D pairs row r with r + n0/2 (ps = n0/2),
 // 3D pairs neighbouring rows (ps = 1).
 __device__ __forceinline__ long long pair_row(long long rp, int ps) { return (rp / ps) * 2 * ps + (rp % ps); }
@@ -88,27 +102,20 @@ __device__ __forceinline__ void tile_to_ws(const float2* tile, float2* __restric
 }
 
 // ------------------------------------------------------------- forward rows
+// One task: RPB row pairs starting at rpb of one volume (activations at
+// `base`, workspace `ztv`).  `work` is the shared region after the tables.
 template <int NL, class T>
-__global__ void __launch_bounds__(kTM, 2) k_rowfwd2(const T* __restrict__ k, const T* __restrict__ v,
-                                                 float2* __restrict__ Zt, long long ord0, int rp_total, int ps,
-                                                 int B, int C) {
+__device__ __forceinline__ void rowfwd_task(const Tabs<NL> t, unsigned char* work, const T* __restrict__ k,
+                                            const T* __restrict__ v, float2* __restrict__ ztv, long long base,
+                                            int rpb, int rp_total, int ps) {
   using R = RT<NL>;
   constexpr int G = R::G, PPW = R::PPW, R1 = P2<NL>::R1, RPB = R::RPB, TS = R::TS;
-  extern __shared__ __align__(16) unsigned char smem[];
-  const Tabs<NL> t = tabs_at<NL>(smem);
-  float2* tile = reinterpret_cast<float2*>(smem + Tabs<NL>::kBytes);
-  float4* xb = reinterpret_cast<float4*>(smem + Tabs<NL>::kBytes);     // shares the tile region
-  tabs_build<NL>(t, g_tw512);
+  float2* tile = reinterpret_cast<float2*>(work);
+  float4* xb = reinterpret_cast<float4*>(work);     // shares the tile region
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long ord = ord0 + blockIdx.x;
-  const int c = static_cast<int>(ord / B), b = static_cast<int>(ord % B);
-  const long long L = static_cast<long long>(rp_total) * 2 * NL;
-  const long long base = (static_cast<long long>(b) * C + c) * L;
-  const int rpb = blockIdx.y * RPB;
   const int nrp = min(RPB, rp_total - rpb);
   const int pen = lane / G, g = lane % G;
   float4* buf = xb + warp * XB<NL>::kWarp + pen * XB<NL>::kPen;
-  __syncthreads();
   static_assert(RPB == kWM * PPW || RPB == 2 * kWM * PPW, "row tile covers one or two rounds");
   constexpr int ROUNDS = RPB / (kWM * PPW);
   cp keep[ROUNDS > 1 ? R1 : 1];
@@ -132,7 +139,7 @@ __global__ void __launch_bounds__(kTM, 2) k_rowfwd2(const T* __restrict__ k, con
       for (int s = 0; s < R1; ++s) keep[ROUNDS > 1 ? s : 0] = x[s];
       continue;
     }
-    __syncthreads();      // every pencil's exchange buffer is free: reuse it as the tile
+    task_sync();      // every pencil's exchange buffer is free: reuse it as the tile
     auto put = [&](const cp (&xx)[R1], int rl_) {
 #pragma unroll
       for (int s = 0; s < R1; ++s) {
@@ -144,31 +151,40 @@ __global__ void __launch_bounds__(kTM, 2) k_rowfwd2(const T* __restrict__ k, con
     if constexpr (ROUNDS > 1) put(keep, warp * PPW + pen);
     put(x, rl);
   }
+  task_sync();
+  tile_to_ws<NL, RPB, TS>(tile, ztv, rp_total, rpb, nrp);
+}
+
+template <int NL, class T>
+__global__ void __launch_bounds__(kTM, 2) k_rowfwd2(const T* __restrict__ k, const T* __restrict__ v,
+                                                 float2* __restrict__ Zt, long long ord0, int rp_total, int ps,
+                                                 int B, int C) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  pdl_release();
+  const Tabs<NL> t = tabs_at<NL>(smem);
+  tabs_build<NL>(t, g_tw512);
+  const long long ord = ord0 + blockIdx.x;
+  const int c = static_cast<int>(ord / B), b = static_cast<int>(ord % B);
+  const long long L = static_cast<long long>(rp_total) * 2 * NL;
   __syncthreads();
-  tile_to_ws<NL, RPB, TS>(tile, Zt + static_cast<long long>(blockIdx.x) * L, rp_total, rpb, nrp);
+  pdl_wait();
+  rowfwd_task<NL, T>(t, smem + Tabs<NL>::kBytes, k, v, Zt + static_cast<long long>(blockIdx.x) * L,
+                     (static_cast<long long>(b) * C + c) * L, blockIdx.y * RT<NL>::RPB, rp_total, ps);
 }
 
 // ------------------------------------------------------------- inverse rows
 template <int NL, class T>
-__global__ void __launch_bounds__(kTM, 2) k_rowinv2(const float2* __restrict__ Zt, const T* __restrict__ q,
-                                                 T* __restrict__ y, long long ord0, int rp_total, int ps, int B,
-                                                 int C) {
+__device__ __forceinline__ void rowinv_task(const Tabs<NL> t, unsigned char* work, const float2* __restrict__ ztv,
+                                            const T* __restrict__ q, T* __restrict__ y, long long base, int rpb,
+                                            int rp_total, int ps) {
   using R = RT<NL>;
   constexpr int G = R::G, PPW = R::PPW, R1 = P2<NL>::R1, RPB = R::RPB, TS = R::TS;
-  extern __shared__ __align__(16) unsigned char smem[];
-  const Tabs<NL> t = tabs_at<NL>(smem);
-  float2* tile = reinterpret_cast<float2*>(smem + Tabs<NL>::kBytes);
-  float4* xb = reinterpret_cast<float4*>(smem + Tabs<NL>::kBytes);     // shares the tile region
-  tabs_build<NL>(t, g_tw512);
+  float2* tile = reinterpret_cast<float2*>(work);
+  float4* xb = reinterpret_cast<float4*>(work);     // shares the tile region
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long ord = ord0 + blockIdx.x;
-  const int c = static_cast<int>(ord / B), b = static_cast<int>(ord % B);
-  const long long L = static_cast<long long>(rp_total) * 2 * NL;
-  const long long base = (static_cast<long long>(b) * C + c) * L;
-  const int rpb = blockIdx.y * RPB;
   const int nrp = min(RPB, rp_total - rpb);
-  tile_from_ws<NL, RPB, TS>(tile, Zt + static_cast<long long>(blockIdx.x) * L, rp_total, rpb, nrp);
-  __syncthreads();
+  tile_from_ws<NL, RPB, TS>(tile, ztv, rp_total, rpb, nrp);
+  task_sync();
   const int pen = lane / G, g = lane % G;
   float4* buf = xb + warp * XB<NL>::kWarp + pen * XB<NL>::kPen;
   static_assert(RPB == kWM * PPW || RPB == 2 * kWM * PPW, "row tile covers one or two rounds");
@@ -186,7 +202,7 @@ __global__ void __launch_bounds__(kTM, 2) k_rowinv2(const float2* __restrict__ Z
       xin[round][s] = {make_float2(e.x, d.x), make_float2(e.y, d.y)};
     }
   }
-  __syncthreads();
+  task_sync();
   for (int round = 0; round < ROUNDS; ++round) {
     const int r0 = round * kWM * PPW + warp * PPW;
     const int rl = r0 + pen;
@@ -215,6 +231,23 @@ __global__ void __launch_bounds__(kTM, 2) k_rowinv2(const float2* __restrict__ Z
   }
 }
 
+template <int NL, class T>
+__global__ void __launch_bounds__(kTM, 2) k_rowinv2(const float2* __restrict__ Zt, const T* __restrict__ q,
+                                                 T* __restrict__ y, long long ord0, int rp_total, int ps, int B,
+                                                 int C) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  pdl_release();
+  const Tabs<NL> t = tabs_at<NL>(smem);
+  tabs_build<NL>(t, g_tw512);
+  const long long ord = ord0 + blockIdx.x;
+  const int c = static_cast<int>(ord / B), b = static_cast<int>(ord % B);
+  const long long L = static_cast<long long>(rp_total) * 2 * NL;
+  __syncthreads();
+  pdl_wait();
+  rowinv_task<NL, T>(t, smem + Tabs<NL>::kBytes, Zt + static_cast<long long>(blockIdx.x) * L, q, y,
+                     (static_cast<long long>(b) * C + c) * L, blockIdx.y * RT<NL>::RPB, rp_total, ps);
+}
+
 // ---------------------------------------------------------- 2D column units
 // Zt[kk][rp] per volume, rp in [0, n0/2) with row pair (rp, rp + n0/2); unit cu
 // = last-axis frequency kx (cu >= 1) or the combined DC/Nyquist unit (cu = 0).
@@ -225,27 +258,15 @@ struct M1 {
   static constexpr size_t kBytes = Tabs<N0>::kBytes + 16ull * XB<N0>::kWarp * kWM;
 };
 
-template <int N0>
-__global__ void __launch_bounds__(kTM, 2) k_mid1v2(float2* __restrict__ Zt, const float4* __restrict__ spec,
-                                                long long sbs4, int N1, long long ord0, int B, int C) {
-  using M = M1<N0>;
-  constexpr int G = M::G, PPW = M::PPW, R1 = P2<N0>::R1, RP = N0 / 2, HS = R1 / 2;
-  extern __shared__ __align__(16) unsigned char smem[];
-  const Tabs<N0> t = tabs_at<N0>(smem);
-  float4* xb = reinterpret_cast<float4*>(smem + Tabs<N0>::kBytes);
-  tabs_build<N0>(t, g_tw512);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long ord = ord0 + blockIdx.x;
-  const int c = static_cast<int>(ord / B), b = static_cast<int>(ord % B);
-  const int u0 = blockIdx.y * M::UPB;
-  const float4* sp = spec + static_cast<long long>(b) * sbs4 + static_cast<long long>(c) * (N1 + 1) * N0;
-  __syncthreads();
-  float2* zt = Zt + static_cast<long long>(blockIdx.x) * 2 * N1 * RP;
-  const int pen = lane / G, g = lane % G;
-  float4* buf = xb + warp * XB<N0>::kWarp + pen * XB<N0>::kPen;
-  const int cu = u0 + warp * PPW + pen;
+// One column unit cu (one pencil of lanes).  GEN: the warp that holds unit
+// 0, the combined DC/Nyquist unit, whose product needs the partner
+// frequency; every pencil of that warp takes this path (for cu != 0 the
+// partner term is multiplied by zero).
+template <int N0, bool GEN>
+__device__ __forceinline__ void mid1_unit(const Tabs<N0> t, float4* buf, float2* __restrict__ zt,
+                                          const float4* __restrict__ sp, int N1, int cu, int g) {
+  constexpr int G = P2<N0>::G, R1 = P2<N0>::R1, RP = N0 / 2, HS = R1 / 2;
   const bool act = cu < N1;
-  const bool general = u0 == 0 && warp == 0;
   const int kx = act ? cu : 1, kxm = cu == 0 ? N1 : 2 * N1 - kx;
   float2 z[R1];
 #pragma unroll
@@ -253,8 +274,8 @@ __global__ void __launch_bounds__(kTM, 2) k_mid1v2(float2* __restrict__ Zt, cons
     const int rp = g + s * G;
     float2 z1 = make_float2(0.f, 0.f), z2 = z1;
     if (act) {
-      z1 = zt[static_cast<long long>(kx) * RP + rp];
-      z2 = zt[static_cast<long long>(kxm) * RP + rp];
+      z1 = __ldcg(zt + static_cast<long long>(kx) * RP + rp);
+      z2 = __ldcg(zt + static_cast<long long>(kxm) * RP + rp);
     }
     if (cu == 0) {
       z[s] = make_float2(z1.x, z2.x);
@@ -267,7 +288,7 @@ __global__ void __launch_bounds__(kTM, 2) k_mid1v2(float2* __restrict__ Zt, cons
   cp x[R1];
   padded_fwd<N0>(z, x, g, buf, 0, t, 0u);
   const float4* su = sp + (cu == 0 ? 0LL : static_cast<long long>(cu + 1) * N0);
-  if (general) {
+  if constexpr (GEN) {
     cp xp[R1];
     fetch_partner<N0>(x, xp, g, buf, 0, 0u);
 #pragma unroll
@@ -279,11 +300,13 @@ __global__ void __launch_bounds__(kTM, 2) k_mid1v2(float2* __restrict__ Zt, cons
       const cp bb = cmulp(xc, make_float2(Bc.x, Bc.y), make_float2(Bc.z, Bc.w));
       x[s] = cadd(a, bb);
     }
-  } else if (act) {
+  } else {
+    if (act) {
 #pragma unroll
-    for (int s = 0; s < R1; ++s) {
-      const float4 S = __ldg(su + s * G + g);
-      x[s] = cmulp(x[s], make_float2(S.x, S.y), make_float2(S.z, S.w));
+      for (int s = 0; s < R1; ++s) {
+        const float4 S = __ldg(su + s * G + g);
+        x[s] = cmulp(x[s], make_float2(S.x, S.y), make_float2(S.z, S.w));
+      }
     }
   }
   float2 o[R1];
@@ -302,6 +325,46 @@ __global__ void __launch_bounds__(kTM, 2) k_mid1v2(float2* __restrict__ Zt, cons
       }
     }
   }
+}
+
+// The DC/Nyquist warp's path, kept out of line so that its extra registers
+// do not weigh on the common path.
+template <int N0>
+__device__ __noinline__ void mid1_unit_gen(const Tabs<N0> t, float4* buf, float2* __restrict__ zt,
+                                           const float4* __restrict__ sp, int N1, int cu, int g) {
+  mid1_unit<N0, true>(t, buf, zt, sp, N1, cu, g);
+}
+
+// One task: UPB column units starting at u0 of one volume; `sp` is the
+// channel's spectrum for this sample.
+template <int N0>
+__device__ __forceinline__ void mid1_task(const Tabs<N0> t, unsigned char* work, float2* __restrict__ zt,
+                                          const float4* __restrict__ sp, int N1, int u0) {
+  using M = M1<N0>;
+  constexpr int G = M::G, PPW = M::PPW;
+  float4* xb = reinterpret_cast<float4*>(work);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pen = lane / G, g = lane % G;
+  float4* buf = xb + warp * XB<N0>::kWarp + pen * XB<N0>::kPen;
+  const int cu = u0 + warp * PPW + pen;
+  if (u0 == 0 && warp == 0) mid1_unit_gen<N0>(t, buf, zt, sp, N1, cu, g);
+  else mid1_unit<N0, false>(t, buf, zt, sp, N1, cu, g);
+}
+
+template <int N0>
+__global__ void __launch_bounds__(kTM, 2) k_mid1v2(float2* __restrict__ Zt, const float4* __restrict__ spec,
+                                                long long sbs4, int N1, long long ord0, int B, int C) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  pdl_release();
+  const Tabs<N0> t = tabs_at<N0>(smem);
+  tabs_build<N0>(t, g_tw512);
+  const long long ord = ord0 + blockIdx.x;
+  const int c = static_cast<int>(ord / B), b = static_cast<int>(ord % B);
+  const float4* sp = spec + static_cast<long long>(b) * sbs4 + static_cast<long long>(c) * (N1 + 1) * N0;
+  __syncthreads();
+  pdl_wait();
+  mid1_task<N0>(t, smem + Tabs<N0>::kBytes, Zt + static_cast<long long>(blockIdx.x) * 2 * N1 * (N0 / 2), sp, N1,
+                blockIdx.y * M1<N0>::UPB);
 }
 
 // ---------------------------------------------------------------- 3D slabs
@@ -331,8 +394,8 @@ __device__ __forceinline__ void slab_rows_in(const float2* __restrict__ zt, long
   for (int s = 0; s < R1; ++s) {
     const int yy = g + s * G;
     const long long rp = (static_cast<long long>(z) * N1 + yy) >> 1;
-    const float2 z1 = zt[kx * RPn + rp];
-    const float2 z2 = self_conj ? z1 : zt[kxm * RPn + rp];
+    const float2 z1 = __ldcg(zt + kx * RPn + rp);
+    const float2 z2 = self_conj ? z1 : __ldcg(zt + kxm * RPn + rp);
     x[s] = (yy & 1) ? unpack_b(z1, z2) : unpack_a(z1, z2);
   }
 }
@@ -365,36 +428,22 @@ __device__ __forceinline__ void slab_rows_out(float2* __restrict__ zt, long long
   }
 }
 
+// One task: the slab of last-axis frequency kx of one volume (`zt`), with the
+// channel's slab spectrum `sslab` for this sample.  `work` holds F, then the
+// exchange buffers.
 template <int N0, int N1, bool HALF>
-__device__ __forceinline__ void k_mid2_body(float2* __restrict__ Zt, const float4* __restrict__ spec, long long sbs4,
-                                            int N2, long long ord0, int B, int C, int vol_local, int h) {
+__device__ __forceinline__ void mid2_task(const Tabs<N0> t0, const Tabs<N1> t1, unsigned char* work,
+                                          float2* __restrict__ zt, const float4* __restrict__ sslab, int N2, int kx,
+                                          int h) {
   using M = M2<N0, N1, HALF>;
   constexpr int FS = M::FS, NKY = M::NKY;
   constexpr int G0 = P2<N0>::G, R0 = P2<N0>::R1, G1 = P2<N1>::G, R1 = P2<N1>::R1;
-  extern __shared__ __align__(16) unsigned char smem[];
-  const Tabs<N0> t0 = tabs_at<N0>(smem);
-  Tabs<N1> t1;
-  if constexpr (N0 == N1) {
-    t1 = t0;
-  } else {
-    t1 = tabs_at<N1>(smem + Tabs<N0>::kBytes);
-  }
-  float2* F = reinterpret_cast<float2*>(smem + M::kTabs);
-  float4* xb = reinterpret_cast<float4*>(smem + M::kTabs + sizeof(float2) * NKY * FS);
-  tabs_build<N0>(t0, g_tw512);
-  if constexpr (N0 != N1) tabs_build<N1>(t1, g_tw512);
+  float2* F = reinterpret_cast<float2*>(work);
+  float4* xb = reinterpret_cast<float4*>(work + sizeof(float2) * NKY * FS);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long ord = ord0 + vol_local;
-  const int c = static_cast<int>(ord / B), b = static_cast<int>(ord % B);
   const long long RPn = static_cast<long long>(N0) * N1 / 2;
-  float2* zt = Zt + static_cast<long long>(vol_local) * 2 * N2 * RPn;
-  const int kx = blockIdx.y;
   const bool self_conj = (kx == 0) || (kx == N2);
   const int kxm = self_conj ? kx : 2 * N2 - kx;
-  const long long slab = 2LL * N1 * N0;                 // float4 per slab
-  const float4* sslab = spec + static_cast<long long>(b) * sbs4 + static_cast<long long>(c) * (N2 + 1) * slab +
-                        static_cast<long long>(kx) * slab;
-  __syncthreads();
   // step 1: y transforms, one pencil per z
   {
     constexpr int PPW = 32 / G1;
@@ -426,7 +475,7 @@ __device__ __forceinline__ void k_mid2_body(float2* __restrict__ Zt, const float
       }
     }
   }
-  __syncthreads();
+  task_sync();
   // step 2: z-pencil convolution per ky row held here; pencils of a warp
   // take rows 8 apart (bank groups of F)
   {
@@ -467,7 +516,7 @@ __device__ __forceinline__ void k_mid2_body(float2* __restrict__ Zt, const float
   if constexpr (HALF) {
     cg::this_cluster().sync();
   } else {
-    __syncthreads();
+    task_sync();
   }
   // step 3: inverse y transforms, repack, write back
   {
@@ -510,10 +559,39 @@ __device__ __forceinline__ void k_mid2_body(float2* __restrict__ Zt, const float
   if constexpr (HALF) cg::this_cluster().sync();
 }
 
+template <int N0, int N1, bool HALF>
+__device__ __forceinline__ void mid2_kernel_body(float2* __restrict__ Zt, const float4* __restrict__ spec,
+                                                 long long sbs4, int N2, long long ord0, int B, int C, int vol_local,
+                                                 int h) {
+  using M = M2<N0, N1, HALF>;
+  extern __shared__ __align__(16) unsigned char smem[];
+  pdl_release();
+  const Tabs<N0> t0 = tabs_at<N0>(smem);
+  Tabs<N1> t1;
+  if constexpr (N0 == N1) {
+    t1 = t0;
+  } else {
+    t1 = tabs_at<N1>(smem + Tabs<N0>::kBytes);
+  }
+  tabs_build<N0>(t0, g_tw512);
+  if constexpr (N0 != N1) tabs_build<N1>(t1, g_tw512);
+  const long long ord = ord0 + vol_local;
+  const int c = static_cast<int>(ord / B), b = static_cast<int>(ord % B);
+  const long long RPn = static_cast<long long>(N0) * N1 / 2;
+  const int kx = blockIdx.y;
+  const long long slab = 2LL * N1 * N0;                 // float4 per slab
+  const float4* sslab = spec + static_cast<long long>(b) * sbs4 + static_cast<long long>(c) * (N2 + 1) * slab +
+                        static_cast<long long>(kx) * slab;
+  __syncthreads();
+  pdl_wait();
+  mid2_task<N0, N1, HALF>(t0, t1, smem + M::kTabs, Zt + static_cast<long long>(vol_local) * 2 * N2 * RPn, sslab, N2,
+                          kx, h);
+}
+
 template <int N0, int N1>
 __global__ void __launch_bounds__(kTM, 2) k_mid2v2(float2* __restrict__ Zt, const float4* __restrict__ spec,
                                                 long long sbs4, int N2, long long ord0, int B, int C) {
-  k_mid2_body<N0, N1, false>(Zt, spec, sbs4, N2, ord0, B, C, blockIdx.x, 0);
+  mid2_kernel_body<N0, N1, false>(Zt, spec, sbs4, N2, ord0, B, C, blockIdx.x, 0);
 }
 
 template <int N0, int N1>
@@ -521,7 +599,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTM)
     k_mid2v2_pair(float2* __restrict__ Zt, const float4* __restrict__ spec, long long sbs4, int N2, long long ord0,
                   int B, int C) {
   const int h = static_cast<int>(cg::this_cluster().block_rank());
-  k_mid2_body<N0, N1, true>(Zt, spec, sbs4, N2, ord0, B, C, blockIdx.x / 2, h);
+  mid2_kernel_body<N0, N1, true>(Zt, spec, sbs4, N2, ord0, B, C, blockIdx.x / 2, h);
 }
 
 // --------------------------------------------------- spectrum layouts (v2)

@@ -60,9 +60,8 @@ static cudaError_t rowfwd_go(const ConvArgs& a, float2* zt, long long ord0, int 
   if (e != cudaSuccess) return e;
   constexpr int RPB = hnd2::RT<NL>::RPB;
   dim3 grid(np, (rp_total + RPB - 1) / RPB);
-  kern<<<grid, hnd2::kTM, sm, a.stream>>>(static_cast<const TT*>(a.k), static_cast<const TT*>(a.v), zt, ord0,
-                                          rp_total, pair_stride(a), a.B, a.C);
-  return cudaGetLastError();
+  return launch_pdl(true, kern, grid, dim3(hnd2::kTM), sm, a.stream, static_cast<const TT*>(a.k),
+                    static_cast<const TT*>(a.v), zt, ord0, rp_total, pair_stride(a), a.B, a.C);
 }
 
 template <int NL, class IO>
@@ -74,9 +73,10 @@ static cudaError_t rowinv_go(const ConvArgs& a, const float2* zt, long long ord0
   if (e != cudaSuccess) return e;
   constexpr int RPB = hnd2::RT<NL>::RPB;
   dim3 grid(np, (rp_total + RPB - 1) / RPB);
-  kern<<<grid, hnd2::kTM, sm, a.stream>>>(zt, static_cast<const TT*>(a.q), static_cast<TT*>(a.y), ord0, rp_total,
-                                          pair_stride(a), a.B, a.C);
-  return cudaGetLastError();
+  // Early launch after the 3D slab kernel measured slower (its CTAs crowd the
+  // slab kernel's tail); after the 2D column kernel it pays.
+  return launch_pdl(a.ndim == 2, kern, grid, dim3(hnd2::kTM), sm, a.stream, zt, static_cast<const TT*>(a.q),
+                    static_cast<TT*>(a.y), ord0, rp_total, pair_stride(a), a.B, a.C);
 }
 
 #define HND_ROWS_SWITCH(FN, IO, ...)                  \

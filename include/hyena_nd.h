@@ -26,6 +26,7 @@
  *     and returned synchronously.  A failed launch returns HYENA_ND_ERR_CUDA.
  *     Errors detected on the device are written to a status word held in the
  *     first 16 bytes of the workspace and read by hyena_nd_device_status.
+ *     The first 256 bytes of the workspace are its control area.
  *   * Activations q, k, v, y: contiguous [B, C, n_1, ..., n_d], last axis
  *     fastest, all of one dtype (fp32 or bf16; bf16 outputs are rounded to
  *     nearest even).  Arithmetic is fp32 throughout.
@@ -103,13 +104,14 @@ typedef struct {
 HYENA_ND_API size_t hyena_nd_spectrum_bytes(const hyena_nd_problem* p);
 
 /* Workspace bytes needed by every call below for problem `p` (a pure
- * function of the descriptor, at least 256 bytes; the first 16 bytes hold the
- * device status word).  0 if `p` is invalid or unsupported.  The same
+ * function of the descriptor, at least 256 bytes: the control area, then
+ * the intermediate spectra of the multi-pass tiers).  0 if `p` is invalid or unsupported.  The same
  * workspace may be reused by consecutive calls on one stream. */
 HYENA_ND_API size_t hyena_nd_workspace_bytes(const hyena_nd_problem* p);
 
-/* Clear the device status word (enqueues a 16-byte memset on `stream`).  Call
- * once on a fresh workspace before the first call that uses it. */
+/* Clear the workspace control area (enqueues a 256-byte memset on
+ * `stream`).  Call once on a fresh workspace before the first call that uses
+ * it; `ws_bytes` must be at least 256. */
 HYENA_ND_API hyena_nd_status hyena_nd_workspace_init(void* ws, size_t ws_bytes, void* cuda_stream);
 
 /* Call 1: evaluate the implicit filter on the offset grid, place it on the

@@ -69,6 +69,7 @@ SMALL = [
     ((8, 128), 1, 2, "f32"), ((128, 128), 1, 2, "f32"), ((128, 8), 2, 1, "bf16"),
     ((256, 64), 1, 2, "f32"), ((64, 256), 2, 1, "bf16"), ((256, 256), 1, 1, "f32"),
     ((8, 8, 8), 2, 2, "f32"), ((16, 8, 32), 1, 3, "f32"), ((32, 32, 32), 1, 2, "bf16"),
+    ((16, 16, 128), 2, 2, "f32"), ((64, 64, 8), 1, 2, "bf16"), ((8, 8, 256), 3, 2, "f32"),
     ((8, 16, 256), 1, 2, "f32"), ((128, 128, 16), 1, 2, "f32"), ((64, 128, 8), 2, 1, "f32"),
 ]
 
@@ -199,7 +200,9 @@ def test_single_volume_entry_point():
 
 
 def test_launch_counts_per_tier():
-    cases = [((64,), 4, 4, 1), ((64, 64), 2, 2, 1), ((256, 256), 2, 2, 3), ((16, 16, 16), 1, 2, 3)]
+    # 1D and 2D <= 64: one fused launch; larger grids: waves of 3 launches
+    cases = [((64,), 4, 4, 1), ((64, 64), 2, 2, 1), ((256, 256), 2, 2, 3), ((16, 16, 16), 1, 2, 3),
+             ((128, 128, 16), 1, 2, 3)]
     for dims, B, C, want in cases:
         wl = W.custom(dims, B, C)
         inp = W.make_inputs(wl)
@@ -207,23 +210,53 @@ def test_launch_counts_per_tier():
         assert H.last_launch_count() == want, dims
 
 
-def test_multi_wave_schedule():
-    """More pairs than one wave of the multi-pass tier holds (2D 256^2: 192
-    pairs per wave), so several waves run back to back (192, 192, 16)."""
+def _check_sampled(wl, inp, got, chans, tol, npts=12):
+    pts = sample_points(wl, npts, seed=2, channels=chans)
+    K = O.implicit_kernel(inp.filt, wl.dims, channels=chans)
+    Kfull = np.zeros((wl.C,) + K.shape[1:])
+    for j, c in enumerate(chans):
+        Kfull[c] = K[j]
+    want = O.conv_direct_at(inp.as_f64("q"), inp.as_f64("k"), inp.as_f64("v"), Kfull, wl.dims, pts)
+    gv = np.array([got[tuple(p)] for p in pts])
+    assert O.rel_l2(gv, want) <= tol
+
+
+def test_multi_wave_schedule_2d():
+    """More volumes (400 of 256^2) than one wave's workspace holds (192), so
+    three balanced waves of 134, 134 and 132 volumes run back to back."""
     dims = (256, 256)
     wl = W.custom(dims, 2, 200, io_dtype="bf16", seed=31)
     inp = W.make_inputs(wl)
     got, _ = run(inp)
     assert H.last_launch_count() == 9
-    chans = [0, 99, 199]
-    pts = sample_points(wl, 12, seed=2, channels=chans)
-    K = O.implicit_kernel(inp.filt, dims, channels=chans)
-    Kfull = np.zeros((wl.C,) + K.shape[1:])
-    for j, c in enumerate(chans):
-        Kfull[c] = K[j]
-    want = O.conv_direct_at(inp.as_f64("q"), inp.as_f64("k"), inp.as_f64("v"), Kfull, dims, pts)
-    gv = np.array([got[tuple(p)] for p in pts])
-    assert O.rel_l2(gv, want) <= 1e-2
+    _check_sampled(wl, inp, got, [0, 66, 67, 133, 199], 1e-2)
+
+
+def test_multi_wave_schedule_3d():
+    """100 volumes of 32x64x64 at 1 MiB of intermediate each run as two
+    balanced waves of 50."""
+    dims = (32, 64, 64)
+    wl = W.custom(dims, 1, 100, io_dtype="bf16", seed=37)
+    inp = W.make_inputs(wl)
+    got, _ = run(inp)
+    assert H.last_launch_count() == 6
+    _check_sampled(wl, inp, got, [0, 49, 50, 99], 1e-2)
+
+
+def test_repeated_calls_on_one_workspace():
+    """Back-to-back calls on one workspace give identical results and leave
+    the device status clear."""
+    dims = (32, 32, 64)
+    wl = W.custom(dims, 2, 5, seed=13)
+    inp = W.make_inputs(wl)
+    op = make_op(wl)
+    set_filter(op, inp.filt)
+    q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
+    outs = [to_host(op(q, k, v)) for _ in range(3)]
+    assert H.device_status(op.ws.data_ptr(), op._stream()) == H.OK
+    assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[0], outs[2])
+    want = O.reference_output(inp)
+    assert O.rel_l2(outs[0], want) < 1e-4
 
 
 # ------------------------------------------------------------ device status
