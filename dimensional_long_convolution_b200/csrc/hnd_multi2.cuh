@@ -41,23 +41,35 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 // 3D pairs neighbouring rows (ps = 1).
 __device__ __forceinline__ long long pair_row(long long rp, int ps) { return (rp / ps) * 2 * ps + (rp % ps); }
 
+// Row tile: for each of the 2 NL frequencies kk, RPB row pairs (float2).
+// Even and odd frequencies sit in two planes, row f = kk / 2 at f TS of its
+// plane.  A pencil's lanes hold consecutive f, so with the pitch TS = 16 / G
+// (mod 16) the lanes and pencils of a half-warp hit 16 distinct 8-byte bank
+// slots when they write or gather a frequency row; an even pitch keeps rows
+// 16-byte aligned for the workspace-side float4 accesses, and for the odd
+// pitch (G = 16) the odd plane is shifted by one slot so that the two planes'
+// rows read by one half-warp interleave.
 template <int NL>
 struct RT {
   static constexpr int G = P2<NL>::G, PPW = 32 / G;
   static constexpr int RPB = (kWM * PPW) * ((kWM * PPW) < 16 ? 2 : 1);   // row pairs per CTA
-  static constexpr int TS = RPB + 1;                                     // tile pitch (float2)
+  static constexpr int TS = RPB + ((16 / G - RPB) % 16 + 16) % 16;       // tile pitch (float2)
+  static constexpr int PL = NL * TS + TS % 2;                            // plane stride (float2)
   // The row tile and the FFT exchange buffers are never live together, so
   // they share one region.
-  static constexpr size_t kTile = sizeof(float2) * 2 * NL * TS;
+  static constexpr size_t kTile = sizeof(float2) * 2 * PL;
   static constexpr size_t kXb = 16ull * XB<NL>::kWarp * kWM;
   static constexpr size_t kBytes = Tabs<NL>::kBytes + (kTile > kXb ? kTile : kXb);
+  static __device__ __forceinline__ int row(int kk) { return (kk & 1) * PL + (kk >> 1) * TS; }
 };
 
 // Tile <-> workspace copies: rows of RPB row pairs (float2) per frequency kk,
 // moved as float4 pairs, every load of a thread issued before its stores.
-template <int NL, int RPB, int TS>
+template <int NL>
 __device__ __forceinline__ void tile_from_ws(float2* tile, const float2* __restrict__ zt, int rp_total, int rpb,
                                              int nrp) {
+  using R = RT<NL>;
+  constexpr int RPB = R::RPB;
   constexpr int PER = NL * RPB / kTM;                     // float4 per thread
   static_assert(PER * kTM == NL * RPB && RPB % 2 == 0, "tile split");
   float4 v[PER];
@@ -77,21 +89,35 @@ __device__ __forceinline__ void tile_from_ws(float2* tile, const float2* __restr
   for (int i = 0; i < PER; ++i) {
     const int e = 2 * (threadIdx.x + i * kTM);
     const int kk = e / RPB, rl = e % RPB;
-    tile[kk * TS + rl] = make_float2(v[i].x, v[i].y);
-    tile[kk * TS + rl + 1] = make_float2(v[i].z, v[i].w);
+    float2* t = tile + R::row(kk) + rl;
+    if constexpr (R::TS % 2 == 0) {
+      *reinterpret_cast<float4*>(t) = v[i];
+    } else {
+      t[0] = make_float2(v[i].x, v[i].y);
+      t[1] = make_float2(v[i].z, v[i].w);
+    }
   }
 }
 
-template <int NL, int RPB, int TS>
+template <int NL>
 __device__ __forceinline__ void tile_to_ws(const float2* tile, float2* __restrict__ zt, int rp_total, int rpb,
                                            int nrp) {
+  using R = RT<NL>;
+  constexpr int RPB = R::RPB;
   constexpr int PER = NL * RPB / kTM;
   static_assert(PER * kTM == NL * RPB && RPB % 2 == 0, "tile split");
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int e = 2 * (threadIdx.x + i * kTM);
     const int kk = e / RPB, rl = e % RPB;
-    const float2 a = tile[kk * TS + rl], b = tile[kk * TS + rl + 1];
+    const float2* t = tile + R::row(kk) + rl;
+    float2 a, b;
+    if constexpr (R::TS % 2 == 0) {
+      const float4 ab = *reinterpret_cast<const float4*>(t);
+      a = make_float2(ab.x, ab.y), b = make_float2(ab.z, ab.w);
+    } else {
+      a = t[0], b = t[1];
+    }
     float2* dst = zt + static_cast<long long>(kk) * rp_total + rpb + rl;
     if (rl + 1 < nrp) {
       __stcg(reinterpret_cast<float4*>(dst), make_float4(a.x, a.y, b.x, b.y));
@@ -109,7 +135,7 @@ __device__ __forceinline__ void rowfwd_task(const Tabs<NL> t, unsigned char* wor
                                             const T* __restrict__ v, float2* __restrict__ ztv, long long base,
                                             int rpb, int rp_total, int ps) {
   using R = RT<NL>;
-  constexpr int G = R::G, PPW = R::PPW, R1 = P2<NL>::R1, RPB = R::RPB, TS = R::TS;
+  constexpr int G = R::G, PPW = R::PPW, R1 = P2<NL>::R1, RPB = R::RPB;
   float2* tile = reinterpret_cast<float2*>(work);
   float4* xb = reinterpret_cast<float4*>(work);     // shares the tile region
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -144,15 +170,15 @@ __device__ __forceinline__ void rowfwd_task(const Tabs<NL> t, unsigned char* wor
 #pragma unroll
       for (int s = 0; s < R1; ++s) {
         const int kk = 2 * spec_idx<NL>(g, s);
-        tile[kk * TS + rl_] = make_float2(xx[s].re.x, xx[s].im.x);
-        tile[(kk + 1) * TS + rl_] = make_float2(xx[s].re.y, xx[s].im.y);
+        tile[R::row(kk) + rl_] = make_float2(xx[s].re.x, xx[s].im.x);
+        tile[R::row(kk + 1) + rl_] = make_float2(xx[s].re.y, xx[s].im.y);
       }
     };
     if constexpr (ROUNDS > 1) put(keep, warp * PPW + pen);
     put(x, rl);
   }
   task_sync();
-  tile_to_ws<NL, RPB, TS>(tile, ztv, rp_total, rpb, nrp);
+  tile_to_ws<NL>(tile, ztv, rp_total, rpb, nrp);
 }
 
 template <int NL, class T>
@@ -178,12 +204,12 @@ __device__ __forceinline__ void rowinv_task(const Tabs<NL> t, unsigned char* wor
                                             const T* __restrict__ q, T* __restrict__ y, long long base, int rpb,
                                             int rp_total, int ps) {
   using R = RT<NL>;
-  constexpr int G = R::G, PPW = R::PPW, R1 = P2<NL>::R1, RPB = R::RPB, TS = R::TS;
+  constexpr int G = R::G, PPW = R::PPW, R1 = P2<NL>::R1, RPB = R::RPB;
   float2* tile = reinterpret_cast<float2*>(work);
   float4* xb = reinterpret_cast<float4*>(work);     // shares the tile region
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nrp = min(RPB, rp_total - rpb);
-  tile_from_ws<NL, RPB, TS>(tile, ztv, rp_total, rpb, nrp);
+  tile_from_ws<NL>(tile, ztv, rp_total, rpb, nrp);
   task_sync();
   const int pen = lane / G, g = lane % G;
   float4* buf = xb + warp * XB<NL>::kWarp + pen * XB<NL>::kPen;
@@ -198,7 +224,7 @@ __device__ __forceinline__ void rowinv_task(const Tabs<NL> t, unsigned char* wor
 #pragma unroll
     for (int s = 0; s < R1; ++s) {
       const int kk = 2 * spec_idx<NL>(g, s);
-      const float2 e = tile[kk * TS + rl], d = tile[(kk + 1) * TS + rl];
+      const float2 e = tile[R::row(kk) + rl], d = tile[R::row(kk + 1) + rl];
       xin[round][s] = {make_float2(e.x, d.x), make_float2(e.y, d.y)};
     }
   }
