@@ -376,6 +376,46 @@ def run_ours(args):
         del sj
         torch.cuda.empty_cache()
 
+    # call 1 (filter spectrum) timed on its own: device-resident weights, the
+    # MLP on the offset grid, the padded transform and the packing
+    f = setup.inp0.filt
+    wdev = [torch.from_numpy(a).to(device) for a in (f.W1, f.b1, f.W2, f.b2, f.alpha)]
+    spec_tmp = setup.op.spectrum.clone()
+    for _ in range(2):
+        setup.op.set_filter(*wdev, f.decay_scale, f.num_freqs)
+    fa, fb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    NF = 5
+    fa.record(stream)
+    for _ in range(NF):
+        setup.op.set_filter(*wdev, f.decay_scale, f.num_freqs)
+    fb.record(stream)
+    fb.synchronize()
+    setup.op.spectrum.copy_(spec_tmp)
+    call1_ms = fa.elapsed_time(fb) / NF
+    filter_call = {"ms_per_call": call1_ms, "conv_steps_per_call": call1_ms / (ms / K),
+                   "note": "not in the metric: the spectrum is computed once per filter update"}
+
+    # backward (dq, dk, dv for a loss gradient dy) on the same grid, timed
+    # apart from the metric; algorithmic bytes: q, k, v, dy read, dq, dk, dv
+    # written, the spectrum read twice (forward and adjoint convolutions)
+    dy0 = torch.empty_like(y0).copy_(setup.sets[-1][0])
+    for _ in range(3):
+        setup.op.backward(q0, k0, v0, dy0, spectrum=spec0)
+    bwd_launches = setup.H.last_launch_count()
+    ba, bb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    NB = max(5, min(200, K // 3))
+    ba.record(stream)
+    for _ in range(NB):
+        setup.op.backward(q0, k0, v0, dy0, spectrum=spec0)
+    bb.record(stream)
+    bb.synchronize()
+    bwd_ms = ba.elapsed_time(bb) / NB
+    bwd_bytes = 7 * units * elt + 2 * (ub - 4 * units * elt)
+    backward = {"ms_per_step": bwd_ms, "value": units / (bwd_ms / 1e3), "unit": UNIT,
+                "launches_per_step": bwd_launches, "gbs": bwd_bytes / (bwd_ms / 1e3) / 1e9,
+                "hbm_frac": bwd_bytes / (bwd_ms / 1e3) / 1e9 / peak,
+                "note": "three convolutions (dq; dk and dv each recompute the adjoint)"}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl, setup.inp0, args.cpu_seconds)
@@ -399,6 +439,8 @@ def run_ours(args):
         "gpu_launches": int(launches * K),
         "clocks": clocks.summary(),
         "e2e": e2e,
+        "filter_call": filter_call,
+        "backward": backward,
         "also": also,
     }
     if cpu is not None:

@@ -113,6 +113,32 @@ bool overlaps(const void* a, const void* b, size_t bytes) {
 
 hyena_nd_status cuda_status(cudaError_t e) { return e == cudaSuccess ? HYENA_ND_OK : HYENA_ND_ERR_CUDA; }
 
+// One gated convolution y = q . (K * (k . v)) (or with the conjugate
+// spectrum) on the plan's tier; adds the kernel launches to *launches.
+cudaError_t run_conv(const Plan& pl, const hnd::ConvArgs& a, void* ws, int* launches) {
+  cudaError_t e = cudaSuccess;
+  if (pl.tier == kRows1D) {
+    e = hnd::launch_rows1d(a);
+    *launches += 1;
+  } else if (pl.tier == kFused2D) {
+    e = pl.bf16 ? hnd::launch_fused2d_bf16(a) : hnd::launch_fused2d_f32(a);
+    *launches += 1;
+  } else {
+    float2* zt = reinterpret_cast<float2*>(static_cast<char*>(ws) + kStatusBytes);
+    const long long pairs = pl.B * pl.C;
+    const int nl = pl.n[pl.ndim - 1];
+    const int rp_total = static_cast<int>(pl.L / nl / 2);
+    for (long long ord0 = 0; ord0 < pairs && e == cudaSuccess; ord0 += pl.wave) {
+      const int np = static_cast<int>(pairs - ord0 < pl.wave ? pairs - ord0 : pl.wave);
+      e = hnd::launch_rowfwd(a, nl, zt, ord0, np, rp_total);
+      if (e == cudaSuccess) e = pl.tier == kMulti2D ? hnd::launch_mid1(a, zt, ord0, np) : hnd::launch_mid2(a, zt, ord0, np);
+      if (e == cudaSuccess) e = hnd::launch_rowinv(a, nl, zt, ord0, np, rp_total);
+      *launches += 3;
+    }
+  }
+  return e;
+}
+
 }  // namespace
 
 extern "C" {
@@ -166,27 +192,7 @@ hyena_nd_status hyena_nd_fftconv_batched(const hyena_nd_problem* p, const void* 
   a.status = static_cast<int*>(ws);
 
   int launches = 0;
-  cudaError_t e = cudaSuccess;
-  if (pl.tier == kRows1D) {
-    e = hnd::launch_rows1d(a);
-    launches = 1;
-  } else if (pl.tier == kFused2D) {
-    e = pl.bf16 ? hnd::launch_fused2d_bf16(a) : hnd::launch_fused2d_f32(a);
-    launches = 1;
-  } else {
-    float2* zt = reinterpret_cast<float2*>(static_cast<char*>(ws) + kStatusBytes);
-    const long long pairs = pl.B * pl.C;
-    const int nl = pl.n[pl.ndim - 1];
-    const int rp_total = static_cast<int>(pl.L / nl / 2);
-    for (long long ord0 = 0; ord0 < pairs && e == cudaSuccess; ord0 += pl.wave) {
-      const int np = static_cast<int>(pairs - ord0 < pl.wave ? pairs - ord0 : pl.wave);
-      e = hnd::launch_rowfwd(a, nl, zt, ord0, np, rp_total);
-      if (e == cudaSuccess) e = pl.tier == kMulti2D ? hnd::launch_mid1(a, zt, ord0, np) : hnd::launch_mid2(a, zt, ord0, np);
-      if (e == cudaSuccess) e = hnd::launch_rowinv(a, nl, zt, ord0, np, rp_total);
-      launches += 3;
-    }
-  }
-  if (e != cudaSuccess) return HYENA_ND_ERR_CUDA;
+  if (run_conv(pl, a, ws, &launches) != cudaSuccess) return HYENA_ND_ERR_CUDA;
   g_last_launches = launches;
   return HYENA_ND_OK;
 }
@@ -196,6 +202,58 @@ hyena_nd_status hyena_nd_fftconv(const hyena_nd_problem* p, const void* q, const
   if (!p) return HYENA_ND_ERR_INVALID_ARG;
   if (p->B != 1 || p->C != 1) return HYENA_ND_ERR_INVALID_ARG;
   return hyena_nd_fftconv_batched(p, q, k, v, spectrum_c, 0, y, ws, ws_bytes, cuda_stream);
+}
+
+hyena_nd_status hyena_nd_fftconv_backward(const hyena_nd_problem* p, const void* q, const void* k, const void* v,
+                                          const void* spectrum, int64_t spectrum_batch_stride, const void* dy,
+                                          void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
+                                          void* cuda_stream) {
+  Plan pl;
+  hyena_nd_status st = make_plan(p, &pl);
+  if (st != HYENA_ND_OK) return st;
+  if (!q || !k || !v || !spectrum || !dy || !dq || !dk || !dv || !ws) return HYENA_ND_ERR_INVALID_ARG;
+  const void* ptrs[9] = {q, k, v, spectrum, dy, dq, dk, dv, ws};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return HYENA_ND_ERR_MISALIGNED;
+  if (spectrum_batch_stride < 0) return HYENA_ND_ERR_INVALID_ARG;
+  if (spectrum_batch_stride % 16 != 0) return HYENA_ND_ERR_MISALIGNED;
+  if (ws_bytes < pl.ws_total) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
+  const size_t act_bytes = static_cast<size_t>(pl.B * pl.C * pl.L) * (pl.bf16 ? 2 : 4);
+  const void* outs[3] = {dq, dk, dv};
+  const void* ins[4] = {q, k, v, dy};
+  for (int i = 0; i < 3; ++i) {
+    for (const void* in : ins)
+      if (overlaps(outs[i], in, act_bytes)) return HYENA_ND_ERR_INVALID_ARG;
+    for (int j = i + 1; j < 3; ++j)
+      if (overlaps(outs[i], outs[j], act_bytes)) return HYENA_ND_ERR_INVALID_ARG;
+  }
+  hnd::ConvArgs a;
+  a.spec = spectrum;
+  a.sbs = spectrum_batch_stride / 8;
+  a.B = static_cast<int>(pl.B);
+  a.C = static_cast<int>(pl.C);
+  a.bf16 = pl.bf16;
+  a.ndim = pl.ndim;
+  for (int i = 0; i < 3; ++i) a.n[i] = pl.n[i];
+  a.stream = static_cast<cudaStream_t>(cuda_stream);
+  a.status = static_cast<int*>(ws);
+  int launches = 0;
+  // dq = dy . (K * (k . v)): the forward with dy as the output gate
+  a.q = dy, a.k = k, a.v = v, a.y = dq, a.sconj = 1.f;
+  cudaError_t e = run_conv(pl, a, ws, &launches);
+  // du = K (adjoint) applied to q . dy: the conjugate spectrum; dk = v . du, dv = k . du
+  a.k = q, a.v = dy, a.sconj = -1.f;
+  if (e == cudaSuccess) {
+    a.q = v, a.y = dk;
+    e = run_conv(pl, a, ws, &launches);
+  }
+  if (e == cudaSuccess) {
+    a.q = k, a.y = dv;
+    e = run_conv(pl, a, ws, &launches);
+  }
+  if (e != cudaSuccess) return HYENA_ND_ERR_CUDA;
+  g_last_launches = launches;
+  return HYENA_ND_OK;
 }
 
 hyena_nd_status hyena_nd_filter_spectrum(const hyena_nd_problem* p, const hyena_nd_filter* f, void* spectrum,

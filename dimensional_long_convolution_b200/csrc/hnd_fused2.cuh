@@ -189,7 +189,7 @@ __device__ __forceinline__ void rows_inv(const T* qst, const float4* Zb, T* yp, 
 // diverge.
 template <int N0, int N1, class T>
 __device__ __forceinline__ void columns(float4* Zb4, float4* xb, const float4* __restrict__ sp, Tabs<N0> t0,
-                                        int warp, int lane) {
+                                        int warp, int lane, float sgn) {
   using L = F3<N0, N1, T>;
   constexpr int G = P2<N0>::G, PPW = 32 / G;
   constexpr int SLOTS = kW3 * PPW;
@@ -209,7 +209,10 @@ __device__ __forceinline__ void columns(float4* Zb4, float4* xb, const float4* _
     if (act) {
       const float4* su = sp + (cu == 0 ? 0LL : static_cast<long long>(cu + 1) * N0);
 #pragma unroll
-      for (int s = 0; s < 8; ++s) S[s] = __ldg(su + s * G + g);
+      for (int s = 0; s < 8; ++s) {
+        S[s] = __ldg(su + s * G + g);
+        S[s].z *= sgn, S[s].w *= sgn;     // sgn = -1: conjugate spectrum (adjoint)
+      }
     }
     float2 z[8];
 #pragma unroll
@@ -236,7 +239,10 @@ __device__ __forceinline__ void columns(float4* Zb4, float4* xb, const float4* _
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
         float4 Bc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (cu == 0) Bc = __ldg(sp + N0 + s * G + g);
+        if (cu == 0) {
+          Bc = __ldg(sp + N0 + s * G + g);
+          Bc.z *= sgn, Bc.w *= sgn;
+        }
         const cp a = cmulp(x[s], make_float2(S[s].x, S[s].y), make_float2(S[s].z, S[s].w));
         const cp xc = {xp[s].re, make_float2(-xp[s].im.x, -xp[s].im.y)};
         const cp bb = cmulp(xc, make_float2(Bc.x, Bc.y), make_float2(Bc.z, Bc.w));
@@ -275,7 +281,8 @@ __device__ __forceinline__ void named_arrive(int id, int nthreads) {
 template <int N0, int N1, class T>
 __global__ void __launch_bounds__(kT3, 1)
     k_fused2d_v3(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-                 const float4* __restrict__ spec, long long sbs4, T* __restrict__ y, int B, int C, int* status) {
+                 const float4* __restrict__ spec, long long sbs4, T* __restrict__ y, int B, int C, int* status,
+                 float sgn) {
   using L = F3<N0, N1, T>;
   extern __shared__ __align__(16) unsigned char smem[];
   uint64_t* bar_kv = reinterpret_cast<uint64_t*>(smem);
@@ -373,7 +380,7 @@ __global__ void __launch_bounds__(kT3, 1)
     // phase B: columns of `vol`.  Group 0 needs every column before its
     // inverse rows; group 1 only signals and goes on to the next volume's
     // forward rows (they touch the other Zb buffer and the staging planes).
-    columns<N0, N1, T>(Zc, xw, sp, t0, warp, lane);
+    columns<N0, N1, T>(Zc, xw, sp, t0, warp, lane, sgn);
     if (grp == 0) named_sync(1, kT3);
     else named_arrive(1, kT3);
 

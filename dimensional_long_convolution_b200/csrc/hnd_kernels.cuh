@@ -247,7 +247,7 @@ __global__ void __launch_bounds__(kThreads) k_rows1d(const typename IO::T* __res
                                                      const typename IO::T* __restrict__ k,
                                                      const typename IO::T* __restrict__ v,
                                                      const float2* __restrict__ spec, long long sbs,
-                                                     typename IO::T* __restrict__ y, int B, int C) {
+                                                     typename IO::T* __restrict__ y, int B, int C, float sgn) {
   using TT = typename IO::T;
   extern __shared__ float4 smem4[];
   float2* T = reinterpret_cast<float2*>(smem4);
@@ -296,6 +296,7 @@ __global__ void __launch_bounds__(kThreads) k_rows1d(const typename IO::T* __res
           Sa = c_conj(__ldg(sa + 2 * N - kk));
           Sb = c_conj(__ldg(sb + 2 * N - kk));
         }
+        Sa.y *= sgn, Sb.y *= sgn;     // sgn = -1: conjugate spectrum (adjoint)
         x[p][s] = pack_pos(c_mul(xa, Sa), c_mul(xbv, Sb));
       }
     }

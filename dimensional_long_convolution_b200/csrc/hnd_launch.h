@@ -22,6 +22,7 @@ struct ConvArgs {
   int ndim;
   cudaStream_t stream;
   int* status = nullptr;  // device status word (may be null)
+  float sconj = 1.f;      // -1: multiply by the conjugate spectrum (the adjoint convolution)
 };
 
 // 2D problems whose axes are both <= 64 run on the persistent fused kernel;

@@ -290,7 +290,7 @@ struct M1 {
 // partner term is multiplied by zero).
 template <int N0, bool GEN>
 __device__ __forceinline__ void mid1_unit(const Tabs<N0> t, float4* buf, float2* __restrict__ zt,
-                                          const float4* __restrict__ sp, int N1, int cu, int g) {
+                                          const float4* __restrict__ sp, int N1, int cu, int g, float sgn) {
   constexpr int G = P2<N0>::G, R1 = P2<N0>::R1, RP = N0 / 2, HS = R1 / 2;
   const bool act = cu < N1;
   const int kx = act ? cu : 1, kxm = cu == 0 ? N1 : 2 * N1 - kx;
@@ -319,8 +319,9 @@ __device__ __forceinline__ void mid1_unit(const Tabs<N0> t, float4* buf, float2*
     fetch_partner<N0>(x, xp, g, buf, 0, 0u);
 #pragma unroll
     for (int s = 0; s < R1; ++s) {
-      const float4 S = act ? __ldg(su + s * G + g) : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float4 Bc = (cu == 0) ? __ldg(sp + N0 + s * G + g) : make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 S = act ? __ldg(su + s * G + g) : make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 Bc = (cu == 0) ? __ldg(sp + N0 + s * G + g) : make_float4(0.f, 0.f, 0.f, 0.f);
+      S.z *= sgn, S.w *= sgn, Bc.z *= sgn, Bc.w *= sgn;     // sgn = -1: conjugate spectrum (adjoint)
       const cp a = cmulp(x[s], make_float2(S.x, S.y), make_float2(S.z, S.w));
       const cp xc = {xp[s].re, make_float2(-xp[s].im.x, -xp[s].im.y)};
       const cp bb = cmulp(xc, make_float2(Bc.x, Bc.y), make_float2(Bc.z, Bc.w));
@@ -331,7 +332,7 @@ __device__ __forceinline__ void mid1_unit(const Tabs<N0> t, float4* buf, float2*
 #pragma unroll
       for (int s = 0; s < R1; ++s) {
         const float4 S = __ldg(su + s * G + g);
-        x[s] = cmulp(x[s], make_float2(S.x, S.y), make_float2(S.z, S.w));
+        x[s] = cmulp(x[s], make_float2(S.x, S.y), make_float2(sgn * S.z, sgn * S.w));
       }
     }
   }
@@ -357,15 +358,15 @@ __device__ __forceinline__ void mid1_unit(const Tabs<N0> t, float4* buf, float2*
 // do not weigh on the common path.
 template <int N0>
 __device__ __noinline__ void mid1_unit_gen(const Tabs<N0> t, float4* buf, float2* __restrict__ zt,
-                                           const float4* __restrict__ sp, int N1, int cu, int g) {
-  mid1_unit<N0, true>(t, buf, zt, sp, N1, cu, g);
+                                           const float4* __restrict__ sp, int N1, int cu, int g, float sgn) {
+  mid1_unit<N0, true>(t, buf, zt, sp, N1, cu, g, sgn);
 }
 
 // One task: UPB column units starting at u0 of one volume; `sp` is the
 // channel's spectrum for this sample.
 template <int N0>
 __device__ __forceinline__ void mid1_task(const Tabs<N0> t, unsigned char* work, float2* __restrict__ zt,
-                                          const float4* __restrict__ sp, int N1, int u0) {
+                                          const float4* __restrict__ sp, int N1, int u0, float sgn) {
   using M = M1<N0>;
   constexpr int G = M::G, PPW = M::PPW;
   float4* xb = reinterpret_cast<float4*>(work);
@@ -373,13 +374,13 @@ __device__ __forceinline__ void mid1_task(const Tabs<N0> t, unsigned char* work,
   const int pen = lane / G, g = lane % G;
   float4* buf = xb + warp * XB<N0>::kWarp + pen * XB<N0>::kPen;
   const int cu = u0 + warp * PPW + pen;
-  if (u0 == 0 && warp == 0) mid1_unit_gen<N0>(t, buf, zt, sp, N1, cu, g);
-  else mid1_unit<N0, false>(t, buf, zt, sp, N1, cu, g);
+  if (u0 == 0 && warp == 0) mid1_unit_gen<N0>(t, buf, zt, sp, N1, cu, g, sgn);
+  else mid1_unit<N0, false>(t, buf, zt, sp, N1, cu, g, sgn);
 }
 
 template <int N0>
 __global__ void __launch_bounds__(kTM, 2) k_mid1v2(float2* __restrict__ Zt, const float4* __restrict__ spec,
-                                                long long sbs4, int N1, long long ord0, int B, int C) {
+                                                long long sbs4, int N1, long long ord0, int B, int C, float sgn) {
   extern __shared__ __align__(16) unsigned char smem[];
   pdl_release();
   const Tabs<N0> t = tabs_at<N0>(smem);
@@ -390,7 +391,7 @@ __global__ void __launch_bounds__(kTM, 2) k_mid1v2(float2* __restrict__ Zt, cons
   __syncthreads();
   pdl_wait();
   mid1_task<N0>(t, smem + Tabs<N0>::kBytes, Zt + static_cast<long long>(blockIdx.x) * 2 * N1 * (N0 / 2), sp, N1,
-                blockIdx.y * M1<N0>::UPB);
+                blockIdx.y * M1<N0>::UPB, sgn);
 }
 
 // ---------------------------------------------------------------- 3D slabs
@@ -460,7 +461,7 @@ __device__ __forceinline__ void slab_rows_out(float2* __restrict__ zt, long long
 template <int N0, int N1, bool HALF>
 __device__ __forceinline__ void mid2_task(const Tabs<N0> t0, const Tabs<N1> t1, unsigned char* work,
                                           float2* __restrict__ zt, const float4* __restrict__ sslab, int N2, int kx,
-                                          int h) {
+                                          int h, float sgn) {
   using M = M2<N0, N1, HALF>;
   constexpr int FS = M::FS, NKY = M::NKY;
   constexpr int G0 = P2<N0>::G, R0 = P2<N0>::R1, G1 = P2<N1>::G, R1 = P2<N1>::R1;
@@ -528,7 +529,7 @@ __device__ __forceinline__ void mid2_task(const Tabs<N0> t0, const Tabs<N1> t1, 
 #pragma unroll
         for (int s = 0; s < R0; ++s) {
           const float4 Sv = (R0 == 8) ? S[s % NPF] : __ldg(su + s * G0 + g);
-          x[s] = cmulp(x[s], make_float2(Sv.x, Sv.y), make_float2(Sv.z, Sv.w));
+          x[s] = cmulp(x[s], make_float2(Sv.x, Sv.y), make_float2(sgn * Sv.z, sgn * Sv.w));
         }
       }
       float2 o[R0];
@@ -588,7 +589,7 @@ __device__ __forceinline__ void mid2_task(const Tabs<N0> t0, const Tabs<N1> t1, 
 template <int N0, int N1, bool HALF>
 __device__ __forceinline__ void mid2_kernel_body(float2* __restrict__ Zt, const float4* __restrict__ spec,
                                                  long long sbs4, int N2, long long ord0, int B, int C, int vol_local,
-                                                 int h) {
+                                                 int h, float sgn) {
   using M = M2<N0, N1, HALF>;
   extern __shared__ __align__(16) unsigned char smem[];
   pdl_release();
@@ -611,21 +612,21 @@ __device__ __forceinline__ void mid2_kernel_body(float2* __restrict__ Zt, const 
   __syncthreads();
   pdl_wait();
   mid2_task<N0, N1, HALF>(t0, t1, smem + M::kTabs, Zt + static_cast<long long>(vol_local) * 2 * N2 * RPn, sslab, N2,
-                          kx, h);
+                          kx, h, sgn);
 }
 
 template <int N0, int N1>
 __global__ void __launch_bounds__(kTM, 2) k_mid2v2(float2* __restrict__ Zt, const float4* __restrict__ spec,
-                                                long long sbs4, int N2, long long ord0, int B, int C) {
-  mid2_kernel_body<N0, N1, false>(Zt, spec, sbs4, N2, ord0, B, C, blockIdx.x, 0);
+                                                long long sbs4, int N2, long long ord0, int B, int C, float sgn) {
+  mid2_kernel_body<N0, N1, false>(Zt, spec, sbs4, N2, ord0, B, C, blockIdx.x, 0, sgn);
 }
 
 template <int N0, int N1>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTM)
     k_mid2v2_pair(float2* __restrict__ Zt, const float4* __restrict__ spec, long long sbs4, int N2, long long ord0,
-                  int B, int C) {
+                  int B, int C, float sgn) {
   const int h = static_cast<int>(cg::this_cluster().block_rank());
-  mid2_kernel_body<N0, N1, true>(Zt, spec, sbs4, N2, ord0, B, C, blockIdx.x / 2, h);
+  mid2_kernel_body<N0, N1, true>(Zt, spec, sbs4, N2, ord0, B, C, blockIdx.x / 2, h, sgn);
 }
 
 // --------------------------------------------------- spectrum layouts (v2)

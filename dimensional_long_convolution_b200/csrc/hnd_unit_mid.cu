@@ -16,7 +16,7 @@ static cudaError_t mid1_go(const ConvArgs& a, float2* zt, long long ord0, int np
   const int n1 = a.n[1];
   dim3 grid(np, (n1 + UPB - 1) / UPB);
   return launch_pdl(true, kern, grid, dim3(hnd2::kTM), sm, a.stream, zt, static_cast<const float4*>(a.spec),
-                    a.sbs / 2, n1, ord0, a.B, a.C);
+                    a.sbs / 2, n1, ord0, a.B, a.C, a.sconj);
 }
 
 cudaError_t launch_mid1(const ConvArgs& a, float2* zt, long long ord0, int np) {
@@ -41,7 +41,7 @@ static cudaError_t mid2_go(const ConvArgs& a, float2* zt, long long ord0, int np
     if (e != cudaSuccess) return e;
     dim3 grid(np, n2 + 1);
     return launch_pdl(true, kern, grid, dim3(hnd2::kTM), sm, a.stream, zt, static_cast<const float4*>(a.spec),
-                      a.sbs / 2, n2, ord0, a.B, a.C);
+                      a.sbs / 2, n2, ord0, a.B, a.C, a.sconj);
   } else {
     auto kern = hnd2::k_mid2v2_pair<N0, N1>;
     const size_t sm = hnd2::M2<N0, N1, true>::kBytes;
@@ -49,7 +49,7 @@ static cudaError_t mid2_go(const ConvArgs& a, float2* zt, long long ord0, int np
     if (e != cudaSuccess) return e;
     dim3 grid(2 * np, n2 + 1);
     return launch_pdl(true, kern, grid, dim3(hnd2::kTM), sm, a.stream, zt, static_cast<const float4*>(a.spec),
-                      a.sbs / 2, n2, ord0, a.B, a.C);
+                      a.sbs / 2, n2, ord0, a.B, a.C, a.sconj);
   }
 }
 

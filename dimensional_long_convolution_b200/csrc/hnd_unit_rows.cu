@@ -19,7 +19,7 @@ static cudaError_t rows1d_go(const ConvArgs& a) {
   if (blocks > 148LL * 64) blocks = 148LL * 64;
   kern<<<static_cast<unsigned>(blocks), kThreads, sm, a.stream>>>(
       static_cast<const TT*>(a.q), static_cast<const TT*>(a.k), static_cast<const TT*>(a.v),
-      static_cast<const float2*>(a.spec), a.sbs, static_cast<TT*>(a.y), a.B, a.C);
+      static_cast<const float2*>(a.spec), a.sbs, static_cast<TT*>(a.y), a.B, a.C, a.sconj);
   return cudaGetLastError();
 }
 

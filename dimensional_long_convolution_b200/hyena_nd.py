@@ -37,6 +37,7 @@ EXPORTED = (
     "hyena_nd_filter_spectrum",
     "hyena_nd_fftconv",
     "hyena_nd_fftconv_batched",
+    "hyena_nd_fftconv_backward",
     "hyena_nd_spectrum_export",
     "hyena_nd_spectrum_import",
     "hyena_nd_device_status",
@@ -100,6 +101,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "hyena_nd_filter_spectrum": (ctypes.c_int, [P, ctypes.POINTER(Filter), vp, vp, sz, vp]),
         "hyena_nd_fftconv": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
         "hyena_nd_fftconv_batched": (ctypes.c_int, [P, vp, vp, vp, vp, i64, vp, vp, sz, vp]),
+        "hyena_nd_fftconv_backward": (ctypes.c_int, [P, vp, vp, vp, vp, i64, vp, vp, vp, vp, vp, sz, vp]),
         "hyena_nd_spectrum_export": (ctypes.c_int, [P, vp, vp, vp]),
         "hyena_nd_spectrum_import": (ctypes.c_int, [P, vp, vp, vp]),
         "hyena_nd_device_status": (ctypes.c_int, [vp, vp]),
@@ -175,6 +177,12 @@ def device_status(ws: int, stream: int = 0) -> int:
 
 def debug_bounded_wait(ws: int, ws_bytes: int, limit_us: int, stream: int = 0) -> int:
     return load().hyena_nd_debug_bounded_wait(ws, ws_bytes, int(limit_us), stream)
+
+
+def fftconv_backward(p: Problem, q: int, k: int, v: int, spectrum: int, spectrum_batch_stride: int, dy: int,
+                     dq: int, dk: int, dv: int, ws: int, ws_bytes: int, stream: int = 0) -> int:
+    return load().hyena_nd_fftconv_backward(ctypes.byref(p), q, k, v, spectrum, int(spectrum_batch_stride), dy,
+                                            dq, dk, dv, ws, ws_bytes, stream)
 
 
 def status_string(code: int) -> str:
@@ -257,6 +265,18 @@ class HyenaND:
                               int(spectrum_batch_stride), y.data_ptr(), self.ws.data_ptr(), self.ws_bytes,
                               self._stream()), "fftconv_batched")
         return y
+
+    def backward(self, q, k, v, dy, spectrum=None, spectrum_batch_stride: int = 0):
+        """(dq, dk, dv) for the loss gradient dy of __call__'s output."""
+        for t in (q, k, v, dy):
+            if t.dtype != self.tdtype or not t.is_contiguous() or t.device != self.device:
+                raise ValueError("q, k, v, dy must be contiguous %s tensors on %s" % (self.tdtype, self.device))
+        dq, dk, dv = (self.torch.empty_like(q) for _ in range(3))
+        spec = self.spectrum if spectrum is None else spectrum
+        check(fftconv_backward(self.p, q.data_ptr(), k.data_ptr(), v.data_ptr(), spec.data_ptr(),
+                               int(spectrum_batch_stride), dy.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                               dv.data_ptr(), self.ws.data_ptr(), self.ws_bytes, self._stream()), "fftconv_backward")
+        return dq, dk, dv
 
     def status(self) -> int:
         return device_status(self.ws.data_ptr(), self._stream())

@@ -145,6 +145,30 @@ HYENA_ND_API hyena_nd_status hyena_nd_fftconv_batched(const hyena_nd_problem* p,
                                          int64_t spectrum_batch_stride, void* y, void* ws,
                                          size_t ws_bytes, void* cuda_stream);
 
+/* Backward of call 3: the gradients of a loss L with respect to q, k and v,
+ * given dy = dL/dy (all [B, C, n...] in the problem's dtype).  With
+ * u = k (.) v and w = crop_n(K_c * u) as in the forward,
+ *   dq = dy (.) w
+ *   du[j] = sum_{i in [0,n)^d} q[i] dy[i] K_c[i - j]      (the adjoint convolution)
+ *   dk = v (.) du,   dv = k (.) du.
+ * The adjoint is the same padded FFT convolution with the conjugate spectrum:
+ * for a real K_c on the 2n grid, the transform of K_c[-t] is conj(S).  The
+ * forward intermediates are recomputed, not stored (blog "Native
+ * multi-dimensional subquadratic operators via input-dependent long
+ * convolutions", sections "勾配フローと数値安定性" (gradient flow and
+ * numerical stability: recompute the forward FFT in the backward) and
+ * "具体的な実装パターン(PyTorch)" (an autograd function that keeps only
+ * the inputs and the kernel parameters)).  Arithmetic is fp32 as in the forward.
+ * Runs three convolutions (9 launches per wave on the multi-pass tiers).
+ * q, k, v, dy: read.  dq, dk, dv: written; none may overlap another output or
+ * an input.  `spectrum`, `spectrum_batch_stride`, `ws`: as in call 3.  The
+ * gradient with respect to the filter is not computed here. */
+HYENA_ND_API hyena_nd_status hyena_nd_fftconv_backward(const hyena_nd_problem* p, const void* q, const void* k,
+                                          const void* v, const void* spectrum,
+                                          int64_t spectrum_batch_stride, const void* dy, void* dq,
+                                          void* dk, void* dv, void* ws, size_t ws_bytes,
+                                          void* cuda_stream);
+
 /* Same operation as hyena_nd_fftconv_batched, for callers that cannot
  * allocate device memory and so have no workspace to pass: for instance a
  * plugin whose interface carries only input and output buffers, or an

@@ -229,6 +229,72 @@ def conv_circular(q: np.ndarray, k: np.ndarray, v: np.ndarray, Kper: np.ndarray,
     return q * x.real
 
 
+# ---------------------------------------------------------------- backward
+# Gradients of L with respect to q, k, v for dy = dL/dy, from the definition
+# above: y = q * w with w[i] = sum_j u[j] K[i - j] and u = k v, so
+#   dq = dy * w,  du[j] = sum_i q[i] dy[i] K[i - j],  dk = v du,  dv = k du.
+# (Blog "Native multi-dimensional subquadratic operators via input-dependent
+# long convolutions", sections on gradient flow and the PyTorch autograd
+# pattern: the backward recomputes the forward FFT convolution.)
+def corr_direct(z: np.ndarray, K: np.ndarray, dims: Sequence[int]) -> np.ndarray:
+    """The adjoint of the cropped linear convolution, written out:
+    du[b,c,j] = sum_{i in [0,n)^d} z[b,c,i] K_c[i - j], j in [0,n)^d.
+    O(L^2); tiny grids only.  K: [C, 2n-1, ...] with index t + (n - 1)."""
+    d = len(dims)
+    B, C = z.shape[:2]
+    zf = z.reshape(B, C, -1)
+    du = np.zeros((B, C) + tuple(dims), dtype=np.float64)
+    igrid = np.stack(np.meshgrid(*[np.arange(n) for n in dims], indexing="ij"), axis=-1).reshape(-1, d)
+    Kf = K.reshape(C, -1)
+    strides = np.array([int(np.prod([2 * m - 1 for m in dims[a + 1:]])) for a in range(d)], dtype=np.int64)
+    for j in itertools.product(*[range(n) for n in dims]):
+        off = (igrid - np.array(j)[None, :]) + (np.array(dims) - 1)[None, :]
+        du[(slice(None), slice(None)) + j] = np.einsum("bci,ci->bc", zf, Kf[:, off @ strides])
+    return du
+
+
+def corr_direct_at(z: np.ndarray, K: np.ndarray, dims: Sequence[int], points: np.ndarray) -> np.ndarray:
+    """corr_direct at chosen outputs only.  points: [M, 2 + d] rows
+    (b, c, j_1..j_d).  O(L) per point."""
+    d = len(dims)
+    igrid = np.stack(np.meshgrid(*[np.arange(n) for n in dims], indexing="ij"), axis=-1).reshape(-1, d)
+    strides = np.array([int(np.prod([2 * m - 1 for m in dims[a + 1:]])) for a in range(d)], dtype=np.int64)
+    out = np.empty(points.shape[0], dtype=np.float64)
+    for r, p in enumerate(points):
+        b, c = int(p[0]), int(p[1])
+        j = np.asarray(p[2:], dtype=np.int64)
+        off = (igrid - j[None, :]) + (np.array(dims) - 1)[None, :]
+        out[r] = float(np.dot(z[b, c].reshape(-1), K[c].reshape(-1)[off @ strides]))
+    return out
+
+
+def corr_dft(z: np.ndarray, S_full: np.ndarray, dims: Sequence[int]) -> np.ndarray:
+    """The adjoint through zero-padded DFTs: on the 2n grid the transform of
+    K[-t] is conj(S) for a real K, so the adjoint is conv_dft's steps with the
+    conjugate spectrum (and no output gate)."""
+    x = z.astype(np.complex128)
+    for a, n in enumerate(dims):
+        x = _apply_along(x, dft_matrix(2 * n)[:, :n], 2 + a)
+    x = x * np.conj(S_full)[None]
+    for a, n in enumerate(dims):
+        x = _apply_along(x, np.conj(dft_matrix(2 * n))[:n, :], 2 + a)
+    return x.real
+
+
+def backward_dft(q, k, v, dy, S_full, dims) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """(dq, dk, dv) through the DFT route (float64)."""
+    w = conv_dft(np.ones_like(q), k, v, S_full, dims)
+    du = corr_dft(q * dy, S_full, dims)
+    return dy * w, v * du, k * du
+
+
+def backward_direct(q, k, v, dy, K, dims) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """(dq, dk, dv) by direct sums (float64, tiny grids)."""
+    w = conv_direct(np.ones_like(q), k, v, K, dims)
+    du = corr_direct(q * dy, K, dims)
+    return dy * w, v * du, k * du
+
+
 # -------------------------------------------------------------- conveniences
 def reference_output(inputs, S_full=None, K=None) -> np.ndarray:
     """y for a seeded workload through O2 (float64)."""

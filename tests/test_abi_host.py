@@ -20,7 +20,7 @@ def _declared():
 def test_library_exports_every_declared_symbol():
     lib = H.load()
     names = _declared()
-    assert len(names) == len(H.EXPORTED) == 13
+    assert len(names) == len(H.EXPORTED) == 14
     assert set(names) == set(H.EXPORTED)
     for n in names:
         assert getattr(lib, n) is not None
@@ -102,6 +102,30 @@ def test_invalid_arguments_are_rejected_before_launch():
     assert _call(bad, q, k, v, s, y, ws, wsb) == H.ERR_UNSUPPORTED
     circ = H.problem((64, 64), 2, 3, circular=1)
     assert _call(circ, q, k, v, s, y, ws, wsb) == H.ERR_UNSUPPORTED
+
+
+def test_backward_arguments_are_rejected_before_launch():
+    p = H.problem((64, 64), 2, 3)
+    q, k, v, s, dy, ws = _ptrs()
+    dq, dk, dv = (A + i * STEP for i in (6, 7, 8))
+    wsb = H.workspace_bytes(p)
+
+    def bwd(*args, sbs=0, wsb_=wsb, prob=p):
+        a = dict(q=q, k=k, v=v, s=s, dy=dy, dq=dq, dk=dk, dv=dv, ws=ws)
+        a.update(args[0] if args else {})
+        return H.fftconv_backward(prob, a["q"], a["k"], a["v"], a["s"], sbs, a["dy"], a["dq"], a["dk"], a["dv"],
+                                  a["ws"], wsb_, 0)
+
+    assert bwd({"dy": 0}) == H.ERR_INVALID_ARG
+    assert bwd({"dv": 0}) == H.ERR_INVALID_ARG
+    assert bwd({"dq": dq + 8}) == H.ERR_MISALIGNED
+    assert bwd({"dk": q}) == H.ERR_INVALID_ARG            # output aliases an input
+    assert bwd({"dv": dy + 64}) == H.ERR_INVALID_ARG      # output overlaps dy
+    assert bwd({"dk": dq}) == H.ERR_INVALID_ARG           # two outputs alias
+    assert bwd(wsb_=wsb - 16) == H.ERR_WORKSPACE_TOO_SMALL
+    assert bwd(sbs=-16) == H.ERR_INVALID_ARG
+    assert bwd(sbs=8) == H.ERR_MISALIGNED
+    assert bwd(prob=H.problem((48, 64), 2, 3)) == H.ERR_UNSUPPORTED
 
 
 def test_single_volume_call_needs_b_and_c_of_one():

@@ -310,3 +310,88 @@ def test_rel_l2_compares_complex_values_as_complex():
     a = np.array([1.0 + 1.0j, 2.0])
     b = np.array([1.0 + 0.0j, 2.0])
     assert abs(O.rel_l2(a, b) - 1.0 / np.sqrt(5.0)) < 1e-15
+
+
+# ------------------------------------------------------------------ backward
+# dq = dy w, du[j] = sum_i q[i] dy[i] K[i - j], dk = v du, dv = k du (the
+# gradients of L = sum dy y; blog sections on gradient flow and the autograd
+# pattern).  Pinned by brute force, by the adjoint identity against the
+# forward oracle, by exact finite differences of L, and by numpy's 1D convolve.
+@pytest.mark.parametrize("dims", [(8,), (5,), (6, 5), (4, 7), (3, 4, 5)])
+def test_adjoint_dft_equals_direct_sum(dims):
+    q, k, v, K = _rand_problem(dims, seed=11)
+    z = q * v
+    S = O.spectrum_full(K, dims)
+    assert O.rel_l2(O.corr_dft(z, S, dims), O.corr_direct(z, K, dims)) < 1e-12
+
+
+def test_adjoint_direct_by_explicit_loops():
+    dims = (3, 4)
+    rng = np.random.default_rng(5)
+    z = rng.standard_normal((1, 2) + dims)
+    K = rng.standard_normal((2, 5, 7))
+    du = O.corr_direct(z, K, dims)
+    for c in range(2):
+        for j0 in range(3):
+            for j1 in range(4):
+                s = sum(z[0, c, i0, i1] * K[c, i0 - j0 + 2, i1 - j1 + 3] for i0 in range(3) for i1 in range(4))
+                assert abs(du[0, c, j0, j1] - s) < 1e-12
+
+
+@pytest.mark.parametrize("dims", [(7,), (5, 6), (3, 4, 4)])
+def test_adjoint_identity_against_the_forward(dims):
+    """<conv(u), z> = <u, adj(z)> for the forward oracle's conv_direct."""
+    rng = np.random.default_rng(7)
+    shape = (2, 3) + dims
+    u, z = rng.standard_normal(shape), rng.standard_normal(shape)
+    K = rng.standard_normal((3,) + tuple(2 * n - 1 for n in dims))
+    lhs = np.sum(O.conv_direct(np.ones(shape), u, np.ones(shape), K, dims) * z)
+    rhs = np.sum(u * O.corr_direct(z, K, dims))
+    assert abs(lhs - rhs) <= 1e-11 * max(1.0, abs(lhs))
+
+
+@pytest.mark.parametrize("dims", [(8,), (6, 5), (3, 4, 5)])
+def test_backward_matches_finite_differences(dims):
+    """L = sum dy * y is linear in each of q, k, v, so the central difference
+    along any direction is exact up to rounding."""
+    q, k, v, K = _rand_problem(dims, seed=21)
+    rng = np.random.default_rng(22)
+    dy = rng.standard_normal(q.shape)
+    S = O.spectrum_full(K, dims)
+    dq, dk, dv = O.backward_dft(q, k, v, dy, S, dims)
+
+    def L(q_, k_, v_):
+        return float(np.sum(dy * O.conv_direct(q_, k_, v_, K, dims)))
+
+    for name, g in (("q", dq), ("k", dk), ("v", dv)):
+        dirn = rng.standard_normal(q.shape)
+        eps = 0.5
+        args_p = {"q_": q, "k_": k, "v_": v}
+        args_m = dict(args_p)
+        args_p[name + "_"] = args_p[name + "_"] + eps * dirn
+        args_m[name + "_"] = args_m[name + "_"] - eps * dirn
+        fd = (L(**args_p) - L(**args_m)) / (2 * eps)
+        an = float(np.sum(g * dirn))
+        assert abs(fd - an) <= 1e-10 * max(1.0, abs(an)), name
+
+
+@pytest.mark.parametrize("n", [5, 8, 13])
+def test_1d_adjoint_matches_numpy_convolve(n):
+    """d = 1: du[j] = sum_i z[i] K[i - j] = convolve(reverse(z), K)[2(n-1) - j]."""
+    rng = np.random.default_rng(n)
+    z = rng.standard_normal(n)
+    Kf = rng.standard_normal(2 * n - 1)
+    du = O.corr_direct(z[None, None], Kf[None], (n,))[0, 0]
+    want = np.convolve(z[::-1], Kf)[n - 1: 2 * n - 1][::-1]
+    assert np.max(np.abs(du - want)) < 1e-12
+
+
+def test_backward_direct_at_points_matches_full():
+    dims = (5, 6)
+    q, k, v, K = _rand_problem(dims, seed=31)
+    z = q * v
+    full = O.corr_direct(z, K, dims)
+    pts = np.array([[1, 2, 0, 0], [0, 1, 4, 5], [1, 0, 2, 3]])
+    got = O.corr_direct_at(z, K, dims, pts)
+    want = np.array([full[tuple(p)] for p in pts])
+    assert np.max(np.abs(got - want)) < 1e-12
