@@ -397,7 +397,7 @@ def run_ours(args):
 
     # backward (dq, dk, dv for a loss gradient dy) on the same grid, timed
     # apart from the metric; algorithmic bytes: q, k, v, dy read, dq, dk, dv
-    # written, the spectrum read twice (forward and adjoint convolutions)
+    # written, the spectrum read twice (the dq and the adjoint convolutions)
     dy0 = torch.empty_like(y0).copy_(setup.sets[-1][0])
     for _ in range(3):
         setup.op.backward(q0, k0, v0, dy0, spectrum=spec0)
@@ -414,7 +414,7 @@ def run_ours(args):
     backward = {"ms_per_step": bwd_ms, "value": units / (bwd_ms / 1e3), "unit": UNIT,
                 "launches_per_step": bwd_launches, "gbs": bwd_bytes / (bwd_ms / 1e3) / 1e9,
                 "hbm_frac": bwd_bytes / (bwd_ms / 1e3) / 1e9 / peak,
-                "note": "three convolutions (dq; dk and dv each recompute the adjoint)"}
+                "note": "two convolutions: dq, then the adjoint writing dk and dv"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

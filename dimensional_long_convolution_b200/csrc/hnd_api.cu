@@ -241,16 +241,12 @@ hyena_nd_status hyena_nd_fftconv_backward(const hyena_nd_problem* p, const void*
   // dq = dy . (K * (k . v)): the forward with dy as the output gate
   a.q = dy, a.k = k, a.v = v, a.y = dq, a.sconj = 1.f;
   cudaError_t e = run_conv(pl, a, ws, &launches);
-  // du = K (adjoint) applied to q . dy: the conjugate spectrum; dk = v . du, dv = k . du
+  // du = K (adjoint) applied to q . dy: the conjugate spectrum; one convolution
+  // writes both gated outputs dk = v . du and dv = k . du
   a.k = q, a.v = dy, a.sconj = -1.f;
-  if (e == cudaSuccess) {
-    a.q = v, a.y = dk;
-    e = run_conv(pl, a, ws, &launches);
-  }
-  if (e == cudaSuccess) {
-    a.q = k, a.y = dv;
-    e = run_conv(pl, a, ws, &launches);
-  }
+  a.q = v, a.y = dk;
+  a.g2 = k, a.y2 = dv;
+  if (e == cudaSuccess) e = run_conv(pl, a, ws, &launches);
   if (e != cudaSuccess) return HYENA_ND_ERR_CUDA;
   g_last_launches = launches;
   return HYENA_ND_OK;

@@ -146,9 +146,9 @@ __device__ __forceinline__ void rows_fwd(const T* kst, const T* vst, float4* Zb,
 }
 
 // Inverse rows, crop, output gate and store of one volume (8 warps).
-template <int N0, int N1, class T>
+template <int N0, int N1, class T, bool DUAL>
 __device__ __forceinline__ void rows_inv(const T* qst, const float4* Zb, T* yp, float4* xb, Tabs<N1> t1, int gw,
-                                         int lane) {
+                                         int lane, const T* __restrict__ g2p, T* __restrict__ y2p) {
   using L = F3<N0, N1, T>;
   constexpr int G = P2<N1>::G, PPW = 32 / G;
   const int pen = lane / G, g = lane % G;
@@ -174,6 +174,15 @@ __device__ __forceinline__ void rows_inv(const T* qst, const float4* Zb, T* yp, 
         const float qb = Act<T>::ld_s(qst + (rp + N0 / 2) * L::PITCH + j);
         Act<T>::st_g(yp + static_cast<long long>(rp) * N1 + j, o[s].x * qa);
         Act<T>::st_g(yp + static_cast<long long>(rp + N0 / 2) * N1 + j, o[s].y * qb);
+      }
+      if constexpr (DUAL) {      // second gated output of the same convolution
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+          const long long ja = static_cast<long long>(rp) * N1 + g + s * G;
+          const long long jb = ja + static_cast<long long>(N0 / 2) * N1;
+          Act<T>::st_g(y2p + ja, o[s].x * Act<T>::ld_g(g2p + ja));
+          Act<T>::st_g(y2p + jb, o[s].y * Act<T>::ld_g(g2p + jb));
+        }
       }
     }
   }
@@ -278,11 +287,11 @@ __device__ __forceinline__ void named_arrive(int id, int nthreads) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-template <int N0, int N1, class T>
+template <int N0, int N1, class T, bool DUAL>
 __global__ void __launch_bounds__(kT3, 1)
     k_fused2d_v3(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                  const float4* __restrict__ spec, long long sbs4, T* __restrict__ y, int B, int C, int* status,
-                 float sgn) {
+                 float sgn, const T* __restrict__ g2, T* __restrict__ y2) {
   using L = F3<N0, N1, T>;
   extern __shared__ __align__(16) unsigned char smem[];
   uint64_t* bar_kv = reinterpret_cast<uint64_t*>(smem);
@@ -388,7 +397,10 @@ __global__ void __launch_bounds__(kT3, 1)
     ok = true;
     if (grp == 0) {
       ok = mbar_wait_bounded(bar_q, ph_q, status);
-      if (ok) rows_inv<N0, N1, T>(qst, Zc, y + (static_cast<long long>(b) * C + c) * Lv, xw, t1, gw, lane);
+      if (ok) {
+        const long long vo = (static_cast<long long>(b) * C + c) * Lv;
+        rows_inv<N0, N1, T, DUAL>(qst, Zc, y + vo, xw, t1, gw, lane, g2 + vo, y2 + vo);
+      }
     } else if (next < nvol) {
       ok = mbar_wait_bounded(bar_kv, ph_kv, status);
       if (ok) rows_fwd<N0, N1, T>(kst, vst, Zn, xw, t1, gw, lane);

@@ -242,12 +242,14 @@ __global__ void __launch_bounds__(kThreads) k_fused2d(const typename IO::T* __re
 // ===================================================================== 1D fused
 // Rows are independent: each warp owns row pairs, transforms, multiplies by the
 // channel spectrum (natural order, kx in [0, N]) and transforms back.
-template <int N, class IO>
+template <int N, class IO, bool DUAL>
 __global__ void __launch_bounds__(kThreads) k_rows1d(const typename IO::T* __restrict__ q,
                                                      const typename IO::T* __restrict__ k,
                                                      const typename IO::T* __restrict__ v,
                                                      const float2* __restrict__ spec, long long sbs,
-                                                     typename IO::T* __restrict__ y, int B, int C, float sgn) {
+                                                     typename IO::T* __restrict__ y, int B, int C, float sgn,
+                                                     const typename IO::T* __restrict__ g2,
+                                                     typename IO::T* __restrict__ y2) {
   using TT = typename IO::T;
   extern __shared__ float4 smem4[];
   float2* T = reinterpret_cast<float2*>(smem4);
@@ -306,6 +308,10 @@ __global__ void __launch_bounds__(kThreads) k_rows1d(const typename IO::T* __res
       const long long j = g + s * G;
       if (act_a) IO::st(y + ra * N + j, x[0][s].x * IO::ld(q + ra * N + j));
       if (act_b) IO::st(y + rb * N + j, x[0][s].y * IO::ld(q + rb * N + j));
+      if constexpr (DUAL) {       // second gated output of the same convolution
+        if (act_a) IO::st(y2 + ra * N + j, x[0][s].x * IO::ld(g2 + ra * N + j));
+        if (act_b) IO::st(y2 + rb * N + j, x[0][s].y * IO::ld(g2 + rb * N + j));
+      }
     }
   }
 }

@@ -23,6 +23,8 @@ struct ConvArgs {
   cudaStream_t stream;
   int* status = nullptr;  // device status word (may be null)
   float sconj = 1.f;      // -1: multiply by the conjugate spectrum (the adjoint convolution)
+  const void* g2 = nullptr;  // optional second output y2 = g2 . conv (same layout as q and y)
+  void* y2 = nullptr;
 };
 
 // 2D problems whose axes are both <= 64 run on the persistent fused kernel;

@@ -202,7 +202,8 @@ __global__ void __launch_bounds__(kTM, 2) k_rowfwd2(const T* __restrict__ k, con
 template <int NL, class T>
 __device__ __forceinline__ void rowinv_task(const Tabs<NL> t, unsigned char* work, const float2* __restrict__ ztv,
                                             const T* __restrict__ q, T* __restrict__ y, long long base, int rpb,
-                                            int rp_total, int ps) {
+                                            int rp_total, int ps, const T* __restrict__ g2 = nullptr,
+                                            T* __restrict__ y2 = nullptr) {
   using R = RT<NL>;
   constexpr int G = R::G, PPW = R::PPW, R1 = P2<NL>::R1, RPB = R::RPB;
   float2* tile = reinterpret_cast<float2*>(work);
@@ -253,6 +254,14 @@ __device__ __forceinline__ void rowinv_task(const Tabs<NL> t, unsigned char* wor
         Act<T>::st_g(y + base + ra + j, o[s].x * qa[s]);
         Act<T>::st_g(y + base + rb + j, o[s].y * qb[s]);
       }
+      if (y2) {       // second gated output of the same convolution
+#pragma unroll
+        for (int s = 0; s < R1; ++s) {
+          const long long j = g + s * G;
+          Act<T>::st_g(y2 + base + ra + j, o[s].x * Act<T>::ld_g(g2 + base + ra + j));
+          Act<T>::st_g(y2 + base + rb + j, o[s].y * Act<T>::ld_g(g2 + base + rb + j));
+        }
+      }
     }
   }
 }
@@ -260,7 +269,7 @@ __device__ __forceinline__ void rowinv_task(const Tabs<NL> t, unsigned char* wor
 template <int NL, class T>
 __global__ void __launch_bounds__(kTM, 2) k_rowinv2(const float2* __restrict__ Zt, const T* __restrict__ q,
                                                  T* __restrict__ y, long long ord0, int rp_total, int ps, int B,
-                                                 int C) {
+                                                 int C, const T* __restrict__ g2, T* __restrict__ y2) {
   extern __shared__ __align__(16) unsigned char smem[];
   pdl_release();
   const Tabs<NL> t = tabs_at<NL>(smem);
@@ -271,7 +280,7 @@ __global__ void __launch_bounds__(kTM, 2) k_rowinv2(const float2* __restrict__ Z
   __syncthreads();
   pdl_wait();
   rowinv_task<NL, T>(t, smem + Tabs<NL>::kBytes, Zt + static_cast<long long>(blockIdx.x) * L, q, y,
-                     (static_cast<long long>(b) * C + c) * L, blockIdx.y * RT<NL>::RPB, rp_total, ps);
+                     (static_cast<long long>(b) * C + c) * L, blockIdx.y * RT<NL>::RPB, rp_total, ps, g2, y2);
 }
 
 // ---------------------------------------------------------- 2D column units

@@ -6,10 +6,10 @@
 
 namespace hnd {
 
-template <int N, class IO>
-static cudaError_t rows1d_go(const ConvArgs& a) {
+template <int N, class IO, bool DUAL>
+static cudaError_t rows1d_launch(const ConvArgs& a) {
   using TT = typename IO::T;
-  auto kern = k_rows1d<N, IO>;
+  auto kern = k_rows1d<N, IO, DUAL>;
   const size_t sm = kMidSmemBase;
   cudaError_t e = ensure_smem(kern, sm);
   if (e != cudaSuccess) return e;
@@ -19,8 +19,14 @@ static cudaError_t rows1d_go(const ConvArgs& a) {
   if (blocks > 148LL * 64) blocks = 148LL * 64;
   kern<<<static_cast<unsigned>(blocks), kThreads, sm, a.stream>>>(
       static_cast<const TT*>(a.q), static_cast<const TT*>(a.k), static_cast<const TT*>(a.v),
-      static_cast<const float2*>(a.spec), a.sbs, static_cast<TT*>(a.y), a.B, a.C, a.sconj);
+      static_cast<const float2*>(a.spec), a.sbs, static_cast<TT*>(a.y), a.B, a.C, a.sconj,
+      static_cast<const TT*>(a.g2), static_cast<TT*>(a.y2));
   return cudaGetLastError();
+}
+
+template <int N, class IO>
+static cudaError_t rows1d_go(const ConvArgs& a) {
+  return a.y2 ? rows1d_launch<N, IO, true>(a) : rows1d_launch<N, IO, false>(a);
 }
 
 template <class IO>
@@ -76,7 +82,8 @@ static cudaError_t rowinv_go(const ConvArgs& a, const float2* zt, long long ord0
   // Early launch after the 3D slab kernel measured slower (its CTAs crowd the
   // slab kernel's tail); after the 2D column kernel it pays.
   return launch_pdl(a.ndim == 2, kern, grid, dim3(hnd2::kTM), sm, a.stream, zt, static_cast<const TT*>(a.q),
-                    static_cast<TT*>(a.y), ord0, rp_total, pair_stride(a), a.B, a.C);
+                    static_cast<TT*>(a.y), ord0, rp_total, pair_stride(a), a.B, a.C,
+                    static_cast<const TT*>(a.g2), static_cast<TT*>(a.y2));
 }
 
 #define HND_ROWS_SWITCH(FN, IO, ...)                  \

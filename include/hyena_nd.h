@@ -159,7 +159,8 @@ HYENA_ND_API hyena_nd_status hyena_nd_fftconv_batched(const hyena_nd_problem* p,
  * numerical stability: recompute the forward FFT in the backward) and
  * "具体的な実装パターン(PyTorch)" (an autograd function that keeps only
  * the inputs and the kernel parameters)).  Arithmetic is fp32 as in the forward.
- * Runs three convolutions (9 launches per wave on the multi-pass tiers).
+ * Runs two convolutions: dq, then the adjoint, whose last stage writes both
+ * dk and dv (6 launches per wave on the multi-pass tiers).
  * q, k, v, dy: read.  dq, dk, dv: written; none may overlap another output or
  * an input.  `spectrum`, `spectrum_batch_stride`, `ws`: as in call 3.  The
  * gradient with respect to the filter is not computed here. */
