@@ -22,7 +22,7 @@ thread_local int g_last_launches = 0;
 constexpr size_t kStatusBytes = 256;                  // status word + padding
 constexpr size_t kWaveBudget = size_t(96) << 20;      // multi-pass intermediate per wave (measured best of 24/48/96 MiB)
 constexpr size_t kFilterBudget = size_t(64) << 20;    // filter grid per channel chunk
-constexpr int kFilterMaxChunk = 16;
+constexpr int kFilterMaxChunk = 64;
 
 enum Tier { kRows1D = 0, kFused2D = 1, kMulti2D = 2, kMulti3D = 3 };
 

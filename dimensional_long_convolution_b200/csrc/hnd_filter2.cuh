@@ -1,0 +1,174 @@
+// hnd_filter2.cuh -- the implicit filter on the offset grid (call 1) as tiled
+// fp32 products: per CTA, 128 offsets; their Fourier features and hidden
+// layer are computed once into shared memory, then the output layer runs as a
+// register-tiled product over tiles of 32 channels of the chunk.
+// (HyenaND pages: gist.science summary of arXiv 2607.19378, "Methodologie",
+// kernel parameterisation -- a coordinate MLP with sine activation on
+// continuous offsets, times a window; blog "Native multi-dimensional
+// subquadratic operators via input-dependent long convolutions", section on
+// the neural parameterisation.)
+//   phi(t) = [sin(pi m t_a / n_a), cos(pi m t_a / n_a)]  m = 1..M, axis-major
+//   h = sin(W1 phi + b1),  K_c(t) = (W2 h + b2)_c exp(-alpha_c |t|_2 / s)
+// written wrap-placed (offset t at slot t mod P on each axis) into a complex
+// grid [nc][P^d] whose other slots the caller has zeroed.
+#pragma once
+
+#include <cuda_runtime.h>
+
+namespace hnd2 {
+
+constexpr int kFT = 256;     // threads per CTA
+constexpr int kFO = 128;     // offsets per CTA
+constexpr int kFC = 32;      // channels per output tile
+
+struct FilterMlpArgs {
+  const float *W1, *b1, *W2, *b2, *alpha;
+  int num_freqs, hidden, fin;    // fin = 2 num_freqs ndim
+  float decay_scale;
+  int ndim;
+  int n[3];
+  int c0, nc;                    // channel chunk [c0, c0 + nc)
+  float2* grid;                  // [nc][P^d]
+};
+
+// Shared layout (floats), HP = hidden rounded up to a multiple of 32:
+//   phi[fin][kFO] | w1[fin][HP] | hid[HP][kFO] | w2[HP][kFC] | b1[HP] | rad[kFO] | slot[kFO] (int)
+template <int HP>
+struct FilterSmem {
+  static size_t bytes(int fin) {
+    return sizeof(float) * (static_cast<size_t>(fin) * kFO + static_cast<size_t>(fin) * HP +
+                            static_cast<size_t>(HP) * kFO + static_cast<size_t>(HP) * kFC + HP + kFO) +
+           sizeof(int) * kFO;
+  }
+};
+
+template <int HP>
+__global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
+  static_assert(HP % 32 == 0 && HP <= 128, "hidden tile");
+  constexpr int HG = HP / 8;                 // hidden outputs per thread in the hidden layer
+  extern __shared__ __align__(16) float fsm[];
+  const int fin = a.fin;
+  float* phi = fsm;                          // [fin][kFO]
+  float* w1 = phi + fin * kFO;               // [fin][HP]
+  float* hid = w1 + fin * HP;                // [HP][kFO]
+  float* w2 = hid + HP * kFO;                // [HP][kFC]
+  float* b1 = w2 + HP * kFC;                 // [HP]
+  float* rad = b1 + HP;                      // [kFO]
+  int* slot = reinterpret_cast<int*>(rad + kFO);
+  const int tid = threadIdx.x;
+  // axes as scalars (an unused axis has extent 1 and offset 0)
+  const int n0 = a.n[0], n1 = a.ndim > 1 ? a.n[1] : 1, n2 = a.ndim > 2 ? a.n[2] : 1;
+  const int E0 = 2 * n0 - 1, E1 = 2 * n1 - 1, E2 = 2 * n2 - 1;
+  const int P0 = 2 * n0, P1 = a.ndim > 1 ? 2 * n1 : 1, P2 = a.ndim > 2 ? 2 * n2 : 1;
+  const long long noff = static_cast<long long>(E0) * E1 * E2;
+  const long long gsz = static_cast<long long>(P0) * P1 * P2;
+  const long long e0 = static_cast<long long>(blockIdx.x) * kFO;
+  // offset t of tile entry o (the last axis fastest; past the end: the last offset)
+  auto offset_of = [&](int o, int& t0, int& t1, int& t2) {
+    long long r = e0 + o < noff ? e0 + o : noff - 1;
+    const int i2 = static_cast<int>(r % E2);
+    r /= E2;
+    const int i1 = static_cast<int>(r % E1);
+    const int i0 = static_cast<int>(r / E1);
+    t0 = i0 - (n0 - 1), t1 = i1 - (n1 - 1), t2 = i2 - (n2 - 1);
+  };
+
+  // first layer weights (zero-padded to HP hidden units: sin(0) = 0 and the
+  // padded output weights are zero, so the padding contributes nothing)
+  for (int i = tid; i < fin * HP; i += kFT) {
+    const int f = i / HP, h = i % HP;
+    w1[i] = h < a.hidden ? __ldg(a.W1 + static_cast<long long>(h) * fin + f) : 0.f;
+  }
+  for (int h = tid; h < HP; h += kFT) b1[h] = h < a.hidden ? __ldg(a.b1 + h) : 0.f;
+  // offsets of this tile: radius and slot (offset t at t mod P per axis)
+  for (int o = tid; o < kFO; o += kFT) {
+    int t0, t1, t2;
+    offset_of(o, t0, t1, t2);
+    const float f0 = static_cast<float>(t0), f1 = static_cast<float>(t1), f2 = static_cast<float>(t2);
+    rad[o] = sqrtf(f0 * f0 + f1 * f1 + f2 * f2);
+    const int s0 = (t0 + P0) % P0, s1 = (t1 + P1) % P1, s2 = (t2 + P2) % P2;
+    slot[o] = (s0 * P1 + s1) * P2 + s2;
+  }
+  // Fourier features, phi[(ax M + m - 1) 2 + {0: sin, 1: cos}][o]
+  const int M = a.num_freqs;
+  for (int i = tid; i < kFO * a.ndim * M; i += kFT) {
+    const int o = i % kFO, q = i / kFO, m = q % M + 1, ax = q / M;
+    int t0, t1, t2;
+    offset_of(o, t0, t1, t2);
+    const int tax = ax == 0 ? t0 : (ax == 1 ? t1 : t2);
+    const int nax = ax == 0 ? n0 : (ax == 1 ? n1 : n2);
+    float sv, cv;
+    sincospif(static_cast<float>(m) * (static_cast<float>(tax) / static_cast<float>(nax)), &sv, &cv);
+    phi[(2 * (ax * M + m - 1)) * kFO + o] = sv;
+    phi[(2 * (ax * M + m - 1) + 1) * kFO + o] = cv;
+  }
+  __syncthreads();
+
+  // hidden layer: thread (og, hg) computes offsets 4 og .. 4 og + 3 x units hg HG ..
+  const int og = tid % 32, grp = tid / 32;
+  {
+    float acc[4][HG];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < HG; ++j) acc[i][j] = b1[grp * HG + j];
+    for (int f = 0; f < fin; ++f) {
+      const float4 p = *reinterpret_cast<const float4*>(phi + f * kFO + 4 * og);
+      const float pv[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+      for (int j4 = 0; j4 < HG / 4; ++j4) {
+        const float4 w = *reinterpret_cast<const float4*>(w1 + f * HP + grp * HG + 4 * j4);
+        const float wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) acc[i][4 * j4 + jj] = fmaf(wv[jj], pv[i], acc[i][4 * j4 + jj]);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < HG; ++j)
+      *reinterpret_cast<float4*>(hid + (grp * HG + j) * kFO + 4 * og) =
+          make_float4(sinf(acc[0][j]), sinf(acc[1][j]), sinf(acc[2][j]), sinf(acc[3][j]));
+  }
+
+  // output layer over channel tiles: thread (og, cg) -> offsets 4 og.., channels 4 cg..
+  for (int ct = 0; ct < a.nc; ct += kFC) {
+    __syncthreads();          // hid complete / previous tile's w2 no longer read
+    for (int i = tid; i < HP * kFC; i += kFT) {
+      const int h = i / kFC, cc = i % kFC;
+      const int c = ct + cc;
+      w2[i] = (h < a.hidden && c < a.nc) ? __ldg(a.W2 + static_cast<long long>(a.c0 + c) * a.hidden + h) : 0.f;
+    }
+    __syncthreads();
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 4
+    for (int h = 0; h < HP; ++h) {
+      const float4 hv = *reinterpret_cast<const float4*>(hid + h * kFO + 4 * og);
+      const float4 wv = *reinterpret_cast<const float4*>(w2 + h * kFC + 4 * grp);
+      const float hh[4] = {hv.x, hv.y, hv.z, hv.w}, ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(hh[i], ww[j], acc[i][j]);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = ct + 4 * grp + j;
+      if (c >= a.nc) continue;
+      const float bb = __ldg(a.b2 + a.c0 + c), al = __ldg(a.alpha + a.c0 + c);
+      float2* gch = a.grid + static_cast<long long>(c) * gsz;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int o = 4 * og + i;
+        if (e0 + o < noff)
+          gch[slot[o]] = make_float2((acc[i][j] + bb) * expf(-al * rad[o] / a.decay_scale), 0.f);
+      }
+    }
+  }
+}
+
+}  // namespace hnd2

@@ -856,63 +856,6 @@ static __global__ void k_spec_export(const float2* __restrict__ lib, float2* __r
 // activation times a window), written wrap-placed into a complex grid P^d
 // per channel of the chunk [c0, c0 + nc).  The grid must be zeroed first
 // (slot n_a of each axis stays 0).
-struct FilterArgs {
-  const float *W1, *b1, *W2, *b2, *alpha;
-  int num_freqs, hidden, fin;
-  float decay_scale;
-};
-
-constexpr int kMaxChunkOut = 16;
-
-static __global__ void __launch_bounds__(128) k_filter_mlp(FilterArgs fa, SpecDims d, int c0, int nc, float2* __restrict__ grid) {
-  int P[3] = {1, 1, 1}, E[3] = {1, 1, 1};
-  for (int a = 0; a < d.ndim; ++a) {
-    P[a] = 2 * d.n[a];
-    E[a] = 2 * d.n[a] - 1;
-  }
-  const long long noff = static_cast<long long>(E[0]) * E[1] * E[2];
-  long long gsz = 1;
-  for (int a = 0; a < d.ndim; ++a) gsz *= P[a];
-  for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < noff;
-       e += static_cast<long long>(gridDim.x) * blockDim.x) {
-    int t[3] = {0, 0, 0};
-    long long r = e;
-    for (int a = d.ndim - 1; a >= 0; --a) {
-      t[a] = static_cast<int>(r % E[a]) - (d.n[a] - 1);
-      r /= E[a];
-    }
-    float phi[96];
-    int f = 0;
-    float r2 = 0.f;
-    for (int a = 0; a < d.ndim; ++a) {
-      const float xa = static_cast<float>(t[a]) / static_cast<float>(d.n[a]);
-      r2 += static_cast<float>(t[a]) * static_cast<float>(t[a]);
-      for (int m = 1; m <= fa.num_freqs; ++m) {
-        float sv, cv;
-        sincospif(static_cast<float>(m) * xa, &sv, &cv);
-        phi[f++] = sv;
-        phi[f++] = cv;
-      }
-    }
-    float acc[kMaxChunkOut];
-    for (int j = 0; j < nc; ++j) acc[j] = 0.f;
-    for (int hh = 0; hh < fa.hidden; ++hh) {
-      float pre = __ldg(fa.b1 + hh);
-      const float* w = fa.W1 + static_cast<long long>(hh) * fa.fin;
-      for (int ff = 0; ff < fa.fin; ++ff) pre = fmaf(__ldg(w + ff), phi[ff], pre);
-      const float hv = sinf(pre);
-      for (int j = 0; j < nc; ++j) acc[j] = fmaf(__ldg(fa.W2 + static_cast<long long>(c0 + j) * fa.hidden + hh), hv, acc[j]);
-    }
-    const float rad = sqrtf(r2);
-    long long slot = 0;
-    for (int a = 0; a < d.ndim; ++a) slot = slot * P[a] + ((t[a] + P[a]) % P[a]);
-    for (int j = 0; j < nc; ++j) {
-      const float kv = (acc[j] + __ldg(fa.b2 + c0 + j)) * expf(-__ldg(fa.alpha + c0 + j) * rad / fa.decay_scale);
-      grid[static_cast<long long>(j) * gsz + slot] = make_float2(kv, 0.f);
-    }
-  }
-}
-
 // In-place complex forward DFT of length P (16..512) along one axis of a
 // batch of arrays: element e of pencil (o, i) sits at o*P*stride + e*stride + i.
 // Radix-2 Stockham in shared memory; P/2 threads per pencil.

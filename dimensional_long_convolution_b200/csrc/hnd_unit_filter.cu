@@ -1,6 +1,7 @@
 // Filter spectrum (call 1), spectrum layout conversion, diagnostics.
 #include "hnd_kernels.cuh"
 #include "hnd_multi2.cuh"
+#include "hnd_filter2.cuh"
 #include "hnd_launch.h"
 #include "hnd_host_util.h"
 
@@ -20,6 +21,16 @@ static unsigned grid_for(long long work, int threads) {
   return static_cast<unsigned>(b);
 }
 
+template <int HP>
+static cudaError_t filter_mlp_go(const hnd2::FilterMlpArgs& fa, long long noff, cudaStream_t st) {
+  auto kern = hnd2::k_filter_mlp2<HP>;
+  cudaError_t e = ensure_smem(kern, hnd2::FilterSmem<HP>::bytes(96));     // the largest feature count
+  if (e != cudaSuccess) return e;
+  const long long blocks = (noff + hnd2::kFO - 1) / hnd2::kFO;
+  kern<<<static_cast<unsigned>(blocks), hnd2::kFT, hnd2::FilterSmem<HP>::bytes(fa.fin), st>>>(fa);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, int c0, int nc, float2* grid,
                                 void* spectrum, cudaStream_t st) {
   const SpecDims d = make_dims(ndim, n);
@@ -30,7 +41,7 @@ cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, i
   }
   cudaError_t e = cudaMemsetAsync(grid, 0, sizeof(float2) * gsz * nc, st);
   if (e != cudaSuccess) return e;
-  FilterArgs fa;
+  hnd2::FilterMlpArgs fa;
   fa.W1 = f.W1;
   fa.b1 = f.b1;
   fa.W2 = f.W2;
@@ -40,8 +51,17 @@ cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, i
   fa.hidden = f.hidden;
   fa.fin = 2 * f.num_freqs * ndim;
   fa.decay_scale = f.decay_scale;
-  k_filter_mlp<<<grid_for(noff, 128), 128, 0, st>>>(fa, d, c0, nc, grid);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  fa.ndim = ndim;
+  for (int a = 0; a < 3; ++a) fa.n[a] = a < ndim ? n[a] : 1;
+  fa.c0 = c0;
+  fa.nc = nc;
+  fa.grid = grid;
+  const int HP = (f.hidden + 31) / 32 * 32;
+  e = HP <= 32 ? filter_mlp_go<32>(fa, noff, st)
+      : HP <= 64 ? filter_mlp_go<64>(fa, noff, st)
+      : HP <= 96 ? filter_mlp_go<96>(fa, noff, st)
+                 : filter_mlp_go<128>(fa, noff, st);
+  if (e != cudaSuccess) return e;
   long long stride = gsz;
   for (int a = 0; a < ndim; ++a) {
     const int P = 2 * n[a];
