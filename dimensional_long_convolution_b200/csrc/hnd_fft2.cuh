@@ -395,6 +395,27 @@ __device__ __forceinline__ void padded_fwd(const float2 (&z)[P2<N>::R1], cp (&x)
   fft_fwd<N>(x, g, buf, key, t, mask);
 }
 
+// Full (unpadded) forward transform of length 2N: on entry lo[s] = x[g + s G]
+// and hi[s] = x[N + g + s G]; on exit x[s] holds (X[2f], X[2f+1]) with
+// f = spec_idx<N>(g, s).  Even frequencies are FFT_N(lo + hi), odd ones
+// FFT_N((lo - hi) W_2N^j): the two paths of the packed core.
+template <int N>
+__device__ __forceinline__ void full_fwd(const float2 (&lo)[P2<N>::R1], const float2 (&hi)[P2<N>::R1],
+                                         cp (&x)[P2<N>::R1], int g, float4* buf, int key, Tabs<N> t,
+                                         unsigned mask) {
+  constexpr int G = P2<N>::G, R1 = P2<N>::R1;
+  const float2 tg = t.b[4 * G + g];
+  sfor<0, R1>([&](auto sc) {
+    constexpr int s = decltype(sc)::value;
+    const float2 w = mul_w32<s * (16 / R1)>(tg);     // W_2N^{g + s G}
+    const float2 a = make_float2(lo[s].x + hi[s].x, lo[s].y + hi[s].y);
+    const float2 d = make_float2(lo[s].x - hi[s].x, lo[s].y - hi[s].y);
+    const float2 b = cmul1(d, w);
+    x[s] = {make_float2(a.x, b.x), make_float2(a.y, b.y)};
+  });
+  fft_fwd<N>(x, g, buf, key, t, mask);
+}
+
 // Inverse padded transform keeping outputs [0, N): on entry x[s] =
 // (Y[2f], Y[2f+1]); on exit out[s] = y[g + s G] (unnormalised).
 template <int N>

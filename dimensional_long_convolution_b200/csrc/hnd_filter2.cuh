@@ -15,6 +15,8 @@
 
 #include <cuda_runtime.h>
 
+#include "hnd_fused2.cuh"     // packed FFT core and the W_512 table
+
 namespace hnd2 {
 
 constexpr int kFT = 256;     // threads per CTA
@@ -166,6 +168,57 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
         const int o = 4 * og + i;
         if (e0 + o < noff)
           gch[slot[o]] = make_float2((acc[i][j] + bb) * expf(-al * rad[o] / a.decay_scale), 0.f);
+      }
+    }
+  }
+}
+
+// In-place full complex forward transform of length P = 2N along one axis of
+// a batch of arrays: element e of pencil (o, i) sits at (o P + e) stride + i.
+// One pencil per G lanes of the packed core; a warp takes pencils with
+// consecutive i (adjacent in memory on a strided axis).  Every lane loads its
+// pencil's values before the core's exchange, so the stores cannot overwrite
+// unread inputs.
+constexpr int kAT = 256;     // threads per CTA of the axis transform
+
+template <int N>
+struct AxisSmem {
+  static constexpr size_t kBytes = Tabs<N>::kBytes + 16ull * XB<N>::kWarp * (kAT / 32);
+};
+
+template <int N>
+__global__ void __launch_bounds__(kAT) k_fft_axis2(float2* __restrict__ data, long long stride, long long npencil) {
+  constexpr int G = P2<N>::G, R1 = P2<N>::R1, PPW = 32 / G, P = 2 * N;
+  extern __shared__ __align__(16) unsigned char asmem[];
+  const Tabs<N> t = tabs_at<N>(asmem);
+  float4* xb = reinterpret_cast<float4*>(asmem + Tabs<N>::kBytes);
+  tabs_build<N>(t, g_tw512);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pen = lane / G, g = lane % G;
+  float4* buf = xb + warp * XB<N>::kWarp + pen * XB<N>::kPen;
+  const long long per_cta = (kAT / 32) * PPW;
+  for (long long p0 = static_cast<long long>(blockIdx.x) * per_cta; p0 < npencil;
+       p0 += static_cast<long long>(gridDim.x) * per_cta) {
+    const long long p = p0 + warp * PPW + pen;
+    const bool act = p < npencil;
+    const long long o = act ? p / stride : 0, i = act ? p % stride : 0;
+    float2* base = data + o * P * stride + i;
+    float2 lo[R1], hi[R1];
+#pragma unroll
+    for (int s = 0; s < R1; ++s) {
+      const long long j = g + s * G;
+      lo[s] = act ? base[j * stride] : make_float2(0.f, 0.f);
+      hi[s] = act ? base[(j + N) * stride] : make_float2(0.f, 0.f);
+    }
+    cp x[R1];
+    full_fwd<N>(lo, hi, x, g, buf, 0, t, 0u);
+    if (act) {
+#pragma unroll
+      for (int s = 0; s < R1; ++s) {
+        const long long kk = 2LL * spec_idx<N>(g, s);
+        base[kk * stride] = make_float2(x[s].re.x, x[s].im.x);
+        base[(kk + 1) * stride] = make_float2(x[s].re.y, x[s].im.y);
       }
     }
   }

@@ -852,58 +852,6 @@ static __global__ void k_spec_export(const float2* __restrict__ lib, float2* __r
 }
 
 // ================================================================ the filter
-// Implicit filter on the offset grid (pages: coordinate MLP with sine
-// activation times a window), written wrap-placed into a complex grid P^d
-// per channel of the chunk [c0, c0 + nc).  The grid must be zeroed first
-// (slot n_a of each axis stays 0).
-// In-place complex forward DFT of length P (16..512) along one axis of a
-// batch of arrays: element e of pencil (o, i) sits at o*P*stride + e*stride + i.
-// Radix-2 Stockham in shared memory; P/2 threads per pencil.
-static __global__ void __launch_bounds__(256) k_fft_axis(float2* __restrict__ data, int P, int logP, long long stride,
-                                                  long long npencil) {
-  __shared__ float2 sm[2][512];
-  __shared__ float2 T[kTab];
-  load_twiddles(T);
-  const int per_cta = 512 / P;                     // pencils per CTA
-  const int tid = threadIdx.x;
-  // contiguous pencils: lanes walk one pencil; strided pencils: lanes walk pencils
-  const int pl = (stride == 1) ? tid / (P / 2) : tid % per_cta;
-  const int tj = (stride == 1) ? tid % (P / 2) : tid / per_cta;
-  const long long pen = static_cast<long long>(blockIdx.x) * per_cta + pl;
-  const bool act = pen < npencil;
-  const long long o = act ? pen / stride : 0, i = act ? pen % stride : 0;
-  float2* base = data + o * P * stride + i;
-  float2* a = sm[0] + pl * P;
-  float2* bsm = sm[1] + pl * P;
-  __syncthreads();
-  if (act) {
-    a[tj] = base[tj * stride];
-    a[tj + P / 2] = base[(tj + P / 2) * stride];
-  }
-  __syncthreads();
-  int ns = 1;
-  for (int st = 0; st < logP; ++st) {
-    // radix-2 Stockham pass: inputs j and j + P/2, twiddle W_{2ns}^{j mod ns}
-    const int j = tj;
-    const int jm = j & (ns - 1);
-    const float2 w = T[jm * (kTab / (2 * ns))];
-    const float2 x0 = a[j];
-    const float2 x1 = c_mul(a[j + P / 2], w);
-    const int outi = (j / ns) * ns * 2 + jm;
-    bsm[outi] = c_add(x0, x1);
-    bsm[outi + ns] = c_sub(x0, x1);
-    __syncthreads();
-    float2* t = a;
-    a = bsm;
-    bsm = t;
-    ns *= 2;
-  }
-  if (act) {
-    base[tj * stride] = a[tj];
-    base[(tj + P / 2) * stride] = a[tj + P / 2];
-  }
-}
-
 // Full-grid natural spectra (chunk of channels) -> library order, scaled.
 static __global__ void k_spec_pack(const float2* __restrict__ grid, float2* __restrict__ out, SpecDims d, int c0, int nc,
                             float scale) {

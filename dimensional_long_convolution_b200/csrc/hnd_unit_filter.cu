@@ -31,6 +31,20 @@ static cudaError_t filter_mlp_go(const hnd2::FilterMlpArgs& fa, long long noff, 
   return cudaGetLastError();
 }
 
+// Full transform of length 2N along one axis of the filter grid.
+template <int N>
+static cudaError_t fft_axis_go(float2* grid, long long stride, long long npen, cudaStream_t st) {
+  auto kern = hnd2::k_fft_axis2<N>;
+  const size_t sm = hnd2::AxisSmem<N>::kBytes;
+  cudaError_t e = ensure_smem(kern, sm);
+  if (e != cudaSuccess) return e;
+  const long long per_cta = (hnd2::kAT / 32) * (32 / hnd2::P2<N>::G);
+  long long blocks = (npen + per_cta - 1) / per_cta;
+  if (blocks > 148LL * 16) blocks = 148LL * 16;
+  kern<<<static_cast<unsigned>(blocks), hnd2::kAT, sm, st>>>(grid, stride, npen);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, int c0, int nc, float2* grid,
                                 void* spectrum, cudaStream_t st) {
   const SpecDims d = make_dims(ndim, n);
@@ -64,14 +78,18 @@ cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, i
   if (e != cudaSuccess) return e;
   long long stride = gsz;
   for (int a = 0; a < ndim; ++a) {
-    const int P = 2 * n[a];
-    stride /= P;
-    int logP = 0;
-    while ((1 << logP) < P) ++logP;
-    const long long npen = gsz * nc / P;
-    const long long per_cta = 512 / P;
-    k_fft_axis<<<static_cast<unsigned>((npen + per_cta - 1) / per_cta), 256, 0, st>>>(grid, P, logP, stride, npen);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    stride /= 2 * n[a];
+    const long long npen = gsz * nc / (2 * n[a]);
+    switch (n[a]) {
+      case 8: e = fft_axis_go<8>(grid, stride, npen, st); break;
+      case 16: e = fft_axis_go<16>(grid, stride, npen, st); break;
+      case 32: e = fft_axis_go<32>(grid, stride, npen, st); break;
+      case 64: e = fft_axis_go<64>(grid, stride, npen, st); break;
+      case 128: e = fft_axis_go<128>(grid, stride, npen, st); break;
+      case 256: e = fft_axis_go<256>(grid, stride, npen, st); break;
+      default: e = cudaErrorInvalidValue;
+    }
+    if (e != cudaSuccess) return e;
   }
   const long long per = spec_per_channel(d);
   const float scale = static_cast<float>(1.0 / static_cast<double>(gsz));
