@@ -258,7 +258,7 @@ hyena_nd_status hyena_nd_filter_spectrum(const hyena_nd_problem* p, const hyena_
   hyena_nd_status st = make_plan(p, &pl);
   if (st != HYENA_ND_OK) return st;
   if (!f || !spectrum || !ws || !f->W1 || !f->b1 || !f->W2 || !f->b2 || !f->alpha) return HYENA_ND_ERR_INVALID_ARG;
-  if (f->window != 0) return HYENA_ND_ERR_UNSUPPORTED;
+  if (f->window != 0 && f->window != 1) return HYENA_ND_ERR_UNSUPPORTED;
   if (f->num_freqs < 1 || f->num_freqs > 16 || f->hidden < 1 || f->hidden > 128) return HYENA_ND_ERR_UNSUPPORTED;
   if (!(f->decay_scale > 0.f) || !std::isfinite(f->decay_scale)) return HYENA_ND_ERR_INVALID_ARG;
   if (!aligned16(spectrum) || !aligned16(ws)) return HYENA_ND_ERR_MISALIGNED;
@@ -275,6 +275,7 @@ hyena_nd_status hyena_nd_filter_spectrum(const hyena_nd_problem* p, const hyena_
   fl.num_freqs = f->num_freqs;
   fl.hidden = f->hidden;
   fl.decay_scale = f->decay_scale;
+  fl.window = f->window;
   float2* grid = reinterpret_cast<float2*>(static_cast<char*>(ws) + kStatusBytes);
   for (long long c0 = 0; c0 < pl.C; c0 += pl.filter_chunk) {
     const int nc = static_cast<int>(pl.C - c0 < pl.filter_chunk ? pl.C - c0 : pl.filter_chunk);

@@ -8,7 +8,8 @@
 // subquadratic operators via input-dependent long convolutions", section on
 // the neural parameterisation.)
 //   phi(t) = [sin(pi m t_a / n_a), cos(pi m t_a / n_a)]  m = 1..M, axis-major
-//   h = sin(W1 phi + b1),  K_c(t) = (W2 h + b2)_c exp(-alpha_c |t|_2 / s)
+//   h = sin(W1 phi + b1),  K_c(t) = (W2 h + b2)_c w_c(t)
+//   w_c(t) = exp(-alpha_c |t|_2 / s), or the Gaussian exp(-alpha_c (|t|_2 / s)^2)
 // written wrap-placed (offset t at slot t mod P on each axis) into a complex
 // grid [nc][P^d] whose other slots the caller has zeroed.
 #pragma once
@@ -27,6 +28,7 @@ struct FilterMlpArgs {
   const float *W1, *b1, *W2, *b2, *alpha;
   int num_freqs, hidden, fin;    // fin = 2 num_freqs ndim
   float decay_scale;
+  int window;                    // 0: exp(-alpha |t| / s), 1: exp(-alpha (|t| / s)^2)
   int ndim;
   int n[3];
   int c0, nc;                    // channel chunk [c0, c0 + nc)
@@ -87,7 +89,9 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
     int t0, t1, t2;
     offset_of(o, t0, t1, t2);
     const float f0 = static_cast<float>(t0), f1 = static_cast<float>(t1), f2 = static_cast<float>(t2);
-    rad[o] = sqrtf(f0 * f0 + f1 * f1 + f2 * f2);
+    // the window's argument |t| / s, squared for the Gaussian window
+    const float rs = sqrtf(f0 * f0 + f1 * f1 + f2 * f2) / a.decay_scale;
+    rad[o] = a.window == 1 ? rs * rs : rs;
     const int s0 = (t0 + P0) % P0, s1 = (t1 + P1) % P1, s2 = (t2 + P2) % P2;
     slot[o] = (s0 * P1 + s1) * P2 + s2;
   }
@@ -167,7 +171,7 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
       for (int i = 0; i < 4; ++i) {
         const int o = 4 * og + i;
         if (e0 + o < noff)
-          gch[slot[o]] = make_float2((acc[i][j] + bb) * expf(-al * rad[o] / a.decay_scale), 0.f);
+          gch[slot[o]] = make_float2((acc[i][j] + bb) * expf(-al * rad[o]), 0.f);
       }
     }
   }

@@ -55,6 +55,7 @@ struct FilterLaunch {
   const float *W1, *b1, *W2, *b2, *alpha;
   int num_freqs, hidden;
   float decay_scale;
+  int window = 0;         // 0: exp(-alpha |t| / s), 1: exp(-alpha (|t| / s)^2)
 };
 cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, int c0, int nc, float2* grid,
                                 void* spectrum, cudaStream_t st);

@@ -65,6 +65,7 @@ cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, i
   fa.hidden = f.hidden;
   fa.fin = 2 * f.num_freqs * ndim;
   fa.decay_scale = f.decay_scale;
+  fa.window = f.window;
   fa.ndim = ndim;
   for (int a = 0; a < 3; ++a) fa.n[a] = a < ndim ? n[a] : 1;
   fa.c0 = c0;

@@ -232,7 +232,7 @@ class HyenaND:
         P = [2 * n for n in self.dims]
         return (self.C,) + tuple(P[:-1]) + (self.dims[-1] + 1,)
 
-    def set_filter(self, W1, b1, W2, b2, alpha, decay_scale: float, num_freqs: int = 8) -> None:
+    def set_filter(self, W1, b1, W2, b2, alpha, decay_scale: float, num_freqs: int = 8, window: int = 0) -> None:
         t = [x.to(self.device, self.torch.float32).contiguous() for x in (W1, b1, W2, b2, alpha)]
         self._filter_params = t        # keep alive until the call has run
         f = Filter()
@@ -240,7 +240,7 @@ class HyenaND:
         f.hidden = int(t[0].shape[0])
         f.W1, f.b1, f.W2, f.b2, f.alpha = (x.data_ptr() for x in t)
         f.decay_scale = float(decay_scale)
-        f.window = 0
+        f.window = int(window)
         check(filter_spectrum(self.p, f, self.spectrum.data_ptr(), self.ws.data_ptr(), self.ws_bytes,
                               self._stream()), "filter_spectrum")
 

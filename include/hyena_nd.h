@@ -89,8 +89,11 @@ typedef struct {
  *   K_c(t)  = ((W2 h + b2)_c) * exp(-alpha_c * ||t||_2 / decay_scale)
  * Device pointers, fp32, row-major: W1 [hidden, 2*num_freqs*ndim], b1 [hidden],
  * W2 [C, hidden], b2 [C], alpha [C].  Limits: 1 <= num_freqs <= 16,
- * 1 <= hidden <= 128, decay_scale > 0.  window must be 0 (exponential decay);
- * the Gaussian window of the pages is not implemented (HYENA_ND_ERR_UNSUPPORTED). */
+ * 1 <= hidden <= 128, decay_scale > 0.  window 0: exp(-alpha_c |t|_2 / s);
+ * window 1: the Gaussian window exp(-alpha_c (|t|_2 / s)^2) (arXiv 2607.19378
+ * summary, "Methodologie", kernel synthesis: a learnable Gaussian window times
+ * the coordinate network; alpha_c is its learnable width); other values:
+ * HYENA_ND_ERR_UNSUPPORTED. */
 typedef struct {
   int num_freqs;
   int hidden;

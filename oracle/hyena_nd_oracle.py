@@ -64,11 +64,15 @@ def fourier_features(t: np.ndarray, dims: Sequence[int], num_freqs: int) -> np.n
     return np.stack(cols, axis=-1)
 
 
-def implicit_kernel(filt, dims: Sequence[int], channels=None, chunk: int = 1 << 18) -> np.ndarray:
+def implicit_kernel(filt, dims: Sequence[int], channels=None, chunk: int = 1 << 18, window: int = 0) -> np.ndarray:
     """K_c(t) for every channel c (or the listed ``channels``) and offset t
-    (pages: coordinate MLP with sine activation times a decay window; reading
-    4).  Computed in float64 from the fp32 parameters, ``chunk`` offsets at a
-    time to bound memory.  Returns [C, 2n_1-1, ..., 2n_d-1]; index t + (n - 1)."""
+    (pages: coordinate MLP with sine activation times a window; reading 4).
+    window 0: exp(-alpha_c ||t||_2 / s); window 1: the Gaussian window of the
+    arXiv summary ("Methodologie", kernel synthesis: a learnable Gaussian
+    window times the coordinate network), read as exp(-alpha_c (||t||_2 / s)^2)
+    with alpha_c the learnable width.  Computed in float64 from the fp32
+    parameters, ``chunk`` offsets at a time to bound memory.  Returns
+    [C, 2n_1-1, ..., 2n_d-1]; index t + (n - 1)."""
     t_all = offsets_grid(dims)
     W1 = filt.W1.astype(np.float64)
     b1 = filt.b1.astype(np.float64)
@@ -83,8 +87,9 @@ def implicit_kernel(filt, dims: Sequence[int], channels=None, chunk: int = 1 << 
         h = np.sin(phi @ W1.T + b1)                      # [N, H]
         mlp = h @ W2.T + b2                              # [N, C]
         r = np.sqrt(np.sum(t * t, axis=-1))              # ||t||_2
-        window = np.exp(-np.outer(r, alpha) / float(filt.decay_scale))
-        K[:, s0: s0 + chunk] = (mlp * window).T
+        rs = r / float(filt.decay_scale)
+        win = np.exp(-np.outer(rs * rs if window == 1 else rs, alpha))
+        K[:, s0: s0 + chunk] = (mlp * win).T
     return K.reshape((len(sel),) + tuple(2 * n - 1 for n in dims))
 
 

@@ -142,8 +142,8 @@ def test_filter_arguments_are_checked():
     f.num_freqs, f.hidden = 8, 64
     f.W1 = f.b1 = f.W2 = f.b2 = f.alpha = A + 7 * STEP
     f.decay_scale, f.window = 32.0, 0
-    f.window = 1
-    assert H.filter_spectrum(p, f, s, ws, wsb) == H.ERR_UNSUPPORTED      # Gaussian window
+    f.window = 2
+    assert H.filter_spectrum(p, f, s, ws, wsb) == H.ERR_UNSUPPORTED      # no such window
     f.window = 0
     f.hidden = 0
     assert H.filter_spectrum(p, f, s, ws, wsb) == H.ERR_UNSUPPORTED

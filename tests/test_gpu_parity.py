@@ -34,6 +34,20 @@ def test_filter_spectrum_matches_oracle(dims, C):
     assert O.rel_l2(got, want) < 2e-5
 
 
+@pytest.mark.parametrize("dims,C", [((32,), 3), ((16, 64), 3), ((256, 256), 2), ((16, 8, 32), 2)])
+def test_filter_spectrum_gaussian_window(dims, C):
+    wl = W.custom(dims, 1, C, seed=17)
+    inp = W.make_inputs(wl, with_qkv=False)
+    op = make_op(wl)
+    t = torch()
+    f = inp.filt
+    op.set_filter(t.from_numpy(f.W1), t.from_numpy(f.b1), t.from_numpy(f.W2), t.from_numpy(f.b2),
+                  t.from_numpy(f.alpha), f.decay_scale, f.num_freqs, window=1)
+    got = to_host(op.export_spectrum())
+    want = O.spectrum_half(O.implicit_kernel(f, dims, window=1), dims)
+    assert O.rel_l2(got, want) < 2e-5
+
+
 @pytest.mark.parametrize("i,channels", [(1, [0, 255]), (2, [0, 127]), (3, [0, 63]), (4, [0, 31])])
 def test_filter_spectrum_benchmark_grids(i, channels):
     wl = W.workload(i)

@@ -244,6 +244,24 @@ def test_filter_window_closed_form():
     assert K[1, 7, 7] == -2.0
 
 
+def test_filter_gaussian_window_closed_form():
+    """window 1: exp(-alpha (||t|| / s)^2) (reading of the learnable Gaussian
+    window); W2 = 0 isolates the window times b2."""
+    dims = (8, 8, 8)
+    p = _params(2, 48)
+    p.W2[:] = 0.0
+    p.b2[:] = [1.0, 3.0]
+    p.alpha[:] = [0.5, 2.0]
+    K = O.implicit_kernel(p, dims, window=1)
+    # offset (1, 2, 2): ||t|| = 3, s = 8
+    assert abs(K[0, 7 + 1, 7 - 2, 7 + 2] - np.exp(-0.5 * (3 / 8.0) ** 2)) < 1e-15
+    assert abs(K[1, 7 - 1, 7 + 2, 7 - 2] - 3.0 * np.exp(-2.0 * (3 / 8.0) ** 2)) < 1e-15
+    assert K[1, 7, 7, 7] == 3.0
+    # the exponential window at the same offset differs (the two readings are distinct)
+    Ke = O.implicit_kernel(p, dims, window=0)
+    assert abs(Ke[0, 8, 5, 9] - np.exp(-0.5 * 3 / 8.0)) < 1e-15
+
+
 @pytest.mark.parametrize("axis,m,cos", [(0, 1, 0), (1, 1, 0), (1, 3, 1), (0, 8, 1), (2, 5, 0)])
 def test_filter_feature_order_closed_form(axis, m, cos):
     """One hidden unit reading one feature: K_0(t) = sin(f(pi m t_axis / n_axis))
