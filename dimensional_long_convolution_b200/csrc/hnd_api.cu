@@ -23,6 +23,7 @@ constexpr size_t kStatusBytes = 256;                  // status word + padding
 constexpr size_t kWaveBudget = size_t(96) << 20;      // multi-pass intermediate per wave (measured best of 24/48/96 MiB)
 constexpr size_t kFilterBudget = size_t(64) << 20;    // filter grid per channel chunk
 constexpr int kFilterMaxChunk = 64;
+constexpr size_t kKgradBudget = size_t(128) << 20;    // kernel-gradient grids per channel chunk
 
 enum Tier { kRows1D = 0, kFused2D = 1, kMulti2D = 2, kMulti3D = 3 };
 
@@ -37,6 +38,7 @@ struct Plan {
   int tier = 0;
   long long wave = 0;       // pairs per wave (multi-pass tiers)
   int filter_chunk = 1;
+  int kgrad_chunk = 1;      // channels per kernel-gradient chunk
   size_t ws_total = 0;
   size_t spec_bytes = 0;
 };
@@ -100,7 +102,17 @@ hyena_nd_status make_plan(const hyena_nd_problem* p, Plan* pl) {
   if (chunk > p->C) chunk = p->C;
   pl->filter_chunk = static_cast<int>(chunk);
   const size_t ws_filter = static_cast<size_t>(chunk) * static_cast<size_t>(pl->gsz) * 8;
-  pl->ws_total = kStatusBytes + (ws_conv > ws_filter ? ws_conv : ws_filter);
+  // kernel gradient: per channel 2B transformed grids (u and z per sample) and
+  // one accumulator, P^d complex each
+  const size_t per_kg = (2 * static_cast<size_t>(p->B) + 1) * static_cast<size_t>(pl->gsz) * 8;
+  long long kgc = static_cast<long long>(kKgradBudget / per_kg);
+  if (kgc < 1) kgc = 1;
+  if (kgc > p->C) kgc = p->C;
+  pl->kgrad_chunk = static_cast<int>(kgc);
+  const size_t ws_kgrad = per_kg * static_cast<size_t>(kgc);
+  size_t need = ws_conv > ws_filter ? ws_conv : ws_filter;
+  if (ws_kgrad > need) need = ws_kgrad;
+  pl->ws_total = kStatusBytes + need;
   return HYENA_ND_OK;
 }
 
@@ -109,6 +121,12 @@ bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u
 bool overlaps(const void* a, const void* b, size_t bytes) {
   const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
   return x < y + bytes && y < x + bytes;
+}
+
+// [a, a + na) and [b, b + nb) share a byte
+bool overlaps2(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
 }
 
 hyena_nd_status cuda_status(cudaError_t e) { return e == cudaSuccess ? HYENA_ND_OK : HYENA_ND_ERR_CUDA; }
@@ -249,6 +267,43 @@ hyena_nd_status hyena_nd_fftconv_backward(const hyena_nd_problem* p, const void*
   if (e == cudaSuccess) e = run_conv(pl, a, ws, &launches);
   if (e != cudaSuccess) return HYENA_ND_ERR_CUDA;
   g_last_launches = launches;
+  return HYENA_ND_OK;
+}
+
+hyena_nd_status hyena_nd_kernel_grad(const hyena_nd_problem* p, const void* q, const void* k, const void* v,
+                                     const void* dy, float* dK, void* ws, size_t ws_bytes, void* cuda_stream) {
+  Plan pl;
+  hyena_nd_status st = make_plan(p, &pl);
+  if (st != HYENA_ND_OK) return st;
+  if (!q || !k || !v || !dy || !dK || !ws) return HYENA_ND_ERR_INVALID_ARG;
+  const void* ptrs[6] = {q, k, v, dy, dK, ws};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return HYENA_ND_ERR_MISALIGNED;
+  if (ws_bytes < pl.ws_total) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
+  long long noff = 1;
+  for (int a = 0; a < pl.ndim; ++a) noff *= 2 * pl.n[a] - 1;
+  const size_t act_bytes = static_cast<size_t>(pl.B * pl.C * pl.L) * (pl.bf16 ? 2 : 4);
+  const size_t dk_bytes = static_cast<size_t>(pl.C * noff) * 4;
+  const void* ins[4] = {q, k, v, dy};
+  for (const void* in : ins)
+    if (overlaps2(dK, dk_bytes, in, act_bytes)) return HYENA_ND_ERR_INVALID_ARG;
+  hnd::KgradLaunch g;
+  g.q = q;
+  g.k = k;
+  g.v = v;
+  g.dy = dy;
+  g.dK = dK;
+  g.grids = reinterpret_cast<float2*>(static_cast<char*>(ws) + kStatusBytes);
+  g.ndim = pl.ndim;
+  for (int i = 0; i < 3; ++i) g.n[i] = pl.n[i];
+  g.B = static_cast<int>(pl.B);
+  g.C = static_cast<int>(pl.C);
+  g.bf16 = pl.bf16;
+  for (long long c0 = 0; c0 < pl.C; c0 += pl.kgrad_chunk) {
+    g.c0 = static_cast<int>(c0);
+    g.ncc = static_cast<int>(pl.C - c0 < pl.kgrad_chunk ? pl.C - c0 : pl.kgrad_chunk);
+    if (hnd::launch_kgrad_chunk(g, static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess) return HYENA_ND_ERR_CUDA;
+  }
   return HYENA_ND_OK;
 }
 

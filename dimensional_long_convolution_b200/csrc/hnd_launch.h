@@ -61,6 +61,18 @@ cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, i
                                 void* spectrum, cudaStream_t st);
 cudaError_t launch_spec_convert(int ndim, const int* n, long long C, const void* src, void* dst, bool to_natural,
                                 cudaStream_t st);
+// In-place full forward transforms along every axis of `ngrids` complex grids
+// [P^d] (P_a = 2 n_a), adjacent in memory.
+cudaError_t launch_fft_axes(float2* grid, int ndim, const int* n, long long ngrids, cudaStream_t st);
+
+// Kernel-value gradient for channels [c0, c0 + ncc) (all B samples of each).
+struct KgradLaunch {
+  const void *q, *k, *v, *dy;
+  float* dK;              // [C][2n-1 ...]
+  float2* grids;          // (2 B + 1) ncc grids of P^d complex
+  int ndim, n[3], B, C, c0, ncc, bf16;
+};
+cudaError_t launch_kgrad_chunk(const KgradLaunch& g, cudaStream_t st);
 cudaError_t launch_bounded_wait(int* status, const int* flag, long long limit_cycles, cudaStream_t st);
 
 }  // namespace hnd

@@ -2,6 +2,7 @@
 #include "hnd_kernels.cuh"
 #include "hnd_multi2.cuh"
 #include "hnd_filter2.cuh"
+#include "hnd_kgrad.cuh"
 #include "hnd_launch.h"
 #include "hnd_host_util.h"
 
@@ -45,6 +46,27 @@ static cudaError_t fft_axis_go(float2* grid, long long stride, long long npen, c
   return cudaGetLastError();
 }
 
+cudaError_t launch_fft_axes(float2* grid, int ndim, const int* n, long long ngrids, cudaStream_t st) {
+  long long gsz = 1;
+  for (int a = 0; a < ndim; ++a) gsz *= 2 * n[a];
+  long long stride = gsz;
+  cudaError_t e = cudaSuccess;
+  for (int a = 0; a < ndim && e == cudaSuccess; ++a) {
+    stride /= 2 * n[a];
+    const long long npen = gsz * ngrids / (2 * n[a]);
+    switch (n[a]) {
+      case 8: e = fft_axis_go<8>(grid, stride, npen, st); break;
+      case 16: e = fft_axis_go<16>(grid, stride, npen, st); break;
+      case 32: e = fft_axis_go<32>(grid, stride, npen, st); break;
+      case 64: e = fft_axis_go<64>(grid, stride, npen, st); break;
+      case 128: e = fft_axis_go<128>(grid, stride, npen, st); break;
+      case 256: e = fft_axis_go<256>(grid, stride, npen, st); break;
+      default: e = cudaErrorInvalidValue;
+    }
+  }
+  return e;
+}
+
 cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, int c0, int nc, float2* grid,
                                 void* spectrum, cudaStream_t st) {
   const SpecDims d = make_dims(ndim, n);
@@ -77,21 +99,8 @@ cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, i
       : HP <= 96 ? filter_mlp_go<96>(fa, noff, st)
                  : filter_mlp_go<128>(fa, noff, st);
   if (e != cudaSuccess) return e;
-  long long stride = gsz;
-  for (int a = 0; a < ndim; ++a) {
-    stride /= 2 * n[a];
-    const long long npen = gsz * nc / (2 * n[a]);
-    switch (n[a]) {
-      case 8: e = fft_axis_go<8>(grid, stride, npen, st); break;
-      case 16: e = fft_axis_go<16>(grid, stride, npen, st); break;
-      case 32: e = fft_axis_go<32>(grid, stride, npen, st); break;
-      case 64: e = fft_axis_go<64>(grid, stride, npen, st); break;
-      case 128: e = fft_axis_go<128>(grid, stride, npen, st); break;
-      case 256: e = fft_axis_go<256>(grid, stride, npen, st); break;
-      default: e = cudaErrorInvalidValue;
-    }
-    if (e != cudaSuccess) return e;
-  }
+  e = launch_fft_axes(grid, ndim, n, nc, st);
+  if (e != cudaSuccess) return e;
   const long long per = spec_per_channel(d);
   const float scale = static_cast<float>(1.0 / static_cast<double>(gsz));
   if (ndim == 2) {
@@ -105,6 +114,44 @@ cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, i
     k_spec_pack<<<grid_for(per * nc, 256), 256, 0, st>>>(grid, static_cast<float2*>(spectrum), d, c0, nc, scale);
   }
   return cudaGetLastError();
+}
+
+template <class T>
+static cudaError_t kgrad_chunk_t(const KgradLaunch& g, cudaStream_t st) {
+  hnd2::KgDims d;
+  d.n0 = g.n[0];
+  d.n1 = g.ndim > 1 ? g.n[1] : 1;
+  d.n2 = g.ndim > 2 ? g.n[2] : 1;
+  d.P0 = 2 * d.n0;
+  d.P1 = g.ndim > 1 ? 2 * d.n1 : 1;
+  d.P2 = g.ndim > 2 ? 2 * d.n2 : 1;
+  const long long gsz = static_cast<long long>(d.P0) * d.P1 * d.P2;
+  const int nvol = g.ncc * g.B;
+  float2* gu = g.grids;
+  float2* gz = gu + gsz * nvol;
+  float2* acc = gz + gsz * nvol;
+  const T* q = static_cast<const T*>(g.q);
+  const T* k = static_cast<const T*>(g.k);
+  const T* v = static_cast<const T*>(g.v);
+  const T* dy = static_cast<const T*>(g.dy);
+  hnd2::k_kg_pad<T><<<grid_for(gsz * nvol, 256), 256, 0, st>>>(k, v, gu, d, g.B, g.C, g.c0, nvol);
+  hnd2::k_kg_pad<T><<<grid_for(gsz * nvol, 256), 256, 0, st>>>(q, dy, gz, d, g.B, g.C, g.c0, nvol);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = launch_fft_axes(gu, g.ndim, g.n, 2LL * nvol, st);      // gu and gz are adjacent
+  if (e != cudaSuccess) return e;
+  hnd2::k_kg_corr<<<grid_for(gsz * g.ncc, 256), 256, 0, st>>>(gu, gz, acc, g.B, g.ncc, gsz);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  e = launch_fft_axes(acc, g.ndim, g.n, g.ncc, st);
+  if (e != cudaSuccess) return e;
+  long long noff = 1;
+  for (int a = 0; a < g.ndim; ++a) noff *= 2 * g.n[a] - 1;
+  hnd2::k_kg_extract<<<grid_for(noff * g.ncc, 256), 256, 0, st>>>(acc, g.dK, d, g.c0, g.ncc,
+                                                                    static_cast<float>(1.0 / static_cast<double>(gsz)));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_kgrad_chunk(const KgradLaunch& g, cudaStream_t st) {
+  return g.bf16 ? kgrad_chunk_t<__nv_bfloat16>(g, st) : kgrad_chunk_t<float>(g, st);
 }
 
 cudaError_t launch_spec_convert(int ndim, const int* n, long long C, const void* src, void* dst, bool to_natural,

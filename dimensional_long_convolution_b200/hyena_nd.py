@@ -38,6 +38,7 @@ EXPORTED = (
     "hyena_nd_fftconv",
     "hyena_nd_fftconv_batched",
     "hyena_nd_fftconv_backward",
+    "hyena_nd_kernel_grad",
     "hyena_nd_spectrum_export",
     "hyena_nd_spectrum_import",
     "hyena_nd_device_status",
@@ -102,6 +103,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "hyena_nd_fftconv": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
         "hyena_nd_fftconv_batched": (ctypes.c_int, [P, vp, vp, vp, vp, i64, vp, vp, sz, vp]),
         "hyena_nd_fftconv_backward": (ctypes.c_int, [P, vp, vp, vp, vp, i64, vp, vp, vp, vp, vp, sz, vp]),
+        "hyena_nd_kernel_grad": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
         "hyena_nd_spectrum_export": (ctypes.c_int, [P, vp, vp, vp]),
         "hyena_nd_spectrum_import": (ctypes.c_int, [P, vp, vp, vp]),
         "hyena_nd_device_status": (ctypes.c_int, [vp, vp]),
@@ -183,6 +185,11 @@ def fftconv_backward(p: Problem, q: int, k: int, v: int, spectrum: int, spectrum
                      dq: int, dk: int, dv: int, ws: int, ws_bytes: int, stream: int = 0) -> int:
     return load().hyena_nd_fftconv_backward(ctypes.byref(p), q, k, v, spectrum, int(spectrum_batch_stride), dy,
                                             dq, dk, dv, ws, ws_bytes, stream)
+
+
+def kernel_grad(p: Problem, q: int, k: int, v: int, dy: int, dK: int, ws: int, ws_bytes: int,
+                stream: int = 0) -> int:
+    return load().hyena_nd_kernel_grad(ctypes.byref(p), q, k, v, dy, dK, ws, ws_bytes, stream)
 
 
 def status_string(code: int) -> str:
@@ -277,6 +284,18 @@ class HyenaND:
                                int(spectrum_batch_stride), dy.data_ptr(), dq.data_ptr(), dk.data_ptr(),
                                dv.data_ptr(), self.ws.data_ptr(), self.ws_bytes, self._stream()), "fftconv_backward")
         return dq, dk, dv
+
+    def kernel_grad(self, q, k, v, dy):
+        """dK [C, 2n-1, ...] (float32): the gradient of the loss with respect to
+        the kernel values, for the loss gradient dy of __call__'s output."""
+        for t in (q, k, v, dy):
+            if t.dtype != self.tdtype or not t.is_contiguous() or t.device != self.device:
+                raise ValueError("q, k, v, dy must be contiguous %s tensors on %s" % (self.tdtype, self.device))
+        dK = self.torch.empty((self.C,) + tuple(2 * n - 1 for n in self.dims), dtype=self.torch.float32,
+                              device=self.device)
+        check(kernel_grad(self.p, q.data_ptr(), k.data_ptr(), v.data_ptr(), dy.data_ptr(), dK.data_ptr(),
+                          self.ws.data_ptr(), self.ws_bytes, self._stream()), "kernel_grad")
+        return dK
 
     def status(self) -> int:
         return device_status(self.ws.data_ptr(), self._stream())

@@ -173,6 +173,22 @@ HYENA_ND_API hyena_nd_status hyena_nd_fftconv_backward(const hyena_nd_problem* p
                                           void* dk, void* dv, void* ws, size_t ws_bytes,
                                           void* cuda_stream);
 
+/* Gradient with respect to the kernel values, given dy = dL/dy of call 3:
+ *   dK[c, t] = sum_b sum_{i in [0,n)^d} q[b,c,i] dy[b,c,i] u[b,c,i - t],  u = k (.) v,
+ * for every offset t in [-(n_1-1), n_1-1] x ... (terms with i - t outside the
+ * grid are absent): the cross-correlation of q (.) dy with u, summed over the
+ * batch (blog "Native multi-dimensional subquadratic operators via
+ * input-dependent long convolutions", gradient sections: dK by correlation).
+ * Computed through zero-padded transforms on the 2n grid with fp32
+ * arithmetic; the sum over b runs in a fixed order (deterministic).
+ * q, k, v, dy: [B, C, n...] in the problem's dtype, read.  dK: float32
+ * [C, 2n_1-1, ..., 2n_d-1] (index t + n - 1), written; it may not overlap an
+ * input.  The chain into the filter's parameters is the caller's (the filter
+ * call is its forward).  `ws`: hyena_nd_workspace_bytes(p) bytes. */
+HYENA_ND_API hyena_nd_status hyena_nd_kernel_grad(const hyena_nd_problem* p, const void* q, const void* k,
+                                     const void* v, const void* dy, float* dK, void* ws, size_t ws_bytes,
+                                     void* cuda_stream);
+
 /* Same operation as hyena_nd_fftconv_batched, for callers that cannot
  * allocate device memory and so have no workspace to pass: for instance a
  * plugin whose interface carries only input and output buffers, or an

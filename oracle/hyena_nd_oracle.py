@@ -300,6 +300,55 @@ def backward_direct(q, k, v, dy, K, dims) -> Tuple[np.ndarray, np.ndarray, np.nd
     return dy * w, v * du, k * du
 
 
+# ------------------------------------------------------- kernel-value gradient
+# dL/dK for L = sum dy y: y[i] = q[i] sum_j u[j] K[i - j] gives
+#   dK[c, t] = sum_b sum_{i in [0,n)^d} q[b,c,i] dy[b,c,i] u[b,c,i - t]
+# for every offset t in [-(n-1), n-1]^d (terms with i - t outside the grid
+# are absent): the cross-correlation of z = q dy with u, summed over the
+# batch (blog, gradient sections: dK by correlation).
+def kernel_grad_direct(q, k, v, dy, dims) -> np.ndarray:
+    """The definition, one offset at a time.  Returns [C, 2n-1, ...]."""
+    d = len(dims)
+    B, C = q.shape[:2]
+    z, u = q * dy, k * v
+    out = np.zeros((C,) + tuple(2 * n - 1 for n in dims))
+    for t in itertools.product(*[range(-(n - 1), n) for n in dims]):
+        zi = tuple(slice(max(0, ta), n + min(0, ta)) for ta, n in zip(t, dims))
+        uj = tuple(slice(max(0, -ta), n - max(0, ta)) for ta, n in zip(t, dims))
+        val = np.sum(z[(slice(None), slice(None)) + zi] * u[(slice(None), slice(None)) + uj],
+                     axis=tuple(range(2, 2 + d)))
+        out[(slice(None),) + tuple(ta + n - 1 for ta, n in zip(t, dims))] = val.sum(axis=0)
+    return out
+
+
+def kernel_grad_at(q, k, v, dy, dims, points: np.ndarray) -> np.ndarray:
+    """kernel_grad_direct at chosen (c, t_1..t_d) rows only.  O(B L) each."""
+    z, u = q * dy, k * v
+    out = np.empty(points.shape[0])
+    for r, p in enumerate(points):
+        c, t = int(p[0]), [int(x) for x in p[1:]]
+        zi = tuple(slice(max(0, ta), n + min(0, ta)) for ta, n in zip(t, dims))
+        uj = tuple(slice(max(0, -ta), n - max(0, ta)) for ta, n in zip(t, dims))
+        out[r] = float(np.sum(z[(slice(None), c) + zi] * u[(slice(None), c) + uj]))
+    return out
+
+
+def kernel_grad_dft(q, k, v, dy, dims) -> np.ndarray:
+    """Through zero-padded DFTs: correlation = IDFT(sum_b Z_b conj(U_b)) on
+    the 2n grid, read back at slot t mod 2n.  Returns [C, 2n-1, ...]."""
+    d = len(dims)
+    z, u = (q * dy).astype(np.complex128), (k * v).astype(np.complex128)
+    for a, n in enumerate(dims):
+        F = dft_matrix(2 * n)[:, :n]
+        z = _apply_along(z, F, 2 + a)
+        u = _apply_along(u, F, 2 + a)
+    acc = np.sum(z * np.conj(u), axis=0)                  # [C, P...]
+    for a, n in enumerate(dims):
+        acc = _apply_along(acc, np.conj(dft_matrix(2 * n)) / (2 * n), 1 + a)
+    idx = [np.arange(-(n - 1), n) % (2 * n) for n in dims]
+    return acc.real[np.ix_(np.arange(acc.shape[0]), *idx)]
+
+
 # -------------------------------------------------------------- conveniences
 def reference_output(inputs, S_full=None, K=None) -> np.ndarray:
     """y for a seeded workload through O2 (float64)."""

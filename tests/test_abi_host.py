@@ -4,6 +4,7 @@ touching the GPU (no call here reaches a kernel launch)."""
 import os
 import re
 
+import numpy as np
 import pytest
 
 from dimensional_long_convolution_b200 import hyena_nd as H
@@ -20,7 +21,7 @@ def _declared():
 def test_library_exports_every_declared_symbol():
     lib = H.load()
     names = _declared()
-    assert len(names) == len(H.EXPORTED) == 14
+    assert len(names) == len(H.EXPORTED) == 15
     assert set(names) == set(H.EXPORTED)
     for n in names:
         assert getattr(lib, n) is not None
@@ -126,6 +127,28 @@ def test_backward_arguments_are_rejected_before_launch():
     assert bwd(sbs=-16) == H.ERR_INVALID_ARG
     assert bwd(sbs=8) == H.ERR_MISALIGNED
     assert bwd(prob=H.problem((48, 64), 2, 3)) == H.ERR_UNSUPPORTED
+
+
+def test_kernel_grad_arguments_are_rejected_before_launch():
+    p = H.problem((32, 16), 2, 3)
+    q, k, v, dy, dK, ws = _ptrs()
+    wsb = H.workspace_bytes(p)
+    assert H.kernel_grad(p, q, k, v, 0, dK, ws, wsb) == H.ERR_INVALID_ARG
+    assert H.kernel_grad(p, q, k, v, dy, 0, ws, wsb) == H.ERR_INVALID_ARG
+    assert H.kernel_grad(p, q, k, v, dy, dK + 4, ws, wsb) == H.ERR_MISALIGNED
+    assert H.kernel_grad(p, q, k, v, dy, dK, ws, wsb - 16) == H.ERR_WORKSPACE_TOO_SMALL
+    assert H.kernel_grad(p, q, k, v, dy, k + 64, ws, wsb) == H.ERR_INVALID_ARG     # dK overlaps k
+    assert H.kernel_grad(H.problem((24, 16), 2, 3), q, k, v, dy, dK, ws, wsb) == H.ERR_UNSUPPORTED
+
+
+def test_workspace_covers_the_kernel_gradient():
+    """The workspace of every grid holds at least one channel's kernel-gradient
+    grids: (2 B + 1) padded complex grids."""
+    for i in range(5):
+        wl = W.workload(i)
+        p = H.problem(wl.dims, wl.B, wl.C, H.BF16 if wl.io_dtype == "bf16" else H.F32)
+        P = int(np.prod([2 * n for n in wl.dims]))
+        assert H.workspace_bytes(p) >= (2 * wl.B + 1) * P * 8
 
 
 def test_single_volume_call_needs_b_and_c_of_one():

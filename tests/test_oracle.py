@@ -413,3 +413,59 @@ def test_backward_direct_at_points_matches_full():
     got = O.corr_direct_at(z, K, dims, pts)
     want = np.array([full[tuple(p)] for p in pts])
     assert np.max(np.abs(got - want)) < 1e-12
+
+
+# ------------------------------------------------------ kernel-value gradient
+@pytest.mark.parametrize("dims", [(6,), (4, 5), (3, 4, 3)])
+def test_kernel_grad_dft_equals_direct(dims):
+    q, k, v, _ = _rand_problem(dims, seed=51)
+    dy = np.random.default_rng(52).standard_normal(q.shape)
+    a = O.kernel_grad_dft(q, k, v, dy, dims)
+    b = O.kernel_grad_direct(q, k, v, dy, dims)
+    assert O.rel_l2(a, b) < 1e-12
+
+
+@pytest.mark.parametrize("dims", [(7,), (5, 4), (3, 3, 4)])
+def test_kernel_grad_matches_finite_differences(dims):
+    """L = sum dy y is linear in K: the central difference along a random
+    direction of K is exact up to rounding."""
+    q, k, v, K = _rand_problem(dims, seed=61)
+    rng = np.random.default_rng(62)
+    dy = rng.standard_normal(q.shape)
+    g = O.kernel_grad_direct(q, k, v, dy, dims)
+    D = rng.standard_normal(K.shape)
+
+    def L(KK):
+        return float(np.sum(dy * O.conv_direct(q, k, v, KK, dims)))
+
+    fd = (L(K + 0.5 * D) - L(K - 0.5 * D)) / 1.0
+    an = float(np.sum(g * D))
+    assert abs(fd - an) <= 1e-10 * max(1.0, abs(an))
+
+
+def test_kernel_grad_by_explicit_loops():
+    dims = (3, 4)
+    q, k, v, _ = _rand_problem(dims, B=2, C=1, seed=71)
+    dy = np.random.default_rng(72).standard_normal(q.shape)
+    g = O.kernel_grad_direct(q, k, v, dy, dims)
+    for t0 in range(-2, 3):
+        for t1 in range(-3, 4):
+            s = 0.0
+            for b in range(2):
+                for i0 in range(3):
+                    for i1 in range(4):
+                        j0, j1 = i0 - t0, i1 - t1
+                        if 0 <= j0 < 3 and 0 <= j1 < 4:
+                            s += q[b, 0, i0, i1] * dy[b, 0, i0, i1] * k[b, 0, j0, j1] * v[b, 0, j0, j1]
+            assert abs(g[0, t0 + 2, t1 + 3] - s) < 1e-12
+
+
+def test_kernel_grad_at_points_matches_full():
+    dims = (5, 6)
+    q, k, v, _ = _rand_problem(dims, seed=81)
+    dy = np.random.default_rng(82).standard_normal(q.shape)
+    full = O.kernel_grad_direct(q, k, v, dy, dims)
+    pts = np.array([[0, -4, 5], [2, 0, 0], [1, 3, -2]])
+    got = O.kernel_grad_at(q, k, v, dy, dims, pts)
+    want = np.array([full[p[0], p[1] + 4, p[2] + 5] for p in pts])
+    assert np.max(np.abs(got - want)) < 1e-12
