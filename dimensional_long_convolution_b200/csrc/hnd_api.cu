@@ -32,6 +32,7 @@ struct Plan {
   int n[3] = {1, 1, 1};
   long long B = 0, C = 0;
   int bf16 = 0;
+  int circular = 0;
   long long L = 1;          // voxels per volume
   long long gsz = 1;        // padded grid points per channel
   long long spec_per = 0;   // complex values per channel spectrum
@@ -52,7 +53,7 @@ hyena_nd_status make_plan(const hyena_nd_problem* p, Plan* pl) {
   if (p->io_dtype != HYENA_ND_F32 && p->io_dtype != HYENA_ND_BF16) return HYENA_ND_ERR_INVALID_ARG;
   for (int a = 0; a < p->ndim; ++a)
     if (p->n[a] < 1) return HYENA_ND_ERR_INVALID_ARG;
-  if (p->circular != 0) return HYENA_ND_ERR_UNSUPPORTED;
+  if (p->circular != 0 && p->circular != 1) return HYENA_ND_ERR_INVALID_ARG;
   for (int a = 0; a < p->ndim; ++a)
     if (!pow2_in(p->n[a], 8, 256)) return HYENA_ND_ERR_UNSUPPORTED;
   if (p->ndim == 3 && (p->n[0] > 128 || p->n[1] > 128)) return HYENA_ND_ERR_UNSUPPORTED;
@@ -61,6 +62,7 @@ hyena_nd_status make_plan(const hyena_nd_problem* p, Plan* pl) {
   pl->B = p->B;
   pl->C = p->C;
   pl->bf16 = p->io_dtype == HYENA_ND_BF16;
+  pl->circular = p->circular;
   pl->L = 1;
   pl->gsz = 1;
   for (int a = 0; a < 3; ++a) pl->n[a] = 1;
@@ -280,8 +282,8 @@ hyena_nd_status hyena_nd_kernel_grad(const hyena_nd_problem* p, const void* q, c
   for (const void* ptr : ptrs)
     if (!aligned16(ptr)) return HYENA_ND_ERR_MISALIGNED;
   if (ws_bytes < pl.ws_total) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
-  long long noff = 1;
-  for (int a = 0; a < pl.ndim; ++a) noff *= 2 * pl.n[a] - 1;
+  long long noff = 1;     // dK entries per channel: linear offsets, or the periodic grid
+  for (int a = 0; a < pl.ndim; ++a) noff *= pl.circular ? pl.n[a] : 2 * pl.n[a] - 1;
   const size_t act_bytes = static_cast<size_t>(pl.B * pl.C * pl.L) * (pl.bf16 ? 2 : 4);
   const size_t dk_bytes = static_cast<size_t>(pl.C * noff) * 4;
   const void* ins[4] = {q, k, v, dy};
@@ -299,6 +301,7 @@ hyena_nd_status hyena_nd_kernel_grad(const hyena_nd_problem* p, const void* q, c
   g.B = static_cast<int>(pl.B);
   g.C = static_cast<int>(pl.C);
   g.bf16 = pl.bf16;
+  g.circular = pl.circular;
   for (long long c0 = 0; c0 < pl.C; c0 += pl.kgrad_chunk) {
     g.c0 = static_cast<int>(c0);
     g.ncc = static_cast<int>(pl.C - c0 < pl.kgrad_chunk ? pl.C - c0 : pl.kgrad_chunk);
@@ -331,6 +334,7 @@ hyena_nd_status hyena_nd_filter_spectrum(const hyena_nd_problem* p, const hyena_
   fl.hidden = f->hidden;
   fl.decay_scale = f->decay_scale;
   fl.window = f->window;
+  fl.circular = pl.circular;
   float2* grid = reinterpret_cast<float2*>(static_cast<char*>(ws) + kStatusBytes);
   for (long long c0 = 0; c0 < pl.C; c0 += pl.filter_chunk) {
     const int nc = static_cast<int>(pl.C - c0 < pl.filter_chunk ? pl.C - c0 : pl.filter_chunk);

@@ -29,6 +29,7 @@ struct FilterMlpArgs {
   int num_freqs, hidden, fin;    // fin = 2 num_freqs ndim
   float decay_scale;
   int window;                    // 0: exp(-alpha |t| / s), 1: exp(-alpha (|t| / s)^2)
+  int circular;                  // 1: evaluate at each offset's periodic representative
   int ndim;
   int n[3];
   int c0, nc;                    // channel chunk [c0, c0 + nc)
@@ -76,6 +77,10 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
     const int i0 = static_cast<int>(r / E1);
     t0 = i0 - (n0 - 1), t1 = i1 - (n1 - 1), t2 = i2 - (n2 - 1);
   };
+  // circular mode: the network sees the representative of t mod n in
+  // [-n/2, n/2) (the linear offsets t and t - n then carry the same value,
+  // which makes the linear convolution on the 2n grid the circular one)
+  auto rep = [&](int t, int n) { return a.circular ? ((t + n / 2) % n + n) % n - n / 2 : t; };
 
   // first layer weights (zero-padded to HP hidden units: sin(0) = 0 and the
   // padded output weights are zero, so the padding contributes nothing)
@@ -88,7 +93,8 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
   for (int o = tid; o < kFO; o += kFT) {
     int t0, t1, t2;
     offset_of(o, t0, t1, t2);
-    const float f0 = static_cast<float>(t0), f1 = static_cast<float>(t1), f2 = static_cast<float>(t2);
+    const float f0 = static_cast<float>(rep(t0, n0)), f1 = static_cast<float>(rep(t1, n1)),
+                f2 = static_cast<float>(rep(t2, n2));
     // the window's argument |t| / s, squared for the Gaussian window
     const float rs = sqrtf(f0 * f0 + f1 * f1 + f2 * f2) / a.decay_scale;
     rad[o] = a.window == 1 ? rs * rs : rs;
@@ -101,8 +107,8 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
     const int o = i % kFO, q = i / kFO, m = q % M + 1, ax = q / M;
     int t0, t1, t2;
     offset_of(o, t0, t1, t2);
-    const int tax = ax == 0 ? t0 : (ax == 1 ? t1 : t2);
     const int nax = ax == 0 ? n0 : (ax == 1 ? n1 : n2);
+    const int tax = rep(ax == 0 ? t0 : (ax == 1 ? t1 : t2), nax);
     float sv, cv;
     sincospif(static_cast<float>(m) * (static_cast<float>(tax) / static_cast<float>(nax)), &sv, &cv);
     phi[(2 * (ax * M + m - 1)) * kFO + o] = sv;

@@ -85,4 +85,32 @@ static __global__ void k_kg_extract(const float2* __restrict__ acc, float* __res
   }
 }
 
+// Circular mode: dKper[c, tau] = sum of dK over the linear offsets t with
+// t = tau mod n (t_a in {tau_a, tau_a - n} within [-(n_a - 1), n_a - 1]).
+static __global__ void k_kg_extract_periodic(const float2* __restrict__ acc, float* __restrict__ dK, KgDims d, int c0,
+                                             int ncc, float scale) {
+  const long long nper = static_cast<long long>(d.n0) * d.n1 * d.n2;
+  const long long gsz = static_cast<long long>(d.P0) * d.P1 * d.P2;
+  const long long total = nper * ncc;
+  for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long c = e / nper, off = e % nper;
+    long long r = off;
+    const int u2 = static_cast<int>(r % d.n2);
+    r /= d.n2;
+    const int u1 = static_cast<int>(r % d.n1);
+    const int u0 = static_cast<int>(r / d.n1);
+    float sum = 0.f;
+    for (int k0 = 0; k0 < (u0 > 0 ? 2 : 1); ++k0)
+      for (int k1 = 0; k1 < (u1 > 0 ? 2 : 1); ++k1)
+        for (int k2 = 0; k2 < (u2 > 0 ? 2 : 1); ++k2) {
+          const int t0 = u0 - k0 * d.n0, t1 = u1 - k1 * d.n1, t2 = u2 - k2 * d.n2;
+          const long long slot = (static_cast<long long>((t0 + d.P0) % d.P0) * d.P1 + (t1 + d.P1) % d.P1) * d.P2 +
+                                 (t2 + d.P2) % d.P2;
+          sum += acc[c * gsz + slot].x;
+        }
+    dK[(c0 + c) * nper + off] = sum * scale;
+  }
+}
+
 }  // namespace hnd2

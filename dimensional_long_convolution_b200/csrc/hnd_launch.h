@@ -56,6 +56,7 @@ struct FilterLaunch {
   int num_freqs, hidden;
   float decay_scale;
   int window = 0;         // 0: exp(-alpha |t| / s), 1: exp(-alpha (|t| / s)^2)
+  int circular = 0;       // 1: periodic representatives (circular mode)
 };
 cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, int c0, int nc, float2* grid,
                                 void* spectrum, cudaStream_t st);
@@ -71,6 +72,7 @@ struct KgradLaunch {
   float* dK;              // [C][2n-1 ...]
   float2* grids;          // (2 B + 1) ncc grids of P^d complex
   int ndim, n[3], B, C, c0, ncc, bf16;
+  int circular;           // 1: fold onto the periodic grid, dK [C][n ...]
 };
 cudaError_t launch_kgrad_chunk(const KgradLaunch& g, cudaStream_t st);
 cudaError_t launch_bounded_wait(int* status, const int* flag, long long limit_cycles, cudaStream_t st);

@@ -85,7 +85,7 @@ extern "C" HYENA_ND_API hyena_nd_status hyena_nd_fftconv_batched_static(
   if (p->io_dtype != HYENA_ND_F32 && p->io_dtype != HYENA_ND_BF16) return HYENA_ND_ERR_INVALID_ARG;
   for (int a = 0; a < p->ndim; ++a)
     if (p->n[a] < 1) return HYENA_ND_ERR_INVALID_ARG;
-  if (p->circular != 0) return HYENA_ND_ERR_UNSUPPORTED;
+  if (p->circular != 0 && p->circular != 1) return HYENA_ND_ERR_INVALID_ARG;
   for (int a = 0; a < p->ndim; ++a)
     if (!pow2_in(p->n[a], 8, 256)) return HYENA_ND_ERR_UNSUPPORTED;
   if (p->ndim == 3 && (p->n[0] > 128 || p->n[1] > 128)) return HYENA_ND_ERR_UNSUPPORTED;

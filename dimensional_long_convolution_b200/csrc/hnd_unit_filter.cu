@@ -88,6 +88,7 @@ cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, i
   fa.fin = 2 * f.num_freqs * ndim;
   fa.decay_scale = f.decay_scale;
   fa.window = f.window;
+  fa.circular = f.circular;
   fa.ndim = ndim;
   for (int a = 0; a < 3; ++a) fa.n[a] = a < ndim ? n[a] : 1;
   fa.c0 = c0;
@@ -143,10 +144,15 @@ static cudaError_t kgrad_chunk_t(const KgradLaunch& g, cudaStream_t st) {
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   e = launch_fft_axes(acc, g.ndim, g.n, g.ncc, st);
   if (e != cudaSuccess) return e;
-  long long noff = 1;
-  for (int a = 0; a < g.ndim; ++a) noff *= 2 * g.n[a] - 1;
-  hnd2::k_kg_extract<<<grid_for(noff * g.ncc, 256), 256, 0, st>>>(acc, g.dK, d, g.c0, g.ncc,
-                                                                    static_cast<float>(1.0 / static_cast<double>(gsz)));
+  const float scale = static_cast<float>(1.0 / static_cast<double>(gsz));
+  if (g.circular) {
+    const long long nper = static_cast<long long>(d.n0) * d.n1 * d.n2;
+    hnd2::k_kg_extract_periodic<<<grid_for(nper * g.ncc, 256), 256, 0, st>>>(acc, g.dK, d, g.c0, g.ncc, scale);
+  } else {
+    long long noff = 1;
+    for (int a = 0; a < g.ndim; ++a) noff *= 2 * g.n[a] - 1;
+    hnd2::k_kg_extract<<<grid_for(noff * g.ncc, 256), 256, 0, st>>>(acc, g.dK, d, g.c0, g.ncc, scale);
+  }
   return cudaGetLastError();
 }
 

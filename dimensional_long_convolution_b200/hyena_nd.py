@@ -210,7 +210,7 @@ class HyenaND:
     """One problem shape bound to a device: owns the spectrum and workspace
     tensors (allocated by torch) and calls the C ABI on the current stream."""
 
-    def __init__(self, dims: Sequence[int], B: int, C: int, io_dtype: str = "f32", device=None):
+    def __init__(self, dims: Sequence[int], B: int, C: int, io_dtype: str = "f32", device=None, circular: int = 0):
         import torch
 
         self.torch = torch
@@ -218,7 +218,8 @@ class HyenaND:
         self.B, self.C = int(B), int(C)
         self.io_dtype = io_dtype
         self.tdtype = torch.bfloat16 if io_dtype == "bf16" else torch.float32
-        self.p = problem(self.dims, B, C, BF16 if io_dtype == "bf16" else F32)
+        self.circular = int(circular)
+        self.p = problem(self.dims, B, C, BF16 if io_dtype == "bf16" else F32, circular=self.circular)
         dev = torch.device(device if device is not None else "cuda")
         if dev.type == "cuda" and dev.index is None:
             dev = torch.device("cuda", torch.cuda.current_device())
@@ -286,13 +287,14 @@ class HyenaND:
         return dq, dk, dv
 
     def kernel_grad(self, q, k, v, dy):
-        """dK [C, 2n-1, ...] (float32): the gradient of the loss with respect to
-        the kernel values, for the loss gradient dy of __call__'s output."""
+        """dK (float32): the gradient of the loss with respect to the kernel
+        values, for the loss gradient dy of __call__'s output; [C, 2n-1, ...]
+        on the linear offsets, [C, n...] on the periodic grid when circular."""
         for t in (q, k, v, dy):
             if t.dtype != self.tdtype or not t.is_contiguous() or t.device != self.device:
                 raise ValueError("q, k, v, dy must be contiguous %s tensors on %s" % (self.tdtype, self.device))
-        dK = self.torch.empty((self.C,) + tuple(2 * n - 1 for n in self.dims), dtype=self.torch.float32,
-                              device=self.device)
+        shape = tuple(self.dims) if self.circular else tuple(2 * n - 1 for n in self.dims)
+        dK = self.torch.empty((self.C,) + shape, dtype=self.torch.float32, device=self.device)
         check(kernel_grad(self.p, q.data_ptr(), k.data_ptr(), v.data_ptr(), dy.data_ptr(), dK.data_ptr(),
                           self.ws.data_ptr(), self.ws_bytes, self._stream()), "kernel_grad")
         return dK

@@ -71,8 +71,17 @@ typedef enum { HYENA_ND_F32 = 0, HYENA_ND_BF16 = 1 } hyena_nd_dtype;
  *            for ndim == 3 the two outer axes are limited to [8, 128].
  *   B, C     batch and channel counts (>= 1).
  *   io_dtype dtype of q, k, v and y.
- *   circular must be 0 (zero-padded linear convolution); the periodic mode of
- *            the pages is not implemented and returns HYENA_ND_ERR_UNSUPPORTED. */
+ *   circular 0: zero-padded linear convolution.  1: circular (periodic)
+ *            convolution y[i] = q[i] sum_j u[j] Kper[(i - j) mod n] (arXiv
+ *            2607.19378 summary, "Methodologie", boundary handling: circular
+ *            convolutions for periodic systems).  The filter call then
+ *            evaluates the network at each offset's representative in
+ *            [-n/2, n/2), which gives the periodic kernel on the linear
+ *            offsets (t and t - n carry the same value); the convolution
+ *            calls are unchanged, since for i, j in [0, n) the linear sum
+ *            over K[i - j] is then the circular one.  It runs through the
+ *            same 2n grid as the linear mode.  Other values:
+ *            HYENA_ND_ERR_INVALID_ARG. */
 typedef struct {
   int ndim;
   int64_t n[3];
@@ -183,7 +192,9 @@ HYENA_ND_API hyena_nd_status hyena_nd_fftconv_backward(const hyena_nd_problem* p
  * arithmetic; the sum over b runs in a fixed order (deterministic).
  * q, k, v, dy: [B, C, n...] in the problem's dtype, read.  dK: float32
  * [C, 2n_1-1, ..., 2n_d-1] (index t + n - 1), written; it may not overlap an
- * input.  The chain into the filter's parameters is the caller's (the filter
+ * input.  Circular problems: dK is the gradient with respect to the periodic
+ * kernel, dKper[c, tau] = sum_b sum_i q dy[i] u[(i - tau) mod n], float32
+ * [C, n_1, ..., n_d] (the linear offsets t = tau mod n summed).  The chain into the filter's parameters is the caller's (the filter
  * call is its forward).  `ws`: hyena_nd_workspace_bytes(p) bytes. */
 HYENA_ND_API hyena_nd_status hyena_nd_kernel_grad(const hyena_nd_problem* p, const void* q, const void* k,
                                      const void* v, const void* dy, float* dK, void* ws, size_t ws_bytes,

@@ -93,6 +93,48 @@ def implicit_kernel(filt, dims: Sequence[int], channels=None, chunk: int = 1 << 
     return K.reshape((len(sel),) + tuple(2 * n - 1 for n in dims))
 
 
+def periodic_rep(t: np.ndarray, n: int) -> np.ndarray:
+    """The representative of t mod n in [-n/2, n/2): the offset the periodic
+    (circular) mode evaluates the filter at."""
+    return (t + n // 2) % n - n // 2
+
+
+def implicit_kernel_periodic(filt, dims: Sequence[int], channels=None, window: int = 0) -> np.ndarray:
+    """Circular mode (arXiv 2607.19378 summary, "Methodologie", boundary
+    handling: circular convolutions for periodic systems): the kernel on the
+    periodic grid, Kper[c, tau] for tau in [0, n)^d, is the filter evaluated at
+    each tau's representative in [-n/2, n/2) per axis (reading: the window
+    then decays with the periodic distance).  Returns [C, n_1, ..., n_d]."""
+    d = len(dims)
+    taus = np.stack(np.meshgrid(*[np.arange(n) for n in dims], indexing="ij"), axis=-1).reshape(-1, d)
+    reps = np.stack([periodic_rep(taus[:, a], n) for a, n in enumerate(dims)], axis=-1)
+    full = implicit_kernel(filt, dims, channels=channels, window=window)      # [C, 2n-1, ...]
+    idx = tuple(reps[:, a] + n - 1 for a, n in enumerate(dims))
+    out = full[(slice(None),) + idx]
+    return out.reshape((out.shape[0],) + tuple(dims))
+
+
+def periodize_to_offsets(Kper: np.ndarray, dims: Sequence[int]) -> np.ndarray:
+    """K_lin[t] = Kper[t mod n] on the linear offsets t in [-(n-1), n-1]^d:
+    for i, j in [0, n) the circular sum over Kper[(i - j) mod n] equals the
+    linear sum over K_lin[i - j]."""
+    idx = [np.arange(-(n - 1), n) % n for n in dims]
+    return Kper[np.ix_(np.arange(Kper.shape[0]), *idx)]
+
+
+def kernel_grad_periodic_direct(q, k, v, dy, dims) -> np.ndarray:
+    """dKper[c, tau] = sum_b sum_i q dy[b,c,i] u[b,c,(i - tau) mod n]: the
+    kernel gradient of the circular mode, from its definition (one tau at a
+    time).  Returns [C, n...]."""
+    z, u = q * dy, k * v
+    d = len(dims)
+    out = np.zeros((q.shape[1],) + tuple(dims))
+    for tau in itertools.product(*[range(n) for n in dims]):
+        us = np.roll(u, shift=tau, axis=tuple(range(2, 2 + d)))          # us[i] = u[(i - tau) mod n]
+        out[(slice(None),) + tau] = np.sum(z * us, axis=(0,) + tuple(range(2, 2 + d)))
+    return out
+
+
 def wrap_place(K: np.ndarray, dims: Sequence[int]) -> np.ndarray:
     """Place K (offsets [-(n-1), n-1] per axis) on the padded periodic grid
     P_a = 2 n_a: offset t goes to slot t mod P_a; slot n_a stays 0 (reading 2)."""

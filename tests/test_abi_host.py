@@ -56,7 +56,7 @@ def test_sizes_of_the_benchmark_grids(i):
     ((256, 64, 64), 1, 1, 0, 0, False),       # outer 3D axis above 128
     ((64, 64), 0, 1, 0, 0, False),            # B < 1
     ((64, 64), 1, 1, 7, 0, False),            # unknown dtype
-    ((64, 64), 1, 1, 0, 1, False),            # circular mode not implemented
+    ((64, 64), 1, 1, 0, 1, True),             # circular mode
 ])
 def test_workspace_bytes_is_zero_for_invalid_problems(dims, B, C, dt, circ, want):
     p = H.problem(dims, B, C, dt, circ)
@@ -101,8 +101,8 @@ def test_invalid_arguments_are_rejected_before_launch():
     assert _call(p, q, k, v, s, y, ws, wsb, sbs=8) == H.ERR_MISALIGNED
     bad = H.problem((48, 64), 2, 3)
     assert _call(bad, q, k, v, s, y, ws, wsb) == H.ERR_UNSUPPORTED
-    circ = H.problem((64, 64), 2, 3, circular=1)
-    assert _call(circ, q, k, v, s, y, ws, wsb) == H.ERR_UNSUPPORTED
+    circ = H.problem((64, 64), 2, 3, circular=2)
+    assert _call(circ, q, k, v, s, y, ws, wsb) == H.ERR_INVALID_ARG
 
 
 def test_backward_arguments_are_rejected_before_launch():

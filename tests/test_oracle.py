@@ -3,6 +3,8 @@ itself: brute force, numpy library routines, closed forms and invariants of the
 gated linear convolution y[i] = q[i] sum_j k[j] v[j] K[i - j]
 (HyenaND blog, section "HyenaND", output equation; zero-padded linear mode from
 the arXiv 2607.19378 summary, "Methodologie", boundary handling)."""
+import itertools
+
 import numpy as np
 import pytest
 
@@ -469,3 +471,66 @@ def test_kernel_grad_at_points_matches_full():
     got = O.kernel_grad_at(q, k, v, dy, dims, pts)
     want = np.array([full[p[0], p[1] + 4, p[2] + 5] for p in pts])
     assert np.max(np.abs(got - want)) < 1e-12
+
+
+# -------------------------------------------------------------- circular mode
+@pytest.mark.parametrize("dims", [(8,), (4, 6), (4, 2, 4)])
+def test_circular_equals_linear_with_periodized_kernel(dims):
+    """sum_j u[j] Kper[(i - j) mod n] = sum_j u[j] K_lin[i - j] for i, j in
+    [0, n): the circular DFT route against the linear direct sum."""
+    rng = np.random.default_rng(91)
+    shape = (2, 3) + dims
+    q, k, v = (rng.standard_normal(shape) for _ in range(3))
+    Kper = rng.standard_normal((3,) + dims)
+    yc = O.conv_circular(q, k, v, Kper, dims)
+    yl = O.conv_direct(q, k, v, O.periodize_to_offsets(Kper, dims), dims)
+    assert O.rel_l2(yc, yl) < 1e-12
+
+
+def test_circular_direct_by_explicit_loops():
+    dims = (3, 4)
+    rng = np.random.default_rng(92)
+    q, k, v = (rng.standard_normal((1, 1) + dims) for _ in range(3))
+    Kper = rng.standard_normal((1,) + dims)
+    y = O.conv_circular(q, k, v, Kper, dims)
+    for i0 in range(3):
+        for i1 in range(4):
+            s = sum(k[0, 0, j0, j1] * v[0, 0, j0, j1] * Kper[0, (i0 - j0) % 3, (i1 - j1) % 4]
+                    for j0 in range(3) for j1 in range(4))
+            assert abs(y[0, 0, i0, i1] - q[0, 0, i0, i1] * s) < 1e-12
+
+
+def test_periodic_kernel_takes_the_centred_representative():
+    dims = (8, 4)
+    p = _params(2, 32)
+    Kp = O.implicit_kernel_periodic(p, dims)
+    K = O.implicit_kernel(p, dims)
+    # tau = (5, 3) -> representatives (-3, -1)
+    assert np.array_equal(Kp[:, 5, 3], K[:, 7 - 3, 3 - 1])
+    # tau = (4, 2) -> (-4, -2): the half-way offset is taken as negative
+    assert np.array_equal(Kp[:, 4, 2], K[:, 7 - 4, 3 - 2])
+    assert np.array_equal(Kp[:, 0, 0], K[:, 7, 3])
+
+
+@pytest.mark.parametrize("dims", [(6,), (4, 3)])
+def test_periodic_kernel_grad_folds_the_linear_one(dims):
+    """dKper[tau] = sum over linear offsets t = tau mod n of dK[t], and it
+    matches exact finite differences of the circular forward."""
+    rng = np.random.default_rng(93)
+    shape = (2, 2) + dims
+    q, k, v, dy = (rng.standard_normal(shape) for _ in range(4))
+    g = O.kernel_grad_periodic_direct(q, k, v, dy, dims)
+    lin = O.kernel_grad_direct(q, k, v, dy, dims)
+    fold = np.zeros_like(g)
+    for t in itertools.product(*[range(-(n - 1), n) for n in dims]):
+        fold[(slice(None),) + tuple(ta % n for ta, n in zip(t, dims))] += \
+            lin[(slice(None),) + tuple(ta + n - 1 for ta, n in zip(t, dims))]
+    assert np.max(np.abs(fold - g)) < 1e-11
+    Kper = rng.standard_normal((2,) + dims)
+    D = rng.standard_normal(Kper.shape)
+
+    def L(KK):
+        return float(np.sum(dy * O.conv_circular(q, k, v, KK, dims)))
+
+    fd = (L(Kper + 0.5 * D) - L(Kper - 0.5 * D)) / 1.0
+    assert abs(fd - float(np.sum(g * D))) <= 1e-10 * max(1.0, abs(fd))
