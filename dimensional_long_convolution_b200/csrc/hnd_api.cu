@@ -25,7 +25,9 @@ constexpr size_t kFilterBudget = size_t(64) << 20;    // filter grid per channel
 constexpr int kFilterMaxChunk = 64;
 constexpr size_t kKgradBudget = size_t(128) << 20;    // kernel-gradient grids per channel chunk
 
-enum Tier { kRows1D = 0, kFused2D = 1, kMulti2D = 2, kMulti3D = 3 };
+enum Tier { kRows1D = 0, kFused2D = 1, kMulti2D = 2, kMulti3D = 3, kLong1D = 4 };
+
+constexpr long long kLong1DMax = 131072;   // two four-step levels of at most 512 points
 
 struct Plan {
   int ndim = 0;
@@ -42,6 +44,7 @@ struct Plan {
   int kgrad_chunk = 1;      // channels per kernel-gradient chunk
   size_t ws_total = 0;
   size_t spec_bytes = 0;
+  size_t nat_bytes = 0;     // natural-order half spectrum (export / import)
 };
 
 bool pow2_in(long long x, long long lo, long long hi) { return x >= lo && x <= hi && (x & (x - 1)) == 0; }
@@ -54,8 +57,12 @@ hyena_nd_status make_plan(const hyena_nd_problem* p, Plan* pl) {
   for (int a = 0; a < p->ndim; ++a)
     if (p->n[a] < 1) return HYENA_ND_ERR_INVALID_ARG;
   if (p->circular != 0 && p->circular != 1) return HYENA_ND_ERR_INVALID_ARG;
-  for (int a = 0; a < p->ndim; ++a)
-    if (!pow2_in(p->n[a], 8, 256)) return HYENA_ND_ERR_UNSUPPORTED;
+  if (p->ndim == 1) {
+    if (!pow2_in(p->n[0], 8, kLong1DMax)) return HYENA_ND_ERR_UNSUPPORTED;
+  } else {
+    for (int a = 0; a < p->ndim; ++a)
+      if (!pow2_in(p->n[a], 8, 256)) return HYENA_ND_ERR_UNSUPPORTED;
+  }
   if (p->ndim == 3 && (p->n[0] > 128 || p->n[1] > 128)) return HYENA_ND_ERR_UNSUPPORTED;
   if (p->B > INT_MAX / p->C) return HYENA_ND_ERR_UNSUPPORTED;
   pl->ndim = p->ndim;
@@ -72,14 +79,24 @@ hyena_nd_status make_plan(const hyena_nd_problem* p, Plan* pl) {
     pl->gsz *= 2 * p->n[a];
   }
   const int nl = pl->n[p->ndim - 1];
-  if (p->ndim == 1) pl->spec_per = nl + 1;
+  if (p->ndim == 1) pl->spec_per = nl > 256 ? 2LL * nl : nl + 1;   // long 1D: the full four-step spectrum
   else if (p->ndim == 2) pl->spec_per = static_cast<long long>(nl + 1) * 2 * pl->n[0];
   else pl->spec_per = static_cast<long long>(nl + 1) * 4 * pl->n[0] * pl->n[1];
   pl->spec_bytes = static_cast<size_t>(pl->spec_per) * 8 * static_cast<size_t>(p->C);
+  pl->nat_bytes = static_cast<size_t>(pl->gsz / (2 * nl) * (nl + 1)) * 8 * static_cast<size_t>(p->C);
 
   const long long pairs = p->B * p->C;
   size_t ws_conv = 0;
-  if (p->ndim == 1) {
+  if (p->ndim == 1 && nl > 256) {
+    pl->tier = kLong1D;
+    const size_t per_vol = static_cast<size_t>(8) * static_cast<size_t>(pl->gsz);
+    long long w = static_cast<long long>(kWaveBudget / per_vol);
+    if (w < 1) w = 1;
+    if (w > pairs) w = pairs;
+    const long long nw = (pairs + w - 1) / w;
+    pl->wave = (pairs + nw - 1) / nw;   // equal waves
+    ws_conv = per_vol * static_cast<size_t>(pl->wave);
+  } else if (p->ndim == 1) {
     pl->tier = kRows1D;
   } else if (hnd::fused_2d(p->ndim, pl->n)) {
     pl->tier = kFused2D;
@@ -137,7 +154,9 @@ hyena_nd_status cuda_status(cudaError_t e) { return e == cudaSuccess ? HYENA_ND_
 // spectrum) on the plan's tier; adds the kernel launches to *launches.
 cudaError_t run_conv(const Plan& pl, const hnd::ConvArgs& a, void* ws, int* launches) {
   cudaError_t e = cudaSuccess;
-  if (pl.tier == kRows1D) {
+  if (pl.tier == kLong1D) {
+    e = hnd::launch_long1d(a, reinterpret_cast<float2*>(static_cast<char*>(ws) + kStatusBytes), pl.wave, launches);
+  } else if (pl.tier == kRows1D) {
     e = hnd::launch_rows1d(a);
     *launches += 1;
   } else if (pl.tier == kFused2D) {
@@ -352,7 +371,9 @@ static hyena_nd_status spec_convert(const hyena_nd_problem* p, const void* src, 
   if (st != HYENA_ND_OK) return st;
   if (!src || !dst) return HYENA_ND_ERR_INVALID_ARG;
   if (!aligned16(src) || !aligned16(dst)) return HYENA_ND_ERR_MISALIGNED;
-  if (overlaps(src, dst, pl.spec_bytes)) return HYENA_ND_ERR_INVALID_ARG;
+  const size_t src_bytes = to_natural ? pl.spec_bytes : pl.nat_bytes;
+  const size_t dst_bytes = to_natural ? pl.nat_bytes : pl.spec_bytes;
+  if (overlaps2(src, src_bytes, dst, dst_bytes)) return HYENA_ND_ERR_INVALID_ARG;
   return cuda_status(hnd::launch_spec_convert(pl.ndim, pl.n, pl.C, src, dst, to_natural,
                                               static_cast<cudaStream_t>(cuda_stream)));
 }

@@ -62,6 +62,12 @@ cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, i
                                 void* spectrum, cudaStream_t st);
 cudaError_t launch_spec_convert(int ndim, const int* n, long long C, const void* src, void* dst, bool to_natural,
                                 cudaStream_t st);
+// In-place full forward transform along one axis of `ngrids` grids [P^d].
+cudaError_t launch_fft_axis(float2* grid, int ndim, const int* n, int axis, long long ngrids, cudaStream_t st);
+// Long 1D tier (n > 256): the four-step split P = 2n = P0 P1, and one
+// convolution over all volumes in waves of `wave` grids (9 launches a wave).
+void long1d_split(int n, int* P0, int* P1);
+cudaError_t launch_long1d(const ConvArgs& a, float2* grid, long long wave, int* launches);
 // In-place full forward transforms along every axis of `ngrids` complex grids
 // [P^d] (P_a = 2 n_a), adjacent in memory.
 cudaError_t launch_fft_axes(float2* grid, int ndim, const int* n, long long ngrids, cudaStream_t st);

@@ -3,6 +3,7 @@
 #include "hnd_multi2.cuh"
 #include "hnd_filter2.cuh"
 #include "hnd_kgrad.cuh"
+#include "hnd_long1d.cuh"
 #include "hnd_launch.h"
 #include "hnd_host_util.h"
 
@@ -44,6 +45,89 @@ static cudaError_t fft_axis_go(float2* grid, long long stride, long long npen, c
   if (blocks > 148LL * 16) blocks = 148LL * 16;
   kern<<<static_cast<unsigned>(blocks), hnd2::kAT, sm, st>>>(grid, stride, npen);
   return cudaGetLastError();
+}
+
+cudaError_t launch_fft_axis(float2* grid, int ndim, const int* n, int axis, long long ngrids, cudaStream_t st) {
+  long long gsz = 1, stride = 1;
+  for (int a = 0; a < ndim; ++a) gsz *= 2 * n[a];
+  for (int a = axis + 1; a < ndim; ++a) stride *= 2 * n[a];
+  const long long npen = gsz * ngrids / (2 * n[axis]);
+  switch (n[axis]) {
+    case 8: return fft_axis_go<8>(grid, stride, npen, st);
+    case 16: return fft_axis_go<16>(grid, stride, npen, st);
+    case 32: return fft_axis_go<32>(grid, stride, npen, st);
+    case 64: return fft_axis_go<64>(grid, stride, npen, st);
+    case 128: return fft_axis_go<128>(grid, stride, npen, st);
+    case 256: return fft_axis_go<256>(grid, stride, npen, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// ------------------------------------------------------------ long 1D
+void long1d_split(int n, int* P0, int* P1) {
+  const long long P = 2LL * n;
+  int lg = 0;
+  while ((1LL << lg) < P) ++lg;
+  *P0 = 1 << (lg / 2);
+  *P1 = static_cast<int>(P / *P0);
+}
+
+// forward four-step on `ngrids` adjacent grids of P = P0 P1
+static cudaError_t four_step_fwd(float2* grid, int P0, int P1, long long ngrids, cudaStream_t st) {
+  const int h[2] = {P0 / 2, P1 / 2};
+  cudaError_t e = launch_fft_axis(grid, 2, h, 0, ngrids, st);
+  if (e != cudaSuccess) return e;
+  hnd2::k_l1_twiddle<<<grid_for(static_cast<long long>(P0) * P1 * ngrids, 256), 256, 0, st>>>(grid, P0, P1, ngrids);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return launch_fft_axis(grid, 2, h, 1, ngrids, st);
+}
+
+// on conjugated spectra [k0][k1]: the conjugate of the unnormalised inverse,
+// in natural order i = P1 i0 + i1
+static cudaError_t four_step_inv_conj(float2* grid, int P0, int P1, long long ngrids, cudaStream_t st) {
+  const int h[2] = {P0 / 2, P1 / 2};
+  cudaError_t e = launch_fft_axis(grid, 2, h, 1, ngrids, st);
+  if (e != cudaSuccess) return e;
+  hnd2::k_l1_twiddle<<<grid_for(static_cast<long long>(P0) * P1 * ngrids, 256), 256, 0, st>>>(grid, P0, P1, ngrids);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return launch_fft_axis(grid, 2, h, 0, ngrids, st);
+}
+
+template <class T>
+static cudaError_t long1d_t(const ConvArgs& a, float2* grid, long long wave, int* launches) {
+  const int n = a.n[0];
+  int P0, P1;
+  long1d_split(n, &P0, &P1);
+  const long long P = 2LL * n, nv = static_cast<long long>(a.B) * a.C;
+  const T* q = static_cast<const T*>(a.q);
+  const T* k = static_cast<const T*>(a.k);
+  const T* v = static_cast<const T*>(a.v);
+  T* y = static_cast<T*>(a.y);
+  cudaError_t e = cudaSuccess;
+  for (long long v0 = 0; v0 < nv && e == cudaSuccess; v0 += wave) {
+    const int cnt = static_cast<int>(nv - v0 < wave ? nv - v0 : wave);
+    hnd2::k_l1_pad<T><<<grid_for(P * cnt, 256), 256, 0, a.stream>>>(k, v, grid, n, P, v0, cnt);
+    if ((e = cudaGetLastError()) != cudaSuccess) break;
+    if ((e = four_step_fwd(grid, P0, P1, cnt, a.stream)) != cudaSuccess) break;
+    hnd2::k_l1_modulate<<<grid_for(P * cnt, 256), 256, 0, a.stream>>>(grid, static_cast<const float2*>(a.spec), a.sbs,
+                                                                     a.sconj, P, a.C, v0, cnt);
+    if ((e = cudaGetLastError()) != cudaSuccess) break;
+    if ((e = four_step_inv_conj(grid, P0, P1, cnt, a.stream)) != cudaSuccess) break;
+    if (a.y2) {
+      hnd2::k_l1_out<T, true><<<grid_for(static_cast<long long>(n) * cnt, 256), 256, 0, a.stream>>>(
+          grid, q, y, static_cast<const T*>(a.g2), static_cast<T*>(a.y2), n, P, v0, cnt);
+    } else {
+      hnd2::k_l1_out<T, false><<<grid_for(static_cast<long long>(n) * cnt, 256), 256, 0, a.stream>>>(
+          grid, q, y, nullptr, nullptr, n, P, v0, cnt);
+    }
+    e = cudaGetLastError();
+    *launches += 9;
+  }
+  return e;
+}
+
+cudaError_t launch_long1d(const ConvArgs& a, float2* grid, long long wave, int* launches) {
+  return a.bf16 ? long1d_t<__nv_bfloat16>(a, grid, wave, launches) : long1d_t<float>(a, grid, wave, launches);
 }
 
 cudaError_t launch_fft_axes(float2* grid, int ndim, const int* n, long long ngrids, cudaStream_t st) {
@@ -100,6 +184,14 @@ cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, i
       : HP <= 96 ? filter_mlp_go<96>(fa, noff, st)
                  : filter_mlp_go<128>(fa, noff, st);
   if (e != cudaSuccess) return e;
+  if (ndim == 1 && n[0] > 256) {
+    int P0, P1;
+    long1d_split(n[0], &P0, &P1);
+    if ((e = four_step_fwd(grid, P0, P1, nc, st)) != cudaSuccess) return e;
+    hnd2::k_l1_spec_store<<<grid_for(gsz * nc, 256), 256, 0, st>>>(
+        grid, static_cast<float2*>(spectrum), gsz, c0, nc, static_cast<float>(1.0 / static_cast<double>(gsz)));
+    return cudaGetLastError();
+  }
   e = launch_fft_axes(grid, ndim, n, nc, st);
   if (e != cudaSuccess) return e;
   const long long per = spec_per_channel(d);
@@ -137,12 +229,18 @@ static cudaError_t kgrad_chunk_t(const KgradLaunch& g, cudaStream_t st) {
   const T* dy = static_cast<const T*>(g.dy);
   hnd2::k_kg_pad<T><<<grid_for(gsz * nvol, 256), 256, 0, st>>>(k, v, gu, d, g.B, g.C, g.c0, nvol);
   hnd2::k_kg_pad<T><<<grid_for(gsz * nvol, 256), 256, 0, st>>>(q, dy, gz, d, g.B, g.C, g.c0, nvol);
+  const bool long1d = g.ndim == 1 && g.n[0] > 256;
+  int P0 = 0, P1 = 0;
+  if (long1d) long1d_split(g.n[0], &P0, &P1);
   cudaError_t e = cudaGetLastError();
-  if (e == cudaSuccess) e = launch_fft_axes(gu, g.ndim, g.n, 2LL * nvol, st);      // gu and gz are adjacent
+  if (e == cudaSuccess)       // gu and gz are adjacent
+    e = long1d ? four_step_fwd(gu, P0, P1, 2LL * nvol, st) : launch_fft_axes(gu, g.ndim, g.n, 2LL * nvol, st);
   if (e != cudaSuccess) return e;
   hnd2::k_kg_corr<<<grid_for(gsz * g.ncc, 256), 256, 0, st>>>(gu, gz, acc, g.B, g.ncc, gsz);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  e = launch_fft_axes(acc, g.ndim, g.n, g.ncc, st);
+  // the accumulator holds conj(sum_b Z conj U): a forward transform gives the
+  // conjugate of the unnormalised inverse, whose real part is wanted
+  e = long1d ? four_step_inv_conj(acc, P0, P1, g.ncc, st) : launch_fft_axes(acc, g.ndim, g.n, g.ncc, st);
   if (e != cudaSuccess) return e;
   const float scale = static_cast<float>(1.0 / static_cast<double>(gsz));
   if (g.circular) {
@@ -162,6 +260,17 @@ cudaError_t launch_kgrad_chunk(const KgradLaunch& g, cudaStream_t st) {
 
 cudaError_t launch_spec_convert(int ndim, const int* n, long long C, const void* src, void* dst, bool to_natural,
                                 cudaStream_t st) {
+  if (ndim == 1 && n[0] > 256) {
+    int P0, P1;
+    long1d_split(n[0], &P0, &P1);
+    if (to_natural)
+      hnd2::k_l1_spec_export<<<grid_for((n[0] + 1LL) * C, 256), 256, 0, st>>>(
+          static_cast<const float2*>(src), static_cast<float2*>(dst), n[0], P0, P1, C);
+    else
+      hnd2::k_l1_spec_import<<<grid_for(2LL * n[0] * C, 256), 256, 0, st>>>(
+          static_cast<const float2*>(src), static_cast<float2*>(dst), n[0], P0, P1, C, n[0] + 1LL, 1.f);
+    return cudaGetLastError();
+  }
   const SpecDims d = make_dims(ndim, n);
   const long long total = spec_per_channel(d) * C;
   if (ndim == 3) {

@@ -68,7 +68,11 @@ typedef enum { HYENA_ND_F32 = 0, HYENA_ND_BF16 = 1 } hyena_nd_dtype;
 /* Problem descriptor.
  *   ndim     1, 2 or 3.
  *   n[a]     grid extent of axis a (a < ndim), a power of two in [8, 256];
- *            for ndim == 3 the two outer axes are limited to [8, 128].
+ *            for ndim == 3 the two outer axes are limited to [8, 128]; for
+ *            ndim == 1 any power of two in [8, 131072] (long 1D context:
+ *            n > 256 runs the padded length-2n transform as a four-step
+ *            split 2n = P0 P1 of two passes of at most 512 points, in waves
+ *            of volumes through the workspace).
  *   B, C     batch and channel counts (>= 1).
  *   io_dtype dtype of q, k, v and y.
  *   circular 0: zero-padded linear convolution.  1: circular (periodic)
@@ -228,8 +232,12 @@ HYENA_ND_API hyena_nd_status hyena_nd_fftconv_batched_static(const hyena_nd_prob
 
 /* Convert between the library's spectrum order and the natural order
  * [C, P_1, ..., P_{d-1}, P_d/2 + 1] complex64 (scale included, i.e. the
- * natural array is DFT(wrap-placed K) / prod(P)).  Both buffers are device
- * memory of hyena_nd_spectrum_bytes(p) bytes and may not alias. */
+ * natural array is DFT(wrap-placed K) / prod(P)).  The library-order buffer
+ * holds hyena_nd_spectrum_bytes(p) bytes, the natural one
+ * 8 C prod_{a<d} P_a (n_d + 1) bytes (the same number except for the long 1D
+ * tier, whose library order keeps all 2n frequencies); both are device memory
+ * and may not overlap.  The import takes the other half by Hermitian symmetry
+ * where the library order keeps it. */
 HYENA_ND_API hyena_nd_status hyena_nd_spectrum_export(const hyena_nd_problem* p, const void* spectrum,
                                          void* natural_c64, void* cuda_stream);
 HYENA_ND_API hyena_nd_status hyena_nd_spectrum_import(const hyena_nd_problem* p, const void* natural_c64,

@@ -182,6 +182,25 @@ def spectrum_half(K: np.ndarray, dims: Sequence[int]) -> np.ndarray:
     return S[..., : dims[-1] + 1]
 
 
+def spectrum_at(K: np.ndarray, dims: Sequence[int], points: np.ndarray) -> np.ndarray:
+    """The spectrum's definition at chosen frequencies only, for grids too long
+    for a dense DFT matrix: S[c, k] = (1/prod(P)) sum_t K_c[t]
+    exp(-2 pi i sum_a k_a (t_a mod P_a) / P_a) over every offset t (reading 5).
+    points: [M, 1 + d] rows (c, k_1..k_d).  Returns [M] complex128.  O(prod(2n-1))
+    per point; the phase index is reduced mod P_a first so the angle is exact."""
+    d = len(dims)
+    P = [2 * n for n in dims]
+    tgrid = np.stack(np.meshgrid(*[np.arange(-(n - 1), n) for n in dims], indexing="ij"), axis=-1).reshape(-1, d)
+    out = np.empty(points.shape[0], dtype=np.complex128)
+    for r, p in enumerate(points):
+        c = int(p[0])
+        ph = np.zeros(tgrid.shape[0], dtype=np.float64)
+        for a in range(d):
+            ph += np.mod(int(p[1 + a]) * np.mod(tgrid[:, a], P[a]), P[a]) / P[a]
+        out[r] = np.sum(K[c].reshape(-1) * np.exp(-2j * np.pi * ph)) / float(np.prod(P))
+    return out
+
+
 def full_from_half(Sh: np.ndarray, dims: Sequence[int]) -> np.ndarray:
     """Rebuild the full spectrum from the half by Hermitian symmetry
     S[-k] = conj(S[k]) of the transform of a real kernel."""

@@ -51,7 +51,11 @@ def test_sizes_of_the_benchmark_grids(i):
 @pytest.mark.parametrize("dims,B,C,dt,circ,want", [
     ((64, 64), 1, 1, 0, 0, True),
     ((300, 300), 1, 1, 0, 0, False),          # not a power of two
-    ((512,), 1, 1, 0, 0, False),              # above 256
+    ((512, 8), 1, 1, 0, 0, False),            # a 2D axis above 256
+    ((512,), 1, 1, 0, 0, True),               # long 1D context
+    ((131072,), 2, 4, 1, 1, True),            # longest 1D grid, circular
+    ((262144,), 1, 1, 0, 0, False),           # above the long 1D limit
+    ((3000,), 1, 1, 0, 0, False),             # long 1D, not a power of two
     ((4, 8), 1, 1, 0, 0, False),              # below 8
     ((256, 64, 64), 1, 1, 0, 0, False),       # outer 3D axis above 128
     ((64, 64), 0, 1, 0, 0, False),            # B < 1
@@ -149,6 +153,36 @@ def test_workspace_covers_the_kernel_gradient():
         p = H.problem(wl.dims, wl.B, wl.C, H.BF16 if wl.io_dtype == "bf16" else H.F32)
         P = int(np.prod([2 * n for n in wl.dims]))
         assert H.workspace_bytes(p) >= (2 * wl.B + 1) * P * 8
+
+
+@pytest.mark.parametrize("n,B,C", [(512, 2, 3), (4096, 1, 8), (131072, 2, 100)])
+def test_long_1d_sizes(n, B, C):
+    """Long 1D grids keep all 2n frequencies in the library order; the
+    workspace holds at least one volume's padded grid (one wave) and the
+    kernel-gradient grids of one channel; the natural export stays n + 1."""
+    p = H.problem((n,), B, C, H.F32)
+    assert H.spectrum_bytes(p) == C * 2 * n * 8
+    ws = H.workspace_bytes(p)
+    assert ws >= 256 + max(2 * n * 8, (2 * B + 1) * 2 * n * 8)
+    assert ws <= 256 + max(96 << 20, 128 << 20, (2 * B + 1) * 2 * n * 8)
+
+
+def test_long_1d_spectrum_conversion_uses_the_natural_size():
+    """The natural half spectrum of a long 1D grid is shorter than the library
+    order; the overlap check measures each buffer by its own size."""
+    n, C = 1024, 2
+    p = H.problem((n,), 1, C)
+    nat = C * (n + 1) * 8
+    nat16 = (nat + 15) // 16 * 16
+    assert H.spectrum_bytes(p) == C * 2 * n * 8
+    assert H.spectrum_import(p, A, A + nat16 - 16, 0) == H.ERR_INVALID_ARG
+    assert H.spectrum_export(p, A + nat16 - 16, A, 0) == H.ERR_INVALID_ARG
+
+
+def test_static_scratch_call_rejects_long_1d():
+    q, k, v, s, y, ws = _ptrs()
+    p = H.problem((1024,), 1, 1)
+    assert H.fftconv_batched_static(p, q, k, v, s, 0, y, 0) == H.ERR_UNSUPPORTED
 
 
 def test_single_volume_call_needs_b_and_c_of_one():

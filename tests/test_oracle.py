@@ -154,6 +154,45 @@ def test_spectrum_of_shifted_delta_is_a_phase_ramp():
     assert np.max(np.abs(S - want)) < 1e-15
 
 
+def test_spectrum_at_points_matches_numpy_fftn():
+    """The sampled definition against numpy's FFT of the wrap-placed kernel."""
+    dims = (5, 4, 3)
+    rng = np.random.default_rng(21)
+    K = rng.standard_normal((2,) + tuple(2 * n - 1 for n in dims))
+    full = np.fft.fftn(O.wrap_place(K, dims), axes=(1, 2, 3)) / np.prod([2 * n for n in dims])
+    pts = np.stack([rng.integers(0, 2, 20)] + [rng.integers(0, 2 * n, 20) for n in dims], axis=1)
+    got = O.spectrum_at(K, dims, pts)
+    want = np.array([full[tuple(p)] for p in pts])
+    assert np.max(np.abs(got - want)) < 1e-14
+
+
+def test_spectrum_at_of_shifted_delta_on_a_long_axis():
+    """Closed form on a 1D grid of the long-context size class: K = delta at
+    t0 gives exp(-2 pi i k t0 / P) / P at every frequency k."""
+    n, t0 = 4096, -1234
+    K = np.zeros((1, 2 * n - 1))
+    K[0, t0 + n - 1] = 1.0
+    ks = np.array([0, 1, 7, n - 1, n, n + 1, 2 * n - 1])
+    got = O.spectrum_at(K, (n,), np.stack([np.zeros_like(ks), ks], axis=1))
+    want = np.exp(-2j * np.pi * ks * t0 / (2 * n)) / (2 * n)
+    assert np.max(np.abs(got - want)) < 1e-15
+
+
+def test_long_1d_direct_at_points_matches_numpy_convolve():
+    """Sampled outputs of the definition on a long 1D grid against numpy's
+    full linear convolution (the crop keeps indices 0..n-1 of u * K shifted by
+    the kernel's centre n - 1)."""
+    n = 8192
+    rng = np.random.default_rng(22)
+    q, k, v = (rng.standard_normal((1, 1, n)) for _ in range(3))
+    K = rng.standard_normal((1, 2 * n - 1))
+    full = np.convolve((k * v)[0, 0], K[0])                 # index i + n - 1 holds output i
+    pts = np.array([[0, 0, i] for i in (0, 1, 777, n // 2, n - 2, n - 1)])
+    got = O.conv_direct_at(q, k, v, K, (n,), pts)
+    want = np.array([q[0, 0, i] * full[i + n - 1] for i in pts[:, 2]])
+    assert np.max(np.abs(got - want)) < 1e-10 * np.max(np.abs(want))
+
+
 # ------------------------------------------------------------------- invariants
 def test_linearity_in_v():
     dims = (6, 7)
