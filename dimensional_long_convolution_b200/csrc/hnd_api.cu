@@ -27,7 +27,7 @@ constexpr size_t kKgradBudget = size_t(128) << 20;    // kernel-gradient grids p
 
 enum Tier { kRows1D = 0, kFused2D = 1, kMulti2D = 2, kMulti3D = 3, kLong1D = 4 };
 
-constexpr long long kLong1DMax = 131072;   // two four-step levels of at most 512 points
+constexpr long long kLong1DMax = 1LL << 26;   // three split levels of at most 512 points
 
 struct Plan {
   int ndim = 0;

@@ -64,9 +64,15 @@ cudaError_t launch_spec_convert(int ndim, const int* n, long long C, const void*
                                 cudaStream_t st);
 // In-place full forward transform along one axis of `ngrids` grids [P^d].
 cudaError_t launch_fft_axis(float2* grid, int ndim, const int* n, int axis, long long ngrids, cudaStream_t st);
-// Long 1D tier (n > 256): the four-step split P = 2n = P0 P1, and one
-// convolution over all volumes in waves of `wave` grids (9 launches a wave).
-void long1d_split(int n, int* P0, int* P1);
+// Long 1D tier (n > 256): the split P = 2n = P0 P1 (P2) into m = 2 or 3
+// factors of at most 512 points (unused factors 1), and one convolution over
+// all volumes in waves of `wave` grids (3 + 2 (2m - 1) launches a wave).
+struct L1Split {
+  int m = 0;
+  int P[3] = {1, 1, 1};
+};
+L1Split long1d_split(int n);
+int long1d_launches_per_transform(int n);
 cudaError_t launch_long1d(const ConvArgs& a, float2* grid, long long wave, int* launches);
 // In-place full forward transforms along every axis of `ngrids` complex grids
 // [P^d] (P_a = 2 n_a), adjacent in memory.

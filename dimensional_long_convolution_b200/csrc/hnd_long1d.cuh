@@ -1,13 +1,18 @@
 // hnd_long1d.cuh -- 1D grids longer than one transform pencil (n in
-// [512, 131072]): the zero-padded length-P transform (P = 2n) as a four-step
-// factorisation P = P0 P1 on the [P0][P1] view of each volume's grid
-// (j = P1 j0 + j1):
-//   forward   transform along j0 (the padded half: j0 >= P0/2 is zero),
-//             twiddle W_P^{k0 j1}, transform along j1
-//             -> X(k0 + P0 k1) at [k0][k1] (the spectrum is kept in this order)
+// [512, 2^26]): the zero-padded length-P transform (P = 2n) as a multi-level
+// split P = P0 P1 (P2) with every factor at most 512, on the row-major view
+// [P0][P1][P2] of each volume's grid (j = (j0 P1 + j1) P2 + j2):
+//   forward   transform along axis 0 (the padded half j0 >= P0/2 is zero),
+//             twiddle W_P^{k0 r} (r the flattened later index), then the same
+//             split recursively on the later axes
+//             -> X(k0 + P0 k1 + P0 P1 k2) at [k0][k1][k2] (the spectrum is kept
+//             in this order)
 //   modulate  Y = X S (or X conj(S) for the adjoint), stored conjugated
-//   inverse   transform along k1, twiddle W_P^{k0 i1}, transform along k0:
-//             the conjugate of the unnormalised inverse at i = P1 i0 + i1
+//   inverse   the same steps in reverse order (last axis first, each twiddle
+//             after the transform of its level's later axes): every step is
+//             a symmetric operator, so the reversed chain applied to data in
+//             split order is the DFT in natural order; on conjugated data it
+//             gives the conjugate of the unnormalised inverse at i = j
 //   output    y[i] = q[i] Re(.) for i < n (the crop), optional second gate
 // (HyenaND pages: arXiv 2607.19378 summary, d = 1 long context through the
 // zero-padded FFT path; blog "Native multi-dimensional subquadratic operators
@@ -36,16 +41,17 @@ static __global__ void k_l1_pad(const T* __restrict__ a, const T* __restrict__ b
   }
 }
 
-// grid[g][r0][r1] *= W_P^{r0 r1} (W_P = exp(-2 pi i / P)), P = P0 P1
-static __global__ void k_l1_twiddle(float2* __restrict__ grid, int P0, int P1, long long ngrids) {
-  const long long P = static_cast<long long>(P0) * P1;
-  const long long total = P * ngrids;
+// Twiddle of level a of the split: on the view [..][P_a][R] (R = Q / P_a the
+// points of the later levels, Q = P_a R), element (k, r) *= W_Q^{k r},
+// W_Q = exp(-2 pi i / Q).  k r < Q, and Q is a power of two, so the angle is
+// the float ratio of two integers (exact while k r < 2^24).
+static __global__ void k_l1_twiddle(float2* __restrict__ grid, int Pa, long long Q, long long total) {
+  const long long R = Q / Pa;
   for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long r = e % P;
-    const long long m = ((r / P1) * (r % P1)) % P;
+    const long long m = ((e / R) % Pa) * (e % R);
     float s, c;
-    sincospif(-2.f * (static_cast<float>(m) / static_cast<float>(P)), &s, &c);   // exact ratio: P is 2^k
+    sincospif(-2.f * (static_cast<float>(m) / static_cast<float>(Q)), &s, &c);
     const float2 x = grid[e];
     grid[e] = make_float2(x.x * c - x.y * s, x.x * s + x.y * c);
   }
@@ -93,25 +99,31 @@ static __global__ void k_l1_spec_store(const float2* __restrict__ grid, float2* 
   }
 }
 
-// library order [C][P0][P1] (X(k0 + P0 k1) at k0 P1 + k1) <-> natural half
-// spectrum [C][n + 1]; the import fills the other half by Hermitian symmetry
+// library order [C][P0][P1][P2] (X(k0 + P0 k1 + P0 P1 k2) at (k0 P1 + k1) P2 + k2;
+// P2 = 1 for a two-level split) <-> natural half spectrum [C][n + 1]; the
+// import fills the other half by Hermitian symmetry
+static __device__ __forceinline__ long long l1_pos(long long k, int P0, int P1, int P2) {
+  return ((k % P0) * P1 + (k / P0) % P1) * P2 + k / (static_cast<long long>(P0) * P1);
+}
+
 static __global__ void k_l1_spec_export(const float2* __restrict__ lib, float2* __restrict__ nat, int n, int P0,
-                                        int P1, long long C) {
-  const long long P = static_cast<long long>(P0) * P1, H = n + 1;
+                                        int P1, int P2, long long C) {
+  const long long P = static_cast<long long>(P0) * P1 * P2, H = n + 1LL;
   for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < H * C;
        e += static_cast<long long>(gridDim.x) * blockDim.x) {
     const long long c = e / H, k = e % H;
-    nat[e] = lib[c * P + (k % P0) * P1 + k / P0];
+    nat[e] = lib[c * P + l1_pos(k, P0, P1, P2)];
   }
 }
 
 static __global__ void k_l1_spec_import(const float2* __restrict__ nat, float2* __restrict__ lib, int n, int P0,
-                                        int P1, long long C, long long pitch, float scale) {
-  const long long P = static_cast<long long>(P0) * P1;
+                                        int P1, int P2, long long C, long long pitch, float scale) {
+  const long long P = static_cast<long long>(P0) * P1 * P2;
   for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < P * C;
        e += static_cast<long long>(gridDim.x) * blockDim.x) {
     const long long c = e / P, r = e % P;
-    const long long k = (r / P1) + static_cast<long long>(P0) * (r % P1);
+    const long long k = r / (static_cast<long long>(P1) * P2) + P0 * ((r / P2) % P1) +
+                        static_cast<long long>(P0) * P1 * (r % P2);
     float2 s;
     if (k <= n) {
       s = nat[c * pitch + k];

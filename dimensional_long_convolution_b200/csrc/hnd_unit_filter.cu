@@ -64,40 +64,67 @@ cudaError_t launch_fft_axis(float2* grid, int ndim, const int* n, int axis, long
 }
 
 // ------------------------------------------------------------ long 1D
-void long1d_split(int n, int* P0, int* P1) {
-  const long long P = 2LL * n;
+L1Split long1d_split(int n) {
   int lg = 0;
-  while ((1LL << lg) < P) ++lg;
-  *P0 = 1 << (lg / 2);
-  *P1 = static_cast<int>(P / *P0);
+  while ((1LL << lg) < 2LL * n) ++lg;
+  L1Split sp;
+  sp.m = lg <= 18 ? 2 : 3;                 // factors of at most 2^9 points
+  int left = lg;
+  for (int a = 0; a < 3; ++a) {
+    const int share = a < sp.m ? (left + (sp.m - a) - 1) / (sp.m - a) : 0;    // the larger shares first
+    sp.P[a] = 1 << share;
+    left -= share;
+  }
+  return sp;
 }
 
-// forward four-step on `ngrids` adjacent grids of P = P0 P1
-static cudaError_t four_step_fwd(float2* grid, int P0, int P1, long long ngrids, cudaStream_t st) {
-  const int h[2] = {P0 / 2, P1 / 2};
-  cudaError_t e = launch_fft_axis(grid, 2, h, 0, ngrids, st);
-  if (e != cudaSuccess) return e;
-  hnd2::k_l1_twiddle<<<grid_for(static_cast<long long>(P0) * P1 * ngrids, 256), 256, 0, st>>>(grid, P0, P1, ngrids);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  return launch_fft_axis(grid, 2, h, 1, ngrids, st);
+// forward split transform on `ngrids` adjacent grids of P points
+static cudaError_t l1_fwd(float2* grid, const L1Split& sp, long long ngrids, cudaStream_t st) {
+  int h[3];
+  long long P = 1;
+  for (int a = 0; a < sp.m; ++a) {
+    h[a] = sp.P[a] / 2;
+    P *= sp.P[a];
+  }
+  long long Q = P;
+  cudaError_t e = cudaSuccess;
+  for (int a = 0; a < sp.m && e == cudaSuccess; ++a) {
+    e = launch_fft_axis(grid, sp.m, h, a, ngrids, st);
+    if (e != cudaSuccess || a == sp.m - 1) break;
+    hnd2::k_l1_twiddle<<<grid_for(P * ngrids, 256), 256, 0, st>>>(grid, sp.P[a], Q, P * ngrids);
+    e = cudaGetLastError();
+    Q /= sp.P[a];
+  }
+  return e;
 }
 
-// on conjugated spectra [k0][k1]: the conjugate of the unnormalised inverse,
-// in natural order i = P1 i0 + i1
-static cudaError_t four_step_inv_conj(float2* grid, int P0, int P1, long long ngrids, cudaStream_t st) {
-  const int h[2] = {P0 / 2, P1 / 2};
-  cudaError_t e = launch_fft_axis(grid, 2, h, 1, ngrids, st);
-  if (e != cudaSuccess) return e;
-  hnd2::k_l1_twiddle<<<grid_for(static_cast<long long>(P0) * P1 * ngrids, 256), 256, 0, st>>>(grid, P0, P1, ngrids);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  return launch_fft_axis(grid, 2, h, 0, ngrids, st);
+// on conjugated spectra in split order: the conjugate of the unnormalised
+// inverse, in natural order
+static cudaError_t l1_inv_conj(float2* grid, const L1Split& sp, long long ngrids, cudaStream_t st) {
+  int h[3];
+  long long P = 1;
+  for (int a = 0; a < sp.m; ++a) {
+    h[a] = sp.P[a] / 2;
+    P *= sp.P[a];
+  }
+  cudaError_t e = cudaSuccess;
+  for (int a = sp.m - 1; a >= 0 && e == cudaSuccess; --a) {
+    e = launch_fft_axis(grid, sp.m, h, a, ngrids, st);
+    if (e != cudaSuccess || a == 0) break;
+    long long Q = 1;               // points of levels a - 1 .. m - 1
+    for (int b = a - 1; b < sp.m; ++b) Q *= sp.P[b];
+    hnd2::k_l1_twiddle<<<grid_for(P * ngrids, 256), 256, 0, st>>>(grid, sp.P[a - 1], Q, P * ngrids);
+    e = cudaGetLastError();
+  }
+  return e;
 }
+
+int long1d_launches_per_transform(int n) { return 2 * long1d_split(n).m - 1; }
 
 template <class T>
 static cudaError_t long1d_t(const ConvArgs& a, float2* grid, long long wave, int* launches) {
   const int n = a.n[0];
-  int P0, P1;
-  long1d_split(n, &P0, &P1);
+  const L1Split sp = long1d_split(n);
   const long long P = 2LL * n, nv = static_cast<long long>(a.B) * a.C;
   const T* q = static_cast<const T*>(a.q);
   const T* k = static_cast<const T*>(a.k);
@@ -108,11 +135,11 @@ static cudaError_t long1d_t(const ConvArgs& a, float2* grid, long long wave, int
     const int cnt = static_cast<int>(nv - v0 < wave ? nv - v0 : wave);
     hnd2::k_l1_pad<T><<<grid_for(P * cnt, 256), 256, 0, a.stream>>>(k, v, grid, n, P, v0, cnt);
     if ((e = cudaGetLastError()) != cudaSuccess) break;
-    if ((e = four_step_fwd(grid, P0, P1, cnt, a.stream)) != cudaSuccess) break;
+    if ((e = l1_fwd(grid, sp, cnt, a.stream)) != cudaSuccess) break;
     hnd2::k_l1_modulate<<<grid_for(P * cnt, 256), 256, 0, a.stream>>>(grid, static_cast<const float2*>(a.spec), a.sbs,
                                                                      a.sconj, P, a.C, v0, cnt);
     if ((e = cudaGetLastError()) != cudaSuccess) break;
-    if ((e = four_step_inv_conj(grid, P0, P1, cnt, a.stream)) != cudaSuccess) break;
+    if ((e = l1_inv_conj(grid, sp, cnt, a.stream)) != cudaSuccess) break;
     if (a.y2) {
       hnd2::k_l1_out<T, true><<<grid_for(static_cast<long long>(n) * cnt, 256), 256, 0, a.stream>>>(
           grid, q, y, static_cast<const T*>(a.g2), static_cast<T*>(a.y2), n, P, v0, cnt);
@@ -121,7 +148,7 @@ static cudaError_t long1d_t(const ConvArgs& a, float2* grid, long long wave, int
           grid, q, y, nullptr, nullptr, n, P, v0, cnt);
     }
     e = cudaGetLastError();
-    *launches += 9;
+    *launches += 3 + 2 * (2 * sp.m - 1);
   }
   return e;
 }
@@ -185,9 +212,7 @@ cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, i
                  : filter_mlp_go<128>(fa, noff, st);
   if (e != cudaSuccess) return e;
   if (ndim == 1 && n[0] > 256) {
-    int P0, P1;
-    long1d_split(n[0], &P0, &P1);
-    if ((e = four_step_fwd(grid, P0, P1, nc, st)) != cudaSuccess) return e;
+    if ((e = l1_fwd(grid, long1d_split(n[0]), nc, st)) != cudaSuccess) return e;
     hnd2::k_l1_spec_store<<<grid_for(gsz * nc, 256), 256, 0, st>>>(
         grid, static_cast<float2*>(spectrum), gsz, c0, nc, static_cast<float>(1.0 / static_cast<double>(gsz)));
     return cudaGetLastError();
@@ -230,17 +255,16 @@ static cudaError_t kgrad_chunk_t(const KgradLaunch& g, cudaStream_t st) {
   hnd2::k_kg_pad<T><<<grid_for(gsz * nvol, 256), 256, 0, st>>>(k, v, gu, d, g.B, g.C, g.c0, nvol);
   hnd2::k_kg_pad<T><<<grid_for(gsz * nvol, 256), 256, 0, st>>>(q, dy, gz, d, g.B, g.C, g.c0, nvol);
   const bool long1d = g.ndim == 1 && g.n[0] > 256;
-  int P0 = 0, P1 = 0;
-  if (long1d) long1d_split(g.n[0], &P0, &P1);
+  const L1Split sp = long1d ? long1d_split(g.n[0]) : L1Split();
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess)       // gu and gz are adjacent
-    e = long1d ? four_step_fwd(gu, P0, P1, 2LL * nvol, st) : launch_fft_axes(gu, g.ndim, g.n, 2LL * nvol, st);
+    e = long1d ? l1_fwd(gu, sp, 2LL * nvol, st) : launch_fft_axes(gu, g.ndim, g.n, 2LL * nvol, st);
   if (e != cudaSuccess) return e;
   hnd2::k_kg_corr<<<grid_for(gsz * g.ncc, 256), 256, 0, st>>>(gu, gz, acc, g.B, g.ncc, gsz);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // the accumulator holds conj(sum_b Z conj U): a forward transform gives the
   // conjugate of the unnormalised inverse, whose real part is wanted
-  e = long1d ? four_step_inv_conj(acc, P0, P1, g.ncc, st) : launch_fft_axes(acc, g.ndim, g.n, g.ncc, st);
+  e = long1d ? l1_inv_conj(acc, sp, g.ncc, st) : launch_fft_axes(acc, g.ndim, g.n, g.ncc, st);
   if (e != cudaSuccess) return e;
   const float scale = static_cast<float>(1.0 / static_cast<double>(gsz));
   if (g.circular) {
@@ -261,14 +285,14 @@ cudaError_t launch_kgrad_chunk(const KgradLaunch& g, cudaStream_t st) {
 cudaError_t launch_spec_convert(int ndim, const int* n, long long C, const void* src, void* dst, bool to_natural,
                                 cudaStream_t st) {
   if (ndim == 1 && n[0] > 256) {
-    int P0, P1;
-    long1d_split(n[0], &P0, &P1);
+    const L1Split sp = long1d_split(n[0]);
     if (to_natural)
       hnd2::k_l1_spec_export<<<grid_for((n[0] + 1LL) * C, 256), 256, 0, st>>>(
-          static_cast<const float2*>(src), static_cast<float2*>(dst), n[0], P0, P1, C);
+          static_cast<const float2*>(src), static_cast<float2*>(dst), n[0], sp.P[0], sp.P[1], sp.P[2], C);
     else
       hnd2::k_l1_spec_import<<<grid_for(2LL * n[0] * C, 256), 256, 0, st>>>(
-          static_cast<const float2*>(src), static_cast<float2*>(dst), n[0], P0, P1, C, n[0] + 1LL, 1.f);
+          static_cast<const float2*>(src), static_cast<float2*>(dst), n[0], sp.P[0], sp.P[1], sp.P[2], C,
+          n[0] + 1LL, 1.f);
     return cudaGetLastError();
   }
   const SpecDims d = make_dims(ndim, n);

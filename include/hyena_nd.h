@@ -69,10 +69,10 @@ typedef enum { HYENA_ND_F32 = 0, HYENA_ND_BF16 = 1 } hyena_nd_dtype;
  *   ndim     1, 2 or 3.
  *   n[a]     grid extent of axis a (a < ndim), a power of two in [8, 256];
  *            for ndim == 3 the two outer axes are limited to [8, 128]; for
- *            ndim == 1 any power of two in [8, 131072] (long 1D context:
- *            n > 256 runs the padded length-2n transform as a four-step
- *            split 2n = P0 P1 of two passes of at most 512 points, in waves
- *            of volumes through the workspace).
+ *            ndim == 1 any power of two in [8, 2^26] (long 1D context:
+ *            n > 256 runs the padded length-2n transform as a split
+ *            2n = P0 P1 (P2) into two or three passes of at most 512 points,
+ *            in waves of volumes through the workspace).
  *   B, C     batch and channel counts (>= 1).
  *   io_dtype dtype of q, k, v and y.
  *   circular 0: zero-padded linear convolution.  1: circular (periodic)

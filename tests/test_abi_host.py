@@ -53,8 +53,9 @@ def test_sizes_of_the_benchmark_grids(i):
     ((300, 300), 1, 1, 0, 0, False),          # not a power of two
     ((512, 8), 1, 1, 0, 0, False),            # a 2D axis above 256
     ((512,), 1, 1, 0, 0, True),               # long 1D context
-    ((131072,), 2, 4, 1, 1, True),            # longest 1D grid, circular
-    ((262144,), 1, 1, 0, 0, False),           # above the long 1D limit
+    ((131072,), 2, 4, 1, 1, True),            # longest two-level split, circular
+    ((1 << 26,), 1, 1, 0, 0, True),           # longest 1D grid (three levels)
+    ((1 << 27,), 1, 1, 0, 0, False),          # above the long 1D limit
     ((3000,), 1, 1, 0, 0, False),             # long 1D, not a power of two
     ((4, 8), 1, 1, 0, 0, False),              # below 8
     ((256, 64, 64), 1, 1, 0, 0, False),       # outer 3D axis above 128
@@ -155,7 +156,7 @@ def test_workspace_covers_the_kernel_gradient():
         assert H.workspace_bytes(p) >= (2 * wl.B + 1) * P * 8
 
 
-@pytest.mark.parametrize("n,B,C", [(512, 2, 3), (4096, 1, 8), (131072, 2, 100)])
+@pytest.mark.parametrize("n,B,C", [(512, 2, 3), (4096, 1, 8), (131072, 2, 100), (1 << 23, 1, 2), (1 << 26, 1, 1)])
 def test_long_1d_sizes(n, B, C):
     """Long 1D grids keep all 2n frequencies in the library order; the
     workspace holds at least one volume's padded grid (one wave) and the
@@ -164,7 +165,7 @@ def test_long_1d_sizes(n, B, C):
     assert H.spectrum_bytes(p) == C * 2 * n * 8
     ws = H.workspace_bytes(p)
     assert ws >= 256 + max(2 * n * 8, (2 * B + 1) * 2 * n * 8)
-    assert ws <= 256 + max(96 << 20, 128 << 20, (2 * B + 1) * 2 * n * 8)
+    assert ws <= 256 + max(96 << 20, 128 << 20, (2 * B + 1) * 2 * n * 8, 64 * 2 * n * 8)
 
 
 def test_long_1d_spectrum_conversion_uses_the_natural_size():

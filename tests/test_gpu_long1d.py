@@ -1,6 +1,6 @@
-"""GPU parity of the long 1D context tier (n from 512 to 131072) against the
-float64 oracle: the padded length-2n transform runs as a four-step split of two
-passes of at most 512 points, volumes go through the workspace in waves.
+"""GPU parity of the long 1D context tier (n from 512 to 2^26) against the
+float64 oracle: the padded length-2n transform runs as a split into two or
+three passes of at most 512 points, volumes go through the workspace in waves.
 Forward, backward, kernel gradient, the filter spectrum and its import/export,
 per-sample spectra, circular mode and the Gaussian window are each checked,
 fully at sizes the dense-DFT oracle finishes quickly and on sampled outputs
@@ -234,3 +234,86 @@ def test_long1d_gaussian_window_sampled():
     K = _kernel_for(f, wl.dims, C, chans, window=1)
     want = O.conv_direct_at(inp.as_f64("q"), inp.as_f64("k"), inp.as_f64("v"), K, wl.dims, pts)
     assert O.rel_l2(np.array([got[tuple(p)] for p in pts]), want) <= TOL["f32"]
+
+
+# ------------------------------------------------ three-level split (n > 2^17)
+@pytest.mark.parametrize("n,B,C,dt", [(1 << 18, 1, 2, "f32"), (1 << 19, 2, 1, "bf16")])
+def test_long1d_three_levels_forward_sampled(n, B, C, dt):
+    wl = W.custom((n,), B, C, io_dtype=dt, seed=61 + C)
+    inp = W.make_inputs(wl)
+    got, _ = run(inp)
+    assert H.last_launch_count() == 13 * _waves(n, B, C)
+    chans = list(range(C))
+    pts = sample_points(wl, 10, seed=9, channels=chans)
+    K = _kernel_for(inp.filt, wl.dims, C, chans)
+    want = O.conv_direct_at(inp.as_f64("q"), inp.as_f64("k"), inp.as_f64("v"), K, wl.dims, pts)
+    assert O.rel_l2(np.array([got[tuple(p)] for p in pts]), want) <= TOL[dt]
+
+
+def test_long1d_three_levels_spectrum_backward_and_kernel_grad():
+    n, B, C = 1 << 18, 2, 2
+    wl = W.custom((n,), B, C, seed=67)
+    inp = W.make_inputs(wl)
+    dy = W.make_inputs(wl, seed=wl.seed + 7).q
+    op = make_op(wl)
+    set_filter(op, inp.filt)
+    K = O.implicit_kernel(inp.filt, wl.dims)
+    spec = to_host(op.export_spectrum())
+    rng = np.random.default_rng(10)
+    ks = np.concatenate([[0, 1, n - 1, n], rng.integers(0, n + 1, 8)])
+    sp = np.stack([np.arange(ks.size) % C, ks], axis=1)
+    assert O.rel_l2(np.array([spec[int(c), int(k)] for c, k in sp]), O.spectrum_at(K, wl.dims, sp)) < 2e-5
+    q, k, v, g = (to_dev(a) for a in (inp.q, inp.k, inp.v, dy))
+    dq, dk, dv = (to_host(x) for x in op.backward(q, k, v, g))
+    dK = to_host(op.kernel_grad(q, k, v, g))
+    torch().cuda.synchronize()
+    assert op.status() == H.OK
+    qf, kf, vf, gf = inp.as_f64("q"), inp.as_f64("k"), inp.as_f64("v"), _f64(dy)
+    pts = sample_points(wl, 8, seed=11)
+    w = O.conv_direct_at(np.ones_like(qf), kf, vf, K, wl.dims, pts)
+    du = O.corr_direct_at(qf * gf, K, wl.dims, pts)
+    idx = [tuple(p) for p in pts]
+    wants = (np.array([gf[i] for i in idx]) * w, np.array([vf[i] for i in idx]) * du,
+             np.array([kf[i] for i in idx]) * du)
+    for name, got, want in zip(("dq", "dk", "dv"), (dq, dk, dv), wants):
+        assert O.rel_l2(np.array([got[i] for i in idx]), want) <= TOL["f32"], name
+    kp = np.stack([rng.integers(0, C, 8), rng.integers(-(n - 1), n, 8)], axis=1)
+    kp[0] = [0, n - 1]
+    kp[1] = [1, -(n - 1)]
+    wantK = O.kernel_grad_at(qf, kf, vf, gf, wl.dims, kp)
+    assert O.rel_l2(np.array([dK[int(c), int(t) + n - 1] for c, t in kp]), wantK) <= TOL["f32"]
+
+
+def test_long1d_eight_million_tokens_sampled():
+    """2^23 tokens (the pages' long-context class of about ten million), the
+    filter network evaluated on all 2^24 - 1 offsets, sampled outputs."""
+    n = 1 << 23
+    wl = W.custom((n,), 1, 1, seed=71)
+    inp = W.make_inputs(wl)
+    got, _ = run(inp)
+    pts = sample_points(wl, 6, seed=12, channels=[0])
+    K = O.implicit_kernel(inp.filt, wl.dims)
+    want = O.conv_direct_at(inp.as_f64("q"), inp.as_f64("k"), inp.as_f64("v"), K, wl.dims, pts)
+    assert O.rel_l2(np.array([got[tuple(p)] for p in pts]), want) <= TOL["f32"]
+
+
+def test_long1d_longest_grid_shifted_delta():
+    """n = 2^26, the largest grid: the natural spectrum of a delta at offset t0
+    (its closed form exp(-2 pi i k t0 / P) / P) must shift the gated input,
+    y[i] = q[i] u[i - t0], at every output."""
+    n, t0 = 1 << 26, 12345
+    wl = W.custom((n,), 1, 1, seed=73)
+    inp = W.make_inputs(wl)
+    op = make_op(wl)
+    kk = np.arange(n + 1, dtype=np.float64)
+    ph = np.mod(kk * t0, 2 * n) / (2 * n)
+    nat = (np.exp(-2j * np.pi * ph) / (2 * n)).astype(np.complex64)[None]
+    op.import_spectrum(torch().from_numpy(nat))
+    del nat, kk, ph
+    got, _ = run(inp, op=op)
+    assert H.last_launch_count() == 13
+    u = inp.as_f64("k")[0, 0] * inp.as_f64("v")[0, 0]
+    want = np.zeros(n)
+    want[t0:] = u[: n - t0]
+    want *= inp.as_f64("q")[0, 0]
+    assert O.rel_l2(got[0, 0], want) <= TOL["f32"]
