@@ -48,8 +48,10 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=0, help="timed steps (0 = enough for about 3 s)")
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--config", type=int, default=2, help="benchmark grid index (0..4)")
-    ap.add_argument("--also", default="1,3", help="extra grids measured kernel-only, comma separated")
+    ap.add_argument("--config", type=lambda x: int(x) if x.isdigit() else x, default=2,
+                    help="benchmark grid index (0..4) or workload name")
+    ap.add_argument("--also", default="1,3", help="extra grids measured kernel-only, comma separated "
+                    "(suite indices or workload names, e.g. seq1d_1m_b1_c64_bf16)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--sets", type=int, default=3, help="rotating input sets")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -357,7 +359,7 @@ def run_ours(args):
 
     also = []
     for tok in [x for x in args.also.split(",") if x.strip() != ""]:
-        j = int(tok)
+        j = int(tok) if tok.strip().isdigit() else tok.strip()
         if j == args.config:
             continue
         wj = W.workload(j)

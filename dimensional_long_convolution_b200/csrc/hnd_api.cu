@@ -24,6 +24,10 @@ constexpr size_t kWaveBudget = size_t(96) << 20;      // multi-pass intermediate
 constexpr size_t kFilterBudget = size_t(64) << 20;    // filter grid per channel chunk
 constexpr int kFilterMaxChunk = 64;
 constexpr size_t kKgradBudget = size_t(128) << 20;    // kernel-gradient grids per channel chunk
+#ifndef HND_L1_WAVE_MB
+#define HND_L1_WAVE_MB 96
+#endif
+constexpr size_t kL1WaveBudget = size_t(HND_L1_WAVE_MB) << 20;   // long 1D grids per wave
 
 enum Tier { kRows1D = 0, kFused2D = 1, kMulti2D = 2, kMulti3D = 3, kLong1D = 4 };
 
@@ -90,7 +94,7 @@ hyena_nd_status make_plan(const hyena_nd_problem* p, Plan* pl) {
   if (p->ndim == 1 && nl > 256) {
     pl->tier = kLong1D;
     const size_t per_vol = static_cast<size_t>(8) * static_cast<size_t>(pl->gsz);
-    long long w = static_cast<long long>(kWaveBudget / per_vol);
+    long long w = static_cast<long long>(kL1WaveBudget / per_vol);
     if (w < 1) w = 1;
     if (w > pairs) w = pairs;
     const long long nw = (pairs + w - 1) / w;

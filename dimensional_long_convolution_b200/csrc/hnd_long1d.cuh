@@ -20,26 +20,9 @@
 // The axis transforms are k_fft_axis2 of hnd_filter2.cuh.
 #pragma once
 
-#include "hnd_fused2.cuh"
+#include "hnd_filter2.cuh"
 
 namespace hnd2 {
-
-// zero-padded a . b of volumes [v0, v0 + nvol) (memory order b C + c)
-template <class T>
-static __global__ void k_l1_pad(const T* __restrict__ a, const T* __restrict__ b, float2* __restrict__ grid, int n,
-                                long long P, long long v0, int nvol) {
-  const long long total = P * nvol;
-  for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < total;
-       e += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long v = e / P, j = e % P;
-    float val = 0.f;
-    if (j < n) {
-      const long long o = (v0 + v) * n + j;
-      val = Act<T>::ld_g(a + o) * Act<T>::ld_g(b + o);
-    }
-    grid[e] = make_float2(val, 0.f);
-  }
-}
 
 // Twiddle of level a of the split: on the view [..][P_a][R] (R = Q / P_a the
 // points of the later levels, Q = P_a R), element (k, r) *= W_Q^{k r},
@@ -57,38 +40,7 @@ static __global__ void k_l1_twiddle(float2* __restrict__ grid, int Pa, long long
   }
 }
 
-// grid = conj(grid S_c) with S_c (or conj S_c when sconj < 0) of the volume's
-// channel and sample; spec: [C][P] per sample set, sample stride sbs (complex)
-static __global__ void k_l1_modulate(float2* __restrict__ grid, const float2* __restrict__ spec, long long sbs,
-                                     float sconj, long long P, int C, long long v0, int nvol) {
-  const long long total = P * nvol;
-  for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < total;
-       e += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long v = v0 + e / P, r = e % P;
-    const long long b = v / C, c = v % C;
-    const float2 S = __ldg(spec + b * sbs + c * P + r);
-    const float si = sconj * S.y;
-    const float2 x = grid[e];
-    grid[e] = make_float2(x.x * S.x - x.y * si, -(x.x * si + x.y * S.x));
-  }
-}
-
-template <class T, bool DUAL>
-static __global__ void k_l1_out(const float2* __restrict__ grid, const T* __restrict__ q, T* __restrict__ y,
-                                const T* __restrict__ g2, T* __restrict__ y2, int n, long long P, long long v0,
-                                int nvol) {
-  const long long total = static_cast<long long>(n) * nvol;
-  for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < total;
-       e += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long v = e / n, i = e % n;
-    const float r = grid[v * P + i].x;
-    const long long o = (v0 + v) * n + i;
-    Act<T>::st_g(y + o, r * Act<T>::ld_g(q + o));
-    if constexpr (DUAL) Act<T>::st_g(y2 + o, r * Act<T>::ld_g(g2 + o));
-  }
-}
-
-// filter grids (after the forward four-step) -> spectrum [c0 + c][P], scaled
+// filter grids (after the forward split transform) -> spectrum [c0 + c][P], scaled
 static __global__ void k_l1_spec_store(const float2* __restrict__ grid, float2* __restrict__ spec, long long P, int c0,
                                        int nc, float scale) {
   const long long total = P * nc;
@@ -132,6 +84,201 @@ static __global__ void k_l1_spec_import(const float2* __restrict__ nat, float2* 
       s.y = -s.y;
     }
     lib[e] = make_float2(s.x * scale, s.y * scale);
+  }
+}
+
+// ------------------------------------------------------------ fused passes
+// One convolution over a wave of volumes as 2m - 1 passes, each an axis
+// transform with its neighbours' elementwise steps folded in:
+//   kFirst   axis 0: k v of the first P0/2 rows (the rest is the zero pad),
+//            padded forward transform, forward twiddle of level 0
+//   kFwdMid  axis 1 of 3: full forward transform, forward twiddle of level 1
+//   kCenter  last axis: full forward transform, spectrum product, full
+//            inverse transform, conjugate twiddle of level m - 2
+//   kInvMid  axis 1 of 3: full inverse transform, conjugate twiddle of level 0
+//   kLast    axis 0: inverse transform of which only the first P0/2 outputs
+//            (the crop i < n) are formed, output gate(s)
+// The inverse chain (inverse transforms, conjugate twiddles, last axis first)
+// is the adjoint of the forward chain, so on spectra in split order it forms
+// the unnormalised inverse in natural order (the spectrum holds the 1/P).
+enum L1Kind { kFirst = 0, kFwdMid = 1, kCenter = 2, kInvMid = 3, kLast = 4 };
+
+struct L1PassArgs {
+  float2* grid;              // wave grids [vol][P]
+  long long P;               // points per grid
+  long long stride;          // stride of the pass's axis (points)
+  long long npen;            // pencils in the wave
+  long long twQ;             // twiddle order Q (W_Q)
+  int twP;                   // inverse twiddles: the level's factor (k = outer index mod twP)
+  int n;                     // volume length
+  long long v0;              // first volume of the wave (memory order b C + c)
+  const void* a;             // kFirst: k
+  const void* b;             // kFirst: v
+  const void* q;             // kLast: output gate
+  void* y;                   // kLast: output
+  const void* g2;            // kLast: second gate (dual output) or null
+  void* y2;
+  const float2* spec;        // kCenter: spectrum [C][P] per sample set
+  long long sbs;             // sample-set stride (complex values)
+  float sconj;               // -1: conjugate spectrum (adjoint)
+  int C;
+};
+
+// W_Q^m for 0 <= m < Q (Q a power of two): the ratio is exact while m < 2^24
+__device__ __forceinline__ float2 l1_w(long long m, long long Q) {
+  float s, c;
+  sincospif(-2.f * (static_cast<float>(m) / static_cast<float>(Q)), &s, &c);
+  return make_float2(c, s);
+}
+
+__device__ __forceinline__ float2 l1_conj(float2 a) { return make_float2(a.x, -a.y); }
+
+template <int N>
+__device__ __forceinline__ void l1_full_inv(cp (&x)[P2<N>::R1], float2 (&lo)[P2<N>::R1], float2 (&hi)[P2<N>::R1],
+                                            int g, float4* buf, Tabs<N> t) {
+  constexpr int G = P2<N>::G, R1 = P2<N>::R1;
+  fft_inv<N>(x, g, buf, 0, t, 0u);
+  const float2 tg = t.b[4 * G + g];
+  sfor<0, R1>([&](auto sc) {
+    constexpr int s = decltype(sc)::value;
+    const float2 w = mul_w32<s * (16 / R1)>(tg);     // W_2N^{g + s G}
+    // path 0: A_j, path 1: B_j; y[j] = A + B conj(w), y[j + N] = A - B conj(w)
+    const float br = fmaf(x[s].re.y, w.x, x[s].im.y * w.y);
+    const float bi = fmaf(x[s].im.y, w.x, -x[s].re.y * w.y);
+    lo[s] = make_float2(x[s].re.x + br, x[s].im.x + bi);
+    hi[s] = make_float2(x[s].re.x - br, x[s].im.x - bi);
+  });
+}
+
+template <int N, int KIND, class T, bool DUAL>
+__global__ void __launch_bounds__(kAT, N >= 128 ? 2 : 1) k_l1_pass(const L1PassArgs a) {
+  constexpr int G = P2<N>::G, R1 = P2<N>::R1, PPW = 32 / G, P = 2 * N;
+  extern __shared__ __align__(16) unsigned char asmem[];
+  const Tabs<N> t = tabs_at<N>(asmem);
+  float4* xb = reinterpret_cast<float4*>(asmem + Tabs<N>::kBytes);
+  tabs_build<N>(t, g_tw512);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pen = lane / G, g = lane % G;
+  float4* buf = xb + warp * XB<N>::kWarp + pen * XB<N>::kPen;
+  const long long per_cta = (kAT / 32) * PPW;
+  const long long S = a.stride;
+  for (long long p0 = static_cast<long long>(blockIdx.x) * per_cta; p0 < a.npen;
+       p0 += static_cast<long long>(gridDim.x) * per_cta) {
+    const long long p = p0 + warp * PPW + pen;
+    const bool act = p < a.npen;
+    const long long o = act ? p / S : 0, i = act ? p % S : 0;
+    const long long start = o * P * S + i;            // first point of the pencil in the wave
+    const long long vol = start / a.P;                // the pencil's volume within the wave
+    float2* base = a.grid + start;
+    cp x[R1];
+    if constexpr (KIND == kFirst) {
+      const T* ka = static_cast<const T*>(a.a);
+      const T* va = static_cast<const T*>(a.b);
+      float2 z[R1];
+      const long long row0 = (a.v0 + vol) * a.n + i;
+#pragma unroll
+      for (int s = 0; s < R1; ++s) {
+        const long long j = row0 + static_cast<long long>(g + s * G) * S;
+        z[s] = act ? make_float2(Act<T>::ld_g(ka + j) * Act<T>::ld_g(va + j), 0.f) : make_float2(0.f, 0.f);
+      }
+      padded_fwd<N>(z, x, g, buf, 0, t, 0u);
+    } else if constexpr (KIND == kFwdMid || KIND == kCenter) {
+      float2 lo[R1], hi[R1];
+#pragma unroll
+      for (int s = 0; s < R1; ++s) {
+        const long long j = g + s * G;
+        lo[s] = act ? base[j * S] : make_float2(0.f, 0.f);
+        hi[s] = act ? base[(j + N) * S] : make_float2(0.f, 0.f);
+      }
+      full_fwd<N>(lo, hi, x, g, buf, 0, t, 0u);
+    } else {
+      // kInvMid, kLast: spectral input, (Y[2f], Y[2f+1]) per slot
+#pragma unroll
+      for (int s = 0; s < R1; ++s) {
+        const long long f = spec_idx<N>(g, s);
+        const float2 e0 = act ? base[(2 * f) * S] : make_float2(0.f, 0.f);
+        const float2 e1 = act ? base[(2 * f + 1) * S] : make_float2(0.f, 0.f);
+        x[s] = {make_float2(e0.x, e1.x), make_float2(e0.y, e1.y)};
+      }
+    }
+
+    if constexpr (KIND == kFirst || KIND == kFwdMid) {
+      // forward twiddle W_Q^{k i} at k = 2f, 2f + 1; store in spectral positions
+      const float2 wi = l1_w(i, a.twQ);
+#pragma unroll
+      for (int s = 0; s < R1; ++s) {
+        const long long f = spec_idx<N>(g, s);
+        const float2 w0 = l1_w(((2 * f) * i) % a.twQ, a.twQ);
+        const float2 w1 = cmul1(w0, wi);
+        if (act) {
+          base[(2 * f) * S] = cmul1(make_float2(x[s].re.x, x[s].im.x), w0);
+          base[(2 * f + 1) * S] = cmul1(make_float2(x[s].re.y, x[s].im.y), w1);
+        }
+      }
+    } else if constexpr (KIND == kCenter) {
+      const long long vg = a.v0 + vol;
+      const long long bb = vg / a.C, cc = vg % a.C;
+      const float2* Sp = a.spec + bb * a.sbs + cc * a.P + (start - vol * a.P);
+#pragma unroll
+      for (int s = 0; s < R1; ++s) {
+        const long long f = spec_idx<N>(g, s);
+        float4 sv = act ? __ldg(reinterpret_cast<const float4*>(Sp + 2 * f)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        sv.y *= a.sconj;
+        sv.w *= a.sconj;
+        const float2 y0 = cmul1(make_float2(x[s].re.x, x[s].im.x), make_float2(sv.x, sv.y));
+        const float2 y1 = cmul1(make_float2(x[s].re.y, x[s].im.y), make_float2(sv.z, sv.w));
+        x[s] = {make_float2(y0.x, y1.x), make_float2(y0.y, y1.y)};
+      }
+      float2 lo[R1], hi[R1];
+      l1_full_inv<N>(x, lo, hi, g, buf, t);
+      // conjugate twiddle of the previous level: conj W_Q^{k e}, k = o mod twP,
+      // e the element's index along this (last) axis
+      const long long k = o % a.twP;
+      const float2 wk = l1_conj(l1_w((k * N) % a.twQ, a.twQ));
+#pragma unroll
+      for (int s = 0; s < R1; ++s) {
+        const long long j = g + s * G;
+        const float2 w0 = l1_conj(l1_w((k * j) % a.twQ, a.twQ));
+        const float2 w1 = cmul1(w0, wk);
+        if (act) {
+          base[j] = cmul1(lo[s], w0);
+          base[j + N] = cmul1(hi[s], w1);
+        }
+      }
+    } else if constexpr (KIND == kInvMid) {
+      float2 lo[R1], hi[R1];
+      l1_full_inv<N>(x, lo, hi, g, buf, t);
+      // conjugate twiddle of level 0: conj W_P^{k0 (e S + i)}, k0 = o mod twP
+      const long long k = o % a.twP;
+      const float2 wk = l1_conj(l1_w((k * N * S) % a.twQ, a.twQ));
+#pragma unroll
+      for (int s = 0; s < R1; ++s) {
+        const long long j = g + s * G;
+        const float2 w0 = l1_conj(l1_w((k * (j * S + i)) % a.twQ, a.twQ));
+        const float2 w1 = cmul1(w0, wk);
+        if (act) {
+          base[j * S] = cmul1(lo[s], w0);
+          base[(j + N) * S] = cmul1(hi[s], w1);
+        }
+      }
+    } else {
+      // kLast: outputs i0 < N only (the crop), real part, output gate(s)
+      float2 out[R1];
+      padded_inv<N>(x, out, g, buf, 0, t, 0u);
+      const T* qa = static_cast<const T*>(a.q);
+      T* ya = static_cast<T*>(a.y);
+      const long long row0 = (a.v0 + vol) * a.n + i;
+#pragma unroll
+      for (int s = 0; s < R1; ++s) {
+        const long long j = row0 + static_cast<long long>(g + s * G) * S;
+        if (act) {
+          Act<T>::st_g(ya + j, out[s].x * Act<T>::ld_g(qa + j));
+          if constexpr (DUAL)
+            Act<T>::st_g(static_cast<T*>(a.y2) + j, out[s].x * Act<T>::ld_g(static_cast<const T*>(a.g2) + j));
+        }
+      }
+    }
   }
 }
 

@@ -121,42 +121,6 @@ static cudaError_t l1_inv_conj(float2* grid, const L1Split& sp, long long ngrids
 
 int long1d_launches_per_transform(int n) { return 2 * long1d_split(n).m - 1; }
 
-template <class T>
-static cudaError_t long1d_t(const ConvArgs& a, float2* grid, long long wave, int* launches) {
-  const int n = a.n[0];
-  const L1Split sp = long1d_split(n);
-  const long long P = 2LL * n, nv = static_cast<long long>(a.B) * a.C;
-  const T* q = static_cast<const T*>(a.q);
-  const T* k = static_cast<const T*>(a.k);
-  const T* v = static_cast<const T*>(a.v);
-  T* y = static_cast<T*>(a.y);
-  cudaError_t e = cudaSuccess;
-  for (long long v0 = 0; v0 < nv && e == cudaSuccess; v0 += wave) {
-    const int cnt = static_cast<int>(nv - v0 < wave ? nv - v0 : wave);
-    hnd2::k_l1_pad<T><<<grid_for(P * cnt, 256), 256, 0, a.stream>>>(k, v, grid, n, P, v0, cnt);
-    if ((e = cudaGetLastError()) != cudaSuccess) break;
-    if ((e = l1_fwd(grid, sp, cnt, a.stream)) != cudaSuccess) break;
-    hnd2::k_l1_modulate<<<grid_for(P * cnt, 256), 256, 0, a.stream>>>(grid, static_cast<const float2*>(a.spec), a.sbs,
-                                                                     a.sconj, P, a.C, v0, cnt);
-    if ((e = cudaGetLastError()) != cudaSuccess) break;
-    if ((e = l1_inv_conj(grid, sp, cnt, a.stream)) != cudaSuccess) break;
-    if (a.y2) {
-      hnd2::k_l1_out<T, true><<<grid_for(static_cast<long long>(n) * cnt, 256), 256, 0, a.stream>>>(
-          grid, q, y, static_cast<const T*>(a.g2), static_cast<T*>(a.y2), n, P, v0, cnt);
-    } else {
-      hnd2::k_l1_out<T, false><<<grid_for(static_cast<long long>(n) * cnt, 256), 256, 0, a.stream>>>(
-          grid, q, y, nullptr, nullptr, n, P, v0, cnt);
-    }
-    e = cudaGetLastError();
-    *launches += 3 + 2 * (2 * sp.m - 1);
-  }
-  return e;
-}
-
-cudaError_t launch_long1d(const ConvArgs& a, float2* grid, long long wave, int* launches) {
-  return a.bf16 ? long1d_t<__nv_bfloat16>(a, grid, wave, launches) : long1d_t<float>(a, grid, wave, launches);
-}
-
 cudaError_t launch_fft_axes(float2* grid, int ndim, const int* n, long long ngrids, cudaStream_t st) {
   long long gsz = 1;
   for (int a = 0; a < ndim; ++a) gsz *= 2 * n[a];

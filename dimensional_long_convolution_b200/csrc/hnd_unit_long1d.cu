@@ -1,0 +1,104 @@
+// Long 1D tier: one convolution over all volumes in waves, each wave the
+// 2m - 1 fused passes of hnd_long1d.cuh over the split P = 2n = P0 P1 (P2).
+#include "hnd_launch.h"
+#include "hnd_host_util.h"
+#include "hnd_long1d.cuh"
+
+namespace hnd {
+
+namespace {
+
+template <int N, int KIND, class T, bool DUAL>
+cudaError_t l1_pass_go(const hnd2::L1PassArgs& a, cudaStream_t st) {
+  auto kern = hnd2::k_l1_pass<N, KIND, T, DUAL>;
+  const size_t sm = hnd2::AxisSmem<N>::kBytes;
+  cudaError_t e = ensure_smem(kern, sm);
+  if (e != cudaSuccess) return e;
+  const long long per_cta = (hnd2::kAT / 32) * (32 / hnd2::P2<N>::G);
+  long long blocks = (a.npen + per_cta - 1) / per_cta;
+  if (blocks > 148LL * 16) blocks = 148LL * 16;
+  if (blocks < 1) blocks = 1;
+  kern<<<static_cast<unsigned>(blocks), hnd2::kAT, sm, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <int KIND, class T, bool DUAL>
+cudaError_t l1_pass(int N, const hnd2::L1PassArgs& a, cudaStream_t st) {
+  switch (N) {
+    case 16: return l1_pass_go<16, KIND, T, DUAL>(a, st);
+    case 32: return l1_pass_go<32, KIND, T, DUAL>(a, st);
+    case 64: return l1_pass_go<64, KIND, T, DUAL>(a, st);
+    case 128: return l1_pass_go<128, KIND, T, DUAL>(a, st);
+    case 256: return l1_pass_go<256, KIND, T, DUAL>(a, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <class T>
+cudaError_t long1d_t(const ConvArgs& c, float2* grid, long long wave, int* launches) {
+  const L1Split sp = long1d_split(c.n[0]);
+  const int m = sp.m;
+  const long long P = 2LL * c.n[0], nv = static_cast<long long>(c.B) * c.C;
+  long long stride[3] = {1, 1, 1};
+  for (int a = m - 2; a >= 0; --a) stride[a] = stride[a + 1] * sp.P[a + 1];
+  hnd2::L1PassArgs a{};
+  a.grid = grid;
+  a.P = P;
+  a.n = c.n[0];
+  a.a = c.k;
+  a.b = c.v;
+  a.q = c.q;
+  a.y = c.y;
+  a.g2 = c.g2;
+  a.y2 = c.y2;
+  a.spec = static_cast<const float2*>(c.spec);
+  a.sbs = c.sbs;
+  a.sconj = c.sconj;
+  a.C = c.C;
+  cudaError_t e = cudaSuccess;
+  for (long long v0 = 0; v0 < nv && e == cudaSuccess; v0 += wave) {
+    const long long cnt = nv - v0 < wave ? nv - v0 : wave;
+    a.v0 = v0;
+    auto set_axis = [&](int ax) {
+      a.stride = stride[ax];
+      a.npen = cnt * P / sp.P[ax];
+    };
+    // forward: axis 0 from k v, then axis 1 (three levels)
+    set_axis(0);
+    a.twQ = P;
+    e = l1_pass<hnd2::kFirst, T, false>(sp.P[0] / 2, a, c.stream);
+    if (e == cudaSuccess && m == 3) {
+      set_axis(1);
+      a.twQ = static_cast<long long>(sp.P[1]) * sp.P[2];
+      e = l1_pass<hnd2::kFwdMid, float, false>(sp.P[1] / 2, a, c.stream);
+    }
+    // spectrum product on the last axis, with the inverse transform back
+    if (e == cudaSuccess) {
+      set_axis(m - 1);
+      a.twP = sp.P[m - 2];
+      a.twQ = static_cast<long long>(sp.P[m - 2]) * sp.P[m - 1];
+      e = l1_pass<hnd2::kCenter, float, false>(sp.P[m - 1] / 2, a, c.stream);
+    }
+    if (e == cudaSuccess && m == 3) {
+      set_axis(1);
+      a.twP = sp.P[0];
+      a.twQ = P;
+      e = l1_pass<hnd2::kInvMid, float, false>(sp.P[1] / 2, a, c.stream);
+    }
+    if (e == cudaSuccess) {
+      set_axis(0);
+      e = c.y2 ? l1_pass<hnd2::kLast, T, true>(sp.P[0] / 2, a, c.stream)
+               : l1_pass<hnd2::kLast, T, false>(sp.P[0] / 2, a, c.stream);
+    }
+    *launches += 2 * m - 1;
+  }
+  return e;
+}
+
+}  // namespace
+
+cudaError_t launch_long1d(const ConvArgs& a, float2* grid, long long wave, int* launches) {
+  return a.bf16 ? long1d_t<__nv_bfloat16>(a, grid, wave, launches) : long1d_t<float>(a, grid, wave, launches);
+}
+
+}  // namespace hnd

@@ -68,10 +68,18 @@ WORKLOADS = (
 )
 
 
+# Long 1D sequences (the pages' long-context class: about a million and about
+# ten million tokens), measured beside the suite as extra lines.
+EXTRA = (
+    Workload("seq1d_1m_b1_c64_bf16", (1 << 20,), 1, 64, "bf16", input_scale=0.5, seed=1240),
+    Workload("seq1d_8m_b1_c8_f32", (1 << 23,), 1, 8, "f32", seed=1241),
+)
+
+
 def workload(i_or_name) -> Workload:
     if isinstance(i_or_name, int):
         return WORKLOADS[i_or_name]
-    for w in WORKLOADS:
+    for w in WORKLOADS + EXTRA:
         if w.name == i_or_name:
             return w
     raise KeyError(i_or_name)
