@@ -110,6 +110,7 @@ struct L1PassArgs {
   long long npen;            // pencils in the wave
   long long twQ;             // twiddle order Q (W_Q)
   int twP;                   // inverse twiddles: the level's factor (k = outer index mod twP)
+  int lgS, lgP, lgQ;         // log2 of stride, P and twQ (all powers of two)
   int n;                     // volume length
   long long v0;              // first volume of the wave (memory order b C + c)
   const void* a;             // kFirst: k
@@ -124,10 +125,11 @@ struct L1PassArgs {
   int C;
 };
 
-// W_Q^m for 0 <= m < Q (Q a power of two): the ratio is exact while m < 2^24
-__device__ __forceinline__ float2 l1_w(long long m, long long Q) {
+// W_Q^m for 0 <= m < Q, with invQ = 1/Q exact (Q a power of two): the
+// ratio m/Q is exact while m < 2^24
+__device__ __forceinline__ float2 l1_w(unsigned m, float invQ) {
   float s, c;
-  sincospif(-2.f * (static_cast<float>(m) / static_cast<float>(Q)), &s, &c);
+  sincospif(-2.f * (static_cast<float>(m) * invQ), &s, &c);
   return make_float2(c, s);
 }
 
@@ -151,7 +153,7 @@ __device__ __forceinline__ void l1_full_inv(cp (&x)[P2<N>::R1], float2 (&lo)[P2<
 }
 
 template <int N, int KIND, class T, bool DUAL>
-__global__ void __launch_bounds__(kAT, N >= 128 ? 2 : 1) k_l1_pass(const L1PassArgs a) {
+__global__ void __launch_bounds__(kAT, 2) k_l1_pass(const L1PassArgs a) {
   constexpr int G = P2<N>::G, R1 = P2<N>::R1, PPW = 32 / G, P = 2 * N;
   extern __shared__ __align__(16) unsigned char asmem[];
   const Tabs<N> t = tabs_at<N>(asmem);
@@ -163,13 +165,17 @@ __global__ void __launch_bounds__(kAT, N >= 128 ? 2 : 1) k_l1_pass(const L1PassA
   float4* buf = xb + warp * XB<N>::kWarp + pen * XB<N>::kPen;
   const long long per_cta = (kAT / 32) * PPW;
   const long long S = a.stride;
+  const float invQ = ldexpf(1.f, -a.lgQ);
+  // every product below is < Q <= 2^27 (the level's factor times the index
+  // range of the later levels), so 32-bit unsigned arithmetic is exact
   for (long long p0 = static_cast<long long>(blockIdx.x) * per_cta; p0 < a.npen;
        p0 += static_cast<long long>(gridDim.x) * per_cta) {
     const long long p = p0 + warp * PPW + pen;
     const bool act = p < a.npen;
-    const long long o = act ? p / S : 0, i = act ? p % S : 0;
-    const long long start = o * P * S + i;            // first point of the pencil in the wave
-    const long long vol = start / a.P;                // the pencil's volume within the wave
+    const long long o = act ? p >> a.lgS : 0;
+    const unsigned i = act ? static_cast<unsigned>(p & (S - 1)) : 0u;
+    const long long start = ((o * P) << a.lgS) + i;   // first point of the pencil in the wave
+    const long long vol = start >> a.lgP;             // the pencil's volume within the wave
     float2* base = a.grid + start;
     cp x[R1];
     if constexpr (KIND == kFirst) {
@@ -205,11 +211,11 @@ __global__ void __launch_bounds__(kAT, N >= 128 ? 2 : 1) k_l1_pass(const L1PassA
 
     if constexpr (KIND == kFirst || KIND == kFwdMid) {
       // forward twiddle W_Q^{k i} at k = 2f, 2f + 1; store in spectral positions
-      const float2 wi = l1_w(i, a.twQ);
+      const float2 wi = l1_w(i, invQ);
 #pragma unroll
       for (int s = 0; s < R1; ++s) {
-        const long long f = spec_idx<N>(g, s);
-        const float2 w0 = l1_w(((2 * f) * i) % a.twQ, a.twQ);
+        const unsigned f = spec_idx<N>(g, s);
+        const float2 w0 = l1_w((2u * f) * i, invQ);
         const float2 w1 = cmul1(w0, wi);
         if (act) {
           base[(2 * f) * S] = cmul1(make_float2(x[s].re.x, x[s].im.x), w0);
@@ -217,7 +223,7 @@ __global__ void __launch_bounds__(kAT, N >= 128 ? 2 : 1) k_l1_pass(const L1PassA
         }
       }
     } else if constexpr (KIND == kCenter) {
-      const long long vg = a.v0 + vol;
+      const int vg = static_cast<int>(a.v0 + vol);     // B C <= INT_MAX
       const long long bb = vg / a.C, cc = vg % a.C;
       const float2* Sp = a.spec + bb * a.sbs + cc * a.P + (start - vol * a.P);
 #pragma unroll
@@ -234,12 +240,12 @@ __global__ void __launch_bounds__(kAT, N >= 128 ? 2 : 1) k_l1_pass(const L1PassA
       l1_full_inv<N>(x, lo, hi, g, buf, t);
       // conjugate twiddle of the previous level: conj W_Q^{k e}, k = o mod twP,
       // e the element's index along this (last) axis
-      const long long k = o % a.twP;
-      const float2 wk = l1_conj(l1_w((k * N) % a.twQ, a.twQ));
+      const unsigned k = static_cast<unsigned>(o & (a.twP - 1));
+      const float2 wk = l1_conj(l1_w(k * N, invQ));
 #pragma unroll
       for (int s = 0; s < R1; ++s) {
-        const long long j = g + s * G;
-        const float2 w0 = l1_conj(l1_w((k * j) % a.twQ, a.twQ));
+        const unsigned j = g + s * G;
+        const float2 w0 = l1_conj(l1_w(k * j, invQ));
         const float2 w1 = cmul1(w0, wk);
         if (act) {
           base[j] = cmul1(lo[s], w0);
@@ -250,12 +256,13 @@ __global__ void __launch_bounds__(kAT, N >= 128 ? 2 : 1) k_l1_pass(const L1PassA
       float2 lo[R1], hi[R1];
       l1_full_inv<N>(x, lo, hi, g, buf, t);
       // conjugate twiddle of level 0: conj W_P^{k0 (e S + i)}, k0 = o mod twP
-      const long long k = o % a.twP;
-      const float2 wk = l1_conj(l1_w((k * N * S) % a.twQ, a.twQ));
+      const unsigned k = static_cast<unsigned>(o & (a.twP - 1));
+      const unsigned Su = static_cast<unsigned>(S);
+      const float2 wk = l1_conj(l1_w(k * N * Su, invQ));
 #pragma unroll
       for (int s = 0; s < R1; ++s) {
         const long long j = g + s * G;
-        const float2 w0 = l1_conj(l1_w((k * (j * S + i)) % a.twQ, a.twQ));
+        const float2 w0 = l1_conj(l1_w(k * (static_cast<unsigned>(j) * Su + i), invQ));
         const float2 w1 = cmul1(w0, wk);
         if (act) {
           base[j * S] = cmul1(lo[s], w0);

@@ -34,6 +34,12 @@ cudaError_t l1_pass(int N, const hnd2::L1PassArgs& a, cudaStream_t st) {
   }
 }
 
+int ilog2(long long x) {
+  int l = 0;
+  while ((1LL << l) < x) ++l;
+  return l;
+}
+
 template <class T>
 cudaError_t long1d_t(const ConvArgs& c, float2* grid, long long wave, int* launches) {
   const L1Split sp = long1d_split(c.n[0]);
@@ -44,6 +50,7 @@ cudaError_t long1d_t(const ConvArgs& c, float2* grid, long long wave, int* launc
   hnd2::L1PassArgs a{};
   a.grid = grid;
   a.P = P;
+  a.lgP = ilog2(P);
   a.n = c.n[0];
   a.a = c.k;
   a.b = c.v;
@@ -61,15 +68,18 @@ cudaError_t long1d_t(const ConvArgs& c, float2* grid, long long wave, int* launc
     a.v0 = v0;
     auto set_axis = [&](int ax) {
       a.stride = stride[ax];
+      a.lgS = ilog2(stride[ax]);
       a.npen = cnt * P / sp.P[ax];
     };
     // forward: axis 0 from k v, then axis 1 (three levels)
     set_axis(0);
     a.twQ = P;
+    a.lgQ = ilog2(a.twQ);
     e = l1_pass<hnd2::kFirst, T, false>(sp.P[0] / 2, a, c.stream);
     if (e == cudaSuccess && m == 3) {
       set_axis(1);
       a.twQ = static_cast<long long>(sp.P[1]) * sp.P[2];
+      a.lgQ = ilog2(a.twQ);
       e = l1_pass<hnd2::kFwdMid, float, false>(sp.P[1] / 2, a, c.stream);
     }
     // spectrum product on the last axis, with the inverse transform back
@@ -77,12 +87,14 @@ cudaError_t long1d_t(const ConvArgs& c, float2* grid, long long wave, int* launc
       set_axis(m - 1);
       a.twP = sp.P[m - 2];
       a.twQ = static_cast<long long>(sp.P[m - 2]) * sp.P[m - 1];
+      a.lgQ = ilog2(a.twQ);
       e = l1_pass<hnd2::kCenter, float, false>(sp.P[m - 1] / 2, a, c.stream);
     }
     if (e == cudaSuccess && m == 3) {
       set_axis(1);
       a.twP = sp.P[0];
       a.twQ = P;
+      a.lgQ = ilog2(a.twQ);
       e = l1_pass<hnd2::kInvMid, float, false>(sp.P[1] / 2, a, c.stream);
     }
     if (e == cudaSuccess) {
