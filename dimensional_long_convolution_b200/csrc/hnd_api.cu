@@ -125,9 +125,9 @@ hyena_nd_status make_plan(const hyena_nd_problem* p, Plan* pl) {
   if (chunk > p->C) chunk = p->C;
   pl->filter_chunk = static_cast<int>(chunk);
   const size_t ws_filter = static_cast<size_t>(chunk) * static_cast<size_t>(pl->gsz) * 8;
-  // kernel gradient: per channel 2B transformed grids (u and z per sample) and
-  // one accumulator, P^d complex each
-  const size_t per_kg = (2 * static_cast<size_t>(p->B) + 1) * static_cast<size_t>(pl->gsz) * 8;
+  // kernel gradient: per channel B transformed grids (u + i z per sample) and
+  // half an accumulator (two channels share one), P^d complex each
+  const size_t per_kg = (static_cast<size_t>(p->B) + 1) * static_cast<size_t>(pl->gsz) * 8;
   long long kgc = static_cast<long long>(kKgradBudget / per_kg);
   if (kgc < 1) kgc = 1;
   if (kgc > p->C) kgc = p->C;

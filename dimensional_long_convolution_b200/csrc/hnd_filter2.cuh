@@ -184,7 +184,12 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
 }
 
 // In-place full complex forward transform of length P = 2N along one axis of
-// a batch of arrays: element e of pencil (o, i) sits at (o P + e) stride + i.
+// a batch of arrays: element e of pencil (o, i) sits at (o P + e) S + i, with
+// S = 2^lgS the axis stride.  Pencils are counted compactly so that ones known
+// to be zero can be skipped: pencil p has o = p >> lgSc and compact inner
+// index c = p & (2^lgSc - 1), mapped to i = ((c >> lgK) << lgPi) | (c & (2^lgK - 1))
+// (the first 2^lgK of every 2^lgPi inner positions; lgSc = lgK = lgPi = lgS
+// visits every pencil).  All extents are powers of two.
 // One pencil per G lanes of the packed core; a warp takes pencils with
 // consecutive i (adjacent in memory on a strided axis).  Every lane loads its
 // pencil's values before the core's exchange, so the stores cannot overwrite
@@ -196,8 +201,13 @@ struct AxisSmem {
   static constexpr size_t kBytes = Tabs<N>::kBytes + 16ull * XB<N>::kWarp * (kAT / 32);
 };
 
+struct AxisMap {
+  long long npencil;
+  int lgS, lgSc, lgK, lgPi;
+};
+
 template <int N>
-__global__ void __launch_bounds__(kAT) k_fft_axis2(float2* __restrict__ data, long long stride, long long npencil) {
+__global__ void __launch_bounds__(kAT) k_fft_axis2(float2* __restrict__ data, const AxisMap m) {
   constexpr int G = P2<N>::G, R1 = P2<N>::R1, PPW = 32 / G, P = 2 * N;
   extern __shared__ __align__(16) unsigned char asmem[];
   const Tabs<N> t = tabs_at<N>(asmem);
@@ -208,12 +218,15 @@ __global__ void __launch_bounds__(kAT) k_fft_axis2(float2* __restrict__ data, lo
   const int pen = lane / G, g = lane % G;
   float4* buf = xb + warp * XB<N>::kWarp + pen * XB<N>::kPen;
   const long long per_cta = (kAT / 32) * PPW;
-  for (long long p0 = static_cast<long long>(blockIdx.x) * per_cta; p0 < npencil;
+  const long long stride = 1LL << m.lgS;
+  for (long long p0 = static_cast<long long>(blockIdx.x) * per_cta; p0 < m.npencil;
        p0 += static_cast<long long>(gridDim.x) * per_cta) {
     const long long p = p0 + warp * PPW + pen;
-    const bool act = p < npencil;
-    const long long o = act ? p / stride : 0, i = act ? p % stride : 0;
-    float2* base = data + o * P * stride + i;
+    const bool act = p < m.npencil;
+    const long long o = act ? p >> m.lgSc : 0;
+    const long long c = act ? p & ((1LL << m.lgSc) - 1) : 0;
+    const long long i = ((c >> m.lgK) << m.lgPi) | (c & ((1LL << m.lgK) - 1));
+    float2* base = data + ((o * P) << m.lgS) + i;
     float2 lo[R1], hi[R1];
 #pragma unroll
     for (int s = 0; s < R1; ++s) {

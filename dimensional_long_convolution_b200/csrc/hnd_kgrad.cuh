@@ -4,12 +4,20 @@
 // summed over the batch, through zero-padded transforms on the 2n grid
 // (blog "Native multi-dimensional subquadratic operators via input-dependent
 // long convolutions", gradient sections: the kernel gradient by correlation).
-//   k_kg_pad      z or u, zero-padded into complex grids [vol][P^d]
-//   (axis transforms of hnd_filter2.cuh on every grid)
-//   k_kg_corr     acc_c = conj(sum_b Z_b conj(U_b)), b in order (deterministic)
-//   (axis transforms again: the inverse as conj(F(conj(.))))
-//   k_kg_extract  dK[c, t] = Re(acc_c)[t mod P] / prod P
-// Axes are scalars (an unused axis has extent 1).
+//   k_kg_pad      w = u + i z (both real) zero-padded into one complex grid
+//                 per volume [vol][P^d]
+//   (axis transforms of hnd_filter2.cuh, zero pencils skipped)
+//   k_kg_corr     with W the transform of w and Wm = W[-k]:
+//                   U = (W + conj Wm) / 2,  Z = (W - conj Wm) / (2i),
+//                   Z conj(U) = Im(W Wm) / 2 - i (|W|^2 - |Wm|^2) / 4,
+//                 A_c = sum_b Z_b conj(U_b), b in order (deterministic); two
+//                 channels share one grid: acc = conj(A_c1) - i conj(A_c2)
+//   (axis transforms again: F(conj(A1 + i A2)) = conj(IDFT(A1) + i IDFT(A2))
+//    and both inverses are real, so the result is dK_c1 - i dK_c2, unnormalised)
+//   k_kg_extract  dK[c, t] = (Re or -Im)(acc)[t mod P] / prod P
+// Axes are scalars (an unused axis has extent 1).  For the long 1D tier the
+// grids are in the split order of hnd_long1d.cuh, whose frequency negation
+// k -> P - k is taken digit by digit with borrows.
 #pragma once
 
 #include "hnd_fused2.cuh"
@@ -22,8 +30,9 @@ struct KgDims {
 };
 
 template <class T>
-static __global__ void k_kg_pad(const T* __restrict__ a, const T* __restrict__ b, float2* __restrict__ grid,
-                                KgDims d, int B, int C, int c0, int nvol) {
+static __global__ void k_kg_pad(const T* __restrict__ k, const T* __restrict__ v, const T* __restrict__ q,
+                                const T* __restrict__ dy, float2* __restrict__ grid, KgDims d, int B, int C, int c0,
+                                int nvol) {
   const long long gsz = static_cast<long long>(d.P0) * d.P1 * d.P2;
   const long long L = static_cast<long long>(d.n0) * d.n1 * d.n2;
   const long long total = gsz * nvol;
@@ -35,33 +44,74 @@ static __global__ void k_kg_pad(const T* __restrict__ a, const T* __restrict__ b
     r /= d.P2;
     const int s1 = static_cast<int>(r % d.P1);
     const int s0 = static_cast<int>(r / d.P1);
-    float val = 0.f;
+    float2 val = make_float2(0.f, 0.f);
     if (s0 < d.n0 && s1 < d.n1 && s2 < d.n2) {
       const int cl = vv / B, bb = vv % B;
       const long long idx = (static_cast<long long>(bb) * C + c0 + cl) * L + (static_cast<long long>(s0) * d.n1 + s1) * d.n2 + s2;
-      val = Act<T>::ld_g(a + idx) * Act<T>::ld_g(b + idx);
+      val = make_float2(Act<T>::ld_g(k + idx) * Act<T>::ld_g(v + idx), Act<T>::ld_g(q + idx) * Act<T>::ld_g(dy + idx));
     }
-    grid[e] = make_float2(val, 0.f);
+    grid[e] = val;
   }
 }
 
-// gu, gz: [ncc B][P^d] transformed grids (channel-major, sample-minor);
-// acc: [ncc][P^d].
-static __global__ void k_kg_corr(const float2* __restrict__ gu, const float2* __restrict__ gz,
-                                 float2* __restrict__ acc, int B, int ncc, long long gsz) {
-  const long long total = gsz * ncc;
+// Position of -k for the frequency at position r: per axis (P_a - k_a) mod P_a
+// on the natural grid; on the long 1D split order (split0 > 0: factors
+// split0, split1, split2) the digits of P - k with borrows.
+__device__ __forceinline__ long long kg_neg(long long r, const KgDims& d, int split0, int split1, int split2) {
+  if (split0 == 0) {
+    const int k2 = static_cast<int>(r % d.P2);
+    const long long r1 = r / d.P2;
+    const int k1 = static_cast<int>(r1 % d.P1);
+    const int k0 = static_cast<int>(r1 / d.P1);
+    return (static_cast<long long>((d.P0 - k0) % d.P0) * d.P1 + (d.P1 - k1) % d.P1) * d.P2 + (d.P2 - k2) % d.P2;
+  }
+  // r = (k0 P1 + k1) P2 + k2 holds X(k0 + P0 k1 + P0 P1 k2)
+  const int k2 = static_cast<int>(r % split2);
+  const long long r1 = r / split2;
+  const int k1 = static_cast<int>(r1 % split1);
+  const int k0 = static_cast<int>(r1 / split1);
+  int m0, m1, m2;
+  if (k0 != 0) {
+    m0 = split0 - k0, m1 = split1 - 1 - k1, m2 = split2 - 1 - k2;
+  } else if (k1 != 0) {
+    m0 = 0, m1 = split1 - k1, m2 = split2 - 1 - k2;
+  } else {
+    m0 = 0, m1 = 0, m2 = (split2 - k2) % split2;
+  }
+  return (static_cast<long long>(m0) * split1 + m1) * split2 + m2;
+}
+
+// gw: [ncc B][P^d] transformed grids (channel-major, sample-minor);
+// acc: [(ncc + 1) / 2][P^d], channels 2h and 2h + 1 in grid h.
+static __global__ void k_kg_corr(const float2* __restrict__ gw, float2* __restrict__ acc, KgDims d, int B, int ncc,
+                                 long long gsz, int split0, int split1, int split2) {
+  const int nh = (ncc + 1) / 2;
+  const long long total = gsz * nh;
   for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long c = e / gsz, r = e % gsz;
-    float re = 0.f, im = 0.f;
-    for (int b = 0; b < B; ++b) {
-      const long long o = (c * B + b) * gsz + r;
-      const float2 z = gz[o], u = gu[o];
-      re += z.x * u.x + z.y * u.y;      // z conj(u)
-      im += z.y * u.x - z.x * u.y;
+    const long long h = e / gsz, r = e % gsz;
+    const long long rn = kg_neg(r, d, split0, split1, split2);
+    float are[2] = {0.f, 0.f}, aim[2] = {0.f, 0.f};
+    for (int j = 0; j < 2; ++j) {
+      const long long c = 2 * h + j;
+      if (c >= ncc) break;
+      for (int b = 0; b < B; ++b) {
+        const long long o = (c * B + b) * gsz;
+        const float2 w = gw[o + r], wm = gw[o + rn];
+        are[j] += 0.5f * (w.x * wm.y + w.y * wm.x);                                  // Im(W Wm) / 2
+        aim[j] -= 0.25f * ((w.x * w.x + w.y * w.y) - (wm.x * wm.x + wm.y * wm.y));   // -(|W|^2 - |Wm|^2) / 4
+      }
     }
-    acc[e] = make_float2(re, -im);     // conjugated: the inverse runs as a forward transform
+    // conj(A1) - i conj(A2) = (a1r - a2i) + i (-a1i - a2r)
+    acc[e] = make_float2(are[0] - aim[1], -aim[0] - are[1]);
   }
+}
+
+// channel c of the chunk sits in grid c / 2: even c the real part, odd c
+// minus the imaginary part
+__device__ __forceinline__ float kg_part(const float2* acc, long long c, long long gsz, long long slot) {
+  const float2 x = acc[(c >> 1) * gsz + slot];
+  return (c & 1) ? -x.y : x.x;
 }
 
 static __global__ void k_kg_extract(const float2* __restrict__ acc, float* __restrict__ dK, KgDims d, int c0, int ncc,
@@ -81,7 +131,7 @@ static __global__ void k_kg_extract(const float2* __restrict__ acc, float* __res
     const int t0 = i0 - (d.n0 - 1), t1 = i1 - (d.n1 - 1), t2 = i2 - (d.n2 - 1);
     const long long slot = (static_cast<long long>((t0 + d.P0) % d.P0) * d.P1 + (t1 + d.P1) % d.P1) * d.P2 +
                            (t2 + d.P2) % d.P2;
-    dK[(c0 + c) * noff + off] = acc[c * gsz + slot].x * scale;
+    dK[(c0 + c) * noff + off] = kg_part(acc, c, gsz, slot) * scale;
   }
 }
 
@@ -107,7 +157,7 @@ static __global__ void k_kg_extract_periodic(const float2* __restrict__ acc, flo
           const int t0 = u0 - k0 * d.n0, t1 = u1 - k1 * d.n1, t2 = u2 - k2 * d.n2;
           const long long slot = (static_cast<long long>((t0 + d.P0) % d.P0) * d.P1 + (t1 + d.P1) % d.P1) * d.P2 +
                                  (t2 + d.P2) % d.P2;
-          sum += acc[c * gsz + slot].x;
+          sum += kg_part(acc, c, gsz, slot);
         }
     dK[(c0 + c) * nper + off] = sum * scale;
   }

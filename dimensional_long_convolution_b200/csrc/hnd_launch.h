@@ -75,8 +75,11 @@ L1Split long1d_split(int n);
 int long1d_launches_per_transform(int n);
 cudaError_t launch_long1d(const ConvArgs& a, float2* grid, long long wave, int* launches);
 // In-place full forward transforms along every axis of `ngrids` complex grids
-// [P^d] (P_a = 2 n_a), adjacent in memory.
-cudaError_t launch_fft_axes(float2* grid, int ndim, const int* n, long long ngrids, cudaStream_t st);
+// [P^d] (P_a = 2 n_a), adjacent in memory.  skip_zero: the grids hold
+// zero-padded data (zero wherever some s_a >= n_a), so the pencils of each
+// pass that only see such zeros are skipped.
+cudaError_t launch_fft_axes(float2* grid, int ndim, const int* n, long long ngrids, cudaStream_t st,
+                            bool skip_zero = false);
 
 // Kernel-value gradient for channels [c0, c0 + ncc) (all B samples of each).
 struct KgradLaunch {

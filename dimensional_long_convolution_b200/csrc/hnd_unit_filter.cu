@@ -35,32 +35,45 @@ static cudaError_t filter_mlp_go(const hnd2::FilterMlpArgs& fa, long long noff, 
 
 // Full transform of length 2N along one axis of the filter grid.
 template <int N>
-static cudaError_t fft_axis_go(float2* grid, long long stride, long long npen, cudaStream_t st) {
+static cudaError_t fft_axis_go(float2* grid, const hnd2::AxisMap& m, cudaStream_t st) {
   auto kern = hnd2::k_fft_axis2<N>;
   const size_t sm = hnd2::AxisSmem<N>::kBytes;
   cudaError_t e = ensure_smem(kern, sm);
   if (e != cudaSuccess) return e;
   const long long per_cta = (hnd2::kAT / 32) * (32 / hnd2::P2<N>::G);
-  long long blocks = (npen + per_cta - 1) / per_cta;
+  long long blocks = (m.npencil + per_cta - 1) / per_cta;
   if (blocks > 148LL * 16) blocks = 148LL * 16;
-  kern<<<static_cast<unsigned>(blocks), hnd2::kAT, sm, st>>>(grid, stride, npen);
+  if (blocks < 1) blocks = 1;
+  kern<<<static_cast<unsigned>(blocks), hnd2::kAT, sm, st>>>(grid, m);
   return cudaGetLastError();
+}
+
+static int lg2(long long x) {
+  int l = 0;
+  while ((1LL << l) < x) ++l;
+  return l;
+}
+
+static cudaError_t fft_axis_n(int N, float2* grid, const hnd2::AxisMap& m, cudaStream_t st) {
+  switch (N) {
+    case 8: return fft_axis_go<8>(grid, m, st);
+    case 16: return fft_axis_go<16>(grid, m, st);
+    case 32: return fft_axis_go<32>(grid, m, st);
+    case 64: return fft_axis_go<64>(grid, m, st);
+    case 128: return fft_axis_go<128>(grid, m, st);
+    case 256: return fft_axis_go<256>(grid, m, st);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_fft_axis(float2* grid, int ndim, const int* n, int axis, long long ngrids, cudaStream_t st) {
   long long gsz = 1, stride = 1;
   for (int a = 0; a < ndim; ++a) gsz *= 2 * n[a];
   for (int a = axis + 1; a < ndim; ++a) stride *= 2 * n[a];
-  const long long npen = gsz * ngrids / (2 * n[axis]);
-  switch (n[axis]) {
-    case 8: return fft_axis_go<8>(grid, stride, npen, st);
-    case 16: return fft_axis_go<16>(grid, stride, npen, st);
-    case 32: return fft_axis_go<32>(grid, stride, npen, st);
-    case 64: return fft_axis_go<64>(grid, stride, npen, st);
-    case 128: return fft_axis_go<128>(grid, stride, npen, st);
-    case 256: return fft_axis_go<256>(grid, stride, npen, st);
-    default: return cudaErrorInvalidValue;
-  }
+  hnd2::AxisMap m;
+  m.npencil = gsz * ngrids / (2 * n[axis]);
+  m.lgS = m.lgSc = m.lgK = m.lgPi = lg2(stride);
+  return fft_axis_n(n[axis], grid, m, st);
 }
 
 // ------------------------------------------------------------ long 1D
@@ -121,23 +134,32 @@ static cudaError_t l1_inv_conj(float2* grid, const L1Split& sp, long long ngrids
 
 int long1d_launches_per_transform(int n) { return 2 * long1d_split(n).m - 1; }
 
-cudaError_t launch_fft_axes(float2* grid, int ndim, const int* n, long long ngrids, cudaStream_t st) {
+cudaError_t launch_fft_axes(float2* grid, int ndim, const int* n, long long ngrids, cudaStream_t st,
+                            bool skip_zero) {
   long long gsz = 1;
   for (int a = 0; a < ndim; ++a) gsz *= 2 * n[a];
-  long long stride = gsz;
   cudaError_t e = cudaSuccess;
   for (int a = 0; a < ndim && e == cudaSuccess; ++a) {
-    stride /= 2 * n[a];
-    const long long npen = gsz * ngrids / (2 * n[a]);
-    switch (n[a]) {
-      case 8: e = fft_axis_go<8>(grid, stride, npen, st); break;
-      case 16: e = fft_axis_go<16>(grid, stride, npen, st); break;
-      case 32: e = fft_axis_go<32>(grid, stride, npen, st); break;
-      case 64: e = fft_axis_go<64>(grid, stride, npen, st); break;
-      case 128: e = fft_axis_go<128>(grid, stride, npen, st); break;
-      case 256: e = fft_axis_go<256>(grid, stride, npen, st); break;
-      default: e = cudaErrorInvalidValue;
+    long long stride = 1;
+    for (int b = a + 1; b < ndim; ++b) stride *= 2 * n[b];
+    hnd2::AxisMap m;
+    m.lgS = lg2(stride);
+    m.lgSc = m.lgK = m.lgPi = m.lgS;
+    long long inner = stride;
+    if (skip_zero && a + 1 < ndim) {
+      // axes after a are still zero-padded: only s_b < n_b is non-zero there
+      if (a + 2 == ndim) {
+        inner = n[a + 1];
+        m.lgSc = m.lgK = m.lgPi = lg2(inner);
+      } else {
+        inner = static_cast<long long>(n[a + 1]) * n[a + 2];
+        m.lgSc = lg2(inner);
+        m.lgK = lg2(n[a + 2]);
+        m.lgPi = lg2(2LL * n[a + 2]);
+      }
     }
+    m.npencil = gsz / (2LL * n[a] * stride) * inner * ngrids;
+    e = fft_axis_n(n[a], grid, m, st);
   }
   return e;
 }
@@ -209,26 +231,24 @@ static cudaError_t kgrad_chunk_t(const KgradLaunch& g, cudaStream_t st) {
   d.P2 = g.ndim > 2 ? 2 * d.n2 : 1;
   const long long gsz = static_cast<long long>(d.P0) * d.P1 * d.P2;
   const int nvol = g.ncc * g.B;
-  float2* gu = g.grids;
-  float2* gz = gu + gsz * nvol;
-  float2* acc = gz + gsz * nvol;
-  const T* q = static_cast<const T*>(g.q);
-  const T* k = static_cast<const T*>(g.k);
-  const T* v = static_cast<const T*>(g.v);
-  const T* dy = static_cast<const T*>(g.dy);
-  hnd2::k_kg_pad<T><<<grid_for(gsz * nvol, 256), 256, 0, st>>>(k, v, gu, d, g.B, g.C, g.c0, nvol);
-  hnd2::k_kg_pad<T><<<grid_for(gsz * nvol, 256), 256, 0, st>>>(q, dy, gz, d, g.B, g.C, g.c0, nvol);
+  float2* gw = g.grids;
+  float2* acc = gw + gsz * nvol;
+  const int nh = (g.ncc + 1) / 2;
+  hnd2::k_kg_pad<T><<<grid_for(gsz * nvol, 256), 256, 0, st>>>(
+      static_cast<const T*>(g.k), static_cast<const T*>(g.v), static_cast<const T*>(g.q), static_cast<const T*>(g.dy),
+      gw, d, g.B, g.C, g.c0, nvol);
   const bool long1d = g.ndim == 1 && g.n[0] > 256;
   const L1Split sp = long1d ? long1d_split(g.n[0]) : L1Split();
   cudaError_t e = cudaGetLastError();
-  if (e == cudaSuccess)       // gu and gz are adjacent
-    e = long1d ? l1_fwd(gu, sp, 2LL * nvol, st) : launch_fft_axes(gu, g.ndim, g.n, 2LL * nvol, st);
+  if (e == cudaSuccess)
+    e = long1d ? l1_fwd(gw, sp, nvol, st) : launch_fft_axes(gw, g.ndim, g.n, nvol, st, true);
   if (e != cudaSuccess) return e;
-  hnd2::k_kg_corr<<<grid_for(gsz * g.ncc, 256), 256, 0, st>>>(gu, gz, acc, g.B, g.ncc, gsz);
+  hnd2::k_kg_corr<<<grid_for(gsz * nh, 256), 256, 0, st>>>(gw, acc, d, g.B, g.ncc, gsz, long1d ? sp.P[0] : 0,
+                                                             long1d ? sp.P[1] : 1, long1d ? sp.P[2] : 1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  // the accumulator holds conj(sum_b Z conj U): a forward transform gives the
-  // conjugate of the unnormalised inverse, whose real part is wanted
-  e = long1d ? l1_inv_conj(acc, sp, g.ncc, st) : launch_fft_axes(acc, g.ndim, g.n, g.ncc, st);
+  // acc holds conj(A_c1 + i A_c2): a forward transform gives the conjugate of
+  // the unnormalised inverse, dK_c1 - i dK_c2
+  e = long1d ? l1_inv_conj(acc, sp, nh, st) : launch_fft_axes(acc, g.ndim, g.n, nh, st);
   if (e != cudaSuccess) return e;
   const float scale = static_cast<float>(1.0 / static_cast<double>(gsz));
   if (g.circular) {

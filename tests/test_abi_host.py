@@ -148,12 +148,12 @@ def test_kernel_grad_arguments_are_rejected_before_launch():
 
 def test_workspace_covers_the_kernel_gradient():
     """The workspace of every grid holds at least one channel's kernel-gradient
-    grids: (2 B + 1) padded complex grids."""
+    grids: B padded complex grids and one accumulator."""
     for i in range(5):
         wl = W.workload(i)
         p = H.problem(wl.dims, wl.B, wl.C, H.BF16 if wl.io_dtype == "bf16" else H.F32)
         P = int(np.prod([2 * n for n in wl.dims]))
-        assert H.workspace_bytes(p) >= (2 * wl.B + 1) * P * 8
+        assert H.workspace_bytes(p) >= (wl.B + 1) * P * 8
 
 
 @pytest.mark.parametrize("n,B,C", [(512, 2, 3), (4096, 1, 8), (131072, 2, 100), (1 << 23, 1, 2), (1 << 26, 1, 1)])
@@ -164,8 +164,8 @@ def test_long_1d_sizes(n, B, C):
     p = H.problem((n,), B, C, H.F32)
     assert H.spectrum_bytes(p) == C * 2 * n * 8
     ws = H.workspace_bytes(p)
-    assert ws >= 256 + max(2 * n * 8, (2 * B + 1) * 2 * n * 8)
-    assert ws <= 256 + max(96 << 20, 128 << 20, (2 * B + 1) * 2 * n * 8, 64 * 2 * n * 8)
+    assert ws >= 256 + max(2 * n * 8, (B + 1) * 2 * n * 8)
+    assert ws <= 256 + max(96 << 20, 128 << 20, (B + 1) * 2 * n * 8, 64 * 2 * n * 8)
 
 
 def test_long_1d_spectrum_conversion_uses_the_natural_size():
