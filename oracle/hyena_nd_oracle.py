@@ -64,15 +64,19 @@ def fourier_features(t: np.ndarray, dims: Sequence[int], num_freqs: int) -> np.n
     return np.stack(cols, axis=-1)
 
 
-def implicit_kernel(filt, dims: Sequence[int], channels=None, chunk: int = 1 << 18, window: int = 0) -> np.ndarray:
+def implicit_kernel(filt, dims: Sequence[int], channels=None, chunk: int = 1 << 18, window: int = 0,
+                    film=None) -> np.ndarray:
     """K_c(t) for every channel c (or the listed ``channels``) and offset t
     (pages: coordinate MLP with sine activation times a window; reading 4).
     window 0: exp(-alpha_c ||t||_2 / s); window 1: the Gaussian window of the
     arXiv summary ("Methodologie", kernel synthesis: a learnable Gaussian
     window times the coordinate network), read as exp(-alpha_c (||t||_2 / s)^2)
-    with alpha_c the learnable width.  Computed in float64 from the fp32
-    parameters, ``chunk`` offsets at a time to bound memory.  Returns
-    [C, 2n_1-1, ..., 2n_d-1]; index t + (n - 1)."""
+    with alpha_c the learnable width.  ``film`` = (gamma, beta), one value per
+    hidden unit: the per-sample feature-wise modulation of the sine layer,
+    h = sin(gamma (W1 phi + b1) + beta) (reading 18; the pages condition the
+    coordinate network on a per-sample control through FiLM).  Computed in
+    float64 from the fp32 parameters, ``chunk`` offsets at a time to bound
+    memory.  Returns [C, 2n_1-1, ..., 2n_d-1]; index t + (n - 1)."""
     t_all = offsets_grid(dims)
     W1 = filt.W1.astype(np.float64)
     b1 = filt.b1.astype(np.float64)
@@ -84,7 +88,10 @@ def implicit_kernel(filt, dims: Sequence[int], channels=None, chunk: int = 1 << 
     for s0 in range(0, t_all.shape[0], chunk):
         t = t_all[s0: s0 + chunk]
         phi = fourier_features(t, dims, filt.num_freqs)
-        h = np.sin(phi @ W1.T + b1)                      # [N, H]
+        pre = phi @ W1.T + b1                            # [N, H]
+        if film is not None:
+            pre = film[0].astype(np.float64) * pre + film[1].astype(np.float64)
+        h = np.sin(pre)
         mlp = h @ W2.T + b2                              # [N, C]
         r = np.sqrt(np.sum(t * t, axis=-1))              # ||t||_2
         rs = r / float(filt.decay_scale)

@@ -334,6 +334,47 @@ def test_filter_bias_and_second_layer():
     assert np.max(np.abs(K[0])) == 0.0
 
 
+def test_film_identity_and_constant_hidden_layer():
+    """FiLM pins: gamma = 1, beta = 0 is the plain network; gamma = 0 makes
+    every hidden unit the constant sin(beta_h), so K_c = (W2 sin(beta) + b2)_c
+    times the window (a closed form, independent of the offset features)."""
+    dims = (4, 6)
+    p = _params(3, 32)
+    H = p.W1.shape[0]
+    one, zero = np.ones(H, np.float32), np.zeros(H, np.float32)
+    assert np.array_equal(O.implicit_kernel(p, dims, film=(one, zero)), O.implicit_kernel(p, dims))
+    beta = np.linspace(-1.0, 1.0, H).astype(np.float32)
+    K = O.implicit_kernel(p, dims, film=(zero, beta))
+    t = O.offsets_grid(dims)
+    r = np.sqrt(np.sum(t * t, axis=-1)) / p.decay_scale
+    mlp = p.W2.astype(np.float64) @ np.sin(beta.astype(np.float64)) + p.b2
+    want = mlp[:, None] * np.exp(-np.outer(p.alpha.astype(np.float64), r))
+    assert np.max(np.abs(K.reshape(3, -1) - want)) < 1e-12
+
+
+def test_film_by_explicit_loops():
+    """One channel, a few offsets: the modulated sine layer written out unit by
+    unit."""
+    dims = (5,)
+    rng = np.random.default_rng(31)
+    H, F = 8, 16
+    p = W.FilterParams(rng.standard_normal((H, F)).astype(np.float32), rng.standard_normal(H).astype(np.float32),
+                       rng.standard_normal((2, H)).astype(np.float32), rng.standard_normal(2).astype(np.float32),
+                       np.array([0.5, 1.5], np.float32), 4.0)
+    g, b = rng.standard_normal(H).astype(np.float32), rng.standard_normal(H).astype(np.float32)
+    K = O.implicit_kernel(p, dims, film=(g, b))
+    for t in (-4, -1, 0, 3):
+        feats = []
+        for m in range(1, p.num_freqs + 1):
+            feats += [np.sin(np.pi * m * t / 5), np.cos(np.pi * m * t / 5)]
+        out = float(p.b2[1])
+        for hh in range(H):
+            pre = sum(float(p.W1[hh, f]) * feats[f] for f in range(F)) + float(p.b1[hh])
+            out += float(p.W2[1, hh]) * np.sin(float(g[hh]) * pre + float(b[hh]))
+        out *= np.exp(-float(p.alpha[1]) * abs(t) / p.decay_scale)
+        assert abs(K[1, t + 4] - out) < 1e-12
+
+
 # ----------------------------------------------------------- input generators
 def test_bf16_rounding_is_round_to_nearest_even():
     x = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -2.5, 1.0 + 2 ** -9], dtype=np.float32)
