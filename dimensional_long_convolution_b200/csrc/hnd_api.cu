@@ -333,36 +333,74 @@ hyena_nd_status hyena_nd_kernel_grad(const hyena_nd_problem* p, const void* q, c
   return HYENA_ND_OK;
 }
 
+// Argument checks shared by the filter calls; fills `fl` from `f`.
+static hyena_nd_status filter_args(const hyena_nd_filter* f, hnd::FilterLaunch* fl) {
+  if (!f || !f->W1 || !f->b1 || !f->W2 || !f->b2 || !f->alpha) return HYENA_ND_ERR_INVALID_ARG;
+  if (f->window != 0 && f->window != 1) return HYENA_ND_ERR_UNSUPPORTED;
+  if (f->num_freqs < 1 || f->num_freqs > 16 || f->hidden < 1 || f->hidden > 128) return HYENA_ND_ERR_UNSUPPORTED;
+  if (!(f->decay_scale > 0.f) || !std::isfinite(f->decay_scale)) return HYENA_ND_ERR_INVALID_ARG;
+  const void* wp[5] = {f->W1, f->b1, f->W2, f->b2, f->alpha};
+  for (const void* w : wp)
+    if (reinterpret_cast<uintptr_t>(w) & 3u) return HYENA_ND_ERR_MISALIGNED;
+  fl->W1 = f->W1;
+  fl->b1 = f->b1;
+  fl->W2 = f->W2;
+  fl->b2 = f->b2;
+  fl->alpha = f->alpha;
+  fl->num_freqs = f->num_freqs;
+  fl->hidden = f->hidden;
+  fl->decay_scale = f->decay_scale;
+  fl->window = f->window;
+  return HYENA_ND_OK;
+}
+
+static cudaError_t filter_all_chunks(const Plan& pl, const hnd::FilterLaunch& fl, void* spectrum, void* ws,
+                                     cudaStream_t st) {
+  float2* grid = reinterpret_cast<float2*>(static_cast<char*>(ws) + kStatusBytes);
+  for (long long c0 = 0; c0 < pl.C; c0 += pl.filter_chunk) {
+    const int nc = static_cast<int>(pl.C - c0 < pl.filter_chunk ? pl.C - c0 : pl.filter_chunk);
+    cudaError_t e = hnd::launch_filter_chunk(fl, pl.ndim, pl.n, static_cast<int>(c0), nc, grid, spectrum, st);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 hyena_nd_status hyena_nd_filter_spectrum(const hyena_nd_problem* p, const hyena_nd_filter* f, void* spectrum,
                                          void* ws, size_t ws_bytes, void* cuda_stream) {
   Plan pl;
   hyena_nd_status st = make_plan(p, &pl);
   if (st != HYENA_ND_OK) return st;
-  if (!f || !spectrum || !ws || !f->W1 || !f->b1 || !f->W2 || !f->b2 || !f->alpha) return HYENA_ND_ERR_INVALID_ARG;
-  if (f->window != 0 && f->window != 1) return HYENA_ND_ERR_UNSUPPORTED;
-  if (f->num_freqs < 1 || f->num_freqs > 16 || f->hidden < 1 || f->hidden > 128) return HYENA_ND_ERR_UNSUPPORTED;
-  if (!(f->decay_scale > 0.f) || !std::isfinite(f->decay_scale)) return HYENA_ND_ERR_INVALID_ARG;
-  if (!aligned16(spectrum) || !aligned16(ws)) return HYENA_ND_ERR_MISALIGNED;
-  const void* wp[5] = {f->W1, f->b1, f->W2, f->b2, f->alpha};
-  for (const void* w : wp)
-    if (reinterpret_cast<uintptr_t>(w) & 3u) return HYENA_ND_ERR_MISALIGNED;
-  if (ws_bytes < pl.ws_total) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
   hnd::FilterLaunch fl;
-  fl.W1 = f->W1;
-  fl.b1 = f->b1;
-  fl.W2 = f->W2;
-  fl.b2 = f->b2;
-  fl.alpha = f->alpha;
-  fl.num_freqs = f->num_freqs;
-  fl.hidden = f->hidden;
-  fl.decay_scale = f->decay_scale;
-  fl.window = f->window;
+  if ((st = filter_args(f, &fl)) != HYENA_ND_OK) return st;
+  if (!spectrum || !ws) return HYENA_ND_ERR_INVALID_ARG;
+  if (!aligned16(spectrum) || !aligned16(ws)) return HYENA_ND_ERR_MISALIGNED;
+  if (ws_bytes < pl.ws_total) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
   fl.circular = pl.circular;
-  float2* grid = reinterpret_cast<float2*>(static_cast<char*>(ws) + kStatusBytes);
-  for (long long c0 = 0; c0 < pl.C; c0 += pl.filter_chunk) {
-    const int nc = static_cast<int>(pl.C - c0 < pl.filter_chunk ? pl.C - c0 : pl.filter_chunk);
-    cudaError_t e = hnd::launch_filter_chunk(fl, pl.ndim, pl.n, static_cast<int>(c0), nc, grid, spectrum,
-                                             static_cast<cudaStream_t>(cuda_stream));
+  return cuda_status(filter_all_chunks(pl, fl, spectrum, ws, static_cast<cudaStream_t>(cuda_stream)));
+}
+
+hyena_nd_status hyena_nd_filter_spectrum_film(const hyena_nd_problem* p, const hyena_nd_filter* f,
+                                              const float* gamma, const float* beta, void* spectrum,
+                                              int64_t spectrum_batch_stride, void* ws, size_t ws_bytes,
+                                              void* cuda_stream) {
+  Plan pl;
+  hyena_nd_status st = make_plan(p, &pl);
+  if (st != HYENA_ND_OK) return st;
+  hnd::FilterLaunch fl;
+  if ((st = filter_args(f, &fl)) != HYENA_ND_OK) return st;
+  if (!gamma || !beta || !spectrum || !ws) return HYENA_ND_ERR_INVALID_ARG;
+  if (!aligned16(spectrum) || !aligned16(ws)) return HYENA_ND_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(gamma) & 3u) || (reinterpret_cast<uintptr_t>(beta) & 3u))
+    return HYENA_ND_ERR_MISALIGNED;
+  if (spectrum_batch_stride % 16 != 0) return HYENA_ND_ERR_MISALIGNED;
+  if (spectrum_batch_stride < static_cast<int64_t>(pl.spec_bytes)) return HYENA_ND_ERR_INVALID_ARG;
+  if (ws_bytes < pl.ws_total) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
+  fl.circular = pl.circular;
+  for (long long b = 0; b < pl.B; ++b) {
+    fl.gamma = gamma + b * f->hidden;
+    fl.beta = beta + b * f->hidden;
+    void* sb = static_cast<char*>(spectrum) + b * spectrum_batch_stride;
+    cudaError_t e = filter_all_chunks(pl, fl, sb, ws, static_cast<cudaStream_t>(cuda_stream));
     if (e != cudaSuccess) return HYENA_ND_ERR_CUDA;
   }
   return HYENA_ND_OK;

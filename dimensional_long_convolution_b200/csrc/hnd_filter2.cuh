@@ -34,6 +34,8 @@ struct FilterMlpArgs {
   int n[3];
   int c0, nc;                    // channel chunk [c0, c0 + nc)
   float2* grid;                  // [nc][P^d]
+  const float* gamma = nullptr;  // FiLM: sin(gamma (W1 phi + b1) + beta), [hidden] each; null = plain
+  const float* beta = nullptr;
 };
 
 // Shared layout (floats), HP = hidden rounded up to a multiple of 32:
@@ -135,6 +137,16 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
         for (int i = 0; i < 4; ++i)
 #pragma unroll
           for (int jj = 0; jj < 4; ++jj) acc[i][4 * j4 + jj] = fmaf(wv[jj], pv[i], acc[i][4 * j4 + jj]);
+      }
+    }
+    if (a.gamma) {       // per-sample feature-wise modulation of the sine layer
+#pragma unroll
+      for (int j = 0; j < HG; ++j) {
+        const int hu = grp * HG + j;
+        const float gm = hu < a.hidden ? __ldg(a.gamma + hu) : 0.f;
+        const float bt = hu < a.hidden ? __ldg(a.beta + hu) : 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i][j] = fmaf(gm, acc[i][j], bt);
       }
     }
 #pragma unroll

@@ -57,6 +57,8 @@ struct FilterLaunch {
   float decay_scale;
   int window = 0;         // 0: exp(-alpha |t| / s), 1: exp(-alpha (|t| / s)^2)
   int circular = 0;       // 1: periodic representatives (circular mode)
+  const float* gamma = nullptr;   // FiLM modulation of the sine layer ([hidden] each), or null
+  const float* beta = nullptr;
 };
 cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, int c0, int nc, float2* grid,
                                 void* spectrum, cudaStream_t st);

@@ -191,6 +191,8 @@ cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, i
   fa.c0 = c0;
   fa.nc = nc;
   fa.grid = grid;
+  fa.gamma = f.gamma;
+  fa.beta = f.beta;
   const int HP = (f.hidden + 31) / 32 * 32;
   e = HP <= 32 ? filter_mlp_go<32>(fa, noff, st)
       : HP <= 64 ? filter_mlp_go<64>(fa, noff, st)

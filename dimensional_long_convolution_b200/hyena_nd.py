@@ -35,6 +35,7 @@ EXPORTED = (
     "hyena_nd_workspace_bytes",
     "hyena_nd_workspace_init",
     "hyena_nd_filter_spectrum",
+    "hyena_nd_filter_spectrum_film",
     "hyena_nd_fftconv",
     "hyena_nd_fftconv_batched",
     "hyena_nd_fftconv_backward",
@@ -100,6 +101,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "hyena_nd_workspace_bytes": (sz, [P]),
         "hyena_nd_workspace_init": (ctypes.c_int, [vp, sz, vp]),
         "hyena_nd_filter_spectrum": (ctypes.c_int, [P, ctypes.POINTER(Filter), vp, vp, sz, vp]),
+        "hyena_nd_filter_spectrum_film": (ctypes.c_int, [P, ctypes.POINTER(Filter), vp, vp, vp, i64, vp, sz, vp]),
         "hyena_nd_fftconv": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
         "hyena_nd_fftconv_batched": (ctypes.c_int, [P, vp, vp, vp, vp, i64, vp, vp, sz, vp]),
         "hyena_nd_fftconv_backward": (ctypes.c_int, [P, vp, vp, vp, vp, i64, vp, vp, vp, vp, vp, sz, vp]),
@@ -144,6 +146,12 @@ def workspace_init(ws: int, ws_bytes: int, stream: int = 0) -> int:
 
 def filter_spectrum(p: Problem, f: Filter, spectrum: int, ws: int, ws_bytes: int, stream: int = 0) -> int:
     return load().hyena_nd_filter_spectrum(ctypes.byref(p), ctypes.byref(f), spectrum, ws, ws_bytes, stream)
+
+
+def filter_spectrum_film(p: Problem, f: Filter, gamma: int, beta: int, spectrum: int, spectrum_batch_stride: int,
+                         ws: int, ws_bytes: int, stream: int = 0) -> int:
+    return load().hyena_nd_filter_spectrum_film(ctypes.byref(p), ctypes.byref(f), gamma, beta, spectrum,
+                                                spectrum_batch_stride, ws, ws_bytes, stream)
 
 
 def fftconv(p: Problem, q: int, k: int, v: int, spectrum_c: int, y: int, ws: int, ws_bytes: int,
@@ -251,6 +259,27 @@ class HyenaND:
         f.window = int(window)
         check(filter_spectrum(self.p, f, self.spectrum.data_ptr(), self.ws.data_ptr(), self.ws_bytes,
                               self._stream()), "filter_spectrum")
+
+    def set_filter_film(self, W1, b1, W2, b2, alpha, decay_scale: float, gamma, beta, num_freqs: int = 8,
+                        window: int = 0):
+        """Per-sample spectra from one filter network under per-sample FiLM
+        modulation gamma, beta [B, hidden]: returns a complex64 tensor holding
+        B spectra back to back (the stride to pass to the convolution calls is
+        ``self.spec_bytes``)."""
+        t = [x.to(self.device, self.torch.float32).contiguous() for x in (W1, b1, W2, b2, alpha, gamma, beta)]
+        f = Filter()
+        f.num_freqs = int(num_freqs)
+        f.hidden = int(t[0].shape[0])
+        f.W1, f.b1, f.W2, f.b2, f.alpha = (x.data_ptr() for x in t[:5])
+        f.decay_scale = float(decay_scale)
+        f.window = int(window)
+        if tuple(t[5].shape) != (self.B, f.hidden) or tuple(t[6].shape) != (self.B, f.hidden):
+            raise ValueError("gamma and beta must be [B, hidden]")
+        out = self.torch.empty(self.B * (self.spec_bytes // 8), dtype=self.torch.complex64, device=self.device)
+        check(filter_spectrum_film(self.p, f, t[5].data_ptr(), t[6].data_ptr(), out.data_ptr(), self.spec_bytes,
+                                   self.ws.data_ptr(), self.ws_bytes, self._stream()), "filter_spectrum_film")
+        self._film_params = t
+        return out
 
     def import_spectrum(self, natural) -> None:
         nat = natural.to(self.device, self.torch.complex64).contiguous()

@@ -116,7 +116,8 @@ typedef struct {
 } hyena_nd_filter;
 
 /* Size in bytes of the spectrum buffer for `p` (C channels of
- * prod_{a<d-1} P_a * (P_d/2 + 1) complex64 values).  0 if `p` is invalid. */
+ * prod_{a<d-1} P_a * (P_d/2 + 1) complex64 values; 2n for the long 1D tier).
+ * 0 if `p` is invalid or unsupported. */
 HYENA_ND_API size_t hyena_nd_spectrum_bytes(const hyena_nd_problem* p);
 
 /* Workspace bytes needed by every call below for problem `p` (a pure
@@ -139,6 +140,25 @@ HYENA_ND_API hyena_nd_status hyena_nd_workspace_init(void* ws, size_t ws_bytes, 
 HYENA_ND_API hyena_nd_status hyena_nd_filter_spectrum(const hyena_nd_problem* p, const hyena_nd_filter* f,
                                          void* spectrum, void* ws, size_t ws_bytes,
                                          void* cuda_stream);
+
+/* Call 1 per sample with FiLM conditioning: the pages make the kernel depend
+ * on the whole input sample through a control z(x) that modulates the
+ * coordinate network feature-wise (FiLM) (arXiv 2607.19378 summary,
+ * "Methodologie", input-dependent kernels via registers and FiLM).  With the
+ * modulation of sample b given as gamma[b], beta[b] (one value per hidden
+ * unit), the hidden layer becomes
+ *     h_b = sin(gamma[b] (.) (W1 phi + b1) + beta[b])
+ * and sample b's spectrum is written at spectrum + b * spectrum_batch_stride
+ * (bytes), in library order, ready for the batched and backward calls with
+ * the same stride.  Mapping z(x) to (gamma, beta) is the caller's.
+ *   gamma, beta  device fp32 [B, hidden], 4-byte aligned.
+ *   spectrum_batch_stride  >= hyena_nd_spectrum_bytes(p), a multiple of 16.
+ * Errors as hyena_nd_filter_spectrum; a stride below one spectrum is
+ * HYENA_ND_ERR_INVALID_ARG. */
+HYENA_ND_API hyena_nd_status hyena_nd_filter_spectrum_film(const hyena_nd_problem* p, const hyena_nd_filter* f,
+                                              const float* gamma, const float* beta, void* spectrum,
+                                              int64_t spectrum_batch_stride, void* ws, size_t ws_bytes,
+                                              void* cuda_stream);
 
 /* Call 2 (one volume): the gated linear convolution for one (b, c) pair.
  * `p->B` and `p->C` must both be 1; `spectrum_c` holds that channel's

@@ -21,7 +21,7 @@ def _declared():
 def test_library_exports_every_declared_symbol():
     lib = H.load()
     names = _declared()
-    assert len(names) == len(H.EXPORTED) == 15
+    assert len(names) == len(H.EXPORTED) == 16
     assert set(names) == set(H.EXPORTED)
     for n in names:
         assert getattr(lib, n) is not None
@@ -215,6 +215,26 @@ def test_filter_arguments_are_checked():
     assert H.filter_spectrum(p, f, s, ws, wsb) == H.ERR_MISALIGNED
     f.W2 = A + 7 * STEP
     assert H.filter_spectrum(p, f, s, ws, wsb - 1) == H.ERR_WORKSPACE_TOO_SMALL
+
+
+def test_film_filter_arguments_are_checked():
+    p = H.problem((32, 32), 2, 4)
+    _, _, _, s, _, ws = _ptrs()
+    wsb = H.workspace_bytes(p)
+    sb = H.spectrum_bytes(p)
+    f = H.Filter()
+    f.num_freqs, f.hidden = 8, 64
+    f.W1 = f.b1 = f.W2 = f.b2 = f.alpha = A + 7 * STEP
+    f.decay_scale, f.window = 32.0, 0
+    g = bt = A + 8 * STEP
+    assert H.filter_spectrum_film(p, f, 0, bt, s, sb, ws, wsb) == H.ERR_INVALID_ARG          # no gamma
+    assert H.filter_spectrum_film(p, f, g, 0, s, sb, ws, wsb) == H.ERR_INVALID_ARG           # no beta
+    assert H.filter_spectrum_film(p, f, g + 2, bt, s, sb, ws, wsb) == H.ERR_MISALIGNED
+    assert H.filter_spectrum_film(p, f, g, bt, s, sb - 16, ws, wsb) == H.ERR_INVALID_ARG     # stride below one spectrum
+    assert H.filter_spectrum_film(p, f, g, bt, s, sb + 8, ws, wsb) == H.ERR_MISALIGNED
+    assert H.filter_spectrum_film(p, f, g, bt, s, sb, ws, wsb - 1) == H.ERR_WORKSPACE_TOO_SMALL
+    f.window = 2
+    assert H.filter_spectrum_film(p, f, g, bt, s, sb, ws, wsb) == H.ERR_UNSUPPORTED
 
 
 def test_spectrum_conversion_checks():
