@@ -21,8 +21,16 @@ thread_local int g_last_launches = 0;
 
 constexpr size_t kStatusBytes = 256;                  // status word + padding
 constexpr size_t kWaveBudget = size_t(96) << 20;      // multi-pass intermediate per wave (measured best of 24/48/96 MiB)
-constexpr size_t kFilterBudget = size_t(64) << 20;    // filter grid per channel chunk
-constexpr int kFilterMaxChunk = 64;
+#ifndef HND_FILTER_MB
+#define HND_FILTER_MB 256
+#endif
+#ifndef HND_FILTER_MAXC
+#define HND_FILTER_MAXC 128
+#endif
+// filter grids per channel chunk: each chunk evaluates the hidden layer once
+// per offset, so fewer, larger chunks save that work at the cost of workspace
+constexpr size_t kFilterBudget = size_t(HND_FILTER_MB) << 20;
+constexpr int kFilterMaxChunk = HND_FILTER_MAXC;
 constexpr size_t kKgradBudget = size_t(128) << 20;    // kernel-gradient grids per channel chunk
 #ifndef HND_L1_WAVE_MB
 #define HND_L1_WAVE_MB 96
@@ -49,6 +57,7 @@ struct Plan {
   size_t ws_total = 0;
   size_t spec_bytes = 0;
   size_t nat_bytes = 0;     // natural-order half spectrum (export / import)
+  size_t filter_grid_bytes = 0;   // filter call: chunk grids (the tables follow)
 };
 
 bool pow2_in(long long x, long long lo, long long hi) { return x >= lo && x <= hi && (x & (x - 1)) == 0; }
@@ -124,7 +133,9 @@ hyena_nd_status make_plan(const hyena_nd_problem* p, Plan* pl) {
   if (chunk > kFilterMaxChunk) chunk = kFilterMaxChunk;
   if (chunk > p->C) chunk = p->C;
   pl->filter_chunk = static_cast<int>(chunk);
-  const size_t ws_filter = static_cast<size_t>(chunk) * static_cast<size_t>(pl->gsz) * 8;
+  // the chunk's grids, then the first-layer tables (for the largest hidden width)
+  pl->filter_grid_bytes = (static_cast<size_t>(chunk) * static_cast<size_t>(pl->gsz) * 8 + 255) / 256 * 256;
+  const size_t ws_filter = pl->filter_grid_bytes + static_cast<size_t>(hnd::filter_table_bytes(128, pl->ndim, pl->n));
   // kernel gradient: per channel B transformed grids (u + i z per sample) and
   // half an accumulator (two channels share one), P^d complex each
   const size_t per_kg = (static_cast<size_t>(p->B) + 1) * static_cast<size_t>(pl->gsz) * 8;
@@ -376,6 +387,12 @@ hyena_nd_status hyena_nd_filter_spectrum(const hyena_nd_problem* p, const hyena_
   if (!aligned16(spectrum) || !aligned16(ws)) return HYENA_ND_ERR_MISALIGNED;
   if (ws_bytes < pl.ws_total) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
   fl.circular = pl.circular;
+  if (hnd::filter_table_bytes(fl.hidden, pl.ndim, pl.n) > 0) {
+    float* tab = reinterpret_cast<float*>(static_cast<char*>(ws) + kStatusBytes + pl.filter_grid_bytes);
+    if (hnd::launch_filter_tables(fl, pl.ndim, pl.n, tab, static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
+      return HYENA_ND_ERR_CUDA;
+    fl.tab = tab;
+  }
   return cuda_status(filter_all_chunks(pl, fl, spectrum, ws, static_cast<cudaStream_t>(cuda_stream)));
 }
 
@@ -396,6 +413,12 @@ hyena_nd_status hyena_nd_filter_spectrum_film(const hyena_nd_problem* p, const h
   if (spectrum_batch_stride < static_cast<int64_t>(pl.spec_bytes)) return HYENA_ND_ERR_INVALID_ARG;
   if (ws_bytes < pl.ws_total) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
   fl.circular = pl.circular;
+  if (hnd::filter_table_bytes(fl.hidden, pl.ndim, pl.n) > 0) {
+    float* tab = reinterpret_cast<float*>(static_cast<char*>(ws) + kStatusBytes + pl.filter_grid_bytes);
+    if (hnd::launch_filter_tables(fl, pl.ndim, pl.n, tab, static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
+      return HYENA_ND_ERR_CUDA;
+    fl.tab = tab;
+  }
   for (long long b = 0; b < pl.B; ++b) {
     fl.gamma = gamma + b * f->hidden;
     fl.beta = beta + b * f->hidden;

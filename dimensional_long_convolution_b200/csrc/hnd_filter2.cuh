@@ -36,32 +36,74 @@ struct FilterMlpArgs {
   float2* grid;                  // [nc][P^d]
   const float* gamma = nullptr;  // FiLM: sin(gamma (W1 phi + b1) + beta), [hidden] each; null = plain
   const float* beta = nullptr;
+  const float* tab = nullptr;    // per-axis first-layer tables (k_filter_tables)
 };
 
+// The first layer is separable over the axes: the features of axis a depend on
+// t_a alone, so W1 phi(t) = sum_a T_a[t_a] with
+//   T_a[h][t_a] = sum_m W1[h, f(a,m,sin)] sin(pi m t_a / n_a) + W1[h, f(a,m,cos)] cos(pi m t_a / n_a),
+// tabulated once per call for t_a in [-(n_a - 1), n_a - 1] (index t_a + n_a - 1),
+// axis a's table at HP * sum_{b<a} (2 n_b - 1), h-major.  The hidden unit of
+// offset t is then sin(b1 + T_0[t_0] + T_1[t_1] + T_2[t_2]) (FiLM applied to
+// the sum): ndim table reads per unit instead of 2 M ndim products.
+inline long long filter_table_floats(int HP, int ndim, const int* n) {
+  long long e = 0;
+  for (int a = 0; a < ndim; ++a) e += 2LL * n[a] - 1;
+  return e * HP;
+}
+
+static __global__ void k_filter_tables(const float* __restrict__ W1, int hidden, int HP, int num_freqs, int ndim,
+                                       int n0, int n1, int n2, float* __restrict__ tab) {
+  const int nn[3] = {n0, n1, n2};
+  const int fin = 2 * num_freqs * ndim;
+  long long base = 0;
+  for (int a = 0; a < ndim; ++a) {
+    const int E = 2 * nn[a] - 1;
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < HP * E; e += gridDim.x * blockDim.x) {
+      const int h = e / E, j = e % E;
+      const int t = j - (nn[a] - 1);
+      float acc = 0.f;
+      if (h < hidden) {
+        for (int m = 1; m <= num_freqs; ++m) {
+          float sv, cv;
+          sincospif(static_cast<float>(m) * (static_cast<float>(t) / static_cast<float>(nn[a])), &sv, &cv);
+          const int f = 2 * (a * num_freqs + m - 1);
+          acc = fmaf(__ldg(W1 + static_cast<long long>(h) * fin + f), sv, acc);
+          acc = fmaf(__ldg(W1 + static_cast<long long>(h) * fin + f + 1), cv, acc);
+        }
+      }
+      tab[base + e] = acc;
+    }
+    base += static_cast<long long>(HP) * E;
+  }
+}
+
 // Shared layout (floats), HP = hidden rounded up to a multiple of 32:
-//   phi[fin][kFO] | w1[fin][HP] | hid[HP][kFO] | w2[HP][kFC] | b1[HP] | rad[kFO] | slot[kFO] (int)
+//   [phi[fin][kFO] | w1[fin][HP]] | hid[HP][kFO] | w2[HP][kFC] | b1[HP] | rad[kFO] |
+//   slot[kFO] (int) | tix[3][kFO] (int); the bracketed part only on the feature path
 template <int HP>
 struct FilterSmem {
-  static size_t bytes(int fin) {
-    return sizeof(float) * (static_cast<size_t>(fin) * kFO + static_cast<size_t>(fin) * HP +
-                            static_cast<size_t>(HP) * kFO + static_cast<size_t>(HP) * kFC + HP + kFO) +
-           sizeof(int) * kFO;
+  static size_t bytes(int fin, bool tab) {
+    const size_t feat = tab ? 0 : static_cast<size_t>(fin) * (kFO + HP);
+    return sizeof(float) * (feat + static_cast<size_t>(HP) * kFO + static_cast<size_t>(HP) * kFC + HP + kFO) +
+           sizeof(int) * 4 * kFO;
   }
 };
 
-template <int HP>
+template <int HP, bool TAB>
 __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
   static_assert(HP % 32 == 0 && HP <= 128, "hidden tile");
   constexpr int HG = HP / 8;                 // hidden outputs per thread in the hidden layer
   extern __shared__ __align__(16) float fsm[];
   const int fin = a.fin;
-  float* phi = fsm;                          // [fin][kFO]
-  float* w1 = phi + fin * kFO;               // [fin][HP]
-  float* hid = w1 + fin * HP;                // [HP][kFO]
+  float* phi = fsm;                          // [fin][kFO] (feature path)
+  float* w1 = phi + (TAB ? 0 : fin * kFO);   // [fin][HP]  (feature path)
+  float* hid = w1 + (TAB ? 0 : fin * HP);    // [HP][kFO]
   float* w2 = hid + HP * kFO;                // [HP][kFC]
   float* b1 = w2 + HP * kFC;                 // [HP]
   float* rad = b1 + HP;                      // [kFO]
   int* slot = reinterpret_cast<int*>(rad + kFO);
+  int* tix = slot + kFO;                     // [3][kFO]: table column per axis (table path)
   const int tid = threadIdx.x;
   // axes as scalars (an unused axis has extent 1 and offset 0)
   const int n0 = a.n[0], n1 = a.ndim > 1 ? a.n[1] : 1, n2 = a.ndim > 2 ? a.n[2] : 1;
@@ -86,9 +128,11 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
 
   // first layer weights (zero-padded to HP hidden units: sin(0) = 0 and the
   // padded output weights are zero, so the padding contributes nothing)
-  for (int i = tid; i < fin * HP; i += kFT) {
-    const int f = i / HP, h = i % HP;
-    w1[i] = h < a.hidden ? __ldg(a.W1 + static_cast<long long>(h) * fin + f) : 0.f;
+  if constexpr (!TAB) {
+    for (int i = tid; i < fin * HP; i += kFT) {
+      const int f = i / HP, h = i % HP;
+      w1[i] = h < a.hidden ? __ldg(a.W1 + static_cast<long long>(h) * fin + f) : 0.f;
+    }
   }
   for (int h = tid; h < HP; h += kFT) b1[h] = h < a.hidden ? __ldg(a.b1 + h) : 0.f;
   // offsets of this tile: radius and slot (offset t at t mod P per axis)
@@ -102,57 +146,81 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
     rad[o] = a.window == 1 ? rs * rs : rs;
     const int s0 = (t0 + P0) % P0, s1 = (t1 + P1) % P1, s2 = (t2 + P2) % P2;
     slot[o] = (s0 * P1 + s1) * P2 + s2;
+    if constexpr (TAB) {
+      tix[o] = rep(t0, n0) + n0 - 1;
+      tix[kFO + o] = rep(t1, n1) + n1 - 1;
+      tix[2 * kFO + o] = rep(t2, n2) + n2 - 1;
+    }
   }
-  // Fourier features, phi[(ax M + m - 1) 2 + {0: sin, 1: cos}][o]
-  const int M = a.num_freqs;
-  for (int i = tid; i < kFO * a.ndim * M; i += kFT) {
-    const int o = i % kFO, q = i / kFO, m = q % M + 1, ax = q / M;
-    int t0, t1, t2;
-    offset_of(o, t0, t1, t2);
-    const int nax = ax == 0 ? n0 : (ax == 1 ? n1 : n2);
-    const int tax = rep(ax == 0 ? t0 : (ax == 1 ? t1 : t2), nax);
-    float sv, cv;
-    sincospif(static_cast<float>(m) * (static_cast<float>(tax) / static_cast<float>(nax)), &sv, &cv);
-    phi[(2 * (ax * M + m - 1)) * kFO + o] = sv;
-    phi[(2 * (ax * M + m - 1) + 1) * kFO + o] = cv;
+  if constexpr (!TAB) {
+    // Fourier features, phi[(ax M + m - 1) 2 + {0: sin, 1: cos}][o]
+    const int M = a.num_freqs;
+    for (int i = tid; i < kFO * a.ndim * M; i += kFT) {
+      const int o = i % kFO, q = i / kFO, m = q % M + 1, ax = q / M;
+      int t0, t1, t2;
+      offset_of(o, t0, t1, t2);
+      const int nax = ax == 0 ? n0 : (ax == 1 ? n1 : n2);
+      const int tax = rep(ax == 0 ? t0 : (ax == 1 ? t1 : t2), nax);
+      float sv, cv;
+      sincospif(static_cast<float>(m) * (static_cast<float>(tax) / static_cast<float>(nax)), &sv, &cv);
+      phi[(2 * (ax * M + m - 1)) * kFO + o] = sv;
+      phi[(2 * (ax * M + m - 1) + 1) * kFO + o] = cv;
+    }
   }
   __syncthreads();
 
-  // hidden layer: thread (og, hg) computes offsets 4 og .. 4 og + 3 x units hg HG ..
   const int og = tid % 32, grp = tid / 32;
-  {
-    float acc[4][HG];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < HG; ++j) acc[i][j] = b1[grp * HG + j];
-    for (int f = 0; f < fin; ++f) {
-      const float4 p = *reinterpret_cast<const float4*>(phi + f * kFO + 4 * og);
-      const float pv[4] = {p.x, p.y, p.z, p.w};
-#pragma unroll
-      for (int j4 = 0; j4 < HG / 4; ++j4) {
-        const float4 w = *reinterpret_cast<const float4*>(w1 + f * HP + grp * HG + 4 * j4);
-        const float wv[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int jj = 0; jj < 4; ++jj) acc[i][4 * j4 + jj] = fmaf(wv[jj], pv[i], acc[i][4 * j4 + jj]);
-      }
+  if constexpr (TAB) {
+    // hidden layer from the per-axis tables: thread i -> offset o = i % kFO
+    // (consecutive offsets read consecutive table columns), unit h = i / kFO
+    const int E0t = 2 * n0 - 1, E1t = 2 * n1 - 1, E2t = 2 * n2 - 1;
+    const float* T0 = a.tab;
+    const float* T1 = T0 + static_cast<long long>(HP) * E0t;
+    const float* T2 = T1 + static_cast<long long>(HP) * (a.ndim > 1 ? E1t : 0);
+    for (int i = tid; i < HP * kFO; i += kFT) {
+      const int o = i % kFO, h = i / kFO;
+      float pre = b1[h] + __ldg(T0 + h * E0t + tix[o]);
+      if (a.ndim > 1) pre += __ldg(T1 + h * E1t + tix[kFO + o]);
+      if (a.ndim > 2) pre += __ldg(T2 + h * E2t + tix[2 * kFO + o]);
+      if (a.gamma && h < a.hidden) pre = fmaf(__ldg(a.gamma + h), pre, __ldg(a.beta + h));
+      hid[h * kFO + o] = h < a.hidden ? sinf(pre) : 0.f;
     }
-    if (a.gamma) {       // per-sample feature-wise modulation of the sine layer
+  } else {
+    // hidden layer: thread (og, hg) computes offsets 4 og .. 4 og + 3 x units hg HG ..
+    {
+      float acc[4][HG];
 #pragma unroll
-      for (int j = 0; j < HG; ++j) {
-        const int hu = grp * HG + j;
-        const float gm = hu < a.hidden ? __ldg(a.gamma + hu) : 0.f;
-        const float bt = hu < a.hidden ? __ldg(a.beta + hu) : 0.f;
+      for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[i][j] = fmaf(gm, acc[i][j], bt);
+        for (int j = 0; j < HG; ++j) acc[i][j] = b1[grp * HG + j];
+      for (int f = 0; f < fin; ++f) {
+        const float4 p = *reinterpret_cast<const float4*>(phi + f * kFO + 4 * og);
+        const float pv[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+        for (int j4 = 0; j4 < HG / 4; ++j4) {
+          const float4 w = *reinterpret_cast<const float4*>(w1 + f * HP + grp * HG + 4 * j4);
+          const float wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) acc[i][4 * j4 + jj] = fmaf(wv[jj], pv[i], acc[i][4 * j4 + jj]);
+        }
       }
-    }
+      if (a.gamma) {       // per-sample feature-wise modulation of the sine layer
 #pragma unroll
-    for (int j = 0; j < HG; ++j)
-      *reinterpret_cast<float4*>(hid + (grp * HG + j) * kFO + 4 * og) =
-          make_float4(sinf(acc[0][j]), sinf(acc[1][j]), sinf(acc[2][j]), sinf(acc[3][j]));
+        for (int j = 0; j < HG; ++j) {
+          const int hu = grp * HG + j;
+          const float gm = hu < a.hidden ? __ldg(a.gamma + hu) : 0.f;
+          const float bt = hu < a.hidden ? __ldg(a.beta + hu) : 0.f;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[i][j] = fmaf(gm, acc[i][j], bt);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < HG; ++j)
+        *reinterpret_cast<float4*>(hid + (grp * HG + j) * kFO + 4 * og) =
+            make_float4(sinf(acc[0][j]), sinf(acc[1][j]), sinf(acc[2][j]), sinf(acc[3][j]));
+    }
   }
 
   // output layer over channel tiles: thread (og, cg) -> offsets 4 og.., channels 4 cg..

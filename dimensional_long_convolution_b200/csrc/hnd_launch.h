@@ -59,7 +59,12 @@ struct FilterLaunch {
   int circular = 0;       // 1: periodic representatives (circular mode)
   const float* gamma = nullptr;   // FiLM modulation of the sine layer ([hidden] each), or null
   const float* beta = nullptr;
+  const float* tab = nullptr;     // per-axis first-layer tables (launch_filter_tables), or null
 };
+// Per-axis first-layer tables of the filter network (bytes; 0 where the
+// feature path is used instead), and the launch that fills them.
+long long filter_table_bytes(int hidden, int ndim, const int* n);
+cudaError_t launch_filter_tables(const FilterLaunch& f, int ndim, const int* n, float* tab, cudaStream_t st);
 cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, int c0, int nc, float2* grid,
                                 void* spectrum, cudaStream_t st);
 cudaError_t launch_spec_convert(int ndim, const int* n, long long C, const void* src, void* dst, bool to_natural,

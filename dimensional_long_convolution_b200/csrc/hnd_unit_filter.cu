@@ -23,13 +23,33 @@ static unsigned grid_for(long long work, int threads) {
   return static_cast<unsigned>(b);
 }
 
-template <int HP>
-static cudaError_t filter_mlp_go(const hnd2::FilterMlpArgs& fa, long long noff, cudaStream_t st) {
-  auto kern = hnd2::k_filter_mlp2<HP>;
-  cudaError_t e = ensure_smem(kern, hnd2::FilterSmem<HP>::bytes(96));     // the largest feature count
+template <int HP, bool TAB>
+static cudaError_t filter_mlp_go_t(const hnd2::FilterMlpArgs& fa, long long noff, cudaStream_t st) {
+  auto kern = hnd2::k_filter_mlp2<HP, TAB>;
+  cudaError_t e = ensure_smem(kern, hnd2::FilterSmem<HP>::bytes(96, TAB));     // the largest feature count
   if (e != cudaSuccess) return e;
   const long long blocks = (noff + hnd2::kFO - 1) / hnd2::kFO;
-  kern<<<static_cast<unsigned>(blocks), hnd2::kFT, hnd2::FilterSmem<HP>::bytes(fa.fin), st>>>(fa);
+  kern<<<static_cast<unsigned>(blocks), hnd2::kFT, hnd2::FilterSmem<HP>::bytes(fa.fin, TAB), st>>>(fa);
+  return cudaGetLastError();
+}
+
+template <int HP>
+static cudaError_t filter_mlp_go(const hnd2::FilterMlpArgs& fa, long long noff, cudaStream_t st) {
+  return fa.tab ? filter_mlp_go_t<HP, true>(fa, noff, st) : filter_mlp_go_t<HP, false>(fa, noff, st);
+}
+
+long long filter_table_bytes(int hidden, int ndim, const int* n) {
+  for (int a = 0; a < ndim; ++a)
+    if (n[a] > 256) return 0;              // long 1D: the feature path (a table would be as large as the grid)
+  const int HP = (hidden + 31) / 32 * 32;
+  return hnd2::filter_table_floats(HP, ndim, n) * 4;
+}
+
+cudaError_t launch_filter_tables(const FilterLaunch& f, int ndim, const int* n, float* tab, cudaStream_t st) {
+  const int HP = (f.hidden + 31) / 32 * 32;
+  const long long cnt = hnd2::filter_table_floats(HP, ndim, n);
+  hnd2::k_filter_tables<<<grid_for(cnt, 256), 256, 0, st>>>(f.W1, f.hidden, HP, f.num_freqs, ndim, n[0],
+                                                            ndim > 1 ? n[1] : 1, ndim > 2 ? n[2] : 1, tab);
   return cudaGetLastError();
 }
 
@@ -193,6 +213,7 @@ cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, i
   fa.grid = grid;
   fa.gamma = f.gamma;
   fa.beta = f.beta;
+  fa.tab = f.tab;
   const int HP = (f.hidden + 31) / 32 * 32;
   e = HP <= 32 ? filter_mlp_go<32>(fa, noff, st)
       : HP <= 64 ? filter_mlp_go<64>(fa, noff, st)
