@@ -50,7 +50,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--config", type=lambda x: int(x) if x.isdigit() else x, default=2,
                     help="benchmark grid index (0..4) or workload name")
-    ap.add_argument("--also", default="1,3", help="extra grids measured kernel-only, comma separated "
+    ap.add_argument("--also", default="1,3,seq1d_1m_b1_c64_bf16", help="extra grids measured kernel-only, comma separated "
                     "(suite indices or workload names, e.g. seq1d_1m_b1_c64_bf16)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--sets", type=int, default=3, help="rotating input sets")
