@@ -27,23 +27,23 @@ namespace hnd2 {
 struct KgDims {
   int n0, n1, n2;       // grid (1 for unused axes)
   int P0, P1, P2;       // padded grid (1 for unused axes)
+  int l0, l1, l2;       // log2 of P0, P1, P2 (all powers of two)
 };
 
 template <class T>
 static __global__ void k_kg_pad(const T* __restrict__ k, const T* __restrict__ v, const T* __restrict__ q,
                                 const T* __restrict__ dy, float2* __restrict__ grid, KgDims d, int B, int C, int c0,
                                 int nvol) {
-  const long long gsz = static_cast<long long>(d.P0) * d.P1 * d.P2;
+  const int lg = d.l0 + d.l1 + d.l2;          // log2 of the grid size
   const long long L = static_cast<long long>(d.n0) * d.n1 * d.n2;
-  const long long total = gsz * nvol;
+  const long long total = static_cast<long long>(nvol) << lg;
   for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int vv = static_cast<int>(e / gsz);
-    long long r = e % gsz;
-    const int s2 = static_cast<int>(r % d.P2);
-    r /= d.P2;
-    const int s1 = static_cast<int>(r % d.P1);
-    const int s0 = static_cast<int>(r / d.P1);
+    const int vv = static_cast<int>(e >> lg);
+    const unsigned r = static_cast<unsigned>(e & ((1LL << lg) - 1));     // grids are below 2^32 points
+    const int s2 = static_cast<int>(r & (d.P2 - 1));
+    const int s1 = static_cast<int>((r >> d.l2) & (d.P1 - 1));
+    const int s0 = static_cast<int>(r >> (d.l1 + d.l2));
     float2 val = make_float2(0.f, 0.f);
     if (s0 < d.n0 && s1 < d.n1 && s2 < d.n2) {
       const int cl = vv / B, bb = vv % B;
@@ -59,11 +59,10 @@ static __global__ void k_kg_pad(const T* __restrict__ k, const T* __restrict__ v
 // split0, split1, split2) the digits of P - k with borrows.
 __device__ __forceinline__ long long kg_neg(long long r, const KgDims& d, int split0, int split1, int split2) {
   if (split0 == 0) {
-    const int k2 = static_cast<int>(r % d.P2);
-    const long long r1 = r / d.P2;
-    const int k1 = static_cast<int>(r1 % d.P1);
-    const int k0 = static_cast<int>(r1 / d.P1);
-    return (static_cast<long long>((d.P0 - k0) % d.P0) * d.P1 + (d.P1 - k1) % d.P1) * d.P2 + (d.P2 - k2) % d.P2;
+    const unsigned ru = static_cast<unsigned>(r);
+    const unsigned k2 = ru & (d.P2 - 1), k1 = (ru >> d.l2) & (d.P1 - 1), k0 = ru >> (d.l1 + d.l2);
+    const unsigned m0 = (d.P0 - k0) & (d.P0 - 1), m1 = (d.P1 - k1) & (d.P1 - 1), m2 = (d.P2 - k2) & (d.P2 - 1);
+    return static_cast<long long>((((m0 << d.l1) | m1) << d.l2) | m2);
   }
   // r = (k0 P1 + k1) P2 + k2 holds X(k0 + P0 k1 + P0 P1 k2)
   const int k2 = static_cast<int>(r % split2);
@@ -86,10 +85,11 @@ __device__ __forceinline__ long long kg_neg(long long r, const KgDims& d, int sp
 static __global__ void k_kg_corr(const float2* __restrict__ gw, float2* __restrict__ acc, KgDims d, int B, int ncc,
                                  long long gsz, int split0, int split1, int split2) {
   const int nh = (ncc + 1) / 2;
+  const int lg = d.l0 + d.l1 + d.l2;
   const long long total = gsz * nh;
   for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long h = e / gsz, r = e % gsz;
+    const long long h = e >> lg, r = e & (gsz - 1);
     const long long rn = kg_neg(r, d, split0, split1, split2);
     float are[2] = {0.f, 0.f}, aim[2] = {0.f, 0.f};
     for (int j = 0; j < 2; ++j) {
@@ -116,22 +116,22 @@ __device__ __forceinline__ float kg_part(const float2* acc, long long c, long lo
 
 static __global__ void k_kg_extract(const float2* __restrict__ acc, float* __restrict__ dK, KgDims d, int c0, int ncc,
                                     float scale) {
-  const int E0 = 2 * d.n0 - 1, E1 = 2 * d.n1 - 1, E2 = 2 * d.n2 - 1;
-  const long long noff = static_cast<long long>(E0) * E1 * E2;
+  // a chunk's outputs are fewer than 2^31 (at most one grid per channel of
+  // the chunk budget), so the index arithmetic stays in 32 bits
+  const unsigned E0 = 2 * d.n0 - 1, E1 = 2 * d.n1 - 1, E2 = 2 * d.n2 - 1;
+  const unsigned noff = E0 * E1 * E2;
   const long long gsz = static_cast<long long>(d.P0) * d.P1 * d.P2;
-  const long long total = noff * ncc;
-  for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < total;
-       e += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long c = e / noff, off = e % noff;
-    long long r = off;
-    const int i2 = static_cast<int>(r % E2);
-    r /= E2;
-    const int i1 = static_cast<int>(r % E1);
-    const int i0 = static_cast<int>(r / E1);
-    const int t0 = i0 - (d.n0 - 1), t1 = i1 - (d.n1 - 1), t2 = i2 - (d.n2 - 1);
-    const long long slot = (static_cast<long long>((t0 + d.P0) % d.P0) * d.P1 + (t1 + d.P1) % d.P1) * d.P2 +
-                           (t2 + d.P2) % d.P2;
-    dK[(c0 + c) * noff + off] = kg_part(acc, c, gsz, slot) * scale;
+  const unsigned total = noff * static_cast<unsigned>(ncc);
+  for (unsigned e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
+    const unsigned c = e / noff, off = e - c * noff;
+    const unsigned i2 = off % E2, r = off / E2;
+    const unsigned i1 = r % E1, i0 = r / E1;
+    const int t0 = static_cast<int>(i0) - (d.n0 - 1), t1 = static_cast<int>(i1) - (d.n1 - 1),
+              t2 = static_cast<int>(i2) - (d.n2 - 1);
+    const unsigned slot = ((static_cast<unsigned>(t0 + d.P0) & (d.P0 - 1)) << (d.l1 + d.l2)) |
+                          ((static_cast<unsigned>(t1 + d.P1) & (d.P1 - 1)) << d.l2) |
+                          (static_cast<unsigned>(t2 + d.P2) & (d.P2 - 1));
+    dK[static_cast<long long>(c0 + c) * noff + off] = kg_part(acc, c, gsz, slot) * scale;
   }
 }
 

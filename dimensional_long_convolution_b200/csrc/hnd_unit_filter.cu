@@ -252,6 +252,9 @@ static cudaError_t kgrad_chunk_t(const KgradLaunch& g, cudaStream_t st) {
   d.P0 = 2 * d.n0;
   d.P1 = g.ndim > 1 ? 2 * d.n1 : 1;
   d.P2 = g.ndim > 2 ? 2 * d.n2 : 1;
+  d.l0 = lg2(d.P0);
+  d.l1 = lg2(d.P1);
+  d.l2 = lg2(d.P2);
   const long long gsz = static_cast<long long>(d.P0) * d.P1 * d.P2;
   const int nvol = g.ncc * g.B;
   float2* gw = g.grids;
