@@ -293,6 +293,10 @@ struct M1 {
   static constexpr size_t kBytes = Tabs<N0>::kBytes + 16ull * XB<N0>::kWarp * kWM;
 };
 
+#ifndef HND_MID1_PREFETCH
+#define HND_MID1_PREFETCH 1
+#endif
+
 // One column unit cu (one pencil of lanes).  GEN: the warp that holds unit
 // 0, the combined DC/Nyquist unit, whose product needs the partner
 // frequency; every pencil of that warp takes this path (for cu != 0 the
@@ -320,9 +324,23 @@ __device__ __forceinline__ void mid1_unit(const Tabs<N0> t, float4* buf, float2*
       z[s + HS] = unpack_b(z1, z2);
     }
   }
+  const float4* su = sp + (cu == 0 ? 0LL : static_cast<long long>(cu + 1) * N0);
+#if HND_MID1_PREFETCH
+  // the unit's spectrum comes from HBM: start fetching it before the forward
+  // transform so that the product after it does not wait the full latency
+  if (act) {
+#pragma unroll
+    for (int s = 0; s < R1; ++s) {
+#if HND_MID1_PREFETCH == 2
+      asm volatile("prefetch.global.L1 [%0];" ::"l"(su + s * G + g));
+#else
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(su + s * G + g));
+#endif
+    }
+  }
+#endif
   cp x[R1];
   padded_fwd<N0>(z, x, g, buf, 0, t, 0u);
-  const float4* su = sp + (cu == 0 ? 0LL : static_cast<long long>(cu + 1) * N0);
   if constexpr (GEN) {
     cp xp[R1];
     fetch_partner<N0>(x, xp, g, buf, 0, 0u);
