@@ -37,6 +37,7 @@ struct FilterMlpArgs {
   const float* gamma = nullptr;  // FiLM: sin(gamma (W1 phi + b1) + beta), [hidden] each; null = plain
   const float* beta = nullptr;
   const float* tab = nullptr;    // per-axis first-layer tables (k_filter_tables)
+  int cgroup = 1 << 30;          // channels per CTA row of the grid (blockIdx.y; a multiple of kFC)
 };
 
 // The first layer is separable over the axes: the features of axis a depend on
@@ -223,8 +224,10 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
     }
   }
 
-  // output layer over channel tiles: thread (og, cg) -> offsets 4 og.., channels 4 cg..
-  for (int ct = 0; ct < a.nc; ct += kFC) {
+  // output layer over the channel tiles of this CTA's group (blockIdx.y):
+  // thread (og, cg) -> offsets 4 og.., channels 4 cg..
+  const int cend = min(a.nc, (static_cast<int>(blockIdx.y) + 1) * a.cgroup);
+  for (int ct = static_cast<int>(blockIdx.y) * a.cgroup; ct < cend; ct += kFC) {
     __syncthreads();          // hid complete / previous tile's w2 no longer read
     for (int i = tid; i < HP * kFC; i += kFT) {
       const int h = i / kFC, cc = i % kFC;

@@ -29,7 +29,17 @@ static cudaError_t filter_mlp_go_t(const hnd2::FilterMlpArgs& fa, long long noff
   cudaError_t e = ensure_smem(kern, hnd2::FilterSmem<HP>::bytes(96, TAB));     // the largest feature count
   if (e != cudaSuccess) return e;
   const long long blocks = (noff + hnd2::kFO - 1) / hnd2::kFO;
-  kern<<<static_cast<unsigned>(blocks), hnd2::kFT, hnd2::FilterSmem<HP>::bytes(fa.fin, TAB), st>>>(fa);
+  // small offset grids: split the channels over a second grid dimension so
+  // that about four CTAs per SM are in flight (each recomputes its hidden tile)
+  hnd2::FilterMlpArgs g = fa;
+  const int tiles = (fa.nc + hnd2::kFC - 1) / hnd2::kFC;
+  long long groups = (4LL * sm_count() + blocks - 1) / blocks;
+  if (groups > tiles) groups = tiles;
+  if (groups < 1) groups = 1;
+  const int per = static_cast<int>((tiles + groups - 1) / groups);
+  g.cgroup = per * hnd2::kFC;
+  const unsigned gy = static_cast<unsigned>((fa.nc + g.cgroup - 1) / g.cgroup);
+  kern<<<dim3(static_cast<unsigned>(blocks), gy), hnd2::kFT, hnd2::FilterSmem<HP>::bytes(fa.fin, TAB), st>>>(g);
   return cudaGetLastError();
 }
 
