@@ -31,7 +31,7 @@ constexpr size_t kWaveBudget = size_t(96) << 20;      // multi-pass intermediate
 // per offset, so fewer, larger chunks save that work at the cost of workspace
 constexpr size_t kFilterBudget = size_t(HND_FILTER_MB) << 20;
 constexpr int kFilterMaxChunk = HND_FILTER_MAXC;
-constexpr size_t kKgradBudget = size_t(128) << 20;    // kernel-gradient grids per channel chunk
+constexpr size_t kKgradBudget = size_t(256) << 20;    // kernel-gradient grids per channel chunk (the filter call already needs 256 MiB)
 #ifndef HND_L1_WAVE_MB
 #define HND_L1_WAVE_MB 96
 #endif

@@ -165,7 +165,7 @@ def test_long_1d_sizes(n, B, C):
     assert H.spectrum_bytes(p) == C * 2 * n * 8
     ws = H.workspace_bytes(p)
     assert ws >= 256 + max(2 * n * 8, (B + 1) * 2 * n * 8)
-    # the largest of: a 96 MiB conv wave, 128 MiB of kernel-gradient grids,
+    # the largest of: a 96 MiB conv wave, 256 MiB of kernel-gradient grids,
     # 256 MiB of filter grids (each at least one volume or channel), plus tables
     assert ws <= 256 + max(96 << 20, 128 << 20, 256 << 20, (B + 1) * 2 * n * 8, 2 * n * 8) + (1 << 20)
 
