@@ -98,7 +98,8 @@ typedef struct {
  * For every offset t in [-(n_a-1), n_a-1]^d:
  *   phi(t)  = [sin(pi m t_a / n_a), cos(pi m t_a / n_a)] for a < ndim, m = 1..num_freqs,
  *             ordered [axis][m][sin, cos]            (2 * num_freqs * ndim features)
- *   h       = sin(W1 phi + b1)                       (hidden units)
+ *   h       = sin(W1 phi + b1)                       (hidden units; with FiLM,
+ *             sin(gamma (W1 phi + b1) + beta), see hyena_nd_filter_spectrum_film)
  *   K_c(t)  = ((W2 h + b2)_c) * exp(-alpha_c * ||t||_2 / decay_scale)
  * Device pointers, fp32, row-major: W1 [hidden, 2*num_freqs*ndim], b1 [hidden],
  * W2 [C, hidden], b2 [C], alpha [C].  Limits: 1 <= num_freqs <= 16,
@@ -121,9 +122,13 @@ typedef struct {
 HYENA_ND_API size_t hyena_nd_spectrum_bytes(const hyena_nd_problem* p);
 
 /* Workspace bytes needed by every call below for problem `p` (a pure
- * function of the descriptor, at least 256 bytes: the control area, then
- * the intermediate spectra of the multi-pass tiers).  0 if `p` is invalid or unsupported.  The same
- * workspace may be reused by consecutive calls on one stream. */
+ * function of the descriptor, at least 256 bytes: the control area, then the
+ * largest of one wave of intermediate spectra of the multi-pass tiers (about
+ * 96 MiB), one channel chunk of the filter call's padded grids plus its
+ * first-layer tables (about 256 MiB) and one channel chunk of the kernel
+ * gradient's grids (about 256 MiB); each at least one volume or channel).
+ * 0 if `p` is invalid or unsupported.  The same workspace may be reused by
+ * consecutive calls on one stream. */
 HYENA_ND_API size_t hyena_nd_workspace_bytes(const hyena_nd_problem* p);
 
 /* Clear the workspace control area (enqueues a 256-byte memset on
