@@ -497,6 +497,29 @@ def test_backward_direct_at_points_matches_full():
     assert np.max(np.abs(got - want)) < 1e-12
 
 
+@pytest.mark.parametrize("dims", [(7,), (4, 6), (3, 3, 4)])
+def test_backward_direct_equals_dft_route(dims):
+    """The two backward routes (direct sums on the grid, and padded DFTs with
+    the conjugate spectrum) agree: a sign or index slip in the adjoint of
+    either fails here."""
+    q, k, v, K = _rand_problem(dims, seed=61)
+    dy = np.random.default_rng(62).standard_normal(q.shape)
+    a = O.backward_direct(q, k, v, dy, K, dims)
+    b = O.backward_dft(q, k, v, dy, O.spectrum_full(K, dims), dims)
+    for x, y in zip(a, b):
+        assert np.max(np.abs(x - y)) < 1e-11 * max(1.0, np.max(np.abs(y)))
+
+
+def test_reference_output_is_the_definition_on_the_smallest_workload():
+    """The convenience route used by the GPU tests (implicit kernel -> spectrum
+    -> DFT convolution) equals the direct sum with the same kernel."""
+    wl = W.custom((6, 5), 1, 2, seed=63)
+    inp = W.make_inputs(wl)
+    K = O.implicit_kernel(inp.filt, wl.dims)
+    want = O.conv_direct(inp.as_f64("q"), inp.as_f64("k"), inp.as_f64("v"), K, wl.dims)
+    assert np.max(np.abs(O.reference_output(inp) - want)) < 1e-11 * np.max(np.abs(want))
+
+
 # ------------------------------------------------------ kernel-value gradient
 @pytest.mark.parametrize("dims", [(6,), (4, 5), (3, 4, 3)])
 def test_kernel_grad_dft_equals_direct(dims):
