@@ -188,6 +188,19 @@ def test_static_scratch_call_rejects_long_1d():
     assert H.fftconv_batched_static(p, q, k, v, s, 0, y, 0) == H.ERR_UNSUPPORTED
 
 
+@pytest.mark.parametrize("i", range(5))
+def test_workspace_stays_within_the_chunk_budgets(i):
+    """Every benchmark grid's workspace is the largest of its scratch parts:
+    a conv wave (96 MiB), a filter chunk (256 MiB plus first-layer tables) and
+    a kernel-gradient chunk (256 MiB), each at least one volume or channel."""
+    wl = W.workload(i)
+    p = H.problem(wl.dims, wl.B, wl.C, H.BF16 if wl.io_dtype == "bf16" else H.F32)
+    P = int(np.prod([2 * n for n in wl.dims]))
+    one = max(8 * P * (wl.B + 1), 8 * P)
+    tables = 3 * 511 * 128 * 4
+    assert H.workspace_bytes(p) <= 256 + max(256 << 20, one) + 256 + tables
+
+
 def test_single_volume_call_needs_b_and_c_of_one():
     q, k, v, s, y, ws = _ptrs()
     p = H.problem((32, 32), 2, 1)
