@@ -66,6 +66,13 @@ def unavoidable_bytes(wl) -> int:
     return 4 * wl.B * wl.C * wl.voxels * elt + wl.C * half * 8
 
 
+def plan_summary(setup) -> dict:
+    """Tier, waves and launches of the measured problem, from the library's
+    host-side plan (no device work)."""
+    info = setup.H.plan_info(setup.op.p)
+    return {k: info[k] for k in ("tier", "wave", "waves", "launches", "split")}
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -442,7 +449,8 @@ def run_ours(args):
                    "parallelism": "batch-sharded x%d (rank 0 samples %d..%d of %d; independent volumes, no "
                                   "collective)" % (world, shard[0], shard[1] - 1, world * wl.B),
                    "l2": "%d rotating input sets of %.0f MB each (> 126 MB L2 between reuses)" %
-                         (args.sets, ub / 1e6)},
+                         (args.sets, ub / 1e6),
+                   "plan": plan_summary(setup)},
         "gbs": ub * K / (ms_max / 1e3) / 1e9 * world,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": recorded_traffic(wl.name), "peak_kind": peak_kind,

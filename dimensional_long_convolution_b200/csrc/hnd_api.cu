@@ -207,6 +207,33 @@ size_t hyena_nd_workspace_bytes(const hyena_nd_problem* p) {
   return make_plan(p, &pl) == HYENA_ND_OK ? pl.ws_total : 0;
 }
 
+hyena_nd_status hyena_nd_plan_info_get(const hyena_nd_problem* p, hyena_nd_plan_info* out) {
+  if (!out) return HYENA_ND_ERR_INVALID_ARG;
+  Plan pl;
+  const hyena_nd_status st = make_plan(p, &pl);
+  if (st != HYENA_ND_OK) return st;
+  hyena_nd_plan_info info{};
+  info.tier = static_cast<hyena_nd_tier>(pl.tier);
+  const long long vols = pl.B * pl.C;
+  info.wave = pl.tier == kRows1D || pl.tier == kFused2D ? 0 : pl.wave;
+  info.waves = info.wave > 0 ? (vols + pl.wave - 1) / pl.wave : 1;
+  info.split[0] = info.split[1] = info.split[2] = 1;
+  if (pl.tier == kLong1D) {
+    const hnd::L1Split sp = hnd::long1d_split(pl.n[0]);
+    info.split_levels = sp.m;
+    for (int a = 0; a < 3; ++a) info.split[a] = sp.P[a];
+    info.launches = static_cast<int>(info.waves) * (2 * sp.m - 1);
+  } else {
+    info.launches = info.wave > 0 ? static_cast<int>(info.waves) * 3 : 1;
+  }
+  info.filter_chunk = pl.filter_chunk;
+  info.kgrad_chunk = pl.kgrad_chunk;
+  info.workspace_bytes = pl.ws_total;
+  info.spectrum_bytes = pl.spec_bytes;
+  *out = info;
+  return HYENA_ND_OK;
+}
+
 hyena_nd_status hyena_nd_workspace_init(void* ws, size_t ws_bytes, void* cuda_stream) {
   if (!ws) return HYENA_ND_ERR_INVALID_ARG;
   if (!aligned16(ws)) return HYENA_ND_ERR_MISALIGNED;

@@ -47,9 +47,27 @@ EXPORTED = (
     "hyena_nd_status_string",
     "hyena_nd_last_launch_count",
     "hyena_nd_fftconv_batched_static",
+    "hyena_nd_plan_info_get",
 )
 
+TIERS = {0: "rows_1d", 1: "fused_2d", 2: "multi_2d", 3: "multi_3d", 4: "long_1d"}
+
 STATIC_SCRATCH_BYTES = 16 << 20
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [
+        ("tier", ctypes.c_int),
+        ("wave", ctypes.c_int64),
+        ("waves", ctypes.c_int64),
+        ("launches", ctypes.c_int),
+        ("split_levels", ctypes.c_int),
+        ("split", ctypes.c_int * 3),
+        ("filter_chunk", ctypes.c_int),
+        ("kgrad_chunk", ctypes.c_int),
+        ("workspace_bytes", ctypes.c_size_t),
+        ("spectrum_bytes", ctypes.c_size_t),
+    ]
 
 
 class Problem(ctypes.Structure):
@@ -113,6 +131,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "hyena_nd_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "hyena_nd_last_launch_count": (ctypes.c_int, []),
         "hyena_nd_fftconv_batched_static": (ctypes.c_int, [P, vp, vp, vp, vp, i64, vp, vp]),
+        "hyena_nd_plan_info_get": (ctypes.c_int, [P, ctypes.POINTER(PlanInfo)]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -198,6 +217,17 @@ def fftconv_backward(p: Problem, q: int, k: int, v: int, spectrum: int, spectrum
 def kernel_grad(p: Problem, q: int, k: int, v: int, dy: int, dK: int, ws: int, ws_bytes: int,
                 stream: int = 0) -> int:
     return load().hyena_nd_kernel_grad(ctypes.byref(p), q, k, v, dy, dK, ws, ws_bytes, stream)
+
+
+def plan_info(p: Problem) -> dict:
+    """The execution plan of a problem (host only): tier, waves, launches per
+    convolution, long-1D split, chunk sizes and buffer sizes."""
+    info = PlanInfo()
+    check(load().hyena_nd_plan_info_get(ctypes.byref(p), ctypes.byref(info)), "plan_info")
+    return {"tier": TIERS.get(info.tier, str(info.tier)), "wave": info.wave, "waves": info.waves,
+            "launches": info.launches, "split_levels": info.split_levels, "split": list(info.split),
+            "filter_chunk": info.filter_chunk, "kgrad_chunk": info.kgrad_chunk,
+            "workspace_bytes": info.workspace_bytes, "spectrum_bytes": info.spectrum_bytes}
 
 
 def status_string(code: int) -> str:

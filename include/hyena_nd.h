@@ -131,6 +131,33 @@ HYENA_ND_API size_t hyena_nd_spectrum_bytes(const hyena_nd_problem* p);
  * consecutive calls on one stream. */
 HYENA_ND_API size_t hyena_nd_workspace_bytes(const hyena_nd_problem* p);
 
+/* Execution plan of a problem, as the calls below run it (host only, no
+ * device work; a pure function of the descriptor). */
+typedef enum {
+  HYENA_ND_TIER_ROWS_1D = 0,   /* 1D, n <= 256: one fused row kernel */
+  HYENA_ND_TIER_FUSED_2D = 1,  /* 2D, both axes <= 64: one persistent fused kernel */
+  HYENA_ND_TIER_MULTI_2D = 2,  /* other 2D grids: rows, column units, rows, in waves */
+  HYENA_ND_TIER_MULTI_3D = 3,  /* 3D grids: rows, (y, z) slabs, rows, in waves */
+  HYENA_ND_TIER_LONG_1D = 4    /* 1D, n > 256: split transform passes, in waves */
+} hyena_nd_tier;
+
+typedef struct {
+  hyena_nd_tier tier;
+  int64_t wave;           /* volumes per wave of the multi-pass tiers (0 for single-launch tiers) */
+  int64_t waves;          /* waves per convolution (1 for single-launch tiers) */
+  int launches;           /* kernel launches per convolution */
+  int split_levels;       /* long 1D: factors of the split 2n = P0 P1 (P2) (0 otherwise) */
+  int split[3];           /* long 1D: the factors (1 where unused) */
+  int filter_chunk;       /* channels per chunk of the filter call */
+  int kgrad_chunk;        /* channels per chunk of the kernel gradient */
+  size_t workspace_bytes; /* hyena_nd_workspace_bytes(p) */
+  size_t spectrum_bytes;  /* hyena_nd_spectrum_bytes(p) */
+} hyena_nd_plan_info;
+
+/* Fill `out` with the plan of `p`.  Errors: HYENA_ND_ERR_INVALID_ARG (null or
+ * invalid problem), HYENA_ND_ERR_UNSUPPORTED (valid but outside the sizes). */
+HYENA_ND_API hyena_nd_status hyena_nd_plan_info_get(const hyena_nd_problem* p, hyena_nd_plan_info* out);
+
 /* Clear the workspace control area (enqueues a 256-byte memset on
  * `stream`).  Call once on a fresh workspace before the first call that uses
  * it; `ws_bytes` must be at least 256. */

@@ -21,7 +21,7 @@ def _declared():
 def test_library_exports_every_declared_symbol():
     lib = H.load()
     names = _declared()
-    assert len(names) == len(H.EXPORTED) == 16
+    assert len(names) == len(H.EXPORTED) == 17
     assert set(names) == set(H.EXPORTED)
     for n in names:
         assert getattr(lib, n) is not None
@@ -199,6 +199,45 @@ def test_workspace_stays_within_the_chunk_budgets(i):
     one = max(8 * P * (wl.B + 1), 8 * P)
     tables = 3 * 511 * 128 * 4
     assert H.workspace_bytes(p) <= 256 + max(256 << 20, one) + 256 + tables
+
+
+@pytest.mark.parametrize("i,tier,waves,launches", [
+    (0, "fused_2d", 1, 1), (1, "fused_2d", 1, 1), (2, "multi_2d", 2, 6), (3, "multi_3d", 3, 9),
+    (4, "multi_3d", 6, 18)])
+def test_plan_info_of_the_benchmark_grids(i, tier, waves, launches):
+    """The plan the calls run, read on the host: the launch counts are the
+    ones the GPU tests and the bench observe."""
+    wl = W.workload(i)
+    p = H.problem(wl.dims, wl.B, wl.C, H.BF16 if wl.io_dtype == "bf16" else H.F32)
+    info = H.plan_info(p)
+    assert (info["tier"], info["waves"], info["launches"]) == (tier, waves, launches)
+    assert info["workspace_bytes"] == H.workspace_bytes(p)
+    assert info["spectrum_bytes"] == H.spectrum_bytes(p)
+    if waves > 1:       # balanced waves of whole channels' samples
+        assert info["wave"] * (waves - 1) < wl.B * wl.C <= info["wave"] * waves
+        assert info["wave"] % wl.B == 0
+
+
+@pytest.mark.parametrize("n,B,C,levels,split,waves", [
+    (256, 1, 4, 0, [1, 1, 1], 1), (512, 2, 3, 2, [32, 32, 1], 1), (1 << 17, 1, 60, 2, [512, 512, 1], 2),
+    (1 << 20, 1, 64, 3, [128, 128, 128], 11), (1 << 26, 1, 1, 3, [512, 512, 512], 1)])
+def test_plan_info_of_long_1d(n, B, C, levels, split, waves):
+    info = H.plan_info(H.problem((n,), B, C))
+    assert info["split_levels"] == levels and info["split"] == split
+    assert info["tier"] == ("long_1d" if n > 256 else "rows_1d")
+    assert info["waves"] == waves
+    if levels:
+        assert info["launches"] == waves * (2 * levels - 1)
+        assert int(np.prod(split)) == 2 * n
+
+
+def test_plan_info_rejects_bad_problems():
+    info = H.PlanInfo()
+    lib = H.load()
+    assert lib.hyena_nd_plan_info_get(None, H.ctypes.byref(info)) == H.ERR_INVALID_ARG
+    assert lib.hyena_nd_plan_info_get(H.ctypes.byref(H.problem((64, 64), 1, 1)), None) == H.ERR_INVALID_ARG
+    assert lib.hyena_nd_plan_info_get(H.ctypes.byref(H.problem((300,), 1, 1)), H.ctypes.byref(info)) == \
+        H.ERR_UNSUPPORTED
 
 
 def test_single_volume_call_needs_b_and_c_of_one():
