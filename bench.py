@@ -41,6 +41,8 @@ from dimensional_long_convolution_b200.parallel import max_over_ranks, shard_ran
 METRIC = "gated nD FFT long-conv voxel*channels/s"
 UNIT = "voxel*ch/s"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0      # B200 HBM3e nominal (DGX figure); the measured copy bandwidth is the roofline peak
+REPEATS = 5                   # the timed steps run as this many equal segments; their median is reported beside the total
 
 
 def parse_args():
@@ -50,7 +52,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--config", type=lambda x: int(x) if x.isdigit() else x, default=2,
                     help="benchmark grid index (0..4) or workload name")
-    ap.add_argument("--also", default="1,3,seq1d_1m_b1_c64_bf16", help="extra grids measured kernel-only, comma separated "
+    ap.add_argument("--also", default="0,1,3,4,seq1d_1m_b1_c64_bf16", help="extra grids measured kernel-only, comma separated "
                     "(suite indices or workload names, e.g. seq1d_1m_b1_c64_bf16)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--sets", type=int, default=3, help="rotating input sets")
@@ -103,6 +105,22 @@ def recorded_traffic(workload_name: str):
         e = d.get(workload_name)
         if e and e.get("source_sha") == kernel_source_sha():
             return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+def recorded_pipes(workload_name: str):
+    """FP32-pipe and issue fractions of a step (time-weighted over its
+    kernels) from a committed ncu summary taken on the current kernel
+    sources, else None."""
+    path = os.path.join(ROOT, "profiles", "pipes.json")
+    try:
+        with open(path) as fh:
+            d = json.load(fh)
+        e = d.get(workload_name)
+        if e and e.get("source_sha") == kernel_source_sha():
+            return {k: e[k] for k in ("fma_pipe_frac", "issue_frac", "dram_bytes_per_step") if k in e}
     except Exception:
         pass
     return None
@@ -272,16 +290,42 @@ class Setup:
         return self.H.last_launch_count()
 
 
-def time_steps(setup, K, stream):
+def time_steps(setup, K, stream, segments: int = 1):
+    """Device time of K back-to-back steps (CUDA events on the launching
+    stream).  With segments > 1 the same K steps are split into that many
+    consecutive equal parts with an event between parts; returns the total
+    and the per-step time of each part."""
     torch = setup.torch
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(K):
-        setup.step(i)
-    e1.record(stream)
-    e1.synchronize()
-    return e0.elapsed_time(e1)
+    segments = max(1, min(segments, K))
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(segments + 1)]
+    bounds = [K * j // segments for j in range(segments + 1)]
+    ev[0].record(stream)
+    for j in range(segments):
+        for i in range(bounds[j], bounds[j + 1]):
+            setup.step(i)
+        ev[j + 1].record(stream)
+    ev[-1].synchronize()
+    parts = [ev[j].elapsed_time(ev[j + 1]) / max(1, bounds[j + 1] - bounds[j]) for j in range(segments)]
+    if segments == 1:
+        return ev[0].elapsed_time(ev[-1])
+    return ev[0].elapsed_time(ev[-1]), parts
+
+
+def time_filter_call(setup, device, stream, n: int) -> float:
+    """ms per call 1 (filter spectrum) with device-resident weights: the MLP
+    on the offset grid, the window, the padded transform and the packing.
+    The spectrum it rewrites is the same one (same weights)."""
+    torch = setup.torch
+    f = setup.inp0.filt
+    wdev = [torch.from_numpy(a).to(device) for a in (f.W1, f.b1, f.W2, f.b2, f.alpha)]
+    setup.op.set_filter(*wdev, f.decay_scale, f.num_freqs)
+    fa, fb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    fa.record(stream)
+    for _ in range(n):
+        setup.op.set_filter(*wdev, f.decay_scale, f.num_freqs)
+    fb.record(stream)
+    fb.synchronize()
+    return fa.elapsed_time(fb) / n
 
 
 def run_ours(args):
@@ -321,7 +365,7 @@ def run_ours(args):
     clocks.start()
     time.sleep(0.3)
     barrier()
-    ms = time_steps(setup, K, stream)
+    ms, parts = time_steps(setup, K, stream, REPEATS)
     barrier()
     clocks.stop()
     ms_max = max_over_ranks(ms, dist, device)
@@ -364,6 +408,22 @@ def run_ours(args):
     e2e = {"value": world * units * E / (te / 1e3), "unit": UNIT,
            "h2d_bytes_per_step": 3 * units * elt, "d2h_bytes_per_step": units * elt}
 
+    # warm: the same grid with one input set reused every step, so whatever of
+    # q, k, v, y and the spectrum L2 keeps between steps is found there
+    warm = None
+    if args.sets > 1:
+        q1, k1, v1, y1, s1 = setup.sets[0]
+        saved = setup.sets
+        setup.sets = [(q1, k1, v1, y1, s1)]
+        for i in range(3):
+            setup.step(i)
+        Kw = max(REPEATS, min(K, 2000))
+        tw, wparts = time_steps(setup, Kw, stream, REPEATS)
+        setup.sets = saved
+        wparts.sort()
+        warm = {"ms_per_step": tw / Kw, "median_ms_per_step": wparts[len(wparts) // 2], "steps": Kw,
+                "note": "one input set reused every step (L2 may keep part of it)"}
+
     also = []
     for tok in [x for x in args.also.split(",") if x.strip() != ""]:
         j = int(tok) if tok.strip().isdigit() else tok.strip()
@@ -376,31 +436,25 @@ def run_ours(args):
         torch.cuda.synchronize(device)
         pj = time_steps(sj, 10, stream) / 10.0
         Kj = int(max(20, min(20000, 1500.0 / max(pj, 1e-3))))
-        msj = time_steps(sj, Kj, stream)
+        msj, pparts = time_steps(sj, Kj, stream, REPEATS)
         sm = msj / Kj
+        pparts.sort()
         ubj = unavoidable_bytes(wj)
-        also.append({"workload": wj.name, "value": wj.B * wj.C * wj.voxels / (sm / 1e3), "unit": UNIT,
-                     "ms_per_step": sm, "gbs": ubj / (sm / 1e3) / 1e9,
-                     "hbm_frac": ubj / (sm / 1e3) / 1e9 / peak, "launches_per_step": sj.launches, "steps": Kj})
+        entry = {"workload": wj.name, "value": wj.B * wj.C * wj.voxels / (sm / 1e3), "unit": UNIT,
+                 "ms_per_step": sm, "median_ms_per_step": pparts[len(pparts) // 2],
+                 "gbs": ubj / (sm / 1e3) / 1e9, "hbm_frac": ubj / (sm / 1e3) / 1e9 / peak,
+                 "hbm_frac_nominal": ubj / (sm / 1e3) / 1e9 / NOMINAL_HBM_GBS,
+                 "launches_per_step": sj.launches, "steps": Kj, "plan": plan_summary(sj)}
+        pj_rec = recorded_pipes(wj.name)
+        if pj_rec:
+            entry["profile"] = pj_rec
+        entry["filter_call_ms"] = time_filter_call(sj, device, stream, 3)
+        entry["filter_call_conv_steps"] = entry["filter_call_ms"] / sm
+        also.append(entry)
         del sj
         torch.cuda.empty_cache()
 
-    # call 1 (filter spectrum) timed on its own: device-resident weights, the
-    # MLP on the offset grid, the padded transform and the packing
-    f = setup.inp0.filt
-    wdev = [torch.from_numpy(a).to(device) for a in (f.W1, f.b1, f.W2, f.b2, f.alpha)]
-    spec_tmp = setup.op.spectrum.clone()
-    for _ in range(2):
-        setup.op.set_filter(*wdev, f.decay_scale, f.num_freqs)
-    fa, fb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    NF = 5
-    fa.record(stream)
-    for _ in range(NF):
-        setup.op.set_filter(*wdev, f.decay_scale, f.num_freqs)
-    fb.record(stream)
-    fb.synchronize()
-    setup.op.spectrum.copy_(spec_tmp)
-    call1_ms = fa.elapsed_time(fb) / NF
+    call1_ms = time_filter_call(setup, device, stream, 5)
     filter_call = {"ms_per_call": call1_ms, "conv_steps_per_call": call1_ms / (ms / K),
                    "note": "not in the metric: the spectrum is computed once per filter update"}
 
@@ -441,6 +495,8 @@ def run_ours(args):
         cpu = cpu_baseline(wl, setup.inp0, args.cpu_seconds)
 
     kernel_desc = {1: "fused single-CTA kernel", 3: "three multi-pass kernels per wave"}
+    parts.sort()
+    pipes = recorded_pipes(wl.name)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -452,14 +508,20 @@ def run_ours(args):
                          (args.sets, ub / 1e6),
                    "plan": plan_summary(setup)},
         "gbs": ub * K / (ms_max / 1e3) / 1e9 * world,
+        "median_ms_per_step": parts[len(parts) // 2],
+        "repeats_ms_per_step": parts,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "frac_nominal": achieved / NOMINAL_HBM_GBS, "nominal_peak": NOMINAL_HBM_GBS,
                      "traffic": recorded_traffic(wl.name), "peak_kind": peak_kind,
+                     "fp32_pipe_frac": pipes.get("fma_pipe_frac") if pipes else None,
+                     "issue_frac": pipes.get("issue_frac") if pipes else None,
                      "kernel": "step (%d launch%s per step: %s)" % (
                          launches, "" if launches == 1 else "es", kernel_desc.get(launches, "multi-pass waves")),
                      "algorithmic_bytes_per_step": ub},
         "gpu_launches": int(launches * K),
         "clocks": clocks.summary(),
         "e2e": e2e,
+        "warm": warm,
         "filter_call": filter_call,
         "backward": backward,
         "also": also,

@@ -2,6 +2,7 @@
 // workspace planning, tier selection and launch sequencing.  Every arithmetic
 // step of the convolution runs in the kernels of hnd_kernels.cuh.
 #include "hyena_nd.h"
+#include "hnd_bounds.cuh"
 #include "hnd_launch.h"
 
 #include <cuda_runtime.h>
@@ -9,6 +10,7 @@
 #include <climits>
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 namespace hnd {
 cudaError_t launch_fused2d_f32(const ConvArgs& a);
@@ -19,8 +21,78 @@ namespace {
 
 thread_local int g_last_launches = 0;
 
+}  // namespace
+
+namespace hnd {
+
+long long balanced_wave(long long pairs, long long B, size_t per_pair, size_t budget, bool whole_channels) {
+  long long w = static_cast<long long>(budget / per_pair);
+  if (w < 1) w = 1;
+  if (w > pairs) w = pairs;
+  if (whole_channels && w >= B) w -= w % B;        // keep a channel's samples in one wave
+  // equal waves: no short last wave
+  const long long nw = (pairs + w - 1) / w;
+  long long we = (pairs + nw - 1) / nw;
+  if (whole_channels && we >= B && we % B) we += B - we % B;
+  return we < w ? we : w;
+}
+
+void note_launches(int n) { g_last_launches = n; }
+
+cudaError_t side_stream(SideStream** out) {
+  static std::mutex mu;
+  static SideStream* per_dev[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!per_dev[dev]) {
+    SideStream* r = new SideStream;
+    if ((e = cudaStreamCreateWithFlags(&r->s, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    for (cudaEvent_t* ev : {&r->fork, &r->stagger, &r->join})
+      if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+    per_dev[dev] = r;
+  }
+  *out = per_dev[dev];
+  return cudaSuccess;
+}
+
+#ifdef HYENA_ND_BOUNDS
+__device__ BoundsTable g_bounds;
+__device__ __align__(16) unsigned char g_bounds_dummy[256];
+
+cudaError_t bounds_register(const BoundsList& l, int* status, cudaStream_t st) {
+  BoundsTable t{};
+  for (int i = 0; i < l.n; ++i) {
+    t.base[i] = reinterpret_cast<unsigned long long>(l.ptr[i]);
+    t.bytes[i] = l.bytes[i];
+  }
+  t.n = l.n;
+  t.status = status;
+  return cudaMemcpyToSymbolAsync(g_bounds, &t, sizeof(t), 0, cudaMemcpyHostToDevice, st);
+}
+#else
+cudaError_t bounds_register(const BoundsList&, int*, cudaStream_t) { return cudaSuccess; }
+#endif
+
+}  // namespace hnd
+
+namespace {
+
 constexpr size_t kStatusBytes = 256;                  // status word + padding
-constexpr size_t kWaveBudget = size_t(96) << 20;      // multi-pass intermediate per wave (measured best of 24/48/96 MiB)
+#ifndef HND_WAVE_MB
+#define HND_WAVE_MB 64
+#endif
+#ifndef HND_STREAMS
+#define HND_STREAMS 2
+#endif
+// Multi-pass tiers: intermediates of the waves in flight, split over
+// HND_STREAMS streams that run alternate waves one stage apart.  Measured on
+// the 256^2, 64^3 and 128^3 grids: two streams with 64 MiB in all (32 MiB
+// waves) beat one stream with 96 MiB by 2-5%, and 128 or 192 MiB in all.
+constexpr size_t kWaveBudget = size_t(HND_WAVE_MB) << 20;
+constexpr int kWaveStreams = HND_STREAMS;
 #ifndef HND_FILTER_MB
 #define HND_FILTER_MB 256
 #endif
@@ -52,9 +124,14 @@ struct Plan {
   long long spec_per = 0;   // complex values per channel spectrum
   int tier = 0;
   long long wave = 0;       // pairs per wave (multi-pass tiers)
+  int streams = 1;          // multi-pass tiers: streams running alternate waves
+  size_t wave_bytes = 0;    // workspace of one wave (multi-pass tiers)
   int filter_chunk = 1;
   int kgrad_chunk = 1;      // channels per kernel-gradient chunk
-  size_t ws_total = 0;
+  size_t ws_total = 0;      // the largest of the three below (hyena_nd_workspace_bytes)
+  size_t ws_conv = 0;       // convolution calls (forward, batched, backward)
+  size_t ws_filter = 0;     // filter calls
+  size_t ws_kgrad = 0;      // kernel gradient
   size_t spec_bytes = 0;
   size_t nat_bytes = 0;     // natural-order half spectrum (export / import)
   size_t filter_grid_bytes = 0;   // filter call: chunk grids (the tables follow)
@@ -103,11 +180,7 @@ hyena_nd_status make_plan(const hyena_nd_problem* p, Plan* pl) {
   if (p->ndim == 1 && nl > 256) {
     pl->tier = kLong1D;
     const size_t per_vol = static_cast<size_t>(8) * static_cast<size_t>(pl->gsz);
-    long long w = static_cast<long long>(kL1WaveBudget / per_vol);
-    if (w < 1) w = 1;
-    if (w > pairs) w = pairs;
-    const long long nw = (pairs + w - 1) / w;
-    pl->wave = (pairs + nw - 1) / nw;   // equal waves
+    pl->wave = hnd::balanced_wave(pairs, p->B, per_vol, kL1WaveBudget, false);
     ws_conv = per_vol * static_cast<size_t>(pl->wave);
   } else if (p->ndim == 1) {
     pl->tier = kRows1D;
@@ -116,17 +189,15 @@ hyena_nd_status make_plan(const hyena_nd_problem* p, Plan* pl) {
   } else {
     pl->tier = p->ndim == 2 ? kMulti2D : kMulti3D;
     const size_t per_pair = static_cast<size_t>(8) * static_cast<size_t>(pl->L);
-    long long w = static_cast<long long>(kWaveBudget / per_pair);
-    if (w < 1) w = 1;
-    if (w > pairs) w = pairs;
-    if (w >= p->B) w -= w % p->B;        // keep a channel's samples in one wave
-    // equal waves: no short last wave
-    const long long nw = (pairs + w - 1) / w;
-    long long we = (pairs + nw - 1) / nw;
-    if (we >= p->B && we % p->B) we += p->B - we % p->B;
-    if (we < w) w = we;
-    pl->wave = w;
-    ws_conv = per_pair * static_cast<size_t>(w);
+    pl->wave = hnd::balanced_wave(pairs, p->B, per_pair, kWaveBudget, true);
+    pl->streams = 1;
+    if (kWaveStreams > 1 && pl->wave < pairs) {
+      // several waves: run them on two streams, each wave in half the budget
+      pl->wave = hnd::balanced_wave(pairs, p->B, per_pair, kWaveBudget / kWaveStreams, true);
+      pl->streams = pl->wave < pairs ? kWaveStreams : 1;
+    }
+    pl->wave_bytes = (per_pair * static_cast<size_t>(pl->wave) + 255) / 256 * 256;
+    ws_conv = pl->wave_bytes * static_cast<size_t>(pl->streams);
   }
   long long chunk = static_cast<long long>(kFilterBudget / (8 * static_cast<size_t>(pl->gsz)));
   if (chunk < 1) chunk = 1;
@@ -147,6 +218,9 @@ hyena_nd_status make_plan(const hyena_nd_problem* p, Plan* pl) {
   size_t need = ws_conv > ws_filter ? ws_conv : ws_filter;
   if (ws_kgrad > need) need = ws_kgrad;
   pl->ws_total = kStatusBytes + need;
+  pl->ws_conv = kStatusBytes + ws_conv;
+  pl->ws_filter = kStatusBytes + ws_filter;
+  pl->ws_kgrad = kStatusBytes + ws_kgrad;
   return HYENA_ND_OK;
 }
 
@@ -165,6 +239,12 @@ bool overlaps2(const void* a, size_t na, const void* b, size_t nb) {
 
 hyena_nd_status cuda_status(cudaError_t e) { return e == cudaSuccess ? HYENA_ND_OK : HYENA_ND_ERR_CUDA; }
 
+// Bytes of spectrum a convolution call may read: one set, or B sets at a
+// byte stride.
+size_t spectrum_span(const Plan& pl, int64_t sbs) {
+  return sbs > 0 ? static_cast<size_t>(pl.B - 1) * static_cast<size_t>(sbs) + pl.spec_bytes : pl.spec_bytes;
+}
+
 // One gated convolution y = q . (K * (k . v)) (or with the conjugate
 // spectrum) on the plan's tier; adds the kernel launches to *launches.
 cudaError_t run_conv(const Plan& pl, const hnd::ConvArgs& a, void* ws, int* launches) {
@@ -178,16 +258,43 @@ cudaError_t run_conv(const Plan& pl, const hnd::ConvArgs& a, void* ws, int* laun
     e = pl.bf16 ? hnd::launch_fused2d_bf16(a) : hnd::launch_fused2d_f32(a);
     *launches += 1;
   } else {
-    float2* zt = reinterpret_cast<float2*>(static_cast<char*>(ws) + kStatusBytes);
+    char* zbase = static_cast<char*>(ws) + kStatusBytes;
     const long long pairs = pl.B * pl.C;
     const int nl = pl.n[pl.ndim - 1];
     const int rp_total = static_cast<int>(pl.L / nl / 2);
-    for (long long ord0 = 0; ord0 < pairs && e == cudaSuccess; ord0 += pl.wave) {
+    hnd::SideStream* side = nullptr;
+    std::unique_lock<std::mutex> lk;
+    if (pl.streams > 1) {
+      // Waves alternate between the caller's stream and a side stream; the
+      // side stream starts one stage late, so that the column stage of one
+      // wave shares the SMs with the row stages of the next.  Each stream
+      // owns one wave-sized slice of the workspace.
+      if ((e = hnd::side_stream(&side)) != cudaSuccess) return e;
+      lk = std::unique_lock<std::mutex>(side->mu);
+      if ((e = cudaEventRecord(side->fork, a.stream)) != cudaSuccess) return e;
+      if ((e = cudaStreamWaitEvent(side->s, side->fork, 0)) != cudaSuccess) return e;
+    }
+    int w = 0;
+    for (long long ord0 = 0; ord0 < pairs && e == cudaSuccess; ord0 += pl.wave, ++w) {
       const int np = static_cast<int>(pairs - ord0 < pl.wave ? pairs - ord0 : pl.wave);
-      e = hnd::launch_rowfwd(a, nl, zt, ord0, np, rp_total);
-      if (e == cudaSuccess) e = pl.tier == kMulti2D ? hnd::launch_mid1(a, zt, ord0, np) : hnd::launch_mid2(a, zt, ord0, np);
-      if (e == cudaSuccess) e = hnd::launch_rowinv(a, nl, zt, ord0, np, rp_total);
+      const int lane = pl.streams > 1 ? w % pl.streams : 0;
+      hnd::ConvArgs aw = a;
+      if (lane == 1) aw.stream = side->s;
+      float2* zt = reinterpret_cast<float2*>(zbase + static_cast<size_t>(lane) * pl.wave_bytes);
+      e = hnd::launch_rowfwd(aw, nl, zt, ord0, np, rp_total);
+      if (e == cudaSuccess && pl.streams > 1 && w == 0) {
+        e = cudaEventRecord(side->stagger, a.stream);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(side->s, side->stagger, 0);
+      }
+      if (e == cudaSuccess) e = pl.tier == kMulti2D ? hnd::launch_mid1(aw, zt, ord0, np) : hnd::launch_mid2(aw, zt, ord0, np);
+      if (e == cudaSuccess) e = hnd::launch_rowinv(aw, nl, zt, ord0, np, rp_total);
       *launches += 3;
+    }
+    if (pl.streams > 1) {
+      // join: the caller's stream waits for the side stream's last wave
+      const cudaError_t e1 = cudaEventRecord(side->join, side->s);
+      const cudaError_t e2 = e1 == cudaSuccess ? cudaStreamWaitEvent(a.stream, side->join, 0) : e1;
+      if (e == cudaSuccess) e = e2;
     }
   }
   return e;
@@ -205,6 +312,18 @@ size_t hyena_nd_spectrum_bytes(const hyena_nd_problem* p) {
 size_t hyena_nd_workspace_bytes(const hyena_nd_problem* p) {
   Plan pl;
   return make_plan(p, &pl) == HYENA_ND_OK ? pl.ws_total : 0;
+}
+
+size_t hyena_nd_workspace_bytes_for(const hyena_nd_problem* p, hyena_nd_call call) {
+  Plan pl;
+  if (make_plan(p, &pl) != HYENA_ND_OK) return 0;
+  switch (call) {
+    case HYENA_ND_CALL_ALL: return pl.ws_total;
+    case HYENA_ND_CALL_CONV: return pl.ws_conv;
+    case HYENA_ND_CALL_FILTER: return pl.ws_filter;
+    case HYENA_ND_CALL_KERNEL_GRAD: return pl.ws_kgrad;
+  }
+  return 0;
 }
 
 hyena_nd_status hyena_nd_plan_info_get(const hyena_nd_problem* p, hyena_nd_plan_info* out) {
@@ -230,6 +349,7 @@ hyena_nd_status hyena_nd_plan_info_get(const hyena_nd_problem* p, hyena_nd_plan_
   info.kgrad_chunk = pl.kgrad_chunk;
   info.workspace_bytes = pl.ws_total;
   info.spectrum_bytes = pl.spec_bytes;
+  info.streams = pl.streams;
   *out = info;
   return HYENA_ND_OK;
 }
@@ -252,7 +372,7 @@ hyena_nd_status hyena_nd_fftconv_batched(const hyena_nd_problem* p, const void* 
     return HYENA_ND_ERR_MISALIGNED;
   if (spectrum_batch_stride < 0) return HYENA_ND_ERR_INVALID_ARG;
   if (spectrum_batch_stride % 16 != 0) return HYENA_ND_ERR_MISALIGNED;
-  if (ws_bytes < pl.ws_total) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
+  if (ws_bytes < pl.ws_conv) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
   const size_t act_bytes = static_cast<size_t>(pl.B * pl.C * pl.L) * (pl.bf16 ? 2 : 4);
   if (overlaps(y, q, act_bytes) || overlaps(y, k, act_bytes) || overlaps(y, v, act_bytes))
     return HYENA_ND_ERR_INVALID_ARG;
@@ -272,6 +392,14 @@ hyena_nd_status hyena_nd_fftconv_batched(const hyena_nd_problem* p, const void* 
   a.stream = static_cast<cudaStream_t>(cuda_stream);
   a.status = static_cast<int*>(ws);
 
+  hnd::BoundsList bl;
+  bl.add(q, act_bytes);
+  bl.add(k, act_bytes);
+  bl.add(v, act_bytes);
+  bl.add(y, act_bytes);
+  bl.add(spectrum, spectrum_span(pl, spectrum_batch_stride));
+  bl.add(ws, ws_bytes);
+  if (hnd::bounds_register(bl, a.status, a.stream) != cudaSuccess) return HYENA_ND_ERR_CUDA;
   int launches = 0;
   if (run_conv(pl, a, ws, &launches) != cudaSuccess) return HYENA_ND_ERR_CUDA;
   g_last_launches = launches;
@@ -298,7 +426,7 @@ hyena_nd_status hyena_nd_fftconv_backward(const hyena_nd_problem* p, const void*
     if (!aligned16(ptr)) return HYENA_ND_ERR_MISALIGNED;
   if (spectrum_batch_stride < 0) return HYENA_ND_ERR_INVALID_ARG;
   if (spectrum_batch_stride % 16 != 0) return HYENA_ND_ERR_MISALIGNED;
-  if (ws_bytes < pl.ws_total) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
+  if (ws_bytes < pl.ws_conv) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
   const size_t act_bytes = static_cast<size_t>(pl.B * pl.C * pl.L) * (pl.bf16 ? 2 : 4);
   const void* outs[3] = {dq, dk, dv};
   const void* ins[4] = {q, k, v, dy};
@@ -318,6 +446,13 @@ hyena_nd_status hyena_nd_fftconv_backward(const hyena_nd_problem* p, const void*
   for (int i = 0; i < 3; ++i) a.n[i] = pl.n[i];
   a.stream = static_cast<cudaStream_t>(cuda_stream);
   a.status = static_cast<int*>(ws);
+  hnd::BoundsList bl;
+  for (const void* ptr : {q, k, v, dy, static_cast<const void*>(dq), static_cast<const void*>(dk),
+                          static_cast<const void*>(dv)})
+    bl.add(ptr, act_bytes);
+  bl.add(spectrum, spectrum_span(pl, spectrum_batch_stride));
+  bl.add(ws, ws_bytes);
+  if (hnd::bounds_register(bl, a.status, a.stream) != cudaSuccess) return HYENA_ND_ERR_CUDA;
   int launches = 0;
   // dq = dy . (K * (k . v)): the forward with dy as the output gate
   a.q = dy, a.k = k, a.v = v, a.y = dq, a.sconj = 1.f;
@@ -342,7 +477,7 @@ hyena_nd_status hyena_nd_kernel_grad(const hyena_nd_problem* p, const void* q, c
   const void* ptrs[6] = {q, k, v, dy, dK, ws};
   for (const void* ptr : ptrs)
     if (!aligned16(ptr)) return HYENA_ND_ERR_MISALIGNED;
-  if (ws_bytes < pl.ws_total) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
+  if (ws_bytes < pl.ws_kgrad) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
   long long noff = 1;     // dK entries per channel: linear offsets, or the periodic grid
   for (int a = 0; a < pl.ndim; ++a) noff *= pl.circular ? pl.n[a] : 2 * pl.n[a] - 1;
   const size_t act_bytes = static_cast<size_t>(pl.B * pl.C * pl.L) * (pl.bf16 ? 2 : 4);
@@ -363,6 +498,12 @@ hyena_nd_status hyena_nd_kernel_grad(const hyena_nd_problem* p, const void* q, c
   g.C = static_cast<int>(pl.C);
   g.bf16 = pl.bf16;
   g.circular = pl.circular;
+  hnd::BoundsList bl;
+  for (const void* in : ins) bl.add(in, act_bytes);
+  bl.add(dK, dk_bytes);
+  bl.add(ws, ws_bytes);
+  if (hnd::bounds_register(bl, static_cast<int*>(ws), static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
+    return HYENA_ND_ERR_CUDA;
   for (long long c0 = 0; c0 < pl.C; c0 += pl.kgrad_chunk) {
     g.c0 = static_cast<int>(c0);
     g.ncc = static_cast<int>(pl.C - c0 < pl.kgrad_chunk ? pl.C - c0 : pl.kgrad_chunk);
@@ -392,6 +533,25 @@ static hyena_nd_status filter_args(const hyena_nd_filter* f, hnd::FilterLaunch* 
   return HYENA_ND_OK;
 }
 
+// The buffers a filter call reads and writes (checked build only).
+static cudaError_t filter_bounds(const Plan& pl, const hyena_nd_filter* f, const void* spectrum, size_t spec_span,
+                                 const void* ws, size_t ws_bytes, const float* gamma, const float* beta,
+                                 cudaStream_t st) {
+  const size_t fin = static_cast<size_t>(2 * f->num_freqs * pl.ndim), H = static_cast<size_t>(f->hidden);
+  const size_t C = static_cast<size_t>(pl.C);
+  hnd::BoundsList bl;
+  bl.add(f->W1, 4 * H * fin);
+  bl.add(f->b1, 4 * H);
+  bl.add(f->W2, 4 * C * H);
+  bl.add(f->b2, 4 * C);
+  bl.add(f->alpha, 4 * C);
+  bl.add(gamma, 4 * H * static_cast<size_t>(pl.B));
+  bl.add(beta, 4 * H * static_cast<size_t>(pl.B));
+  bl.add(spectrum, spec_span);
+  bl.add(ws, ws_bytes);
+  return hnd::bounds_register(bl, static_cast<int*>(const_cast<void*>(ws)), st);
+}
+
 static cudaError_t filter_all_chunks(const Plan& pl, const hnd::FilterLaunch& fl, void* spectrum, void* ws,
                                      cudaStream_t st) {
   float2* grid = reinterpret_cast<float2*>(static_cast<char*>(ws) + kStatusBytes);
@@ -412,8 +572,11 @@ hyena_nd_status hyena_nd_filter_spectrum(const hyena_nd_problem* p, const hyena_
   if ((st = filter_args(f, &fl)) != HYENA_ND_OK) return st;
   if (!spectrum || !ws) return HYENA_ND_ERR_INVALID_ARG;
   if (!aligned16(spectrum) || !aligned16(ws)) return HYENA_ND_ERR_MISALIGNED;
-  if (ws_bytes < pl.ws_total) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
+  if (ws_bytes < pl.ws_filter) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
   fl.circular = pl.circular;
+  if (filter_bounds(pl, f, spectrum, pl.spec_bytes, ws, ws_bytes, nullptr, nullptr,
+                    static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
+    return HYENA_ND_ERR_CUDA;
   if (hnd::filter_table_bytes(fl.hidden, pl.ndim, pl.n) > 0) {
     float* tab = reinterpret_cast<float*>(static_cast<char*>(ws) + kStatusBytes + pl.filter_grid_bytes);
     if (hnd::launch_filter_tables(fl, pl.ndim, pl.n, tab, static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
@@ -438,8 +601,12 @@ hyena_nd_status hyena_nd_filter_spectrum_film(const hyena_nd_problem* p, const h
     return HYENA_ND_ERR_MISALIGNED;
   if (spectrum_batch_stride % 16 != 0) return HYENA_ND_ERR_MISALIGNED;
   if (spectrum_batch_stride < static_cast<int64_t>(pl.spec_bytes)) return HYENA_ND_ERR_INVALID_ARG;
-  if (ws_bytes < pl.ws_total) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
+  if (ws_bytes < pl.ws_filter) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
   fl.circular = pl.circular;
+  if (filter_bounds(pl, f, spectrum, static_cast<size_t>(pl.B - 1) * static_cast<size_t>(spectrum_batch_stride) +
+                                         pl.spec_bytes,
+                    ws, ws_bytes, gamma, beta, static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
+    return HYENA_ND_ERR_CUDA;
   if (hnd::filter_table_bytes(fl.hidden, pl.ndim, pl.n) > 0) {
     float* tab = reinterpret_cast<float*>(static_cast<char*>(ws) + kStatusBytes + pl.filter_grid_bytes);
     if (hnd::launch_filter_tables(fl, pl.ndim, pl.n, tab, static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
@@ -466,6 +633,11 @@ static hyena_nd_status spec_convert(const hyena_nd_problem* p, const void* src, 
   const size_t src_bytes = to_natural ? pl.spec_bytes : pl.nat_bytes;
   const size_t dst_bytes = to_natural ? pl.nat_bytes : pl.spec_bytes;
   if (overlaps2(src, src_bytes, dst, dst_bytes)) return HYENA_ND_ERR_INVALID_ARG;
+  hnd::BoundsList bl;
+  bl.add(src, src_bytes);
+  bl.add(dst, dst_bytes);
+  if (hnd::bounds_register(bl, nullptr, static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
+    return HYENA_ND_ERR_CUDA;
   return cuda_status(hnd::launch_spec_convert(pl.ndim, pl.n, pl.C, src, dst, to_natural,
                                               static_cast<cudaStream_t>(cuda_stream)));
 }
@@ -481,7 +653,12 @@ hyena_nd_status hyena_nd_spectrum_import(const hyena_nd_problem* p, const void* 
 }
 
 hyena_nd_status hyena_nd_device_status(void* ws, void* cuda_stream) {
-  if (!ws) return HYENA_ND_ERR_INVALID_ARG;
+  if (!ws) {
+    // the status word of the fixed array of hyena_nd_fftconv_batched_static
+    int* w = nullptr;
+    if (hnd::static_status_word(&w) != cudaSuccess) return HYENA_ND_ERR_CUDA;
+    ws = w;
+  }
   if (!aligned16(ws)) return HYENA_ND_ERR_MISALIGNED;
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return HYENA_ND_ERR_CUDA;

@@ -27,6 +27,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "hnd_bounds.cuh"
+
 namespace hnd {
 
 constexpr int kTab = 512;   // twiddle table: W_512^e, e in [0, 512)
@@ -141,7 +143,7 @@ __device__ __forceinline__ void pass2(float2 (&x)[2][8], int g, const float2* __
       const int jm = (g + G * b) & (NS - 1);
 #pragma unroll
       for (int r = 1; r < RP; ++r) {
-        const float2 w = T[(jm * r) * (kTab / (NS * RP))];
+        const float2 w = (*HND_S(&T[(jm * r) * (kTab / (NS * RP))]));
         x[0][b * RP + r] = c_tw<INV>(x[0][b * RP + r], w);
         x[1][b * RP + r] = c_tw<INV>(x[1][b * RP + r], w);
       }
@@ -168,7 +170,7 @@ __device__ __forceinline__ void exch2(float2 (&x)[2][8], int g, float4* buf, uns
 #pragma unroll
     for (int r = 0; r < RPO; ++r) {
       const int s = b * RPO + r;
-      buf[xpad(base + r * NSO)] = make_float4(x[0][s].x, x[0][s].y, x[1][s].x, x[1][s].y);
+      (*HND_S(&buf[xpad(base + r * NSO)])) = make_float4(x[0][s].x, x[0][s].y, x[1][s].x, x[1][s].y);
     }
   }
   __syncwarp(mask);
@@ -178,7 +180,7 @@ __device__ __forceinline__ void exch2(float2 (&x)[2][8], int g, float4* buf, uns
 #pragma unroll
     for (int r = 0; r < RPI; ++r) {
       const int s = b * RPI + r;
-      const float4 t = buf[xpad(j + r * (N / RPI))];
+      const float4 t = (*HND_S(&buf[xpad(j + r * (N / RPI))]));
       x[0][s] = make_float2(t.x, t.y);
       x[1][s] = make_float2(t.z, t.w);
     }
@@ -225,7 +227,7 @@ template <int N>
 __device__ __forceinline__ void padded_fwd(float2 (&x)[2][8], int g, float4* buf, const float2* T, unsigned mask) {
   constexpr int G = Plan<N>::G;
 #pragma unroll
-  for (int s = 0; s < 8; ++s) x[1][s] = c_mul(x[0][s], T[(g + s * G) * (kTab / (2 * N))]);
+  for (int s = 0; s < 8; ++s) x[1][s] = c_mul(x[0][s], (*HND_S(&T[(g + s * G) * (kTab / (2 * N))])));
   fft2<N, false>(x, g, buf, T, mask);
 }
 
@@ -236,7 +238,7 @@ __device__ __forceinline__ void padded_inv(float2 (&x)[2][8], int g, float4* buf
   constexpr int G = Plan<N>::G;
   fft2<N, true>(x, g, buf, T, mask);
 #pragma unroll
-  for (int s = 0; s < 8; ++s) x[0][s] = c_add(x[0][s], c_mulc(x[1][s], T[(g + s * G) * (kTab / (2 * N))]));
+  for (int s = 0; s < 8; ++s) x[0][s] = c_add(x[0][s], c_mulc(x[1][s], (*HND_S(&T[(g + s * G) * (kTab / (2 * N))]))));
 }
 
 // Natural index of the partner frequency -k (mod 2N) of spectral slot (f, p):
@@ -255,14 +257,14 @@ __device__ __forceinline__ void fetch_partner(const float2 (&x)[2][8], float2 (&
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
     const int f = spec_index<N>(g, s);
-    buf[xpad(f)] = make_float4(x[0][s].x, x[0][s].y, x[1][s].x, x[1][s].y);
+    (*HND_S(&buf[xpad(f)])) = make_float4(x[0][s].x, x[0][s].y, x[1][s].x, x[1][s].y);
   }
   __syncwarp(mask);
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
     const int f = spec_index<N>(g, s);
-    const float4 te = buf[xpad(partner_even<N>(f))];
-    const float4 to = buf[xpad(partner_odd<N>(f))];
+    const float4 te = (*HND_S(&buf[xpad(partner_even<N>(f))]));
+    const float4 to = (*HND_S(&buf[xpad(partner_odd<N>(f))]));
     xp[0][s] = make_float2(te.x, te.y);
     xp[1][s] = make_float2(to.z, to.w);
   }
@@ -271,18 +273,18 @@ __device__ __forceinline__ void fetch_partner(const float2 (&x)[2][8], float2 (&
 // ------------------------------------------------------------ activations
 struct IOF32 {
   using T = float;
-  static __device__ __forceinline__ float ld(const float* p) { return __ldcs(p); }
-  static __device__ __forceinline__ void st(float* p, float x) { __stcs(p, x); }
+  static __device__ __forceinline__ float ld(const float* p) { return __ldcs(HND_G(p)); }
+  static __device__ __forceinline__ void st(float* p, float x) { __stcs(HND_G(p), x); }
 };
 struct IOBF16 {
   using T = __nv_bfloat16;
   static __device__ __forceinline__ float ld(const __nv_bfloat16* p) {
-    const unsigned short b = __ldcs(reinterpret_cast<const unsigned short*>(p));
+    const unsigned short b = __ldcs(HND_G(reinterpret_cast<const unsigned short*>(p)));
     return __uint_as_float(static_cast<unsigned>(b) << 16);
   }
   static __device__ __forceinline__ void st(__nv_bfloat16* p, float x) {
     const __nv_bfloat16 h = __float2bfloat16_rn(x);
-    __stcs(reinterpret_cast<unsigned short*>(p), *reinterpret_cast<const unsigned short*>(&h));
+    __stcs(HND_G(reinterpret_cast<unsigned short*>(p)), *reinterpret_cast<const unsigned short*>(&h));
   }
 };
 

@@ -28,6 +28,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "hnd_bounds.cuh"
+
 namespace hnd2 {
 
 // ------------------------------------------------------------ packed fp32
@@ -251,7 +253,7 @@ __device__ __forceinline__ void tabs_build(Tabs<N> t, const float2* __restrict__
   constexpr int G = P2<N>::G;
   for (int e = threadIdx.x; e < 5 * G; e += blockDim.x) {
     const int j = e / G, g = e % G;
-    t.b[e] = j < 4 ? wtab(W512, N, g << j) : wtab(W512, 2 * N, g);
+    *HND_S(&t.b[e]) = j < 4 ? wtab(W512, N, g << j) : wtab(W512, 2 * N, g);
   }
 }
 
@@ -281,10 +283,10 @@ __device__ __forceinline__ float2 mul_w32(float2 x) {
 template <int N>
 __device__ __forceinline__ void load_bases(Tabs<N> t, int g, float2 (&u)[4]) {
   constexpr int G = P2<N>::G, R1 = P2<N>::R1;
-  u[0] = t.b[g];
-  u[1] = t.b[G + g];
-  u[2] = t.b[2 * G + g];
-  u[3] = R1 == 16 ? t.b[3 * G + g] : make_float2(1.f, 0.f);
+  u[0] = *HND_S(&t.b[g]);
+  u[1] = *HND_S(&t.b[G + g]);
+  u[2] = *HND_S(&t.b[2 * G + g]);
+  u[3] = R1 == 16 ? *HND_S(&t.b[3 * G + g]) : make_float2(1.f, 0.f);
 }
 
 __device__ __forceinline__ float4 w4of(float2 w) { return make_float4(w.x, w.x, w.y, w.y); }
@@ -313,7 +315,7 @@ __device__ __forceinline__ void fft_fwd(cp (&x)[P2<N>::R1], int g, float4* buf, 
     __syncwarp();
 #pragma unroll
     for (int r = 0; r < R1; ++r)
-      buf[padx<R1>(g * R1 + r)] = make_float4(x[r].re.x, x[r].re.y, x[r].im.x, x[r].im.y);
+      *HND_S(&buf[padx<R1>(g * R1 + r)]) = make_float4(x[r].re.x, x[r].re.y, x[r].im.x, x[r].im.y);
     __syncwarp();
     float2 u[4];
     load_bases<N>(t, g, u);
@@ -321,7 +323,7 @@ __device__ __forceinline__ void fft_fwd(cp (&x)[P2<N>::R1], int g, float4* buf, 
       constexpr int b = decltype(bc)::value;
       sfor<0, R2>([&](auto rc) {
         constexpr int r = decltype(rc)::value;
-        const float4 v = buf[padx<R1>(g + G * b + r * R1)];
+        const float4 v = *HND_S(&buf[padx<R1>(g + G * b + r * R1)]);
         cp y = {make_float2(v.x, v.y), make_float2(v.z, v.w)};
         if constexpr (r > 0) {
           // W_N^{(g + G b) r} = u^r W_R1^{b r}
@@ -359,7 +361,7 @@ __device__ __forceinline__ void fft_inv(cp (&x)[P2<N>::R1], int g, float4* buf, 
 #pragma unroll
       for (int r = 0; r < R2; ++r) {
         const int s = b * R2 + r;
-        buf[padx<PD>((g + G * b) * R2 + r)] = make_float4(x[s].re.x, x[s].re.y, x[s].im.x, x[s].im.y);
+        *HND_S(&buf[padx<PD>((g + G * b) * R2 + r)]) = make_float4(x[s].re.x, x[s].re.y, x[s].im.x, x[s].im.y);
       }
     }
     __syncwarp();
@@ -367,7 +369,7 @@ __device__ __forceinline__ void fft_inv(cp (&x)[P2<N>::R1], int g, float4* buf, 
     load_bases<N>(t, g, u);
     sfor<0, R1>([&](auto rc) {
       constexpr int r = decltype(rc)::value;
-      const float4 v = buf[padx<PD>(g + r * G)];
+      const float4 v = *HND_S(&buf[padx<PD>(g + r * G)]);
       cp y = {make_float2(v.x, v.y), make_float2(v.z, v.w)};
       if constexpr (r > 0) y = ctw<true>(y, w4of(upow<r>(u)));     // W_N^{g r}
       x[r] = y;
@@ -384,7 +386,7 @@ template <int N>
 __device__ __forceinline__ void padded_fwd(const float2 (&z)[P2<N>::R1], cp (&x)[P2<N>::R1], int g, float4* buf,
                                            int key, Tabs<N> t, unsigned mask) {
   constexpr int G = P2<N>::G, R1 = P2<N>::R1;
-  const float2 tg = t.b[4 * G + g];
+  const float2 tg = *HND_S(&t.b[4 * G + g]);
   sfor<0, R1>([&](auto sc) {
     constexpr int s = decltype(sc)::value;
     const float2 w = mul_w32<s * (16 / R1)>(tg);     // W_2N^{g + s G} = W_2N^g W_{2 R1}^s
@@ -404,7 +406,7 @@ __device__ __forceinline__ void full_fwd(const float2 (&lo)[P2<N>::R1], const fl
                                          cp (&x)[P2<N>::R1], int g, float4* buf, int key, Tabs<N> t,
                                          unsigned mask) {
   constexpr int G = P2<N>::G, R1 = P2<N>::R1;
-  const float2 tg = t.b[4 * G + g];
+  const float2 tg = *HND_S(&t.b[4 * G + g]);
   sfor<0, R1>([&](auto sc) {
     constexpr int s = decltype(sc)::value;
     const float2 w = mul_w32<s * (16 / R1)>(tg);     // W_2N^{g + s G}
@@ -423,7 +425,7 @@ __device__ __forceinline__ void padded_inv(cp (&x)[P2<N>::R1], float2 (&out)[P2<
                                            Tabs<N> t, unsigned mask) {
   constexpr int G = P2<N>::G, R1 = P2<N>::R1;
   fft_inv<N>(x, g, buf, key, t, mask);
-  const float2 tg = t.b[4 * G + g];
+  const float2 tg = *HND_S(&t.b[4 * G + g]);
   sfor<0, R1>([&](auto sc) {
     constexpr int s = decltype(sc)::value;
     const float2 w = mul_w32<s * (16 / R1)>(tg);   // untwist by conj(W_2N^{g + s G})
@@ -441,13 +443,13 @@ __device__ __forceinline__ void fetch_partner(const cp (&x)[P2<N>::R1], cp (&xp)
   __syncwarp();
 #pragma unroll
   for (int s = 0; s < P2<N>::R1; ++s)
-    buf[swz(spec_idx<N>(g, s)) ^ key] = make_float4(x[s].re.x, x[s].re.y, x[s].im.x, x[s].im.y);
+    *HND_S(&buf[swz(spec_idx<N>(g, s)) ^ key]) = make_float4(x[s].re.x, x[s].re.y, x[s].im.x, x[s].im.y);
   __syncwarp();
 #pragma unroll
   for (int s = 0; s < P2<N>::R1; ++s) {
     const int f = spec_idx<N>(g, s);
-    const float4 a = buf[swz((N - f) & (N - 1)) ^ key];
-    const float4 b = buf[swz(N - 1 - f) ^ key];
+    const float4 a = *HND_S(&buf[swz((N - f) & (N - 1)) ^ key]);
+    const float4 b = *HND_S(&buf[swz(N - 1 - f) ^ key]);
     xp[s] = {make_float2(a.x, b.y), make_float2(a.z, b.w)};
   }
 }

@@ -69,11 +69,11 @@ static __global__ void k_filter_tables(const float* __restrict__ W1, int hidden,
           float sv, cv;
           sincospif(static_cast<float>(m) * (static_cast<float>(t) / static_cast<float>(nn[a])), &sv, &cv);
           const int f = 2 * (a * num_freqs + m - 1);
-          acc = fmaf(__ldg(W1 + static_cast<long long>(h) * fin + f), sv, acc);
-          acc = fmaf(__ldg(W1 + static_cast<long long>(h) * fin + f + 1), cv, acc);
+          acc = fmaf(__ldg(HND_G(W1 + static_cast<long long>(h) * fin + f)), sv, acc);
+          acc = fmaf(__ldg(HND_G(W1 + static_cast<long long>(h) * fin + f + 1)), cv, acc);
         }
       }
-      tab[base + e] = acc;
+      (*HND_G(&tab[base + e])) = acc;
     }
     base += static_cast<long long>(HP) * E;
   }
@@ -90,6 +90,18 @@ struct FilterSmem {
            sizeof(int) * 4 * kFO;
   }
 };
+
+// sin(x) for the sine layer: Cody-Waite reduction of x to r = x - 2 pi m in
+// [-pi, pi] (m = rint(x / 2 pi), 2 pi split into a head exact in fp32 and a
+// tail), then the hardware sine approximation __sinf on r, whose absolute
+// error on [-pi, pi] is about 2^-21.  The hidden units feed the kernel
+// values, whose spectrum is checked against the float64 oracle at 2e-5.
+__device__ __forceinline__ float sine_layer(float x) {
+  const float m = rintf(x * 0.15915494309189535f);         // 1 / (2 pi)
+  float r = fmaf(m, -6.28125f, x);                          // 2 pi head (exact times m for |m| < 2^15)
+  r = fmaf(m, -1.9353071795864769e-3f, r);                  // 2 pi - 6.28125
+  return __sinf(r);
+}
 
 template <int HP, bool TAB>
 __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
@@ -132,10 +144,10 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
   if constexpr (!TAB) {
     for (int i = tid; i < fin * HP; i += kFT) {
       const int f = i / HP, h = i % HP;
-      w1[i] = h < a.hidden ? __ldg(a.W1 + static_cast<long long>(h) * fin + f) : 0.f;
+      (*HND_S(&w1[i])) = h < a.hidden ? __ldg(HND_G(a.W1 + static_cast<long long>(h) * fin + f)) : 0.f;
     }
   }
-  for (int h = tid; h < HP; h += kFT) b1[h] = h < a.hidden ? __ldg(a.b1 + h) : 0.f;
+  for (int h = tid; h < HP; h += kFT) (*HND_S(&b1[h])) = h < a.hidden ? __ldg(HND_G(a.b1 + h)) : 0.f;
   // offsets of this tile: radius and slot (offset t at t mod P per axis)
   for (int o = tid; o < kFO; o += kFT) {
     int t0, t1, t2;
@@ -144,13 +156,13 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
                 f2 = static_cast<float>(rep(t2, n2));
     // the window's argument |t| / s, squared for the Gaussian window
     const float rs = sqrtf(f0 * f0 + f1 * f1 + f2 * f2) / a.decay_scale;
-    rad[o] = a.window == 1 ? rs * rs : rs;
+    (*HND_S(&rad[o])) = a.window == 1 ? rs * rs : rs;
     const int s0 = (t0 + P0) % P0, s1 = (t1 + P1) % P1, s2 = (t2 + P2) % P2;
-    slot[o] = (s0 * P1 + s1) * P2 + s2;
+    (*HND_S(&slot[o])) = (s0 * P1 + s1) * P2 + s2;
     if constexpr (TAB) {
-      tix[o] = rep(t0, n0) + n0 - 1;
-      tix[kFO + o] = rep(t1, n1) + n1 - 1;
-      tix[2 * kFO + o] = rep(t2, n2) + n2 - 1;
+      (*HND_S(&tix[o])) = rep(t0, n0) + n0 - 1;
+      (*HND_S(&tix[kFO + o])) = rep(t1, n1) + n1 - 1;
+      (*HND_S(&tix[2 * kFO + o])) = rep(t2, n2) + n2 - 1;
     }
   }
   if constexpr (!TAB) {
@@ -164,8 +176,8 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
       const int tax = rep(ax == 0 ? t0 : (ax == 1 ? t1 : t2), nax);
       float sv, cv;
       sincospif(static_cast<float>(m) * (static_cast<float>(tax) / static_cast<float>(nax)), &sv, &cv);
-      phi[(2 * (ax * M + m - 1)) * kFO + o] = sv;
-      phi[(2 * (ax * M + m - 1) + 1) * kFO + o] = cv;
+      (*HND_S(&phi[(2 * (ax * M + m - 1)) * kFO + o])) = sv;
+      (*HND_S(&phi[(2 * (ax * M + m - 1) + 1) * kFO + o])) = cv;
     }
   }
   __syncthreads();
@@ -180,11 +192,11 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
     const float* T2 = T1 + static_cast<long long>(HP) * (a.ndim > 1 ? E1t : 0);
     for (int i = tid; i < HP * kFO; i += kFT) {
       const int o = i % kFO, h = i / kFO;
-      float pre = b1[h] + __ldg(T0 + h * E0t + tix[o]);
-      if (a.ndim > 1) pre += __ldg(T1 + h * E1t + tix[kFO + o]);
-      if (a.ndim > 2) pre += __ldg(T2 + h * E2t + tix[2 * kFO + o]);
-      if (a.gamma && h < a.hidden) pre = fmaf(__ldg(a.gamma + h), pre, __ldg(a.beta + h));
-      hid[h * kFO + o] = h < a.hidden ? sinf(pre) : 0.f;
+      float pre = (*HND_S(&b1[h])) + __ldg(HND_G(T0 + h * E0t + (*HND_S(&tix[o]))));
+      if (a.ndim > 1) pre += __ldg(HND_G(T1 + h * E1t + (*HND_S(&tix[kFO + o]))));
+      if (a.ndim > 2) pre += __ldg(HND_G(T2 + h * E2t + (*HND_S(&tix[2 * kFO + o]))));
+      if (a.gamma && h < a.hidden) pre = fmaf(__ldg(HND_G(a.gamma + h)), pre, __ldg(HND_G(a.beta + h)));
+      (*HND_S(&hid[h * kFO + o])) = h < a.hidden ? sine_layer(pre) : 0.f;
     }
   } else {
     // hidden layer: thread (og, hg) computes offsets 4 og .. 4 og + 3 x units hg HG ..
@@ -193,13 +205,13 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < HG; ++j) acc[i][j] = b1[grp * HG + j];
+        for (int j = 0; j < HG; ++j) acc[i][j] = (*HND_S(&b1[grp * HG + j]));
       for (int f = 0; f < fin; ++f) {
-        const float4 p = *reinterpret_cast<const float4*>(phi + f * kFO + 4 * og);
+        const float4 p = *HND_S(reinterpret_cast<const float4*>(phi + f * kFO + 4 * og));
         const float pv[4] = {p.x, p.y, p.z, p.w};
 #pragma unroll
         for (int j4 = 0; j4 < HG / 4; ++j4) {
-          const float4 w = *reinterpret_cast<const float4*>(w1 + f * HP + grp * HG + 4 * j4);
+          const float4 w = *HND_S(reinterpret_cast<const float4*>(w1 + f * HP + grp * HG + 4 * j4));
           const float wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i)
@@ -211,16 +223,16 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
 #pragma unroll
         for (int j = 0; j < HG; ++j) {
           const int hu = grp * HG + j;
-          const float gm = hu < a.hidden ? __ldg(a.gamma + hu) : 0.f;
-          const float bt = hu < a.hidden ? __ldg(a.beta + hu) : 0.f;
+          const float gm = hu < a.hidden ? __ldg(HND_G(a.gamma + hu)) : 0.f;
+          const float bt = hu < a.hidden ? __ldg(HND_G(a.beta + hu)) : 0.f;
 #pragma unroll
           for (int i = 0; i < 4; ++i) acc[i][j] = fmaf(gm, acc[i][j], bt);
         }
       }
 #pragma unroll
       for (int j = 0; j < HG; ++j)
-        *reinterpret_cast<float4*>(hid + (grp * HG + j) * kFO + 4 * og) =
-            make_float4(sinf(acc[0][j]), sinf(acc[1][j]), sinf(acc[2][j]), sinf(acc[3][j]));
+        *HND_S(reinterpret_cast<float4*>(hid + (grp * HG + j) * kFO + 4 * og)) =
+            make_float4(sine_layer(acc[0][j]), sine_layer(acc[1][j]), sine_layer(acc[2][j]), sine_layer(acc[3][j]));
     }
   }
 
@@ -232,7 +244,7 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
     for (int i = tid; i < HP * kFC; i += kFT) {
       const int h = i / kFC, cc = i % kFC;
       const int c = ct + cc;
-      w2[i] = (h < a.hidden && c < a.nc) ? __ldg(a.W2 + static_cast<long long>(a.c0 + c) * a.hidden + h) : 0.f;
+      (*HND_S(&w2[i])) = (h < a.hidden && c < a.nc) ? __ldg(HND_G(a.W2 + static_cast<long long>(a.c0 + c) * a.hidden + h)) : 0.f;
     }
     __syncthreads();
     float acc[4][4];
@@ -242,8 +254,8 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
       for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
 #pragma unroll 4
     for (int h = 0; h < HP; ++h) {
-      const float4 hv = *reinterpret_cast<const float4*>(hid + h * kFO + 4 * og);
-      const float4 wv = *reinterpret_cast<const float4*>(w2 + h * kFC + 4 * grp);
+      const float4 hv = *HND_S(reinterpret_cast<const float4*>(hid + h * kFO + 4 * og));
+      const float4 wv = *HND_S(reinterpret_cast<const float4*>(w2 + h * kFC + 4 * grp));
       const float hh[4] = {hv.x, hv.y, hv.z, hv.w}, ww[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i)
@@ -254,13 +266,13 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
     for (int j = 0; j < 4; ++j) {
       const int c = ct + 4 * grp + j;
       if (c >= a.nc) continue;
-      const float bb = __ldg(a.b2 + a.c0 + c), al = __ldg(a.alpha + a.c0 + c);
+      const float bb = __ldg(HND_G(a.b2 + a.c0 + c)), al = __ldg(HND_G(a.alpha + a.c0 + c));
       float2* gch = a.grid + static_cast<long long>(c) * gsz;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int o = 4 * og + i;
         if (e0 + o < noff)
-          gch[slot[o]] = make_float2((acc[i][j] + bb) * expf(-al * rad[o]), 0.f);
+          (*HND_G(&gch[(*HND_S(&slot[o]))])) = make_float2((acc[i][j] + bb) * __expf(-al * (*HND_S(&rad[o]))), 0.f);
       }
     }
   }
@@ -314,8 +326,8 @@ __global__ void __launch_bounds__(kAT) k_fft_axis2(float2* __restrict__ data, co
 #pragma unroll
     for (int s = 0; s < R1; ++s) {
       const long long j = g + s * G;
-      lo[s] = act ? base[j * stride] : make_float2(0.f, 0.f);
-      hi[s] = act ? base[(j + N) * stride] : make_float2(0.f, 0.f);
+      lo[s] = act ? (*HND_G(&base[j * stride])) : make_float2(0.f, 0.f);
+      hi[s] = act ? (*HND_G(&base[(j + N) * stride])) : make_float2(0.f, 0.f);
     }
     cp x[R1];
     full_fwd<N>(lo, hi, x, g, buf, 0, t, 0u);
@@ -323,8 +335,8 @@ __global__ void __launch_bounds__(kAT) k_fft_axis2(float2* __restrict__ data, co
 #pragma unroll
       for (int s = 0; s < R1; ++s) {
         const long long kk = 2LL * spec_idx<N>(g, s);
-        base[kk * stride] = make_float2(x[s].re.x, x[s].im.x);
-        base[(kk + 1) * stride] = make_float2(x[s].re.y, x[s].im.y);
+        (*HND_G(&base[kk * stride])) = make_float2(x[s].re.x, x[s].im.x);
+        (*HND_G(&base[(kk + 1) * stride])) = make_float2(x[s].re.y, x[s].im.y);
       }
     }
   }

@@ -73,21 +73,21 @@ template <class T>
 struct Act;
 template <>
 struct Act<float> {
-  static __device__ __forceinline__ float ld_s(const float* p) { return *p; }
-  static __device__ __forceinline__ float ld_g(const float* p) { return __ldcs(p); }
-  static __device__ __forceinline__ void st_g(float* p, float x) { __stcs(p, x); }
+  static __device__ __forceinline__ float ld_s(const float* p) { return *HND_S(p); }
+  static __device__ __forceinline__ float ld_g(const float* p) { return __ldcs(HND_G(p)); }
+  static __device__ __forceinline__ void st_g(float* p, float x) { __stcs(HND_G(p), x); }
 };
 template <>
 struct Act<__nv_bfloat16> {
   static __device__ __forceinline__ float ld_s(const __nv_bfloat16* p) {
-    return __uint_as_float(static_cast<unsigned>(*reinterpret_cast<const unsigned short*>(p)) << 16);
+    return __uint_as_float(static_cast<unsigned>(*HND_S(reinterpret_cast<const unsigned short*>(p))) << 16);
   }
   static __device__ __forceinline__ float ld_g(const __nv_bfloat16* p) {
-    return __uint_as_float(static_cast<unsigned>(__ldcs(reinterpret_cast<const unsigned short*>(p))) << 16);
+    return __uint_as_float(static_cast<unsigned>(__ldcs(HND_G(reinterpret_cast<const unsigned short*>(p)))) << 16);
   }
   static __device__ __forceinline__ void st_g(__nv_bfloat16* p, float x) {
     const __nv_bfloat16 h = __float2bfloat16_rn(x);
-    __stcs(reinterpret_cast<unsigned short*>(p), *reinterpret_cast<const unsigned short*>(&h));
+    __stcs(HND_G(reinterpret_cast<unsigned short*>(p)), *reinterpret_cast<const unsigned short*>(&h));
   }
 };
 
@@ -140,7 +140,7 @@ __device__ __forceinline__ void rows_fwd(const T* kst, const T* vst, float4* Zb,
     if (act) {
 #pragma unroll
       for (int s = 0; s < 8; ++s)
-        Zb[spec_idx<N1>(g, s) * L::RPS + rp] = make_float4(x[s].re.x, x[s].im.x, x[s].re.y, x[s].im.y);
+        *HND_S(&Zb[spec_idx<N1>(g, s) * L::RPS + rp]) = make_float4(x[s].re.x, x[s].im.x, x[s].re.y, x[s].im.y);
     }
   }
 }
@@ -161,7 +161,7 @@ __device__ __forceinline__ void rows_inv(const T* qst, const float4* Zb, T* yp, 
     cp x[8];
 #pragma unroll
     for (int s = 0; s < 8; ++s) {
-      const float4 e = act ? Zb[spec_idx<N1>(g, s) * L::RPS + rp] : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 e = act ? *HND_S(&Zb[spec_idx<N1>(g, s) * L::RPS + rp]) : make_float4(0.f, 0.f, 0.f, 0.f);
       x[s] = {make_float2(e.x, e.z), make_float2(e.y, e.w)};
     }
     float2 o[8];
@@ -219,7 +219,7 @@ __device__ __forceinline__ void columns(float4* Zb4, float4* xb, const float4* _
       const float4* su = sp + (cu == 0 ? 0LL : static_cast<long long>(cu + 1) * N0);
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
-        S[s] = __ldg(su + s * G + g);
+        S[s] = __ldg(HND_G(su + s * G + g));
         S[s].z *= sgn, S[s].w *= sgn;     // sgn = -1: conjugate spectrum (adjoint)
       }
     }
@@ -229,8 +229,8 @@ __device__ __forceinline__ void columns(float4* Zb4, float4* xb, const float4* _
       const int rp = g + s * G;
       float2 z1 = make_float2(0.f, 0.f), z2 = z1;
       if (act) {
-        z1 = Zb[zidx(kx, rp)];
-        z2 = Zb[zidx(kxm, rp)];
+        z1 = *HND_S(&Zb[zidx(kx, rp)]);
+        z2 = *HND_S(&Zb[zidx(kxm, rp)]);
       }
       if (cu == 0) {
         z[s] = make_float2(z1.x, z2.x);       // row a: (DC, Nyquist)
@@ -249,7 +249,7 @@ __device__ __forceinline__ void columns(float4* Zb4, float4* xb, const float4* _
       for (int s = 0; s < 8; ++s) {
         float4 Bc = make_float4(0.f, 0.f, 0.f, 0.f);
         if (cu == 0) {
-          Bc = __ldg(sp + N0 + s * G + g);
+          Bc = __ldg(HND_G(sp + N0 + s * G + g));
           Bc.z *= sgn, Bc.w *= sgn;
         }
         const cp a = cmulp(x[s], make_float2(S[s].x, S[s].y), make_float2(S[s].z, S[s].w));
@@ -269,11 +269,11 @@ __device__ __forceinline__ void columns(float4* Zb4, float4* xb, const float4* _
         const int rp = g + s * G;
         const float2 ya = o[s], yb = o[s + 4];
         if (cu == 0) {
-          Zb[zidx(0, rp)] = make_float2(ya.x, yb.x);
-          Zb[zidx(N1, rp)] = make_float2(ya.y, yb.y);
+          *HND_S(&Zb[zidx(0, rp)]) = make_float2(ya.x, yb.x);
+          *HND_S(&Zb[zidx(N1, rp)]) = make_float2(ya.y, yb.y);
         } else {
-          Zb[zidx(kx, rp)] = pack_pos(ya, yb);
-          Zb[zidx(kxm, rp)] = pack_neg(ya, yb);
+          *HND_S(&Zb[zidx(kx, rp)]) = pack_pos(ya, yb);
+          *HND_S(&Zb[zidx(kxm, rp)]) = pack_neg(ya, yb);
         }
       }
     }
@@ -338,18 +338,24 @@ __global__ void __launch_bounds__(kT3, 1)
     if (r < 2 * N0) {
       const int row = r % N0;
       const T* src = (r < N0 ? k : v) + base + static_cast<long long>(row) * N1;
+      T* dst = (r < N0 ? kst : vst) + row * L::PITCH;
+      // (checked build: a copy outside its buffers is skipped and delivers no bytes)
+      const bool okc = HND_RANGE_OK(src, N1 * sizeof(T)) && HND_RANGE_OK(dst, N1 * sizeof(T));
       fence_proxy_async();
-      mbar_expect_tx(bar_kv, N1 * sizeof(T));
-      bulk_g2s((r < N0 ? kst : vst) + row * L::PITCH, src, N1 * sizeof(T), bar_kv);
+      mbar_expect_tx(bar_kv, okc ? N1 * sizeof(T) : 0u);
+      if (okc) bulk_g2s(dst, src, N1 * sizeof(T), bar_kv);
     }
   };
   auto copy_q = [&](int vv) {
     const long long base = vol_base(vv);
     const int r = threadIdx.x;
     if (r < N0) {
+      const T* src = q + base + static_cast<long long>(r) * N1;
+      T* dst = qst + r * L::PITCH;
+      const bool okc = HND_RANGE_OK(src, N1 * sizeof(T)) && HND_RANGE_OK(dst, N1 * sizeof(T));
       fence_proxy_async();
-      mbar_expect_tx(bar_q, N1 * sizeof(T));
-      bulk_g2s(qst + r * L::PITCH, q + base + static_cast<long long>(r) * N1, N1 * sizeof(T), bar_q);
+      mbar_expect_tx(bar_q, okc ? N1 * sizeof(T) : 0u);
+      if (okc) bulk_g2s(dst, src, N1 * sizeof(T), bar_q);
     }
   };
 
@@ -470,16 +476,16 @@ static __global__ void k_spec_import_v2(const float2* __restrict__ nat, float4* 
     const float2* src = nat + c * src_per;
     float2 s0, s1;
     if (ps.kind == 0) {
-      s0 = src[ps.ky0 * full_pitch + ps.kx];
-      s1 = src[ps.ky1 * full_pitch + ps.kx];
+      s0 = *HND_G(&src[ps.ky0 * full_pitch + ps.kx]);
+      s1 = *HND_G(&src[ps.ky1 * full_pitch + ps.kx]);
     } else {
       const float sg = ps.kind == 1 ? 1.f : -1.f;
-      const float2 a0 = src[ps.ky0 * full_pitch], b0 = src[ps.ky0 * full_pitch + n1];
-      const float2 a1 = src[ps.ky1 * full_pitch], b1 = src[ps.ky1 * full_pitch + n1];
+      const float2 a0 = *HND_G(&src[ps.ky0 * full_pitch]), b0 = *HND_G(&src[ps.ky0 * full_pitch + n1]);
+      const float2 a1 = *HND_G(&src[ps.ky1 * full_pitch]), b1 = *HND_G(&src[ps.ky1 * full_pitch + n1]);
       s0 = make_float2(0.5f * (a0.x + sg * b0.x), 0.5f * (a0.y + sg * b0.y));
       s1 = make_float2(0.5f * (a1.x + sg * b1.x), 0.5f * (a1.y + sg * b1.y));
     }
-    out[e] = make_float4(scale * s0.x, scale * s1.x, scale * s0.y, scale * s1.y);
+    *HND_G(&out[e]) = make_float4(scale * s0.x, scale * s1.x, scale * s0.y, scale * s1.y);
   }
 }
 
@@ -493,16 +499,16 @@ static __global__ void k_spec_export_v2(const float4* __restrict__ lib, float2* 
     const long long c = e / per, e4 = e % per;
     const Pos2 ps = pos2_of(n0, n1, e4);
     float2* dst = nat + c * per * 2;
-    const float4 f = lib[e];
+    const float4 f = *HND_G(&lib[e]);
     if (ps.kind == 0) {
-      dst[ps.ky0 * W + ps.kx] = make_float2(f.x, f.z);
-      dst[ps.ky1 * W + ps.kx] = make_float2(f.y, f.w);
+      *HND_G(&dst[ps.ky0 * W + ps.kx]) = make_float2(f.x, f.z);
+      *HND_G(&dst[ps.ky1 * W + ps.kx]) = make_float2(f.y, f.w);
     } else if (ps.kind == 1) {
-      const float4 g = lib[e + n0];     // the B payload at the same position
-      dst[ps.ky0 * W] = make_float2(f.x + g.x, f.z + g.z);
-      dst[ps.ky0 * W + n1] = make_float2(f.x - g.x, f.z - g.z);
-      dst[ps.ky1 * W] = make_float2(f.y + g.y, f.w + g.w);
-      dst[ps.ky1 * W + n1] = make_float2(f.y - g.y, f.w - g.w);
+      const float4 g = *HND_G(&lib[e + n0]);     // the B payload at the same position
+      *HND_G(&dst[ps.ky0 * W]) = make_float2(f.x + g.x, f.z + g.z);
+      *HND_G(&dst[ps.ky0 * W + n1]) = make_float2(f.x - g.x, f.z - g.z);
+      *HND_G(&dst[ps.ky1 * W]) = make_float2(f.y + g.y, f.w + g.w);
+      *HND_G(&dst[ps.ky1 * W + n1]) = make_float2(f.y - g.y, f.w - g.w);
     }
   }
 }

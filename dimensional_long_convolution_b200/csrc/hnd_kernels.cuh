@@ -40,7 +40,7 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kXWarp = 4608 / 16;       // float4 per warp of exchange buffers
 
 __device__ __forceinline__ void load_twiddles(float2* T) {
-  for (int i = threadIdx.x; i < kTab; i += blockDim.x) T[i] = g_tw[i];
+  for (int i = threadIdx.x; i < kTab; i += blockDim.x) (*HND_S(&T[i])) = g_tw[i];
 }
 
 // Shared memory of the 1D row kernel: the twiddle table and its warps' exchange buffers.
@@ -99,11 +99,11 @@ __global__ void __launch_bounds__(kThreads) k_rows1d(const typename IO::T* __res
         const float2 xa = unpack_a(x[p][s], xp[p][s]), xbv = unpack_b(x[p][s], xp[p][s]);
         float2 Sa, Sb;
         if (kk <= N) {
-          Sa = __ldg(sa + kk);
-          Sb = __ldg(sb + kk);
+          Sa = __ldg(HND_G(sa + kk));
+          Sb = __ldg(HND_G(sb + kk));
         } else {
-          Sa = c_conj(__ldg(sa + 2 * N - kk));
-          Sb = c_conj(__ldg(sb + 2 * N - kk));
+          Sa = c_conj(__ldg(HND_G(sa + 2 * N - kk)));
+          Sb = c_conj(__ldg(HND_G(sb + 2 * N - kk)));
         }
         Sa.y *= sgn, Sb.y *= sgn;     // sgn = -1: conjugate spectrum (adjoint)
         x[p][s] = pack_pos(c_mul(xa, Sa), c_mul(xbv, Sb));
@@ -145,14 +145,14 @@ static __global__ void k_spec_import(const float2* __restrict__ nat, float2* __r
   const long long total = spec_per_channel(d) * C;
   for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<long long>(gridDim.x) * blockDim.x)
-    out[e] = nat[e];
+    (*HND_G(&out[e])) = (*HND_G(&nat[e]));
 }
 
 static __global__ void k_spec_export(const float2* __restrict__ lib, float2* __restrict__ nat, SpecDims d, long long C) {
   const long long total = spec_per_channel(d) * C;
   for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<long long>(gridDim.x) * blockDim.x)
-    nat[e] = lib[e];
+    (*HND_G(&nat[e])) = (*HND_G(&lib[e]));
 }
 
 // ================================================================ the filter
@@ -166,7 +166,7 @@ static __global__ void k_spec_pack(const float2* __restrict__ grid, float2* __re
   for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<long long>(gridDim.x) * blockDim.x) {
     const long long cl = e / per, o = e % per;
-    out[(c0 + cl) * per + o] = c_scale(grid[cl * P + o], scale);
+    (*HND_G(&out[(c0 + cl) * per + o])) = c_scale((*HND_G(&grid[cl * P + o])), scale);
   }
 }
 

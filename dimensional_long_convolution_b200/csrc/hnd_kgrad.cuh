@@ -50,7 +50,7 @@ static __global__ void k_kg_pad(const T* __restrict__ k, const T* __restrict__ v
       const long long idx = (static_cast<long long>(bb) * C + c0 + cl) * L + (static_cast<long long>(s0) * d.n1 + s1) * d.n2 + s2;
       val = make_float2(Act<T>::ld_g(k + idx) * Act<T>::ld_g(v + idx), Act<T>::ld_g(q + idx) * Act<T>::ld_g(dy + idx));
     }
-    grid[e] = val;
+    (*HND_G(&grid[e])) = val;
   }
 }
 
@@ -97,20 +97,20 @@ static __global__ void k_kg_corr(const float2* __restrict__ gw, float2* __restri
       if (c >= ncc) break;
       for (int b = 0; b < B; ++b) {
         const long long o = (c * B + b) * gsz;
-        const float2 w = gw[o + r], wm = gw[o + rn];
+        const float2 w = (*HND_G(&gw[o + r])), wm = (*HND_G(&gw[o + rn]));
         are[j] += 0.5f * (w.x * wm.y + w.y * wm.x);                                  // Im(W Wm) / 2
         aim[j] -= 0.25f * ((w.x * w.x + w.y * w.y) - (wm.x * wm.x + wm.y * wm.y));   // -(|W|^2 - |Wm|^2) / 4
       }
     }
     // conj(A1) - i conj(A2) = (a1r - a2i) + i (-a1i - a2r)
-    acc[e] = make_float2(are[0] - aim[1], -aim[0] - are[1]);
+    (*HND_G(&acc[e])) = make_float2(are[0] - aim[1], -aim[0] - are[1]);
   }
 }
 
 // channel c of the chunk sits in grid c / 2: even c the real part, odd c
 // minus the imaginary part
 __device__ __forceinline__ float kg_part(const float2* acc, long long c, long long gsz, long long slot) {
-  const float2 x = acc[(c >> 1) * gsz + slot];
+  const float2 x = (*HND_G(&acc[(c >> 1) * gsz + slot]));
   return (c & 1) ? -x.y : x.x;
 }
 
@@ -131,7 +131,7 @@ static __global__ void k_kg_extract(const float2* __restrict__ acc, float* __res
     const unsigned slot = ((static_cast<unsigned>(t0 + d.P0) & (d.P0 - 1)) << (d.l1 + d.l2)) |
                           ((static_cast<unsigned>(t1 + d.P1) & (d.P1 - 1)) << d.l2) |
                           (static_cast<unsigned>(t2 + d.P2) & (d.P2 - 1));
-    dK[static_cast<long long>(c0 + c) * noff + off] = kg_part(acc, c, gsz, slot) * scale;
+    (*HND_G(&dK[static_cast<long long>(c0 + c) * noff + off])) = kg_part(acc, c, gsz, slot) * scale;
   }
 }
 
@@ -159,7 +159,7 @@ static __global__ void k_kg_extract_periodic(const float2* __restrict__ acc, flo
                                  (t2 + d.P2) % d.P2;
           sum += kg_part(acc, c, gsz, slot);
         }
-    dK[(c0 + c) * nper + off] = sum * scale;
+    (*HND_G(&dK[(c0 + c) * nper + off])) = sum * scale;
   }
 }
 

@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <mutex>
+
 namespace hnd {
 
 struct ConvArgs {
@@ -34,6 +36,28 @@ inline bool fused_2d(int ndim, const int* n) { return ndim == 2 && n[0] <= 64 &&
 
 // Streaming multiprocessors of the current device (cached per device).
 int sm_count();
+
+// Volumes per wave of a multi-pass tier: as many as `budget` bytes of
+// intermediates hold (per_pair bytes each, at least one), then evened out so
+// that no wave is short; with whole_channels, a multiple of B where possible
+// so that the B samples sharing a channel spectrum run in one wave.
+long long balanced_wave(long long pairs, long long B, size_t per_pair, size_t budget, bool whole_channels);
+// A second stream per device (created on first use, kept until exit) with
+// the events that fork it from, stagger it against and join it back to the
+// caller's stream; `mu` serialises the enqueue of calls that use it.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, stagger = nullptr, join = nullptr;
+  std::mutex mu;
+};
+cudaError_t side_stream(SideStream** out);
+// Record the kernel count of the latest successful convolution call on this
+// host thread (read by hyena_nd_last_launch_count).
+void note_launches(int n);
+// Device address of the status word at the head of the fixed array used by
+// hyena_nd_fftconv_batched_static, on the current device (looked up once per
+// device).
+cudaError_t static_status_word(int** out);
 
 // Maximum dynamic shared memory per CTA on sm_100 (227 KB).
 constexpr size_t kMaxSmem = 232448;

@@ -35,8 +35,8 @@ static __global__ void k_l1_twiddle(float2* __restrict__ grid, int Pa, long long
     const long long m = ((e / R) % Pa) * (e % R);
     float s, c;
     sincospif(-2.f * (static_cast<float>(m) / static_cast<float>(Q)), &s, &c);
-    const float2 x = grid[e];
-    grid[e] = make_float2(x.x * c - x.y * s, x.x * s + x.y * c);
+    const float2 x = *HND_G(&grid[e]);
+    *HND_G(&grid[e]) = make_float2(x.x * c - x.y * s, x.x * s + x.y * c);
   }
 }
 
@@ -46,8 +46,8 @@ static __global__ void k_l1_spec_store(const float2* __restrict__ grid, float2* 
   const long long total = P * nc;
   for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const float2 x = grid[e];
-    spec[static_cast<long long>(c0) * P + e] = make_float2(x.x * scale, x.y * scale);
+    const float2 x = *HND_G(&grid[e]);
+    *HND_G(&spec[static_cast<long long>(c0) * P + e]) = make_float2(x.x * scale, x.y * scale);
   }
 }
 
@@ -64,7 +64,7 @@ static __global__ void k_l1_spec_export(const float2* __restrict__ lib, float2* 
   for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < H * C;
        e += static_cast<long long>(gridDim.x) * blockDim.x) {
     const long long c = e / H, k = e % H;
-    nat[e] = lib[c * P + l1_pos(k, P0, P1, P2)];
+    *HND_G(&nat[e]) = *HND_G(&lib[c * P + l1_pos(k, P0, P1, P2)]);
   }
 }
 
@@ -78,12 +78,12 @@ static __global__ void k_l1_spec_import(const float2* __restrict__ nat, float2* 
                         static_cast<long long>(P0) * P1 * (r % P2);
     float2 s;
     if (k <= n) {
-      s = nat[c * pitch + k];
+      s = *HND_G(&nat[c * pitch + k]);
     } else {
-      s = nat[c * pitch + (P - k)];
+      s = *HND_G(&nat[c * pitch + (P - k)]);
       s.y = -s.y;
     }
-    lib[e] = make_float2(s.x * scale, s.y * scale);
+    *HND_G(&lib[e]) = make_float2(s.x * scale, s.y * scale);
   }
 }
 
@@ -194,8 +194,8 @@ __global__ void __launch_bounds__(kAT, 2) k_l1_pass(const L1PassArgs a) {
 #pragma unroll
       for (int s = 0; s < R1; ++s) {
         const long long j = g + s * G;
-        lo[s] = act ? base[j * S] : make_float2(0.f, 0.f);
-        hi[s] = act ? base[(j + N) * S] : make_float2(0.f, 0.f);
+        lo[s] = act ? *HND_G(&base[j * S]) : make_float2(0.f, 0.f);
+        hi[s] = act ? *HND_G(&base[(j + N) * S]) : make_float2(0.f, 0.f);
       }
       full_fwd<N>(lo, hi, x, g, buf, 0, t, 0u);
     } else {
@@ -203,8 +203,8 @@ __global__ void __launch_bounds__(kAT, 2) k_l1_pass(const L1PassArgs a) {
 #pragma unroll
       for (int s = 0; s < R1; ++s) {
         const long long f = spec_idx<N>(g, s);
-        const float2 e0 = act ? base[(2 * f) * S] : make_float2(0.f, 0.f);
-        const float2 e1 = act ? base[(2 * f + 1) * S] : make_float2(0.f, 0.f);
+        const float2 e0 = act ? *HND_G(&base[(2 * f) * S]) : make_float2(0.f, 0.f);
+        const float2 e1 = act ? *HND_G(&base[(2 * f + 1) * S]) : make_float2(0.f, 0.f);
         x[s] = {make_float2(e0.x, e1.x), make_float2(e0.y, e1.y)};
       }
     }
@@ -218,8 +218,8 @@ __global__ void __launch_bounds__(kAT, 2) k_l1_pass(const L1PassArgs a) {
         const float2 w0 = l1_w((2u * f) * i, invQ);
         const float2 w1 = cmul1(w0, wi);
         if (act) {
-          base[(2 * f) * S] = cmul1(make_float2(x[s].re.x, x[s].im.x), w0);
-          base[(2 * f + 1) * S] = cmul1(make_float2(x[s].re.y, x[s].im.y), w1);
+          *HND_G(&base[(2 * f) * S]) = cmul1(make_float2(x[s].re.x, x[s].im.x), w0);
+          *HND_G(&base[(2 * f + 1) * S]) = cmul1(make_float2(x[s].re.y, x[s].im.y), w1);
         }
       }
     } else if constexpr (KIND == kCenter) {
@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(kAT, 2) k_l1_pass(const L1PassArgs a) {
 #pragma unroll
       for (int s = 0; s < R1; ++s) {
         const long long f = spec_idx<N>(g, s);
-        float4 sv = act ? __ldg(reinterpret_cast<const float4*>(Sp + 2 * f)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 sv = act ? __ldg(HND_G(reinterpret_cast<const float4*>(Sp + 2 * f))) : make_float4(0.f, 0.f, 0.f, 0.f);
         sv.y *= a.sconj;
         sv.w *= a.sconj;
         const float2 y0 = cmul1(make_float2(x[s].re.x, x[s].im.x), make_float2(sv.x, sv.y));
@@ -248,8 +248,8 @@ __global__ void __launch_bounds__(kAT, 2) k_l1_pass(const L1PassArgs a) {
         const float2 w0 = l1_conj(l1_w(k * j, invQ));
         const float2 w1 = cmul1(w0, wk);
         if (act) {
-          base[j] = cmul1(lo[s], w0);
-          base[j + N] = cmul1(hi[s], w1);
+          *HND_G(&base[j]) = cmul1(lo[s], w0);
+          *HND_G(&base[j + N]) = cmul1(hi[s], w1);
         }
       }
     } else if constexpr (KIND == kInvMid) {
@@ -265,8 +265,8 @@ __global__ void __launch_bounds__(kAT, 2) k_l1_pass(const L1PassArgs a) {
         const float2 w0 = l1_conj(l1_w(k * (static_cast<unsigned>(j) * Su + i), invQ));
         const float2 w1 = cmul1(w0, wk);
         if (act) {
-          base[j * S] = cmul1(lo[s], w0);
-          base[(j + N) * S] = cmul1(hi[s], w1);
+          *HND_G(&base[j * S]) = cmul1(lo[s], w0);
+          *HND_G(&base[(j + N) * S]) = cmul1(hi[s], w1);
         }
       }
     } else {

@@ -21,6 +21,7 @@ namespace hnd2 {
 namespace cg = cooperative_groups;
 
 constexpr int kTM = 256;          // threads per CTA in the multi-pass kernels
+
 constexpr int kWM = kTM / 32;
 
 // Barrier over the kTM task threads (named barrier 1).  In the stage kernels
@@ -36,6 +37,16 @@ __device__ __forceinline__ void task_sync() { asm volatile("bar.sync 1, %0;" ::"
 // launch without the programmatic-serialization attribute.
 __device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// ------------------------------------------------------ workspace access
+// The wave workspace (packed row spectra) bypasses L1: it is written by one
+// stage kernel and read by the next.  (An L2 evict-last policy on these
+// accesses, to keep a wave resident while the activations stream past, was
+// measured 2% slower on the 256^2 grid and is not used.)
+__device__ __forceinline__ float2 zt_ld(const float2* p) { return __ldcg(HND_G(p)); }
+__device__ __forceinline__ float4 zt_ld(const float4* p) { return __ldcg(HND_G(p)); }
+__device__ __forceinline__ void zt_st(float2* p, float2 v) { __stcg(HND_G(p), v); }
+__device__ __forceinline__ void zt_st(float4* p, float4 v) { __stcg(HND_G(p), v); }
 
 // Row pair rp = rows (ra, ra + ps): 2D pairs row r with r + n0/2 (ps = n0/2),
 // 3D pairs neighbouring rows (ps = 1).
@@ -79,9 +90,9 @@ __device__ __forceinline__ void tile_from_ws(float2* tile, const float2* __restr
     const int kk = e / RPB, rl = e % RPB;
     const float2* src = zt + static_cast<long long>(kk) * rp_total + rpb + rl;
     if (rl + 1 < nrp) {
-      v[i] = __ldcg(reinterpret_cast<const float4*>(src));
+      v[i] = zt_ld(reinterpret_cast<const float4*>(src));
     } else {
-      const float2 a = rl < nrp ? __ldcg(src) : make_float2(0.f, 0.f);
+      const float2 a = rl < nrp ? zt_ld(src) : make_float2(0.f, 0.f);
       v[i] = make_float4(a.x, a.y, 0.f, 0.f);
     }
   }
@@ -91,10 +102,10 @@ __device__ __forceinline__ void tile_from_ws(float2* tile, const float2* __restr
     const int kk = e / RPB, rl = e % RPB;
     float2* t = tile + R::row(kk) + rl;
     if constexpr (R::TS % 2 == 0) {
-      *reinterpret_cast<float4*>(t) = v[i];
+      *HND_S(reinterpret_cast<float4*>(t)) = v[i];
     } else {
-      t[0] = make_float2(v[i].x, v[i].y);
-      t[1] = make_float2(v[i].z, v[i].w);
+      *HND_S(&t[0]) = make_float2(v[i].x, v[i].y);
+      *HND_S(&t[1]) = make_float2(v[i].z, v[i].w);
     }
   }
 }
@@ -113,16 +124,16 @@ __device__ __forceinline__ void tile_to_ws(const float2* tile, float2* __restric
     const float2* t = tile + R::row(kk) + rl;
     float2 a, b;
     if constexpr (R::TS % 2 == 0) {
-      const float4 ab = *reinterpret_cast<const float4*>(t);
+      const float4 ab = *HND_S(reinterpret_cast<const float4*>(t));
       a = make_float2(ab.x, ab.y), b = make_float2(ab.z, ab.w);
     } else {
-      a = t[0], b = t[1];
+      a = *HND_S(&t[0]), b = *HND_S(&t[1]);
     }
     float2* dst = zt + static_cast<long long>(kk) * rp_total + rpb + rl;
     if (rl + 1 < nrp) {
-      __stcg(reinterpret_cast<float4*>(dst), make_float4(a.x, a.y, b.x, b.y));
+      zt_st(reinterpret_cast<float4*>(dst), make_float4(a.x, a.y, b.x, b.y));
     } else if (rl < nrp) {
-      __stcg(dst, a);
+      zt_st(dst, a);
     }
   }
 }
@@ -170,8 +181,8 @@ __device__ __forceinline__ void rowfwd_task(const Tabs<NL> t, unsigned char* wor
 #pragma unroll
       for (int s = 0; s < R1; ++s) {
         const int kk = 2 * spec_idx<NL>(g, s);
-        tile[R::row(kk) + rl_] = make_float2(xx[s].re.x, xx[s].im.x);
-        tile[R::row(kk + 1) + rl_] = make_float2(xx[s].re.y, xx[s].im.y);
+        *HND_S(&tile[R::row(kk) + rl_]) = make_float2(xx[s].re.x, xx[s].im.x);
+        *HND_S(&tile[R::row(kk + 1) + rl_]) = make_float2(xx[s].re.y, xx[s].im.y);
       }
     };
     if constexpr (ROUNDS > 1) put(keep, warp * PPW + pen);
@@ -225,7 +236,7 @@ __device__ __forceinline__ void rowinv_task(const Tabs<NL> t, unsigned char* wor
 #pragma unroll
     for (int s = 0; s < R1; ++s) {
       const int kk = 2 * spec_idx<NL>(g, s);
-      const float2 e = tile[R::row(kk) + rl], d = tile[R::row(kk + 1) + rl];
+      const float2 e = *HND_S(&tile[R::row(kk) + rl]), d = *HND_S(&tile[R::row(kk + 1) + rl]);
       xin[round][s] = {make_float2(e.x, d.x), make_float2(e.y, d.y)};
     }
   }
@@ -313,8 +324,8 @@ __device__ __forceinline__ void mid1_unit(const Tabs<N0> t, float4* buf, float2*
     const int rp = g + s * G;
     float2 z1 = make_float2(0.f, 0.f), z2 = z1;
     if (act) {
-      z1 = __ldcg(zt + static_cast<long long>(kx) * RP + rp);
-      z2 = __ldcg(zt + static_cast<long long>(kxm) * RP + rp);
+      z1 = zt_ld(zt + static_cast<long long>(kx) * RP + rp);
+      z2 = zt_ld(zt + static_cast<long long>(kxm) * RP + rp);
     }
     if (cu == 0) {
       z[s] = make_float2(z1.x, z2.x);
@@ -332,9 +343,9 @@ __device__ __forceinline__ void mid1_unit(const Tabs<N0> t, float4* buf, float2*
 #pragma unroll
     for (int s = 0; s < R1; ++s) {
 #if HND_MID1_PREFETCH == 2
-      asm volatile("prefetch.global.L1 [%0];" ::"l"(su + s * G + g));
+      if (HND_RANGE_OK(su + s * G + g, 16)) asm volatile("prefetch.global.L1 [%0];" ::"l"(su + s * G + g));
 #else
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(su + s * G + g));
+      if (HND_RANGE_OK(su + s * G + g, 16)) asm volatile("prefetch.global.L2 [%0];" ::"l"(su + s * G + g));
 #endif
     }
   }
@@ -346,8 +357,8 @@ __device__ __forceinline__ void mid1_unit(const Tabs<N0> t, float4* buf, float2*
     fetch_partner<N0>(x, xp, g, buf, 0, 0u);
 #pragma unroll
     for (int s = 0; s < R1; ++s) {
-      float4 S = act ? __ldg(su + s * G + g) : make_float4(0.f, 0.f, 0.f, 0.f);
-      float4 Bc = (cu == 0) ? __ldg(sp + N0 + s * G + g) : make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 S = act ? __ldg(HND_G(su + s * G + g)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 Bc = (cu == 0) ? __ldg(HND_G(sp + N0 + s * G + g)) : make_float4(0.f, 0.f, 0.f, 0.f);
       S.z *= sgn, S.w *= sgn, Bc.z *= sgn, Bc.w *= sgn;     // sgn = -1: conjugate spectrum (adjoint)
       const cp a = cmulp(x[s], make_float2(S.x, S.y), make_float2(S.z, S.w));
       const cp xc = {xp[s].re, make_float2(-xp[s].im.x, -xp[s].im.y)};
@@ -358,7 +369,7 @@ __device__ __forceinline__ void mid1_unit(const Tabs<N0> t, float4* buf, float2*
     if (act) {
 #pragma unroll
       for (int s = 0; s < R1; ++s) {
-        const float4 S = __ldg(su + s * G + g);
+        const float4 S = __ldg(HND_G(su + s * G + g));
         x[s] = cmulp(x[s], make_float2(S.x, S.y), make_float2(sgn * S.z, sgn * S.w));
       }
     }
@@ -371,20 +382,27 @@ __device__ __forceinline__ void mid1_unit(const Tabs<N0> t, float4* buf, float2*
       const int rp = g + s * G;
       const float2 ya = o[s], yb = o[s + HS];
       if (cu == 0) {
-        zt[rp] = make_float2(ya.x, yb.x);
-        zt[static_cast<long long>(N1) * RP + rp] = make_float2(ya.y, yb.y);
+        zt_st(zt + rp, make_float2(ya.x, yb.x));
+        zt_st(zt + static_cast<long long>(N1) * RP + rp, make_float2(ya.y, yb.y));
       } else {
-        zt[static_cast<long long>(kx) * RP + rp] = pack_pos(ya, yb);
-        zt[static_cast<long long>(kxm) * RP + rp] = pack_neg(ya, yb);
+        zt_st(zt + static_cast<long long>(kx) * RP + rp, pack_pos(ya, yb));
+        zt_st(zt + static_cast<long long>(kxm) * RP + rp, pack_neg(ya, yb));
       }
     }
   }
 }
 
 // The DC/Nyquist warp's path, kept out of line so that its extra registers
-// do not weigh on the common path.
+// do not weigh on the common path.  (The checked build, with relocatable
+// device code, keeps it inline: an out-of-line function there gets its own
+// register budget, above the kernel's.)
+#ifdef HYENA_ND_BOUNDS
+#define HND_OUT_OF_LINE __forceinline__
+#else
+#define HND_OUT_OF_LINE __noinline__
+#endif
 template <int N0>
-__device__ __noinline__ void mid1_unit_gen(const Tabs<N0> t, float4* buf, float2* __restrict__ zt,
+__device__ HND_OUT_OF_LINE void mid1_unit_gen(const Tabs<N0> t, float4* buf, float2* __restrict__ zt,
                                            const float4* __restrict__ sp, int N1, int cu, int g, float sgn) {
   mid1_unit<N0, true>(t, buf, zt, sp, N1, cu, g, sgn);
 }
@@ -448,8 +466,8 @@ __device__ __forceinline__ void slab_rows_in(const float2* __restrict__ zt, long
   for (int s = 0; s < R1; ++s) {
     const int yy = g + s * G;
     const long long rp = (static_cast<long long>(z) * N1 + yy) >> 1;
-    const float2 z1 = __ldcg(zt + kx * RPn + rp);
-    const float2 z2 = self_conj ? z1 : __ldcg(zt + kxm * RPn + rp);
+    const float2 z1 = zt_ld(zt + kx * RPn + rp);
+    const float2 z2 = self_conj ? z1 : zt_ld(zt + kxm * RPn + rp);
     x[s] = (yy & 1) ? unpack_b(z1, z2) : unpack_a(z1, z2);
   }
 }
@@ -474,10 +492,10 @@ __device__ __forceinline__ void slab_rows_out(float2* __restrict__ zt, long long
     const float2 ya = odd ? oth : own, yb = odd ? own : oth;
     if (!act) continue;
     if (self_conj) {
-      if (!odd) zt[kx * RPn + rp] = make_float2(ya.x, yb.x);
+      if (!odd) zt_st(zt + kx * RPn + rp, make_float2(ya.x, yb.x));
     } else {
-      if (!odd) zt[kx * RPn + rp] = pack_pos(ya, yb);
-      else zt[kxm * RPn + rp] = pack_neg(ya, yb);
+      if (!odd) zt_st(zt + kx * RPn + rp, pack_pos(ya, yb));
+      else zt_st(zt + kxm * RPn + rp, pack_neg(ya, yb));
     }
   }
 }
@@ -520,10 +538,10 @@ __device__ __forceinline__ void mid2_task(const Tabs<N0> t0, const Tabs<N1> t1, 
         for (int s = 0; s < R1; ++s) {
           const int f = spec_idx<N1>(g, s);
           if (HALF) {
-            F[f * FS + z] = h == 0 ? make_float2(x[s].re.x, x[s].im.x) : make_float2(x[s].re.y, x[s].im.y);
+            *HND_S(&F[f * FS + z]) = h == 0 ? make_float2(x[s].re.x, x[s].im.x) : make_float2(x[s].re.y, x[s].im.y);
           } else {
-            F[(2 * f) * FS + z] = make_float2(x[s].re.x, x[s].im.x);
-            F[(2 * f + 1) * FS + z] = make_float2(x[s].re.y, x[s].im.y);
+            *HND_S(&F[(2 * f) * FS + z]) = make_float2(x[s].re.x, x[s].im.x);
+            *HND_S(&F[(2 * f + 1) * FS + z]) = make_float2(x[s].re.y, x[s].im.y);
           }
         }
       }
@@ -545,17 +563,17 @@ __device__ __forceinline__ void mid2_task(const Tabs<N0> t0, const Tabs<N1> t1, 
       float4 S[NPF];
       if (R0 == 8 && act) {
 #pragma unroll
-        for (int s = 0; s < NPF; ++s) S[s] = __ldg(su + s * G0 + g);
+        for (int s = 0; s < NPF; ++s) S[s] = __ldg(HND_G(su + s * G0 + g));
       }
       float2 in[R0];
 #pragma unroll
-      for (int s = 0; s < R0; ++s) in[s] = act ? F[kyl * FS + g + s * G0] : make_float2(0.f, 0.f);
+      for (int s = 0; s < R0; ++s) in[s] = act ? *HND_S(&F[kyl * FS + g + s * G0]) : make_float2(0.f, 0.f);
       cp x[R0];
       padded_fwd<N0>(in, x, g, buf, 0, t0, 0u);
       if (act) {
 #pragma unroll
         for (int s = 0; s < R0; ++s) {
-          const float4 Sv = (R0 == 8) ? S[s % NPF] : __ldg(su + s * G0 + g);
+          const float4 Sv = (R0 == 8) ? S[s % NPF] : __ldg(HND_G(su + s * G0 + g));
           x[s] = cmulp(x[s], make_float2(Sv.x, Sv.y), make_float2(sgn * Sv.z, sgn * Sv.w));
         }
       }
@@ -563,7 +581,7 @@ __device__ __forceinline__ void mid2_task(const Tabs<N0> t0, const Tabs<N1> t1, 
       padded_inv<N0>(x, o, g, buf, 0, t0, 0u);
       if (act) {
 #pragma unroll
-        for (int s = 0; s < R0; ++s) F[kyl * FS + g + s * G0] = o[s];
+        for (int s = 0; s < R0; ++s) *HND_S(&F[kyl * FS + g + s * G0]) = o[s];
       }
     }
   }
@@ -596,11 +614,13 @@ __device__ __forceinline__ void mid2_task(const Tabs<N0> t0, const Tabs<N1> t1, 
         float2 e = make_float2(0.f, 0.f), d = e;
         if (act) {
           if (HALF) {
-            e = Fe[f * FS + z];
-            d = Fo[f * FS + z];
+            if (HND_RANGE_OK(&F[f * FS + z], sizeof(float2))) {
+              e = Fe[f * FS + z];
+              d = Fo[f * FS + z];
+            }
           } else {
-            e = F[(2 * f) * FS + z];
-            d = F[(2 * f + 1) * FS + z];
+            e = *HND_S(&F[(2 * f) * FS + z]);
+            d = *HND_S(&F[(2 * f + 1) * FS + z]);
           }
         }
         x[s] = {make_float2(e.x, d.x), make_float2(e.y, d.y)};
@@ -682,9 +702,9 @@ static __global__ void k_spec3_in(const float2* __restrict__ nat, float4* __rest
     const int ky = static_cast<int>(r2 / n0), m = static_cast<int>(r2 % n0);
     const int f = spec_idx_gen(n0, m % G, m / G);
     const float2* src = nat + c * src_per;
-    const float2 s0 = src[((2LL * f) * (2 * n1) + ky) * pitch + kx];
-    const float2 s1 = src[((2LL * f + 1) * (2 * n1) + ky) * pitch + kx];
-    out[e] = make_float4(scale * s0.x, scale * s1.x, scale * s0.y, scale * s1.y);
+    const float2 s0 = *HND_G(&src[((2LL * f) * (2 * n1) + ky) * pitch + kx]);
+    const float2 s1 = *HND_G(&src[((2LL * f + 1) * (2 * n1) + ky) * pitch + kx]);
+    *HND_G(&out[e]) = make_float4(scale * s0.x, scale * s1.x, scale * s0.y, scale * s1.y);
   }
 }
 
@@ -700,9 +720,9 @@ static __global__ void k_spec3_out(const float4* __restrict__ lib, float2* __res
     const int ky = static_cast<int>(r2 / n0), m = static_cast<int>(r2 % n0);
     const int f = spec_idx_gen(n0, m % G, m / G);
     float2* dst = nat + c * per * 2;
-    const float4 v = lib[e];
-    dst[((2LL * f) * (2 * n1) + ky) * (n2 + 1) + kx] = make_float2(v.x, v.z);
-    dst[((2LL * f + 1) * (2 * n1) + ky) * (n2 + 1) + kx] = make_float2(v.y, v.w);
+    const float4 v = *HND_G(&lib[e]);
+    *HND_G(&dst[((2LL * f) * (2 * n1) + ky) * (n2 + 1) + kx]) = make_float2(v.x, v.z);
+    *HND_G(&dst[((2LL * f + 1) * (2 * n1) + ky) * (n2 + 1) + kx]) = make_float2(v.y, v.w);
   }
 }
 

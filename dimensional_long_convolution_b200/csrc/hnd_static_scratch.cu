@@ -5,25 +5,33 @@
 // interface passes only input and output buffers, or an application that
 // reserves every byte of device memory at start-up and forbids allocations
 // afterwards.  This entry point serves them.  The only scratch it needs (the
-// packed row spectra of the multi-pass tiers) lives in a fixed array that is
-// part of the library's device image, so nothing is allocated per call.
+// packed row spectra of the multi-pass tiers, the split grids of the long 1D
+// tier) lives in a fixed array that is part of the library's device image, so
+// nothing is allocated per call.
 //
 // Properties a caller must know:
-//  * The array holds kStaticScratchBytes (16 MiB).  Every GPU that loads the
+//  * The array holds a 256-byte control area (the device status word) and
+//    then kStaticScratchBytes (16 MiB) of scratch.  Every GPU that loads the
 //    library keeps it until the process exits.
-//  * Problems whose single (b, c) volume needs more intermediate space than
-//    that (8 bytes per voxel; for example a 128 x 128 x 256 volume) are
+//  * Problems whose single (b, c) volume needs more scratch than that (8
+//    bytes per voxel in the multi-pass tiers, for example a 128 x 128 x 256
+//    volume; 16 bytes per token in the long 1D tier, so n > 2^20) are
 //    rejected with HYENA_ND_ERR_WORKSPACE_TOO_SMALL before anything runs.
 //  * The first call on a device looks up the array's device address (once
 //    per device, with that device current).  Make that first call before any
 //    stream capture.
 //  * All calls share the one array, and it keeps whatever the previous call
 //    left there.  Each call writes every intermediate it later reads, so
-//    nothing needs to start at zero.  Two calls whose kernels overlap on the
-//    GPU (different streams, or different host threads on one device) race on
-//    the array: serialise them.
+//    nothing needs to start at zero; the status word starts at zero when the
+//    library loads and is cleared only by hyena_nd_device_status(NULL, ...).
+//    Two calls whose kernels overlap on the GPU (different streams, or
+//    different host threads on one device) race on the array: serialise them.
+//  * Device-side errors (a bounded wait of the fused 2D kernel that gives up)
+//    are recorded in the array's status word; hyena_nd_device_status with a
+//    null workspace pointer reads and clears it.
 //  * Nothing here calls cudaMalloc, cudaFree or any allocating routine.
 #include "hyena_nd.h"
+#include "hnd_bounds.cuh"
 #include "hnd_launch.h"
 
 #include <cuda_runtime.h>
@@ -40,11 +48,12 @@ cudaError_t launch_fused2d_bf16(const ConvArgs& a);
 namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(16) << 20;
+constexpr size_t kStaticControlBytes = 256;      // status word + padding, ahead of the scratch
 
-// The scratch itself.  Host code must not pass this name to a kernel: on the
+// The array itself.  Host code must not pass this name to a kernel: on the
 // host it is only a stand-in for the symbol.  Its device address comes from
 // cudaGetSymbolAddress below.
-static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticControlBytes + kStaticScratchBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
@@ -67,6 +76,8 @@ cudaError_t scratch_address(void** out) {
   return cudaSuccess;
 }
 
+constexpr long long kLong1DMax = 1LL << 26;    // the longest 1D grid of the library
+
 bool pow2_in(long long x, long long lo, long long hi) { return x >= lo && x <= hi && (x & (x - 1)) == 0; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool overlaps(const void* a, const void* b, size_t n) {
@@ -75,6 +86,16 @@ bool overlaps(const void* a, const void* b, size_t n) {
 }
 
 }  // namespace
+
+namespace hnd {
+cudaError_t static_status_word(int** out) {
+  void* base = nullptr;
+  const cudaError_t e = scratch_address(&base);
+  if (e != cudaSuccess) return e;
+  *out = static_cast<int*>(base);
+  return cudaSuccess;
+}
+}  // namespace hnd
 
 extern "C" HYENA_ND_API hyena_nd_status hyena_nd_fftconv_batched_static(
     const hyena_nd_problem* p, const void* q, const void* k, const void* v, const void* spectrum,
@@ -87,7 +108,7 @@ extern "C" HYENA_ND_API hyena_nd_status hyena_nd_fftconv_batched_static(
     if (p->n[a] < 1) return HYENA_ND_ERR_INVALID_ARG;
   if (p->circular != 0 && p->circular != 1) return HYENA_ND_ERR_INVALID_ARG;
   for (int a = 0; a < p->ndim; ++a)
-    if (!pow2_in(p->n[a], 8, 256)) return HYENA_ND_ERR_UNSUPPORTED;
+    if (!pow2_in(p->n[a], 8, p->ndim == 1 ? kLong1DMax : 256)) return HYENA_ND_ERR_UNSUPPORTED;
   if (p->ndim == 3 && (p->n[0] > 128 || p->n[1] > 128)) return HYENA_ND_ERR_UNSUPPORTED;
   if (p->B > INT_MAX / p->C) return HYENA_ND_ERR_UNSUPPORTED;
   if (!q || !k || !v || !spectrum || !y) return HYENA_ND_ERR_INVALID_ARG;
@@ -107,9 +128,15 @@ extern "C" HYENA_ND_API hyena_nd_status hyena_nd_fftconv_batched_static(
   if (overlaps(y, q, act_bytes) || overlaps(y, k, act_bytes) || overlaps(y, v, act_bytes))
     return HYENA_ND_ERR_INVALID_ARG;
 
-  const bool fused = p->ndim == 1 || hnd::fused_2d(p->ndim, n);
-  const size_t per_pair = static_cast<size_t>(8) * static_cast<size_t>(L);
+  const bool long1d = p->ndim == 1 && n[0] > 256;
+  const bool fused = (p->ndim == 1 && !long1d) || hnd::fused_2d(p->ndim, n);
+  // scratch per (b, c) volume: packed row spectra (multi-pass) or the padded
+  // split grid (long 1D)
+  const size_t per_pair = static_cast<size_t>(long1d ? 16 : 8) * static_cast<size_t>(L);
   if (!fused && per_pair > kStaticScratchBytes) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
+
+  void* base = nullptr;
+  if (scratch_address(&base) != cudaSuccess) return HYENA_ND_ERR_CUDA;
 
   hnd::ConvArgs a;
   a.q = q;
@@ -124,21 +151,36 @@ extern "C" HYENA_ND_API hyena_nd_status hyena_nd_fftconv_batched_static(
   a.ndim = p->ndim;
   for (int i = 0; i < 3; ++i) a.n[i] = n[i];
   a.stream = static_cast<cudaStream_t>(cuda_stream);
+  a.status = static_cast<int*>(base);
+  float2* zt = reinterpret_cast<float2*>(static_cast<unsigned char*>(base) + kStaticControlBytes);
+
+  hnd::BoundsList bl;
+  for (const void* ptr : {q, k, v, static_cast<const void*>(y)}) bl.add(ptr, act_bytes);
+  long long spec_per = 1;     // complex values per channel spectrum (library order)
+  if (p->ndim == 1) spec_per = long1d ? 2LL * n[0] : n[0] + 1LL;
+  else if (p->ndim == 2) spec_per = (n[1] + 1LL) * 2 * n[0];
+  else spec_per = (n[2] + 1LL) * 4 * n[0] * n[1];
+  const size_t spec_bytes = static_cast<size_t>(spec_per) * 8 * static_cast<size_t>(p->C);
+  bl.add(spectrum, spectrum_batch_stride > 0
+                       ? static_cast<size_t>(p->B - 1) * static_cast<size_t>(spectrum_batch_stride) + spec_bytes
+                       : spec_bytes);
+  bl.add(base, kStaticControlBytes + kStaticScratchBytes);
+  if (hnd::bounds_register(bl, a.status, a.stream) != cudaSuccess) return HYENA_ND_ERR_CUDA;
 
   cudaError_t e = cudaSuccess;
-  if (p->ndim == 1) {
+  int launches = 0;
+  const long long pairs = p->B * p->C;
+  if (long1d) {
+    const long long wave = hnd::balanced_wave(pairs, p->B, per_pair, kStaticScratchBytes, false);
+    e = hnd::launch_long1d(a, zt, wave, &launches);
+  } else if (p->ndim == 1) {
     e = hnd::launch_rows1d(a);
+    launches = 1;
   } else if (fused) {
     e = bf16 ? hnd::launch_fused2d_bf16(a) : hnd::launch_fused2d_f32(a);
+    launches = 1;
   } else {
-    void* base = nullptr;
-    e = scratch_address(&base);
-    if (e != cudaSuccess) return HYENA_ND_ERR_CUDA;
-    float2* zt = static_cast<float2*>(base);
-    const long long pairs = p->B * p->C;
-    long long wave = static_cast<long long>(kStaticScratchBytes / per_pair);
-    if (wave > pairs) wave = pairs;
-    if (wave >= p->B) wave -= wave % p->B;
+    const long long wave = hnd::balanced_wave(pairs, p->B, per_pair, kStaticScratchBytes, true);
     const int nl = n[p->ndim - 1];
     const int rp_total = static_cast<int>(L / nl / 2);
     for (long long ord0 = 0; ord0 < pairs && e == cudaSuccess; ord0 += wave) {
@@ -146,7 +188,10 @@ extern "C" HYENA_ND_API hyena_nd_status hyena_nd_fftconv_batched_static(
       e = hnd::launch_rowfwd(a, nl, zt, ord0, np, rp_total);
       if (e == cudaSuccess) e = p->ndim == 2 ? hnd::launch_mid1(a, zt, ord0, np) : hnd::launch_mid2(a, zt, ord0, np);
       if (e == cudaSuccess) e = hnd::launch_rowinv(a, nl, zt, ord0, np, rp_total);
+      launches += 3;
     }
   }
-  return e == cudaSuccess ? HYENA_ND_OK : HYENA_ND_ERR_CUDA;
+  if (e != cudaSuccess) return HYENA_ND_ERR_CUDA;
+  hnd::note_launches(launches);
+  return HYENA_ND_OK;
 }

@@ -30,9 +30,16 @@ ERR_DEVICE_BOUNDS = 7
 F32 = 0
 BF16 = 1
 
+# calls that use a workspace (hyena_nd_workspace_bytes_for)
+CALL_ALL = 0
+CALL_CONV = 1
+CALL_FILTER = 2
+CALL_KERNEL_GRAD = 3
+
 EXPORTED = (
     "hyena_nd_spectrum_bytes",
     "hyena_nd_workspace_bytes",
+    "hyena_nd_workspace_bytes_for",
     "hyena_nd_workspace_init",
     "hyena_nd_filter_spectrum",
     "hyena_nd_filter_spectrum_film",
@@ -67,6 +74,7 @@ class PlanInfo(ctypes.Structure):
         ("kgrad_chunk", ctypes.c_int),
         ("workspace_bytes", ctypes.c_size_t),
         ("spectrum_bytes", ctypes.c_size_t),
+        ("streams", ctypes.c_int),
     ]
 
 
@@ -117,6 +125,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     sigs = {
         "hyena_nd_spectrum_bytes": (sz, [P]),
         "hyena_nd_workspace_bytes": (sz, [P]),
+        "hyena_nd_workspace_bytes_for": (ctypes.c_size_t, [P, ctypes.c_int]),
         "hyena_nd_workspace_init": (ctypes.c_int, [vp, sz, vp]),
         "hyena_nd_filter_spectrum": (ctypes.c_int, [P, ctypes.POINTER(Filter), vp, vp, sz, vp]),
         "hyena_nd_filter_spectrum_film": (ctypes.c_int, [P, ctypes.POINTER(Filter), vp, vp, vp, i64, vp, sz, vp]),
@@ -157,6 +166,10 @@ def spectrum_bytes(p: Problem) -> int:
 
 def workspace_bytes(p: Problem) -> int:
     return int(load().hyena_nd_workspace_bytes(ctypes.byref(p)))
+
+
+def workspace_bytes_for(p: Problem, call: int) -> int:
+    return int(load().hyena_nd_workspace_bytes_for(ctypes.byref(p), int(call)))
 
 
 def workspace_init(ws: int, ws_bytes: int, stream: int = 0) -> int:
@@ -227,7 +240,8 @@ def plan_info(p: Problem) -> dict:
     return {"tier": TIERS.get(info.tier, str(info.tier)), "wave": info.wave, "waves": info.waves,
             "launches": info.launches, "split_levels": info.split_levels, "split": list(info.split),
             "filter_chunk": info.filter_chunk, "kgrad_chunk": info.kgrad_chunk,
-            "workspace_bytes": info.workspace_bytes, "spectrum_bytes": info.spectrum_bytes}
+            "workspace_bytes": info.workspace_bytes, "spectrum_bytes": info.spectrum_bytes,
+            "streams": info.streams}
 
 
 def status_string(code: int) -> str:

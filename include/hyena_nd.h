@@ -22,6 +22,12 @@
  *     or frees.  Every call is asynchronous on the given CUDA stream
  *     (cudaStream_t passed as void*; NULL = legacy default stream) and
  *     performs no host synchronisation, except hyena_nd_device_status.
+ *     Convolutions on the multi-pass tiers with several waves run alternate
+ *     waves on a side stream the library creates per device on first use:
+ *     it is forked from the caller's stream with an event and joined back to
+ *     it before the call returns, so the call stays ordered on the caller's
+ *     stream (and may be captured into a CUDA graph with it).  Calls from
+ *     several host threads serialise their enqueue on that side stream.
  *   * Argument errors are detected on the host before anything is launched
  *     and returned synchronously.  A failed launch returns HYENA_ND_ERR_CUDA.
  *     Errors detected on the device are written to a status word held in the
@@ -131,6 +137,25 @@ HYENA_ND_API size_t hyena_nd_spectrum_bytes(const hyena_nd_problem* p);
  * consecutive calls on one stream. */
 HYENA_ND_API size_t hyena_nd_workspace_bytes(const hyena_nd_problem* p);
 
+/* The calls that use a workspace, for hyena_nd_workspace_bytes_for. */
+typedef enum {
+  HYENA_ND_CALL_ALL = 0,          /* every call: hyena_nd_workspace_bytes(p) */
+  HYENA_ND_CALL_CONV = 1,         /* hyena_nd_fftconv, _batched, _backward */
+  HYENA_ND_CALL_FILTER = 2,       /* hyena_nd_filter_spectrum, _film */
+  HYENA_ND_CALL_KERNEL_GRAD = 3   /* hyena_nd_kernel_grad */
+} hyena_nd_call;
+
+/* Workspace bytes that the calls of one kind need for problem `p` (a pure
+ * function of the descriptor, at least 256 bytes for the control area): the
+ * convolution calls need only their waves' intermediates (none on the
+ * single-launch tiers), the filter calls a channel chunk of grids and
+ * tables, the kernel gradient a chunk of its grids.  A caller that only runs
+ * convolutions can hold this much instead of hyena_nd_workspace_bytes(p);
+ * each call checks its own figure.  0 if `p` is invalid or unsupported or
+ * `call` is not one of the values above.  (A deployment convenience of this
+ * library; the pages only ask for a preallocated, deterministic workspace.) */
+HYENA_ND_API size_t hyena_nd_workspace_bytes_for(const hyena_nd_problem* p, hyena_nd_call call);
+
 /* Execution plan of a problem, as the calls below run it (host only, no
  * device work; a pure function of the descriptor). */
 typedef enum {
@@ -152,6 +177,8 @@ typedef struct {
   int kgrad_chunk;        /* channels per chunk of the kernel gradient */
   size_t workspace_bytes; /* hyena_nd_workspace_bytes(p) */
   size_t spectrum_bytes;  /* hyena_nd_spectrum_bytes(p) */
+  int streams;            /* multi-pass tiers: streams running alternate waves (the caller's and, for 2,
+                             a side stream of the library forked from and joined back to it); else 1 */
 } hyena_nd_plan_info;
 
 /* Fill `out` with the plan of `p`.  Errors: HYENA_ND_ERR_INVALID_ARG (null or
@@ -262,18 +289,25 @@ HYENA_ND_API hyena_nd_status hyena_nd_kernel_grad(const hyena_nd_problem* p, con
  * application that reserves all device memory at start-up and allows no
  * allocation afterwards.  (The HyenaND pages have no counterpart; this is a
  * deployment convenience of this library.)
- * Scratch: a fixed array of HYENA_ND_STATIC_SCRATCH_BYTES (16 MiB) inside the
- * library's device image, held by every GPU that loads the library until the
+ * Scratch: a fixed array inside the library's device image -- a 256-byte
+ * control area (the status word) followed by HYENA_ND_STATIC_SCRATCH_BYTES
+ * (16 MiB) of scratch -- held by every GPU that loads the library until the
  * process exits.  Nothing is allocated or freed by the call.
- *   * A problem whose single (b, c) volume needs more than that (8 bytes per
- *     voxel in the multi-pass tiers, e.g. a 128 x 128 x 256 volume) returns
- *     HYENA_ND_ERR_WORKSPACE_TOO_SMALL before anything is launched.
+ *   * A problem whose single (b, c) volume needs more scratch than that
+ *     (8 bytes per voxel in the multi-pass tiers, e.g. a 128 x 128 x 256
+ *     volume; 16 bytes per token in the long 1D tier, i.e. n > 2^20) returns
+ *     HYENA_ND_ERR_WORKSPACE_TOO_SMALL before anything is launched.  Every
+ *     other supported shape runs, on the same tier as the workspace call.
  *   * The first call on a device looks up the array's device address once;
  *     make that first call before any stream capture.
  *   * Every call shares the array and it keeps the previous call's contents
  *     (each call writes what it reads, so nothing has to start at zero).
  *     Calls whose kernels overlap on one GPU race on it: serialise them.
- *   * Device-side status words are not used by this call.
+ *   * Device-side errors (a bounded wait of the fused 2D kernel that gives
+ *     up) go to the array's status word, which is zero when the library loads
+ *     and stays set until hyena_nd_device_status(NULL, stream) reads and
+ *     clears it on the current device.
+ *   * hyena_nd_last_launch_count reports the call's kernel launches.
  * Other arguments and errors: as hyena_nd_fftconv_batched. */
 #define HYENA_ND_STATIC_SCRATCH_BYTES (16u << 20)
 HYENA_ND_API hyena_nd_status hyena_nd_fftconv_batched_static(const hyena_nd_problem* p, const void* q,
@@ -295,7 +329,9 @@ HYENA_ND_API hyena_nd_status hyena_nd_spectrum_export(const hyena_nd_problem* p,
 HYENA_ND_API hyena_nd_status hyena_nd_spectrum_import(const hyena_nd_problem* p, const void* natural_c64,
                                          void* spectrum, void* cuda_stream);
 
-/* Synchronise `stream`, then read and clear the device status word in `ws`.
+/* Synchronise `stream`, then read and clear the device status word in `ws`
+ * (a workspace), or, with ws == NULL, the status word of the fixed array of
+ * hyena_nd_fftconv_batched_static on the current device.
  * Returns HYENA_ND_OK, the recorded device error, or HYENA_ND_ERR_CUDA. */
 HYENA_ND_API hyena_nd_status hyena_nd_device_status(void* ws, void* cuda_stream);
 
@@ -309,8 +345,9 @@ HYENA_ND_API hyena_nd_status hyena_nd_debug_bounded_wait(void* ws, size_t ws_byt
 /* Human-readable name of a status code (static string). */
 HYENA_ND_API const char* hyena_nd_status_string(hyena_nd_status s);
 
-/* Number of kernels the most recent successful call to hyena_nd_fftconv or
- * hyena_nd_fftconv_batched on this host thread enqueued. */
+/* Number of kernels the most recent successful call to hyena_nd_fftconv,
+ * hyena_nd_fftconv_batched, hyena_nd_fftconv_batched_static or
+ * hyena_nd_fftconv_backward on this host thread enqueued. */
 HYENA_ND_API int hyena_nd_last_launch_count(void);
 
 #ifdef __cplusplus

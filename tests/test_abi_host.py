@@ -21,7 +21,7 @@ def _declared():
 def test_library_exports_every_declared_symbol():
     lib = H.load()
     names = _declared()
-    assert len(names) == len(H.EXPORTED) == 17
+    assert len(names) == len(H.EXPORTED) == 18
     assert set(names) == set(H.EXPORTED)
     for n in names:
         assert getattr(lib, n) is not None
@@ -93,7 +93,7 @@ def _call(p, q, k, v, s, y, ws, wsb, sbs=0):
 def test_invalid_arguments_are_rejected_before_launch():
     p = H.problem((64, 64), 2, 3)
     q, k, v, s, y, ws = _ptrs()
-    wsb = H.workspace_bytes(p)
+    wsb = H.workspace_bytes_for(p, H.CALL_CONV)
     assert _call(p, 0, k, v, s, y, ws, wsb) == H.ERR_INVALID_ARG
     assert _call(p, q, k, v, 0, y, ws, wsb) == H.ERR_INVALID_ARG
     assert _call(p, q, k, v, s, y, 0, wsb) == H.ERR_INVALID_ARG
@@ -114,7 +114,7 @@ def test_backward_arguments_are_rejected_before_launch():
     p = H.problem((64, 64), 2, 3)
     q, k, v, s, dy, ws = _ptrs()
     dq, dk, dv = (A + i * STEP for i in (6, 7, 8))
-    wsb = H.workspace_bytes(p)
+    wsb = H.workspace_bytes_for(p, H.CALL_CONV)
 
     def bwd(*args, sbs=0, wsb_=wsb, prob=p):
         a = dict(q=q, k=k, v=v, s=s, dy=dy, dq=dq, dk=dk, dv=dv, ws=ws)
@@ -182,10 +182,14 @@ def test_long_1d_spectrum_conversion_uses_the_natural_size():
     assert H.spectrum_export(p, A + nat16 - 16, A, 0) == H.ERR_INVALID_ARG
 
 
-def test_static_scratch_call_rejects_long_1d():
+def test_static_scratch_call_limits_long_1d():
+    """The no-allocation call runs long 1D grids while one volume's split grid
+    (16 bytes per token) fits its 16 MiB array: 2^21 tokens do not, and 2^27
+    is beyond every tier.  Both are refused on the host (fake pointers)."""
     q, k, v, s, y, ws = _ptrs()
-    p = H.problem((1024,), 1, 1)
-    assert H.fftconv_batched_static(p, q, k, v, s, 0, y, 0) == H.ERR_UNSUPPORTED
+    assert H.fftconv_batched_static(H.problem((1 << 21,), 1, 1), q, k, v, s, 0, y, 0) == \
+        H.ERR_WORKSPACE_TOO_SMALL
+    assert H.fftconv_batched_static(H.problem((1 << 27,), 1, 1), q, k, v, s, 0, y, 0) == H.ERR_UNSUPPORTED
 
 
 @pytest.mark.parametrize("i", range(5))
@@ -201,16 +205,17 @@ def test_workspace_stays_within_the_chunk_budgets(i):
     assert H.workspace_bytes(p) <= 256 + max(256 << 20, one) + 256 + tables
 
 
-@pytest.mark.parametrize("i,tier,waves,launches", [
-    (0, "fused_2d", 1, 1), (1, "fused_2d", 1, 1), (2, "multi_2d", 2, 6), (3, "multi_3d", 3, 9),
-    (4, "multi_3d", 6, 18)])
-def test_plan_info_of_the_benchmark_grids(i, tier, waves, launches):
+@pytest.mark.parametrize("i,tier,waves,launches,streams", [
+    (0, "fused_2d", 1, 1, 1), (1, "fused_2d", 1, 1, 1), (2, "multi_2d", 4, 12, 2), (3, "multi_3d", 8, 24, 2),
+    (4, "multi_3d", 16, 48, 2)])
+def test_plan_info_of_the_benchmark_grids(i, tier, waves, launches, streams):
     """The plan the calls run, read on the host: the launch counts are the
-    ones the GPU tests and the bench observe."""
+    ones the GPU tests and the bench observe; multi-pass grids with several
+    waves run alternate waves on two streams, each wave in 32 MiB."""
     wl = W.workload(i)
     p = H.problem(wl.dims, wl.B, wl.C, H.BF16 if wl.io_dtype == "bf16" else H.F32)
     info = H.plan_info(p)
-    assert (info["tier"], info["waves"], info["launches"]) == (tier, waves, launches)
+    assert (info["tier"], info["waves"], info["launches"], info["streams"]) == (tier, waves, launches, streams)
     assert info["workspace_bytes"] == H.workspace_bytes(p)
     assert info["spectrum_bytes"] == H.spectrum_bytes(p)
     if waves > 1:       # balanced waves of whole channels' samples
@@ -249,7 +254,7 @@ def test_single_volume_call_needs_b_and_c_of_one():
 def test_filter_arguments_are_checked():
     p = H.problem((32, 32), 1, 4)
     _, _, _, s, _, ws = _ptrs()
-    wsb = H.workspace_bytes(p)
+    wsb = H.workspace_bytes_for(p, H.CALL_FILTER)
     f = H.Filter()
     f.num_freqs, f.hidden = 8, 64
     f.W1 = f.b1 = f.W2 = f.b2 = f.alpha = A + 7 * STEP
@@ -274,7 +279,7 @@ def test_filter_arguments_are_checked():
 def test_film_filter_arguments_are_checked():
     p = H.problem((32, 32), 2, 4)
     _, _, _, s, _, ws = _ptrs()
-    wsb = H.workspace_bytes(p)
+    wsb = H.workspace_bytes_for(p, H.CALL_FILTER)
     sb = H.spectrum_bytes(p)
     f = H.Filter()
     f.num_freqs, f.hidden = 8, 64
@@ -300,8 +305,41 @@ def test_spectrum_conversion_checks():
 
 
 def test_status_and_debug_calls_check_arguments():
-    assert H.device_status(0, 0) == H.ERR_INVALID_ARG
+    # a null workspace names the no-allocation call's status word, which needs
+    # a device: without one the lookup fails as a CUDA error
+    assert H.device_status(0, 0) == H.ERR_CUDA
     assert H.device_status(A + 4, 0) == H.ERR_MISALIGNED
     assert H.workspace_init(A, 16, 0) == H.ERR_WORKSPACE_TOO_SMALL
     assert H.debug_bounded_wait(A, 4096, 0, 0) == H.ERR_INVALID_ARG
     assert H.debug_bounded_wait(A, 8, 100, 0) == H.ERR_WORKSPACE_TOO_SMALL
+
+
+@pytest.mark.parametrize("i", range(5))
+def test_workspace_bytes_per_call(i):
+    """Each call kind needs only its own scratch: the convolution calls their
+    waves (nothing beyond the control area on the single-launch tiers), the
+    filter and kernel-gradient calls their channel chunks; the largest of the
+    three is hyena_nd_workspace_bytes."""
+    wl = W.workload(i)
+    p = H.problem(wl.dims, wl.B, wl.C, H.BF16 if wl.io_dtype == "bf16" else H.F32)
+    conv, filt, kg = (H.workspace_bytes_for(p, c) for c in (H.CALL_CONV, H.CALL_FILTER, H.CALL_KERNEL_GRAD))
+    assert H.workspace_bytes_for(p, H.CALL_ALL) == H.workspace_bytes(p) == max(conv, filt, kg)
+    info = H.plan_info(p)
+    if info["tier"] == "fused_2d":
+        assert conv == 256
+    else:
+        per = 8 * wl.voxels * int(info["wave"])
+        assert conv == 256 + info["streams"] * ((per + 255) // 256 * 256)
+    assert H.workspace_bytes_for(p, 99) == 0
+
+
+def test_calls_check_their_own_workspace_size():
+    """Host-side rejects against each call's own figure (fake pointers: these
+    return before any launch)."""
+    q, k, v, s, y, ws = _ptrs()
+    p = H.problem((256, 256), 2, 128, H.BF16)
+    conv = H.workspace_bytes_for(p, H.CALL_CONV)
+    assert conv < H.workspace_bytes(p)
+    assert H.fftconv_batched(p, q, k, v, s, 0, y, ws, conv - 16, 0) == H.ERR_WORKSPACE_TOO_SMALL
+    kg = H.workspace_bytes_for(p, H.CALL_KERNEL_GRAD)
+    assert H.kernel_grad(p, q, k, v, s, y, ws, kg - 16, 0) == H.ERR_WORKSPACE_TOO_SMALL

@@ -67,7 +67,7 @@ def test_backward_matches_oracle(dims, B, C, dt):
 
 
 def test_backward_full_size_sampled():
-    """The 2D 256^2, B=2, C=128, bf16 workload (two waves per convolution):
+    """The 2D 256^2, B=2, C=128, bf16 workload (several waves per convolution):
     sampled outputs of all three gradients against direct sums."""
     wl = W.workload(2)
     inp = W.make_inputs(wl)
@@ -75,7 +75,7 @@ def test_backward_full_size_sampled():
     op = make_op(wl)
     set_filter(op, inp.filt)
     dq, dk, dv = _gpu_backward(op, inp, dy)
-    assert H.last_launch_count() == 12
+    assert H.last_launch_count() == 2 * H.plan_info(op.p)["launches"]
     chans = [0, 77, 127]
     pts = sample_points(wl, 10, seed=5, channels=chans)
     K = O.implicit_kernel(inp.filt, wl.dims, channels=chans)

@@ -6,7 +6,7 @@ Every output of every (b, c) volume is compared on the 2D 256^2 (B2, C128,
 bf16) and 3D 64^3 (B2, C64, fp32) grids; the 3D 128^3 grid (B1, C32, bf16) is
 compared on four whole volumes at the ends of its waves.  The backward (dq, dk,
 dv) and the kernel gradient are compared on 16 whole 256^2 volumes that span
-both waves of a convolution.  Tolerances: relative L2 <= 1e-4 (fp32 I/O) and
+every wave of a convolution.  Tolerances: relative L2 <= 1e-4 (fp32 I/O) and
 <= 1e-2 (bf16 I/O), over the whole tensor and over each volume on its own.
 
 The operation: HyenaND blog, section "HyenaND" (output equation); the arXiv
@@ -88,8 +88,8 @@ def test_full_grid_large_volume_wave_edges():
         _check_volumes(got[:, c:c + 1], want, TOL["bf16"], (wl.name, c))
 
 
-# Channels of the 256^2 grid whose 2 x 8 volumes span both waves of a
-# convolution (the waves hold channels 0..63 and 64..127).
+# Channels of the 256^2 grid whose 2 x 8 volumes span every wave of a
+# convolution (four waves of 32 channels: 0..31, 32..63, 64..95, 96..127).
 _BWD_CHANS = [0, 1, 31, 62, 63, 64, 65, 127]
 
 
@@ -115,7 +115,7 @@ def test_backward_full_volumes():
 
 
 def test_kernel_grad_full_channels():
-    """dK of 8 channels (16 volumes, both waves) at every offset."""
+    """dK of 8 channels (16 volumes) at every offset."""
     wl = W.workload(2)
     inp = W.make_inputs(wl)
     dy = W.make_inputs(wl, seed=wl.seed + 9).q

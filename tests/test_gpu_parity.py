@@ -235,26 +235,39 @@ def _check_sampled(wl, inp, got, chans, tol, npts=12):
     assert O.rel_l2(gv, want) <= tol
 
 
+def _wave_edge_channels(wl):
+    """Channels at the start and end of the first two waves and the last
+    channel, from the library's plan (volumes run in channel-major order)."""
+    info = H.plan_info(H.problem(wl.dims, wl.B, wl.C, H.BF16 if wl.io_dtype == "bf16" else H.F32))
+    w = int(info["wave"])
+    ords = [0, w - 1, w, 2 * w - 1, wl.B * wl.C - 1]
+    return info, sorted({o // wl.B for o in ords})
+
+
 def test_multi_wave_schedule_2d():
-    """More volumes (400 of 256^2) than one wave's workspace holds (192), so
-    three balanced waves of 134, 134 and 132 volumes run back to back."""
+    """More volumes (400 of 256^2) than one wave's workspace holds: seven
+    balanced waves of 58 volumes (the last 52) on two alternating streams."""
     dims = (256, 256)
     wl = W.custom(dims, 2, 200, io_dtype="bf16", seed=31)
+    info, chans = _wave_edge_channels(wl)
+    assert info["waves"] == 7 and info["streams"] == 2
     inp = W.make_inputs(wl)
     got, _ = run(inp)
-    assert H.last_launch_count() == 9
-    _check_sampled(wl, inp, got, [0, 66, 67, 133, 199], 1e-2)
+    assert H.last_launch_count() == info["launches"] == 21
+    _check_sampled(wl, inp, got, chans, 1e-2)
 
 
 def test_multi_wave_schedule_3d():
-    """100 volumes of 32x64x64 at 1 MiB of intermediate each run as two
-    balanced waves of 50."""
+    """100 volumes of 32x64x64 at 1 MiB of intermediate each run as four
+    balanced waves of 25 on two alternating streams."""
     dims = (32, 64, 64)
     wl = W.custom(dims, 1, 100, io_dtype="bf16", seed=37)
+    info, chans = _wave_edge_channels(wl)
+    assert info["waves"] == 4 and info["streams"] == 2
     inp = W.make_inputs(wl)
     got, _ = run(inp)
-    assert H.last_launch_count() == 6
-    _check_sampled(wl, inp, got, [0, 49, 50, 99], 1e-2)
+    assert H.last_launch_count() == info["launches"] == 12
+    _check_sampled(wl, inp, got, chans, 1e-2)
 
 
 def test_repeated_calls_on_one_workspace():
@@ -285,3 +298,36 @@ def test_bounded_wait_reports_timeout_and_recovers():
     # the context is still usable
     x = t.ones(16, device="cuda")
     assert float((x * 2).sum()) == 32.0
+
+
+def test_calls_run_in_their_own_workspace_size():
+    """The filter call in exactly hyena_nd_workspace_bytes_for(FILTER) bytes
+    and the convolution in exactly ..._for(CONV) bytes (several waves on two
+    streams), against the oracle."""
+    t = torch()
+    dims = (256, 256)
+    wl = W.custom(dims, 2, 70, io_dtype="bf16", seed=45)
+    inp = W.make_inputs(wl)
+    op = make_op(wl)
+    p = op.p
+    s = int(t.cuda.current_stream().cuda_stream)
+    wf = t.empty(H.workspace_bytes_for(p, H.CALL_FILTER), dtype=t.uint8, device="cuda")
+    wc = t.empty(H.workspace_bytes_for(p, H.CALL_CONV), dtype=t.uint8, device="cuda")
+    assert wc.numel() < op.ws_bytes
+    for w in (wf, wc):
+        assert H.workspace_init(w.data_ptr(), w.numel(), s) == H.OK
+    f = inp.filt
+    wts = [t.from_numpy(a).cuda() for a in (f.W1, f.b1, f.W2, f.b2, f.alpha)]
+    fl = H.Filter()
+    fl.num_freqs, fl.hidden = f.num_freqs, f.hidden
+    fl.W1, fl.b1, fl.W2, fl.b2, fl.alpha = (x.data_ptr() for x in wts)
+    fl.decay_scale, fl.window = f.decay_scale, 0
+    assert H.filter_spectrum(p, fl, op.spectrum.data_ptr(), wf.data_ptr(), wf.numel(), s) == H.OK
+    q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
+    y = t.empty_like(q)
+    assert H.fftconv_batched(p, q.data_ptr(), k.data_ptr(), v.data_ptr(), op.spectrum.data_ptr(), 0, y.data_ptr(),
+                             wc.data_ptr(), wc.numel(), s) == H.OK
+    assert H.plan_info(p)["waves"] > 1
+    t.cuda.synchronize()
+    assert H.device_status(wc.data_ptr(), s) == H.OK
+    _check_sampled(wl, inp, to_host(y), [0, 34, 35, 69], 1e-2)

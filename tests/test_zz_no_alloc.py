@@ -1,14 +1,22 @@
 """hyena_nd_fftconv_batched_static: the batched call for callers that cannot
-allocate device memory (no workspace argument; its scratch is a fixed 16 MiB
-array inside the library).  Its output must match the workspace-taking entry
-point within the parity tolerances, on two calls in a row (the second call
-finds the first call's leftovers in the shared array).  This file is collected
-last so a failure here never hides the rest of the suite."""
+allocate device memory -- a plugin interface that hands over only input and
+output buffers, or an application that reserves all device memory at
+start-up -- so there is no workspace argument; the call's scratch is a fixed
+16 MiB array inside the library.
+
+Checked here, through the C ABI: on two calls in a row (the second finds the
+first call's leftovers in the shared array) the output matches the
+workspace-taking entry point within the parity tolerances and the float64
+oracle within the same tolerances; repeated calls leave the device's free
+memory unchanged; the array's status word reads clear afterwards; and the
+launch count is reported.  This file is collected last, so a failure here
+never hides the rest of the suite."""
 import numpy as np
 import pytest
 
 from dimensional_long_convolution_b200 import hyena_nd as H
 from dimensional_long_convolution_b200 import workloads as W
+from oracle import hyena_nd_oracle as O
 
 TOL = {"f32": 1e-4, "bf16": 1e-2}
 
@@ -17,13 +25,19 @@ def _rel(a, b):
     return float(np.linalg.norm((a - b).ravel()) / max(np.linalg.norm(b.ravel()), 1e-300))
 
 
+def _static(op, q, k, v, y):
+    return H.fftconv_batched_static(op.p, q.data_ptr(), k.data_ptr(), v.data_ptr(), op.spectrum.data_ptr(), 0,
+                                    y.data_ptr(), op._stream())
+
+
 @pytest.mark.gpu
-@pytest.mark.parametrize("dims,B,C,dt", [
-    ((256, 256), 2, 40, "bf16"),     # multi-pass 2D: three waves through the fixed array
-    ((64, 64, 64), 1, 10, "f32"),    # multi-pass 3D: two waves
-    ((64, 64), 2, 3, "f32"),         # fused tier: needs no scratch at all
+@pytest.mark.parametrize("dims,B,C,dt,launches", [
+    ((256, 256), 2, 40, "bf16", 9),      # multi-pass 2D: three waves through the fixed array
+    ((64, 64, 64), 1, 10, "f32", 6),     # multi-pass 3D: two waves
+    ((64, 64), 2, 3, "f32", 1),          # fused 2D tier: no scratch, status word only
+    ((1024,), 2, 5, "f32", None),        # long 1D: split passes over the fixed array
 ])
-def test_static_scratch_matches_workspace_entry_point(dims, B, C, dt):
+def test_static_scratch_matches_workspace_entry_point(dims, B, C, dt, launches):
     from gpu_util import make_op, set_filter, to_dev, to_host, torch
     t = torch()
     wl = W.custom(dims, B, C, io_dtype=dt, seed=77)
@@ -33,15 +47,42 @@ def test_static_scratch_matches_workspace_entry_point(dims, B, C, dt):
     q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
     ref = to_host(op(q, k, v))
     t.cuda.synchronize()
+    want = O.reference_output(inp)
     for _ in range(2):
         y = t.empty_like(q)
-        st = H.fftconv_batched_static(op.p, q.data_ptr(), k.data_ptr(), v.data_ptr(), op.spectrum.data_ptr(), 0,
-                                      y.data_ptr(), op._stream())
+        st = _static(op, q, k, v, y)
         assert st == H.OK, H.status_string(st)
+        if launches is not None:
+            assert H.last_launch_count() == launches
         t.cuda.synchronize()
         got = to_host(y)
         assert np.all(np.isfinite(got))
         assert _rel(got, ref) <= TOL[dt]
+        assert O.rel_l2(got, want) <= TOL[dt]
+    assert H.device_status(0, op._stream()) == H.OK
+
+
+@pytest.mark.gpu
+def test_static_scratch_allocates_nothing():
+    """After the first calls (which load the kernels and look up the array),
+    further calls leave cudaMemGetInfo's free bytes exactly unchanged."""
+    from gpu_util import make_op, set_filter, to_dev, torch
+    t = torch()
+    wl = W.custom((256, 256), 2, 40, io_dtype="bf16", seed=78)
+    inp = W.make_inputs(wl)
+    op = make_op(wl)
+    set_filter(op, inp.filt)
+    q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
+    y = t.empty_like(q)
+    for _ in range(2):
+        assert _static(op, q, k, v, y) == H.OK
+    t.cuda.synchronize()
+    free0, _ = t.cuda.mem_get_info()
+    for _ in range(5):
+        assert _static(op, q, k, v, y) == H.OK
+    t.cuda.synchronize()
+    free1, _ = t.cuda.mem_get_info()
+    assert free1 == free0
 
 
 def test_static_scratch_rejects_volumes_beyond_its_size():
