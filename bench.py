@@ -517,7 +517,7 @@ def run_ours(args):
                      "issue_frac": pipes.get("issue_frac") if pipes else None,
                      "kernel": "step (%d launch%s per step: %s)" % (
                          launches, "" if launches == 1 else "es", kernel_desc.get(launches, "multi-pass waves")),
-                     "algorithmic_bytes_per_step": ub},
+                     "algorithmic_bytes_per_step": ub, "kernel_source_sha": kernel_source_sha()},
         "gpu_launches": int(launches * K),
         "clocks": clocks.summary(),
         "e2e": e2e,

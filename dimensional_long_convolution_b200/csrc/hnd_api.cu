@@ -49,9 +49,13 @@ cudaError_t side_stream(SideStream** out) {
   std::lock_guard<std::mutex> lk(mu);
   if (!per_dev[dev]) {
     SideStream* r = new SideStream;
-    if ((e = cudaStreamCreateWithFlags(&r->s, cudaStreamNonBlocking)) != cudaSuccess) return e;
-    for (cudaEvent_t* ev : {&r->fork, &r->stagger, &r->join})
-      if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+    for (int j = 1; j < SideStream::kMax; ++j)
+      if ((e = cudaStreamCreateWithFlags(&r->s[j], cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&r->fork, cudaEventDisableTiming)) != cudaSuccess) return e;
+    for (int j = 0; j < SideStream::kMax; ++j) {
+      if ((e = cudaEventCreateWithFlags(&r->stagger[j], cudaEventDisableTiming)) != cudaSuccess) return e;
+      if ((e = cudaEventCreateWithFlags(&r->join[j], cudaEventDisableTiming)) != cudaSuccess) return e;
+    }
     per_dev[dev] = r;
   }
   *out = per_dev[dev];
@@ -85,14 +89,16 @@ constexpr size_t kStatusBytes = 256;                  // status word + padding
 #define HND_WAVE_MB 64
 #endif
 #ifndef HND_STREAMS
-#define HND_STREAMS 2
+#define HND_STREAMS 3
 #endif
 // Multi-pass tiers: intermediates of the waves in flight, split over
-// HND_STREAMS streams that run alternate waves one stage apart.  Measured on
-// the 256^2, 64^3 and 128^3 grids: two streams with 64 MiB in all (32 MiB
-// waves) beat one stream with 96 MiB by 2-5%, and 128 or 192 MiB in all.
+// HND_STREAMS streams that run the waves round-robin, each one stage behind
+// the previous.  Measured on the 256^2, 64^3 and 128^3 grids: three streams
+// with 64 MiB in all beat one stream with 96 MiB by 5%, 5% and 7%, and two
+// or four streams, or larger budgets, by up to 4%.
 constexpr size_t kWaveBudget = size_t(HND_WAVE_MB) << 20;
 constexpr int kWaveStreams = HND_STREAMS;
+static_assert(kWaveStreams >= 1 && kWaveStreams <= hnd::SideStream::kMax, "streams per convolution");
 #ifndef HND_FILTER_MB
 #define HND_FILTER_MB 256
 #endif
@@ -194,18 +200,24 @@ hyena_nd_status make_plan(const hyena_nd_problem* p, Plan* pl) {
     if (kWaveStreams > 1 && pl->wave < pairs) {
       // several waves: run them on two streams, each wave in half the budget
       pl->wave = hnd::balanced_wave(pairs, p->B, per_pair, kWaveBudget / kWaveStreams, true);
-      pl->streams = pl->wave < pairs ? kWaveStreams : 1;
+      const long long waves = (pairs + pl->wave - 1) / pl->wave;
+      pl->streams = static_cast<int>(waves < kWaveStreams ? waves : kWaveStreams);
     }
     pl->wave_bytes = (per_pair * static_cast<size_t>(pl->wave) + 255) / 256 * 256;
     ws_conv = pl->wave_bytes * static_cast<size_t>(pl->streams);
   }
-  long long chunk = static_cast<long long>(kFilterBudget / (8 * static_cast<size_t>(pl->gsz)));
+  // filter call: 2D and 3D grids hold two channels per complex grid (the
+  // kernel values are real), so a channel costs half a grid
+  const bool fpair = p->ndim >= 2;
+  long long chunk = static_cast<long long>(kFilterBudget / ((fpair ? 4 : 8) * static_cast<size_t>(pl->gsz)));
   if (chunk < 1) chunk = 1;
   if (chunk > kFilterMaxChunk) chunk = kFilterMaxChunk;
+  if (fpair && chunk > 1) chunk -= chunk % 2;        // whole pairs per chunk
   if (chunk > p->C) chunk = p->C;
   pl->filter_chunk = static_cast<int>(chunk);
   // the chunk's grids, then the first-layer tables (for the largest hidden width)
-  pl->filter_grid_bytes = (static_cast<size_t>(chunk) * static_cast<size_t>(pl->gsz) * 8 + 255) / 256 * 256;
+  const long long fgrids = fpair ? (chunk + 1) / 2 : chunk;
+  pl->filter_grid_bytes = (static_cast<size_t>(fgrids) * static_cast<size_t>(pl->gsz) * 8 + 255) / 256 * 256;
   const size_t ws_filter = pl->filter_grid_bytes + static_cast<size_t>(hnd::filter_table_bytes(128, pl->ndim, pl->n));
   // kernel gradient: per channel B transformed grids (u + i z per sample) and
   // half an accumulator (two channels share one), P^d complex each
@@ -264,36 +276,41 @@ cudaError_t run_conv(const Plan& pl, const hnd::ConvArgs& a, void* ws, int* laun
     const int rp_total = static_cast<int>(pl.L / nl / 2);
     hnd::SideStream* side = nullptr;
     std::unique_lock<std::mutex> lk;
-    if (pl.streams > 1) {
-      // Waves alternate between the caller's stream and a side stream; the
-      // side stream starts one stage late, so that the column stage of one
-      // wave shares the SMs with the row stages of the next.  Each stream
-      // owns one wave-sized slice of the workspace.
+    const int ns = pl.streams;
+    if (ns > 1) {
+      // Waves go round-robin over the caller's stream and ns - 1 side
+      // streams; side stream j starts one stage after stream j - 1 (it waits
+      // for that stream's first forward rows), so that the column stage of
+      // one wave shares the SMs with the row stages of the next.  Each
+      // stream owns one wave-sized slice of the workspace.
       if ((e = hnd::side_stream(&side)) != cudaSuccess) return e;
       lk = std::unique_lock<std::mutex>(side->mu);
       if ((e = cudaEventRecord(side->fork, a.stream)) != cudaSuccess) return e;
-      if ((e = cudaStreamWaitEvent(side->s, side->fork, 0)) != cudaSuccess) return e;
+      for (int j = 1; j < ns && e == cudaSuccess; ++j) e = cudaStreamWaitEvent(side->s[j], side->fork, 0);
+      if (e != cudaSuccess) return e;
     }
+    auto stream_of = [&](int lane) { return lane == 0 ? a.stream : side->s[lane]; };
     int w = 0;
     for (long long ord0 = 0; ord0 < pairs && e == cudaSuccess; ord0 += pl.wave, ++w) {
       const int np = static_cast<int>(pairs - ord0 < pl.wave ? pairs - ord0 : pl.wave);
-      const int lane = pl.streams > 1 ? w % pl.streams : 0;
+      const int lane = ns > 1 ? w % ns : 0;
       hnd::ConvArgs aw = a;
-      if (lane == 1) aw.stream = side->s;
+      aw.stream = ns > 1 ? stream_of(lane) : a.stream;
       float2* zt = reinterpret_cast<float2*>(zbase + static_cast<size_t>(lane) * pl.wave_bytes);
       e = hnd::launch_rowfwd(aw, nl, zt, ord0, np, rp_total);
-      if (e == cudaSuccess && pl.streams > 1 && w == 0) {
-        e = cudaEventRecord(side->stagger, a.stream);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(side->s, side->stagger, 0);
+      if (e == cudaSuccess && ns > 1 && w + 1 < ns) {
+        // the next stream's first wave starts after this one's forward rows
+        e = cudaEventRecord(side->stagger[lane], aw.stream);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(side->s[lane + 1], side->stagger[lane], 0);
       }
       if (e == cudaSuccess) e = pl.tier == kMulti2D ? hnd::launch_mid1(aw, zt, ord0, np) : hnd::launch_mid2(aw, zt, ord0, np);
       if (e == cudaSuccess) e = hnd::launch_rowinv(aw, nl, zt, ord0, np, rp_total);
       *launches += 3;
     }
-    if (pl.streams > 1) {
-      // join: the caller's stream waits for the side stream's last wave
-      const cudaError_t e1 = cudaEventRecord(side->join, side->s);
-      const cudaError_t e2 = e1 == cudaSuccess ? cudaStreamWaitEvent(a.stream, side->join, 0) : e1;
+    for (int j = 1; j < ns; ++j) {
+      // join: the caller's stream waits for every side stream's last wave
+      const cudaError_t e1 = cudaEventRecord(side->join[j], side->s[j]);
+      const cudaError_t e2 = e1 == cudaSuccess ? cudaStreamWaitEvent(a.stream, side->join[j], 0) : e1;
       if (e == cudaSuccess) e = e2;
     }
   }
@@ -504,10 +521,15 @@ hyena_nd_status hyena_nd_kernel_grad(const hyena_nd_problem* p, const void* q, c
   bl.add(ws, ws_bytes);
   if (hnd::bounds_register(bl, static_cast<int*>(ws), static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
     return HYENA_ND_ERR_CUDA;
+  // 2D multi-pass grids (linear mode) run the row-pair stages, which need half
+  // the chunk workspace of the full-grid route
+  const bool stages = pl.tier == kMulti2D && !pl.circular;
   for (long long c0 = 0; c0 < pl.C; c0 += pl.kgrad_chunk) {
     g.c0 = static_cast<int>(c0);
     g.ncc = static_cast<int>(pl.C - c0 < pl.kgrad_chunk ? pl.C - c0 : pl.kgrad_chunk);
-    if (hnd::launch_kgrad_chunk(g, static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess) return HYENA_ND_ERR_CUDA;
+    const cudaError_t e = stages ? hnd::launch_kgrad2d_chunk(g, static_cast<cudaStream_t>(cuda_stream))
+                                 : hnd::launch_kgrad_chunk(g, static_cast<cudaStream_t>(cuda_stream));
+    if (e != cudaSuccess) return HYENA_ND_ERR_CUDA;
   }
   return HYENA_ND_OK;
 }

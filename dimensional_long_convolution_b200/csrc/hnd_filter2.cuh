@@ -23,6 +23,7 @@ namespace hnd2 {
 constexpr int kFT = 256;     // threads per CTA
 constexpr int kFO = 128;     // offsets per CTA
 constexpr int kFC = 32;      // channels per output tile
+constexpr int kFNarrow = 8;  // a tile with at most this many channels left takes the narrow path
 
 struct FilterMlpArgs {
   const float *W1, *b1, *W2, *b2, *alpha;
@@ -33,7 +34,8 @@ struct FilterMlpArgs {
   int ndim;
   int n[3];
   int c0, nc;                    // channel chunk [c0, c0 + nc)
-  float2* grid;                  // [nc][P^d]
+  float2* grid;                  // [nc][P^d], or with pair: [(nc + 1) / 2][P^d], channel c in component c & 1
+  int pair = 0;
   const float* gamma = nullptr;  // FiLM: sin(gamma (W1 phi + b1) + beta), [hidden] each; null = plain
   const float* beta = nullptr;
   const float* tab = nullptr;    // per-axis first-layer tables (k_filter_tables)
@@ -101,6 +103,22 @@ __device__ __forceinline__ float sine_layer(float x) {
   float r = fmaf(m, -6.28125f, x);                          // 2 pi head (exact times m for |m| < 2^15)
   r = fmaf(m, -1.9353071795864769e-3f, r);                  // 2 pi - 6.28125
   return __sinf(r);
+}
+
+// Kernel values of channels c .. c + 3 (c a multiple of 4; channels at or
+// beyond nc carry 0 and are not stored) at grid slot `so`: one real grid per
+// channel, or with pair two channels per complex grid (c even in the real
+// part, c + 1 in the imaginary part).
+__device__ __forceinline__ void store_k4(const FilterMlpArgs& a, int c, long long gsz, int so, const float (&kv)[4]) {
+  if (a.pair) {
+#pragma unroll
+    for (int j = 0; j < 4; j += 2)
+      if (c + j < a.nc) *HND_G(&a.grid[static_cast<long long>((c + j) >> 1) * gsz + so]) = make_float2(kv[j], kv[j + 1]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (c + j < a.nc) *HND_G(&a.grid[static_cast<long long>(c + j) * gsz + so]) = make_float2(kv[j], 0.f);
+  }
 }
 
 template <int HP, bool TAB>
@@ -247,6 +265,40 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
       (*HND_S(&w2[i])) = (h < a.hidden && c < a.nc) ? __ldg(HND_G(a.W2 + static_cast<long long>(a.c0 + c) * a.hidden + h)) : 0.f;
     }
     __syncthreads();
+    if (a.nc - ct <= kFNarrow) {
+      // narrow tile (a chunk of at most 8 channels, e.g. the large 3D grids):
+      // thread -> offset tid % kFO, channels 4 (tid / kFO) .. + 3, so no
+      // thread computes padding channels beyond the chunk's 8
+      const int o = tid % kFO, cb = 4 * (tid / kFO);
+      if (cb < a.nc - ct) {
+        float acc1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+        for (int h = 0; h < HP; ++h) {
+          const float hv = *HND_S(hid + h * kFO + o);
+          const float4 wv = *HND_S(reinterpret_cast<const float4*>(w2 + h * kFC + cb));
+          acc1[0] = fmaf(hv, wv.x, acc1[0]);
+          acc1[1] = fmaf(hv, wv.y, acc1[1]);
+          acc1[2] = fmaf(hv, wv.z, acc1[2]);
+          acc1[3] = fmaf(hv, wv.w, acc1[3]);
+        }
+        if (e0 + o < noff) {
+          const float ro = *HND_S(&rad[o]);
+          const int so = *HND_S(&slot[o]);
+          float kv[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int c = ct + cb + j;
+            kv[j] = 0.f;
+            if (c < a.nc) {
+              const float bb = __ldg(HND_G(a.b2 + a.c0 + c)), al = __ldg(HND_G(a.alpha + a.c0 + c));
+              kv[j] = (acc1[j] + bb) * __expf(-al * ro);
+            }
+          }
+          store_k4(a, ct + cb, gsz, so, kv);
+        }
+      }
+      continue;
+    }
     float acc[4][4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -262,18 +314,22 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(hh[i], ww[j], acc[i][j]);
     }
+    float bb[4], al[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int c = ct + 4 * grp + j;
-      if (c >= a.nc) continue;
-      const float bb = __ldg(HND_G(a.b2 + a.c0 + c)), al = __ldg(HND_G(a.alpha + a.c0 + c));
-      float2* gch = a.grid + static_cast<long long>(c) * gsz;
+      bb[j] = c < a.nc ? __ldg(HND_G(a.b2 + a.c0 + c)) : 0.f;
+      al[j] = c < a.nc ? __ldg(HND_G(a.alpha + a.c0 + c)) : 0.f;
+    }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int o = 4 * og + i;
-        if (e0 + o < noff)
-          (*HND_G(&gch[(*HND_S(&slot[o]))])) = make_float2((acc[i][j] + bb) * __expf(-al * (*HND_S(&rad[o]))), 0.f);
-      }
+    for (int i = 0; i < 4; ++i) {
+      const int o = 4 * og + i;
+      if (e0 + o >= noff) continue;
+      const float ro = *HND_S(&rad[o]);
+      float kv[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) kv[j] = ct + 4 * grp + j < a.nc ? (acc[i][j] + bb[j]) * __expf(-al[j] * ro) : 0.f;
+      store_k4(a, ct + 4 * grp, gsz, *HND_S(&slot[o]), kv);
     }
   }
 }

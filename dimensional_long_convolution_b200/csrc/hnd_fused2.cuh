@@ -463,9 +463,23 @@ __host__ __device__ __forceinline__ Pos2 pos2_of(int n0, int n1, long long e4) {
   return r;
 }
 
-// natural half spectrum [C][2 n0][n1 + 1] -> library order (v2)
+// Value at (row ky, column kx) of channel c of a source: a natural array
+// [C][2 n0][pitch], or (pair) the full grids of the filter call that hold two
+// channels per complex grid, K_c + i K_{c+1} for even c, whose transform W
+// gives S_c = (W[k] + conj W[-k]) / 2 and S_{c+1} = (W[k] - conj W[-k]) / (2i).
+__device__ __forceinline__ float2 src2_at(const float2* __restrict__ nat, long long c, long long src_per,
+                                          long long pitch, int ky, int kx, int n0, int n1, int pair) {
+  if (!pair) return *HND_G(&nat[c * src_per + ky * pitch + kx]);
+  const float2* g = nat + (c >> 1) * src_per;
+  const float2 w = *HND_G(&g[ky * pitch + kx]);
+  const float2 m = *HND_G(&g[static_cast<long long>((2 * n0 - ky) & (2 * n0 - 1)) * pitch + ((2 * n1 - kx) & (2 * n1 - 1))]);
+  return (c & 1) ? make_float2(0.5f * (w.y + m.y), 0.5f * (m.x - w.x)) : make_float2(0.5f * (w.x + m.x), 0.5f * (w.y - m.y));
+}
+
+// natural half spectrum [C][2 n0][n1 + 1] (or the filter call's full grids,
+// pitch 2 n1, pair: two channels per grid) -> library order (v2)
 static __global__ void k_spec_import_v2(const float2* __restrict__ nat, float4* __restrict__ out, int n0, int n1,
-                                 long long C, long long full_pitch, float scale) {
+                                 long long C, long long full_pitch, float scale, int pair = 0) {
   // full_pitch: row length of the source (n1 + 1 for a half spectrum, 2 n1 for a full grid)
   const long long per = static_cast<long long>(n1 + 1) * n0;         // float4 per channel
   const long long src_per = static_cast<long long>(2 * n0) * full_pitch;
@@ -473,15 +487,16 @@ static __global__ void k_spec_import_v2(const float2* __restrict__ nat, float4* 
        e += static_cast<long long>(gridDim.x) * blockDim.x) {
     const long long c = e / per, e4 = e % per;
     const Pos2 ps = pos2_of(n0, n1, e4);
-    const float2* src = nat + c * src_per;
     float2 s0, s1;
     if (ps.kind == 0) {
-      s0 = *HND_G(&src[ps.ky0 * full_pitch + ps.kx]);
-      s1 = *HND_G(&src[ps.ky1 * full_pitch + ps.kx]);
+      s0 = src2_at(nat, c, src_per, full_pitch, ps.ky0, ps.kx, n0, n1, pair);
+      s1 = src2_at(nat, c, src_per, full_pitch, ps.ky1, ps.kx, n0, n1, pair);
     } else {
       const float sg = ps.kind == 1 ? 1.f : -1.f;
-      const float2 a0 = *HND_G(&src[ps.ky0 * full_pitch]), b0 = *HND_G(&src[ps.ky0 * full_pitch + n1]);
-      const float2 a1 = *HND_G(&src[ps.ky1 * full_pitch]), b1 = *HND_G(&src[ps.ky1 * full_pitch + n1]);
+      const float2 a0 = src2_at(nat, c, src_per, full_pitch, ps.ky0, 0, n0, n1, pair);
+      const float2 b0 = src2_at(nat, c, src_per, full_pitch, ps.ky0, n1, n0, n1, pair);
+      const float2 a1 = src2_at(nat, c, src_per, full_pitch, ps.ky1, 0, n0, n1, pair);
+      const float2 b1 = src2_at(nat, c, src_per, full_pitch, ps.ky1, n1, n0, n1, pair);
       s0 = make_float2(0.5f * (a0.x + sg * b0.x), 0.5f * (a0.y + sg * b0.y));
       s1 = make_float2(0.5f * (a1.x + sg * b1.x), 0.5f * (a1.y + sg * b1.y));
     }

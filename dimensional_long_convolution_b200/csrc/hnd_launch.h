@@ -42,12 +42,14 @@ int sm_count();
 // that no wave is short; with whole_channels, a multiple of B where possible
 // so that the B samples sharing a channel spectrum run in one wave.
 long long balanced_wave(long long pairs, long long B, size_t per_pair, size_t budget, bool whole_channels);
-// A second stream per device (created on first use, kept until exit) with
-// the events that fork it from, stagger it against and join it back to the
-// caller's stream; `mu` serialises the enqueue of calls that use it.
+// Side streams per device (created on first use, kept until exit; s[0] is
+// unused: lane 0 is the caller's stream) with the events that fork them from,
+// stagger them against each other and join them back to the caller's
+// stream; `mu` serialises the enqueue of calls that use them.
 struct SideStream {
-  cudaStream_t s = nullptr;
-  cudaEvent_t fork = nullptr, stagger = nullptr, join = nullptr;
+  static constexpr int kMax = 4;
+  cudaStream_t s[kMax] = {};
+  cudaEvent_t fork = nullptr, stagger[kMax] = {}, join[kMax] = {};
   std::mutex mu;
 };
 cudaError_t side_stream(SideStream** out);
@@ -121,6 +123,10 @@ struct KgradLaunch {
   int circular;           // 1: fold onto the periodic grid, dK [C][n ...]
 };
 cudaError_t launch_kgrad_chunk(const KgradLaunch& g, cudaStream_t st);
+// The same on the 2D multi-pass tier (linear mode) through the row-pair and
+// half-spectrum stages: `grids` holds 2 B ncc volumes of packed row spectra
+// (8 n0 n1 bytes each) and ncc channel grids (16 n0 n1 bytes each).
+cudaError_t launch_kgrad2d_chunk(const KgradLaunch& g, cudaStream_t st);
 cudaError_t launch_bounded_wait(int* status, const int* flag, long long limit_cycles, cudaStream_t st);
 
 }  // namespace hnd

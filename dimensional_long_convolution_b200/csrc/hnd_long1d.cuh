@@ -140,7 +140,7 @@ __device__ __forceinline__ void l1_full_inv(cp (&x)[P2<N>::R1], float2 (&lo)[P2<
                                             int g, float4* buf, Tabs<N> t) {
   constexpr int G = P2<N>::G, R1 = P2<N>::R1;
   fft_inv<N>(x, g, buf, 0, t, 0u);
-  const float2 tg = t.b[4 * G + g];
+  const float2 tg = *HND_S(&t.b[4 * G + g]);
   sfor<0, R1>([&](auto sc) {
     constexpr int s = decltype(sc)::value;
     const float2 w = mul_w32<s * (16 / R1)>(tg);     // W_2N^{g + s G}

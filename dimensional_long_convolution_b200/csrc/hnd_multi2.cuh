@@ -221,26 +221,28 @@ __device__ __forceinline__ void rowinv_task(const Tabs<NL> t, unsigned char* wor
   float4* xb = reinterpret_cast<float4*>(work);     // shares the tile region
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nrp = min(RPB, rp_total - rpb);
-  tile_from_ws<NL>(tile, ztv, rp_total, rpb, nrp);
-  task_sync();
   const int pen = lane / G, g = lane % G;
   float4* buf = xb + warp * XB<NL>::kWarp + pen * XB<NL>::kPen;
   static_assert(RPB == kWM * PPW || RPB == 2 * kWM * PPW, "row tile covers one or two rounds");
   constexpr int ROUNDS = RPB / (kWM * PPW);
-  // pull every round's inputs out of the tile before the tile region turns
-  // into exchange buffers
   cp xin[ROUNDS][R1];
+  {
+    tile_from_ws<NL>(tile, ztv, rp_total, rpb, nrp);
+    task_sync();
+    // pull every round's inputs out of the tile before the tile region turns
+    // into exchange buffers
 #pragma unroll
-  for (int round = 0; round < ROUNDS; ++round) {
-    const int rl = round * kWM * PPW + warp * PPW + pen;
+    for (int round = 0; round < ROUNDS; ++round) {
+      const int rl = round * kWM * PPW + warp * PPW + pen;
 #pragma unroll
-    for (int s = 0; s < R1; ++s) {
-      const int kk = 2 * spec_idx<NL>(g, s);
-      const float2 e = *HND_S(&tile[R::row(kk) + rl]), d = *HND_S(&tile[R::row(kk + 1) + rl]);
-      xin[round][s] = {make_float2(e.x, d.x), make_float2(e.y, d.y)};
+      for (int s = 0; s < R1; ++s) {
+        const int kk = 2 * spec_idx<NL>(g, s);
+        const float2 e = *HND_S(&tile[R::row(kk) + rl]), d = *HND_S(&tile[R::row(kk + 1) + rl]);
+        xin[round][s] = {make_float2(e.x, d.x), make_float2(e.y, d.y)};
+      }
     }
+    task_sync();
   }
-  task_sync();
   for (int round = 0; round < ROUNDS; ++round) {
     const int r0 = round * kWM * PPW + warp * PPW;
     const int rl = r0 + pen;
@@ -312,9 +314,10 @@ struct M1 {
 // 0, the combined DC/Nyquist unit, whose product needs the partner
 // frequency; every pencil of that warp takes this path (for cu != 0 the
 // partner term is multiplied by zero).
-template <int N0, bool GEN>
+template <int N0, bool GEN, bool CONJ>
 __device__ __forceinline__ void mid1_unit(const Tabs<N0> t, float4* buf, float2* __restrict__ zt,
-                                          const float4* __restrict__ sp, int N1, int cu, int g, float sgn) {
+                                          const float4* __restrict__ sp, int N1, int cu, int g) {
+  constexpr float sgn = CONJ ? -1.f : 1.f;      // -1: conjugate spectrum (the adjoint)
   constexpr int G = P2<N0>::G, R1 = P2<N0>::R1, RP = N0 / 2, HS = R1 / 2;
   const bool act = cu < N1;
   const int kx = act ? cu : 1, kxm = cu == 0 ? N1 : 2 * N1 - kx;
@@ -401,17 +404,17 @@ __device__ __forceinline__ void mid1_unit(const Tabs<N0> t, float4* buf, float2*
 #else
 #define HND_OUT_OF_LINE __noinline__
 #endif
-template <int N0>
+template <int N0, bool CONJ>
 __device__ HND_OUT_OF_LINE void mid1_unit_gen(const Tabs<N0> t, float4* buf, float2* __restrict__ zt,
-                                           const float4* __restrict__ sp, int N1, int cu, int g, float sgn) {
-  mid1_unit<N0, true>(t, buf, zt, sp, N1, cu, g, sgn);
+                                           const float4* __restrict__ sp, int N1, int cu, int g) {
+  mid1_unit<N0, true, CONJ>(t, buf, zt, sp, N1, cu, g);
 }
 
 // One task: UPB column units starting at u0 of one volume; `sp` is the
 // channel's spectrum for this sample.
-template <int N0>
+template <int N0, bool CONJ>
 __device__ __forceinline__ void mid1_task(const Tabs<N0> t, unsigned char* work, float2* __restrict__ zt,
-                                          const float4* __restrict__ sp, int N1, int u0, float sgn) {
+                                          const float4* __restrict__ sp, int N1, int u0) {
   using M = M1<N0>;
   constexpr int G = M::G, PPW = M::PPW;
   float4* xb = reinterpret_cast<float4*>(work);
@@ -419,13 +422,13 @@ __device__ __forceinline__ void mid1_task(const Tabs<N0> t, unsigned char* work,
   const int pen = lane / G, g = lane % G;
   float4* buf = xb + warp * XB<N0>::kWarp + pen * XB<N0>::kPen;
   const int cu = u0 + warp * PPW + pen;
-  if (u0 == 0 && warp == 0) mid1_unit_gen<N0>(t, buf, zt, sp, N1, cu, g, sgn);
-  else mid1_unit<N0, false>(t, buf, zt, sp, N1, cu, g, sgn);
+  if (u0 == 0 && warp == 0) mid1_unit_gen<N0, CONJ>(t, buf, zt, sp, N1, cu, g);
+  else mid1_unit<N0, false, CONJ>(t, buf, zt, sp, N1, cu, g);
 }
 
-template <int N0>
+template <int N0, bool CONJ>
 __global__ void __launch_bounds__(kTM, 2) k_mid1v2(float2* __restrict__ Zt, const float4* __restrict__ spec,
-                                                long long sbs4, int N1, long long ord0, int B, int C, float sgn) {
+                                                long long sbs4, int N1, long long ord0, int B, int C) {
   extern __shared__ __align__(16) unsigned char smem[];
   pdl_release();
   const Tabs<N0> t = tabs_at<N0>(smem);
@@ -435,8 +438,8 @@ __global__ void __launch_bounds__(kTM, 2) k_mid1v2(float2* __restrict__ Zt, cons
   const float4* sp = spec + static_cast<long long>(b) * sbs4 + static_cast<long long>(c) * (N1 + 1) * N0;
   __syncthreads();
   pdl_wait();
-  mid1_task<N0>(t, smem + Tabs<N0>::kBytes, Zt + static_cast<long long>(blockIdx.x) * 2 * N1 * (N0 / 2), sp, N1,
-                blockIdx.y * M1<N0>::UPB, sgn);
+  mid1_task<N0, CONJ>(t, smem + Tabs<N0>::kBytes, Zt + static_cast<long long>(blockIdx.x) * 2 * N1 * (N0 / 2), sp, N1,
+                blockIdx.y * M1<N0>::UPB);
 }
 
 // ---------------------------------------------------------------- 3D slabs
@@ -503,10 +506,11 @@ __device__ __forceinline__ void slab_rows_out(float2* __restrict__ zt, long long
 // One task: the slab of last-axis frequency kx of one volume (`zt`), with the
 // channel's slab spectrum `sslab` for this sample.  `work` holds F, then the
 // exchange buffers.
-template <int N0, int N1, bool HALF>
+template <int N0, int N1, bool HALF, bool CONJ>
 __device__ __forceinline__ void mid2_task(const Tabs<N0> t0, const Tabs<N1> t1, unsigned char* work,
                                           float2* __restrict__ zt, const float4* __restrict__ sslab, int N2, int kx,
-                                          int h, float sgn) {
+                                          int h) {
+  constexpr float sgn = CONJ ? -1.f : 1.f;      // -1: conjugate spectrum (the adjoint)
   using M = M2<N0, N1, HALF>;
   constexpr int FS = M::FS, NKY = M::NKY;
   constexpr int G0 = P2<N0>::G, R0 = P2<N0>::R1, G1 = P2<N1>::G, R1 = P2<N1>::R1;
@@ -633,10 +637,10 @@ __device__ __forceinline__ void mid2_task(const Tabs<N0> t0, const Tabs<N1> t1, 
   if constexpr (HALF) cg::this_cluster().sync();
 }
 
-template <int N0, int N1, bool HALF>
+template <int N0, int N1, bool HALF, bool CONJ>
 __device__ __forceinline__ void mid2_kernel_body(float2* __restrict__ Zt, const float4* __restrict__ spec,
                                                  long long sbs4, int N2, long long ord0, int B, int C, int vol_local,
-                                                 int h, float sgn) {
+                                                 int h) {
   using M = M2<N0, N1, HALF>;
   extern __shared__ __align__(16) unsigned char smem[];
   pdl_release();
@@ -658,22 +662,22 @@ __device__ __forceinline__ void mid2_kernel_body(float2* __restrict__ Zt, const 
                         static_cast<long long>(kx) * slab;
   __syncthreads();
   pdl_wait();
-  mid2_task<N0, N1, HALF>(t0, t1, smem + M::kTabs, Zt + static_cast<long long>(vol_local) * 2 * N2 * RPn, sslab, N2,
-                          kx, h, sgn);
+  mid2_task<N0, N1, HALF, CONJ>(t0, t1, smem + M::kTabs, Zt + static_cast<long long>(vol_local) * 2 * N2 * RPn, sslab,
+                                N2, kx, h);
 }
 
-template <int N0, int N1>
+template <int N0, int N1, bool CONJ>
 __global__ void __launch_bounds__(kTM, 2) k_mid2v2(float2* __restrict__ Zt, const float4* __restrict__ spec,
-                                                long long sbs4, int N2, long long ord0, int B, int C, float sgn) {
-  mid2_kernel_body<N0, N1, false>(Zt, spec, sbs4, N2, ord0, B, C, blockIdx.x, 0, sgn);
+                                                long long sbs4, int N2, long long ord0, int B, int C) {
+  mid2_kernel_body<N0, N1, false, CONJ>(Zt, spec, sbs4, N2, ord0, B, C, blockIdx.x, 0);
 }
 
-template <int N0, int N1>
+template <int N0, int N1, bool CONJ>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTM)
     k_mid2v2_pair(float2* __restrict__ Zt, const float4* __restrict__ spec, long long sbs4, int N2, long long ord0,
-                  int B, int C, float sgn) {
+                  int B, int C) {
   const int h = static_cast<int>(cg::this_cluster().block_rank());
-  mid2_kernel_body<N0, N1, true>(Zt, spec, sbs4, N2, ord0, B, C, blockIdx.x / 2, h, sgn);
+  mid2_kernel_body<N0, N1, true, CONJ>(Zt, spec, sbs4, N2, ord0, B, C, blockIdx.x / 2, h);
 }
 
 // --------------------------------------------------- spectrum layouts (v2)
@@ -687,10 +691,27 @@ __host__ __device__ __forceinline__ int spec_idx_gen(int N, int g, int s) {
 }
 __host__ __device__ __forceinline__ int lanes_of(int N) { return N == 8 ? 1 : N / (N >= 128 ? 16 : 8); }
 
+// Value at (kz, ky, kx) of channel c of a source [C][2 n0][2 n1][pitch], or
+// (pair) of the filter call's full grids holding two channels per complex
+// grid (channel c even in the real part; S_c = (W[k] + conj W[-k]) / 2,
+// S_{c+1} = (W[k] - conj W[-k]) / (2i)).
+__device__ __forceinline__ float2 src3_at(const float2* __restrict__ nat, long long c, long long src_per,
+                                          long long pitch, int kz, int ky, int kx, int n0, int n1, int n2,
+                                          int pair) {
+  const long long row = 2LL * n1;
+  if (!pair) return *HND_G(&nat[c * src_per + (kz * row + ky) * pitch + kx]);
+  const float2* g = nat + (c >> 1) * src_per;
+  const float2 w = *HND_G(&g[(kz * row + ky) * pitch + kx]);
+  const int mz = (2 * n0 - kz) & (2 * n0 - 1), my = (2 * n1 - ky) & (2 * n1 - 1), mx = (2 * n2 - kx) & (2 * n2 - 1);
+  const float2 m = *HND_G(&g[(mz * row + my) * pitch + mx]);
+  return (c & 1) ? make_float2(0.5f * (w.y + m.y), 0.5f * (m.x - w.x)) : make_float2(0.5f * (w.x + m.x), 0.5f * (w.y - m.y));
+}
+
 // natural half spectrum [C][2n0][2n1][n2 + 1] (pitch = last-axis length of the
-// source: n2 + 1 for a half spectrum, 2 n2 for a full grid) -> library order
+// source: n2 + 1 for a half spectrum, 2 n2 for a full grid; pair: the filter
+// call's full grids, two channels per grid) -> library order
 static __global__ void k_spec3_in(const float2* __restrict__ nat, float4* __restrict__ out, int n0, int n1, int n2,
-                                  long long C, long long pitch, float scale) {
+                                  long long C, long long pitch, float scale, int pair = 0) {
   const long long per = static_cast<long long>(n2 + 1) * 2 * n1 * n0;     // float4 per channel
   const long long src_per = 4LL * n0 * n1 * pitch;
   const int G = lanes_of(n0);
@@ -701,9 +722,8 @@ static __global__ void k_spec3_in(const float2* __restrict__ nat, float4* __rest
     const long long r2 = r % (2LL * n1 * n0);
     const int ky = static_cast<int>(r2 / n0), m = static_cast<int>(r2 % n0);
     const int f = spec_idx_gen(n0, m % G, m / G);
-    const float2* src = nat + c * src_per;
-    const float2 s0 = *HND_G(&src[((2LL * f) * (2 * n1) + ky) * pitch + kx]);
-    const float2 s1 = *HND_G(&src[((2LL * f + 1) * (2 * n1) + ky) * pitch + kx]);
+    const float2 s0 = src3_at(nat, c, src_per, pitch, 2 * f, ky, kx, n0, n1, n2, pair);
+    const float2 s1 = src3_at(nat, c, src_per, pitch, 2 * f + 1, ky, kx, n0, n1, n2, pair);
     *HND_G(&out[e]) = make_float4(scale * s0.x, scale * s1.x, scale * s0.y, scale * s1.y);
   }
 }

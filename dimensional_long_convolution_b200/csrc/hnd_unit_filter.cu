@@ -202,7 +202,10 @@ cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, i
     gsz *= 2 * n[a];
     noff *= 2 * n[a] - 1;
   }
-  cudaError_t e = cudaMemsetAsync(grid, 0, sizeof(float2) * gsz * nc, st);
+  // 2D and 3D: two channels per complex grid (the kernel values are real)
+  const int pair = ndim >= 2 ? 1 : 0;
+  const int ngrids = pair ? (nc + 1) / 2 : nc;
+  cudaError_t e = cudaMemsetAsync(grid, 0, sizeof(float2) * gsz * ngrids, st);
   if (e != cudaSuccess) return e;
   hnd2::FilterMlpArgs fa;
   fa.W1 = f.W1;
@@ -224,6 +227,7 @@ cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, i
   fa.gamma = f.gamma;
   fa.beta = f.beta;
   fa.tab = f.tab;
+  fa.pair = pair;
   const int HP = (f.hidden + 31) / 32 * 32;
   e = HP <= 32 ? filter_mlp_go<32>(fa, noff, st)
       : HP <= 64 ? filter_mlp_go<64>(fa, noff, st)
@@ -236,17 +240,18 @@ cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, i
         grid, static_cast<float2*>(spectrum), gsz, c0, nc, static_cast<float>(1.0 / static_cast<double>(gsz)));
     return cudaGetLastError();
   }
-  e = launch_fft_axes(grid, ndim, n, nc, st);
+  e = launch_fft_axes(grid, ndim, n, ngrids, st);
   if (e != cudaSuccess) return e;
   const long long per = spec_per_channel(d);
   const float scale = static_cast<float>(1.0 / static_cast<double>(gsz));
   if (ndim == 2) {
     float4* out = static_cast<float4*>(spectrum) + static_cast<long long>(c0) * (per / 2);
     hnd2::k_spec_import_v2<<<grid_for(per / 2 * nc, 256), 256, 0, st>>>(grid, out, n[0], n[1], nc, 2LL * n[1],
-                                                                        scale);
+                                                                        scale, pair);
   } else if (ndim == 3) {
     float4* out = static_cast<float4*>(spectrum) + static_cast<long long>(c0) * (per / 2);
-    hnd2::k_spec3_in<<<grid_for(per / 2 * nc, 256), 256, 0, st>>>(grid, out, n[0], n[1], n[2], nc, 2LL * n[2], scale);
+    hnd2::k_spec3_in<<<grid_for(per / 2 * nc, 256), 256, 0, st>>>(grid, out, n[0], n[1], n[2], nc, 2LL * n[2], scale,
+                                                                  pair);
   } else {
     k_spec_pack<<<grid_for(per * nc, 256), 256, 0, st>>>(grid, static_cast<float2*>(spectrum), d, c0, nc, scale);
   }

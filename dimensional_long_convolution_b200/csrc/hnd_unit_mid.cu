@@ -6,9 +6,9 @@
 
 namespace hnd {
 
-template <int N0>
-static cudaError_t mid1_go(const ConvArgs& a, float2* zt, long long ord0, int np) {
-  auto kern = hnd2::k_mid1v2<N0>;
+template <int N0, bool CONJ>
+static cudaError_t mid1_go_c(const ConvArgs& a, float2* zt, long long ord0, int np) {
+  auto kern = hnd2::k_mid1v2<N0, CONJ>;
   const size_t sm = hnd2::M1<N0>::kBytes;
   cudaError_t e = ensure_smem(kern, sm);
   if (e != cudaSuccess) return e;
@@ -16,7 +16,13 @@ static cudaError_t mid1_go(const ConvArgs& a, float2* zt, long long ord0, int np
   const int n1 = a.n[1];
   dim3 grid(np, (n1 + UPB - 1) / UPB);
   return launch_pdl(true, kern, grid, dim3(hnd2::kTM), sm, a.stream, zt, static_cast<const float4*>(a.spec),
-                    a.sbs / 2, n1, ord0, a.B, a.C, a.sconj);
+                    a.sbs / 2, n1, ord0, a.B, a.C);
+}
+
+// sconj = -1: the adjoint (conjugate spectrum), a separate instantiation
+template <int N0>
+static cudaError_t mid1_go(const ConvArgs& a, float2* zt, long long ord0, int np) {
+  return a.sconj < 0.f ? mid1_go_c<N0, true>(a, zt, ord0, np) : mid1_go_c<N0, false>(a, zt, ord0, np);
 }
 
 cudaError_t launch_mid1(const ConvArgs& a, float2* zt, long long ord0, int np) {
@@ -31,26 +37,31 @@ cudaError_t launch_mid1(const ConvArgs& a, float2* zt, long long ord0, int np) {
   }
 }
 
-template <int N0, int N1>
-static cudaError_t mid2_go(const ConvArgs& a, float2* zt, long long ord0, int np) {
+template <int N0, int N1, bool CONJ>
+static cudaError_t mid2_go_c(const ConvArgs& a, float2* zt, long long ord0, int np) {
   const int n2 = a.n[2];
   if (hnd2::M2<N0, N1, false>::kBytes <= kMaxSmem) {
-    auto kern = hnd2::k_mid2v2<N0, N1>;
+    auto kern = hnd2::k_mid2v2<N0, N1, CONJ>;
     const size_t sm = hnd2::M2<N0, N1, false>::kBytes;
     cudaError_t e = ensure_smem(kern, sm);
     if (e != cudaSuccess) return e;
     dim3 grid(np, n2 + 1);
     return launch_pdl(true, kern, grid, dim3(hnd2::kTM), sm, a.stream, zt, static_cast<const float4*>(a.spec),
-                      a.sbs / 2, n2, ord0, a.B, a.C, a.sconj);
+                      a.sbs / 2, n2, ord0, a.B, a.C);
   } else {
-    auto kern = hnd2::k_mid2v2_pair<N0, N1>;
+    auto kern = hnd2::k_mid2v2_pair<N0, N1, CONJ>;
     const size_t sm = hnd2::M2<N0, N1, true>::kBytes;
     cudaError_t e = ensure_smem(kern, sm);
     if (e != cudaSuccess) return e;
     dim3 grid(2 * np, n2 + 1);
     return launch_pdl(true, kern, grid, dim3(hnd2::kTM), sm, a.stream, zt, static_cast<const float4*>(a.spec),
-                      a.sbs / 2, n2, ord0, a.B, a.C, a.sconj);
+                      a.sbs / 2, n2, ord0, a.B, a.C);
   }
+}
+
+template <int N0, int N1>
+static cudaError_t mid2_go(const ConvArgs& a, float2* zt, long long ord0, int np) {
+  return a.sconj < 0.f ? mid2_go_c<N0, N1, true>(a, zt, ord0, np) : mid2_go_c<N0, N1, false>(a, zt, ord0, np);
 }
 
 template <int N0>

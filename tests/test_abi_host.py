@@ -206,12 +206,13 @@ def test_workspace_stays_within_the_chunk_budgets(i):
 
 
 @pytest.mark.parametrize("i,tier,waves,launches,streams", [
-    (0, "fused_2d", 1, 1, 1), (1, "fused_2d", 1, 1, 1), (2, "multi_2d", 4, 12, 2), (3, "multi_3d", 8, 24, 2),
-    (4, "multi_3d", 16, 48, 2)])
+    (0, "fused_2d", 1, 1, 1), (1, "fused_2d", 1, 1, 1), (2, "multi_2d", 7, 21, 3), (3, "multi_3d", 13, 39, 3),
+    (4, "multi_3d", 32, 96, 3)])
 def test_plan_info_of_the_benchmark_grids(i, tier, waves, launches, streams):
     """The plan the calls run, read on the host: the launch counts are the
     ones the GPU tests and the bench observe; multi-pass grids with several
-    waves run alternate waves on two streams, each wave in 32 MiB."""
+    waves run them round-robin on three streams, each wave in a third of
+    64 MiB."""
     wl = W.workload(i)
     p = H.problem(wl.dims, wl.B, wl.C, H.BF16 if wl.io_dtype == "bf16" else H.F32)
     info = H.plan_info(p)

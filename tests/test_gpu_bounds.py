@@ -26,7 +26,7 @@ BOUNDS_LIB = os.path.join(ROOT, "dimensional_long_convolution_b200", "libhyena_n
 CONV = [((64,), 2, 3, "f32"), ((1024,), 1, 2, "f32"), ((32, 64), 2, 2, "bf16"), ((128, 256), 1, 2, "f32"),
         ((16, 32, 64), 1, 2, "f32"), ((128, 128, 8), 1, 1, "f32")]
 BWD = [((32, 32), 1, 2, "f32"), ((64, 128), 1, 2, "f32"), ((8, 16, 32), 1, 2, "f32")]
-KGRAD = [((32, 16), 2, 2, "f32"), ((8, 8, 16), 1, 2, "f32"), ((512,), 1, 2, "f32")]
+KGRAD = [((32, 16), 2, 2, "f32"), ((64, 128), 2, 2, "f32"), ((8, 8, 16), 1, 2, "f32"), ((512,), 1, 2, "f32")]
 
 
 def _child() -> None:

@@ -29,7 +29,11 @@ def _gpu(wl, inp, dy):
 
 @pytest.mark.parametrize("dims,B,C,dt", [((32,), 2, 3, "f32"), ((256,), 1, 2, "bf16"), ((16, 32), 2, 2, "f32"),
                                          ((64, 64), 1, 2, "bf16"), ((8, 16, 8), 2, 2, "f32"),
-                                         ((128, 128), 2, 53, "f32")])
+                                         ((128, 128), 2, 53, "f32"),
+                                         # 2D multi-pass grids: the row-pair / half-spectrum route, every
+                                         # column-kernel geometry (n0 = 8 .. 256) and a single sample
+                                         ((128, 256), 1, 2, "bf16"), ((256, 128), 3, 3, "f32"), ((8, 128), 2, 3, "f32"),
+                                         ((256, 8), 2, 2, "f32"), ((16, 256), 1, 3, "f32"), ((32, 128), 2, 2, "bf16")])
 def test_kernel_grad_matches_oracle(dims, B, C, dt):
     wl = W.custom(dims, B, C, io_dtype=dt, seed=5 + sum(dims))
     inp = W.make_inputs(wl, with_qkv=True)

@@ -245,28 +245,28 @@ def _wave_edge_channels(wl):
 
 
 def test_multi_wave_schedule_2d():
-    """More volumes (400 of 256^2) than one wave's workspace holds: seven
-    balanced waves of 58 volumes (the last 52) on two alternating streams."""
+    """More volumes (400 of 256^2) than one wave's workspace holds: ten
+    balanced waves of 40 volumes, round-robin on three streams."""
     dims = (256, 256)
     wl = W.custom(dims, 2, 200, io_dtype="bf16", seed=31)
     info, chans = _wave_edge_channels(wl)
-    assert info["waves"] == 7 and info["streams"] == 2
+    assert info["waves"] == 10 and info["streams"] == 3
     inp = W.make_inputs(wl)
     got, _ = run(inp)
-    assert H.last_launch_count() == info["launches"] == 21
+    assert H.last_launch_count() == info["launches"] == 30
     _check_sampled(wl, inp, got, chans, 1e-2)
 
 
 def test_multi_wave_schedule_3d():
-    """100 volumes of 32x64x64 at 1 MiB of intermediate each run as four
-    balanced waves of 25 on two alternating streams."""
+    """100 volumes of 32x64x64 at 1 MiB of intermediate each run as five
+    balanced waves of 20, round-robin on three streams."""
     dims = (32, 64, 64)
     wl = W.custom(dims, 1, 100, io_dtype="bf16", seed=37)
     info, chans = _wave_edge_channels(wl)
-    assert info["waves"] == 4 and info["streams"] == 2
+    assert info["waves"] == 5 and info["streams"] == 3
     inp = W.make_inputs(wl)
     got, _ = run(inp)
-    assert H.last_launch_count() == info["launches"] == 12
+    assert H.last_launch_count() == info["launches"] == 15
     _check_sampled(wl, inp, got, chans, 1e-2)
 
 
@@ -302,8 +302,8 @@ def test_bounded_wait_reports_timeout_and_recovers():
 
 def test_calls_run_in_their_own_workspace_size():
     """The filter call in exactly hyena_nd_workspace_bytes_for(FILTER) bytes
-    and the convolution in exactly ..._for(CONV) bytes (several waves on two
-    streams), against the oracle."""
+    and the convolution in exactly ..._for(CONV) bytes (several waves on
+    several streams), against the oracle."""
     t = torch()
     dims = (256, 256)
     wl = W.custom(dims, 2, 70, io_dtype="bf16", seed=45)
