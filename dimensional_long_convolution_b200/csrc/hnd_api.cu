@@ -127,7 +127,6 @@ struct Plan {
   int circular = 0;
   long long L = 1;          // voxels per volume
   long long gsz = 1;        // padded grid points per channel
-  long long spec_per = 0;   // complex values per channel spectrum
   int tier = 0;
   long long wave = 0;       // pairs per wave (multi-pass tiers)
   int streams = 1;          // multi-pass tiers: streams running alternate waves
@@ -175,19 +174,18 @@ hyena_nd_status make_plan(const hyena_nd_problem* p, Plan* pl) {
     pl->gsz *= 2 * p->n[a];
   }
   const int nl = pl->n[p->ndim - 1];
-  if (p->ndim == 1) pl->spec_per = nl > 256 ? 2LL * nl : nl + 1;   // long 1D: the full four-step spectrum
-  else if (p->ndim == 2) pl->spec_per = static_cast<long long>(nl + 1) * 2 * pl->n[0];
-  else pl->spec_per = static_cast<long long>(nl + 1) * 4 * pl->n[0] * pl->n[1];
-  pl->spec_bytes = static_cast<size_t>(pl->spec_per) * 8 * static_cast<size_t>(p->C);
+  pl->spec_bytes = hnd::spectrum_set_bytes(p->ndim, pl->n, p->C);
   pl->nat_bytes = static_cast<size_t>(pl->gsz / (2 * nl) * (nl + 1)) * 8 * static_cast<size_t>(p->C);
 
   const long long pairs = p->B * p->C;
   size_t ws_conv = 0;
   if (p->ndim == 1 && nl > 256) {
     pl->tier = kLong1D;
-    const size_t per_vol = static_cast<size_t>(8) * static_cast<size_t>(pl->gsz);
-    pl->wave = hnd::balanced_wave(pairs, p->B, per_vol, kL1WaveBudget, false);
-    ws_conv = per_vol * static_cast<size_t>(pl->wave);
+    // one complex grid per channel pair of a sample
+    const size_t per_grid = static_cast<size_t>(8) * static_cast<size_t>(pl->gsz);
+    const long long grids = p->B * ((p->C + 1) / 2);
+    pl->wave = hnd::balanced_wave(grids, 1, per_grid, kL1WaveBudget, false);
+    ws_conv = per_grid * static_cast<size_t>(pl->wave);
   } else if (p->ndim == 1) {
     pl->tier = kRows1D;
   } else if (hnd::fused_2d(p->ndim, pl->n)) {
@@ -206,9 +204,9 @@ hyena_nd_status make_plan(const hyena_nd_problem* p, Plan* pl) {
     pl->wave_bytes = (per_pair * static_cast<size_t>(pl->wave) + 255) / 256 * 256;
     ws_conv = pl->wave_bytes * static_cast<size_t>(pl->streams);
   }
-  // filter call: 2D and 3D grids hold two channels per complex grid (the
-  // kernel values are real), so a channel costs half a grid
-  const bool fpair = p->ndim >= 2;
+  // filter call: two channels per complex grid (the kernel values are real),
+  // so a channel costs half a grid; the short 1D rows keep one per channel
+  const bool fpair = p->ndim >= 2 || pl->tier == kLong1D;
   long long chunk = static_cast<long long>(kFilterBudget / ((fpair ? 4 : 8) * static_cast<size_t>(pl->gsz)));
   if (chunk < 1) chunk = 1;
   if (chunk > kFilterMaxChunk) chunk = kFilterMaxChunk;
@@ -350,7 +348,8 @@ hyena_nd_status hyena_nd_plan_info_get(const hyena_nd_problem* p, hyena_nd_plan_
   if (st != HYENA_ND_OK) return st;
   hyena_nd_plan_info info{};
   info.tier = static_cast<hyena_nd_tier>(pl.tier);
-  const long long vols = pl.B * pl.C;
+  // wave items: (b, c) volumes, or channel-pair grids in the long 1D tier
+  const long long vols = pl.tier == kLong1D ? pl.B * ((pl.C + 1) / 2) : pl.B * pl.C;
   info.wave = pl.tier == kRows1D || pl.tier == kFused2D ? 0 : pl.wave;
   info.waves = info.wave > 0 ? (vols + pl.wave - 1) / pl.wave : 1;
   info.split[0] = info.split[1] = info.split[2] = 1;

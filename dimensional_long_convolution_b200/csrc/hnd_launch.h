@@ -106,7 +106,12 @@ struct L1Split {
 };
 L1Split long1d_split(int n);
 int long1d_launches_per_transform(int n);
+// Channels 2j and 2j + 1 of a sample share one complex grid; `wave` counts
+// these channel-pair grids (B ceil(C/2) in all).
 cudaError_t launch_long1d(const ConvArgs& a, float2* grid, long long wave, int* launches);
+// Bytes of one spectrum set in library order (C channels; long 1D: the pair
+// layout of ceil(C/2) channel pairs).
+size_t spectrum_set_bytes(int ndim, const int* n, long long C);
 // In-place full forward transforms along every axis of `ngrids` complex grids
 // [P^d] (P_a = 2 n_a), adjacent in memory.  skip_zero: the grids hold
 // zero-padded data (zero wherever some s_a >= n_a), so the pencils of each

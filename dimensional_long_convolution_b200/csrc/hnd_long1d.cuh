@@ -1,23 +1,29 @@
 // hnd_long1d.cuh -- 1D grids longer than one transform pencil (n in
 // [512, 2^26]): the zero-padded length-P transform (P = 2n) as a multi-level
 // split P = P0 P1 (P2) with every factor at most 512, on the row-major view
-// [P0][P1][P2] of each volume's grid (j = (j0 P1 + j1) P2 + j2):
+// [P0][P1][P2] of each grid (j = (j0 P1 + j1) P2 + j2):
 //   forward   transform along axis 0 (the padded half j0 >= P0/2 is zero),
 //             twiddle W_P^{k0 r} (r the flattened later index), then the same
 //             split recursively on the later axes
-//             -> X(k0 + P0 k1 + P0 P1 k2) at [k0][k1][k2] (the spectrum is kept
-//             in this order)
-//   modulate  Y = X S (or X conj(S) for the adjoint), stored conjugated
+//             -> X(k0 + P0 k1 + P0 P1 k2) at [k0][k1][k2]
+//   modulate  on the last axis (the center)
 //   inverse   the same steps in reverse order (last axis first, each twiddle
 //             after the transform of its level's later axes): every step is
 //             a symmetric operator, so the reversed chain applied to data in
 //             split order is the DFT in natural order; on conjugated data it
 //             gives the conjugate of the unnormalised inverse at i = j
-//   output    y[i] = q[i] Re(.) for i < n (the crop), optional second gate
+//   output    y[i] = q[i] (.) for i < n (the crop), optional second gate
+// Channel pairs: the inputs of channels 2j and 2j + 1 of one sample are real,
+// so they share one complex grid, z = u_a + i u_b.  With Z = U_a + i U_b and
+// Z_m = Z(-k), the product that the two channels need is
+//   Y = K_a U_a + i K_b U_b = A Z + D conj(Z_m),  A = (K_a + K_b)/2, D = (K_a - K_b)/2
+// and the inverse of Y is y_a + i y_b (both convolutions are real).  The
+// spectrum of a pair therefore holds (A, D) per frequency, and only for half
+// of them: A(-k) = conj A(k), D(-k) = conj D(k).
 // (HyenaND pages: arXiv 2607.19378 summary, d = 1 long context through the
 // zero-padded FFT path; blog "Native multi-dimensional subquadratic operators
 // via input-dependent long convolutions", section "HyenaND".)
-// The axis transforms are k_fft_axis2 of hnd_filter2.cuh.
+// The filter's axis transforms are k_fft_axis2 of hnd_filter2.cuh.
 #pragma once
 
 #include "hnd_filter2.cuh"
@@ -40,87 +46,142 @@ static __global__ void k_l1_twiddle(float2* __restrict__ grid, int Pa, long long
   }
 }
 
-// filter grids (after the forward split transform) -> spectrum [c0 + c][P], scaled
-static __global__ void k_l1_spec_store(const float2* __restrict__ grid, float2* __restrict__ spec, long long P, int c0,
-                                       int nc, float scale) {
-  const long long total = P * nc;
-  for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < total;
+// Pair spectrum layout.  The center axis is the last level (length Pc); the
+// earlier levels form the pencil frequency kap = k0 + P0 k1 in [0, Po)
+// (Po = P / Pc), so k = kap + Po kc.  The pencil of -k is Po - kap (mod Po)
+// with kc reversed (Pc - 1 - kc) for kap != 0, and kc negated for kap = 0.
+// Pencils kap = 0 and kap = Po/2 are their own partners; the others pair up.
+// The spectrum of channel pair j keeps the pencils kap = 0 .. Po/2 only:
+//   float4 {A, D} at [j][kap][kc],  (Po/2 + 1) Pc per pair.
+// Memory pencil (row-major grid) of pencil frequency kap.
+__host__ __device__ __forceinline__ long long l1_pencil(long long kap, int P0, int Pm) {
+  return (kap % P0) * Pm + kap / P0;
+}
+// Grid position of frequency k (split order).
+__host__ __device__ __forceinline__ long long l1_pos(long long k, int P0, int Pm, int Pc) {
+  const long long Po = static_cast<long long>(P0) * Pm;
+  return l1_pencil(k % Po, P0, Pm) * Pc + k / Po;
+}
+
+struct L1Spec {
+  int P0, Pm, Pc;            // first, middle (1 for two levels) and center factors
+  long long Po, R;           // pencils per grid, stored pencils per pair (Po/2 + 1)
+  __host__ __device__ long long per_pair() const { return R * Pc; }      // float4
+};
+
+// the pair layout of an m-level split P[0..m-1]
+inline L1Spec l1_spec_of(int m, const int* P) {
+  L1Spec d;
+  d.P0 = P[0];
+  d.Pm = m == 3 ? P[1] : 1;
+  d.Pc = P[m - 1];
+  d.Po = static_cast<long long>(d.P0) * d.Pm;
+  d.R = d.Po / 2 + 1;
+  return d;
+}
+
+// filter grids (channels c0 + 2jp + {0, 1} as the real and imaginary part,
+// after the forward split transform) -> pair spectrum, scaled by 1/P
+static __global__ void k_l1_pair_store(const float2* __restrict__ grid, float4* __restrict__ spec, L1Spec d, int jp0,
+                                       int ngrids, float scale) {
+  const long long P = d.Po * d.Pc, per = d.per_pair();
+  for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < per * ngrids;
        e += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const float2 x = *HND_G(&grid[e]);
-    *HND_G(&spec[static_cast<long long>(c0) * P + e]) = make_float2(x.x * scale, x.y * scale);
+    const long long jp = e / per, rem = e % per, kap = rem / d.Pc, kc = rem % d.Pc;
+    const long long k = kap + d.Po * kc, km = (P - k) % P;
+    const float2* gj = grid + jp * P;
+    const float2 w = *HND_G(&gj[l1_pos(k, d.P0, d.Pm, d.Pc)]);
+    const float2 wm = *HND_G(&gj[l1_pos(km, d.P0, d.Pm, d.Pc)]);
+    // K_a = (W + conj Wm)/2, K_b = (W - conj Wm)/(2i)
+    const float2 ka = make_float2(0.5f * (w.x + wm.x), 0.5f * (w.y - wm.y));
+    const float2 kb = make_float2(0.5f * (w.y + wm.y), 0.5f * (wm.x - w.x));
+    const float h = 0.5f * scale;
+    *HND_G(&spec[(jp0 + jp) * per + rem]) =
+        make_float4(h * (ka.x + kb.x), h * (ka.y + kb.y), h * (ka.x - kb.x), h * (ka.y - kb.y));
   }
 }
 
-// library order [C][P0][P1][P2] (X(k0 + P0 k1 + P0 P1 k2) at (k0 P1 + k1) P2 + k2;
-// P2 = 1 for a two-level split) <-> natural half spectrum [C][n + 1]; the
-// import fills the other half by Hermitian symmetry
-static __device__ __forceinline__ long long l1_pos(long long k, int P0, int P1, int P2) {
-  return ((k % P0) * P1 + (k / P0) % P1) * P2 + k / (static_cast<long long>(P0) * P1);
+// (A, D) of frequency k from the stored half, conjugated for the other half
+__device__ __forceinline__ float4 l1_pair_at(const float4* __restrict__ sp, const L1Spec& d, long long k) {
+  const long long kap = k % d.Po, kc = k / d.Po;
+  if (kap <= d.Po / 2) return *HND_G(&sp[kap * d.Pc + kc]);
+  const float4 v = *HND_G(&sp[(d.Po - kap) * d.Pc + (d.Pc - 1 - kc)]);
+  return make_float4(v.x, -v.y, v.z, -v.w);
 }
 
-static __global__ void k_l1_spec_export(const float2* __restrict__ lib, float2* __restrict__ nat, int n, int P0,
-                                        int P1, int P2, long long C) {
-  const long long P = static_cast<long long>(P0) * P1 * P2, H = n + 1LL;
+// pair spectra [ceil(C/2)] <-> natural half spectra [C][n + 1]
+static __global__ void k_l1_spec_export(const float4* __restrict__ lib, float2* __restrict__ nat, int n, L1Spec d,
+                                        long long C) {
+  const long long H = n + 1LL;
   for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < H * C;
        e += static_cast<long long>(gridDim.x) * blockDim.x) {
     const long long c = e / H, k = e % H;
-    *HND_G(&nat[e]) = *HND_G(&lib[c * P + l1_pos(k, P0, P1, P2)]);
+    const float4 ad = l1_pair_at(lib + (c / 2) * d.per_pair(), d, k);
+    // K_a = A + D, K_b = A - D
+    *HND_G(&nat[e]) = (c & 1) ? make_float2(ad.x - ad.z, ad.y - ad.w) : make_float2(ad.x + ad.z, ad.y + ad.w);
   }
 }
 
-static __global__ void k_l1_spec_import(const float2* __restrict__ nat, float2* __restrict__ lib, int n, int P0,
-                                        int P1, int P2, long long C, long long pitch, float scale) {
-  const long long P = static_cast<long long>(P0) * P1 * P2;
-  for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < P * C;
+__device__ __forceinline__ float2 l1_nat_at(const float2* __restrict__ nat, long long P, int n, long long k) {
+  if (k <= n) return *HND_G(&nat[k]);
+  const float2 s = *HND_G(&nat[P - k]);
+  return make_float2(s.x, -s.y);
+}
+
+static __global__ void k_l1_spec_import(const float2* __restrict__ nat, float4* __restrict__ lib, int n, L1Spec d,
+                                        long long C, long long pitch) {
+  const long long P = d.Po * d.Pc, per = d.per_pair(), npair = (C + 1) / 2;
+  for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < per * npair;
        e += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long c = e / P, r = e % P;
-    const long long k = r / (static_cast<long long>(P1) * P2) + P0 * ((r / P2) % P1) +
-                        static_cast<long long>(P0) * P1 * (r % P2);
-    float2 s;
-    if (k <= n) {
-      s = *HND_G(&nat[c * pitch + k]);
-    } else {
-      s = *HND_G(&nat[c * pitch + (P - k)]);
-      s.y = -s.y;
-    }
-    *HND_G(&lib[e]) = make_float2(s.x * scale, s.y * scale);
+    const long long j = e / per, rem = e % per;
+    const long long k = rem / d.Pc + d.Po * (rem % d.Pc);
+    const float2 ka = l1_nat_at(nat + 2 * j * pitch, P, n, k);
+    const float2 kb = 2 * j + 1 < C ? l1_nat_at(nat + (2 * j + 1) * pitch, P, n, k) : make_float2(0.f, 0.f);
+    *HND_G(&lib[e]) = make_float4(0.5f * (ka.x + kb.x), 0.5f * (ka.y + kb.y), 0.5f * (ka.x - kb.x),
+                                  0.5f * (ka.y - kb.y));
   }
 }
 
 // ------------------------------------------------------------ fused passes
-// One convolution over a wave of volumes as 2m - 1 passes, each an axis
+// One convolution over a wave of channel pairs as 2m - 1 passes, each an axis
 // transform with its neighbours' elementwise steps folded in:
-//   kFirst   axis 0: k v of the first P0/2 rows (the rest is the zero pad),
-//            padded forward transform, forward twiddle of level 0
+//   kFirst   axis 0: k v of both channels of the pair (real and imaginary
+//            part) on the first P0/2 rows (the rest is the zero pad), padded
+//            forward transform, forward twiddle of level 0
 //   kFwdMid  axis 1 of 3: full forward transform, forward twiddle of level 1
-//   kCenter  last axis: full forward transform, spectrum product, full
-//            inverse transform, conjugate twiddle of level m - 2
+//   center   last axis (k_l1_center): the pencils kap and Po - kap together,
+//            full forward transforms, Y = A Z + D conj(Z_m), full inverse
+//            transforms, conjugate twiddle of level m - 2
 //   kInvMid  axis 1 of 3: full inverse transform, conjugate twiddle of level 0
 //   kLast    axis 0: inverse transform of which only the first P0/2 outputs
-//            (the crop i < n) are formed, output gate(s)
+//            (the crop i < n) are formed; real part to channel a, imaginary
+//            part to channel b, output gate(s)
 // The inverse chain (inverse transforms, conjugate twiddles, last axis first)
 // is the adjoint of the forward chain, so on spectra in split order it forms
 // the unnormalised inverse in natural order (the spectrum holds the 1/P).
-enum L1Kind { kFirst = 0, kFwdMid = 1, kCenter = 2, kInvMid = 3, kLast = 4 };
+enum L1Kind { kFirst = 0, kFwdMid = 1, kInvMid = 3, kLast = 4 };
 
 struct L1PassArgs {
-  float2* grid;              // wave grids [vol][P]
+  float2* grid;              // wave grids [pair][P]
   long long P;               // points per grid
   long long stride;          // stride of the pass's axis (points)
-  long long npen;            // pencils in the wave
+  long long npen;            // pencils in the wave (center: pencil pairs)
   long long twQ;             // twiddle order Q (W_Q)
   int twP;                   // inverse twiddles: the level's factor (k = outer index mod twP)
   int lgS, lgP, lgQ;         // log2 of stride, P and twQ (all powers of two)
   int n;                     // volume length
-  long long v0;              // first volume of the wave (memory order b C + c)
+  long long v0;              // first channel pair of the wave (order b H + j)
+  int H;                     // channel pairs per sample, (C + 1) / 2
   const void* a;             // kFirst: k
   const void* b;             // kFirst: v
   const void* q;             // kLast: output gate
   void* y;                   // kLast: output
   const void* g2;            // kLast: second gate (dual output) or null
   void* y2;
-  const float2* spec;        // kCenter: spectrum [C][P] per sample set
-  long long sbs;             // sample-set stride (complex values)
+  const float4* spec;        // center: pair spectra [H] per sample set
+  long long sbs4;            // sample-set stride (float4)
+  L1Spec sd;                 // center: split of the pair spectrum
+  int lgP0;                  // center: log2 P0 (pencil frequency -> memory pencil)
   float sconj;               // -1: conjugate spectrum (adjoint)
   int C;
 };
@@ -150,6 +211,14 @@ __device__ __forceinline__ void l1_full_inv(cp (&x)[P2<N>::R1], float2 (&lo)[P2<
     lo[s] = make_float2(x[s].re.x + br, x[s].im.x + bi);
     hi[s] = make_float2(x[s].re.x - br, x[s].im.x - bi);
   });
+}
+
+// channels of pair pg: first volume (memory order b C + c) and whether the
+// second channel exists (odd C leaves the last pair of a sample half empty)
+__device__ __forceinline__ long long l1_pair_vol(long long pg, int H, int C, bool* has_b) {
+  const long long b = pg / H, j = pg - b * H;
+  *has_b = 2 * j + 1 < C;
+  return b * C + 2 * j;
 }
 
 template <int N, int KIND, class T, bool DUAL>
@@ -182,14 +251,17 @@ __global__ void __launch_bounds__(kAT, 2) k_l1_pass(const L1PassArgs a) {
       const T* ka = static_cast<const T*>(a.a);
       const T* va = static_cast<const T*>(a.b);
       float2 z[R1];
-      const long long row0 = (a.v0 + vol) * a.n + i;
+      bool has_b;
+      const long long row0 = l1_pair_vol(a.v0 + vol, a.H, a.C, &has_b) * a.n + i;
+      const bool actb = act && has_b;
 #pragma unroll
       for (int s = 0; s < R1; ++s) {
         const long long j = row0 + static_cast<long long>(g + s * G) * S;
-        z[s] = act ? make_float2(Act<T>::ld_g(ka + j) * Act<T>::ld_g(va + j), 0.f) : make_float2(0.f, 0.f);
+        z[s] = make_float2(act ? Act<T>::ld_g(ka + j) * Act<T>::ld_g(va + j) : 0.f,
+                           actb ? Act<T>::ld_g(ka + j + a.n) * Act<T>::ld_g(va + j + a.n) : 0.f);
       }
       padded_fwd<N>(z, x, g, buf, 0, t, 0u);
-    } else if constexpr (KIND == kFwdMid || KIND == kCenter) {
+    } else if constexpr (KIND == kFwdMid) {
       float2 lo[R1], hi[R1];
 #pragma unroll
       for (int s = 0; s < R1; ++s) {
@@ -222,36 +294,6 @@ __global__ void __launch_bounds__(kAT, 2) k_l1_pass(const L1PassArgs a) {
           *HND_G(&base[(2 * f + 1) * S]) = cmul1(make_float2(x[s].re.y, x[s].im.y), w1);
         }
       }
-    } else if constexpr (KIND == kCenter) {
-      const int vg = static_cast<int>(a.v0 + vol);     // B C <= INT_MAX
-      const long long bb = vg / a.C, cc = vg % a.C;
-      const float2* Sp = a.spec + bb * a.sbs + cc * a.P + (start - vol * a.P);
-#pragma unroll
-      for (int s = 0; s < R1; ++s) {
-        const long long f = spec_idx<N>(g, s);
-        float4 sv = act ? __ldg(HND_G(reinterpret_cast<const float4*>(Sp + 2 * f))) : make_float4(0.f, 0.f, 0.f, 0.f);
-        sv.y *= a.sconj;
-        sv.w *= a.sconj;
-        const float2 y0 = cmul1(make_float2(x[s].re.x, x[s].im.x), make_float2(sv.x, sv.y));
-        const float2 y1 = cmul1(make_float2(x[s].re.y, x[s].im.y), make_float2(sv.z, sv.w));
-        x[s] = {make_float2(y0.x, y1.x), make_float2(y0.y, y1.y)};
-      }
-      float2 lo[R1], hi[R1];
-      l1_full_inv<N>(x, lo, hi, g, buf, t);
-      // conjugate twiddle of the previous level: conj W_Q^{k e}, k = o mod twP,
-      // e the element's index along this (last) axis
-      const unsigned k = static_cast<unsigned>(o & (a.twP - 1));
-      const float2 wk = l1_conj(l1_w(k * N, invQ));
-#pragma unroll
-      for (int s = 0; s < R1; ++s) {
-        const unsigned j = g + s * G;
-        const float2 w0 = l1_conj(l1_w(k * j, invQ));
-        const float2 w1 = cmul1(w0, wk);
-        if (act) {
-          *HND_G(&base[j]) = cmul1(lo[s], w0);
-          *HND_G(&base[j + N]) = cmul1(hi[s], w1);
-        }
-      }
     } else if constexpr (KIND == kInvMid) {
       float2 lo[R1], hi[R1];
       l1_full_inv<N>(x, lo, hi, g, buf, t);
@@ -270,12 +312,14 @@ __global__ void __launch_bounds__(kAT, 2) k_l1_pass(const L1PassArgs a) {
         }
       }
     } else {
-      // kLast: outputs i0 < N only (the crop), real part, output gate(s)
+      // kLast: outputs i0 < N only (the crop); real part -> channel a,
+      // imaginary part -> channel b; output gate(s)
       float2 out[R1];
       padded_inv<N>(x, out, g, buf, 0, t, 0u);
       const T* qa = static_cast<const T*>(a.q);
       T* ya = static_cast<T*>(a.y);
-      const long long row0 = (a.v0 + vol) * a.n + i;
+      bool has_b;
+      const long long row0 = l1_pair_vol(a.v0 + vol, a.H, a.C, &has_b) * a.n + i;
 #pragma unroll
       for (int s = 0; s < R1; ++s) {
         const long long j = row0 + static_cast<long long>(g + s * G) * S;
@@ -283,7 +327,125 @@ __global__ void __launch_bounds__(kAT, 2) k_l1_pass(const L1PassArgs a) {
           Act<T>::st_g(ya + j, out[s].x * Act<T>::ld_g(qa + j));
           if constexpr (DUAL)
             Act<T>::st_g(static_cast<T*>(a.y2) + j, out[s].x * Act<T>::ld_g(static_cast<const T*>(a.g2) + j));
+          if (has_b) {
+            Act<T>::st_g(ya + j + a.n, out[s].y * Act<T>::ld_g(qa + j + a.n));
+            if constexpr (DUAL)
+              Act<T>::st_g(static_cast<T*>(a.y2) + j + a.n,
+                           out[s].y * Act<T>::ld_g(static_cast<const T*>(a.g2) + j + a.n));
+          }
         }
+      }
+    }
+  }
+}
+
+// Center pass: one unit = the pencil frequencies kap and Po - kap of one
+// channel-pair grid, on two neighbouring pencil slots of a warp (side 0 and
+// side 1); the self-paired pencils kap = 0 and kap = Po/2 use side 0 alone.
+// After the forward transforms each pencil leaves its spectrum in its own
+// exchange buffer, and each side reads its partner's values Z_m there:
+//   side 0 (kap):       Y[kc] = A[kc] Z[kc] + D[kc] conj(Z_m[pi(kc)])
+//   side 1 (Po - kap):  Y[j]  = conj(A[pi(j)]) Z[j] + conj(D[pi(j)]) conj(Z_m[pi(j)])
+// with pi(kc) = Pc - 1 - kc (kap != 0) or -kc mod Pc (kap = 0), and (A, D)
+// of the stored pencil kap; the adjoint conjugates (A, D) once more.
+template <int N>
+__global__ void __launch_bounds__(kAT, 2) k_l1_center(const L1PassArgs a) {
+  constexpr int G = P2<N>::G, R1 = P2<N>::R1, PPW = 32 / G, UPW = PPW / 2, Pc = 2 * N;
+  static_assert(PPW >= 2, "a unit takes two pencil slots of one warp");
+  extern __shared__ __align__(16) unsigned char asmem[];
+  const Tabs<N> t = tabs_at<N>(asmem);
+  float4* xb = reinterpret_cast<float4*>(asmem + Tabs<N>::kBytes);
+  tabs_build<N>(t, g_tw512);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pen = lane / G, g = lane % G, side = pen & 1;
+  float4* buf = xb + warp * XB<N>::kWarp + pen * XB<N>::kPen;
+  const float4* pbuf = xb + warp * XB<N>::kWarp + (pen ^ 1) * XB<N>::kPen;
+  const L1Spec& d = a.sd;
+  const unsigned Po = static_cast<unsigned>(d.Po), R = static_cast<unsigned>(d.R);
+  const unsigned total = static_cast<unsigned>(a.npen);            // units in the wave
+  const unsigned per_cta = (kAT / 32) * UPW;
+  const float invQ = ldexpf(1.f, -a.lgQ);
+  const bool conj_spec = a.sconj < 0.f;
+  for (unsigned u0 = blockIdx.x * per_cta; u0 < total; u0 += gridDim.x * per_cta) {
+    const unsigned u = u0 + warp * UPW + (pen >> 1);
+    const bool valid = u < total;
+    const unsigned wv = valid ? u / R : 0u, r = valid ? u - wv * R : 0u;
+    const bool self = (r == 0u) || (r == Po / 2);
+    const bool act = valid && (side == 0 || !self);
+    const unsigned kap = side == 0 ? r : (self ? r : Po - r);
+    const long long o = (static_cast<long long>(kap & (d.P0 - 1)) * d.Pm) + (kap >> a.lgP0);
+    float2* base = a.grid + (static_cast<long long>(wv) * Po + o) * Pc;
+    float2 lo[R1], hi[R1];
+#pragma unroll
+    for (int s = 0; s < R1; ++s) {
+      const int j = g + s * G;
+      lo[s] = act ? *HND_G(&base[j]) : make_float2(0.f, 0.f);
+      hi[s] = act ? *HND_G(&base[j + N]) : make_float2(0.f, 0.f);
+    }
+    cp x[R1];
+    full_fwd<N>(lo, hi, x, g, buf, 0, t, 0u);
+    // every pencil's spectrum into its exchange buffer, slot f holding
+    // (Z[2f], Z[2f + 1])
+    __syncwarp();
+#pragma unroll
+    for (int s = 0; s < R1; ++s)
+      *HND_S(&buf[swz(spec_idx<N>(g, s))]) = make_float4(x[s].re.x, x[s].re.y, x[s].im.x, x[s].im.y);
+    __syncwarp();
+    const float4* src = self ? buf : pbuf;
+    const long long pg = a.v0 + wv;                 // the channel pair
+    const long long smp = pg / a.H, jj = pg - smp * a.H;
+    const float4* row = a.spec + smp * a.sbs4 + jj * d.per_pair() + static_cast<long long>(r) * Pc;
+    const bool flip = (side == 1) != conj_spec;
+#pragma unroll
+    for (int s = 0; s < R1; ++s) {
+      const int f = spec_idx<N>(g, s);
+      // partner values at pi(2f) and pi(2f + 1)
+      float2 zm0, zm1;
+      if (r == 0u && side == 0) {
+        const float4 pa = *HND_S(&src[swz((N - f) & (N - 1))]);     // -2f: slot (N - f) mod N, path 0
+        const float4 pb = *HND_S(&src[swz(N - 1 - f)]);             // -(2f + 1): slot N - 1 - f, path 1
+        zm0 = make_float2(pa.x, pa.z);
+        zm1 = make_float2(pb.y, pb.w);
+      } else {
+        const float4 pb = *HND_S(&src[swz(N - 1 - f)]);             // Pc - 1 - 2f: path 1; Pc - 2 - 2f: path 0
+        zm0 = make_float2(pb.y, pb.w);
+        zm1 = make_float2(pb.x, pb.z);
+      }
+      // (A, D) of the stored pencil at kc (side 0) or pi(kc) (side 1)
+      float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
+      if (act) {
+        s0 = __ldg(HND_G(row + (side == 0 ? 2 * f : Pc - 1 - 2 * f)));
+        s1 = __ldg(HND_G(row + (side == 0 ? 2 * f + 1 : Pc - 2 - 2 * f)));
+      }
+      if (flip) {
+        s0.y = -s0.y;
+        s0.w = -s0.w;
+        s1.y = -s1.y;
+        s1.w = -s1.w;
+      }
+      // Y = A Z + D conj(Z_m)
+      const float2 z0 = make_float2(x[s].re.x, x[s].im.x), z1 = make_float2(x[s].re.y, x[s].im.y);
+      const float y0r = s0.x * z0.x - s0.y * z0.y + s0.z * zm0.x + s0.w * zm0.y;
+      const float y0i = s0.x * z0.y + s0.y * z0.x + s0.w * zm0.x - s0.z * zm0.y;
+      const float y1r = s1.x * z1.x - s1.y * z1.y + s1.z * zm1.x + s1.w * zm1.y;
+      const float y1i = s1.x * z1.y + s1.y * z1.x + s1.w * zm1.x - s1.z * zm1.y;
+      x[s] = {make_float2(y0r, y1r), make_float2(y0i, y1i)};
+    }
+    __syncwarp();                                   // the partner is done with this buffer
+    l1_full_inv<N>(x, lo, hi, g, buf, t);
+    // conjugate twiddle of the previous level: conj W_Q^{k e}, k = o mod twP,
+    // e the element's index along this (last) axis
+    const unsigned k = static_cast<unsigned>(o & (a.twP - 1));
+    const float2 wk = l1_conj(l1_w(k * N, invQ));
+#pragma unroll
+    for (int s = 0; s < R1; ++s) {
+      const unsigned j = g + s * G;
+      const float2 w0 = l1_conj(l1_w(k * j, invQ));
+      const float2 w1 = cmul1(w0, wk);
+      if (act) {
+        *HND_G(&base[j]) = cmul1(lo[s], w0);
+        *HND_G(&base[j + N]) = cmul1(hi[s], w1);
       }
     }
   }

@@ -130,8 +130,8 @@ extern "C" HYENA_ND_API hyena_nd_status hyena_nd_fftconv_batched_static(
 
   const bool long1d = p->ndim == 1 && n[0] > 256;
   const bool fused = (p->ndim == 1 && !long1d) || hnd::fused_2d(p->ndim, n);
-  // scratch per (b, c) volume: packed row spectra (multi-pass) or the padded
-  // split grid (long 1D)
+  // scratch per wave item: the packed row spectra of a (b, c) volume
+  // (multi-pass) or the padded split grid of a channel pair (long 1D)
   const size_t per_pair = static_cast<size_t>(long1d ? 16 : 8) * static_cast<size_t>(L);
   if (!fused && per_pair > kStaticScratchBytes) return HYENA_ND_ERR_WORKSPACE_TOO_SMALL;
 
@@ -156,11 +156,7 @@ extern "C" HYENA_ND_API hyena_nd_status hyena_nd_fftconv_batched_static(
 
   hnd::BoundsList bl;
   for (const void* ptr : {q, k, v, static_cast<const void*>(y)}) bl.add(ptr, act_bytes);
-  long long spec_per = 1;     // complex values per channel spectrum (library order)
-  if (p->ndim == 1) spec_per = long1d ? 2LL * n[0] : n[0] + 1LL;
-  else if (p->ndim == 2) spec_per = (n[1] + 1LL) * 2 * n[0];
-  else spec_per = (n[2] + 1LL) * 4 * n[0] * n[1];
-  const size_t spec_bytes = static_cast<size_t>(spec_per) * 8 * static_cast<size_t>(p->C);
+  const size_t spec_bytes = hnd::spectrum_set_bytes(p->ndim, n, p->C);
   bl.add(spectrum, spectrum_batch_stride > 0
                        ? static_cast<size_t>(p->B - 1) * static_cast<size_t>(spectrum_batch_stride) + spec_bytes
                        : spec_bytes);
@@ -171,7 +167,8 @@ extern "C" HYENA_ND_API hyena_nd_status hyena_nd_fftconv_batched_static(
   int launches = 0;
   const long long pairs = p->B * p->C;
   if (long1d) {
-    const long long wave = hnd::balanced_wave(pairs, p->B, per_pair, kStaticScratchBytes, false);
+    const long long grids = p->B * ((p->C + 1) / 2);
+    const long long wave = hnd::balanced_wave(grids, 1, per_pair, kStaticScratchBytes, false);
     e = hnd::launch_long1d(a, zt, wave, &launches);
   } else if (p->ndim == 1) {
     e = hnd::launch_rows1d(a);

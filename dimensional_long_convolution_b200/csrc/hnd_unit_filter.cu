@@ -164,6 +164,14 @@ static cudaError_t l1_inv_conj(float2* grid, const L1Split& sp, long long ngrids
 
 int long1d_launches_per_transform(int n) { return 2 * long1d_split(n).m - 1; }
 
+size_t spectrum_set_bytes(int ndim, const int* n, long long C) {
+  if (ndim == 1 && n[0] > 256) {
+    const L1Split sp = long1d_split(n[0]);
+    return static_cast<size_t>(hnd2::l1_spec_of(sp.m, sp.P).per_pair()) * 16 * static_cast<size_t>((C + 1) / 2);
+  }
+  return static_cast<size_t>(spec_per_channel(make_dims(ndim, n))) * 8 * static_cast<size_t>(C);
+}
+
 cudaError_t launch_fft_axes(float2* grid, int ndim, const int* n, long long ngrids, cudaStream_t st,
                             bool skip_zero) {
   long long gsz = 1;
@@ -202,8 +210,9 @@ cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, i
     gsz *= 2 * n[a];
     noff *= 2 * n[a] - 1;
   }
-  // 2D and 3D: two channels per complex grid (the kernel values are real)
-  const int pair = ndim >= 2 ? 1 : 0;
+  // 2D, 3D and long 1D: two channels per complex grid (the kernel values are real)
+  const bool long1d = ndim == 1 && n[0] > 256;
+  const int pair = ndim >= 2 || long1d ? 1 : 0;
   const int ngrids = pair ? (nc + 1) / 2 : nc;
   cudaError_t e = cudaMemsetAsync(grid, 0, sizeof(float2) * gsz * ngrids, st);
   if (e != cudaSuccess) return e;
@@ -234,10 +243,12 @@ cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, i
       : HP <= 96 ? filter_mlp_go<96>(fa, noff, st)
                  : filter_mlp_go<128>(fa, noff, st);
   if (e != cudaSuccess) return e;
-  if (ndim == 1 && n[0] > 256) {
-    if ((e = l1_fwd(grid, long1d_split(n[0]), nc, st)) != cudaSuccess) return e;
-    hnd2::k_l1_spec_store<<<grid_for(gsz * nc, 256), 256, 0, st>>>(
-        grid, static_cast<float2*>(spectrum), gsz, c0, nc, static_cast<float>(1.0 / static_cast<double>(gsz)));
+  if (long1d) {
+    const L1Split sp = long1d_split(n[0]);
+    if ((e = l1_fwd(grid, sp, ngrids, st)) != cudaSuccess) return e;
+    const hnd2::L1Spec d1 = hnd2::l1_spec_of(sp.m, sp.P);
+    hnd2::k_l1_pair_store<<<grid_for(d1.per_pair() * ngrids, 256), 256, 0, st>>>(
+        grid, static_cast<float4*>(spectrum), d1, c0 / 2, ngrids, static_cast<float>(1.0 / static_cast<double>(gsz)));
     return cudaGetLastError();
   }
   e = launch_fft_axes(grid, ndim, n, ngrids, st);
@@ -311,13 +322,13 @@ cudaError_t launch_spec_convert(int ndim, const int* n, long long C, const void*
                                 cudaStream_t st) {
   if (ndim == 1 && n[0] > 256) {
     const L1Split sp = long1d_split(n[0]);
+    const hnd2::L1Spec d1 = hnd2::l1_spec_of(sp.m, sp.P);
     if (to_natural)
       hnd2::k_l1_spec_export<<<grid_for((n[0] + 1LL) * C, 256), 256, 0, st>>>(
-          static_cast<const float2*>(src), static_cast<float2*>(dst), n[0], sp.P[0], sp.P[1], sp.P[2], C);
+          static_cast<const float4*>(src), static_cast<float2*>(dst), n[0], d1, C);
     else
-      hnd2::k_l1_spec_import<<<grid_for(2LL * n[0] * C, 256), 256, 0, st>>>(
-          static_cast<const float2*>(src), static_cast<float2*>(dst), n[0], sp.P[0], sp.P[1], sp.P[2], C,
-          n[0] + 1LL, 1.f);
+      hnd2::k_l1_spec_import<<<grid_for(d1.per_pair() * ((C + 1) / 2), 256), 256, 0, st>>>(
+          static_cast<const float2*>(src), static_cast<float4*>(dst), n[0], d1, C, n[0] + 1LL);
     return cudaGetLastError();
   }
   const SpecDims d = make_dims(ndim, n);

@@ -1,4 +1,4 @@
-// Long 1D tier: one convolution over all volumes in waves, each wave the
+// Long 1D tier: one convolution over all channel pairs in waves, each wave the
 // 2m - 1 fused passes of hnd_long1d.cuh over the split P = 2n = P0 P1 (P2).
 #include "hnd_launch.h"
 #include "hnd_host_util.h"
@@ -20,6 +20,31 @@ cudaError_t l1_pass_go(const hnd2::L1PassArgs& a, cudaStream_t st) {
   if (blocks < 1) blocks = 1;
   kern<<<static_cast<unsigned>(blocks), hnd2::kAT, sm, st>>>(a);
   return cudaGetLastError();
+}
+
+template <int N>
+cudaError_t l1_center_go(const hnd2::L1PassArgs& a, cudaStream_t st) {
+  auto kern = hnd2::k_l1_center<N>;
+  const size_t sm = hnd2::AxisSmem<N>::kBytes;
+  cudaError_t e = ensure_smem(kern, sm);
+  if (e != cudaSuccess) return e;
+  const long long per_cta = (hnd2::kAT / 32) * (32 / hnd2::P2<N>::G / 2);
+  long long blocks = (a.npen + per_cta - 1) / per_cta;
+  if (blocks > 148LL * 16) blocks = 148LL * 16;
+  if (blocks < 1) blocks = 1;
+  kern<<<static_cast<unsigned>(blocks), hnd2::kAT, sm, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t l1_center(int N, const hnd2::L1PassArgs& a, cudaStream_t st) {
+  switch (N) {
+    case 16: return l1_center_go<16>(a, st);
+    case 32: return l1_center_go<32>(a, st);
+    case 64: return l1_center_go<64>(a, st);
+    case 128: return l1_center_go<128>(a, st);
+    case 256: return l1_center_go<256>(a, st);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 template <int KIND, class T, bool DUAL>
@@ -44,7 +69,9 @@ template <class T>
 cudaError_t long1d_t(const ConvArgs& c, float2* grid, long long wave, int* launches) {
   const L1Split sp = long1d_split(c.n[0]);
   const int m = sp.m;
-  const long long P = 2LL * c.n[0], nv = static_cast<long long>(c.B) * c.C;
+  const long long P = 2LL * c.n[0];
+  const int H = (c.C + 1) / 2;
+  const long long nunits = static_cast<long long>(c.B) * H;      // channel-pair grids
   long long stride[3] = {1, 1, 1};
   for (int a = m - 2; a >= 0; --a) stride[a] = stride[a + 1] * sp.P[a + 1];
   hnd2::L1PassArgs a{};
@@ -52,19 +79,22 @@ cudaError_t long1d_t(const ConvArgs& c, float2* grid, long long wave, int* launc
   a.P = P;
   a.lgP = ilog2(P);
   a.n = c.n[0];
+  a.H = H;
   a.a = c.k;
   a.b = c.v;
   a.q = c.q;
   a.y = c.y;
   a.g2 = c.g2;
   a.y2 = c.y2;
-  a.spec = static_cast<const float2*>(c.spec);
-  a.sbs = c.sbs;
+  a.spec = static_cast<const float4*>(c.spec);
+  a.sbs4 = c.sbs / 2;
+  a.sd = hnd2::l1_spec_of(m, sp.P);
+  a.lgP0 = ilog2(sp.P[0]);
   a.sconj = c.sconj;
   a.C = c.C;
   cudaError_t e = cudaSuccess;
-  for (long long v0 = 0; v0 < nv && e == cudaSuccess; v0 += wave) {
-    const long long cnt = nv - v0 < wave ? nv - v0 : wave;
+  for (long long v0 = 0; v0 < nunits && e == cudaSuccess; v0 += wave) {
+    const long long cnt = nunits - v0 < wave ? nunits - v0 : wave;
     a.v0 = v0;
     auto set_axis = [&](int ax) {
       a.stride = stride[ax];
@@ -82,13 +112,15 @@ cudaError_t long1d_t(const ConvArgs& c, float2* grid, long long wave, int* launc
       a.lgQ = ilog2(a.twQ);
       e = l1_pass<hnd2::kFwdMid, float, false>(sp.P[1] / 2, a, c.stream);
     }
-    // spectrum product on the last axis, with the inverse transform back
+    // spectrum product on the last axis, pencil pairs, with the inverse
+    // transform back
     if (e == cudaSuccess) {
       set_axis(m - 1);
+      a.npen = cnt * a.sd.R;
       a.twP = sp.P[m - 2];
       a.twQ = static_cast<long long>(sp.P[m - 2]) * sp.P[m - 1];
       a.lgQ = ilog2(a.twQ);
-      e = l1_pass<hnd2::kCenter, float, false>(sp.P[m - 1] / 2, a, c.stream);
+      e = l1_center(sp.P[m - 1] / 2, a, c.stream);
     }
     if (e == cudaSuccess && m == 3) {
       set_axis(1);

@@ -122,8 +122,13 @@ typedef struct {
   int window;
 } hyena_nd_filter;
 
-/* Size in bytes of the spectrum buffer for `p` (C channels of
- * prod_{a<d-1} P_a * (P_d/2 + 1) complex64 values; 2n for the long 1D tier).
+/* Size in bytes of the spectrum buffer for `p`: C channels of
+ * prod_{a<d-1} P_a * (P_d/2 + 1) complex64 values.  The long 1D tier
+ * (n > 256) stores channel pairs instead: for channels 2j and 2j + 1 of the
+ * split 2n = Po Pc (Pc the last factor of the split), the two complex64
+ * values A = (K_a + K_b)/2 and D = (K_a - K_b)/2 at the (Po/2 + 1) Pc
+ * frequencies whose first-level index is at most Po/2 (the rest follow by
+ * Hermitian symmetry); a missing last channel (odd C) counts as zero.
  * 0 if `p` is invalid or unsupported. */
 HYENA_ND_API size_t hyena_nd_spectrum_bytes(const hyena_nd_problem* p);
 
@@ -168,7 +173,8 @@ typedef enum {
 
 typedef struct {
   hyena_nd_tier tier;
-  int64_t wave;           /* volumes per wave of the multi-pass tiers (0 for single-launch tiers) */
+  int64_t wave;           /* volumes per wave of the multi-pass tiers (long 1D: channel-pair grids;
+                             0 for single-launch tiers) */
   int64_t waves;          /* waves per convolution (1 for single-launch tiers) */
   int launches;           /* kernel launches per convolution */
   int split_levels;       /* long 1D: factors of the split 2n = P0 P1 (P2) (0 otherwise) */
@@ -321,9 +327,10 @@ HYENA_ND_API hyena_nd_status hyena_nd_fftconv_batched_static(const hyena_nd_prob
  * natural array is DFT(wrap-placed K) / prod(P)).  The library-order buffer
  * holds hyena_nd_spectrum_bytes(p) bytes, the natural one
  * 8 C prod_{a<d} P_a (n_d + 1) bytes (the same number except for the long 1D
- * tier, whose library order keeps all 2n frequencies); both are device memory
- * and may not overlap.  The import takes the other half by Hermitian symmetry
- * where the library order keeps it. */
+ * tier, whose library order is the channel-pair layout described at
+ * hyena_nd_spectrum_bytes); both are device memory and may not overlap.  The
+ * import takes the other half by Hermitian symmetry where the library order
+ * keeps it. */
 HYENA_ND_API hyena_nd_status hyena_nd_spectrum_export(const hyena_nd_problem* p, const void* spectrum,
                                          void* natural_c64, void* cuda_stream);
 HYENA_ND_API hyena_nd_status hyena_nd_spectrum_import(const hyena_nd_problem* p, const void* natural_c64,

@@ -156,13 +156,33 @@ def test_workspace_covers_the_kernel_gradient():
         assert H.workspace_bytes(p) >= (wl.B + 1) * P * 8
 
 
+def _long_1d_split(n):
+    """Factors of 2n: two levels up to 2^18, else three, each at most 2^9,
+    the larger shares first."""
+    lg = (2 * n).bit_length() - 1
+    m = 2 if lg <= 18 else 3
+    out, left = [], lg
+    for a in range(m):
+        share = -(-left // (m - a))
+        out.append(1 << share)
+        left -= share
+    return out
+
+
 @pytest.mark.parametrize("n,B,C", [(512, 2, 3), (4096, 1, 8), (131072, 2, 100), (1 << 23, 1, 2), (1 << 26, 1, 1)])
 def test_long_1d_sizes(n, B, C):
-    """Long 1D grids keep all 2n frequencies in the library order; the
-    workspace holds at least one volume's padded grid (one wave) and the
-    kernel-gradient grids of one channel; the natural export stays n + 1."""
+    """Long 1D spectra are stored per channel pair: (A, D) = ((K_a + K_b)/2,
+    (K_a - K_b)/2) as two complex64 values for the pencils kap = 0 .. Po/2 of
+    the split (Po = P / Pc, Pc the last factor), i.e. about half of the 2n
+    frequencies; the workspace holds at least one pair's padded grid (one
+    wave) and the kernel-gradient grids of one channel; the natural export
+    stays n + 1."""
     p = H.problem((n,), B, C, H.F32)
-    assert H.spectrum_bytes(p) == C * 2 * n * 8
+    sp = _long_1d_split(n)
+    assert int(np.prod(sp)) == 2 * n and max(sp) <= 512
+    Pc, Po = sp[-1], 2 * n // sp[-1]
+    assert H.spectrum_bytes(p) == (C + 1) // 2 * (Po // 2 + 1) * Pc * 16
+    assert H.spectrum_bytes(p) == (C + 1) // 2 * (2 * n * 8 + 16 * Pc)   # half the frequencies, two values each
     ws = H.workspace_bytes(p)
     assert ws >= 256 + max(2 * n * 8, (B + 1) * 2 * n * 8)
     # the largest of: a 96 MiB conv wave, 256 MiB of kernel-gradient grids,
@@ -171,13 +191,14 @@ def test_long_1d_sizes(n, B, C):
 
 
 def test_long_1d_spectrum_conversion_uses_the_natural_size():
-    """The natural half spectrum of a long 1D grid is shorter than the library
-    order; the overlap check measures each buffer by its own size."""
+    """The natural half spectrum of a long 1D grid and the library's pair
+    layout differ in size; the overlap check measures each buffer by its own
+    size."""
     n, C = 1024, 2
     p = H.problem((n,), 1, C)
     nat = C * (n + 1) * 8
     nat16 = (nat + 15) // 16 * 16
-    assert H.spectrum_bytes(p) == C * 2 * n * 8
+    assert H.spectrum_bytes(p) == (64 // 2 + 1) * 32 * 16     # 2048 = 64 x 32, one channel pair
     assert H.spectrum_import(p, A, A + nat16 - 16, 0) == H.ERR_INVALID_ARG
     assert H.spectrum_export(p, A + nat16 - 16, A, 0) == H.ERR_INVALID_ARG
 
@@ -225,9 +246,11 @@ def test_plan_info_of_the_benchmark_grids(i, tier, waves, launches, streams):
 
 
 @pytest.mark.parametrize("n,B,C,levels,split,waves", [
-    (256, 1, 4, 0, [1, 1, 1], 1), (512, 2, 3, 2, [32, 32, 1], 1), (1 << 17, 1, 60, 2, [512, 512, 1], 2),
-    (1 << 20, 1, 64, 3, [128, 128, 128], 11), (1 << 26, 1, 1, 3, [512, 512, 512], 1)])
+    (256, 1, 4, 0, [1, 1, 1], 1), (512, 2, 3, 2, [32, 32, 1], 1), (1 << 17, 1, 60, 2, [512, 512, 1], 1),
+    (1 << 20, 1, 64, 3, [128, 128, 128], 6), (1 << 26, 1, 1, 3, [512, 512, 512], 1)])
 def test_plan_info_of_long_1d(n, B, C, levels, split, waves):
+    """Long 1D waves count channel-pair grids (8 bytes per padded point each,
+    96 MiB per wave): 2^20 tokens, C = 64 -> 32 grids of 16 MiB -> 6 waves."""
     info = H.plan_info(H.problem((n,), B, C))
     assert info["split_levels"] == levels and info["split"] == split
     assert info["tier"] == ("long_1d" if n > 256 else "rows_1d")

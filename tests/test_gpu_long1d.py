@@ -27,9 +27,11 @@ def _f64(a):
 
 
 def _waves(n, B, C):
+    """Channels 2j and 2j + 1 of a sample share one padded complex grid."""
     per = 2 * n * 8
-    w = max(1, min(WAVE_BYTES // per, B * C))
-    return -(-(B * C) // w)
+    grids = B * ((C + 1) // 2)
+    w = max(1, min(WAVE_BYTES // per, grids))
+    return -(-grids // w)
 
 
 def _per_wave(n):
@@ -94,8 +96,11 @@ def test_long1d_filter_spectrum(dims, C):
 
 
 def test_long1d_import_export_roundtrip_and_conv():
-    """A random kernel's natural half spectrum goes in, comes back unchanged,
-    and drives a convolution equal to the oracle's with that kernel."""
+    """A random kernel's natural half spectrum goes in, comes back unchanged
+    up to the two float32 roundings of the channel-pair layout ((K_a + K_b)/2
+    and (K_a - K_b)/2 in, their sum and difference out), and drives a
+    convolution equal to the oracle's with that kernel.  C = 3 leaves the
+    second pair half empty."""
     dims, B, C = (1024,), 2, 3
     rng = np.random.default_rng(8)
     K = rng.standard_normal((C, 2 * dims[0] - 1)) / 64.0
@@ -105,7 +110,7 @@ def test_long1d_import_export_roundtrip_and_conv():
     op = make_op(wl)
     op.import_spectrum(torch().from_numpy(nat.astype(np.complex64)))
     back = to_host(op.export_spectrum())
-    assert np.max(np.abs(back - nat.astype(np.complex64))) <= 1e-7 * np.max(np.abs(nat))
+    assert np.max(np.abs(back - nat.astype(np.complex64))) <= 4e-7 * np.max(np.abs(nat))
     got, _ = run(inp, op=op)
     want = O.conv_direct(inp.as_f64("q"), inp.as_f64("k"), inp.as_f64("v"), K, dims)
     assert O.rel_l2(got, want) <= TOL["f32"]
