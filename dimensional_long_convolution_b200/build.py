@@ -21,6 +21,7 @@ import glob
 import os
 import shutil
 import subprocess
+import time
 import sys
 
 PKG = os.path.dirname(os.path.abspath(__file__))
@@ -71,6 +72,7 @@ def build(force: bool = False, extra_flags=None, verbose: bool = False, jobs: in
     bdir = BUILD_BOUNDS if bounds else BUILD
     if not force and up_to_date(lib):
         return lib
+    t0 = time.time()
     subprocess.check_call([sys.executable, os.path.join(CSRC, "gen_tables.py"), os.path.join(CSRC, "hnd_twiddles.inc")])
     os.makedirs(bdir, exist_ok=True)
     flags = NVCC_FLAGS + list(extra_flags or []) + (BOUNDS_FLAGS if bounds else [])
@@ -93,6 +95,9 @@ def build(force: bool = False, extra_flags=None, verbose: bool = False, jobs: in
     cmd = [exe] + ARCH + (["-rdc=true"] if bounds else []) + ["-shared", "-o", tmp] + objs + ["-lcudart"]
     subprocess.check_call(cmd)
     os.replace(tmp, lib)
+    # stamp the library with the build's start, so that a source edited while
+    # it compiled leaves it out of date
+    os.utime(lib, (t0, t0))
     return lib
 
 

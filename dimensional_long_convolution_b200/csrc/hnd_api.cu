@@ -100,20 +100,26 @@ constexpr size_t kWaveBudget = size_t(HND_WAVE_MB) << 20;
 constexpr int kWaveStreams = HND_STREAMS;
 static_assert(kWaveStreams >= 1 && kWaveStreams <= hnd::SideStream::kMax, "streams per convolution");
 #ifndef HND_FILTER_MB
-#define HND_FILTER_MB 256
+#define HND_FILTER_MB 1024
 #endif
 #ifndef HND_FILTER_MAXC
 #define HND_FILTER_MAXC 128
 #endif
 // filter grids per channel chunk: each chunk evaluates the hidden layer once
 // per offset, so fewer, larger chunks save that work at the cost of workspace
+// (3D 128^3, C = 32: 28.0 / 18.7 / 14.7 ms per call at 256 / 512 / 1024 MiB;
+// only the filter call needs this workspace)
 constexpr size_t kFilterBudget = size_t(HND_FILTER_MB) << 20;
 constexpr int kFilterMaxChunk = HND_FILTER_MAXC;
-constexpr size_t kKgradBudget = size_t(256) << 20;    // kernel-gradient grids per channel chunk (the filter call already needs 256 MiB)
+constexpr size_t kKgradBudget = size_t(256) << 20;    // kernel-gradient grids per channel chunk
 #ifndef HND_L1_WAVE_MB
-#define HND_L1_WAVE_MB 96
+#define HND_L1_WAVE_MB 48
 #endif
-constexpr size_t kL1WaveBudget = size_t(HND_L1_WAVE_MB) << 20;   // long 1D grids per wave
+// long 1D grids in flight: with several waves, three streams of 16 MiB each,
+// so that a wave's grid stays in L2 across its passes (measured on 2^20
+// tokens, C = 64: 1.96 ms against 2.09 with 3 x 32 MiB and 2.24 with one
+// stream of 96 MiB)
+constexpr size_t kL1WaveBudget = size_t(HND_L1_WAVE_MB) << 20;
 
 enum Tier { kRows1D = 0, kFused2D = 1, kMulti2D = 2, kMulti3D = 3, kLong1D = 4 };
 
@@ -185,7 +191,16 @@ hyena_nd_status make_plan(const hyena_nd_problem* p, Plan* pl) {
     const size_t per_grid = static_cast<size_t>(8) * static_cast<size_t>(pl->gsz);
     const long long grids = p->B * ((p->C + 1) / 2);
     pl->wave = hnd::balanced_wave(grids, 1, per_grid, kL1WaveBudget, false);
-    ws_conv = per_grid * static_cast<size_t>(pl->wave);
+    pl->streams = 1;
+    if (kWaveStreams > 1 && pl->wave < grids && per_grid * kWaveStreams <= kL1WaveBudget) {
+      // several waves of grids small enough to share the budget: alternate
+      // streams, each wave in its share
+      pl->wave = hnd::balanced_wave(grids, 1, per_grid, kL1WaveBudget / kWaveStreams, false);
+      const long long waves = (grids + pl->wave - 1) / pl->wave;
+      pl->streams = static_cast<int>(waves < kWaveStreams ? waves : kWaveStreams);
+    }
+    pl->wave_bytes = (per_grid * static_cast<size_t>(pl->wave) + 255) / 256 * 256;
+    ws_conv = pl->wave_bytes * static_cast<size_t>(pl->streams);
   } else if (p->ndim == 1) {
     pl->tier = kRows1D;
   } else if (hnd::fused_2d(p->ndim, pl->n)) {
@@ -259,17 +274,18 @@ size_t spectrum_span(const Plan& pl, int64_t sbs) {
 // spectrum) on the plan's tier; adds the kernel launches to *launches.
 cudaError_t run_conv(const Plan& pl, const hnd::ConvArgs& a, void* ws, int* launches) {
   cudaError_t e = cudaSuccess;
-  if (pl.tier == kLong1D) {
-    e = hnd::launch_long1d(a, reinterpret_cast<float2*>(static_cast<char*>(ws) + kStatusBytes), pl.wave, launches);
-  } else if (pl.tier == kRows1D) {
+  if (pl.tier == kRows1D) {
     e = hnd::launch_rows1d(a);
     *launches += 1;
   } else if (pl.tier == kFused2D) {
     e = pl.bf16 ? hnd::launch_fused2d_bf16(a) : hnd::launch_fused2d_f32(a);
     *launches += 1;
   } else {
+    // multi-pass tiers: waves of (b, c) volumes, or of channel-pair grids in
+    // the long 1D tier
     char* zbase = static_cast<char*>(ws) + kStatusBytes;
-    const long long pairs = pl.B * pl.C;
+    const bool l1 = pl.tier == kLong1D;
+    const long long pairs = l1 ? pl.B * ((pl.C + 1) / 2) : pl.B * pl.C;
     const int nl = pl.n[pl.ndim - 1];
     const int rp_total = static_cast<int>(pl.L / nl / 2);
     hnd::SideStream* side = nullptr;
@@ -295,15 +311,24 @@ cudaError_t run_conv(const Plan& pl, const hnd::ConvArgs& a, void* ws, int* laun
       hnd::ConvArgs aw = a;
       aw.stream = ns > 1 ? stream_of(lane) : a.stream;
       float2* zt = reinterpret_cast<float2*>(zbase + static_cast<size_t>(lane) * pl.wave_bytes);
-      e = hnd::launch_rowfwd(aw, nl, zt, ord0, np, rp_total);
+      if (l1) {
+        e = hnd::launch_long1d_wave(aw, zt, ord0, np, 0, launches);
+      } else {
+        e = hnd::launch_rowfwd(aw, nl, zt, ord0, np, rp_total);
+        *launches += 1;
+      }
       if (e == cudaSuccess && ns > 1 && w + 1 < ns) {
-        // the next stream's first wave starts after this one's forward rows
+        // the next stream's first wave starts after this one's first stage
         e = cudaEventRecord(side->stagger[lane], aw.stream);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(side->s[lane + 1], side->stagger[lane], 0);
       }
+      if (l1) {
+        if (e == cudaSuccess) e = hnd::launch_long1d_wave(aw, zt, ord0, np, 1, launches);
+        continue;
+      }
       if (e == cudaSuccess) e = pl.tier == kMulti2D ? hnd::launch_mid1(aw, zt, ord0, np) : hnd::launch_mid2(aw, zt, ord0, np);
       if (e == cudaSuccess) e = hnd::launch_rowinv(aw, nl, zt, ord0, np, rp_total);
-      *launches += 3;
+      *launches += 2;
     }
     for (int j = 1; j < ns; ++j) {
       // join: the caller's stream waits for every side stream's last wave
@@ -638,6 +663,9 @@ hyena_nd_status hyena_nd_filter_spectrum_film(const hyena_nd_problem* p, const h
     fl.gamma = gamma + b * f->hidden;
     fl.beta = beta + b * f->hidden;
     void* sb = static_cast<char*>(spectrum) + b * spectrum_batch_stride;
+    if (fl.tab && hnd::launch_filter_trig(fl, pl.ndim, pl.n, const_cast<float*>(fl.tab),
+                                          static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
+      return HYENA_ND_ERR_CUDA;
     cudaError_t e = filter_all_chunks(pl, fl, sb, ws, static_cast<cudaStream_t>(cuda_stream));
     if (e != cudaSuccess) return HYENA_ND_ERR_CUDA;
   }

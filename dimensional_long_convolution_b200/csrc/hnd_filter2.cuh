@@ -49,7 +49,20 @@ struct FilterMlpArgs {
 // axis a's table at HP * sum_{b<a} (2 n_b - 1), h-major.  The hidden unit of
 // offset t is then sin(b1 + T_0[t_0] + T_1[t_1] + T_2[t_2]) (FiLM applied to
 // the sum): ndim table reads per unit instead of 2 M ndim products.
+// The last axis L = ndim - 1 varies fastest over a tile of offsets, so the
+// sum splits into a row part R = b1 + sum_{a<L} T_a (one value per row of the
+// tile) and T_L, and with FiLM's gamma and beta
+//   sin(gamma (R + T_L) + beta) = sin(A) cos(gamma T_L) + cos(A) sin(gamma T_L),  A = gamma R + beta:
+// sin and cos of gamma T_L follow the tables (k_filter_trig, [HP][E_L] each),
+// sin A and cos A are computed once per row and unit, and each hidden unit of
+// an offset costs two table reads and two products.
 inline long long filter_table_floats(int HP, int ndim, const int* n) {
+  long long e = 0;
+  for (int a = 0; a < ndim; ++a) e += 2LL * n[a] - 1;
+  return (e + 2LL * (2LL * n[ndim - 1] - 1)) * HP;
+}
+// float offset of the sine table of the last axis (the cosine table follows)
+inline __host__ __device__ long long filter_trig_offset(int HP, int ndim, const int* n) {
   long long e = 0;
   for (int a = 0; a < ndim; ++a) e += 2LL * n[a] - 1;
   return e * HP;
@@ -81,15 +94,40 @@ static __global__ void k_filter_tables(const float* __restrict__ W1, int hidden,
   }
 }
 
+// sin and cos of gamma_h T_L[h][t] for the last axis (gamma = 1 without FiLM),
+// by the full-range library sincosf
+static __global__ void k_filter_trig(float* __restrict__ tab, int HP, int hidden, int ndim, int n0, int n1, int n2,
+                                     const float* __restrict__ gamma) {
+  const int nn[3] = {n0, n1, n2};
+  const long long off = filter_trig_offset(HP, ndim, nn);
+  const int E = 2 * nn[ndim - 1] - 1;
+  const float* TL = tab + off - static_cast<long long>(HP) * E;
+  float* S = tab + off;
+  float* Cc = S + static_cast<long long>(HP) * E;
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < HP * E; e += gridDim.x * blockDim.x) {
+    const int h = e / E;
+    float x = *HND_G(&TL[e]);
+    if (gamma && h < hidden) x *= __ldg(HND_G(gamma + h));
+    float sv, cv;
+    sincosf(x, &sv, &cv);
+    *HND_G(&S[e]) = sv;
+    *HND_G(&Cc[e]) = cv;
+  }
+}
+
 // Shared layout (floats), HP = hidden rounded up to a multiple of 32:
 //   [phi[fin][kFO] | w1[fin][HP]] | hid[HP][kFO] | w2[HP][kFC] | b1[HP] | rad[kFO] |
-//   slot[kFO] (int) | tix[3][kFO] (int); the bracketed part only on the feature path
+//   slot[kFO] (int) | tix[3][kFO] (int) | {sA, cA}[HP][kFR] | rtix[2][kFR] (int);
+//   the bracketed part only on the feature path, the braced one only on the
+//   table path
+constexpr int kFR = 12;      // rows of the last axis a tile of kFO offsets can touch (2 n_L - 1 >= 15)
 template <int HP>
 struct FilterSmem {
   static size_t bytes(int fin, bool tab) {
     const size_t feat = tab ? 0 : static_cast<size_t>(fin) * (kFO + HP);
-    return sizeof(float) * (feat + static_cast<size_t>(HP) * kFO + static_cast<size_t>(HP) * kFC + HP + kFO) +
-           sizeof(int) * 4 * kFO;
+    const size_t rows = tab ? 2 * static_cast<size_t>(HP) * kFR : 0;
+    return sizeof(float) * (feat + static_cast<size_t>(HP) * kFO + static_cast<size_t>(HP) * kFC + HP + kFO + rows) +
+           sizeof(int) * (4 * kFO + 2 * kFR);
   }
 };
 
@@ -135,6 +173,9 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
   float* rad = b1 + HP;                      // [kFO]
   int* slot = reinterpret_cast<int*>(rad + kFO);
   int* tix = slot + kFO;                     // [3][kFO]: table column per axis (table path)
+  float* sA = reinterpret_cast<float*>(tix + 3 * kFO);   // [HP][kFR] (table path)
+  float* cA = sA + HP * kFR;
+  int* rtix = reinterpret_cast<int*>(cA + HP * kFR);     // [2][kFR]: the row's columns of axes 0, 1
   const int tid = threadIdx.x;
   // axes as scalars (an unused axis has extent 1 and offset 0)
   const int n0 = a.n[0], n1 = a.ndim > 1 ? a.n[1] : 1, n2 = a.ndim > 2 ? a.n[2] : 1;
@@ -178,9 +219,27 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
     const int s0 = (t0 + P0) % P0, s1 = (t1 + P1) % P1, s2 = (t2 + P2) % P2;
     (*HND_S(&slot[o])) = (s0 * P1 + s1) * P2 + s2;
     if constexpr (TAB) {
-      (*HND_S(&tix[o])) = rep(t0, n0) + n0 - 1;
-      (*HND_S(&tix[kFO + o])) = rep(t1, n1) + n1 - 1;
-      (*HND_S(&tix[2 * kFO + o])) = rep(t2, n2) + n2 - 1;
+      // tix[0]: the tile row of the offset; tix[1]: its last-axis column
+      const int la = a.ndim - 1;
+      const int EL = la == 0 ? E0 : (la == 1 ? E1 : E2);
+      const int tl = la == 0 ? t0 : (la == 1 ? t1 : t2), nl = la == 0 ? n0 : (la == 1 ? n1 : n2);
+      const long long r = e0 + o < noff ? e0 + o : noff - 1;
+      (*HND_S(&tix[o])) = static_cast<int>(r / EL - e0 / EL);
+      (*HND_S(&tix[kFO + o])) = rep(tl, nl) + nl - 1;
+    }
+  }
+  if constexpr (TAB) {
+    // the rows' columns on the axes before the last
+    const int la = a.ndim - 1;
+    const int EL = la == 0 ? E0 : (la == 1 ? E1 : E2);
+    const long long last = (e0 + kFO < noff ? e0 + kFO : noff) - 1;
+    const int nrows = static_cast<int>(last / EL - e0 / EL) + 1;
+    for (int rr = tid; rr < nrows; rr += kFT) {
+      const long long R = e0 / EL + rr;           // row index over the axes before the last
+      const int i0 = la == 2 ? static_cast<int>(R / E1) : static_cast<int>(R);
+      const int i1 = la == 2 ? static_cast<int>(R % E1) : 0;
+      (*HND_S(&rtix[rr])) = rep(i0 - (n0 - 1), n0) + n0 - 1;
+      (*HND_S(&rtix[kFR + rr])) = rep(i1 - (n1 - 1), n1) + n1 - 1;
     }
   }
   if constexpr (!TAB) {
@@ -202,19 +261,40 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
 
   const int og = tid % 32, grp = tid / 32;
   if constexpr (TAB) {
-    // hidden layer from the per-axis tables: thread i -> offset o = i % kFO
-    // (consecutive offsets read consecutive table columns), unit h = i / kFO
-    const int E0t = 2 * n0 - 1, E1t = 2 * n1 - 1, E2t = 2 * n2 - 1;
+    // hidden layer by angle addition over the last axis (see filter_table_floats)
+    const int la = a.ndim - 1;
+    const int EL = la == 0 ? E0 : (la == 1 ? E1 : E2);
+    const long long last = (e0 + kFO < noff ? e0 + kFO : noff) - 1;
+    const int nrows = static_cast<int>(last / EL - e0 / EL) + 1;
     const float* T0 = a.tab;
-    const float* T1 = T0 + static_cast<long long>(HP) * E0t;
-    const float* T2 = T1 + static_cast<long long>(HP) * (a.ndim > 1 ? E1t : 0);
-    for (int i = tid; i < HP * kFO; i += kFT) {
-      const int o = i % kFO, h = i / kFO;
-      float pre = (*HND_S(&b1[h])) + __ldg(HND_G(T0 + h * E0t + (*HND_S(&tix[o]))));
-      if (a.ndim > 1) pre += __ldg(HND_G(T1 + h * E1t + (*HND_S(&tix[kFO + o]))));
-      if (a.ndim > 2) pre += __ldg(HND_G(T2 + h * E2t + (*HND_S(&tix[2 * kFO + o]))));
-      if (a.gamma && h < a.hidden) pre = fmaf(__ldg(HND_G(a.gamma + h)), pre, __ldg(HND_G(a.beta + h)));
-      (*HND_S(&hid[h * kFO + o])) = h < a.hidden ? sine_layer(pre) : 0.f;
+    const float* T1 = T0 + static_cast<long long>(HP) * E0;
+    const int nn[3] = {n0, n1, n2};
+    const float* Sl = a.tab + filter_trig_offset(HP, a.ndim, nn);
+    const float* Cl = Sl + static_cast<long long>(HP) * EL;
+    // sin A, cos A per (unit, row): A = gamma (b1 + sum of the earlier axes) + beta
+    for (int i = tid; i < HP * nrows; i += kFT) {
+      const int h = i / nrows, rr = i % nrows;
+      float A = *HND_S(&b1[h]);
+      if (la >= 1) A += __ldg(HND_G(T0 + h * E0 + (*HND_S(&rtix[rr]))));
+      if (la >= 2) A += __ldg(HND_G(T1 + h * E1 + (*HND_S(&rtix[kFR + rr]))));
+      if (a.gamma && h < a.hidden) A = fmaf(__ldg(HND_G(a.gamma + h)), A, __ldg(HND_G(a.beta + h)));
+      float sv, cv;
+      sincosf(A, &sv, &cv);
+      (*HND_S(&sA[h * kFR + rr])) = sv;
+      (*HND_S(&cA[h * kFR + rr])) = cv;
+    }
+    __syncthreads();
+    // thread -> offset o (consecutive offsets read consecutive table columns),
+    // units h = tid / kFO, + kFT / kFO, ...
+    const int o = tid % kFO;
+    const int rr = *HND_S(&tix[o]), tl = *HND_S(&tix[kFO + o]);
+    for (int h = tid / kFO; h < HP; h += kFT / kFO) {
+      float v = 0.f;
+      if (h < a.hidden) {
+        const long long j = static_cast<long long>(h) * EL + tl;
+        v = fmaf(*HND_S(&sA[h * kFR + rr]), __ldg(HND_G(Cl + j)), *HND_S(&cA[h * kFR + rr]) * __ldg(HND_G(Sl + j)));
+      }
+      (*HND_S(&hid[h * kFO + o])) = v;
     }
   } else {
     // hidden layer: thread (og, hg) computes offsets 4 og .. 4 og + 3 x units hg HG ..

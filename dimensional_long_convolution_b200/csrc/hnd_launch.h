@@ -74,6 +74,9 @@ cudaError_t launch_rowfwd(const ConvArgs& a, int nl, float2* zt, long long ord0,
 cudaError_t launch_rowinv(const ConvArgs& a, int nl, const float2* zt, long long ord0, int np, int rp_total);
 cudaError_t launch_mid1(const ConvArgs& a, float2* zt, long long ord0, int np);
 cudaError_t launch_mid2(const ConvArgs& a, float2* zt, long long ord0, int np);
+// the 3D slab stage per conjugation sign (launch_mid2 picks one by sconj)
+cudaError_t launch_mid2_fwd(const ConvArgs& a, float2* zt, long long ord0, int np);
+cudaError_t launch_mid2_adj(const ConvArgs& a, float2* zt, long long ord0, int np);
 size_t mid2_smem(int n0, int n1, bool* pair_variant);
 
 // Filter spectrum and layout conversion.
@@ -91,6 +94,10 @@ struct FilterLaunch {
 // feature path is used instead), and the launch that fills them.
 long long filter_table_bytes(int hidden, int ndim, const int* n);
 cudaError_t launch_filter_tables(const FilterLaunch& f, int ndim, const int* n, float* tab, cudaStream_t st);
+// The sine and cosine tables of the last axis, scaled by f.gamma (FiLM) when
+// set: launch_filter_tables fills them with f's gamma, and a per-sample
+// gamma refills them with this before that sample's chunks.
+cudaError_t launch_filter_trig(const FilterLaunch& f, int ndim, const int* n, float* tab, cudaStream_t st);
 cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, int c0, int nc, float2* grid,
                                 void* spectrum, cudaStream_t st);
 cudaError_t launch_spec_convert(int ndim, const int* n, long long C, const void* src, void* dst, bool to_natural,
@@ -109,6 +116,10 @@ int long1d_launches_per_transform(int n);
 // Channels 2j and 2j + 1 of a sample share one complex grid; `wave` counts
 // these channel-pair grids (B ceil(C/2) in all).
 cudaError_t launch_long1d(const ConvArgs& a, float2* grid, long long wave, int* launches);
+// One wave of `cnt` channel-pair grids from pair v0 on a.stream: part 0 the
+// first pass, part 1 the remaining 2m - 2, part 2 all 2m - 1.
+cudaError_t launch_long1d_wave(const ConvArgs& a, float2* grid, long long v0, long long cnt, int part,
+                               int* launches);
 // Bytes of one spectrum set in library order (C channels; long 1D: the pair
 // layout of ceil(C/2) channel pairs).
 size_t spectrum_set_bytes(int ndim, const int* n, long long C);

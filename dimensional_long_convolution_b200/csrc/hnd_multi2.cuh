@@ -709,22 +709,44 @@ __device__ __forceinline__ float2 src3_at(const float2* __restrict__ nat, long l
 
 // natural half spectrum [C][2n0][2n1][n2 + 1] (pitch = last-axis length of the
 // source: n2 + 1 for a half spectrum, 2 n2 for a full grid; pair: the filter
-// call's full grids, two channels per grid) -> library order
-static __global__ void k_spec3_in(const float2* __restrict__ nat, float4* __restrict__ out, int n0, int n1, int n2,
-                                  long long C, long long pitch, float scale, int pair = 0) {
-  const long long per = static_cast<long long>(n2 + 1) * 2 * n1 * n0;     // float4 per channel
+// call's full grids, two channels per grid) -> library order.
+// A CTA takes one (c, ky) and kS3 consecutive kx: it reads the z-pencils of
+// those kx (kx adjacent in the source, so every kz row is one contiguous
+// read; the partner values -k form the mirrored contiguous run) into shared
+// memory indexed by the z frequency pair f, then writes the library's n0
+// float4 of each kx in slot order, contiguous.
+constexpr int kS3 = 32;
+__host__ __device__ __forceinline__ size_t spec3_in_smem(int n0) { return sizeof(float4) * n0 * (kS3 + 1); }
+
+static __global__ void __launch_bounds__(256) k_spec3_in(const float2* __restrict__ nat, float4* __restrict__ out,
+                                                         int n0, int n1, int n2, long long C, long long pitch,
+                                                         float scale, int pair = 0) {
+  extern __shared__ __align__(16) float4 ts[];     // [f][kS3 + 1]
   const long long src_per = 4LL * n0 * n1 * pitch;
+  const int nkb = (n2 + 1 + kS3 - 1) / kS3;
+  const long long cta = blockIdx.x;
+  const int kb0 = static_cast<int>(cta % nkb) * kS3;
+  const int ky = static_cast<int>((cta / nkb) % (2 * n1));
+  const long long c = cta / (static_cast<long long>(nkb) * 2 * n1);
+  const int nk = min(kS3, n2 + 1 - kb0);
+  float* tsf = reinterpret_cast<float*>(ts);
+  for (int i = threadIdx.x; i < 2 * n0 * kS3; i += blockDim.x) {
+    const int kz = i / kS3, kb = i % kS3;
+    if (kb >= nk) continue;
+    const float2 v = src3_at(nat, c, src_per, pitch, kz, ky, kb0 + kb, n0, n1, n2, pair);
+    // float4 (S[2f].re, S[2f+1].re, S[2f].im, S[2f+1].im), f = kz / 2
+    float* d = tsf + 4 * ((kz >> 1) * (kS3 + 1) + kb) + (kz & 1);
+    *HND_S(d) = scale * v.x;
+    *HND_S(d + 2) = scale * v.y;
+  }
+  __syncthreads();
   const int G = lanes_of(n0);
-  for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < per * C;
-       e += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long c = e / per, r = e % per;
-    const int kx = static_cast<int>(r / (2LL * n1 * n0));
-    const long long r2 = r % (2LL * n1 * n0);
-    const int ky = static_cast<int>(r2 / n0), m = static_cast<int>(r2 % n0);
+  for (int i = threadIdx.x; i < n0 * kS3; i += blockDim.x) {
+    const int kb = i / n0, m = i % n0;
+    if (kb >= nk) continue;
     const int f = spec_idx_gen(n0, m % G, m / G);
-    const float2 s0 = src3_at(nat, c, src_per, pitch, 2 * f, ky, kx, n0, n1, n2, pair);
-    const float2 s1 = src3_at(nat, c, src_per, pitch, 2 * f + 1, ky, kx, n0, n1, n2, pair);
-    *HND_G(&out[e]) = make_float4(scale * s0.x, scale * s1.x, scale * s0.y, scale * s1.y);
+    const long long e = ((c * (n2 + 1) + kb0 + kb) * (2LL * n1) + ky) * n0 + m;
+    *HND_G(&out[e]) = *HND_S(&ts[f * (kS3 + 1) + kb]);
   }
 }
 

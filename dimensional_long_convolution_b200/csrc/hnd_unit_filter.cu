@@ -23,6 +23,19 @@ static unsigned grid_for(long long work, int threads) {
   return static_cast<unsigned>(b);
 }
 
+// 3D: natural spectrum or the filter's full grids -> library order
+static cudaError_t spec3_in_go(const float2* src, float4* out, const int* n, long long C, long long pitch, float scale,
+                               int pair, cudaStream_t st) {
+  const size_t sm = hnd2::spec3_in_smem(n[0]);
+  cudaError_t e = ensure_smem(hnd2::k_spec3_in, sm);
+  if (e != cudaSuccess) return e;
+  const long long nkb = (n[2] + 1 + hnd2::kS3 - 1) / hnd2::kS3;
+  const long long ctas = C * 2LL * n[1] * nkb;
+  if (ctas > 0x7fffffffLL) return cudaErrorInvalidValue;
+  hnd2::k_spec3_in<<<static_cast<unsigned>(ctas), 256, sm, st>>>(src, out, n[0], n[1], n[2], C, pitch, scale, pair);
+  return cudaGetLastError();
+}
+
 template <int HP, bool TAB>
 static cudaError_t filter_mlp_go_t(const hnd2::FilterMlpArgs& fa, long long noff, cudaStream_t st) {
   auto kern = hnd2::k_filter_mlp2<HP, TAB>;
@@ -57,9 +70,18 @@ long long filter_table_bytes(int hidden, int ndim, const int* n) {
 
 cudaError_t launch_filter_tables(const FilterLaunch& f, int ndim, const int* n, float* tab, cudaStream_t st) {
   const int HP = (f.hidden + 31) / 32 * 32;
-  const long long cnt = hnd2::filter_table_floats(HP, ndim, n);
+  const long long cnt = hnd2::filter_trig_offset(HP, ndim, n);
   hnd2::k_filter_tables<<<grid_for(cnt, 256), 256, 0, st>>>(f.W1, f.hidden, HP, f.num_freqs, ndim, n[0],
                                                             ndim > 1 ? n[1] : 1, ndim > 2 ? n[2] : 1, tab);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? launch_filter_trig(f, ndim, n, tab, st) : e;
+}
+
+cudaError_t launch_filter_trig(const FilterLaunch& f, int ndim, const int* n, float* tab, cudaStream_t st) {
+  const int HP = (f.hidden + 31) / 32 * 32;
+  const long long cnt = static_cast<long long>(HP) * (2 * n[ndim - 1] - 1);
+  hnd2::k_filter_trig<<<grid_for(cnt, 256), 256, 0, st>>>(tab, HP, f.hidden, ndim, n[0], ndim > 1 ? n[1] : 1,
+                                                          ndim > 2 ? n[2] : 1, f.gamma);
   return cudaGetLastError();
 }
 
@@ -261,8 +283,7 @@ cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, i
                                                                         scale, pair);
   } else if (ndim == 3) {
     float4* out = static_cast<float4*>(spectrum) + static_cast<long long>(c0) * (per / 2);
-    hnd2::k_spec3_in<<<grid_for(per / 2 * nc, 256), 256, 0, st>>>(grid, out, n[0], n[1], n[2], nc, 2LL * n[2], scale,
-                                                                  pair);
+    if ((e = spec3_in_go(grid, out, n, nc, 2LL * n[2], scale, pair, st)) != cudaSuccess) return e;
   } else {
     k_spec_pack<<<grid_for(per * nc, 256), 256, 0, st>>>(grid, static_cast<float2*>(spectrum), d, c0, nc, scale);
   }
@@ -338,9 +359,7 @@ cudaError_t launch_spec_convert(int ndim, const int* n, long long C, const void*
       hnd2::k_spec3_out<<<grid_for(total / 2, 256), 256, 0, st>>>(static_cast<const float4*>(src),
                                                                  static_cast<float2*>(dst), n[0], n[1], n[2], C);
     else
-      hnd2::k_spec3_in<<<grid_for(total / 2, 256), 256, 0, st>>>(static_cast<const float2*>(src),
-                                                                static_cast<float4*>(dst), n[0], n[1], n[2], C,
-                                                                n[2] + 1, 1.0f);
+      return spec3_in_go(static_cast<const float2*>(src), static_cast<float4*>(dst), n, C, n[2] + 1, 1.0f, 0, st);
     return cudaGetLastError();
   }
   if (ndim == 2) {

@@ -65,13 +65,13 @@ int ilog2(long long x) {
   return l;
 }
 
+// One wave: `cnt` channel-pair grids from pair v0.  part 0: the first pass
+// only; part 1: the rest; part 2: all of it.
 template <class T>
-cudaError_t long1d_t(const ConvArgs& c, float2* grid, long long wave, int* launches) {
+cudaError_t long1d_t(const ConvArgs& c, float2* grid, long long v0, long long cnt, int part, int* launches) {
   const L1Split sp = long1d_split(c.n[0]);
   const int m = sp.m;
   const long long P = 2LL * c.n[0];
-  const int H = (c.C + 1) / 2;
-  const long long nunits = static_cast<long long>(c.B) * H;      // channel-pair grids
   long long stride[3] = {1, 1, 1};
   for (int a = m - 2; a >= 0; --a) stride[a] = stride[a + 1] * sp.P[a + 1];
   hnd2::L1PassArgs a{};
@@ -79,7 +79,7 @@ cudaError_t long1d_t(const ConvArgs& c, float2* grid, long long wave, int* launc
   a.P = P;
   a.lgP = ilog2(P);
   a.n = c.n[0];
-  a.H = H;
+  a.H = (c.C + 1) / 2;
   a.a = c.k;
   a.b = c.v;
   a.q = c.q;
@@ -92,57 +92,69 @@ cudaError_t long1d_t(const ConvArgs& c, float2* grid, long long wave, int* launc
   a.lgP0 = ilog2(sp.P[0]);
   a.sconj = c.sconj;
   a.C = c.C;
+  a.v0 = v0;
+  auto set_axis = [&](int ax) {
+    a.stride = stride[ax];
+    a.lgS = ilog2(stride[ax]);
+    a.npen = cnt * P / sp.P[ax];
+  };
   cudaError_t e = cudaSuccess;
-  for (long long v0 = 0; v0 < nunits && e == cudaSuccess; v0 += wave) {
-    const long long cnt = nunits - v0 < wave ? nunits - v0 : wave;
-    a.v0 = v0;
-    auto set_axis = [&](int ax) {
-      a.stride = stride[ax];
-      a.lgS = ilog2(stride[ax]);
-      a.npen = cnt * P / sp.P[ax];
-    };
-    // forward: axis 0 from k v, then axis 1 (three levels)
+  if (part != 1) {
+    // forward: axis 0 from k v
     set_axis(0);
     a.twQ = P;
     a.lgQ = ilog2(a.twQ);
     e = l1_pass<hnd2::kFirst, T, false>(sp.P[0] / 2, a, c.stream);
-    if (e == cudaSuccess && m == 3) {
-      set_axis(1);
-      a.twQ = static_cast<long long>(sp.P[1]) * sp.P[2];
-      a.lgQ = ilog2(a.twQ);
-      e = l1_pass<hnd2::kFwdMid, float, false>(sp.P[1] / 2, a, c.stream);
-    }
-    // spectrum product on the last axis, pencil pairs, with the inverse
-    // transform back
-    if (e == cudaSuccess) {
-      set_axis(m - 1);
-      a.npen = cnt * a.sd.R;
-      a.twP = sp.P[m - 2];
-      a.twQ = static_cast<long long>(sp.P[m - 2]) * sp.P[m - 1];
-      a.lgQ = ilog2(a.twQ);
-      e = l1_center(sp.P[m - 1] / 2, a, c.stream);
-    }
-    if (e == cudaSuccess && m == 3) {
-      set_axis(1);
-      a.twP = sp.P[0];
-      a.twQ = P;
-      a.lgQ = ilog2(a.twQ);
-      e = l1_pass<hnd2::kInvMid, float, false>(sp.P[1] / 2, a, c.stream);
-    }
-    if (e == cudaSuccess) {
-      set_axis(0);
-      e = c.y2 ? l1_pass<hnd2::kLast, T, true>(sp.P[0] / 2, a, c.stream)
-               : l1_pass<hnd2::kLast, T, false>(sp.P[0] / 2, a, c.stream);
-    }
-    *launches += 2 * m - 1;
+    *launches += 1;
+    if (part == 0 || e != cudaSuccess) return e;
   }
+  if (m == 3) {
+    // forward axis 1 (three levels)
+    set_axis(1);
+    a.twQ = static_cast<long long>(sp.P[1]) * sp.P[2];
+    a.lgQ = ilog2(a.twQ);
+    e = l1_pass<hnd2::kFwdMid, float, false>(sp.P[1] / 2, a, c.stream);
+  }
+  // spectrum product on the last axis, pencil pairs, with the inverse
+  // transform back
+  if (e == cudaSuccess) {
+    set_axis(m - 1);
+    a.npen = cnt * a.sd.R;
+    a.twP = sp.P[m - 2];
+    a.twQ = static_cast<long long>(sp.P[m - 2]) * sp.P[m - 1];
+    a.lgQ = ilog2(a.twQ);
+    e = l1_center(sp.P[m - 1] / 2, a, c.stream);
+  }
+  if (e == cudaSuccess && m == 3) {
+    set_axis(1);
+    a.twP = sp.P[0];
+    a.twQ = P;
+    a.lgQ = ilog2(a.twQ);
+    e = l1_pass<hnd2::kInvMid, float, false>(sp.P[1] / 2, a, c.stream);
+  }
+  if (e == cudaSuccess) {
+    set_axis(0);
+    e = c.y2 ? l1_pass<hnd2::kLast, T, true>(sp.P[0] / 2, a, c.stream)
+             : l1_pass<hnd2::kLast, T, false>(sp.P[0] / 2, a, c.stream);
+  }
+  *launches += 2 * m - 2;
   return e;
 }
 
 }  // namespace
 
+cudaError_t launch_long1d_wave(const ConvArgs& a, float2* grid, long long v0, long long cnt, int part,
+                               int* launches) {
+  return a.bf16 ? long1d_t<__nv_bfloat16>(a, grid, v0, cnt, part, launches)
+                : long1d_t<float>(a, grid, v0, cnt, part, launches);
+}
+
 cudaError_t launch_long1d(const ConvArgs& a, float2* grid, long long wave, int* launches) {
-  return a.bf16 ? long1d_t<__nv_bfloat16>(a, grid, wave, launches) : long1d_t<float>(a, grid, wave, launches);
+  const long long grids = static_cast<long long>(a.B) * ((a.C + 1) / 2);
+  cudaError_t e = cudaSuccess;
+  for (long long v0 = 0; v0 < grids && e == cudaSuccess; v0 += wave)
+    e = launch_long1d_wave(a, grid, v0, grids - v0 < wave ? grids - v0 : wave, 2, launches);
+  return e;
 }
 
 }  // namespace hnd
