@@ -379,6 +379,43 @@ __global__ void __launch_bounds__(kFT) k_filter_mlp2(const FilterMlpArgs a) {
       }
       continue;
     }
+    if (a.nc - ct <= kFC / 2) {
+      // half tile (9 to 16 channels left, e.g. the 128^3 grids' chunks):
+      // thread -> offsets 2 (tid % 64) + {0, 1}, channels 4 (tid / 64) + {0..3}
+      const int o2 = 2 * (tid % 64), cb = 4 * (tid / 64);
+      float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll 8
+      for (int h = 0; h < HP; ++h) {
+        const float2 hv = *HND_S(reinterpret_cast<const float2*>(hid + h * kFO + o2));
+        const float4 wv = *HND_S(reinterpret_cast<const float4*>(w2 + h * kFC + cb));
+        const float ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          acc2[0][j] = fmaf(hv.x, ww[j], acc2[0][j]);
+          acc2[1][j] = fmaf(hv.y, ww[j], acc2[1][j]);
+        }
+      }
+      if (cb < a.nc - ct) {
+        float bb[4], al[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int c = ct + cb + j;
+          bb[j] = c < a.nc ? __ldg(HND_G(a.b2 + a.c0 + c)) : 0.f;
+          al[j] = c < a.nc ? __ldg(HND_G(a.alpha + a.c0 + c)) : 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int o = o2 + i;
+          if (e0 + o >= noff) continue;
+          const float ro = *HND_S(&rad[o]);
+          float kv[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) kv[j] = ct + cb + j < a.nc ? (acc2[i][j] + bb[j]) * __expf(-al[j] * ro) : 0.f;
+          store_k4(a, ct + cb, gsz, *HND_S(&slot[o]), kv);
+        }
+      }
+      continue;
+    }
     float acc[4][4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)

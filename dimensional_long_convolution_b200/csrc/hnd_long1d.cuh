@@ -280,6 +280,30 @@ __global__ void __launch_bounds__(kAT, 2) k_l1_pass(const L1PassArgs a) {
         x[s] = {make_float2(e0.x, e1.x), make_float2(e0.y, e1.y)};
       }
     }
+    // kLast: with 8 slots a lane, the output gates are loaded before the
+    // inverse transform, so that their latency overlaps it (the pass is
+    // otherwise bound by waiting on these strided loads); with 16 slots the
+    // registers are not there, and they are loaded at the store
+    constexpr bool PRE = KIND == kLast && R1 == 8;
+    constexpr int RQ = PRE ? R1 : 1;
+    float qa_v[RQ], qb_v[RQ], ga_v[PRE && DUAL ? RQ : 1], gb_v[PRE && DUAL ? RQ : 1];
+    bool has_b = false;
+    long long orow = 0;
+    if constexpr (KIND == kLast) orow = l1_pair_vol(a.v0 + vol, a.H, a.C, &has_b) * a.n + i;
+    if constexpr (PRE) {
+      const T* qa = static_cast<const T*>(a.q);
+#pragma unroll
+      for (int s = 0; s < R1; ++s) {
+        const long long j = orow + static_cast<long long>(g + s * G) * S;
+        qa_v[s] = act ? Act<T>::ld_g(qa + j) : 0.f;
+        qb_v[s] = act && has_b ? Act<T>::ld_g(qa + j + a.n) : 0.f;
+        if constexpr (DUAL) {
+          const T* g2 = static_cast<const T*>(a.g2);
+          ga_v[s] = act ? Act<T>::ld_g(g2 + j) : 0.f;
+          gb_v[s] = act && has_b ? Act<T>::ld_g(g2 + j + a.n) : 0.f;
+        }
+      }
+    }
 
     if constexpr (KIND == kFirst || KIND == kFwdMid) {
       // forward twiddle W_Q^{k i} at k = 2f, 2f + 1; store in spectral positions
@@ -316,22 +340,21 @@ __global__ void __launch_bounds__(kAT, 2) k_l1_pass(const L1PassArgs a) {
       // imaginary part -> channel b; output gate(s)
       float2 out[R1];
       padded_inv<N>(x, out, g, buf, 0, t, 0u);
-      const T* qa = static_cast<const T*>(a.q);
       T* ya = static_cast<T*>(a.y);
-      bool has_b;
-      const long long row0 = l1_pair_vol(a.v0 + vol, a.H, a.C, &has_b) * a.n + i;
+      const T* qa = static_cast<const T*>(a.q);
+      const T* g2 = static_cast<const T*>(a.g2);
 #pragma unroll
       for (int s = 0; s < R1; ++s) {
-        const long long j = row0 + static_cast<long long>(g + s * G) * S;
+        const long long j = orow + static_cast<long long>(g + s * G) * S;
         if (act) {
-          Act<T>::st_g(ya + j, out[s].x * Act<T>::ld_g(qa + j));
+          Act<T>::st_g(ya + j, out[s].x * (PRE ? qa_v[s % RQ] : Act<T>::ld_g(qa + j)));
           if constexpr (DUAL)
-            Act<T>::st_g(static_cast<T*>(a.y2) + j, out[s].x * Act<T>::ld_g(static_cast<const T*>(a.g2) + j));
+            Act<T>::st_g(static_cast<T*>(a.y2) + j, out[s].x * (PRE ? ga_v[s % RQ] : Act<T>::ld_g(g2 + j)));
           if (has_b) {
-            Act<T>::st_g(ya + j + a.n, out[s].y * Act<T>::ld_g(qa + j + a.n));
+            Act<T>::st_g(ya + j + a.n, out[s].y * (PRE ? qb_v[s % RQ] : Act<T>::ld_g(qa + j + a.n)));
             if constexpr (DUAL)
               Act<T>::st_g(static_cast<T*>(a.y2) + j + a.n,
-                           out[s].y * Act<T>::ld_g(static_cast<const T*>(a.g2) + j + a.n));
+                           out[s].y * (PRE ? gb_v[s % RQ] : Act<T>::ld_g(g2 + j + a.n)));
           }
         }
       }
@@ -376,6 +399,14 @@ __global__ void __launch_bounds__(kAT, 2) k_l1_center(const L1PassArgs a) {
     const unsigned kap = side == 0 ? r : (self ? r : Po - r);
     const long long o = (static_cast<long long>(kap & (d.P0 - 1)) * d.Pm) + (kap >> a.lgP0);
     float2* base = a.grid + (static_cast<long long>(wv) * Po + o) * Pc;
+    const long long pg = a.v0 + wv;                 // the channel pair
+    const long long smp = pg / a.H, jj = pg - smp * a.H;
+    const float4* row = a.spec + smp * a.sbs4 + jj * d.per_pair() + static_cast<long long>(r) * Pc;
+    // the unit's spectrum row (Pc float4) into L2 while the transforms run
+    if (valid && side == 0) {
+      for (int q = g; q < Pc / 8; q += G)
+        if (HND_RANGE_OK(row + 8 * q, 16)) asm volatile("prefetch.global.L2 [%0];" ::"l"(row + 8 * q));
+    }
     float2 lo[R1], hi[R1];
 #pragma unroll
     for (int s = 0; s < R1; ++s) {
@@ -393,9 +424,6 @@ __global__ void __launch_bounds__(kAT, 2) k_l1_center(const L1PassArgs a) {
       *HND_S(&buf[swz(spec_idx<N>(g, s))]) = make_float4(x[s].re.x, x[s].re.y, x[s].im.x, x[s].im.y);
     __syncwarp();
     const float4* src = self ? buf : pbuf;
-    const long long pg = a.v0 + wv;                 // the channel pair
-    const long long smp = pg / a.H, jj = pg - smp * a.H;
-    const float4* row = a.spec + smp * a.sbs4 + jj * d.per_pair() + static_cast<long long>(r) * Pc;
     const bool flip = (side == 1) != conj_spec;
 #pragma unroll
     for (int s = 0; s < R1; ++s) {
