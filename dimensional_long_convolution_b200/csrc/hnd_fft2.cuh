@@ -32,6 +32,15 @@
 
 namespace hnd2 {
 
+// Programmatic dependent launch: the stage kernels run back to back on one
+// stream.  Each lets the next stage's CTAs be scheduled as soon as all of its
+// own CTAs have started (they then build their tables on SMs freed by this
+// stage's tail), and waits for the previous grid to complete, with its
+// memory visible, before its first global access.  Both are no-ops for a
+// launch without the programmatic-serialization attribute.
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------ packed fp32
 __device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
 __device__ __forceinline__ float2 padd(float2 a, float2 b) { return __fadd2_rn(a, b); }

@@ -225,10 +225,12 @@ template <int N, int KIND, class T, bool DUAL>
 __global__ void __launch_bounds__(kAT, 2) k_l1_pass(const L1PassArgs a) {
   constexpr int G = P2<N>::G, R1 = P2<N>::R1, PPW = 32 / G, P = 2 * N;
   extern __shared__ __align__(16) unsigned char asmem[];
+  pdl_release();
   const Tabs<N> t = tabs_at<N>(asmem);
   float4* xb = reinterpret_cast<float4*>(asmem + Tabs<N>::kBytes);
   tabs_build<N>(t, g_tw512);
   __syncthreads();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pen = lane / G, g = lane % G;
   float4* buf = xb + warp * XB<N>::kWarp + pen * XB<N>::kPen;
@@ -376,10 +378,12 @@ __global__ void __launch_bounds__(kAT, 2) k_l1_center(const L1PassArgs a) {
   constexpr int G = P2<N>::G, R1 = P2<N>::R1, PPW = 32 / G, UPW = PPW / 2, Pc = 2 * N;
   static_assert(PPW >= 2, "a unit takes two pencil slots of one warp");
   extern __shared__ __align__(16) unsigned char asmem[];
+  pdl_release();
   const Tabs<N> t = tabs_at<N>(asmem);
   float4* xb = reinterpret_cast<float4*>(asmem + Tabs<N>::kBytes);
   tabs_build<N>(t, g_tw512);
   __syncthreads();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pen = lane / G, g = lane % G, side = pen & 1;
   float4* buf = xb + warp * XB<N>::kWarp + pen * XB<N>::kPen;

@@ -29,14 +29,6 @@ constexpr int kWM = kTM / 32;
 // scheduler warp that does not take part.
 __device__ __forceinline__ void task_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kTM) : "memory"); }
 
-// Programmatic dependent launch: the stage kernels run back to back on one
-// stream.  Each lets the next stage's CTAs be scheduled as soon as all of its
-// own CTAs have started (they then build their tables on SMs freed by this
-// stage's tail), and waits for the previous grid to complete, with its
-// memory visible, before its first global access.  Both are no-ops for a
-// launch without the programmatic-serialization attribute.
-__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // ------------------------------------------------------ workspace access
 // The wave workspace (packed row spectra) bypasses L1: it is written by one
@@ -691,62 +683,67 @@ __host__ __device__ __forceinline__ int spec_idx_gen(int N, int g, int s) {
 }
 __host__ __device__ __forceinline__ int lanes_of(int N) { return N == 8 ? 1 : N / (N >= 128 ? 16 : 8); }
 
-// Value at (kz, ky, kx) of channel c of a source [C][2 n0][2 n1][pitch], or
-// (pair) of the filter call's full grids holding two channels per complex
-// grid (channel c even in the real part; S_c = (W[k] + conj W[-k]) / 2,
-// S_{c+1} = (W[k] - conj W[-k]) / (2i)).
-__device__ __forceinline__ float2 src3_at(const float2* __restrict__ nat, long long c, long long src_per,
-                                          long long pitch, int kz, int ky, int kx, int n0, int n1, int n2,
-                                          int pair) {
-  const long long row = 2LL * n1;
-  if (!pair) return *HND_G(&nat[c * src_per + (kz * row + ky) * pitch + kx]);
-  const float2* g = nat + (c >> 1) * src_per;
-  const float2 w = *HND_G(&g[(kz * row + ky) * pitch + kx]);
-  const int mz = (2 * n0 - kz) & (2 * n0 - 1), my = (2 * n1 - ky) & (2 * n1 - 1), mx = (2 * n2 - kx) & (2 * n2 - 1);
-  const float2 m = *HND_G(&g[(mz * row + my) * pitch + mx]);
-  return (c & 1) ? make_float2(0.5f * (w.y + m.y), 0.5f * (m.x - w.x)) : make_float2(0.5f * (w.x + m.x), 0.5f * (w.y - m.y));
-}
-
 // natural half spectrum [C][2n0][2n1][n2 + 1] (pitch = last-axis length of the
 // source: n2 + 1 for a half spectrum, 2 n2 for a full grid; pair: the filter
 // call's full grids, two channels per grid) -> library order.
-// A CTA takes one (c, ky) and kS3 consecutive kx: it reads the z-pencils of
-// those kx (kx adjacent in the source, so every kz row is one contiguous
-// read; the partner values -k form the mirrored contiguous run) into shared
-// memory indexed by the z frequency pair f, then writes the library's n0
-// float4 of each kx in slot order, contiguous.
-constexpr int kS3 = 32;
-__host__ __device__ __forceinline__ size_t spec3_in_smem(int n0) { return sizeof(float4) * n0 * (kS3 + 1); }
+// A CTA takes one ky and kS3 consecutive kx of one source grid: it reads the
+// z-pencils of those kx into shared memory (kx adjacent in the source, so a
+// kz row is one contiguous read) and, for a pair grid, the z-pencils of the
+// mirrored frequencies (-ky, -kx), again contiguous runs; it then writes the
+// library's n0 float4 of each kx in slot order, contiguous -- for a pair grid
+// both channels from the same reads (S_c = (W + conj W_m)/2,
+// S_{c+1} = (W - conj W_m)/(2i)).
+constexpr int kS3 = 16;
+__host__ __device__ __forceinline__ size_t spec3_in_smem(int n0) { return sizeof(float2) * 2 * (2 * n0) * (kS3 + 1); }
 
 static __global__ void __launch_bounds__(256) k_spec3_in(const float2* __restrict__ nat, float4* __restrict__ out,
                                                          int n0, int n1, int n2, long long C, long long pitch,
                                                          float scale, int pair = 0) {
-  extern __shared__ __align__(16) float4 ts[];     // [f][kS3 + 1]
+  extern __shared__ __align__(16) float2 tw[];     // W [kz][kS3 + 1], then W_m [kz][kS3 + 1]
+  float2* tm = tw + 2 * n0 * (kS3 + 1);
   const long long src_per = 4LL * n0 * n1 * pitch;
   const int nkb = (n2 + 1 + kS3 - 1) / kS3;
   const long long cta = blockIdx.x;
   const int kb0 = static_cast<int>(cta % nkb) * kS3;
   const int ky = static_cast<int>((cta / nkb) % (2 * n1));
-  const long long c = cta / (static_cast<long long>(nkb) * 2 * n1);
+  const long long gi = cta / (static_cast<long long>(nkb) * 2 * n1);   // source grid (pair) or channel
   const int nk = min(kS3, n2 + 1 - kb0);
-  float* tsf = reinterpret_cast<float*>(ts);
+  const float2* g = nat + gi * src_per;
+  const long long row = 2LL * n1;
+  const int my = (2 * n1 - ky) & (2 * n1 - 1);
   for (int i = threadIdx.x; i < 2 * n0 * kS3; i += blockDim.x) {
     const int kz = i / kS3, kb = i % kS3;
     if (kb >= nk) continue;
-    const float2 v = src3_at(nat, c, src_per, pitch, kz, ky, kb0 + kb, n0, n1, n2, pair);
-    // float4 (S[2f].re, S[2f+1].re, S[2f].im, S[2f+1].im), f = kz / 2
-    float* d = tsf + 4 * ((kz >> 1) * (kS3 + 1) + kb) + (kz & 1);
-    *HND_S(d) = scale * v.x;
-    *HND_S(d + 2) = scale * v.y;
+    const int kx = kb0 + kb;
+    *HND_S(&tw[kz * (kS3 + 1) + kb]) = *HND_G(&g[(kz * row + ky) * pitch + kx]);
+    if (pair) {
+      const int mx = (2 * n2 - kx) & (2 * n2 - 1);
+      *HND_S(&tm[kz * (kS3 + 1) + kb]) = *HND_G(&g[(kz * row + my) * pitch + mx]);
+    }
   }
   __syncthreads();
   const int G = lanes_of(n0);
-  for (int i = threadIdx.x; i < n0 * kS3; i += blockDim.x) {
-    const int kb = i / n0, m = i % n0;
+  const int nch = pair ? static_cast<int>(min(2LL, C - 2 * gi)) : 1;
+  for (int i = threadIdx.x; i < nch * n0 * kS3; i += blockDim.x) {
+    const int ch = i / (n0 * kS3), kb = (i / n0) % kS3, m = i % n0;
     if (kb >= nk) continue;
     const int f = spec_idx_gen(n0, m % G, m / G);
+    float2 s2[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int kz = 2 * f + h;
+      const float2 w = *HND_S(&tw[kz * (kS3 + 1) + kb]);
+      if (!pair) {
+        s2[h] = w;
+      } else {
+        const float2 wm = *HND_S(&tm[((2 * n0 - kz) & (2 * n0 - 1)) * (kS3 + 1) + kb]);
+        s2[h] = ch ? make_float2(0.5f * (w.y + wm.y), 0.5f * (wm.x - w.x))
+                   : make_float2(0.5f * (w.x + wm.x), 0.5f * (w.y - wm.y));
+      }
+    }
+    const long long c = pair ? 2 * gi + ch : gi;
     const long long e = ((c * (n2 + 1) + kb0 + kb) * (2LL * n1) + ky) * n0 + m;
-    *HND_G(&out[e]) = *HND_S(&ts[f * (kS3 + 1) + kb]);
+    *HND_G(&out[e]) = make_float4(scale * s2[0].x, scale * s2[1].x, scale * s2[0].y, scale * s2[1].y);
   }
 }
 

@@ -30,7 +30,8 @@ static cudaError_t spec3_in_go(const float2* src, float4* out, const int* n, lon
   cudaError_t e = ensure_smem(hnd2::k_spec3_in, sm);
   if (e != cudaSuccess) return e;
   const long long nkb = (n[2] + 1 + hnd2::kS3 - 1) / hnd2::kS3;
-  const long long ctas = C * 2LL * n[1] * nkb;
+  const long long grids = pair ? (C + 1) / 2 : C;      // a pair grid's CTAs write both channels
+  const long long ctas = grids * 2LL * n[1] * nkb;
   if (ctas > 0x7fffffffLL) return cudaErrorInvalidValue;
   hnd2::k_spec3_in<<<static_cast<unsigned>(ctas), 256, sm, st>>>(src, out, n[0], n[1], n[2], C, pitch, scale, pair);
   return cudaGetLastError();

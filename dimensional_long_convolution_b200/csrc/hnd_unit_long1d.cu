@@ -18,8 +18,7 @@ cudaError_t l1_pass_go(const hnd2::L1PassArgs& a, cudaStream_t st) {
   long long blocks = (a.npen + per_cta - 1) / per_cta;
   if (blocks > 148LL * 16) blocks = 148LL * 16;
   if (blocks < 1) blocks = 1;
-  kern<<<static_cast<unsigned>(blocks), hnd2::kAT, sm, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(true, kern, dim3(static_cast<unsigned>(blocks)), dim3(hnd2::kAT), sm, st, a);
 }
 
 template <int N>
@@ -32,8 +31,7 @@ cudaError_t l1_center_go(const hnd2::L1PassArgs& a, cudaStream_t st) {
   long long blocks = (a.npen + per_cta - 1) / per_cta;
   if (blocks > 148LL * 16) blocks = 148LL * 16;
   if (blocks < 1) blocks = 1;
-  kern<<<static_cast<unsigned>(blocks), hnd2::kAT, sm, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(true, kern, dim3(static_cast<unsigned>(blocks)), dim3(hnd2::kAT), sm, st, a);
 }
 
 cudaError_t l1_center(int N, const hnd2::L1PassArgs& a, cudaStream_t st) {
