@@ -64,10 +64,14 @@ def test_long1d_forward_matches_oracle(dims, B, C, dt):
     assert O.rel_l2(got, O.reference_output(inp)) <= TOL[dt]
 
 
-@pytest.mark.parametrize("n,B,C,dt", [(65536, 2, 60, "f32"), (131072, 1, 4, "bf16"), (16384, 3, 5, "f32")])
+@pytest.mark.parametrize("n,B,C,dt", [(65536, 2, 60, "f32"), (131072, 1, 4, "bf16"), (16384, 3, 5, "f32"),
+                                     (1 << 19, 3, 7, "bf16")])
 def test_long1d_forward_sampled(n, B, C, dt):
-    """Longest grids and a two-wave schedule (120 volumes of 1 MiB grids),
-    sampled outputs against direct sums."""
+    """Longest grids and multi-wave schedules, sampled outputs against direct
+    sums.  2^19 tokens, B = 3, C = 7: 12 channel-pair grids of 8 MiB, so six
+    waves of two on three streams, and the last pair of every sample holds
+    one channel (channels 0, 3 and 6 are sampled: both halves of a pair and
+    the lone channel)."""
     wl = W.custom((n,), B, C, io_dtype=dt, seed=n % 97 + C)
     inp = W.make_inputs(wl)
     got, _ = run(inp)
