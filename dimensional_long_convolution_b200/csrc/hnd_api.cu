@@ -382,7 +382,7 @@ hyena_nd_status hyena_nd_plan_info_get(const hyena_nd_problem* p, hyena_nd_plan_
     const hnd::L1Split sp = hnd::long1d_split(pl.n[0]);
     info.split_levels = sp.m;
     for (int a = 0; a < 3; ++a) info.split[a] = sp.P[a];
-    info.launches = static_cast<int>(info.waves) * (2 * sp.m - 1);
+    info.launches = static_cast<int>(info.waves) * hnd::long1d_conv_launches(pl.n[0]);
   } else {
     info.launches = info.wave > 0 ? static_cast<int>(info.waves) * 3 : 1;
   }

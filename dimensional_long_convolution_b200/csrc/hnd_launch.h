@@ -112,7 +112,8 @@ struct L1Split {
   int P[3] = {1, 1, 1};
 };
 L1Split long1d_split(int n);
-int long1d_launches_per_transform(int n);
+// Kernel launches of one convolution wave: 2m - 1.
+int long1d_conv_launches(int n);
 // Channels 2j and 2j + 1 of a sample share one complex grid; `wave` counts
 // these channel-pair grids (B ceil(C/2) in all).
 cudaError_t launch_long1d(const ConvArgs& a, float2* grid, long long wave, int* launches);

@@ -237,8 +237,8 @@ __global__ void __launch_bounds__(kAT, 2) k_l1_pass(const L1PassArgs a) {
   const long long per_cta = (kAT / 32) * PPW;
   const long long S = a.stride;
   const float invQ = ldexpf(1.f, -a.lgQ);
-  // every product below is < Q <= 2^27 (the level's factor times the index
-  // range of the later levels), so 32-bit unsigned arithmetic is exact
+  // twiddle exponents are taken mod Q (Q <= 2^27 a power of two, so 32-bit
+  // unsigned products that wrap keep their value mod Q)
   for (long long p0 = static_cast<long long>(blockIdx.x) * per_cta; p0 < a.npen;
        p0 += static_cast<long long>(gridDim.x) * per_cta) {
     const long long p = p0 + warp * PPW + pen;
@@ -308,12 +308,26 @@ __global__ void __launch_bounds__(kAT, 2) k_l1_pass(const L1PassArgs a) {
     }
 
     if constexpr (KIND == kFirst || KIND == kFwdMid) {
-      // forward twiddle W_Q^{k i} at k = 2f, 2f + 1; store in spectral positions
-      const float2 wi = l1_w(i, invQ);
+      // forward twiddle W_Q^{k i} at k = 2f, 2f + 1; store in spectral
+      // positions.  With 2f i = 2i (g + G (s / R2) + R1 (s % R2)) the lane
+      // builds its twiddles from four exact ones by products (a few float
+      // roundings each) instead of one sine-cosine per slot.
+      const unsigned qm = (1u << a.lgQ) - 1u;
+      const float2 wi = l1_w(i & qm, invQ);
+      const float2 bG = l1_w((2u * G * i) & qm, invQ);
+      const float2 bR = l1_w((2u * R1 * i) & qm, invQ);
+      float2 wo = l1_w((2u * g * i) & qm, invQ), w0 = wo;
 #pragma unroll
       for (int s = 0; s < R1; ++s) {
+        if (s > 0) {
+          if (s % P2<N>::R2 == 0) {
+            wo = cmul1(wo, bG);
+            w0 = wo;
+          } else {
+            w0 = cmul1(w0, bR);
+          }
+        }
         const unsigned f = spec_idx<N>(g, s);
-        const float2 w0 = l1_w((2u * f) * i, invQ);
         const float2 w1 = cmul1(w0, wi);
         if (act) {
           *HND_G(&base[(2 * f) * S]) = cmul1(make_float2(x[s].re.x, x[s].im.x), w0);
@@ -324,13 +338,18 @@ __global__ void __launch_bounds__(kAT, 2) k_l1_pass(const L1PassArgs a) {
       float2 lo[R1], hi[R1];
       l1_full_inv<N>(x, lo, hi, g, buf, t);
       // conjugate twiddle of level 0: conj W_P^{k0 (e S + i)}, k0 = o mod twP
+      // (exponents mod Q, Q a power of two dividing 2^32; w0 for slot s is
+      // conj W^{k (g S + i)} conj W^{k G S}^s)
       const unsigned k = static_cast<unsigned>(o & (a.twP - 1));
       const unsigned Su = static_cast<unsigned>(S);
-      const float2 wk = l1_conj(l1_w(k * N * Su, invQ));
+      const unsigned qm = (1u << a.lgQ) - 1u;
+      const float2 wk = l1_conj(l1_w((k * N * Su) & qm, invQ));
+      const float2 cG = l1_conj(l1_w((k * G * Su) & qm, invQ));
+      float2 w0 = l1_conj(l1_w((k * (static_cast<unsigned>(g) * Su + i)) & qm, invQ));
 #pragma unroll
       for (int s = 0; s < R1; ++s) {
         const long long j = g + s * G;
-        const float2 w0 = l1_conj(l1_w(k * (static_cast<unsigned>(j) * Su + i), invQ));
+        if (s > 0) w0 = cmul1(w0, cG);
         const float2 w1 = cmul1(w0, wk);
         if (act) {
           *HND_G(&base[j * S]) = cmul1(lo[s], w0);
@@ -468,12 +487,16 @@ __global__ void __launch_bounds__(kAT, 2) k_l1_center(const L1PassArgs a) {
     l1_full_inv<N>(x, lo, hi, g, buf, t);
     // conjugate twiddle of the previous level: conj W_Q^{k e}, k = o mod twP,
     // e the element's index along this (last) axis
+    // (w0 for slot s is conj W^{k g} conj W^{k G}^s)
     const unsigned k = static_cast<unsigned>(o & (a.twP - 1));
-    const float2 wk = l1_conj(l1_w(k * N, invQ));
+    const unsigned qm = (1u << a.lgQ) - 1u;
+    const float2 wk = l1_conj(l1_w((k * N) & qm, invQ));
+    const float2 cG = l1_conj(l1_w((k * G) & qm, invQ));
+    float2 w0 = l1_conj(l1_w((k * g) & qm, invQ));
 #pragma unroll
     for (int s = 0; s < R1; ++s) {
       const unsigned j = g + s * G;
-      const float2 w0 = l1_conj(l1_w(k * j, invQ));
+      if (s > 0) w0 = cmul1(w0, cG);
       const float2 w1 = cmul1(w0, wk);
       if (act) {
         *HND_G(&base[j]) = cmul1(lo[s], w0);

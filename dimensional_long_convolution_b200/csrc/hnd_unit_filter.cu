@@ -185,8 +185,6 @@ static cudaError_t l1_inv_conj(float2* grid, const L1Split& sp, long long ngrids
   return e;
 }
 
-int long1d_launches_per_transform(int n) { return 2 * long1d_split(n).m - 1; }
-
 size_t spectrum_set_bytes(int ndim, const int* n, long long C) {
   if (ndim == 1 && n[0] > 256) {
     const L1Split sp = long1d_split(n[0]);

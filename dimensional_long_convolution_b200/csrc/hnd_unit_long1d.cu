@@ -141,6 +141,8 @@ cudaError_t long1d_t(const ConvArgs& c, float2* grid, long long v0, long long cn
 
 }  // namespace
 
+int long1d_conv_launches(int n) { return 2 * long1d_split(n).m - 1; }
+
 cudaError_t launch_long1d_wave(const ConvArgs& a, float2* grid, long long v0, long long cnt, int part,
                                int* launches) {
   return a.bf16 ? long1d_t<__nv_bfloat16>(a, grid, v0, cnt, part, launches)

@@ -27,6 +27,8 @@ CONV = [((64,), 2, 3, "f32"), ((1024,), 1, 2, "f32"), ((32, 64), 2, 2, "bf16"), 
         ((16, 32, 64), 1, 2, "f32"), ((128, 128, 8), 1, 1, "f32")]
 BWD = [((32, 32), 1, 2, "f32"), ((64, 128), 1, 2, "f32"), ((8, 16, 32), 1, 2, "f32")]
 KGRAD = [((32, 16), 2, 2, "f32"), ((64, 128), 2, 2, "f32"), ((8, 8, 16), 1, 2, "f32"), ((512,), 1, 2, "f32")]
+# a three-level long 1D grid: 2^19 points split 128 x 64 x 64, odd C
+PLANE = [(1 << 18, 1, 3, "f32")]
 
 
 def _child() -> None:
@@ -64,6 +66,23 @@ def _child() -> None:
         if want is not None:
             out.append({"what": "export %s" % (dims,), "dt": "f32", "err": O.rel_l2(nat, want),
                         "status": int(H.device_status(op.ws.data_ptr(), op._stream()))})
+    # a three-level long 1D split (five passes, the channel-pair center
+    # pass), sampled against direct sums
+    from gpu_util import sample_points
+    for n, B, C, dt in PLANE:
+        wl = W.custom((n,), B, C, io_dtype=dt, seed=29)
+        inp = W.make_inputs(wl)
+        got, op = run(inp)
+        chans = sorted({0, C - 1})
+        pts = sample_points(wl, 8, seed=5, channels=chans)
+        K = np.zeros((C, 2 * n - 1))
+        Kc = O.implicit_kernel(inp.filt, (n,), channels=chans)
+        for j, c in enumerate(chans):
+            K[c] = Kc[j]
+        want = O.conv_direct_at(inp.as_f64("q"), inp.as_f64("k"), inp.as_f64("v"), K, (n,), pts)
+        gv = np.array([got[tuple(p)] for p in pts])
+        out.append({"what": "long 1D %d" % n, "dt": dt, "err": O.rel_l2(gv, want),
+                    "status": int(H.device_status(op.ws.data_ptr(), op._stream()))})
     for dims, B, C, dt in BWD:
         wl = W.custom(dims, B, C, io_dtype=dt, seed=11 + sum(dims))
         inp = W.make_inputs(wl)
