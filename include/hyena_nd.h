@@ -22,12 +22,13 @@
  *     or frees.  Every call is asynchronous on the given CUDA stream
  *     (cudaStream_t passed as void*; NULL = legacy default stream) and
  *     performs no host synchronisation, except hyena_nd_device_status.
- *     Convolutions on the multi-pass tiers with several waves run alternate
- *     waves on a side stream the library creates per device on first use:
- *     it is forked from the caller's stream with an event and joined back to
- *     it before the call returns, so the call stays ordered on the caller's
- *     stream (and may be captured into a CUDA graph with it).  Calls from
- *     several host threads serialise their enqueue on that side stream.
+ *     Convolutions on the multi-pass and long 1D tiers with several waves
+ *     run the waves round-robin on the caller's stream and up to two side
+ *     streams the library creates per device on first use: they are forked
+ *     from the caller's stream with an event and joined back to it before
+ *     the call returns, so the call stays ordered on the caller's stream.
+ *     Calls from several host threads serialise their enqueue on those side
+ *     streams.
  *   * Argument errors are detected on the host before anything is launched
  *     and returned synchronously.  A failed launch returns HYENA_ND_ERR_CUDA.
  *     Errors detected on the device are written to a status word held in the
@@ -185,8 +186,9 @@ typedef struct {
   int kgrad_chunk;        /* channels per chunk of the kernel gradient */
   size_t workspace_bytes; /* hyena_nd_workspace_bytes(p) */
   size_t spectrum_bytes;  /* hyena_nd_spectrum_bytes(p) */
-  int streams;            /* multi-pass tiers: streams running alternate waves (the caller's and, for 2,
-                             a side stream of the library forked from and joined back to it); else 1 */
+  int streams;            /* multi-pass and long 1D tiers: streams running the waves round-robin (the
+                             caller's and up to two side streams of the library, forked from and
+                             joined back to it); else 1 */
 } hyena_nd_plan_info;
 
 /* Fill `out` with the plan of `p`.  Errors: HYENA_ND_ERR_INVALID_ARG (null or
