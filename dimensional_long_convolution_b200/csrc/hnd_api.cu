@@ -100,15 +100,16 @@ constexpr size_t kWaveBudget = size_t(HND_WAVE_MB) << 20;
 constexpr int kWaveStreams = HND_STREAMS;
 static_assert(kWaveStreams >= 1 && kWaveStreams <= hnd::SideStream::kMax, "streams per convolution");
 #ifndef HND_FILTER_MB
-#define HND_FILTER_MB 1024
+#define HND_FILTER_MB 2304
 #endif
 #ifndef HND_FILTER_MAXC
 #define HND_FILTER_MAXC 128
 #endif
 // filter grids per channel chunk: each chunk evaluates the hidden layer once
 // per offset, so fewer, larger chunks save that work at the cost of workspace
-// (3D 128^3, C = 32: 28.0 / 18.7 / 14.7 ms per call at 256 / 512 / 1024 MiB;
-// only the filter call needs this workspace)
+// (3D 128^3, C = 32: 28.0 / 18.7 / 14.7 ms per call at 256 / 512 / 1024 MiB
+// before the later filter changes; 2.25 GiB holds all 32 channels of that
+// grid in one chunk; only the filter call needs this workspace)
 constexpr size_t kFilterBudget = size_t(HND_FILTER_MB) << 20;
 constexpr int kFilterMaxChunk = HND_FILTER_MAXC;
 constexpr size_t kKgradBudget = size_t(256) << 20;    // kernel-gradient grids per channel chunk

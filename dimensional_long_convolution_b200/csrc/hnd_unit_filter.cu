@@ -23,6 +23,29 @@ static unsigned grid_for(long long work, int threads) {
   return static_cast<unsigned>(b);
 }
 
+// Zero the slots of `ngrids` grids [P0][P1][P2] with index P_a / 2 on some
+// used axis a (the planes no kernel offset t in [-(n_a - 1), n_a - 1] is
+// wrap-placed on); a slot on two such planes is written twice, with zero.
+static __global__ void k_filter_clear_unmapped(float2* __restrict__ grid, int ndim, long long P0, long long P1,
+                                               long long P2, long long plane_pts, long long ngrids) {
+  const long long gsz = P0 * P1 * P2;
+  for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < plane_pts * ngrids;
+       e += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long gi = e / plane_pts;
+    long long r = e % plane_pts;
+    long long s0, s1, s2;
+    if (r < P1 * P2) {                               // axis 0 at P0 / 2
+      s0 = P0 / 2, s1 = r / P2, s2 = r % P2;
+    } else if (ndim > 1 && (r -= P1 * P2) < P0 * P2) {   // axis 1 at P1 / 2
+      s0 = r / P2, s1 = P1 / 2, s2 = r % P2;
+    } else {                                          // axis 2 at P2 / 2
+      if (ndim > 1) r -= P0 * P2;
+      s0 = r / P1, s1 = r % P1, s2 = P2 / 2;
+    }
+    *HND_G(&grid[gi * gsz + (s0 * P1 + s1) * P2 + s2]) = make_float2(0.f, 0.f);
+  }
+}
+
 // 3D: natural spectrum or the filter's full grids -> library order
 static cudaError_t spec3_in_go(const float2* src, float4* out, const int* n, long long C, long long pitch, float scale,
                                int pair, cudaStream_t st) {
@@ -235,7 +258,15 @@ cudaError_t launch_filter_chunk(const FilterLaunch& f, int ndim, const int* n, i
   const bool long1d = ndim == 1 && n[0] > 256;
   const int pair = ndim >= 2 || long1d ? 1 : 0;
   const int ngrids = pair ? (nc + 1) / 2 : nc;
-  cudaError_t e = cudaMemsetAsync(grid, 0, sizeof(float2) * gsz * ngrids, st);
+  // the network writes every slot an offset maps to; only the slots at index
+  // n_a on some axis stay (no offset lands there), so those are cleared
+  long long pa[3] = {1, 1, 1};
+  for (int ax = 0; ax < ndim; ++ax) pa[ax] = 2LL * n[ax];
+  long long plane_pts = 0;
+  for (int ax = 0; ax < ndim; ++ax) plane_pts += gsz / pa[ax];
+  k_filter_clear_unmapped<<<grid_for(plane_pts * ngrids, 256), 256, 0, st>>>(grid, ndim, pa[0], pa[1], pa[2],
+                                                                              plane_pts, ngrids);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   hnd2::FilterMlpArgs fa;
   fa.W1 = f.W1;

@@ -137,7 +137,7 @@ HYENA_ND_API size_t hyena_nd_spectrum_bytes(const hyena_nd_problem* p);
  * function of the descriptor, at least 256 bytes: the control area, then the
  * largest of the convolution's waves of intermediates (64 MiB in the 2D
  * and 3D multi-pass tiers, 48 MiB in the long 1D tier), one channel chunk of
- * the filter call's padded grids plus its first-layer tables (up to 1 GiB)
+ * the filter call's padded grids plus its first-layer tables (up to 2.25 GiB)
  * and one channel chunk of the kernel gradient's grids (about 256 MiB); each
  * at least one volume or channel).  hyena_nd_workspace_bytes_for gives each
  * call's own, smaller need.

@@ -186,8 +186,8 @@ def test_long_1d_sizes(n, B, C):
     ws = H.workspace_bytes(p)
     assert ws >= 256 + max(2 * n * 8, (B + 1) * 2 * n * 8)
     # the largest of: a 48 MiB conv wave, 256 MiB of kernel-gradient grids,
-    # 1 GiB of filter grids (each at least one volume or channel), plus tables
-    assert ws <= 256 + max(48 << 20, 256 << 20, 1 << 30, (B + 1) * 2 * n * 8, 2 * n * 8) + (1 << 20)
+    # 2.25 GiB of filter grids (each at least one volume or channel), plus tables
+    assert ws <= 256 + max(48 << 20, 256 << 20, 2304 << 20, (B + 1) * 2 * n * 8, 2 * n * 8) + (1 << 20)
 
 
 def test_long_1d_spectrum_conversion_uses_the_natural_size():
@@ -216,14 +216,14 @@ def test_static_scratch_call_limits_long_1d():
 @pytest.mark.parametrize("i", range(5))
 def test_workspace_stays_within_the_chunk_budgets(i):
     """Every benchmark grid's workspace is the largest of its scratch parts:
-    a conv wave (64 MiB), a filter chunk (1 GiB plus first-layer tables) and
+    a conv wave (64 MiB), a filter chunk (2.25 GiB plus first-layer tables) and
     a kernel-gradient chunk (256 MiB), each at least one volume or channel."""
     wl = W.workload(i)
     p = H.problem(wl.dims, wl.B, wl.C, H.BF16 if wl.io_dtype == "bf16" else H.F32)
     P = int(np.prod([2 * n for n in wl.dims]))
     one = max(8 * P * (wl.B + 1), 8 * P)
     tables = 5 * 511 * 128 * 4        # three axes' tables and the last axis' sine and cosine
-    assert H.workspace_bytes(p) <= 256 + max(1 << 30, one) + 256 + tables
+    assert H.workspace_bytes(p) <= 256 + max(2304 << 20, one) + 256 + tables
 
 
 @pytest.mark.parametrize("i,tier,waves,launches,streams", [
