@@ -65,13 +65,15 @@ def test_long1d_forward_matches_oracle(dims, B, C, dt):
 
 
 @pytest.mark.parametrize("n,B,C,dt", [(65536, 2, 60, "f32"), (131072, 1, 4, "bf16"), (16384, 3, 5, "f32"),
-                                     (1 << 19, 3, 7, "bf16")])
+                                     (1 << 19, 3, 7, "bf16"), (1 << 20, 1, 64, "bf16")])
 def test_long1d_forward_sampled(n, B, C, dt):
     """Longest grids and multi-wave schedules, sampled outputs against direct
     sums.  2^19 tokens, B = 3, C = 7: 12 channel-pair grids of 8 MiB, so six
     waves of two on three streams, and the last pair of every sample holds
     one channel (channels 0, 3 and 6 are sampled: both halves of a pair and
-    the lone channel)."""
+    the lone channel).  2^20 tokens, B = 1, C = 64 is the benchmark's long
+    1D line in its own launch configuration (32 waves of one grid on three
+    streams)."""
     wl = W.custom((n,), B, C, io_dtype=dt, seed=n % 97 + C)
     inp = W.make_inputs(wl)
     got, _ = run(inp)
