@@ -506,4 +506,100 @@ __global__ void __launch_bounds__(kAT, 2) k_l1_center(const L1PassArgs a) {
   }
 }
 
+// The middle axis passes (kFwdMid, kInvMid) for pencils of 8 slots a lane
+// (N <= 64), with two pencil groups a CTA iteration: both groups' strided
+// loads are issued before the first group's transform, so the second group's
+// latency overlaps it (the same arithmetic as k_l1_pass; with 16 slots a
+// lane the second group's registers spill, and k_l1_pass runs instead).
+template <int N, bool INV>
+__global__ void __launch_bounds__(kAT, 2) k_l1_mid2g(const L1PassArgs a) {
+  constexpr int G = P2<N>::G, R1 = P2<N>::R1, PPW = 32 / G, P = 2 * N;
+  extern __shared__ __align__(16) unsigned char asmem[];
+  pdl_release();
+  const Tabs<N> t = tabs_at<N>(asmem);
+  float4* xb = reinterpret_cast<float4*>(asmem + Tabs<N>::kBytes);
+  tabs_build<N>(t, g_tw512);
+  __syncthreads();
+  pdl_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pen = lane / G, g = lane % G;
+  float4* buf = xb + warp * XB<N>::kWarp + pen * XB<N>::kPen;
+  const long long per_cta = (kAT / 32) * PPW;
+  const long long S = a.stride;
+  const float invQ = ldexpf(1.f, -a.lgQ);
+  const unsigned qm = (1u << a.lgQ) - 1u;
+  for (long long p0 = static_cast<long long>(blockIdx.x) * 2 * per_cta; p0 < a.npen;
+       p0 += static_cast<long long>(gridDim.x) * 2 * per_cta) {
+    long long pp[2];
+    bool act[2];
+    long long o[2];
+    unsigned ii[2];
+    float2* base[2];
+    float2 va[2][R1], vb[2][R1];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      pp[h] = p0 + h * per_cta + warp * PPW + pen;
+      act[h] = pp[h] < a.npen;
+      o[h] = act[h] ? pp[h] >> a.lgS : 0;
+      ii[h] = act[h] ? static_cast<unsigned>(pp[h] & (S - 1)) : 0u;
+      base[h] = a.grid + (((o[h] * P) << a.lgS) + ii[h]);
+#pragma unroll
+      for (int s = 0; s < R1; ++s) {
+        const long long j = INV ? 2LL * spec_idx<N>(g, s) : static_cast<long long>(g + s * G);
+        va[h][s] = act[h] ? *HND_G(&base[h][j * S]) : make_float2(0.f, 0.f);
+        vb[h][s] = act[h] ? *HND_G(&base[h][(INV ? j + 1 : j + N) * S]) : make_float2(0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      cp x[R1];
+      const unsigned i = ii[h];
+      if constexpr (!INV) {
+        full_fwd<N>(va[h], vb[h], x, g, buf, 0, t, 0u);
+        const float2 wi = l1_w(i & qm, invQ);
+        const float2 bG = l1_w((2u * G * i) & qm, invQ);
+        const float2 bR = l1_w((2u * R1 * i) & qm, invQ);
+        float2 wo = l1_w((2u * g * i) & qm, invQ), w0 = wo;
+#pragma unroll
+        for (int s = 0; s < R1; ++s) {
+          if (s > 0) {
+            if (s % P2<N>::R2 == 0) {
+              wo = cmul1(wo, bG);
+              w0 = wo;
+            } else {
+              w0 = cmul1(w0, bR);
+            }
+          }
+          const unsigned f = spec_idx<N>(g, s);
+          const float2 w1 = cmul1(w0, wi);
+          if (act[h]) {
+            *HND_G(&base[h][(2 * f) * S]) = cmul1(make_float2(x[s].re.x, x[s].im.x), w0);
+            *HND_G(&base[h][(2 * f + 1) * S]) = cmul1(make_float2(x[s].re.y, x[s].im.y), w1);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int s = 0; s < R1; ++s) x[s] = {make_float2(va[h][s].x, vb[h][s].x), make_float2(va[h][s].y, vb[h][s].y)};
+        float2 lo[R1], hi[R1];
+        l1_full_inv<N>(x, lo, hi, g, buf, t);
+        const unsigned k = static_cast<unsigned>(o[h] & (a.twP - 1));
+        const unsigned Su = static_cast<unsigned>(S);
+        const float2 wk = l1_conj(l1_w((k * N * Su) & qm, invQ));
+        const float2 cG = l1_conj(l1_w((k * G * Su) & qm, invQ));
+        float2 w0 = l1_conj(l1_w((k * (static_cast<unsigned>(g) * Su + i)) & qm, invQ));
+#pragma unroll
+        for (int s = 0; s < R1; ++s) {
+          const long long j = g + s * G;
+          if (s > 0) w0 = cmul1(w0, cG);
+          const float2 w1 = cmul1(w0, wk);
+          if (act[h]) {
+            *HND_G(&base[h][j * S]) = cmul1(lo[s], w0);
+            *HND_G(&base[h][(j + N) * S]) = cmul1(hi[s], w1);
+          }
+        }
+      }
+    }
+  }
+}
+
 }  // namespace hnd2

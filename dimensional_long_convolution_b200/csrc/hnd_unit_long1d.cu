@@ -45,6 +45,34 @@ cudaError_t l1_center(int N, const hnd2::L1PassArgs& a, cudaStream_t st) {
   }
 }
 
+template <int N, bool INV>
+cudaError_t l1_mid_go(const hnd2::L1PassArgs& a, cudaStream_t st) {
+  auto kern = hnd2::k_l1_mid2g<N, INV>;
+  const size_t sm = hnd2::AxisSmem<N>::kBytes;
+  cudaError_t e = ensure_smem(kern, sm);
+  if (e != cudaSuccess) return e;
+  const long long per_cta = 2 * (hnd2::kAT / 32) * (32 / hnd2::P2<N>::G);   // two pencil groups
+  long long blocks = (a.npen + per_cta - 1) / per_cta;
+  if (blocks > 148LL * 16) blocks = 148LL * 16;
+  if (blocks < 1) blocks = 1;
+  return launch_pdl(true, kern, dim3(static_cast<unsigned>(blocks)), dim3(hnd2::kAT), sm, st, a);
+}
+
+template <int KIND, class T, bool DUAL>
+cudaError_t l1_pass(int N, const hnd2::L1PassArgs& a, cudaStream_t st);
+
+// a middle pass: the two-group kernel for 8-slot pencils, else k_l1_pass
+template <bool INV>
+cudaError_t l1_mid(int N, const hnd2::L1PassArgs& a, cudaStream_t st) {
+  switch (N) {
+    case 16: return l1_mid_go<16, INV>(a, st);
+    case 32: return l1_mid_go<32, INV>(a, st);
+    case 64: return l1_mid_go<64, INV>(a, st);
+    default:
+      return INV ? l1_pass<hnd2::kInvMid, float, false>(N, a, st) : l1_pass<hnd2::kFwdMid, float, false>(N, a, st);
+  }
+}
+
 template <int KIND, class T, bool DUAL>
 cudaError_t l1_pass(int N, const hnd2::L1PassArgs& a, cudaStream_t st) {
   switch (N) {
@@ -111,7 +139,7 @@ cudaError_t long1d_t(const ConvArgs& c, float2* grid, long long v0, long long cn
     set_axis(1);
     a.twQ = static_cast<long long>(sp.P[1]) * sp.P[2];
     a.lgQ = ilog2(a.twQ);
-    e = l1_pass<hnd2::kFwdMid, float, false>(sp.P[1] / 2, a, c.stream);
+    e = l1_mid<false>(sp.P[1] / 2, a, c.stream);
   }
   // spectrum product on the last axis, pencil pairs, with the inverse
   // transform back
@@ -128,7 +156,7 @@ cudaError_t long1d_t(const ConvArgs& c, float2* grid, long long v0, long long cn
     a.twP = sp.P[0];
     a.twQ = P;
     a.lgQ = ilog2(a.twQ);
-    e = l1_pass<hnd2::kInvMid, float, false>(sp.P[1] / 2, a, c.stream);
+    e = l1_mid<true>(sp.P[1] / 2, a, c.stream);
   }
   if (e == cudaSuccess) {
     set_axis(0);
